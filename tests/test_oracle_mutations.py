@@ -1,0 +1,55 @@
+"""Each plausible mistake planted in a copy of the oracle must fail a pin.
+
+The mutants are built from oracle/milo_oracle.c with one textual change each
+(a dropped term, a wrong sign, a swapped index, a wrong tie-break ...), compiled
+into a temporary directory, and the pin suite is run against them in a child
+process.  The real oracle is never modified.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "milo_oracle.c")
+
+MUTANTS = {
+    "dequant_sign": ("((double)codes[k] - z) * s", "(z - (double)codes[k]) * s"),
+    "drop_lorc": ("J->Y[(size_t)m * J->N + n] = acc + lorc;", "J->Y[(size_t)m * J->N + n] = acc;"),
+    "transposed_U": ("J->P->U[(size_t)n * r + p]", "J->P->U[(size_t)p * J->N + n]"),
+    "zero_not_negated": ("float z_f = -mn / s;", "float z_f = mn / s;"),
+    "scale_by_8": ("float s_f = range / 7.0f;", "float s_f = range / 8.0f;"),
+    "round_half_up": ("float r = nearbyintf(v);", "float r = floorf(v + 0.5f);"),
+    "tie_to_higher_id": ("milo_ref_h2d(l[e]) > milo_ref_h2d(l[best])", "milo_ref_h2d(l[e]) >= milo_ref_h2d(l[best])"),
+    "renorm_over_all": ("if (renorm) {", "if (0) {"),
+    "unit_group_swap": ("int c = rr / 16, m = rr % 16 + 16 * half;", "int c = rr / 16, m = rr % 16 + 16 * (1 - half);"),
+    "spare_bits_swapped": ("pos = (m == 30) ? 15 : 31;", "pos = (m == 30) ? 31 : 15;"),
+    "hi_lo_swapped": ("pos = 16 * (within % 2) + 3 * (within / 2) + beta;", "pos = 16 * (1 - within % 2) + 3 * (within / 2) + beta;"),
+    "scale_index_transposed": ("scale[(size_t)j * J->N + n]", "scale[(size_t)n * (J->K / J->group) + j]"),
+    "silu_sign": ("return a / (1.0 + exp(-a));", "return a / (1.0 + exp(a));"),
+    "h_not_rounded": ("h[i] = milo_ref_h2d(h_bits[i]);", "h[i] = milo_ref_silu(a[i]) * b[i];"),
+    "combine_drops_weight": ("acc += w[f] * y_slot[(size_t)f * H + n];", "acc += y_slot[(size_t)f * H + n];"),
+    "shared_dropped": ("for (int s = 0; s < S; ++s) acc += y_sh[((size_t)s * T + t) * H + n];", ""),
+    "gather_wrong_token": ("X + (size_t)(rows[m] / k) * H", "X + (size_t)(rows[m] % T) * H"),
+    "perm_descending": ("int p = offsets[e] + count[e]++;", "int p = offsets[e + 1] - 1 - count[e]++;"),
+    "f2h_truncate": ("double m = nearbyint(ldexp(a, 10 - e));", "double m = floor(ldexp(a, 10 - e));"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
+    mutated = src.replace(old, new)
+    c_path = tmp_path / "mutant.c"
+    so_path = tmp_path / "mutant.so"
+    c_path.write_text(mutated)
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-D_GNU_SOURCE", "-ffp-contract=off", "-fPIC",
+                           "-shared", "-pthread", str(c_path), "-o", str(so_path), "-lm"])
+    env = dict(os.environ, MILO_ORACLE_LIB=str(so_path))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
