@@ -1,0 +1,251 @@
+/*
+ * milo.h -- C ABI of the B200 (sm_100a) int3 + low-rank-compensator MoE forward.
+ *
+ * The operation is the inference hot path of "MiLo: Efficient Quantized MoE
+ * Inference with Mixture of Low-Rank Compensators":
+ *
+ *   - section "MiLo Algorithm: Mixture of Low-Rank Compensators": every expert
+ *     weight is W_out = W_quant + U V, a quantised matrix plus a rank-r
+ *     compensator, with a rank that may differ per expert (and may be 0).  For
+ *     an out x in weight this library stores U [N, r] and V [r, K] and computes
+ *         y = x W_quant^T + (x V^T) U^T ;
+ *   - section "MiLo Kernel: Efficient Int3 Quantized GEMM Backend": int3
+ *     weights times FP16 activations (W3A16), 32 three-bit values packed in
+ *     three 32-bit words without a wasted bit, dequantisation asymmetric with a
+ *     zero point and fused into the GEMM;
+ *   - sections "Background" and "Experimental Setup & Results": the MoE layer
+ *     routes each token to a subset of experts (Mixtral-8x7B-style top-k).
+ *
+ * Conventions (all entry points):
+ *   - Pointers are device pointers owned by the caller unless a comment says
+ *     "host".  The library never allocates device memory and never
+ *     synchronises the host, except milo_*_prepare (documented below).
+ *   - Raw 16-bit floats are passed as uint16_t (fp16 or bf16 bit patterns).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     enqueued on it; results are ready when the stream reaches that point.
+ *   - Argument errors are returned synchronously as milo_status and nothing is
+ *     enqueued.  Data-dependent errors found on the device are OR-ed into the
+ *     caller's `dev_status` word (MILO_DEV_* bits); the caller zeroes it and
+ *     reads it after the stream completes.  `dev_status` may be NULL only where
+ *     stated.
+ *   - Every call is deterministic: identical inputs give identical bits.
+ *   - Calls sharing one workspace must not overlap.
+ */
+#ifndef MILO_H
+#define MILO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MILO_API __attribute__((visibility("default")))
+#else
+#define MILO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MILO_F16 = 0, MILO_BF16 = 1, MILO_F32 = 2 } milo_dtype;
+
+typedef enum {
+    MILO_OK = 0,
+    MILO_ERR_INVALID_ARG = 1,       /* NULL pointer, negative size, bad enum */
+    MILO_ERR_UNSUPPORTED_SHAPE = 2, /* e.g. K not a multiple of 128, group != 64 */
+    MILO_ERR_WORKSPACE = 3,         /* workspace or table too small / misaligned */
+    MILO_ERR_CUDA = 4               /* a CUDA runtime call failed (see milo_last_error) */
+} milo_status;
+
+/* Device status bits, OR-ed into *dev_status by the kernels. */
+#define MILO_DEV_BAD_EXPERT_ID 0x1  /* a routed id outside [0, E): the slot is dropped */
+#define MILO_DEV_NONFINITE 0x2      /* NaN/Inf in weights, logits or activations */
+#define MILO_DEV_FP16_RANGE 0x4     /* a value does not fit fp16 (activation, s or z) */
+#define MILO_DEV_TIMEOUT 0x8        /* a bounded pipeline wait gave up; outputs invalid */
+
+/* Router flags. */
+#define MILO_ROUTE_RENORM 0x1u      /* renormalise the softmax over the k picked experts */
+#define MILO_ROUTE_IDS_GIVEN 0x2u   /* topk_ids are inputs (logits NULL, topk_w untouched) */
+
+/* Limits of this build. */
+#define MILO_GROUP 64               /* scale/zero group along K */
+#define MILO_MAX_RANK 64            /* compensator rank, a multiple of 8 */
+#define MILO_MAX_EXPERTS 256        /* routed + shared */
+#define MILO_MAX_TOPK 16
+
+MILO_API const char* milo_status_str(milo_status s);
+/* Host string describing the last failure on the calling thread ("" if none). */
+MILO_API const char* milo_last_error(void);
+MILO_API int32_t milo_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Packed int3 weights                                                      */
+/* ------------------------------------------------------------------------ */
+/*
+ * Packing format (self-defined; the page describes three 32-bit words holding
+ * 32 three-bit values with no wasted bit but its bit positions are garbled):
+ * a row of K codes, K a multiple of 128, is cut into super-blocks of 128 codes
+ * (two scale groups of 64).  Super-block b occupies words 12b..12b+11 of the
+ * row, as four 3-word units.  Unit c (0..3) carries the 32 codes
+ *     u_m = q[128b + 16c + m]             m = 0..15   (first group)
+ *     u_m = q[128b + 64 + 16c + m - 16]   m = 16..31  (second group)
+ * and word t (0..2) of the unit holds, for i = 0..4,
+ *     bits [3i, 3i+3) = u_{10t+2i},   bits [16+3i, 16+3i+3) = u_{10t+2i+1},
+ * bit 15 = bit t of u_30, bit 31 = bit t of u_31.
+ * Q is u32 [N, 3K/32] row-major (row pitch 3K/8 bytes).  scale and zero are
+ * fp16 [K/64, N] (group-major, N contiguous).  Dequantisation:
+ *     w_hat[n, k] = (q[n, k] - zero[k/64, n]) * scale[k/64, n].
+ */
+
+/*
+ * milo_pack -- quantise W fp16 [N, K] (row-major) to int3 and pack it.
+ * Round-to-nearest asymmetric min/max per group of 64 along K (the paper's HQQ
+ * initialiser is replaced by RTN for synthetic weights):
+ *     s = fp16((max - min) / 7)   (s := 1 when it rounds to 0)
+ *     z = fp16(-min / s)
+ *     q = clamp(rint(w / s + z), 0, 7)    (fp32, ties to even, no FMA)
+ * Writes Q u32 [N, 3K/32], scale and zero fp16 [K/64, N].
+ * Errors: group != 64 or K % 128 != 0 -> UNSUPPORTED_SHAPE; N, K <= 0 or NULL
+ * pointers -> INVALID_ARG.  Device: NONFINITE for NaN/Inf weights, FP16_RANGE
+ * when s or z overflows fp16.  dev_status may be NULL.
+ */
+MILO_API milo_status milo_pack(const uint16_t* W, int32_t N, int32_t K, int32_t group,
+                      uint32_t* Q, uint16_t* scale, uint16_t* zero,
+                      int32_t* dev_status, void* stream);
+
+/*
+ * milo_unpack -- extract the codes of Q u32 [N, 3K/32] into codes u8 [N, K],
+ * with the same register-level field extraction the GEMM kernels use.
+ */
+MILO_API milo_status milo_unpack(const uint32_t* Q, int32_t N, int32_t K, uint8_t* codes,
+                        void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Routing                                                                  */
+/* ------------------------------------------------------------------------ */
+/*
+ * milo_route -- top-k router and expert grouping (histogram, exclusive scan,
+ * stable scatter).
+ *   logits      fp16 [T, E] (ignored, may be NULL, with MILO_ROUTE_IDS_GIVEN)
+ *   topk_ids    int32 [T, k]: output, slot j = j-th largest logit, ties to the
+ *               lower expert id; input with MILO_ROUTE_IDS_GIVEN
+ *   topk_w      f32 [T, k]: softmax weight exp(l_j - l_max) / sum, the sum over
+ *               the k picked experts (MILO_ROUTE_RENORM) or over all E.
+ *               Not written with MILO_ROUTE_IDS_GIVEN (may be NULL then).
+ *   expert_offsets int32 [E+1]: exclusive scan of the per-expert slot counts
+ *   perm        int32 [T*k]: the flat slots f = t*k + j of expert 0 in
+ *               ascending order, then expert 1, ...
+ *   inv_perm    int32 [T*k]: inv_perm[perm[p]] = p; -1 for a dropped slot
+ * Limits: 1 <= E <= MILO_MAX_EXPERTS, 1 <= k <= min(E, MILO_MAX_TOPK), T >= 0.
+ * Device: BAD_EXPERT_ID (given ids outside [0, E); the slot is dropped),
+ * NONFINITE (NaN/Inf logits; ids then unspecified).
+ */
+MILO_API milo_status milo_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k,
+                       uint32_t flags, int32_t* topk_ids, float* topk_w,
+                       int32_t* expert_offsets, int32_t* perm, int32_t* inv_perm,
+                       int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Quantised projections and layers                                         */
+/* ------------------------------------------------------------------------ */
+
+/* One quantised projection W [N, K] with its rank-r compensator (host struct
+ * holding device pointers).  U fp16 [N, r] and V fp16 [r, K] row-major; both
+ * may be NULL when rank == 0.  rank is a multiple of 8, at most MILO_MAX_RANK. */
+typedef struct milo_qweight {
+    const uint32_t* q;
+    const uint16_t* scale;
+    const uint16_t* zero;
+    const uint16_t* U;
+    const uint16_t* V;
+    int32_t rank;
+} milo_qweight;
+
+/* One SwiGLU expert: w1, w3 [I, H] and w2 [H, I]. */
+typedef struct milo_expert {
+    milo_qweight w1, w3, w2;
+} milo_expert;
+
+/* A grouped projection: n_experts weights of the same shape [N, K]. */
+typedef struct milo_linear {
+    int32_t N, K, n_experts, group;
+    int32_t max_rank;       /* set by milo_linear_prepare */
+    const void* table;      /* device table written by milo_linear_prepare */
+} milo_linear;
+
+/* A SwiGLU MoE layer: experts 0..n_routed-1 are routed, the n_shared experts
+ * after them see every token with weight 1. */
+typedef struct milo_moe_layer {
+    int32_t hidden, inter, n_routed, n_shared, top_k, group;
+    int32_t max_rank;       /* set by milo_layer_prepare */
+    const void* table;      /* device table written by milo_layer_prepare */
+} milo_moe_layer;
+
+/* Bytes of the device table for n projections (64-byte aligned buffer). */
+MILO_API milo_status milo_table_bytes(int32_t n_projections, size_t* bytes);
+
+/*
+ * milo_linear_prepare / milo_layer_prepare -- validate the weights (host
+ * array `weights` / `experts` of device pointers) and write the device table
+ * (TMA tensor maps and pointers) to `device_table`, which the caller keeps
+ * alive and unmodified while the layer is used.  One-time set-up: the table is
+ * copied with a synchronous cudaMemcpy.  lin/layer are host structs; the
+ * caller fills the shape fields and the call sets max_rank and table.
+ * Errors: UNSUPPORTED_SHAPE (K % 128, N % 16, group != 64, rank not a multiple
+ * of 8 or above MILO_MAX_RANK), WORKSPACE (table too small or not 64-byte
+ * aligned), INVALID_ARG (NULL or misaligned weight pointers).
+ */
+MILO_API milo_status milo_linear_prepare(milo_linear* lin, const milo_qweight* weights,
+                                void* device_table, size_t table_bytes);
+MILO_API milo_status milo_layer_prepare(milo_moe_layer* layer, const milo_expert* experts,
+                               void* device_table, size_t table_bytes);
+
+/* Workspace bytes for milo_grouped_linear / milo_moe_forward over T tokens. */
+MILO_API milo_status milo_linear_workspace_bytes(const milo_linear* lin, int32_t T, int32_t k,
+                                        size_t* bytes);
+MILO_API milo_status milo_moe_workspace_bytes(const milo_moe_layer* layer, int32_t T, size_t* bytes);
+
+/*
+ * milo_grouped_linear -- per routed slot, y = x W_e^T + (x V_e^T) U_e^T.
+ *   x        [T, K] fp16 or bf16 (x_dt), row-major
+ *   expert_offsets, perm  from milo_route over n_experts experts and k slots
+ *            per token (perm may be NULL: the identity, x already grouped, k = 1)
+ *   y        [T*k, N] in y_dt (F32, F16 or BF16), row f = t*k + j; rows of
+ *            dropped slots are written as zeros
+ *   ws       >= milo_linear_workspace_bytes(lin, T, k), 256-byte aligned
+ * Device: FP16_RANGE (|x| > 65504), NONFINITE, TIMEOUT.
+ */
+MILO_API milo_status milo_grouped_linear(const milo_linear* lin, const void* x, milo_dtype x_dt,
+                                int32_t T, int32_t k, const int32_t* expert_offsets,
+                                const int32_t* perm, void* y, milo_dtype y_dt,
+                                void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * milo_moe_forward -- the SwiGLU MoE layer:
+ *     h  = fp16( silu(x W1_e^T + LoRC1) * (x W3_e^T + LoRC3) )
+ *     y_slot = h W2_e^T + LoRC2
+ *     y[t] = sum_j topk_w[t, j] * y_slot[t*k + j]  +  sum_s shared_s(x_t)
+ *   x        [T, hidden] fp16 or bf16, row-major
+ *   topk_w, expert_offsets, perm, inv_perm  from milo_route (k = layer->top_k)
+ *   y        [T, hidden] in y_dt (F32, F16, BF16); the fp16/bf16 outputs are the
+ *            round-to-nearest of the f32 result
+ *   ws       >= milo_moe_workspace_bytes(layer, T), 256-byte aligned.  The
+ *            fp16 SwiGLU activations h [T*k + n_shared*T, inter] sit at byte
+ *            offset milo_moe_h_offset(layer, T) of ws after the call, row p =
+ *            expert-sorted slot p (shared-expert rows after the routed ones).
+ * Device: FP16_RANGE, NONFINITE, TIMEOUT.
+ */
+MILO_API milo_status milo_moe_forward(const milo_moe_layer* layer, const void* x, milo_dtype x_dt,
+                             int32_t T, const float* topk_w, const int32_t* expert_offsets,
+                             const int32_t* perm, const int32_t* inv_perm, void* y,
+                             milo_dtype y_dt, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream);
+
+/* Byte offset of h inside the forward workspace (see milo_moe_forward). */
+MILO_API size_t milo_moe_h_offset(const milo_moe_layer* layer, int32_t T);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MILO_H */

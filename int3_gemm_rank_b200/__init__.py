@@ -1,0 +1,314 @@
+"""Python binding of libmilo (include/milo.h): argument marshalling only.
+
+Every step of the int3 + low-rank-compensator MoE forward runs in the sm_100a
+kernels of ``libmilo.so``; this module passes torch tensors' device pointers
+and the current CUDA stream through ctypes.  torch is used for device memory
+and streams only.  There is no CPU fallback: if the library is missing or no
+GPU is present the calls raise.
+
+The operation is the inference hot path of "MiLo: Efficient Quantized MoE
+Inference with Mixture of Low-Rank Compensators" (W_out = W_quant + U V with
+int3 W_quant, routed over a Mixtral-style top-k MoE layer).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmilo.so")
+
+MILO_F16, MILO_BF16, MILO_F32 = 0, 1, 2
+MILO_OK, MILO_ERR_INVALID_ARG, MILO_ERR_UNSUPPORTED_SHAPE, MILO_ERR_WORKSPACE, MILO_ERR_CUDA = range(5)
+MILO_DEV_BAD_EXPERT_ID, MILO_DEV_NONFINITE, MILO_DEV_FP16_RANGE, MILO_DEV_TIMEOUT = 1, 2, 4, 8
+MILO_ROUTE_RENORM, MILO_ROUTE_IDS_GIVEN = 1, 2
+MILO_GROUP, MILO_MAX_RANK = 64, 64
+
+# The C ABI symbols of include/milo.h (checked by the tests).
+EXPORTS = ("milo_status_str", "milo_last_error", "milo_version", "milo_pack", "milo_unpack",
+           "milo_route", "milo_table_bytes", "milo_linear_prepare", "milo_layer_prepare",
+           "milo_linear_workspace_bytes", "milo_moe_workspace_bytes", "milo_grouped_linear",
+           "milo_moe_forward", "milo_moe_h_offset")
+
+
+class MiloError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"milo status {status}: {msg}")
+        self.status = status
+
+
+class milo_qweight(C.Structure):
+    _fields_ = [("q", C.c_void_p), ("scale", C.c_void_p), ("zero", C.c_void_p),
+                ("U", C.c_void_p), ("V", C.c_void_p), ("rank", C.c_int32)]
+
+
+class milo_expert(C.Structure):
+    _fields_ = [("w1", milo_qweight), ("w3", milo_qweight), ("w2", milo_qweight)]
+
+
+class milo_linear(C.Structure):
+    _fields_ = [("N", C.c_int32), ("K", C.c_int32), ("n_experts", C.c_int32), ("group", C.c_int32),
+                ("max_rank", C.c_int32), ("table", C.c_void_p)]
+
+
+class milo_moe_layer(C.Structure):
+    _fields_ = [("hidden", C.c_int32), ("inter", C.c_int32), ("n_routed", C.c_int32),
+                ("n_shared", C.c_int32), ("top_k", C.c_int32), ("group", C.c_int32),
+                ("max_rank", C.c_int32), ("table", C.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load libmilo.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m int3_gemm_rank_b200.build` (nvcc, sm_100a)")
+        L = C.CDLL(LIB_PATH)
+        vp, i32, u32, sz = C.c_void_p, C.c_int32, C.c_uint32, C.c_size_t
+        L.milo_status_str.argtypes = [C.c_int]; L.milo_status_str.restype = C.c_char_p
+        L.milo_last_error.argtypes = []; L.milo_last_error.restype = C.c_char_p
+        L.milo_version.argtypes = []; L.milo_version.restype = i32
+        L.milo_pack.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp]; L.milo_pack.restype = C.c_int
+        L.milo_unpack.argtypes = [vp, i32, i32, vp, vp]; L.milo_unpack.restype = C.c_int
+        L.milo_route.argtypes = [vp, i32, i32, i32, u32, vp, vp, vp, vp, vp, vp, vp]
+        L.milo_route.restype = C.c_int
+        L.milo_table_bytes.argtypes = [i32, C.POINTER(sz)]; L.milo_table_bytes.restype = C.c_int
+        L.milo_linear_prepare.argtypes = [C.POINTER(milo_linear), C.POINTER(milo_qweight), vp, sz]
+        L.milo_linear_prepare.restype = C.c_int
+        L.milo_layer_prepare.argtypes = [C.POINTER(milo_moe_layer), C.POINTER(milo_expert), vp, sz]
+        L.milo_layer_prepare.restype = C.c_int
+        L.milo_linear_workspace_bytes.argtypes = [C.POINTER(milo_linear), i32, i32, C.POINTER(sz)]
+        L.milo_linear_workspace_bytes.restype = C.c_int
+        L.milo_moe_workspace_bytes.argtypes = [C.POINTER(milo_moe_layer), i32, C.POINTER(sz)]
+        L.milo_moe_workspace_bytes.restype = C.c_int
+        L.milo_grouped_linear.argtypes = [C.POINTER(milo_linear), vp, C.c_int, i32, i32, vp, vp, vp,
+                                          C.c_int, vp, sz, vp, vp]
+        L.milo_grouped_linear.restype = C.c_int
+        L.milo_moe_forward.argtypes = [C.POINTER(milo_moe_layer), vp, C.c_int, i32, vp, vp, vp, vp,
+                                       vp, C.c_int, vp, sz, vp, vp]
+        L.milo_moe_forward.restype = C.c_int
+        L.milo_moe_h_offset.argtypes = [C.POINTER(milo_moe_layer), i32]
+        L.milo_moe_h_offset.restype = sz
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != MILO_OK:
+        msg = lib().milo_last_error().decode() or lib().milo_status_str(status).decode()
+        raise MiloError(status, f"{what}: {msg}")
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    return {torch.float16: MILO_F16, torch.bfloat16: MILO_BF16, torch.float32: MILO_F32}[t.dtype]
+
+
+def _cuda(t: torch.Tensor, name: str):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def new_status(device=None) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+# ---------------------------------------------------------------------------
+# packing
+# ---------------------------------------------------------------------------
+
+def milo_pack(W: torch.Tensor, group: int = MILO_GROUP, dev_status: torch.Tensor | None = None):
+    """Quantise W fp16 [N, K] to int3 and pack: returns (Q u32-as-int32 [N, 3K/32], scale, zero [K/64, N])."""
+    _cuda(W, "W")
+    N, K = W.shape
+    Q = torch.empty((N, 3 * K // 32), dtype=torch.int32, device=W.device)
+    s = torch.empty((K // group, N), dtype=torch.float16, device=W.device)
+    z = torch.empty((K // group, N), dtype=torch.float16, device=W.device)
+    _check(lib().milo_pack(_ptr(W), N, K, group, _ptr(Q), _ptr(s), _ptr(z), _ptr(dev_status),
+                           _stream()), "milo_pack")
+    return Q, s, z
+
+
+def milo_unpack(Q: torch.Tensor, K: int) -> torch.Tensor:
+    _cuda(Q, "Q")
+    N = Q.shape[0]
+    codes = torch.empty((N, K), dtype=torch.uint8, device=Q.device)
+    _check(lib().milo_unpack(_ptr(Q), N, K, _ptr(codes), _stream()), "milo_unpack")
+    return codes
+
+
+# ---------------------------------------------------------------------------
+# routing
+# ---------------------------------------------------------------------------
+
+def milo_route(logits: torch.Tensor | None, k: int, renorm: bool, E: int | None = None,
+               ids: torch.Tensor | None = None, dev_status: torch.Tensor | None = None) -> dict:
+    """Top-k router + grouping.  With `ids` given ([T, k] int32) the top-k is skipped."""
+    flags = MILO_ROUTE_RENORM if renorm else 0
+    if ids is not None:
+        flags |= MILO_ROUTE_IDS_GIVEN
+        _cuda(ids, "ids")
+        T = ids.shape[0]
+        dev = ids.device
+        w = None
+    else:
+        _cuda(logits, "logits")
+        T, E = logits.shape
+        dev = logits.device
+        ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+        w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+    inv = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+    _check(lib().milo_route(_ptr(logits), T, E, k, flags, _ptr(ids), _ptr(w), _ptr(off), _ptr(perm),
+                            _ptr(inv), _ptr(dev_status), _stream()), "milo_route")
+    return {"ids": ids, "w": w, "offsets": off, "perm": perm[:T * k], "inv_perm": inv[:T * k]}
+
+
+# ---------------------------------------------------------------------------
+# projections and layers
+# ---------------------------------------------------------------------------
+
+class QWeight:
+    """A packed projection on the device: Q, scale, zero and the compensator U [N, r], V [r, K]."""
+
+    def __init__(self, Q, scale, zero, U=None, V=None):
+        self.Q, self.scale, self.zero = Q, scale, zero
+        self.rank = 0 if U is None or U.numel() == 0 else int(U.shape[1])
+        self.U = U if self.rank else None
+        self.V = V if self.rank else None
+        self.N = Q.shape[0]
+        self.K = Q.shape[1] * 32 // 3
+
+    @classmethod
+    def quantize(cls, W: torch.Tensor, U=None, V=None, dev_status=None):
+        Q, s, z = milo_pack(W, dev_status=dev_status)
+        return cls(Q, s, z, U, V)
+
+    def cstruct(self) -> milo_qweight:
+        return milo_qweight(self.Q.data_ptr(), self.scale.data_ptr(), self.zero.data_ptr(),
+                            self.U.data_ptr() if self.rank else None,
+                            self.V.data_ptr() if self.rank else None, self.rank)
+
+
+def _table(n_proj: int, device) -> torch.Tensor:
+    nb = C.c_size_t()
+    _check(lib().milo_table_bytes(n_proj, C.byref(nb)), "milo_table_bytes")
+    return torch.empty(nb.value + 64, dtype=torch.uint8, device=device)
+
+
+def _aligned_view(buf: torch.Tensor, align: int, nbytes: int) -> tuple:
+    off = (-buf.data_ptr()) % align
+    return buf.data_ptr() + off, nbytes
+
+
+class GroupedLinear:
+    """milo_grouped_linear over n_experts packed projections of shape [N, K]."""
+
+    def __init__(self, weights: list, device="cuda"):
+        self.weights = weights
+        self.cs = milo_linear(weights[0].N, weights[0].K, len(weights), MILO_GROUP, 0, None)
+        arr = (milo_qweight * len(weights))(*[w.cstruct() for w in weights])
+        self._table = _table(len(weights), device)
+        ptr, nb = _aligned_view(self._table, 64, self._table.numel() - 64)
+        _check(lib().milo_linear_prepare(C.byref(self.cs), arr, C.c_void_p(ptr), nb), "milo_linear_prepare")
+        self._ws = None
+
+    def workspace_bytes(self, T: int, k: int) -> int:
+        nb = C.c_size_t()
+        _check(lib().milo_linear_workspace_bytes(C.byref(self.cs), T, k, C.byref(nb)),
+               "milo_linear_workspace_bytes")
+        return nb.value
+
+    def workspace(self, T: int, k: int, device="cuda") -> torch.Tensor:
+        need = self.workspace_bytes(T, k) + 256
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=device)
+        return self._ws
+
+    def __call__(self, x: torch.Tensor, offsets: torch.Tensor, perm: torch.Tensor | None, k: int = 1,
+                 out_dtype=torch.float32, dev_status=None, y=None, ws=None) -> torch.Tensor:
+        return milo_grouped_linear(self, x, offsets, perm, k, out_dtype, dev_status, y, ws)
+
+
+def milo_grouped_linear(lin: GroupedLinear, x, offsets, perm, k=1, out_dtype=torch.float32,
+                        dev_status=None, y=None, ws=None) -> torch.Tensor:
+    _cuda(x, "x")
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty((T * k, lin.cs.N), dtype=out_dtype, device=x.device)
+    if ws is None:
+        ws = lin.workspace(T, k, x.device)
+    wp, wn = _aligned_view(ws, 256, ws.numel() - 256)
+    _check(lib().milo_grouped_linear(C.byref(lin.cs), _ptr(x), _dt(x), T, k, _ptr(offsets), _ptr(perm),
+                                     _ptr(y), _dt(y), C.c_void_p(wp), wn, _ptr(dev_status), _stream()),
+           "milo_grouped_linear")
+    return y
+
+
+class MoELayer:
+    """milo_moe_forward over routed + shared SwiGLU experts (list of dict(w1=, w3=, w2=) QWeights)."""
+
+    def __init__(self, experts: list, n_routed: int, n_shared: int, top_k: int, device="cuda"):
+        self.experts = experts
+        H = experts[0]["w2"].N
+        I = experts[0]["w1"].N
+        self.cs = milo_moe_layer(H, I, n_routed, n_shared, top_k, MILO_GROUP, 0, None)
+        arr = (milo_expert * len(experts))(*[milo_expert(e["w1"].cstruct(), e["w3"].cstruct(),
+                                                         e["w2"].cstruct()) for e in experts])
+        self._table = _table(3 * len(experts), device)
+        ptr, nb = _aligned_view(self._table, 64, self._table.numel() - 64)
+        _check(lib().milo_layer_prepare(C.byref(self.cs), arr, C.c_void_p(ptr), nb), "milo_layer_prepare")
+        self._ws = None
+
+    def workspace_bytes(self, T: int) -> int:
+        nb = C.c_size_t()
+        _check(lib().milo_moe_workspace_bytes(C.byref(self.cs), T, C.byref(nb)), "milo_moe_workspace_bytes")
+        return nb.value
+
+    def workspace(self, T: int, device="cuda") -> torch.Tensor:
+        need = self.workspace_bytes(T) + 256
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=device)
+        return self._ws
+
+    def h_view(self, T: int, ws: torch.Tensor | None = None) -> torch.Tensor:
+        """The fp16 SwiGLU activations [T*k + S*T, I] left in the workspace by the last forward."""
+        ws = self._ws if ws is None else ws
+        wp, _ = _aligned_view(ws, 256, 0)
+        off = (wp - ws.data_ptr()) + lib().milo_moe_h_offset(C.byref(self.cs), T)
+        R = T * self.cs.top_k + self.cs.n_shared * T
+        return ws[off:off + R * self.cs.inter * 2].view(torch.float16).view(R, self.cs.inter)
+
+    def __call__(self, x, route: dict, out_dtype=torch.float32, dev_status=None, y=None, ws=None):
+        return milo_moe_forward(self, x, route, out_dtype, dev_status, y, ws)
+
+
+def milo_moe_forward(layer: MoELayer, x, route: dict, out_dtype=torch.float32, dev_status=None,
+                     y=None, ws=None) -> torch.Tensor:
+    _cuda(x, "x")
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty((T, layer.cs.hidden), dtype=out_dtype, device=x.device)
+    if ws is None:
+        ws = layer.workspace(T, x.device)
+    wp, wn = _aligned_view(ws, 256, ws.numel() - 256)
+    _check(lib().milo_moe_forward(C.byref(layer.cs), _ptr(x), _dt(x), T, _ptr(route["w"]),
+                                  _ptr(route["offsets"]), _ptr(route["perm"]), _ptr(route["inv_perm"]),
+                                  _ptr(y), _dt(y), C.c_void_p(wp), wn, _ptr(dev_status), _stream()),
+           "milo_moe_forward")
+    return y

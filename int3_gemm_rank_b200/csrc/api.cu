@@ -1,0 +1,515 @@
+// api.cu -- host side of libmilo: argument validation, device tables (TMA
+// tensor maps), workspace layout and the launch sequence of the forward.
+//
+// The sequence for one MoE layer ("MiLo: Efficient Quantized MoE Inference
+// with Mixture of Low-Rank Compensators": routed experts, each a quantised
+// weight plus a rank-r compensator, outputs mixed by the router weights):
+//   rows -> prep(x) -> lorc(x, V1|V3) -> gemv<SwiGLU>(w1|w3) -> prep(h)
+//        -> lorc(h, V2) -> gemv(w2) -> combine
+// Every step is a kernel on the caller's stream; the host never waits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "milo_host.h"
+#include "milo_kernels.h"
+
+namespace milo {
+
+static thread_local std::string g_last_error;
+void clear_error() { g_last_error.clear(); }
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+// ---------------------------------------------------------------------------
+// tensor maps (driver entry point fetched through the runtime; no -lcuda)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `esize`-byte elements with row pitch
+// `pitch` bytes; box {bcols, brows}.
+static milo_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize,
+                            uint64_t cols, uint64_t rows, uint64_t pitch, uint32_t bcols,
+                            uint32_t brows, const char* what) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(MILO_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {pitch};
+    cuuint32_t box[2] = {bcols, brows};
+    cuuint32_t estr[2] = {1, 1};
+    (void)esize;
+    CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(MILO_ERR_INVALID_ARG, std::string("tensor map encoding failed for ") + what +
+                                              " (code " + std::to_string(static_cast<int>(r)) + ")");
+    return MILO_OK;
+}
+
+static int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// ---------------------------------------------------------------------------
+// tables
+// ---------------------------------------------------------------------------
+static milo_status fill_proj(ProjDev* d, const milo_qweight& w, int N, int K, int tile_rows,
+                             const char* what) {
+    memset(d, 0, sizeof(*d));
+    if (!w.q || !w.scale || !w.zero)
+        return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": NULL weight pointer");
+    if (w.rank < 0 || w.rank % 8 || w.rank > MILO_MAX_RANK)
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE,
+                    std::string(what) + ": rank must be a multiple of 8 in [0, 64]");
+    if (w.rank > 0 && (!w.U || !w.V))
+        return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": U and V are required when rank > 0");
+    if (!aligned(w.q, 16) || !aligned(w.scale, 16) || !aligned(w.zero, 16) ||
+        (w.rank > 0 && (!aligned(w.U, 16) || !aligned(w.V, 16))))
+        return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": pointers must be 16-byte aligned");
+    const int G = K / MILO_GROUP;
+    milo_status s;
+    if ((s = make_map(&d->q_map, w.q, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 3 * K / 32, N,
+                      static_cast<uint64_t>(3 * K / 32) * 4, 12, tile_rows, what)) != MILO_OK) return s;
+    if ((s = make_map(&d->s_map, w.scale, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, N, G,
+                      static_cast<uint64_t>(N) * 2, tile_rows, 4, what)) != MILO_OK) return s;
+    if ((s = make_map(&d->z_map, w.zero, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, N, G,
+                      static_cast<uint64_t>(N) * 2, tile_rows, 4, what)) != MILO_OK) return s;
+    if (w.rank > 0 &&
+        (s = make_map(&d->u_map, w.U, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w.rank, N,
+                      static_cast<uint64_t>(w.rank) * 2, w.rank, tile_rows, what)) != MILO_OK) return s;
+    d->q = w.q;
+    d->scale = w.scale;
+    d->zero = w.zero;
+    d->U = w.rank > 0 ? w.U : nullptr;
+    d->V = w.rank > 0 ? w.V : nullptr;
+    d->rank = w.rank;
+    d->N = N;
+    d->K = K;
+    d->tile_rows = tile_rows;
+    return MILO_OK;
+}
+
+static milo_status check_nk(int N, int K, const char* what) {
+    if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": sizes must be positive");
+    if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": K must be a multiple of 128");
+    if (N % 16) return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": N must be a multiple of 16");
+    return MILO_OK;
+}
+
+static milo_status upload(void* device_table, size_t table_bytes, const std::vector<ProjDev>& t) {
+    if (!device_table || !aligned(device_table, 64))
+        return fail(MILO_ERR_WORKSPACE, "device table must be a 64-byte aligned device buffer");
+    const size_t need = t.size() * sizeof(ProjDev);
+    if (table_bytes < need) return fail(MILO_ERR_WORKSPACE, "device table too small");
+    return check_cuda(cudaMemcpy(device_table, t.data(), need, cudaMemcpyHostToDevice), "table upload");
+}
+
+// ---------------------------------------------------------------------------
+// workspace layouts
+// ---------------------------------------------------------------------------
+struct Carve {
+    size_t off = 0;
+    size_t take(size_t bytes) {
+        const size_t o = off;
+        off = round_up(off + bytes, 256);
+        return o;
+    }
+};
+
+static int gpad_of(int K) { return static_cast<int>(round_up(K / MILO_GROUP, 4)); }
+static size_t frag_row_bytes(int K) { return static_cast<size_t>(K / 128) * 288; }
+
+struct LinearWs {
+    size_t grp, rows, inv, frag, gsum, t, part, total;
+    int R, splits, tcols;
+};
+
+static int tiles_of(int N, int rows) { return (N + rows - 1) / rows; }
+
+// Split-K factor for the plain kernel: make the estimated item count fill the
+// persistent grid in whole waves (the tail "shift" of the work distribution).
+static int choose_splits(long long base_items, int chunks) {
+    const int slots = 2 * sm_count();
+    if (base_items <= 0) return 1;
+    int best = 1;
+    double best_eff = -1.0;
+    for (int s = 1; s <= 16 && s <= chunks; ++s) {
+        const double items = static_cast<double>(base_items) * s;
+        const double waves = items / slots;
+        double eff = waves / std::ceil(waves);
+        if (waves < 1.0) eff = waves;                     // under-filled grid
+        eff -= 0.004 * (s - 1);                           // partial-sum traffic
+        if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
+    }
+    return best;
+}
+
+static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
+    LinearWs w;
+    Carve c;
+    w.R = T * k;
+    const int n_exp = lin->n_experts;
+    const int chunks = (lin->K + kChunkK - 1) / kChunkK;
+    const long long groups = std::min<long long>(n_exp, std::max(1LL, static_cast<long long>(T) * k));
+    const long long tt = std::max(1LL, (static_cast<long long>(T) * k + kTokTile - 1) / kTokTile);
+    w.splits = choose_splits(std::max(groups, tt) * tiles_of(lin->N, kRowsPlain), chunks);
+    w.tcols = std::max(8, lin->max_rank);
+    w.grp = c.take(static_cast<size_t>(n_exp) * 8);
+    w.rows = c.take(static_cast<size_t>(w.R) * 4);
+    w.inv = c.take(static_cast<size_t>(w.R) * 4);
+    w.frag = c.take(static_cast<size_t>(w.R) * frag_row_bytes(lin->K));
+    w.gsum = c.take(static_cast<size_t>(w.R) * gpad_of(lin->K) * 4);
+    w.t = c.take(static_cast<size_t>(w.R) * w.tcols * 2);
+    w.part = c.take(static_cast<size_t>(w.splits) * w.R * lin->N * 4);
+    w.total = c.off;
+    return w;
+}
+
+struct MoeWs {
+    size_t grp, rows, xfrag, xg, t13, h, hfrag, hg, t2, part, total;
+    int R, R_routed, splits, tc13, tc2;
+};
+
+static MoeWs moe_ws(const milo_moe_layer* L, int T) {
+    MoeWs w;
+    Carve c;
+    const int H = L->hidden, I = L->inter;
+    w.R_routed = T * L->top_k;
+    w.R = w.R_routed + L->n_shared * T;
+    const int n_exp = L->n_routed + L->n_shared;
+    const int chunks = (I + kChunkK - 1) / kChunkK;
+    const long long groups = std::min<long long>(L->n_routed, std::max(1LL, static_cast<long long>(w.R_routed))) + L->n_shared;
+    w.splits = choose_splits(groups * tiles_of(H, kRowsPlain), chunks);
+    w.tc13 = std::max(8, 2 * L->max_rank);
+    w.tc2 = std::max(8, L->max_rank);
+    w.grp = c.take(static_cast<size_t>(n_exp) * 8);
+    w.rows = c.take(static_cast<size_t>(w.R) * 4);
+    w.xfrag = c.take(static_cast<size_t>(w.R) * frag_row_bytes(H));
+    w.xg = c.take(static_cast<size_t>(w.R) * gpad_of(H) * 4);
+    w.t13 = c.take(static_cast<size_t>(w.R) * w.tc13 * 2);
+    w.h = c.take(static_cast<size_t>(w.R) * I * 2);
+    w.hfrag = c.take(static_cast<size_t>(w.R) * frag_row_bytes(I));
+    w.hg = c.take(static_cast<size_t>(w.R) * gpad_of(I) * 4);
+    w.t2 = c.take(static_cast<size_t>(w.R) * w.tc2 * 2);
+    w.part = c.take(static_cast<size_t>(w.splits) * w.R * H * 4);
+    w.total = c.off;
+    return w;
+}
+
+// ---------------------------------------------------------------------------
+// launch helpers
+// ---------------------------------------------------------------------------
+static milo_status act_maps(GemvParams& g, void* frag, void* gsum, void* t, int R, int K, int tcols,
+                            bool has_t) {
+    milo_status s;
+    const int SB = K / 128;
+    const int Rm = std::max(R, 1);
+    if ((s = make_map(&g.x_map, frag, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<uint64_t>(SB) * 144, Rm,
+                      frag_row_bytes(K), 144, kTokTile, "activations")) != MILO_OK) return s;
+    if ((s = make_map(&g.g_map, gsum, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, gpad_of(K), Rm,
+                      static_cast<uint64_t>(gpad_of(K)) * 4, 4, kTokTile, "group sums")) != MILO_OK) return s;
+    if (has_t) {
+        if ((s = make_map(&g.t_map, t, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, tcols, Rm,
+                          static_cast<uint64_t>(tcols) * 2, tcols, kTokTile, "compensator rows")) != MILO_OK)
+            return s;
+    } else {
+        memset(&g.t_map, 0, sizeof(g.t_map));
+    }
+    return MILO_OK;
+}
+
+static milo_status run_gemv(GemvParams& g, bool glu, cudaStream_t st, const char* what) {
+    const int grid = 2 * sm_count();
+    return check_cuda(launch_gemv(g, glu, grid, st), what);
+}
+
+}  // namespace milo
+
+using namespace milo;
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+
+extern "C" const char* milo_status_str(milo_status s) {
+    switch (s) {
+        case MILO_OK: return "ok";
+        case MILO_ERR_INVALID_ARG: return "invalid argument";
+        case MILO_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case MILO_ERR_WORKSPACE: return "workspace or table too small or misaligned";
+        case MILO_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+extern "C" const char* milo_last_error(void) { return g_last_error.c_str(); }
+
+extern "C" int32_t milo_version(void) { return 1; }
+
+extern "C" milo_status milo_table_bytes(int32_t n_projections, size_t* bytes) {
+    clear_error();
+    if (n_projections < 0 || !bytes) return fail(MILO_ERR_INVALID_ARG, "milo_table_bytes: bad argument");
+    *bytes = static_cast<size_t>(n_projections) * sizeof(ProjDev);
+    return MILO_OK;
+}
+
+extern "C" milo_status milo_linear_prepare(milo_linear* lin, const milo_qweight* weights,
+                                           void* device_table, size_t table_bytes) {
+    clear_error();
+    if (!lin || !weights) return fail(MILO_ERR_INVALID_ARG, "milo_linear_prepare: NULL argument");
+    if (lin->group != MILO_GROUP) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "group must be 64");
+    if (lin->n_experts < 1 || lin->n_experts > MILO_MAX_EXPERTS)
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE, "n_experts must be in [1, 256]");
+    milo_status s = check_nk(lin->N, lin->K, "milo_linear_prepare");
+    if (s != MILO_OK) return s;
+    std::vector<ProjDev> t(lin->n_experts);
+    int rmax = 0;
+    for (int e = 0; e < lin->n_experts; ++e) {
+        if ((s = fill_proj(&t[e], weights[e], lin->N, lin->K, kRowsPlain, "milo_linear_prepare")) != MILO_OK)
+            return s;
+        rmax = std::max(rmax, weights[e].rank);
+    }
+    if ((s = upload(device_table, table_bytes, t)) != MILO_OK) return s;
+    lin->max_rank = rmax;
+    lin->table = device_table;
+    return MILO_OK;
+}
+
+extern "C" milo_status milo_layer_prepare(milo_moe_layer* L, const milo_expert* experts,
+                                          void* device_table, size_t table_bytes) {
+    clear_error();
+    if (!L || !experts) return fail(MILO_ERR_INVALID_ARG, "milo_layer_prepare: NULL argument");
+    if (L->group != MILO_GROUP) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "group must be 64");
+    const int n_exp = L->n_routed + L->n_shared;
+    if (L->n_routed < 1 || L->n_shared < 0 || n_exp > MILO_MAX_EXPERTS)
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE, "experts: need n_routed >= 1 and n_routed + n_shared <= 256");
+    if (L->top_k < 1 || L->top_k > L->n_routed || L->top_k > MILO_MAX_TOPK)
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE, "top_k must be in [1, min(n_routed, 16)]");
+    milo_status s;
+    if ((s = check_nk(L->inter, L->hidden, "w1/w3")) != MILO_OK) return s;
+    if ((s = check_nk(L->hidden, L->inter, "w2")) != MILO_OK) return s;
+    if (L->hidden % 4) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "hidden must be a multiple of 4");
+    std::vector<ProjDev> t(3 * static_cast<size_t>(n_exp));
+    int rmax = 0;
+    for (int e = 0; e < n_exp; ++e) {
+        if ((s = fill_proj(&t[3 * e + 0], experts[e].w1, L->inter, L->hidden, kRowsGlu, "w1")) != MILO_OK) return s;
+        if ((s = fill_proj(&t[3 * e + 1], experts[e].w3, L->inter, L->hidden, kRowsGlu, "w3")) != MILO_OK) return s;
+        if ((s = fill_proj(&t[3 * e + 2], experts[e].w2, L->hidden, L->inter, kRowsPlain, "w2")) != MILO_OK) return s;
+        rmax = std::max({rmax, experts[e].w1.rank, experts[e].w3.rank, experts[e].w2.rank});
+    }
+    if ((s = upload(device_table, table_bytes, t)) != MILO_OK) return s;
+    L->max_rank = rmax;
+    L->table = device_table;
+    return MILO_OK;
+}
+
+extern "C" milo_status milo_linear_workspace_bytes(const milo_linear* lin, int32_t T, int32_t k,
+                                                   size_t* bytes) {
+    clear_error();
+    if (!lin || !bytes || T < 0 || k < 1) return fail(MILO_ERR_INVALID_ARG, "milo_linear_workspace_bytes");
+    *bytes = linear_ws(lin, T, k).total;
+    return MILO_OK;
+}
+
+extern "C" milo_status milo_moe_workspace_bytes(const milo_moe_layer* L, int32_t T, size_t* bytes) {
+    clear_error();
+    if (!L || !bytes || T < 0) return fail(MILO_ERR_INVALID_ARG, "milo_moe_workspace_bytes");
+    *bytes = moe_ws(L, T).total;
+    return MILO_OK;
+}
+
+extern "C" size_t milo_moe_h_offset(const milo_moe_layer* L, int32_t T) {
+    return L ? moe_ws(L, T).h : 0;
+}
+
+extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x, milo_dtype x_dt,
+                                           int32_t T, int32_t k, const int32_t* expert_offsets,
+                                           const int32_t* perm, void* y, milo_dtype y_dt, void* ws,
+                                           size_t ws_bytes, int32_t* dev_status, void* stream) {
+    clear_error();
+    if (!lin || !lin->table) return fail(MILO_ERR_INVALID_ARG, "milo_grouped_linear: layer not prepared");
+    if (T < 0 || k < 1 || k > MILO_MAX_TOPK) return fail(MILO_ERR_INVALID_ARG, "milo_grouped_linear: bad T or k");
+    if (x_dt != MILO_F16 && x_dt != MILO_BF16) return fail(MILO_ERR_INVALID_ARG, "x must be fp16 or bf16");
+    if (y_dt != MILO_F16 && y_dt != MILO_BF16 && y_dt != MILO_F32) return fail(MILO_ERR_INVALID_ARG, "bad y dtype");
+    if (!perm && k != 1) return fail(MILO_ERR_INVALID_ARG, "perm may be NULL only with k == 1");
+    if (T == 0) return MILO_OK;
+    if (!x || !y || !expert_offsets || !ws) return fail(MILO_ERR_INVALID_ARG, "milo_grouped_linear: NULL pointer");
+    if (!aligned(x, 16) || !aligned(y, 16)) return fail(MILO_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
+    if (!aligned(ws, 256)) return fail(MILO_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    if (lin->N % 4) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "N must be a multiple of 4");
+    const LinearWs w = linear_ws(lin, T, k);
+    if (ws_bytes < w.total) return fail(MILO_ERR_WORKSPACE, "milo_grouped_linear: workspace too small");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* base = static_cast<char*>(ws);
+    int32_t* grp = reinterpret_cast<int32_t*>(base + w.grp);
+    int32_t* rows = reinterpret_cast<int32_t*>(base + w.rows);
+    int32_t* inv = reinterpret_cast<int32_t*>(base + w.inv);
+
+    RowsParams rp{expert_offsets, perm, grp, rows, inv, dev_status, T, k, lin->n_experts, 0, w.R};
+    milo_status s = check_cuda(launch_rows(rp, st), "rows");
+    if (s != MILO_OK) return s;
+
+    PrepParams pp{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.frag),
+                  reinterpret_cast<float*>(base + w.gsum), dev_status, w.R, lin->K, gpad_of(lin->K),
+                  x_dt == MILO_BF16};
+    if ((s = check_cuda(launch_prep(pp, st), "prep")) != MILO_OK) return s;
+
+    const bool has_t = lin->max_rank > 0;
+    const ProjDev* table = static_cast<const ProjDev*>(lin->table);
+    if (has_t) {
+        LorcParams lp{static_cast<const uint16_t*>(x), rows, table, grp,
+                      reinterpret_cast<uint16_t*>(base + w.t), dev_status, 1, 0, -1,
+                      lin->n_experts, lin->K, w.R, w.tcols, 0, x_dt == MILO_BF16};
+        if ((s = check_cuda(launch_lorc(lp, st), "lorc")) != MILO_OK) return s;
+    }
+
+    GemvParams g;
+    memset(&g, 0, sizeof(g));
+    if ((s = act_maps(g, base + w.frag, base + w.gsum, base + w.t, w.R, lin->K, w.tcols, has_t)) != MILO_OK)
+        return s;
+    g.table = table;
+    g.grp = grp;
+    g.y_part = reinterpret_cast<float*>(base + w.part);
+    g.dev_status = dev_status;
+    g.stride = 1;
+    g.proj_a = 0;
+    g.proj_b = 0;
+    g.n_exp = lin->n_experts;
+    g.N = lin->N;
+    g.K = lin->K;
+    g.R = w.R;
+    g.chunks = (lin->K + kChunkK - 1) / kChunkK;
+    g.splits = w.splits;
+    g.cps = (g.chunks + w.splits - 1) / w.splits;
+    g.has_t = has_t;
+    g.tcols = w.tcols;
+    if ((s = run_gemv(g, false, st, "gemv")) != MILO_OK) return s;
+
+    CombineParams cp{reinterpret_cast<const float*>(base + w.part), inv, nullptr, y, dev_status,
+                     T, k, 0, lin->N, w.R, w.splits, w.R, static_cast<int>(y_dt), 1};
+    return check_cuda(launch_combine(cp, st), "combine");
+}
+
+extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, milo_dtype x_dt,
+                                        int32_t T, const float* topk_w, const int32_t* expert_offsets,
+                                        const int32_t* perm, const int32_t* inv_perm, void* y,
+                                        milo_dtype y_dt, void* ws, size_t ws_bytes,
+                                        int32_t* dev_status, void* stream) {
+    clear_error();
+    if (!L || !L->table) return fail(MILO_ERR_INVALID_ARG, "milo_moe_forward: layer not prepared");
+    if (T < 0) return fail(MILO_ERR_INVALID_ARG, "milo_moe_forward: T must be >= 0");
+    if (x_dt != MILO_F16 && x_dt != MILO_BF16) return fail(MILO_ERR_INVALID_ARG, "x must be fp16 or bf16");
+    if (y_dt != MILO_F16 && y_dt != MILO_BF16 && y_dt != MILO_F32) return fail(MILO_ERR_INVALID_ARG, "bad y dtype");
+    if (T == 0) return MILO_OK;
+    if (!x || !y || !topk_w || !expert_offsets || !perm || !inv_perm || !ws)
+        return fail(MILO_ERR_INVALID_ARG, "milo_moe_forward: NULL pointer");
+    if (!aligned(x, 16) || !aligned(y, 16)) return fail(MILO_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
+    if (!aligned(ws, 256)) return fail(MILO_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    const MoeWs w = moe_ws(L, T);
+    if (ws_bytes < w.total) return fail(MILO_ERR_WORKSPACE, "milo_moe_forward: workspace too small");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* base = static_cast<char*>(ws);
+    const int n_exp = L->n_routed + L->n_shared;
+    const int H = L->hidden, I = L->inter;
+    int32_t* grp = reinterpret_cast<int32_t*>(base + w.grp);
+    int32_t* rows = reinterpret_cast<int32_t*>(base + w.rows);
+    const ProjDev* table = static_cast<const ProjDev*>(L->table);
+    const bool has_t = L->max_rank > 0;
+    milo_status s;
+
+    RowsParams rp{expert_offsets, perm, grp, rows, nullptr, dev_status, T, L->top_k, L->n_routed,
+                  L->n_shared, w.R_routed};
+    if ((s = check_cuda(launch_rows(rp, st), "rows")) != MILO_OK) return s;
+
+    PrepParams px{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.xfrag),
+                  reinterpret_cast<float*>(base + w.xg), dev_status, w.R, H, gpad_of(H), x_dt == MILO_BF16};
+    if ((s = check_cuda(launch_prep(px, st), "prep x")) != MILO_OK) return s;
+    if (has_t) {
+        LorcParams lp{static_cast<const uint16_t*>(x), rows, table, grp,
+                      reinterpret_cast<uint16_t*>(base + w.t13), dev_status, 3, 0, 1, n_exp, H, w.R,
+                      w.tc13, L->max_rank, x_dt == MILO_BF16};
+        if ((s = check_cuda(launch_lorc(lp, st), "lorc w1|w3")) != MILO_OK) return s;
+    }
+
+    GemvParams g1;
+    memset(&g1, 0, sizeof(g1));
+    if ((s = act_maps(g1, base + w.xfrag, base + w.xg, base + w.t13, w.R, H, w.tc13, has_t)) != MILO_OK) return s;
+    g1.table = table;
+    g1.grp = grp;
+    g1.h = reinterpret_cast<uint16_t*>(base + w.h);
+    g1.dev_status = dev_status;
+    g1.stride = 3;
+    g1.proj_a = 0;
+    g1.proj_b = 1;
+    g1.n_exp = n_exp;
+    g1.N = I;
+    g1.K = H;
+    g1.R = w.R;
+    g1.chunks = (H + kChunkK - 1) / kChunkK;
+    g1.splits = 1;
+    g1.cps = g1.chunks;
+    g1.has_t = has_t;
+    g1.tcols = w.tc13;
+    g1.t_col_b = L->max_rank;
+    if ((s = run_gemv(g1, true, st, "gemv w1|w3")) != MILO_OK) return s;
+
+    PrepParams ph{reinterpret_cast<const uint16_t*>(base + w.h), nullptr,
+                  reinterpret_cast<uint16_t*>(base + w.hfrag), reinterpret_cast<float*>(base + w.hg),
+                  dev_status, w.R, I, gpad_of(I), 0};
+    if ((s = check_cuda(launch_prep(ph, st), "prep h")) != MILO_OK) return s;
+    if (has_t) {
+        LorcParams lp{reinterpret_cast<const uint16_t*>(base + w.h), nullptr, table, grp,
+                      reinterpret_cast<uint16_t*>(base + w.t2), dev_status, 3, 2, -1, n_exp, I, w.R,
+                      w.tc2, 0, 0};
+        if ((s = check_cuda(launch_lorc(lp, st), "lorc w2")) != MILO_OK) return s;
+    }
+
+    GemvParams g2;
+    memset(&g2, 0, sizeof(g2));
+    if ((s = act_maps(g2, base + w.hfrag, base + w.hg, base + w.t2, w.R, I, w.tc2, has_t)) != MILO_OK) return s;
+    g2.table = table;
+    g2.grp = grp;
+    g2.y_part = reinterpret_cast<float*>(base + w.part);
+    g2.dev_status = dev_status;
+    g2.stride = 3;
+    g2.proj_a = 2;
+    g2.proj_b = 2;
+    g2.n_exp = n_exp;
+    g2.N = H;
+    g2.K = I;
+    g2.R = w.R;
+    g2.chunks = (I + kChunkK - 1) / kChunkK;
+    g2.splits = w.splits;
+    g2.cps = (g2.chunks + w.splits - 1) / w.splits;
+    g2.has_t = has_t;
+    g2.tcols = w.tc2;
+    if ((s = run_gemv(g2, false, st, "gemv w2")) != MILO_OK) return s;
+
+    CombineParams cp{reinterpret_cast<const float*>(base + w.part), inv_perm, topk_w, y, dev_status,
+                     T, L->top_k, L->n_shared, H, w.R, w.splits, w.R_routed, static_cast<int>(y_dt), 0};
+    return check_cuda(launch_combine(cp, st), "combine");
+}

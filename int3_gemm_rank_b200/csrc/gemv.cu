@@ -1,0 +1,428 @@
+// gemv.cu -- grouped int3 x fp16 GEMM with the low-rank compensator, for
+// decode-sized rows per expert (sm_100a).
+//
+// "MiLo: Efficient Quantized MoE Inference with Mixture of Low-Rank
+// Compensators":
+//   - "MiLo Algorithm: Mixture of Low-Rank Compensators": W_out = W_quant + U V,
+//     so y = x W_quant^T + (x V^T) U^T; the rank differs per expert and may be 0.
+//   - "MiLo Kernel: Efficient Int3 Quantized GEMM Backend": int3 x FP16 GEMM
+//     with dequantisation fused in (no separate dequantisation pass),
+//     asynchronous global loads overlapping the math, and the asymmetric zero
+//     point folded into the kernel.
+//
+// B200 design (not a translation of the page's kernel):
+//   - One producer warp streams each CTA's weight tile with 2-D TMA loads
+//     (packed codes, scales, zeros) plus the prepared activation fragments and
+//     per-group activation sums into a 4-stage shared-memory ring guarded by
+//     mbarriers.  Weights are read from HBM exactly once per token tile.
+//   - Four consumer warps each own 32 weight rows.  A lane reads its 3-word
+//     unit of two rows and extracts code pairs with one LOP3 each (plus one
+//     shift per word): the masked fp16 pattern already is code * 8^i * 2^-24,
+//     and the power of 8 is folded into the activations, which are shared by
+//     all rows.  mma.sync m16n8k16 (A = codes, B = tokens) accumulates
+//     D_g = 2^-24 * sum_k x_k q_k per scale group g; after each group the lane
+//     folds  acc += s * 2^24 * D_g - s * z * sum_k x_k  in fp32.  The zero point
+//     thus costs nothing per weight and the result is exact to fp32 rounding.
+//   - The compensator runs as extra K-steps on the same accumulators:
+//     A = U rows (fp16), B = t = x V^T (fp16, computed beforehand per expert).
+//   - Epilogue: SwiGLU h = silu(a) * b in the w1|w3 kernel (both rows live in
+//     the same lane), or fp32 partial sums per K split for the plain one.
+//   - Work items (expert, row tile, K split, 16-row token tile) are enumerated
+//     on the device from the expert offsets, so the host never synchronises;
+//     CTAs are persistent (two per SM) and walk the items round-robin, the
+//     token tiles of one weight tile being adjacent so that they share L2.
+#include <cuda_runtime.h>
+
+#include "milo_device.cuh"
+#include "milo_kernels.h"
+
+namespace milo {
+
+constexpr int kStages = 4;
+constexpr int kConsumerWarps = 4;
+constexpr int kGemvThreads = 32 * (kConsumerWarps + 1);
+// Stage layout (bytes).  Q tiles are [2 super-blocks][rows][12 words]; the
+// GLU kernel keeps w1's 64 rows at kOffQ and w3's at kOffQB.
+constexpr int kOffQ = 0;
+constexpr int kOffQB = 6144;
+constexpr int kOffS = 12288;       // scale/zero tiles [4 groups][rows] fp16, 2048 B in all
+constexpr int kOffX = 14336;       // activation fragments [2 sb][16 rows][144 fp16]
+constexpr int kOffG = 23552;       // group sums [16 rows][4 groups] f32
+constexpr int kStageBytes = 23808;
+constexpr int kOffUA = 0, kOffUB = 8192, kOffT = 16384;   // compensator stage
+constexpr int kXBytesSB = kTokTile * kFragHalvesPerSB * 2;  // 4608
+constexpr int kBarOffset = kStages * kStageBytes;
+constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 3 * (MILO_MAX_EXPERTS + 1) * 4 + 16;
+
+static_assert(kOffQB == 2 * kRowsGlu * 48, "Q tile layout");
+static_assert(kOffS == 2 * kRowsPlain * 48, "Q tile layout");
+static_assert(kOffG + kTokTile * 4 * 4 == kStageBytes, "stage layout");
+static_assert(kOffT + kTokTile * 2 * MILO_MAX_RANK * 2 <= kStageBytes, "compensator stage");
+
+struct Item {
+    int e, ntile, split, tt;
+};
+
+__device__ __forceinline__ Item decode_item(int it, const int* start, const int* cnt, int n_exp,
+                                            int splits) {
+    int lo = 0, hi = n_exp - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (start[mid] <= it) lo = mid;
+        else hi = mid - 1;
+    }
+    Item r;
+    r.e = lo;
+    const int local = it - start[lo];
+    const int tte = (cnt[lo] + kTokTile - 1) / kTokTile;
+    r.tt = local % tte;
+    const int rest = local / tte;
+    r.split = rest % splits;
+    r.ntile = rest / splits;
+    return r;
+}
+
+// One k16 step of the code part: extract the A fragments of both row tiles
+// and multiply them with the prepared activation fragments of NT n8 tiles.
+template <int S, int NT>
+__device__ __forceinline__ void code_step(const uint32_t (&wd)[2][2][3], const uint32_t (&hw)[2][2][3],
+                                          const uint8_t* xs, int g, int c, float (&dz)[2][2][4]) {
+    constexpr int t0 = sched_word(S, 0), f0 = sched_field(S, 0);
+    constexpr int t1 = sched_word(S, 1), f1 = sched_field(S, 1);
+    uint2 b[NT];
+#pragma unroll
+    for (int n8 = 0; n8 < NT; ++n8)
+        b[n8] = *reinterpret_cast<const uint2*>(
+            xs + ((n8 * 8 + g) * kFragHalvesPerSB + S * 16 + c * 4) * 2);
+#pragma unroll
+    for (int ti = 0; ti < 2; ++ti) {
+        const uint32_t a0 = field<f0>(wd[ti][0][t0], hw[ti][0][t0]);
+        const uint32_t a1 = field<f0>(wd[ti][1][t0], hw[ti][1][t0]);
+        const uint32_t a2 = field<f1>(wd[ti][0][t1], hw[ti][0][t1]);
+        const uint32_t a3 = field<f1>(wd[ti][1][t1], hw[ti][1][t1]);
+#pragma unroll
+        for (int n8 = 0; n8 < NT; ++n8) {
+            if constexpr (S == 0 || S == 4) mma16816_zc(dz[ti][n8], a0, a1, a2, a3, b[n8].x, b[n8].y);
+            else mma16816(dz[ti][n8], a0, a1, a2, a3, b[n8].x, b[n8].y);
+        }
+    }
+}
+
+// acc += s * 2^24 * D_g - s * z * X_g for the scale group `grp` of the stage.
+template <bool GLU, int NT>
+__device__ __forceinline__ void fold_group(float (&acc)[2][2][4], const float (&dz)[2][2][4],
+                                           const uint8_t* st, int grp, const int (&rbase)[2],
+                                           int g, int c) {
+    constexpr int RA = GLU ? kRowsGlu : kRowsPlain;
+    const float* gs = reinterpret_cast<const float*>(st + kOffG);
+    float xg[NT][2];
+#pragma unroll
+    for (int n8 = 0; n8 < NT; ++n8) {
+        xg[n8][0] = gs[(n8 * 8 + 2 * c) * 4 + grp];
+        xg[n8][1] = gs[(n8 * 8 + 2 * c + 1) * 4 + grp];
+    }
+#pragma unroll
+    for (int ti = 0; ti < 2; ++ti) {
+        const __half* S = reinterpret_cast<const __half*>(st + kOffS + (GLU ? ti * 1024 : 0));
+        const __half* Z = S + (GLU ? 256 : 512);
+        float s24[2], nsz[2];
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            const int row = rbase[ti] + g + 8 * rr;
+            const float sv = __half2float(S[grp * RA + row]);
+            const float zv = __half2float(Z[grp * RA + row]);
+            s24[rr] = sv * 16777216.0f;
+            nsz[rr] = -sv * zv;
+        }
+#pragma unroll
+        for (int n8 = 0; n8 < NT; ++n8) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int rr = i >> 1;
+                acc[ti][n8][i] = fmaf(nsz[rr], xg[n8][i & 1], fmaf(s24[rr], dz[ti][n8][i], acc[ti][n8][i]));
+            }
+        }
+    }
+}
+
+template <bool GLU, int NT>
+__device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2][2][4], int warp,
+                                              int lane) {
+    constexpr int RA = GLU ? kRowsGlu : kRowsPlain;
+    const int g = lane >> 2, c = lane & 3;
+    const int rbase[2] = {GLU ? 16 * warp : 32 * warp, GLU ? 16 * warp : 32 * warp + 16};
+    const uint32_t* qt[2] = {reinterpret_cast<const uint32_t*>(st + kOffQ),
+                             reinterpret_cast<const uint32_t*>(st + (GLU ? kOffQB : kOffQ))};
+#pragma unroll
+    for (int sbl = 0; sbl < 2; ++sbl) {
+        uint32_t wd[2][2][3], hw[2][2][3];
+#pragma unroll
+        for (int ti = 0; ti < 2; ++ti)
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                for (int t = 0; t < 3; ++t) {
+                    wd[ti][rr][t] = qt[ti][(sbl * RA + rbase[ti] + g + 8 * rr) * 12 + 3 * c + t];
+                    hw[ti][rr][t] = wd[ti][rr][t] >> 9;
+                }
+        const uint8_t* xs = st + kOffX + sbl * kXBytesSB;
+        float dz[2][2][4];
+        code_step<0, NT>(wd, hw, xs, g, c, dz);
+        code_step<1, NT>(wd, hw, xs, g, c, dz);
+        code_step<2, NT>(wd, hw, xs, g, c, dz);
+        code_step<3, NT>(wd, hw, xs, g, c, dz);
+        fold_group<GLU, NT>(acc, dz, st, 2 * sbl, rbase, g, c);
+        code_step<4, NT>(wd, hw, xs, g, c, dz);
+        code_step<5, NT>(wd, hw, xs, g, c, dz);
+        code_step<6, NT>(wd, hw, xs, g, c, dz);
+        code_step<7, NT>(wd, hw, xs, g, c, dz);
+        code_step<8, NT>(wd, hw, xs, g, c, dz);
+        fold_group<GLU, NT>(acc, dz, st, 2 * sbl + 1, rbase, g, c);
+    }
+}
+
+// Compensator K-steps: acc += U_tile * t^T over the rank (multiple of 8).
+template <bool GLU, int NT>
+__device__ __forceinline__ void lorc_compute(const uint8_t* st, float (&acc)[2][2][4], int warp,
+                                             int lane, int ra, int rb, int tcols, int t_col_b) {
+    const int g = lane >> 2, c = lane & 3;
+    const uint16_t* tt = reinterpret_cast<const uint16_t*>(st + kOffT);
+#pragma unroll
+    for (int ti = 0; ti < 2; ++ti) {
+        const int r = (GLU && ti == 1) ? rb : ra;
+        const uint16_t* U = reinterpret_cast<const uint16_t*>(st + ((GLU && ti == 1) ? kOffUB : kOffUA));
+        const int rbase = GLU ? 16 * warp : 32 * warp + 16 * ti;
+        const int tc0 = (GLU && ti == 1) ? t_col_b : 0;
+        for (int kk = 0; kk < r; kk += 16) {
+            const int col = kk + 2 * c;
+            const bool upper = col + 8 < r;
+            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(U + (rbase + g) * r + col);
+            const uint32_t a1 = *reinterpret_cast<const uint32_t*>(U + (rbase + g + 8) * r + col);
+            const uint32_t a2 = upper ? *reinterpret_cast<const uint32_t*>(U + (rbase + g) * r + col + 8) : 0u;
+            const uint32_t a3 = upper ? *reinterpret_cast<const uint32_t*>(U + (rbase + g + 8) * r + col + 8) : 0u;
+#pragma unroll
+            for (int n8 = 0; n8 < NT; ++n8) {
+                const uint16_t* trow = tt + (n8 * 8 + g) * tcols + tc0;
+                const uint32_t b0 = *reinterpret_cast<const uint32_t*>(trow + col);
+                const uint32_t b1 = upper ? *reinterpret_cast<const uint32_t*>(trow + col + 8) : 0u;
+                mma16816(acc[ti][n8], a0, a1, a2, a3, b0, b1);
+            }
+        }
+    }
+}
+
+template <bool GLU>
+__global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_constant__ GemvParams p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
+    uint64_t* empty = full + kStages;
+    int* start = reinterpret_cast<int*>(empty + kStages);
+    int* cnt = start + (MILO_MAX_EXPERTS + 1);
+    int* row0s = cnt + (MILO_MAX_EXPERTS + 1);
+    volatile int* abort_flag = row0s + (MILO_MAX_EXPERTS + 1);
+
+    constexpr int RA = GLU ? kRowsGlu : kRowsPlain;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles = (p.N + RA - 1) / RA;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        int run = 0;
+        for (int e = 0; e < p.n_exp; ++e) {
+            const int r0 = p.grp[2 * e], m = p.grp[2 * e + 1];
+            const bool ok = m > 0 && r0 >= 0 && r0 + m <= p.R;
+            start[e] = run;
+            cnt[e] = ok ? m : 0;
+            row0s[e] = r0;
+            if (ok) run += ((m + kTokTile - 1) / kTokTile) * n_tiles * p.splits;
+        }
+        start[p.n_exp] = run;
+    }
+    __syncthreads();
+    const int n_items = start[p.n_exp];
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------------ producer
+        if (lane != 0) return;
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+            const Item w = decode_item(it, start, cnt, p.n_exp, p.splits);
+            const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
+            const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
+            const int n0 = w.ntile * RA;
+            const int row0 = row0s[w.e] + w.tt * kTokTile;
+            const int c0 = w.split * p.cps;
+            const int c1 = min(p.chunks, c0 + p.cps);
+            tmap_acquire(&pa->q_map);
+            tmap_acquire(&pa->s_map);
+            tmap_acquire(&pa->z_map);
+            if (GLU) {
+                tmap_acquire(&pb->q_map);
+                tmap_acquire(&pb->s_map);
+                tmap_acquire(&pb->z_map);
+            }
+            for (int ch = c0; ch < c1; ++ch) {
+                if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                    flag(p.dev_status, MILO_DEV_TIMEOUT);
+                    *abort_flag = 1;
+                    return;
+                }
+                uint8_t* st = smem + stage * kStageBytes;
+                uint64_t* fb = &full[stage];
+                mbar_arrive_expect_tx(fb, kStageBytes);
+#pragma unroll
+                for (int sbl = 0; sbl < 2; ++sbl) {
+                    const int sb = 2 * ch + sbl;
+                    tma_load_2d(st + kOffQ + sbl * RA * 48, &pa->q_map, fb, 12 * sb, n0);
+                    if (GLU) tma_load_2d(st + kOffQB + sbl * RA * 48, &pb->q_map, fb, 12 * sb, n0);
+                    tma_load_2d(st + kOffX + sbl * kXBytesSB, &p.x_map, fb, kFragHalvesPerSB * sb, row0);
+                }
+                if (GLU) {
+                    tma_load_2d(st + kOffS, &pa->s_map, fb, n0, 4 * ch);
+                    tma_load_2d(st + kOffS + 512, &pa->z_map, fb, n0, 4 * ch);
+                    tma_load_2d(st + kOffS + 1024, &pb->s_map, fb, n0, 4 * ch);
+                    tma_load_2d(st + kOffS + 1536, &pb->z_map, fb, n0, 4 * ch);
+                } else {
+                    tma_load_2d(st + kOffS, &pa->s_map, fb, n0, 4 * ch);
+                    tma_load_2d(st + kOffS + 1024, &pa->z_map, fb, n0, 4 * ch);
+                }
+                tma_load_2d(st + kOffG, &p.g_map, fb, 4 * ch, row0);
+                if (++stage == kStages) { stage = 0; phase ^= 1; }
+            }
+            const int ra = pa->rank, rb = GLU ? pb->rank : 0;
+            if (w.split == 0 && p.has_t && (ra > 0 || rb > 0)) {
+                if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                    flag(p.dev_status, MILO_DEV_TIMEOUT);
+                    *abort_flag = 1;
+                    return;
+                }
+                uint8_t* st = smem + stage * kStageBytes;
+                uint64_t* fb = &full[stage];
+                const uint32_t bytes = ra * RA * 2 + (GLU ? rb * RA * 2 : 0) + p.tcols * kTokTile * 2;
+                mbar_arrive_expect_tx(fb, bytes);
+                if (ra > 0) {
+                    tmap_acquire(&pa->u_map);
+                    tma_load_2d(st + kOffUA, &pa->u_map, fb, 0, n0);
+                }
+                if (GLU && rb > 0) {
+                    tmap_acquire(&pb->u_map);
+                    tma_load_2d(st + kOffUB, &pb->u_map, fb, 0, n0);
+                }
+                tma_load_2d(st + kOffT, &p.t_map, fb, 0, row0);
+                if (++stage == kStages) { stage = 0; phase ^= 1; }
+            }
+        }
+        return;
+    }
+
+    // -------------------------------------------------------------- consumers
+    int stage = 0;
+    uint32_t phase = 0;
+    const int g = lane >> 2, c = lane & 3;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+        const Item w = decode_item(it, start, cnt, p.n_exp, p.splits);
+        const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
+        const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
+        const int n0 = w.ntile * RA;
+        const int row0 = row0s[w.e] + w.tt * kTokTile;
+        const int ntok = min(kTokTile, cnt[w.e] - w.tt * kTokTile);
+        const int c0 = w.split * p.cps;
+        const int c1 = min(p.chunks, c0 + p.cps);
+        float acc[2][2][4];
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[a][b][i] = 0.0f;
+
+        for (int ch = c0; ch < c1; ++ch) {
+            if (!mbar_wait(&full[stage], phase)) {
+                flag(p.dev_status, MILO_DEV_TIMEOUT);
+                *abort_flag = 1;
+                return;
+            }
+            const uint8_t* st = smem + stage * kStageBytes;
+            if (ntok > 8) chunk_compute<GLU, 2>(st, acc, warp, lane);
+            else chunk_compute<GLU, 1>(st, acc, warp, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+        const int ra = pa->rank, rb = GLU ? pb->rank : 0;
+        if (w.split == 0 && p.has_t && (ra > 0 || rb > 0)) {
+            if (!mbar_wait(&full[stage], phase)) {
+                flag(p.dev_status, MILO_DEV_TIMEOUT);
+                *abort_flag = 1;
+                return;
+            }
+            const uint8_t* st = smem + stage * kStageBytes;
+            if (ntok > 8) lorc_compute<GLU, 2>(st, acc, warp, lane, ra, rb, p.tcols, p.t_col_b);
+            else lorc_compute<GLU, 1>(st, acc, warp, lane, ra, rb, p.tcols, p.t_col_b);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+
+        // ------------------------------------------------------------ epilogue
+        if constexpr (GLU) {
+            int32_t st = 0;
+#pragma unroll
+            for (int n8 = 0; n8 < 2; ++n8)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int f = n0 + 16 * warp + g + 8 * (i >> 1);
+                    const int tok = n8 * 8 + 2 * c + (i & 1);
+                    if (tok < ntok && f < p.N) {
+                        const float a = acc[0][n8][i], b = acc[1][n8][i];
+                        const float hv = a / (1.0f + expf(-a)) * b;
+                        const __half hh = __float2half_rn(hv);
+                        if (!isfinite(hv)) st |= MILO_DEV_NONFINITE;
+                        else if (__hisinf(hh)) st |= MILO_DEV_FP16_RANGE;
+                        p.h[static_cast<size_t>(row0 + tok) * p.N + f] = __half_as_ushort(hh);
+                    }
+                }
+            flag(p.dev_status, st);
+        } else {
+            float* out = p.y_part + static_cast<size_t>(w.split) * p.R * p.N;
+#pragma unroll
+            for (int ti = 0; ti < 2; ++ti)
+#pragma unroll
+                for (int n8 = 0; n8 < 2; ++n8)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int n = n0 + 32 * warp + 16 * ti + g + 8 * (i >> 1);
+                        const int tok = n8 * 8 + 2 * c + (i & 1);
+                        if (tok < ntok && n < p.N)
+                            out[static_cast<size_t>(row0 + tok) * p.N + n] = acc[ti][n8][i];
+                    }
+        }
+    }
+}
+
+size_t gemv_smem_bytes(bool) { return kSmemBytes; }
+
+cudaError_t launch_gemv(const GemvParams& p, bool glu, int grid, cudaStream_t s) {
+    // The shared-memory opt-in is a per-device function attribute.
+    static bool configured[64][2] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !configured[dev][glu]) {
+        e = glu ? cudaFuncSetAttribute(gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)
+                : cudaFuncSetAttribute(gemv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev][glu] = true;
+    }
+    if (glu) gemv_kernel<true><<<grid, kGemvThreads, kSmemBytes, s>>>(p);
+    else gemv_kernel<false><<<grid, kGemvThreads, kSmemBytes, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace milo

@@ -1,0 +1,194 @@
+// milo_device.cuh -- device helpers shared by the sm_100a kernels of libmilo.
+//
+// PTX wrappers (mbarrier, TMA bulk-tensor loads, mma.sync), the int3 field
+// extraction of the packing format and its register schedule, and small
+// conversions.  Nothing here is shared with the CPU oracle.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/milo.h"
+
+namespace milo {
+
+// ---------------------------------------------------------------------------
+// status
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void flag(int32_t* st, int32_t bits) {
+    if (st != nullptr && bits) atomicOr(st, bits);
+}
+
+// ---------------------------------------------------------------------------
+// conversions
+// ---------------------------------------------------------------------------
+
+// Activation element -> fp16, round to nearest even.  bf16 values between
+// 2^-17 and 65504 in magnitude convert exactly; larger ones set FP16_RANGE.
+__device__ __forceinline__ __half to_half(uint16_t bits, bool is_bf16, int32_t& st) {
+    float f;
+    if (is_bf16) {
+        f = __uint_as_float(static_cast<uint32_t>(bits) << 16);
+    } else {
+        f = __half2float(__ushort_as_half(bits));
+    }
+    if (!isfinite(f)) st |= MILO_DEV_NONFINITE;
+    else if (fabsf(f) > 65504.0f) st |= MILO_DEV_FP16_RANGE;
+    return __float2half_rn(f);
+}
+
+// ---------------------------------------------------------------------------
+// int3 format: field extraction
+// ---------------------------------------------------------------------------
+//
+// A word holds five 3-bit fields in each 16-bit half (bits 3i..3i+2 and
+// 16+3i..16+3i+2, i = 0..4) plus one spare bit per half (bits 15 and 31).
+// Masking a field that lies in bits 0..8 of a half leaves an fp16 whose value
+// is code * 8^i * 2^-24 (fields 0, 1, 2: the pattern is an integer below 2^11,
+// and fp16 patterns below 2^11 are that integer times 2^-24).  Fields 3 and 4
+// and the spare bit are brought down by one shift of 9.  So each pair of codes
+// costs one LOP3 (plus one shared shift per word) and the power-of-8 factor is
+// undone on the activation side, where it costs nothing per weight.
+constexpr uint32_t kField0 = 0x00070007u;   // bits 0-2   -> code * 1
+constexpr uint32_t kField1 = 0x00380038u;   // bits 3-5   -> code * 8
+constexpr uint32_t kField2 = 0x01C001C0u;   // bits 6-8   -> code * 64
+constexpr uint32_t kSpare = 0x00400040u;    // bit 15 >> 9 -> bit * 64
+
+// Extracted register f (0..5) of a word; `hi` is the word shifted right by 9.
+template <int F>
+__device__ __forceinline__ uint32_t field(uint32_t w, uint32_t hi) {
+    if constexpr (F == 0) return w & kField0;
+    else if constexpr (F == 1) return w & kField1;
+    else if constexpr (F == 2) return w & kField2;
+    else if constexpr (F == 3) return hi & kField0;
+    else if constexpr (F == 4) return hi & kField1;
+    else return hi & kSpare;
+}
+
+// Register schedule of one 3-word unit over the nine k16 MMA steps of a
+// 128-code super-block.  Step s uses register kSchedWord/kSchedField[s][0]
+// for A-fragment slots (2c, 2c+1) and [s][1] for slots (2c+8, 2c+9).  Steps
+// 0..3 cover the first scale group (unit codes u_0..u_15), steps 4..8 the
+// second (u_16..u_29 and the three spare bits of u_30/u_31).
+__host__ __device__ constexpr int sched_word(int s, int h) {
+    constexpr int w[9][2] = {{0, 0}, {0, 0}, {0, 1}, {1, 1}, {1, 1},
+                             {2, 2}, {2, 2}, {2, 0}, {1, 2}};
+    return w[s][h];
+}
+__host__ __device__ constexpr int sched_field(int s, int h) {
+    constexpr int f[9][2] = {{0, 1}, {2, 3}, {4, 0}, {1, 2}, {3, 4},
+                             {0, 1}, {2, 3}, {4, 5}, {5, 5}};
+    return f[s][h];
+}
+// Unit code index of the low half of register (word t, field f); the high
+// half holds the next code.  Spare registers carry bit t of u_30 (low) and
+// u_31 (high).
+__host__ __device__ constexpr int reg_code(int t, int f) { return f < 5 ? 10 * t + 2 * f : 30; }
+// Offset inside the 128-code super-block of unit code m of unit c.
+__host__ __device__ constexpr int unit_k(int c, int m) {
+    return m < 16 ? 16 * c + m : 64 + 16 * c + (m - 16);
+}
+// Factor applied to the activation paired with register (t, f): the inverse of
+// the power of 8 left in the extracted value, or 2^t / 64 for the spare bits.
+__host__ __device__ constexpr float act_scale(int t, int f) {
+    return f == 0 || f == 3 ? 1.0f
+         : f == 1 || f == 4 ? 0.125f
+         : f == 2           ? 0.015625f
+                            : (float)(1 << t) * 0.015625f;
+}
+// Fragment layout of the prepared activations: per row, per super-block,
+// 9 steps x 4 lanes-in-quad (c) x 4 fp16 = 144 fp16 (288 bytes).
+constexpr int kFragHalvesPerSB = 144;
+
+// ---------------------------------------------------------------------------
+// PTX: mbarrier
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: each try_wait suspends for a hardware-chosen interval, so the
+// limit below amounts to well over a second before the wait gives up.
+constexpr uint32_t kWaitLimit = 1u << 24;
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// ---------------------------------------------------------------------------
+// PTX: TMA (no multicast anywhere in this library)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void tmap_acquire(const CUtensorMap* map) {
+    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;"
+                 ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+          "r"(x), "r"(y)
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// PTX: warp-level MMA  D[16x8] (+)= A[16x16] * B[16x8], fp16 in, fp32 accumulate
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma16816_zc(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                            uint32_t a3, uint32_t b0, uint32_t b1) {
+    float z = 0.0f;
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
+}
+
+}  // namespace milo

@@ -1,0 +1,176 @@
+// pack.cu -- int3 quantise + pack, and the field-extraction unpack.
+//
+// "MiLo: Efficient Quantized MoE Inference with Mixture of Low-Rank
+// Compensators", section "MiLo Kernel: Efficient Int3 Quantized GEMM Backend":
+// 32 three-bit values per three 32-bit words, no wasted bit, asymmetric
+// dequantisation with a zero point.  The quantiser is round-to-nearest
+// asymmetric min/max (the paper starts from HQQ; synthetic weights use RTN).
+#include <cuda_runtime.h>
+
+#include "milo_device.cuh"
+#include "milo_host.h"
+
+namespace milo {
+
+// One thread per (row, 128-code super-block): two scale groups.
+__global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ W, int N, int K,
+                                                   uint32_t* __restrict__ Q,
+                                                   uint16_t* __restrict__ scale,
+                                                   uint16_t* __restrict__ zero,
+                                                   int32_t* __restrict__ dev_status) {
+    const int SB = K / 128;
+    const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (gid >= static_cast<long long>(N) * SB) return;
+    const int n = static_cast<int>(gid / SB);
+    const int b = static_cast<int>(gid % SB);
+    const uint16_t* w = W + static_cast<size_t>(n) * K + static_cast<size_t>(b) * 128;
+
+    int32_t st = 0;
+    uint8_t q[128];
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        float mn = INFINITY, mx = -INFINITY;
+        for (int i = 0; i < 64; ++i) {
+            const float v = __half2float(__ushort_as_half(w[64 * g + i]));
+            if (!isfinite(v)) st |= MILO_DEV_NONFINITE;
+            if (v < mn) mn = v;
+            if (v > mx) mx = v;
+        }
+        const float range = __fsub_rn(mx, mn);
+        __half sh = __float2half_rn(__fdiv_rn(range, 7.0f));
+        if ((__half_as_ushort(sh) & 0x7FFF) == 0) sh = __ushort_as_half(0x3C00);   // s := 1
+        const float s = __half2float(sh);
+        const __half zh = __float2half_rn(__fdiv_rn(-mn, s));
+        const float z = __half2float(zh);
+        if (!isfinite(s) || !isfinite(z)) st |= MILO_DEV_FP16_RANGE;
+        const int j = 2 * b + g;
+        scale[static_cast<size_t>(j) * N + n] = __half_as_ushort(sh);
+        zero[static_cast<size_t>(j) * N + n] = __half_as_ushort(zh);
+        for (int i = 0; i < 64; ++i) {
+            const float v = __fadd_rn(__fdiv_rn(__half2float(__ushort_as_half(w[64 * g + i])), s), z);
+            float r = rintf(v);
+            if (!(r >= 0.0f)) r = 0.0f;
+            if (r > 7.0f) r = 7.0f;
+            q[64 * g + i] = static_cast<uint8_t>(r);
+        }
+    }
+
+    // Place the 128 codes: unit c, unit code m -> word 3c + t, see milo.h.
+    uint32_t words[12];
+#pragma unroll
+    for (int i = 0; i < 12; ++i) words[i] = 0u;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int m = 0; m < 30; ++m) {
+            const int t = m / 10, r = m % 10;
+            const int pos = 16 * (r & 1) + 3 * (r >> 1);
+            words[3 * c + t] |= static_cast<uint32_t>(q[unit_k(c, m)]) << pos;
+        }
+        const uint32_t u30 = q[unit_k(c, 30)], u31 = q[unit_k(c, 31)];
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+            words[3 * c + t] |= (((u30 >> t) & 1u) << 15) | (((u31 >> t) & 1u) << 31);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(Q + static_cast<size_t>(n) * (3 * K / 32) + 12 * b);
+    dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+    dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+    dst[2] = make_uint4(words[8], words[9], words[10], words[11]);
+    flag(dev_status, st);
+}
+
+// One thread per (row, super-block, unit): recover the 32 codes of a unit with
+// the register-level extraction of the GEMM (field masks, one shift by 9, the
+// nine-step schedule), so that its bit-exact parity covers that logic.
+template <int S, int H>
+__device__ __forceinline__ void unpack_reg(const uint32_t (&w)[3], const uint32_t (&hi)[3],
+                                           uint8_t (&u)[32], uint32_t& u30, uint32_t& u31) {
+    constexpr int t = sched_word(S, H), f = sched_field(S, H);
+    const uint32_t r = field<f>(w[t], hi[t]);
+    const uint32_t lo = r & 0xFFFFu, up = r >> 16;
+    if constexpr (f < 5) {
+        constexpr int sh = (f == 0 || f == 3) ? 0 : (f == 1 || f == 4) ? 3 : 6;
+        constexpr int m = reg_code(t, f);
+        u[m] = static_cast<uint8_t>(lo >> sh);
+        u[m + 1] = static_cast<uint8_t>(up >> sh);
+    } else {
+        u30 |= (lo >> 6) << t;
+        u31 |= (up >> 6) << t;
+    }
+}
+
+template <int S>
+__device__ __forceinline__ void unpack_step(const uint32_t (&w)[3], const uint32_t (&hi)[3],
+                                            uint8_t (&u)[32], uint32_t& u30, uint32_t& u31) {
+    unpack_reg<S, 0>(w, hi, u, u30, u31);
+    unpack_reg<S, 1>(w, hi, u, u30, u31);
+}
+
+__global__ void __launch_bounds__(128) unpack_kernel(const uint32_t* __restrict__ Q, int N, int K,
+                                                     uint8_t* __restrict__ codes) {
+    const int SB = K / 128;
+    const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (gid >= static_cast<long long>(N) * SB * 4) return;
+    const int c = static_cast<int>(gid % 4);
+    const long long nb = gid / 4;
+    const int n = static_cast<int>(nb / SB), b = static_cast<int>(nb % SB);
+    const uint32_t* src = Q + static_cast<size_t>(n) * (3 * K / 32) + 12 * b + 3 * c;
+    uint32_t w[3] = {src[0], src[1], src[2]};
+    uint32_t hi[3] = {w[0] >> 9, w[1] >> 9, w[2] >> 9};
+    uint8_t u[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) u[i] = 0xFF;   // a code the schedule misses stays 0xFF
+    uint32_t u30 = 0, u31 = 0;
+    unpack_step<0>(w, hi, u, u30, u31);
+    unpack_step<1>(w, hi, u, u30, u31);
+    unpack_step<2>(w, hi, u, u30, u31);
+    unpack_step<3>(w, hi, u, u30, u31);
+    unpack_step<4>(w, hi, u, u30, u31);
+    unpack_step<5>(w, hi, u, u30, u31);
+    unpack_step<6>(w, hi, u, u30, u31);
+    unpack_step<7>(w, hi, u, u30, u31);
+    unpack_step<8>(w, hi, u, u30, u31);
+    u[30] = static_cast<uint8_t>(u30);
+    u[31] = static_cast<uint8_t>(u31);
+    uint8_t* out = codes + static_cast<size_t>(n) * K + 128 * b;
+#pragma unroll
+    for (int m = 0; m < 32; ++m) out[unit_k(c, m)] = u[m];
+}
+
+}  // namespace milo
+
+using namespace milo;
+
+extern "C" milo_status milo_pack(const uint16_t* W, int32_t N, int32_t K, int32_t group,
+                                 uint32_t* Q, uint16_t* scale, uint16_t* zero,
+                                 int32_t* dev_status, void* stream) {
+    clear_error();
+    if (!W || !Q || !scale || !zero) return fail(MILO_ERR_INVALID_ARG, "milo_pack: NULL pointer");
+    if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, "milo_pack: N and K must be positive");
+    if (group != MILO_GROUP) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_pack: group must be 64");
+    if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_pack: K must be a multiple of 128");
+    if (!aligned(Q, 16) || !aligned(W, 2))
+        return fail(MILO_ERR_INVALID_ARG, "milo_pack: Q must be 16-byte aligned");
+    const long long threads = static_cast<long long>(N) * (K / 128);
+    const int block = 128;
+    const long long grid = (threads + block - 1) / block;
+    if (grid > 0x7FFFFFFFLL) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_pack: too large");
+    pack_kernel<<<static_cast<unsigned>(grid), block, 0, static_cast<cudaStream_t>(stream)>>>(
+        W, N, K, Q, scale, zero, dev_status);
+    return check_launch("milo_pack");
+}
+
+extern "C" milo_status milo_unpack(const uint32_t* Q, int32_t N, int32_t K, uint8_t* codes,
+                                   void* stream) {
+    clear_error();
+    if (!Q || !codes) return fail(MILO_ERR_INVALID_ARG, "milo_unpack: NULL pointer");
+    if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, "milo_unpack: N and K must be positive");
+    if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_unpack: K must be a multiple of 128");
+    const long long threads = static_cast<long long>(N) * (K / 128) * 4;
+    const int block = 128;
+    const long long grid = (threads + block - 1) / block;
+    if (grid > 0x7FFFFFFFLL) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_unpack: too large");
+    unpack_kernel<<<static_cast<unsigned>(grid), block, 0, static_cast<cudaStream_t>(stream)>>>(
+        Q, N, K, codes);
+    return check_launch("milo_unpack");
+}

@@ -329,11 +329,11 @@ static void* linear_rows(void* arg) {
     for (int n = J->n0; n < J->n1; ++n) {
         /* scalar unpack and dequantisation of row n */
         milo_ref_unpack(J->P->Q + (size_t)n * W, 1, K, codes);
-        for (int k = 0; k < K; ++k) {
-            int j = k / J->group;
+        for (int j = 0; j < K / J->group; ++j) {
             double s = milo_ref_h2d(J->P->scale[(size_t)j * J->N + n]);
             double z = milo_ref_h2d(J->P->zero[(size_t)j * J->N + n]);
-            wrow[k] = ((double)codes[k] - z) * s;
+            for (int k = j * J->group; k < (j + 1) * J->group; ++k)
+                wrow[k] = ((double)codes[k] - z) * s;
         }
         for (int m = 0; m < J->M; ++m) {
             const double* x = J->X + (size_t)m * K;

@@ -1,0 +1,94 @@
+"""The C-ABI library builds, loads and exports every entry point that
+include/milo.h declares; host-side argument validation (no GPU needed)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "milo.h")).read()
+    return sorted(set(re.findall(r"^MILO_API[^;(]*?\b(milo_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def milo():
+    from int3_gemm_rank_b200 import build
+    build.build()
+    import int3_gemm_rank_b200 as m
+    return m
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for required in ("milo_pack", "milo_route", "milo_moe_forward", "milo_grouped_linear",
+                     "milo_layer_prepare", "milo_moe_workspace_bytes"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(milo):
+    L = milo.lib()
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert set(milo.EXPORTS) == set(_declared())
+
+
+def test_status_strings_and_version(milo):
+    L = milo.lib()
+    assert L.milo_version() >= 1
+    assert L.milo_status_str(0) == b"ok"
+    assert b"shape" in L.milo_status_str(2)
+
+
+def test_host_validation_rejects_before_launch(milo):
+    L = milo.lib()
+    fake = C.c_void_p(0x1000)
+    # group != 64
+    assert L.milo_pack(fake, 16, 128, 32, fake, fake, fake, None, None) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    # K not a multiple of 128
+    assert L.milo_pack(fake, 16, 100, 64, fake, fake, fake, None, None) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    assert b"multiple of 128" in L.milo_last_error()
+    # NULL pointers
+    assert L.milo_pack(None, 16, 128, 64, fake, fake, fake, None, None) == milo.MILO_ERR_INVALID_ARG
+    # router limits
+    assert L.milo_route(fake, 4, 300, 2, 0, fake, fake, fake, fake, fake, None, None) == \
+        milo.MILO_ERR_UNSUPPORTED_SHAPE
+    assert L.milo_route(fake, 4, 8, 9, 0, fake, fake, fake, fake, fake, None, None) == \
+        milo.MILO_ERR_UNSUPPORTED_SHAPE
+    assert L.milo_route(fake, 4, 8, 2, 0x80, fake, fake, fake, fake, fake, None, None) == \
+        milo.MILO_ERR_INVALID_ARG
+
+
+def test_prepare_validates_shapes_and_ranks(milo):
+    L = milo.lib()
+    nb = C.c_size_t()
+    assert L.milo_table_bytes(3, C.byref(nb)) == 0 and nb.value % 64 == 0 and nb.value > 0
+    fake = 0x10000
+    w = milo.milo_qweight(fake, fake, fake, None, None, 12)   # rank not a multiple of 8
+    lin = milo.milo_linear(64, 128, 1, 64, 0, None)
+    assert L.milo_linear_prepare(C.byref(lin), C.byref(w), C.c_void_p(fake), 1 << 20) == \
+        milo.MILO_ERR_UNSUPPORTED_SHAPE
+    lin = milo.milo_linear(64, 200, 1, 64, 0, None)            # K % 128
+    w = milo.milo_qweight(fake, fake, fake, None, None, 0)
+    assert L.milo_linear_prepare(C.byref(lin), C.byref(w), C.c_void_p(fake), 1 << 20) == \
+        milo.MILO_ERR_UNSUPPORTED_SHAPE
+    lin = milo.milo_linear(64, 128, 1, 32, 0, None)            # group
+    assert L.milo_linear_prepare(C.byref(lin), C.byref(w), C.c_void_p(fake), 1 << 20) == \
+        milo.MILO_ERR_UNSUPPORTED_SHAPE
+    layer = milo.milo_moe_layer(4096, 14336, 8, 0, 9, 64, 0, None)   # top_k > n_routed
+    e = milo.milo_expert(w, w, w)
+    assert L.milo_layer_prepare(C.byref(layer), C.byref(e), C.c_void_p(fake), 1 << 20) == \
+        milo.MILO_ERR_UNSUPPORTED_SHAPE
+
+
+def test_workspace_sizes_grow_with_tokens(milo):
+    L = milo.lib()
+    layer = milo.milo_moe_layer(4096, 14336, 8, 0, 2, 64, 64, None)
+    a, b = C.c_size_t(), C.c_size_t()
+    assert L.milo_moe_workspace_bytes(C.byref(layer), 16, C.byref(a)) == 0
+    assert L.milo_moe_workspace_bytes(C.byref(layer), 8192, C.byref(b)) == 0
+    assert 0 < a.value < b.value
+    assert L.milo_moe_h_offset(C.byref(layer), 16) % 256 == 0

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "milo_oracle.c")
 
 MUTANTS = {
-    "dequant_sign": ("((double)codes[k] - z) * s", "(z - (double)codes[k]) * s"),
+    "dequant_sign": ("wrow[k] = ((double)codes[k] - z) * s;", "wrow[k] = (z - (double)codes[k]) * s;"),
     "drop_lorc": ("J->Y[(size_t)m * J->N + n] = acc + lorc;", "J->Y[(size_t)m * J->N + n] = acc;"),
     "transposed_U": ("J->P->U[(size_t)n * r + p]", "J->P->U[(size_t)p * J->N + n]"),
     "zero_not_negated": ("float z_f = -mn / s;", "float z_f = mn / s;"),
