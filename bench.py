@@ -1,0 +1,549 @@
+#!/usr/bin/env python
+"""Benchmark: MoE layer tokens/s and achieved HBM bandwidth of the int3 +
+low-rank-compensator forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl milo|reference]
+                    [--workload mixtral|deepseek|prefill|single|sweep256]
+
+One step = one pass of the whole hot path over one batch of synthetic tokens:
+router (top-k + grouping) -> activation preparation -> compensator
+down-projection -> grouped int3 GEMM w1|w3 + SwiGLU -> preparation of h ->
+compensator down-projection -> grouped int3 GEMM w2 -> weighted combine.
+Weight packing is offline and not timed.
+
+Default workload: the Mixtral-8x7B-shaped decode layer (H 4096, I 14336, 8
+experts, top-2, ranks drawn from {0,16,32,64}, 16 bf16 tokens).  Its packed
+weights (~0.6 GB) are larger than the 126 MB L2, so every step streams them
+from HBM; no flush is needed.
+
+Multi-GPU: each rank runs its own replica on its own batch (the layer has no
+cross-GPU exchange on one node), the time is the max over ranks and `value`
+counts the tokens of all ranks ("weak" scaling).
+
+--impl reference times the CPU oracle (plain C, fp64) on the host cores, each
+step a bounded sample of tokens of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "MoE layer tokens/s and achieved HBM TB/s (% roofline) for int3+LoRC forward"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (also exercised by the gloo tests on CPU)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def dist_init(backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    rank, local, world = dist_env()
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, local, world
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.out = open(f"/tmp/milo_clocks_{os.getpid()}.csv", "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=self.out,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.out.name) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+        os.unlink(self.out.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        power = [num(r[3]) or 0.0 for r in rows]
+        pmax = max(power) if power else 0.0
+        load = [num(r[1]) for r, pw in zip(rows, power) if pw >= 0.5 * pmax and num(r[1]) is not None]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(load or sm) if (load or sm) else None,
+                "sm_max_mhz": num(rows[0][2]), "reasons": reasons, "samples": len(rows),
+                "power_w_max": pmax}
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+
+def make_workload(name: str, experts: int | None = None, tokens: int | None = None):
+    """The named workload; `experts` / `tokens` shrink it for profiler captures."""
+    if name == "mixtral":
+        return wl.mixtral(T=tokens or 16, n_experts=experts or 8)
+    if name == "deepseek":
+        return wl.deepseek(T=tokens or 64)
+    if name == "prefill":
+        return wl.prefill(T=tokens or 8192, n_experts=experts or 8)
+    raise ValueError(name)
+
+
+def describe(wk) -> str:
+    return (f"{wk.name}: H{wk.hidden} I{wk.inter} E{wk.n_routed}+{wk.n_shared}shared top{wk.top_k} "
+            f"T{wk.T} int3 g64 ranks={list(map(int, wk.ranks))}")
+
+
+def gpu_layer(milo, wk, torch):
+    experts = []
+    for e in range(wk.n_experts):
+        d = {}
+        for n in ("w1", "w3", "w2"):
+            P = wk.experts[e][n]
+
+            def dev(a):
+                return torch.from_numpy(a.view(np.int16)).view(torch.float16).cuda()
+            d[n] = milo.QWeight.quantize(dev(P.W), dev(P.U) if P.rank else None,
+                                         dev(P.V) if P.rank else None)
+        experts.append(d)
+    torch.cuda.synchronize()
+    return milo.MoELayer(experts, wk.n_routed, wk.n_shared, wk.top_k)
+
+
+def layer_bytes(wk, counts) -> dict:
+    """Algorithmic HBM bytes of one step: every active expert's packed codes
+    (3/8 B per weight), fp16 scale and zero (4/64 B per weight), compensator U
+    and V (fp16), plus activations in and out, for each kernel."""
+    H, I = wk.hidden, wk.inter
+    active = [e for e in range(wk.n_routed) if counts[e] > 0] + list(range(wk.n_routed, wk.n_experts))
+    rows = int(sum(counts[:wk.n_routed])) + wk.n_shared * wk.T
+    qz = lambda n, k: n * k * 3 // 8 + 2 * (k // 64) * n * 2   # codes + scale + zero
+    glu = dict(weights=0, lorc_u=0, lorc_v=0)
+    w2 = dict(weights=0, lorc_u=0, lorc_v=0)
+    for e in active:
+        r1, r3, r2 = (wk.experts[e][n].rank for n in ("w1", "w3", "w2"))
+        glu["weights"] += 2 * qz(I, H)
+        glu["lorc_u"] += (r1 + r3) * I * 2
+        glu["lorc_v"] += (r1 + r3) * H * 2
+        w2["weights"] += qz(H, I)
+        w2["lorc_u"] += r2 * H * 2
+        w2["lorc_v"] += r2 * I * 2
+    act_x = rows * H * 2
+    act_h = rows * I * 2
+    glu_kernel = glu["weights"] + glu["lorc_u"] + act_x + act_h + rows * 2 * 64 * 2
+    w2_kernel = w2["weights"] + w2["lorc_u"] + act_h + rows * H * 4
+    step = (glu["weights"] + glu["lorc_u"] + glu["lorc_v"] + w2["weights"] + w2["lorc_u"] + w2["lorc_v"]
+            + wk.T * H * 2 + act_x + 2 * act_h + wk.T * H * 2)
+    return {"glu_kernel": glu_kernel, "w2_kernel": w2_kernel, "step": step,
+            "weights_only": glu["weights"] + w2["weights"], "active_experts": len(active), "rows": rows}
+
+
+def peaks() -> dict:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in ("int3_gemm_rank_b200/csrc/gemv.cu", "int3_gemm_rank_b200/csrc/milo_device.cuh",
+                "int3_gemm_rank_b200/csrc/milo_kernels.h"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(name: str):
+    """DRAM bytes per launch of the GEMM kernel from the committed ncu summary,
+    or None when the summary is missing or the kernel source changed since."""
+    path = os.path.join(ROOT, "profiles", name)
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and line.startswith("- "):
+                    k, v = line[2:].split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+            return None
+        return float(kv["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs
+# ---------------------------------------------------------------------------
+
+def oracle_sample_step(wk, tokens, ref_cache, nthreads):
+    """Run the oracle's full layer on `tokens` (routing included); returns seconds."""
+    import oracle
+    L = wk.logits[tokens]
+    t0 = time.perf_counter()
+    ids, w, *_ = oracle.route(L, wk.top_k, wk.renorm)
+    need = sorted(set(int(e) for e in ids.ravel())) + list(range(wk.n_routed, wk.n_experts))
+    for e in need:
+        if e not in ref_cache:
+            raise RuntimeError("expert not prepared")
+    experts = [ref_cache.get(e) or ref_cache[need[0]] for e in range(wk.n_experts)]
+    oracle.moe_forward(wk.x[tokens], wk.x_dtype == "bf16", ids, w, experts, wk.n_routed, wk.n_shared,
+                       wk.hidden, wk.inter, nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def prepare_oracle_experts(wk, experts_needed):
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    jobs = [(e, n) for e in experts_needed for n in ("w1", "w3", "w2")]
+    with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as ex:
+        res = list(ex.map(lambda j: oracle.quantize_projection(wk.experts[j[0]][j[1]].W,
+                                                               wk.experts[j[0]][j[1]].U,
+                                                               wk.experts[j[0]][j[1]].V), jobs))
+    cache = {}
+    for (e, n), p in zip(jobs, res):
+        cache.setdefault(e, {})[n] = p
+    return cache
+
+
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def sample_tokens(wk, n: int, seed: int) -> np.ndarray:
+    return np.sort(np.random.default_rng(seed).choice(wk.T, size=min(n, wk.T), replace=False))
+
+
+def cpu_baseline(wk, n_tokens: int = 4, passes: int = 3, budget_s: float = 25.0) -> dict:
+    """The oracle, as it stands, on the host cores: `passes` full-layer passes
+    over `n_tokens` sampled tokens each (bounded by `budget_s`)."""
+    import oracle
+    nthreads = cpu_threads()
+    samples = [sample_tokens(wk, n_tokens, s) for s in range(1, passes + 1)]
+    need = set(range(wk.n_routed, wk.n_experts))
+    for tok in samples:
+        ids, *_ = oracle.route(wk.logits[tok], wk.top_k, wk.renorm)
+        need |= set(int(e) for e in ids.ravel())
+    cache = prepare_oracle_experts(wk, sorted(need))
+    times = []
+    for tok in samples:
+        times.append(oracle_sample_step(wk, tok, cache, nthreads))
+        if sum(times) > budget_s:
+            break
+    total = sum(times)
+    return {"value": len(times) * n_tokens / total, "unit": "tokens/s", "cores": nthreads,
+            "kind": "oracle",
+            "sample": f"{len(times)} oracle passes over {n_tokens} of the {wk.T} tokens each "
+                      f"(full layer for those tokens, routing included), {total:.1f} s of CPU work"}
+
+
+def run_reference(args):
+    """--impl reference: the oracle as the reference arm (rank 0 only)."""
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    wk = make_workload(args.workload, args.experts, args.tokens)
+    n_tok = 2
+    nthreads = cpu_threads()
+    steps = max(1, args.steps)
+    warm = max(0, args.warmup)
+    # prepare every expert the sampled steps will touch
+    seeds = list(range(100, 100 + warm + steps))
+    import oracle
+    need = set(range(wk.n_routed, wk.n_experts))
+    for s in seeds:
+        ids, *_ = oracle.route(wk.logits[sample_tokens(wk, n_tok, s)], wk.top_k, wk.renorm)
+        need |= set(int(e) for e in ids.ravel())
+    cache = prepare_oracle_experts(wk, sorted(need))
+    for s in seeds[:warm]:
+        oracle_sample_step(wk, sample_tokens(wk, n_tok, s), cache, nthreads)
+    times = [oracle_sample_step(wk, sample_tokens(wk, n_tok, s), cache, nthreads) for s in seeds[warm:]]
+    total = sum(times)
+    value = steps * n_tok / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": steps, "warmup": warm, "ms_per_step": 1e3 * total / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(wk), "tokens_per_step": n_tok,
+                       "sample": f"{n_tok} of {wk.T} tokens per step"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                             "sample": f"{n_tok} of {wk.T} tokens per step, full layer for those tokens"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_milo(args):
+    import torch
+
+    import int3_gemm_rank_b200 as milo
+    from int3_gemm_rank_b200 import build as milo_build
+
+    rank, local, world = dist_env()
+    if not os.path.exists(milo.LIB_PATH):
+        milo_build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+
+    wk = make_workload(args.workload, args.experts, args.tokens)
+    layer = gpu_layer(milo, wk, torch)
+
+    def to_dev(a, dt):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(dt).to(dev)
+
+    x = to_dev(wk.x, torch.bfloat16 if wk.x_dtype == "bf16" else torch.float16)
+    logits = to_dev(wk.logits, torch.float16)
+    out_dt = torch.bfloat16
+    T, k, E = wk.T, wk.top_k, wk.n_routed
+    st = milo.new_status(dev)
+    ws = layer.workspace(T, dev)
+    y = torch.empty((T, wk.hidden), dtype=out_dt, device=dev)
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    wts = torch.empty((T, k), dtype=torch.float32, device=dev)
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty(T * k, dtype=torch.int32, device=dev)
+    route = {"w": wts, "offsets": off, "perm": perm, "inv_perm": inv}
+    L = milo.lib()
+    import ctypes as C
+    flags = milo.MILO_ROUTE_RENORM if wk.renorm else 0
+    stream = torch.cuda.current_stream(dev)
+    sp = C.c_void_p(stream.cuda_stream)
+
+    def step(xin, lin):
+        s = L.milo_route(C.c_void_p(lin.data_ptr()), T, E, k, flags, C.c_void_p(ids.data_ptr()),
+                         C.c_void_p(wts.data_ptr()), C.c_void_p(off.data_ptr()),
+                         C.c_void_p(perm.data_ptr()), C.c_void_p(inv.data_ptr()),
+                         C.c_void_p(st.data_ptr()), sp)
+        if s:
+            milo._check(s, "milo_route")
+        milo.milo_moe_forward(layer, xin, route, out_dtype=out_dt, dev_status=st, y=y, ws=ws)
+
+    launches_per_step = 9   # route, rows, prep x, lorc w1|w3, gemm w1|w3, prep h, lorc w2, gemm w2, combine
+
+    # --- correctness gate on the bench configuration itself
+    step(x, logits)
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} on the bench workload")
+    counts = np.diff(off.cpu().numpy())
+    bytes_ = layer_bytes(wk, counts)
+
+    # --- warm-up and clock soak (also brings the clocks to their loaded state)
+    for _ in range(args.warmup):
+        step(x, logits)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_soak = time.perf_counter()
+    while time.perf_counter() - t_soak < args.soak:
+        for _ in range(20):
+            step(x, logits)
+        torch.cuda.synchronize()
+
+    # --- timed region: K steps, events on the launching stream
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4 * args.steps)]
+    for e in ev:            # torch creates the CUDA event on its first record
+        e.record(stream)
+    milo.milo_set_profile_events(None)
+    barrier(dev)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        milo.milo_set_profile_events(ev[4 * i:4 * i + 4])
+        step(x, logits)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    milo.milo_set_profile_events(None)
+    barrier(dev)
+    clocks = sampler.stop()
+    ms_total = start.elapsed_time(stop)
+    glu_ms = statistics.mean(ev[4 * i].elapsed_time(ev[4 * i + 1]) for i in range(args.steps))
+    w2_ms = statistics.mean(ev[4 * i + 2].elapsed_time(ev[4 * i + 3]) for i in range(args.steps))
+    ms_total = max_over_ranks(ms_total, dev)
+    ms_step = ms_total / args.steps
+    value = world * T * args.steps / (ms_total / 1e3)
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} after the timed region")
+
+    # --- end to end through the public API with host buffers
+    if args.no_e2e:
+        e2e_value, e2e_ms = None, None
+    else:
+        e2e_value, e2e_ms = run_e2e(args, torch, step, x, logits, y, out_dt, T, wk, dev, stream, world)
+    return finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, logits, y,
+                  e2e_value, launches_per_step, clocks)
+
+
+def run_e2e(args, torch, step, x, logits, y, out_dt, T, wk, dev, stream, world):
+    x_h = torch.empty_like(x, device="cpu").pin_memory()
+    x_h.copy_(x.cpu())
+    l_h = torch.empty_like(logits, device="cpu").pin_memory()
+    l_h.copy_(logits.cpu())
+    y_h = torch.empty((T, wk.hidden), dtype=out_dt).pin_memory()
+    x_d, l_d = torch.empty_like(x), torch.empty_like(logits)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        l_d.copy_(l_h, non_blocking=True)
+        step(x_d, l_d)
+        y_h.copy_(y, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(dev)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(s2.elapsed_time(e2), dev)
+    e2e_value = world * T * args.steps / (e2e_ms / 1e3)
+    return e2e_value, e2e_ms
+
+
+def finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, logits, y, e2e_value,
+           launches_per_step, clocks):
+    pk = peaks()
+    glu_gbs = bytes_["glu_kernel"] / (glu_ms / 1e3) / 1e9
+    step_gbs = bytes_["step"] / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": describe(wk), "tokens_per_step": T, "x_dtype": wk.x_dtype,
+                   "y_dtype": "bf16",
+                   "l2": f"inputs larger than L2: {bytes_['weights_only'] / 1e6:.0f} MB of packed weights "
+                         f"streamed per step vs {L2_BYTES / 1e6:.0f} MB L2; no flush",
+                   "parallelism": f"replica per GPU x{world}", "active_experts": bytes_["active_experts"]},
+        "roofline": {"bound": "hbm", "achieved": glu_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": glu_gbs / pk["hbm_gbs"], "traffic": profiled_traffic("gemv_glu_mixtral_decode.md")
+                     if args.workload == "mixtral" else None,
+                     "kernel": "gemv_kernel<true> (w1|w3 grouped int3 GEMM + compensator + SwiGLU)",
+                     "algorithmic_bytes_per_launch": bytes_["glu_kernel"], "ms_per_launch": glu_ms,
+                     "peak_source": f"{pk['source']} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                     if pk["source"] == "measured" else "fallback 6650 GB/s"},
+        "layer_hbm": {"bytes_per_step": bytes_["step"], "achieved_gbs": step_gbs,
+                      "frac": step_gbs / pk["hbm_gbs"]},
+        "kernels": {"gemm_w1w3_ms": glu_ms, "gemm_w2_ms": w2_ms,
+                    "gemm_w2_gbs": bytes_["w2_kernel"] / (w2_ms / 1e3) / 1e9,
+                    "gemm_w1w3_gbs": glu_gbs},
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": x.numel() * x.element_size() + logits.numel() * logits.element_size(),
+                "d2h_bytes_per_step": y.numel() * y.element_size()},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wk)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("milo", "reference"), default="milo")
+    ap.add_argument("--workload", choices=("mixtral", "deepseek", "prefill"), default="mixtral")
+    ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--experts", type=int, default=None, help="routed experts (profiler captures)")
+    ap.add_argument("--tokens", type=int, default=None, help="tokens per step (profiler captures)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_milo(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -244,6 +244,17 @@ MILO_API milo_status milo_moe_forward(const milo_moe_layer* layer, const void* x
 /* Byte offset of h inside the forward workspace (see milo_moe_forward). */
 MILO_API size_t milo_moe_h_offset(const milo_moe_layer* layer, int32_t T);
 
+/*
+ * milo_set_profile_events -- measurement hook.  `events` is a host array of n
+ * cudaEvent_t (n = 0 or events = NULL disables).  While set, every
+ * milo_moe_forward records events[0] / events[1] on its stream right before /
+ * after the launch of the w1|w3 grouped GEMM and events[2] / events[3] around
+ * the w2 grouped GEMM; milo_grouped_linear records events[0] / events[1] around
+ * its grouped GEMM.  The caller owns the events and reads them with
+ * cudaEventElapsedTime after the stream completes.  Process-wide setting.
+ */
+MILO_API milo_status milo_set_profile_events(void* const* events, int32_t n);
+
 #ifdef __cplusplus
 }
 #endif

@@ -30,7 +30,7 @@ MILO_GROUP, MILO_MAX_RANK = 64, 64
 EXPORTS = ("milo_status_str", "milo_last_error", "milo_version", "milo_pack", "milo_unpack",
            "milo_route", "milo_table_bytes", "milo_linear_prepare", "milo_layer_prepare",
            "milo_linear_workspace_bytes", "milo_moe_workspace_bytes", "milo_grouped_linear",
-           "milo_moe_forward", "milo_moe_h_offset")
+           "milo_moe_forward", "milo_moe_h_offset", "milo_set_profile_events")
 
 
 class MiloError(RuntimeError):
@@ -95,6 +95,8 @@ def lib() -> C.CDLL:
         L.milo_moe_forward.restype = C.c_int
         L.milo_moe_h_offset.argtypes = [C.POINTER(milo_moe_layer), i32]
         L.milo_moe_h_offset.restype = sz
+        L.milo_set_profile_events.argtypes = [C.POINTER(C.c_void_p), i32]
+        L.milo_set_profile_events.restype = C.c_int
         _lib = L
     return _lib
 
@@ -121,6 +123,15 @@ def _dt(t: torch.Tensor) -> int:
 def _cuda(t: torch.Tensor, name: str):
     if not t.is_cuda or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def milo_set_profile_events(events: list | None):
+    """Record torch.cuda.Event objects around the grouped GEMM launches (None disables)."""
+    if not events:
+        _check(lib().milo_set_profile_events(None, 0), "milo_set_profile_events")
+        return
+    arr = (C.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _check(lib().milo_set_profile_events(arr, len(events)), "milo_set_profile_events")
 
 
 def new_status(device=None) -> torch.Tensor:

@@ -4,8 +4,8 @@
 // The sequence for one MoE layer ("MiLo: Efficient Quantized MoE Inference
 // with Mixture of Low-Rank Compensators": routed experts, each a quantised
 // weight plus a rank-r compensator, outputs mixed by the router weights):
-//   rows -> prep(x) -> lorc(x, V1|V3) -> gemv<SwiGLU>(w1|w3) -> prep(h)
-//        -> lorc(h, V2) -> gemv(w2) -> combine
+//   prep(x, row bookkeeping) -> lorc(x, V1|V3) -> gemv<SwiGLU>(w1|w3)
+//        -> prep(h) -> lorc(h, V2) -> gemv(w2) -> combine
 // Every step is a kernel on the caller's stream; the host never waits.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -66,6 +66,14 @@ static milo_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataTyp
         return fail(MILO_ERR_INVALID_ARG, std::string("tensor map encoding failed for ") + what +
                                               " (code " + std::to_string(static_cast<int>(r)) + ")");
     return MILO_OK;
+}
+
+// Measurement hook (milo_set_profile_events).
+static cudaEvent_t g_prof[4] = {nullptr, nullptr, nullptr, nullptr};
+static int g_prof_n = 0;
+
+static void prof_record(int i, cudaStream_t st) {
+    if (i < g_prof_n && g_prof[i]) cudaEventRecord(g_prof[i], st);
 }
 
 static int sm_count() {
@@ -143,9 +151,14 @@ struct Carve {
 static int gpad_of(int K) { return static_cast<int>(round_up(K / MILO_GROUP, 4)); }
 static size_t frag_row_bytes(int K) { return static_cast<size_t>(K / 128) * 288; }
 
+struct LorcPlan {
+    int splits, row_groups;
+};
+
 struct LinearWs {
-    size_t grp, rows, inv, frag, gsum, t, part, total;
+    size_t grp, rows, inv, frag, gsum, t, tpart, part, total;
     int R, splits, tcols;
+    LorcPlan lp;
 };
 
 static int tiles_of(int N, int rows) { return (N + rows - 1) / rows; }
@@ -153,7 +166,7 @@ static int tiles_of(int N, int rows) { return (N + rows - 1) / rows; }
 // Split-K factor for the plain kernel: make the estimated item count fill the
 // persistent grid in whole waves (the tail "shift" of the work distribution).
 static int choose_splits(long long base_items, int chunks) {
-    const int slots = 2 * sm_count();
+    const int slots = 3 * sm_count();
     if (base_items <= 0) return 1;
     int best = 1;
     double best_eff = -1.0;
@@ -166,6 +179,22 @@ static int choose_splits(long long base_items, int chunks) {
         if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
     }
     return best;
+}
+
+// K slices and row-tile groups of the compensator down-projection: enough
+// blocks to fill the GPU (about four per SM), K slices dividing K/128.
+static LorcPlan lorc_plan(int n_exp, int nproj, int K, long long rows_per_exp) {
+    const long long target = 8LL * sm_count();
+    const long long base = static_cast<long long>(n_exp) * nproj * ((MILO_MAX_RANK + 15) / 16);
+    const int sb = K / 128;
+    const long long tiles = std::max(1LL, (rows_per_exp + 15) / 16);
+    LorcPlan pl{1, 1};
+    pl.row_groups = static_cast<int>(std::min<long long>(tiles, std::max(1LL, target / std::max(1LL, base))));
+    // K slices only while the row tiles do not fill the GPU (they cost partial sums)
+    const long long want = tiles > 4 ? 1 : std::max(1LL, target / std::max(1LL, base * pl.row_groups));
+    for (int d = 1; d <= sb; ++d)
+        if (sb % d == 0 && d <= want) pl.splits = d;
+    return pl;
 }
 
 static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
@@ -184,14 +213,17 @@ static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
     w.frag = c.take(static_cast<size_t>(w.R) * frag_row_bytes(lin->K));
     w.gsum = c.take(static_cast<size_t>(w.R) * gpad_of(lin->K) * 4);
     w.t = c.take(static_cast<size_t>(w.R) * w.tcols * 2);
+    w.lp = lorc_plan(n_exp, 1, lin->K, std::max(1LL, static_cast<long long>(w.R) / std::max<long long>(1, groups)));
+    w.tpart = c.take(static_cast<size_t>(w.lp.splits) * w.R * w.tcols * 4);
     w.part = c.take(static_cast<size_t>(w.splits) * w.R * lin->N * 4);
     w.total = c.off;
     return w;
 }
 
 struct MoeWs {
-    size_t grp, rows, xfrag, xg, t13, h, hfrag, hg, t2, part, total;
+    size_t grp, rows, xfrag, xg, t13, h, hfrag, hg, t2, tpart, part, total;
     int R, R_routed, splits, tc13, tc2;
+    LorcPlan lp13, lp2;
 };
 
 static MoeWs moe_ws(const milo_moe_layer* L, int T) {
@@ -215,6 +247,11 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
     w.hfrag = c.take(static_cast<size_t>(w.R) * frag_row_bytes(I));
     w.hg = c.take(static_cast<size_t>(w.R) * gpad_of(I) * 4);
     w.t2 = c.take(static_cast<size_t>(w.R) * w.tc2 * 2);
+    const long long rows_per_exp = std::max(1LL, static_cast<long long>(w.R) / std::max<long long>(1, groups));
+    w.lp13 = lorc_plan(n_exp, 2, H, rows_per_exp);
+    w.lp2 = lorc_plan(n_exp, 1, I, rows_per_exp);
+    w.tpart = c.take(std::max(static_cast<size_t>(w.lp13.splits) * w.tc13,
+                              static_cast<size_t>(w.lp2.splits) * w.tc2) * w.R * 4);
     w.part = c.take(static_cast<size_t>(w.splits) * w.R * H * 4);
     w.total = c.off;
     return w;
@@ -243,7 +280,7 @@ static milo_status act_maps(GemvParams& g, void* frag, void* gsum, void* t, int 
 }
 
 static milo_status run_gemv(GemvParams& g, bool glu, cudaStream_t st, const char* what) {
-    const int grid = 2 * sm_count();
+    const int grid = 3 * sm_count();
     return check_cuda(launch_gemv(g, glu, grid, st), what);
 }
 
@@ -269,6 +306,15 @@ extern "C" const char* milo_status_str(milo_status s) {
 extern "C" const char* milo_last_error(void) { return g_last_error.c_str(); }
 
 extern "C" int32_t milo_version(void) { return 1; }
+
+extern "C" milo_status milo_set_profile_events(void* const* events, int32_t n) {
+    clear_error();
+    if (n < 0 || n > 4 || (n > 0 && !events))
+        return fail(MILO_ERR_INVALID_ARG, "milo_set_profile_events: n must be in [0, 4]");
+    for (int i = 0; i < 4; ++i) g_prof[i] = i < n ? static_cast<cudaEvent_t>(events[i]) : nullptr;
+    g_prof_n = n;
+    return MILO_OK;
+}
 
 extern "C" milo_status milo_table_bytes(int32_t n_projections, size_t* bytes) {
     clear_error();
@@ -369,21 +415,19 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     int32_t* rows = reinterpret_cast<int32_t*>(base + w.rows);
     int32_t* inv = reinterpret_cast<int32_t*>(base + w.inv);
 
-    RowsParams rp{expert_offsets, perm, grp, rows, inv, dev_status, T, k, lin->n_experts, 0, w.R};
-    milo_status s = check_cuda(launch_rows(rp, st), "rows");
-    if (s != MILO_OK) return s;
-
     PrepParams pp{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.frag),
                   reinterpret_cast<float*>(base + w.gsum), dev_status, w.R, lin->K, gpad_of(lin->K),
-                  x_dt == MILO_BF16};
-    if ((s = check_cuda(launch_prep(pp, st), "prep")) != MILO_OK) return s;
+                  x_dt == MILO_BF16, 1, expert_offsets, perm, grp, inv, T, k, lin->n_experts, 0, w.R};
+    milo_status s = check_cuda(launch_prep(pp, st), "prep");
+    if (s != MILO_OK) return s;
 
     const bool has_t = lin->max_rank > 0;
     const ProjDev* table = static_cast<const ProjDev*>(lin->table);
     if (has_t) {
         LorcParams lp{static_cast<const uint16_t*>(x), rows, table, grp,
-                      reinterpret_cast<uint16_t*>(base + w.t), dev_status, 1, 0, -1,
-                      lin->n_experts, lin->K, w.R, w.tcols, 0, x_dt == MILO_BF16};
+                      reinterpret_cast<uint16_t*>(base + w.t), reinterpret_cast<float*>(base + w.tpart),
+                      dev_status, 1, 0, -1, lin->n_experts, lin->K, w.R, w.tcols, 0, x_dt == MILO_BF16,
+                      w.lp.splits, w.lp.row_groups};
         if ((s = check_cuda(launch_lorc(lp, st), "lorc")) != MILO_OK) return s;
     }
 
@@ -407,7 +451,9 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     g.cps = (g.chunks + w.splits - 1) / w.splits;
     g.has_t = has_t;
     g.tcols = w.tcols;
+    prof_record(0, st);
     if ((s = run_gemv(g, false, st, "gemv")) != MILO_OK) return s;
+    prof_record(1, st);
 
     CombineParams cp{reinterpret_cast<const float*>(base + w.part), inv, nullptr, y, dev_status,
                      T, k, 0, lin->N, w.R, w.splits, w.R, static_cast<int>(y_dt), 1};
@@ -441,17 +487,15 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     const bool has_t = L->max_rank > 0;
     milo_status s;
 
-    RowsParams rp{expert_offsets, perm, grp, rows, nullptr, dev_status, T, L->top_k, L->n_routed,
-                  L->n_shared, w.R_routed};
-    if ((s = check_cuda(launch_rows(rp, st), "rows")) != MILO_OK) return s;
-
     PrepParams px{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.xfrag),
-                  reinterpret_cast<float*>(base + w.xg), dev_status, w.R, H, gpad_of(H), x_dt == MILO_BF16};
+                  reinterpret_cast<float*>(base + w.xg), dev_status, w.R, H, gpad_of(H), x_dt == MILO_BF16,
+                  1, expert_offsets, perm, grp, nullptr, T, L->top_k, L->n_routed, L->n_shared, w.R_routed};
     if ((s = check_cuda(launch_prep(px, st), "prep x")) != MILO_OK) return s;
     if (has_t) {
         LorcParams lp{static_cast<const uint16_t*>(x), rows, table, grp,
-                      reinterpret_cast<uint16_t*>(base + w.t13), dev_status, 3, 0, 1, n_exp, H, w.R,
-                      w.tc13, L->max_rank, x_dt == MILO_BF16};
+                      reinterpret_cast<uint16_t*>(base + w.t13), reinterpret_cast<float*>(base + w.tpart),
+                      dev_status, 3, 0, 1, n_exp, H, w.R, w.tc13, L->max_rank, x_dt == MILO_BF16,
+                      w.lp13.splits, w.lp13.row_groups};
         if ((s = check_cuda(launch_lorc(lp, st), "lorc w1|w3")) != MILO_OK) return s;
     }
 
@@ -475,16 +519,18 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     g1.has_t = has_t;
     g1.tcols = w.tc13;
     g1.t_col_b = L->max_rank;
+    prof_record(0, st);
     if ((s = run_gemv(g1, true, st, "gemv w1|w3")) != MILO_OK) return s;
+    prof_record(1, st);
 
     PrepParams ph{reinterpret_cast<const uint16_t*>(base + w.h), nullptr,
                   reinterpret_cast<uint16_t*>(base + w.hfrag), reinterpret_cast<float*>(base + w.hg),
-                  dev_status, w.R, I, gpad_of(I), 0};
+                  dev_status, w.R, I, gpad_of(I), 0, 0, nullptr, nullptr, nullptr, nullptr, 0, 0, 0, 0, 0};
     if ((s = check_cuda(launch_prep(ph, st), "prep h")) != MILO_OK) return s;
     if (has_t) {
         LorcParams lp{reinterpret_cast<const uint16_t*>(base + w.h), nullptr, table, grp,
-                      reinterpret_cast<uint16_t*>(base + w.t2), dev_status, 3, 2, -1, n_exp, I, w.R,
-                      w.tc2, 0, 0};
+                      reinterpret_cast<uint16_t*>(base + w.t2), reinterpret_cast<float*>(base + w.tpart),
+                      dev_status, 3, 2, -1, n_exp, I, w.R, w.tc2, 0, 0, w.lp2.splits, w.lp2.row_groups};
         if ((s = check_cuda(launch_lorc(lp, st), "lorc w2")) != MILO_OK) return s;
     }
 
@@ -507,7 +553,9 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     g2.cps = (g2.chunks + w.splits - 1) / w.splits;
     g2.has_t = has_t;
     g2.tcols = w.tc2;
+    prof_record(2, st);
     if ((s = run_gemv(g2, false, st, "gemv w2")) != MILO_OK) return s;
+    prof_record(3, st);
 
     CombineParams cp{reinterpret_cast<const float*>(base + w.part), inv_perm, topk_w, y, dev_status,
                      T, L->top_k, L->n_shared, H, w.R, w.splits, w.R_routed, static_cast<int>(y_dt), 0};

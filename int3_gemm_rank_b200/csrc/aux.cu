@@ -1,8 +1,9 @@
 // aux.cu -- the kernels around the grouped int3 GEMM:
-//   rows_kernel    routed/shared row bookkeeping from the router's offsets/perm
 //   prep_kernel    activations -> fp16 MMA fragments (power-of-8 factors of the
-//                  int3 field extraction folded in) and per-group sums
-//   lorc_kernel    compensator down-projection t = x V^T per expert
+//                  int3 field extraction folded in) and per-group sums; the
+//                  first one of a call also does the row bookkeeping (expert
+//                  groups, row -> token) from the router's offsets and perm
+//   lorc_*_kernel  compensator down-projection t = x V^T per expert
 //   combine_kernel weighted un-permute back to token order, split-K reduction
 //
 // "MiLo: Efficient Quantized MoE Inference with Mixture of Low-Rank
@@ -17,14 +18,28 @@
 namespace milo {
 
 // ---------------------------------------------------------------------------
-// rows: groups (first row, count) for routed + shared experts, row -> token
+// prep: fragment-ordered activations and group sums, one block per row
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) rows_kernel(const RowsParams p) {
+template <int S, int H>
+__device__ __forceinline__ uint32_t frag_pair(const __half (&x)[32]) {
+    constexpr int t = sched_word(S, H), f = sched_field(S, H);
+    constexpr int m = reg_code(t, f);
+    const __half sc = __float2half_rn(act_scale(f));
+    const __half lo = __hmul(x[m], sc), hi = __hmul(x[m + 1], sc);
+    return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+}
+
+template <int S>
+__device__ __forceinline__ uint2 frag_step(const __half (&x)[32]) {
+    return make_uint2(frag_pair<S, 0>(x), frag_pair<S, 1>(x));
+}
+
+// Expert groups (first row, count), clamped into a non-decreasing sequence
+// within [0, T*k]; shared experts follow the routed rows.  Block (0, 0) only.
+__device__ void build_groups(const PrepParams& p, int32_t& st) {
     __shared__ int ok_off[MILO_MAX_EXPERTS + 1];
     const int F = p.T * p.k;
-    int32_t st = 0;
     if (threadIdx.x == 0) {
-        // Clamp the offsets into a non-decreasing sequence within [0, F].
         int prev = 0;
         for (int e = 0; e <= p.E; ++e) {
             int o = p.offsets[e];
@@ -45,56 +60,46 @@ __global__ void __launch_bounds__(256) rows_kernel(const RowsParams p) {
             p.grp[2 * (p.E + s) + 1] = p.T;
         }
     }
-    __syncthreads();
-    const int used = ok_off[p.E];
-    if (p.inv)
+    if (p.inv) {
+        __syncthreads();
         for (int f = threadIdx.x; f < F; f += blockDim.x) p.inv[f] = -1;
-    __syncthreads();
-    for (int r = threadIdx.x; r < p.R_routed; r += blockDim.x) {
-        int src = -1;
-        if (r < used) {
+        __syncthreads();
+        const int used = ok_off[p.E];
+        for (int r = threadIdx.x; r < used; r += blockDim.x) {
             const int f = p.perm ? p.perm[r] : r;
-            if (f >= 0 && f < F) {
-                src = f / p.k;
-                if (p.inv) p.inv[f] = r;
-            } else {
-                st |= MILO_DEV_BAD_EXPERT_ID;
-            }
+            if (f >= 0 && f < F) p.inv[f] = r;
         }
-        p.row_src[r] = src;
     }
-    for (int r = threadIdx.x; r < p.S * p.T; r += blockDim.x) p.row_src[p.R_routed + r] = r % p.T;
-    flag(p.dev_status, st);
 }
 
-cudaError_t launch_rows(const RowsParams& p, cudaStream_t s) {
-    rows_kernel<<<1, 256, 0, s>>>(p);
-    return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
-// prep: fragment-ordered activations and group sums, one block per row
-// ---------------------------------------------------------------------------
-template <int S, int H>
-__device__ __forceinline__ uint32_t frag_pair(const __half (&x)[32]) {
-    constexpr int t = sched_word(S, H), f = sched_field(S, H);
-    constexpr int m = reg_code(t, f);
-    const __half sc = __float2half_rn(act_scale(t, f));
-    const __half lo = __hmul(x[m], sc), hi = __hmul(x[m + 1], sc);
-    return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
-}
-
-template <int S>
-__device__ __forceinline__ uint2 frag_step(const __half (&x)[32]) {
-    return make_uint2(frag_pair<S, 0>(x), frag_pair<S, 1>(x));
+// Source row (token) of row `row`, or -1.
+__device__ __forceinline__ int row_source(const PrepParams& p, int row, int32_t& st) {
+    if (row >= p.R_routed) return (row - p.R_routed) % p.T;
+    const int F = p.T * p.k;
+    int used = p.offsets[p.E];
+    used = used < 0 ? 0 : (used > F ? F : used);
+    if (row >= used) return -1;
+    const int f = p.perm ? p.perm[row] : row;
+    if (f < 0 || f >= F) {
+        st |= MILO_DEV_BAD_EXPERT_ID;
+        return -1;
+    }
+    return f / p.k;
 }
 
 __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     const int row = blockIdx.x;
     const int SB = p.K / 128;
-    const int src = p.row_src ? p.row_src[row] : row;
     int32_t st = 0;
-    for (int base = 0; base < SB * 4; base += blockDim.x) {
+    int src;
+    if (p.rows) {
+        if (blockIdx.x == 0 && blockIdx.y == 0) build_groups(p, st);
+        src = row_source(p, row, st);
+        if (blockIdx.y == 0 && threadIdx.x == 0) p.row_src[row] = src;
+    } else {
+        src = p.row_src ? p.row_src[row] : row;
+    }
+    for (int base = blockIdx.y * blockDim.x; base < SB * 4; base += gridDim.y * blockDim.x) {
         const int idx = base + threadIdx.x;
         const bool active = idx < SB * 4;
         const int sb = idx >> 2, c = idx & 3;
@@ -140,23 +145,29 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
         out[5 * 4] = frag_step<5>(x);
         out[6 * 4] = frag_step<6>(x);
         out[7 * 4] = frag_step<7>(x);
-        out[8 * 4] = frag_step<8>(x);
+        out[8 * 4] = make_uint2(0u, 0u);      // padding (bank spread)
     }
-    for (int j = 2 * SB + threadIdx.x; j < p.gpad; j += blockDim.x)
-        p.gsum[static_cast<size_t>(row) * p.gpad + j] = 0.0f;
+    if (blockIdx.y == 0)
+        for (int j = 2 * SB + threadIdx.x; j < p.gpad; j += blockDim.x)
+            p.gsum[static_cast<size_t>(row) * p.gpad + j] = 0.0f;
     flag(p.dev_status, st);
 }
 
 cudaError_t launch_prep(const PrepParams& p, cudaStream_t s) {
     if (p.R <= 0) return cudaSuccess;
-    prep_kernel<<<p.R, 128, 0, s>>>(p);
+    // 32 super-blocks per block; enough blocks per row to fill the GPU at decode sizes
+    const int chunks = (p.K / 128 * 4 + 127) / 128;
+    prep_kernel<<<dim3(p.R, chunks), 128, 0, s>>>(p);
     return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// lorc: t[p, col0 + j] = sum_k x[p, k] V[j, k] for the rows of each expert,
-// one block per (expert, projection, 16-rank block); four warps split K and
-// the partial tiles are added in a fixed order.
+// lorc: t[p, col0 + j] = sum_k x[p, k] V[j, k] for the rows of each expert.
+// Pass 1 (lorc_partial_kernel): one block per (expert, projection, 16-rank
+// block, K slice, row-tile group); its four warps split the K slice and their
+// 16x16 tiles are added in a fixed order into part[slice].  Pass 2
+// (lorc_reduce_kernel) adds the slices in order and rounds to fp16.  Both
+// orders are fixed, so the result does not depend on scheduling.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t load_x_pair(const uint16_t* row, int k, bool bf16, int32_t& st) {
     const uint32_t w = *reinterpret_cast<const uint32_t*>(row + k);
@@ -165,12 +176,23 @@ __device__ __forceinline__ uint32_t load_x_pair(const uint16_t* row, int k, bool
     return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
 }
 
-__global__ void __launch_bounds__(128) lorc_kernel(const LorcParams p, int rank_blocks) {
+constexpr int kLorcRankBlocks = (MILO_MAX_RANK + 15) / 16;
+constexpr int kLorcChunk = 256;             // K staged per step (per block)
+constexpr int kLorcPitch = kLorcChunk + 8;  // fp16; rows fall on different banks
+
+__global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
+    __shared__ __align__(16) uint16_t xs[16][kLorcPitch];
+    __shared__ __align__(16) uint16_t vs[16][kLorcPitch];
     __shared__ float part[4][16][17];
+    __shared__ int src_row[16];
     const int nproj = p.proj_b >= 0 ? 2 : 1;
-    const int e = blockIdx.x / (nproj * rank_blocks);
-    const int rem = blockIdx.x % (nproj * rank_blocks);
-    const int which = rem / rank_blocks, rblk = rem % rank_blocks;
+    int b = blockIdx.x;
+    const int split = b % p.splits;
+    b /= p.splits;
+    const int rblk = b % kLorcRankBlocks;
+    b /= kLorcRankBlocks;
+    const int which = b % nproj;
+    const int e = b / nproj;
     const ProjDev* P = p.table + e * p.stride + (which == 0 ? p.proj_a : p.proj_b);
     const int r = P->rank;
     const int j0 = 16 * rblk;
@@ -179,30 +201,62 @@ __global__ void __launch_bounds__(128) lorc_kernel(const LorcParams p, int rank_
     if (m <= 0 || row0 < 0 || row0 + m > p.R) return;
     const int col0 = which == 0 ? 0 : p.t_col_b;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-    const int kq = p.K / 4;   // K is a multiple of 128
-    const int kbeg = warp * kq;
+    const int slice = p.K / p.splits;                 // a multiple of 128
+    const int kbeg = split * slice;
+    float* out = p.part + static_cast<size_t>(split) * p.R * p.tcols;
     int32_t st = 0;
-    for (int mt = 0; mt < m; mt += 16) {
+    for (int mt = 16 * blockIdx.y; mt < m; mt += 16 * p.row_groups) {
+        __syncthreads();
+        if (threadIdx.x < 16) {
+            const int i = threadIdx.x;
+            src_row[i] = mt + i < m ? (p.row_src ? p.row_src[row0 + mt + i] : row0 + mt + i) : -1;
+        }
         float acc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
-        const int ra = mt + g, rb = mt + g + 8;
-        const int sa = ra < m ? (p.row_src ? p.row_src[row0 + ra] : row0 + ra) : -1;
-        const int sb_ = rb < m ? (p.row_src ? p.row_src[row0 + rb] : row0 + rb) : -1;
-        const uint16_t* xa = sa >= 0 ? p.src + static_cast<size_t>(sa) * p.K : nullptr;
-        const uint16_t* xb = sb_ >= 0 ? p.src + static_cast<size_t>(sb_) * p.K : nullptr;
-        const uint16_t* v0 = (j0 + g < r) ? P->V + static_cast<size_t>(j0 + g) * p.K : nullptr;
-        const uint16_t* v1 = (j0 + 8 + g < r) ? P->V + static_cast<size_t>(j0 + 8 + g) * p.K : nullptr;
-        for (int k = kbeg; k < kbeg + kq; k += 16) {
-            const int kc = k + 2 * c;
-            const uint32_t a0 = xa ? load_x_pair(xa, kc, p.src_bf16, st) : 0u;
-            const uint32_t a1 = xb ? load_x_pair(xb, kc, p.src_bf16, st) : 0u;
-            const uint32_t a2 = xa ? load_x_pair(xa, kc + 8, p.src_bf16, st) : 0u;
-            const uint32_t a3 = xb ? load_x_pair(xb, kc + 8, p.src_bf16, st) : 0u;
-            const uint32_t b00 = v0 ? *reinterpret_cast<const uint32_t*>(v0 + kc) : 0u;
-            const uint32_t b01 = v0 ? *reinterpret_cast<const uint32_t*>(v0 + kc + 8) : 0u;
-            const uint32_t b10 = v1 ? *reinterpret_cast<const uint32_t*>(v1 + kc) : 0u;
-            const uint32_t b11 = v1 ? *reinterpret_cast<const uint32_t*>(v1 + kc + 8) : 0u;
-            mma16816(acc[0], a0, a1, a2, a3, b00, b01);
-            mma16816(acc[1], a0, a1, a2, a3, b10, b11);
+        for (int kc = kbeg; kc < kbeg + slice; kc += kLorcChunk) {
+            // this chunk: 256 or, at the end of a slice, 128 (slices are multiples of 128)
+            const int cs = min(kLorcChunk, kbeg + slice - kc);
+            const int kw = cs / 4;                    // K per warp: 32 or 64
+            __syncthreads();
+            // stage x rows and V rows [16][cs] with 16-byte loads
+            const int per_row = cs / 8;
+            for (int i = threadIdx.x; i < 32 * per_row; i += blockDim.x) {
+                const int rr = (i / per_row) & 15, ch = i % per_row, isv = i / (16 * per_row);
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (isv) {
+                    if (j0 + rr < r)
+                        v = *reinterpret_cast<const uint4*>(P->V + static_cast<size_t>(j0 + rr) * p.K + kc + 8 * ch);
+                    *reinterpret_cast<uint4*>(&vs[rr][8 * ch]) = v;
+                } else {
+                    const int sr = src_row[rr];
+                    if (sr >= 0) {
+                        v = *reinterpret_cast<const uint4*>(p.src + static_cast<size_t>(sr) * p.K + kc + 8 * ch);
+                        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const __half lo = to_half(static_cast<uint16_t>(w[q] & 0xFFFFu), p.src_bf16, st);
+                            const __half hi = to_half(static_cast<uint16_t>(w[q] >> 16), p.src_bf16, st);
+                            w[q] = static_cast<uint32_t>(__half_as_ushort(lo)) |
+                                   (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+                        }
+                        v = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                    *reinterpret_cast<uint4*>(&xs[rr][8 * ch]) = v;
+                }
+            }
+            __syncthreads();
+            for (int k = warp * kw; k < warp * kw + kw; k += 16) {
+                const int kk = k + 2 * c;
+                const uint32_t a0 = *reinterpret_cast<const uint32_t*>(&xs[g][kk]);
+                const uint32_t a1 = *reinterpret_cast<const uint32_t*>(&xs[g + 8][kk]);
+                const uint32_t a2 = *reinterpret_cast<const uint32_t*>(&xs[g][kk + 8]);
+                const uint32_t a3 = *reinterpret_cast<const uint32_t*>(&xs[g + 8][kk + 8]);
+                const uint32_t b00 = *reinterpret_cast<const uint32_t*>(&vs[g][kk]);
+                const uint32_t b01 = *reinterpret_cast<const uint32_t*>(&vs[g][kk + 8]);
+                const uint32_t b10 = *reinterpret_cast<const uint32_t*>(&vs[g + 8][kk]);
+                const uint32_t b11 = *reinterpret_cast<const uint32_t*>(&vs[g + 8][kk + 8]);
+                mma16816(acc[0], a0, a1, a2, a3, b00, b01);
+                mma16816(acc[1], a0, a1, a2, a3, b10, b11);
+            }
         }
         // acc[h][i]: row g + 8*(i>>1), rank 8h + 2c + (i&1)
 #pragma unroll
@@ -214,20 +268,40 @@ __global__ void __launch_bounds__(128) lorc_kernel(const LorcParams p, int rank_
             const int rr = idx / 16, jj = idx % 16;
             const float v = ((part[0][rr][jj] + part[1][rr][jj]) + part[2][rr][jj]) + part[3][rr][jj];
             if (mt + rr < m && j0 + jj < r)
-                p.t[static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j0 + jj] =
-                    __half_as_ushort(__float2half_rn(v));
+                out[static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j0 + jj] = v;
         }
-        __syncthreads();
     }
     flag(p.dev_status, st);
 }
 
+__global__ void __launch_bounds__(256) lorc_reduce_kernel(const LorcParams p) {
+    const size_t n = static_cast<size_t>(p.R) * p.tcols;
+    const size_t stride = n;
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        // eight running sums (slices s, s+8, ...) so the loads overlap, added in a fixed order
+        float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        int s = 0;
+        for (; s + 8 <= p.splits; s += 8)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) a[j] += p.part[(s + j) * stride + i];
+        for (int j = 0; s + j < p.splits; ++j) a[j] += p.part[(s + j) * stride + i];
+        const float v = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+        p.t[i] = __half_as_ushort(__float2half_rn(v));
+    }
+}
+
 cudaError_t launch_lorc(const LorcParams& p, cudaStream_t s) {
-    const int rank_blocks = (MILO_MAX_RANK + 15) / 16;
     const int nproj = p.proj_b >= 0 ? 2 : 1;
-    const int blocks = p.n_exp * nproj * rank_blocks;
-    if (blocks <= 0) return cudaSuccess;
-    lorc_kernel<<<blocks, 128, 0, s>>>(p, rank_blocks);
+    const long long blocks = static_cast<long long>(p.n_exp) * nproj * kLorcRankBlocks * p.splits;
+    if (blocks <= 0 || p.R <= 0) return cudaSuccess;
+    lorc_partial_kernel<<<dim3(static_cast<unsigned>(blocks), p.row_groups), 128, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long n = static_cast<long long>(p.R) * p.tcols;
+    long long rb = (n + 255) / 256;
+    if (rb > 2048) rb = 2048;
+    lorc_reduce_kernel<<<static_cast<unsigned>(rb), 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 

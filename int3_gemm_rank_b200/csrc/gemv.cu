@@ -13,7 +13,7 @@
 // B200 design (not a translation of the page's kernel):
 //   - One producer warp streams each CTA's weight tile with 2-D TMA loads
 //     (packed codes, scales, zeros) plus the prepared activation fragments and
-//     per-group activation sums into a 4-stage shared-memory ring guarded by
+//     per-group activation sums into a 3-stage shared-memory ring guarded by
 //     mbarriers.  Weights are read from HBM exactly once per token tile.
 //   - Four consumer warps each own 32 weight rows.  A lane reads its 3-word
 //     unit of two rows and extracts code pairs with one LOP3 each (plus one
@@ -29,7 +29,7 @@
 //     the same lane), or fp32 partial sums per K split for the plain one.
 //   - Work items (expert, row tile, K split, 16-row token tile) are enumerated
 //     on the device from the expert offsets, so the host never synchronises;
-//     CTAs are persistent (two per SM) and walk the items round-robin, the
+//     CTAs are persistent (three per SM) and walk the items round-robin, the
 //     token tiles of one weight tile being adjacent so that they share L2.
 #include <cuda_runtime.h>
 
@@ -38,7 +38,7 @@
 
 namespace milo {
 
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kConsumerWarps = 4;
 constexpr int kGemvThreads = 32 * (kConsumerWarps + 1);
 // Stage layout (bytes).  Q tiles are [2 super-blocks][rows][12 words]; the
@@ -89,6 +89,7 @@ __device__ __forceinline__ void code_step(const uint32_t (&wd)[2][2][3], const u
                                           const uint8_t* xs, int g, int c, float (&dz)[2][2][4]) {
     constexpr int t0 = sched_word(S, 0), f0 = sched_field(S, 0);
     constexpr int t1 = sched_word(S, 1), f1 = sched_field(S, 1);
+    static_assert(S < kSteps, "schedule");
     uint2 b[NT];
 #pragma unroll
     for (int n8 = 0; n8 < NT; ++n8)
@@ -96,10 +97,10 @@ __device__ __forceinline__ void code_step(const uint32_t (&wd)[2][2][3], const u
             xs + ((n8 * 8 + g) * kFragHalvesPerSB + S * 16 + c * 4) * 2);
 #pragma unroll
     for (int ti = 0; ti < 2; ++ti) {
-        const uint32_t a0 = field<f0>(wd[ti][0][t0], hw[ti][0][t0]);
-        const uint32_t a1 = field<f0>(wd[ti][1][t0], hw[ti][1][t0]);
-        const uint32_t a2 = field<f1>(wd[ti][0][t1], hw[ti][0][t1]);
-        const uint32_t a3 = field<f1>(wd[ti][1][t1], hw[ti][1][t1]);
+        const uint32_t a0 = unit_reg<t0, f0>(wd[ti][0], hw[ti][0]);
+        const uint32_t a1 = unit_reg<t0, f0>(wd[ti][1], hw[ti][1]);
+        const uint32_t a2 = unit_reg<t1, f1>(wd[ti][0], hw[ti][0]);
+        const uint32_t a3 = unit_reg<t1, f1>(wd[ti][1], hw[ti][1]);
 #pragma unroll
         for (int n8 = 0; n8 < NT; ++n8) {
             if constexpr (S == 0 || S == 4) mma16816_zc(dz[ti][n8], a0, a1, a2, a3, b[n8].x, b[n8].y);
@@ -176,7 +177,6 @@ __device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2]
         code_step<5, NT>(wd, hw, xs, g, c, dz);
         code_step<6, NT>(wd, hw, xs, g, c, dz);
         code_step<7, NT>(wd, hw, xs, g, c, dz);
-        code_step<8, NT>(wd, hw, xs, g, c, dz);
         fold_group<GLU, NT>(acc, dz, st, 2 * sbl + 1, rbase, g, c);
     }
 }
@@ -212,7 +212,7 @@ __device__ __forceinline__ void lorc_compute(const uint8_t* st, float (&acc)[2][
 }
 
 template <bool GLU>
-__global__ void __launch_bounds__(kGemvThreads, 2) gemv_kernel(const __grid_constant__ GemvParams p) {
+__global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_constant__ GemvParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
     uint64_t* empty = full + kStages;

@@ -51,56 +51,59 @@ __device__ __forceinline__ __half to_half(uint16_t bits, bool is_bf16, int32_t& 
 // and fp16 patterns below 2^11 are that integer times 2^-24).  Fields 3 and 4
 // and the spare bit are brought down by one shift of 9.  So each pair of codes
 // costs one LOP3 (plus one shared shift per word) and the power-of-8 factor is
-// undone on the activation side, where it costs nothing per weight.
+// undone on the activation side, where it costs nothing per weight.  The six
+// spare bits of a unit (bit t of u_30 in bit 15 of word t, bit t of u_31 in
+// bit 31) are gathered into bits 6..8 / 22..24 of one more register, i.e.
+// u_30 * 64 and u_31 * 64 in the fp16 halves.
 constexpr uint32_t kField0 = 0x00070007u;   // bits 0-2   -> code * 1
 constexpr uint32_t kField1 = 0x00380038u;   // bits 3-5   -> code * 8
 constexpr uint32_t kField2 = 0x01C001C0u;   // bits 6-8   -> code * 64
-constexpr uint32_t kSpare = 0x00400040u;    // bit 15 >> 9 -> bit * 64
+constexpr uint32_t kSpare = 0x00400040u;    // bit 15 >> 9 -> bit 6 (bit 31 >> 9 -> bit 22)
 
-// Extracted register f (0..5) of a word; `hi` is the word shifted right by 9.
-template <int F>
-__device__ __forceinline__ uint32_t field(uint32_t w, uint32_t hi) {
-    if constexpr (F == 0) return w & kField0;
-    else if constexpr (F == 1) return w & kField1;
-    else if constexpr (F == 2) return w & kField2;
-    else if constexpr (F == 3) return hi & kField0;
-    else if constexpr (F == 4) return hi & kField1;
-    else return hi & kSpare;
+// Register f (0..5) of a unit; w[] are its three words, hw[] the words >> 9.
+// Fields 0..4 come from word t; register 5 gathers the spare bits.
+template <int T, int F>
+__device__ __forceinline__ uint32_t unit_reg(const uint32_t (&w)[3], const uint32_t (&hw)[3]) {
+    if constexpr (F == 0) return w[T] & kField0;
+    else if constexpr (F == 1) return w[T] & kField1;
+    else if constexpr (F == 2) return w[T] & kField2;
+    else if constexpr (F == 3) return hw[T] & kField0;
+    else if constexpr (F == 4) return hw[T] & kField1;
+    else return (hw[0] & kSpare) + (hw[1] & kSpare) * 2u + (hw[2] & kSpare) * 4u;
 }
 
-// Register schedule of one 3-word unit over the nine k16 MMA steps of a
-// 128-code super-block.  Step s uses register kSchedWord/kSchedField[s][0]
+// Register schedule of one 3-word unit over the eight k16 MMA steps of a
+// 128-code super-block.  Step s uses register (sched_word, sched_field)[s][0]
 // for A-fragment slots (2c, 2c+1) and [s][1] for slots (2c+8, 2c+9).  Steps
-// 0..3 cover the first scale group (unit codes u_0..u_15), steps 4..8 the
-// second (u_16..u_29 and the three spare bits of u_30/u_31).
+// 0..3 cover the first scale group (unit codes u_0..u_15), steps 4..7 the
+// second (u_16..u_31).  Field 5 is the gathered spare register (word unused).
 __host__ __device__ constexpr int sched_word(int s, int h) {
-    constexpr int w[9][2] = {{0, 0}, {0, 0}, {0, 1}, {1, 1}, {1, 1},
-                             {2, 2}, {2, 2}, {2, 0}, {1, 2}};
+    constexpr int w[8][2] = {{0, 0}, {0, 0}, {0, 1}, {1, 1}, {1, 1}, {2, 2}, {2, 2}, {2, 0}};
     return w[s][h];
 }
 __host__ __device__ constexpr int sched_field(int s, int h) {
-    constexpr int f[9][2] = {{0, 1}, {2, 3}, {4, 0}, {1, 2}, {3, 4},
-                             {0, 1}, {2, 3}, {4, 5}, {5, 5}};
+    constexpr int f[8][2] = {{0, 1}, {2, 3}, {4, 0}, {1, 2}, {3, 4}, {0, 1}, {2, 3}, {4, 5}};
     return f[s][h];
 }
+constexpr int kSteps = 8;
 // Unit code index of the low half of register (word t, field f); the high
-// half holds the next code.  Spare registers carry bit t of u_30 (low) and
-// u_31 (high).
+// half holds the next code.  The spare register holds u_30 (low), u_31 (high).
 __host__ __device__ constexpr int reg_code(int t, int f) { return f < 5 ? 10 * t + 2 * f : 30; }
 // Offset inside the 128-code super-block of unit code m of unit c.
 __host__ __device__ constexpr int unit_k(int c, int m) {
     return m < 16 ? 16 * c + m : 64 + 16 * c + (m - 16);
 }
-// Factor applied to the activation paired with register (t, f): the inverse of
-// the power of 8 left in the extracted value, or 2^t / 64 for the spare bits.
-__host__ __device__ constexpr float act_scale(int t, int f) {
-    return f == 0 || f == 3 ? 1.0f
-         : f == 1 || f == 4 ? 0.125f
-         : f == 2           ? 0.015625f
-                            : (float)(1 << t) * 0.015625f;
+// Power of 8 left in the extracted value of field f, and its inverse, which
+// multiplies the activation paired with it.
+__host__ __device__ constexpr int field_shift(int f) {
+    return f == 0 || f == 3 ? 0 : f == 1 || f == 4 ? 3 : 6;
 }
-// Fragment layout of the prepared activations: per row, per super-block,
-// 9 steps x 4 lanes-in-quad (c) x 4 fp16 = 144 fp16 (288 bytes).
+__host__ __device__ constexpr float act_scale(int f) {
+    return f == 0 || f == 3 ? 1.0f : f == 1 || f == 4 ? 0.125f : 0.015625f;
+}
+// Prepared activations: per row and super-block, 8 steps x 4 lanes-in-quad
+// (c) x 4 fp16, then 16 fp16 of padding so that rows of a 16-row tile fall on
+// different shared-memory banks: 144 fp16 (288 bytes).
 constexpr int kFragHalvesPerSB = 144;
 
 // ---------------------------------------------------------------------------

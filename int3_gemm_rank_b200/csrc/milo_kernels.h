@@ -48,11 +48,20 @@ struct GemvParams {
 
 struct PrepParams {
     const uint16_t* src;        // [*, K] bf16/fp16 (or fp16 h)
-    const int32_t* row_src;     // row p -> source row (NULL: identity); -1 = zero row
+    int32_t* row_src;           // row p -> source row; built here when `rows` is set, else
+                                // read (NULL: identity); -1 = zero row
     uint16_t* frag;             // [R, SB*144] fp16
     float* gsum;                // [R, Gpad] f32
     int32_t* dev_status;
     int R, K, gpad, src_bf16;
+    // Row bookkeeping (first preparation of a call only): routed rows come from
+    // the router's offsets/perm, the n_shared*T shared-expert rows follow them.
+    int rows;                   // 1: build grp / row_src / inv from offsets and perm
+    const int32_t* offsets;     // [E+1]
+    const int32_t* perm;        // [T*k] or NULL (identity)
+    int32_t* grp;               // [E+S][2]: first row, row count
+    int32_t* inv;               // optional [T*k] inverse of perm (-1 = dropped)
+    int T, k, E, S, R_routed;
 };
 
 struct LorcParams {
@@ -61,19 +70,11 @@ struct LorcParams {
     const ProjDev* table;
     const int32_t* grp;         // [n_exp][2]
     uint16_t* t;                // [R, tcols] fp16
+    float* part;                // [splits][R][tcols] f32 partial sums over K slices
     int32_t* dev_status;
     int stride, proj_a, proj_b; // proj_b < 0: single projection
     int n_exp, K, R, tcols, t_col_b, src_bf16;
-};
-
-struct RowsParams {
-    const int32_t* offsets;     // [E+1] routed offsets
-    const int32_t* perm;        // [T*k] or NULL (identity)
-    int32_t* grp;               // [E+S][2]: first row, row count
-    int32_t* row_src;           // [R] source row (token) of each row, -1 if invalid
-    int32_t* inv;               // optional [T*k] inverse of perm (-1 = dropped)
-    int32_t* dev_status;
-    int T, k, E, S, R_routed;
+    int splits, row_groups;     // K slices (each a multiple of 128); row-tile strides
 };
 
 struct CombineParams {
@@ -90,7 +91,6 @@ size_t gemv_smem_bytes(bool glu);
 cudaError_t launch_gemv(const GemvParams& p, bool glu, int grid, cudaStream_t s);
 cudaError_t launch_prep(const PrepParams& p, cudaStream_t s);
 cudaError_t launch_lorc(const LorcParams& p, cudaStream_t s);
-cudaError_t launch_rows(const RowsParams& p, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 
 }  // namespace milo

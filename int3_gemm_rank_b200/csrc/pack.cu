@@ -81,29 +81,23 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
 
 // One thread per (row, super-block, unit): recover the 32 codes of a unit with
 // the register-level extraction of the GEMM (field masks, one shift by 9, the
-// nine-step schedule), so that its bit-exact parity covers that logic.
+// gathered spare register, the eight-step schedule), so that its bit-exact
+// parity covers that logic.
 template <int S, int H>
-__device__ __forceinline__ void unpack_reg(const uint32_t (&w)[3], const uint32_t (&hi)[3],
-                                           uint8_t (&u)[32], uint32_t& u30, uint32_t& u31) {
+__device__ __forceinline__ void unpack_reg(const uint32_t (&w)[3], const uint32_t (&hw)[3],
+                                           uint8_t (&u)[32]) {
     constexpr int t = sched_word(S, H), f = sched_field(S, H);
-    const uint32_t r = field<f>(w[t], hi[t]);
-    const uint32_t lo = r & 0xFFFFu, up = r >> 16;
-    if constexpr (f < 5) {
-        constexpr int sh = (f == 0 || f == 3) ? 0 : (f == 1 || f == 4) ? 3 : 6;
-        constexpr int m = reg_code(t, f);
-        u[m] = static_cast<uint8_t>(lo >> sh);
-        u[m + 1] = static_cast<uint8_t>(up >> sh);
-    } else {
-        u30 |= (lo >> 6) << t;
-        u31 |= (up >> 6) << t;
-    }
+    constexpr int m = reg_code(t, f), sh = field_shift(f);
+    const uint32_t r = unit_reg<t, f>(w, hw);
+    u[m] = static_cast<uint8_t>((r & 0xFFFFu) >> sh);
+    u[m + 1] = static_cast<uint8_t>((r >> 16) >> sh);
 }
 
 template <int S>
-__device__ __forceinline__ void unpack_step(const uint32_t (&w)[3], const uint32_t (&hi)[3],
-                                            uint8_t (&u)[32], uint32_t& u30, uint32_t& u31) {
-    unpack_reg<S, 0>(w, hi, u, u30, u31);
-    unpack_reg<S, 1>(w, hi, u, u30, u31);
+__device__ __forceinline__ void unpack_step(const uint32_t (&w)[3], const uint32_t (&hw)[3],
+                                            uint8_t (&u)[32]) {
+    unpack_reg<S, 0>(w, hw, u);
+    unpack_reg<S, 1>(w, hw, u);
 }
 
 __global__ void __launch_bounds__(128) unpack_kernel(const uint32_t* __restrict__ Q, int N, int K,
@@ -115,23 +109,19 @@ __global__ void __launch_bounds__(128) unpack_kernel(const uint32_t* __restrict_
     const long long nb = gid / 4;
     const int n = static_cast<int>(nb / SB), b = static_cast<int>(nb % SB);
     const uint32_t* src = Q + static_cast<size_t>(n) * (3 * K / 32) + 12 * b + 3 * c;
-    uint32_t w[3] = {src[0], src[1], src[2]};
-    uint32_t hi[3] = {w[0] >> 9, w[1] >> 9, w[2] >> 9};
+    const uint32_t w[3] = {src[0], src[1], src[2]};
+    const uint32_t hw[3] = {w[0] >> 9, w[1] >> 9, w[2] >> 9};
     uint8_t u[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) u[i] = 0xFF;   // a code the schedule misses stays 0xFF
-    uint32_t u30 = 0, u31 = 0;
-    unpack_step<0>(w, hi, u, u30, u31);
-    unpack_step<1>(w, hi, u, u30, u31);
-    unpack_step<2>(w, hi, u, u30, u31);
-    unpack_step<3>(w, hi, u, u30, u31);
-    unpack_step<4>(w, hi, u, u30, u31);
-    unpack_step<5>(w, hi, u, u30, u31);
-    unpack_step<6>(w, hi, u, u30, u31);
-    unpack_step<7>(w, hi, u, u30, u31);
-    unpack_step<8>(w, hi, u, u30, u31);
-    u[30] = static_cast<uint8_t>(u30);
-    u[31] = static_cast<uint8_t>(u31);
+    unpack_step<0>(w, hw, u);
+    unpack_step<1>(w, hw, u);
+    unpack_step<2>(w, hw, u);
+    unpack_step<3>(w, hw, u);
+    unpack_step<4>(w, hw, u);
+    unpack_step<5>(w, hw, u);
+    unpack_step<6>(w, hw, u);
+    unpack_step<7>(w, hw, u);
     uint8_t* out = codes + static_cast<size_t>(n) * K + 128 * b;
 #pragma unroll
     for (int m = 0; m < 32; ++m) out[unit_k(c, m)] = u[m];

@@ -180,8 +180,8 @@ def single(seed_workload: str = "single", n: int = 1024, k: int = 1024, rank: in
 
 
 def mixtral(T: int = 16, name: str = "mixtral", hidden: int = 4096, inter: int = 14336,
-            ranks=None, rank_choices=(0, 16, 32, 64)) -> MoEWorkload:
-    E = 8
+            ranks=None, rank_choices=(0, 16, 32, 64), n_experts: int = 8) -> MoEWorkload:
+    E = n_experts
     if ranks is None:
         ranks = list(rng_for(name, "ranks").choice(rank_choices, size=E).astype(int))
     x = gen_activations(rng_for(name, "x"), T, hidden, "bf16")
@@ -202,8 +202,8 @@ def deepseek(T: int = 64, name: str = "deepseek", hidden: int = 2048, inter: int
                        ranks, _experts(name, hidden, inter, ranks))
 
 
-def prefill(T: int = 8192, name: str = "prefill") -> MoEWorkload:
-    return mixtral(T=T, name=name, ranks=[64] * 8)
+def prefill(T: int = 8192, name: str = "prefill", n_experts: int = 8) -> MoEWorkload:
+    return mixtral(T=T, name=name, ranks=[64] * n_experts, n_experts=n_experts)
 
 
 def sweep(T: int, name: str = "sweep", hidden: int = 4096, inter: int = 14336,
