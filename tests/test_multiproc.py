@@ -1,0 +1,55 @@
+"""Multi-process plumbing of bench.py on CPU (gloo, world size 2).
+
+The layer has no cross-GPU exchange: each rank runs a replica on its own batch.
+What multi-GPU runs rely on is the host-side plumbing: the barrier, the max
+over ranks of the device time, and the reference arm running on rank 0 only.
+"""
+import os
+import socket
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out_dir):
+    sys.path.insert(0, ROOT)
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import bench
+    import torch.distributed as dist
+    bench.dist_init("gloo")
+    assert dist.get_world_size() == world
+    # each rank "measures" a different time; every rank must see the maximum
+    got = bench.max_over_ranks(10.0 + 5.0 * rank)
+    bench.barrier()
+    # the reference arm prints on rank 0 only; other ranks return 0 without work
+    ref_rc = bench.run_reference(type("A", (), {"steps": 1, "warmup": 0, "workload": "mixtral",
+                                                "experts": None, "tokens": None})()) if rank else 0
+    with open(os.path.join(out_dir, f"r{rank}.txt"), "w") as f:
+        f.write(f"{got} {ref_rc}")
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_rank0_only_reference(tmp_path):
+    import torch.multiprocessing as mp
+    port = _free_port()
+    mp.spawn(_worker, args=(2, port, str(tmp_path)), nprocs=2, join=True)
+    for r in range(2):
+        got, rc = open(tmp_path / f"r{r}.txt").read().split()
+        assert float(got) == 15.0
+        assert int(rc) == 0
+
+
+def test_single_process_max_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.25) == 3.25
+    assert bench.dist_env()[2] >= 1
