@@ -241,6 +241,37 @@ MILO_API milo_status milo_moe_forward(const milo_moe_layer* layer, const void* x
                              milo_dtype y_dt, void* ws, size_t ws_bytes,
                              int32_t* dev_status, void* stream);
 
+/*
+ * milo_grouped_linear_noalloc -- milo_grouped_linear for callers that cannot
+ * allocate device memory: code that is handed only its input and output
+ * buffers (for example behind a plugin or custom-operator interface with no
+ * allocator), or that must not call cudaMalloc on its path because the call
+ * can synchronise the device.  This entry point has no counterpart in the
+ * paper; it exists only for such callers.
+ *
+ * Same arguments and results as milo_grouped_linear, without ws / ws_bytes:
+ * the scratch lives in a buffer of MILO_NOALLOC_SCRATCH_BYTES compiled into
+ * the library, which every GPU that loads the library holds until the process
+ * exits.  Nothing here allocates (no cudaMalloc, cudaFree or allocating
+ * library routine).
+ *   - A call whose scratch need (milo_linear_workspace_bytes for the same
+ *     lin, T, k) exceeds MILO_NOALLOC_SCRATCH_BYTES returns MILO_ERR_WORKSPACE
+ *     and enqueues nothing; decode-sized calls (tens of rows) fit.
+ *   - The first call on each device looks up the buffer's device address
+ *     with that device current (cudaGetSymbolAddress); make that first call
+ *     before any stream capture.  A failed lookup returns MILO_ERR_CUDA.
+ *   - Every call on a device shares the one buffer and finds the previous
+ *     call's contents in it; nothing in it needs to start at zero (each call
+ *     writes what it reads).  Calls that overlap on the GPU (other streams,
+ *     other threads) race on the buffer: order them on one stream.
+ */
+#define MILO_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+MILO_API milo_status milo_grouped_linear_noalloc(const milo_linear* lin, const void* x,
+                                                 milo_dtype x_dt, int32_t T, int32_t k,
+                                                 const int32_t* expert_offsets,
+                                                 const int32_t* perm, void* y, milo_dtype y_dt,
+                                                 int32_t* dev_status, void* stream);
+
 /* Byte offset of h inside the forward workspace (see milo_moe_forward). */
 MILO_API size_t milo_moe_h_offset(const milo_moe_layer* layer, int32_t T);
 

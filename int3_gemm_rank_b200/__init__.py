@@ -30,7 +30,8 @@ MILO_GROUP, MILO_MAX_RANK = 64, 64
 EXPORTS = ("milo_status_str", "milo_last_error", "milo_version", "milo_pack", "milo_unpack",
            "milo_route", "milo_table_bytes", "milo_linear_prepare", "milo_layer_prepare",
            "milo_linear_workspace_bytes", "milo_moe_workspace_bytes", "milo_grouped_linear",
-           "milo_moe_forward", "milo_moe_h_offset", "milo_set_profile_events")
+           "milo_moe_forward", "milo_moe_h_offset", "milo_set_profile_events",
+           "milo_grouped_linear_noalloc")
 
 
 class MiloError(RuntimeError):
@@ -97,6 +98,9 @@ def lib() -> C.CDLL:
         L.milo_moe_h_offset.restype = sz
         L.milo_set_profile_events.argtypes = [C.POINTER(C.c_void_p), i32]
         L.milo_set_profile_events.restype = C.c_int
+        L.milo_grouped_linear_noalloc.argtypes = [C.POINTER(milo_linear), vp, C.c_int, i32, i32, vp, vp,
+                                                  vp, C.c_int, vp, vp]
+        L.milo_grouped_linear_noalloc.restype = C.c_int
         _lib = L
     return _lib
 
@@ -268,6 +272,20 @@ def milo_grouped_linear(lin: GroupedLinear, x, offsets, perm, k=1, out_dtype=tor
     _check(lib().milo_grouped_linear(C.byref(lin.cs), _ptr(x), _dt(x), T, k, _ptr(offsets), _ptr(perm),
                                      _ptr(y), _dt(y), C.c_void_p(wp), wn, _ptr(dev_status), _stream()),
            "milo_grouped_linear")
+    return y
+
+
+def milo_grouped_linear_noalloc(lin: GroupedLinear, x, offsets, perm, k=1, out_dtype=torch.float32,
+                                dev_status=None, y=None) -> torch.Tensor:
+    """milo_grouped_linear without a workspace argument: for callers that cannot
+    allocate device memory; the scratch is the library's built-in buffer."""
+    _cuda(x, "x")
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty((T * k, lin.cs.N), dtype=out_dtype, device=x.device)
+    _check(lib().milo_grouped_linear_noalloc(C.byref(lin.cs), _ptr(x), _dt(x), T, k, _ptr(offsets),
+                                             _ptr(perm), _ptr(y), _dt(y), _ptr(dev_status), _stream()),
+           "milo_grouped_linear_noalloc")
     return y
 
 
