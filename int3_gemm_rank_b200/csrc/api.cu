@@ -9,6 +9,7 @@
 // Every step is a kernel on the caller's stream; the host never waits.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -51,7 +52,8 @@ static EncodeTiledFn encode_fn() {
 // `pitch` bytes; box {bcols, brows}.
 static milo_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize,
                             uint64_t cols, uint64_t rows, uint64_t pitch, uint32_t bcols,
-                            uint32_t brows, const char* what) {
+                            uint32_t brows, const char* what,
+                            CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(MILO_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     cuuint64_t dims[2] = {cols, rows};
@@ -60,7 +62,7 @@ static milo_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataTyp
     cuuint32_t estr[2] = {1, 1};
     (void)esize;
     CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return fail(MILO_ERR_INVALID_ARG, std::string("tensor map encoding failed for ") + what +
@@ -284,6 +286,53 @@ static milo_status run_gemv(GemvParams& g, bool glu, cudaStream_t st, const char
     return check_cuda(launch_gemv(g, glu, grid, st), what);
 }
 
+// Which grouped-GEMM kernel runs: the tcgen05/TMEM one (default) or the
+// mma.sync one (MILO_GEMM=mma).  Both give the same results within fp32
+// rounding and are covered by the same parity tests.
+static bool use_tc() {
+    const char* v = getenv("MILO_GEMM");
+    return !(v && v[0] == 'm');
+}
+
+// Run the grouped GEMM described by g with the tcgen05 kernel: the activation
+// buffer holds the A-column-ordered layout ([R][K] fp16).
+static milo_status run_tc(const GemvParams& g, bool glu, void* acts, void* gsum, void* t,
+                          cudaStream_t st, const char* what) {
+    TcParams p;
+    memset(&p, 0, sizeof(p));
+    milo_status s;
+    const int Rm = std::max(g.R, 1);
+    if ((s = make_map(&p.b_map, acts, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, g.K, Rm,
+                      static_cast<uint64_t>(g.K) * 2, 64, kTokTile, "activations",
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != MILO_OK) return s;
+    if ((s = make_map(&p.g_map, gsum, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, gpad_of(g.K), Rm,
+                      static_cast<uint64_t>(gpad_of(g.K)) * 4, 4, kTokTile, "group sums")) != MILO_OK)
+        return s;
+    if (g.has_t &&
+        (s = make_map(&p.t_map, t, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, g.tcols, Rm,
+                      static_cast<uint64_t>(g.tcols) * 2, 64, kTokTile, "compensator rows",
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != MILO_OK) return s;
+    p.table = g.table;
+    p.grp = g.grp;
+    p.y_part = g.y_part;
+    p.h = g.h;
+    p.dev_status = g.dev_status;
+    p.stride = g.stride;
+    p.proj_a = g.proj_a;
+    p.proj_b = g.proj_b;
+    p.n_exp = g.n_exp;
+    p.N = g.N;
+    p.K = g.K;
+    p.R = g.R;
+    p.splits = g.splits;
+    p.chunks = g.chunks;
+    p.cps = g.cps;
+    p.has_t = g.has_t;
+    p.tcols = g.tcols;
+    p.t_col_b = g.t_col_b;
+    return check_cuda(launch_tc_gemm(p, glu, 2 * sm_count(), st), what);
+}
+
 }  // namespace milo
 
 using namespace milo;
@@ -415,9 +464,11 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     int32_t* rows = reinterpret_cast<int32_t*>(base + w.rows);
     int32_t* inv = reinterpret_cast<int32_t*>(base + w.inv);
 
+    const bool tc = use_tc();
     PrepParams pp{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.frag),
                   reinterpret_cast<float*>(base + w.gsum), dev_status, w.R, lin->K, gpad_of(lin->K),
-                  x_dt == MILO_BF16, 1, expert_offsets, perm, grp, inv, T, k, lin->n_experts, 0, w.R};
+                  x_dt == MILO_BF16, tc ? 1 : 0, 1, expert_offsets, perm, grp, inv, T, k, lin->n_experts, 0,
+                  w.R};
     milo_status s = check_cuda(launch_prep(pp, st), "prep");
     if (s != MILO_OK) return s;
 
@@ -433,7 +484,7 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
 
     GemvParams g;
     memset(&g, 0, sizeof(g));
-    if ((s = act_maps(g, base + w.frag, base + w.gsum, base + w.t, w.R, lin->K, w.tcols, has_t)) != MILO_OK)
+    if (!tc && (s = act_maps(g, base + w.frag, base + w.gsum, base + w.t, w.R, lin->K, w.tcols, has_t)) != MILO_OK)
         return s;
     g.table = table;
     g.grp = grp;
@@ -452,7 +503,9 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     g.has_t = has_t;
     g.tcols = w.tcols;
     prof_record(0, st);
-    if ((s = run_gemv(g, false, st, "gemv")) != MILO_OK) return s;
+    if (tc) s = run_tc(g, false, base + w.frag, base + w.gsum, base + w.t, st, "tc gemm");
+    else s = run_gemv(g, false, st, "gemv");
+    if (s != MILO_OK) return s;
     prof_record(1, st);
 
     CombineParams cp{reinterpret_cast<const float*>(base + w.part), inv, nullptr, y, dev_status,
@@ -487,9 +540,11 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     const bool has_t = L->max_rank > 0;
     milo_status s;
 
+    const bool tc = use_tc();
     PrepParams px{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.xfrag),
                   reinterpret_cast<float*>(base + w.xg), dev_status, w.R, H, gpad_of(H), x_dt == MILO_BF16,
-                  1, expert_offsets, perm, grp, nullptr, T, L->top_k, L->n_routed, L->n_shared, w.R_routed};
+                  tc ? 1 : 0, 1, expert_offsets, perm, grp, nullptr, T, L->top_k, L->n_routed, L->n_shared,
+                  w.R_routed};
     if ((s = check_cuda(launch_prep(px, st), "prep x")) != MILO_OK) return s;
     if (has_t) {
         LorcParams lp{static_cast<const uint16_t*>(x), rows, table, grp,
@@ -501,7 +556,8 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
 
     GemvParams g1;
     memset(&g1, 0, sizeof(g1));
-    if ((s = act_maps(g1, base + w.xfrag, base + w.xg, base + w.t13, w.R, H, w.tc13, has_t)) != MILO_OK) return s;
+    if (!tc && (s = act_maps(g1, base + w.xfrag, base + w.xg, base + w.t13, w.R, H, w.tc13, has_t)) != MILO_OK)
+        return s;
     g1.table = table;
     g1.grp = grp;
     g1.h = reinterpret_cast<uint16_t*>(base + w.h);
@@ -520,12 +576,15 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     g1.tcols = w.tc13;
     g1.t_col_b = L->max_rank;
     prof_record(0, st);
-    if ((s = run_gemv(g1, true, st, "gemv w1|w3")) != MILO_OK) return s;
+    if (tc) s = run_tc(g1, true, base + w.xfrag, base + w.xg, base + w.t13, st, "tc gemm w1|w3");
+    else s = run_gemv(g1, true, st, "gemv w1|w3");
+    if (s != MILO_OK) return s;
     prof_record(1, st);
 
     PrepParams ph{reinterpret_cast<const uint16_t*>(base + w.h), nullptr,
                   reinterpret_cast<uint16_t*>(base + w.hfrag), reinterpret_cast<float*>(base + w.hg),
-                  dev_status, w.R, I, gpad_of(I), 0, 0, nullptr, nullptr, nullptr, nullptr, 0, 0, 0, 0, 0};
+                  dev_status, w.R, I, gpad_of(I), 0, tc ? 1 : 0, 0, nullptr, nullptr, nullptr, nullptr, 0, 0, 0,
+                  0, 0};
     if ((s = check_cuda(launch_prep(ph, st), "prep h")) != MILO_OK) return s;
     if (has_t) {
         LorcParams lp{reinterpret_cast<const uint16_t*>(base + w.h), nullptr, table, grp,
@@ -536,7 +595,8 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
 
     GemvParams g2;
     memset(&g2, 0, sizeof(g2));
-    if ((s = act_maps(g2, base + w.hfrag, base + w.hg, base + w.t2, w.R, I, w.tc2, has_t)) != MILO_OK) return s;
+    if (!tc && (s = act_maps(g2, base + w.hfrag, base + w.hg, base + w.t2, w.R, I, w.tc2, has_t)) != MILO_OK)
+        return s;
     g2.table = table;
     g2.grp = grp;
     g2.y_part = reinterpret_cast<float*>(base + w.part);
@@ -554,7 +614,9 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     g2.has_t = has_t;
     g2.tcols = w.tc2;
     prof_record(2, st);
-    if ((s = run_gemv(g2, false, st, "gemv w2")) != MILO_OK) return s;
+    if (tc) s = run_tc(g2, false, base + w.hfrag, base + w.hg, base + w.t2, st, "tc gemm w2");
+    else s = run_gemv(g2, false, st, "gemv w2");
+    if (s != MILO_OK) return s;
     prof_record(3, st);
 
     CombineParams cp{reinterpret_cast<const float*>(base + w.part), inv_perm, topk_w, y, dev_status,

@@ -136,16 +136,30 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
             p.gsum[static_cast<size_t>(row) * p.gpad + 2 * sb] = s0;
             p.gsum[static_cast<size_t>(row) * p.gpad + 2 * sb + 1] = s1;
         }
-        uint2* out = reinterpret_cast<uint2*>(p.frag + (static_cast<size_t>(row) * SB + sb) * kFragHalvesPerSB) + c;
-        out[0 * 4] = frag_step<0>(x);
-        out[1 * 4] = frag_step<1>(x);
-        out[2 * 4] = frag_step<2>(x);
-        out[3 * 4] = frag_step<3>(x);
-        out[4 * 4] = frag_step<4>(x);
-        out[5 * 4] = frag_step<5>(x);
-        out[6 * 4] = frag_step<6>(x);
-        out[7 * 4] = frag_step<7>(x);
-        out[8 * 4] = make_uint2(0u, 0u);      // padding (bank spread)
+        if (p.layout == 0) {
+            // mma.sync: per super-block, step-major, lane-in-quad c, 4 fp16 each
+            uint2* out = reinterpret_cast<uint2*>(p.frag + (static_cast<size_t>(row) * SB + sb) * kFragHalvesPerSB) + c;
+            out[0 * 4] = frag_step<0>(x);
+            out[1 * 4] = frag_step<1>(x);
+            out[2 * 4] = frag_step<2>(x);
+            out[3 * 4] = frag_step<3>(x);
+            out[4 * 4] = frag_step<4>(x);
+            out[5 * 4] = frag_step<5>(x);
+            out[6 * 4] = frag_step<6>(x);
+            out[7 * 4] = frag_step<7>(x);
+            out[8 * 4] = make_uint2(0u, 0u);      // padding (bank spread)
+        } else {
+            // tcgen05: K slots in the order of the A columns (unit c's first-group
+            // registers at columns 8c..8c+7, its second-group ones at 32+8c..)
+            uint4* o1 = reinterpret_cast<uint4*>(p.frag + static_cast<size_t>(row) * p.K + 128 * sb + 16 * c);
+            uint4* o2 = reinterpret_cast<uint4*>(p.frag + static_cast<size_t>(row) * p.K + 128 * sb + 64 + 16 * c);
+            const uint2 f0 = frag_step<0>(x), f1 = frag_step<1>(x), f2 = frag_step<2>(x), f3 = frag_step<3>(x);
+            const uint2 f4 = frag_step<4>(x), f5 = frag_step<5>(x), f6 = frag_step<6>(x), f7 = frag_step<7>(x);
+            o1[0] = make_uint4(f0.x, f0.y, f1.x, f1.y);
+            o1[1] = make_uint4(f2.x, f2.y, f3.x, f3.y);
+            o2[0] = make_uint4(f4.x, f4.y, f5.x, f5.y);
+            o2[1] = make_uint4(f6.x, f6.y, f7.x, f7.y);
+        }
     }
     if (blockIdx.y == 0)
         for (int j = 2 * SB + threadIdx.x; j < p.gpad; j += blockDim.x)
@@ -196,7 +210,10 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
     const ProjDev* P = p.table + e * p.stride + (which == 0 ? p.proj_a : p.proj_b);
     const int r = P->rank;
     const int j0 = 16 * rblk;
-    if (j0 >= r) return;
+    // Columns [col0, col0 + span) of t belong to this projection.  Ranks past r
+    // are written as zeros so that an MMA over the whole span sees finite values.
+    const int span = p.proj_b >= 0 ? p.t_col_b : p.tcols;
+    if (j0 >= span) return;
     const int row0 = p.grp[2 * e], m = p.grp[2 * e + 1];
     if (m <= 0 || row0 < 0 || row0 + m > p.R) return;
     const int col0 = which == 0 ? 0 : p.t_col_b;
@@ -205,6 +222,15 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
     const int kbeg = split * slice;
     float* out = p.part + static_cast<size_t>(split) * p.R * p.tcols;
     int32_t st = 0;
+    if (j0 >= r) {   // ranks of this block are all past r: zeros only
+        for (int mt = 16 * blockIdx.y; mt < m; mt += 16 * p.row_groups)
+            for (int idx = threadIdx.x; idx < 256; idx += blockDim.x) {
+                const int rr = idx / 16, jj = idx % 16;
+                if (mt + rr < m && j0 + jj < span)
+                    out[static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j0 + jj] = 0.0f;
+            }
+        return;
+    }
     for (int mt = 16 * blockIdx.y; mt < m; mt += 16 * p.row_groups) {
         __syncthreads();
         if (threadIdx.x < 16) {
@@ -267,8 +293,8 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
         for (int idx = threadIdx.x; idx < 256; idx += blockDim.x) {
             const int rr = idx / 16, jj = idx % 16;
             const float v = ((part[0][rr][jj] + part[1][rr][jj]) + part[2][rr][jj]) + part[3][rr][jj];
-            if (mt + rr < m && j0 + jj < r)
-                out[static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j0 + jj] = v;
+            if (mt + rr < m && j0 + jj < span)
+                out[static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j0 + jj] = j0 + jj < r ? v : 0.0f;
         }
     }
     flag(p.dev_status, st);

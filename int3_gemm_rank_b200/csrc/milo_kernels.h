@@ -54,6 +54,7 @@ struct PrepParams {
     float* gsum;                // [R, Gpad] f32
     int32_t* dev_status;
     int R, K, gpad, src_bf16;
+    int layout;                 // 0: mma.sync fragments [R][K/128][144]; 1: tcgen05 A-column order [R][K]
     // Row bookkeeping (first preparation of a call only): routed rows come from
     // the router's offsets/perm, the n_shared*T shared-expert rows follow them.
     int rows;                   // 1: build grp / row_src / inv from offsets and perm
@@ -87,6 +88,24 @@ struct CombineParams {
     int per_slot;               // 1: y row per flat slot (grouped linear), 0: per token
 };
 
+// Parameters of the tcgen05 grouped GEMM (gemm_tc.cu).
+struct TcParams {
+    CUtensorMap b_map;          // activations in A-column order [R, K] fp16, box {64, 16}, 128B swizzle
+    CUtensorMap g_map;          // group sums [R, Gpad] f32, box {4, 16}
+    CUtensorMap t_map;          // compensator activations [R, tcols] fp16, box {64, 16}, 128B swizzle
+    const ProjDev* table;
+    const int32_t* grp;
+    float* y_part;
+    uint16_t* h;
+    int32_t* dev_status;
+    int stride, proj_a, proj_b;
+    int n_exp, N, K, R;
+    int splits, chunks, cps;
+    int has_t, tcols, t_col_b;
+};
+
+size_t tc_smem_bytes();
+cudaError_t launch_tc_gemm(const TcParams& p, bool glu, int grid, cudaStream_t s);
 size_t gemv_smem_bytes(bool glu);
 cudaError_t launch_gemv(const GemvParams& p, bool glu, int grid, cudaStream_t s);
 cudaError_t launch_prep(const PrepParams& p, cudaStream_t s);
