@@ -286,12 +286,14 @@ static milo_status run_gemv(GemvParams& g, bool glu, cudaStream_t st, const char
     return check_cuda(launch_gemv(g, glu, grid, st), what);
 }
 
-// Which grouped-GEMM kernel runs: the tcgen05/TMEM one (default) or the
-// mma.sync one (MILO_GEMM=mma).  Both give the same results within fp32
-// rounding and are covered by the same parity tests.
+// Which grouped-GEMM kernel runs: the mma.sync one (default) or the
+// tcgen05/TMEM one (MILO_GEMM=tc).  Both give the same results within fp32
+// rounding and are covered by the same parity tests.  At decode sizes (16
+// routed rows per tile) a tcgen05.mma of M=128, K=16 costs about as much to
+// issue as one with N=64, so the warp-level MMA is faster there.
 static bool use_tc() {
     const char* v = getenv("MILO_GEMM");
-    return !(v && v[0] == 'm');
+    return v && v[0] == 't';
 }
 
 // Run the grouped GEMM described by g with the tcgen05 kernel: the activation
