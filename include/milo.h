@@ -92,10 +92,19 @@ MILO_API int32_t milo_version(void);
  * and word t (0..2) of the unit holds, for i = 0..4,
  *     bits [3i, 3i+3) = u_{10t+2i},   bits [16+3i, 16+3i+3) = u_{10t+2i+1},
  * bit 15 = bit t of u_30, bit 31 = bit t of u_31.
- * Q is u32 [N, 3K/32] row-major (row pitch 3K/8 bytes).  scale and zero are
- * fp16 [K/64, N] (group-major, N contiguous).  Dequantisation:
- *     w_hat[n, k] = (q[n, k] - zero[k/64, n]) * scale[k/64, n].
+ *
+ * Device layout: rows are grouped in tiles of 64 (the last tile padded with
+ * zero rows, Npad = 64 * ceil(N/64)), so that the kernels fetch the words of
+ * a tile for one K chunk, and its scales and zeros, as contiguous blocks:
+ *     Q     u32  [Npad/64][K/128][64][12]:  Q[n/64][b][n%64][j] = word 12b+j of row n
+ *     scale fp16 [Npad/64][K/64][64]:       scale[n/64][g][n%64] = s of row n, group g
+ *     zero  fp16 [Npad/64][K/64][64]        (same layout)
+ * Dequantisation: w_hat[n, k] = (q[n, k] - z[n, k/64]) * s[n, k/64].
+ * milo_packed_bytes gives the buffer sizes.
  */
+
+/* Bytes of Q and of each of scale, zero for a weight [N, K] (K % 128 == 0). */
+MILO_API milo_status milo_packed_bytes(int32_t N, int32_t K, size_t* q_bytes, size_t* group_bytes);
 
 /*
  * milo_pack -- quantise W fp16 [N, K] (row-major) to int3 and pack it.
@@ -104,7 +113,8 @@ MILO_API int32_t milo_version(void);
  *     s = fp16((max - min) / 7)   (s := 1 when it rounds to 0)
  *     z = fp16(-min / s)
  *     q = clamp(rint(w / s + z), 0, 7)    (fp32, ties to even, no FMA)
- * Writes Q u32 [N, 3K/32], scale and zero fp16 [K/64, N].
+ * Writes Q, scale and zero in the device layout above, padding rows included
+ * (sizes from milo_packed_bytes; Q 16-byte aligned).
  * Errors: group != 64 or K % 128 != 0 -> UNSUPPORTED_SHAPE; N, K <= 0 or NULL
  * pointers -> INVALID_ARG.  Device: NONFINITE for NaN/Inf weights, FP16_RANGE
  * when s or z overflows fp16.  dev_status may be NULL.
@@ -114,8 +124,9 @@ MILO_API milo_status milo_pack(const uint16_t* W, int32_t N, int32_t K, int32_t 
                       int32_t* dev_status, void* stream);
 
 /*
- * milo_unpack -- extract the codes of Q u32 [N, 3K/32] into codes u8 [N, K],
- * with the same register-level field extraction the GEMM kernels use.
+ * milo_unpack -- extract the codes of Q (device layout above) into codes
+ * u8 [N, K] row-major, with the same register-level field extraction the GEMM
+ * kernels use.
  */
 MILO_API milo_status milo_unpack(const uint32_t* Q, int32_t N, int32_t K, uint8_t* codes,
                         void* stream);
@@ -187,7 +198,7 @@ MILO_API milo_status milo_table_bytes(int32_t n_projections, size_t* bytes);
 /*
  * milo_linear_prepare / milo_layer_prepare -- validate the weights (host
  * array `weights` / `experts` of device pointers) and write the device table
- * (TMA tensor maps and pointers) to `device_table`, which the caller keeps
+ * (pointers and shapes) to `device_table`, which the caller keeps
  * alive and unmodified while the layer is used.  One-time set-up: the table is
  * copied with a synchronous cudaMemcpy.  lin/layer are host structs; the
  * caller fills the shape fields and the call sets max_rank and table.

@@ -31,7 +31,7 @@ EXPORTS = ("milo_status_str", "milo_last_error", "milo_version", "milo_pack", "m
            "milo_route", "milo_table_bytes", "milo_linear_prepare", "milo_layer_prepare",
            "milo_linear_workspace_bytes", "milo_moe_workspace_bytes", "milo_grouped_linear",
            "milo_moe_forward", "milo_moe_h_offset", "milo_set_profile_events",
-           "milo_grouped_linear_noalloc")
+           "milo_grouped_linear_noalloc", "milo_packed_bytes")
 
 
 class MiloError(RuntimeError):
@@ -77,6 +77,8 @@ def lib() -> C.CDLL:
         L.milo_version.argtypes = []; L.milo_version.restype = i32
         L.milo_pack.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp]; L.milo_pack.restype = C.c_int
         L.milo_unpack.argtypes = [vp, i32, i32, vp, vp]; L.milo_unpack.restype = C.c_int
+        L.milo_packed_bytes.argtypes = [i32, i32, C.POINTER(sz), C.POINTER(sz)]
+        L.milo_packed_bytes.restype = C.c_int
         L.milo_route.argtypes = [vp, i32, i32, i32, u32, vp, vp, vp, vp, vp, vp, vp]
         L.milo_route.restype = C.c_int
         L.milo_table_bytes.argtypes = [i32, C.POINTER(sz)]; L.milo_table_bytes.restype = C.c_int
@@ -147,20 +149,31 @@ def new_status(device=None) -> torch.Tensor:
 # ---------------------------------------------------------------------------
 
 def milo_pack(W: torch.Tensor, group: int = MILO_GROUP, dev_status: torch.Tensor | None = None):
-    """Quantise W fp16 [N, K] to int3 and pack: returns (Q u32-as-int32 [N, 3K/32], scale, zero [K/64, N])."""
+    """Quantise W fp16 [N, K] to int3 and pack it in the device layout of milo.h.
+
+    Returns (Q int32 [Npad/64, K/128, 64, 12], scale, zero fp16 [Npad/64, K/64, 64]),
+    Npad = 64 * ceil(N / 64)."""
     _cuda(W, "W")
     N, K = W.shape
-    Q = torch.empty((N, 3 * K // 32), dtype=torch.int32, device=W.device)
-    s = torch.empty((K // group, N), dtype=torch.float16, device=W.device)
-    z = torch.empty((K // group, N), dtype=torch.float16, device=W.device)
+    NT = (N + 63) // 64
+    Q = torch.empty((NT, K // 128, 64, 12), dtype=torch.int32, device=W.device)
+    s = torch.empty((NT, K // group, 64), dtype=torch.float16, device=W.device)
+    z = torch.empty((NT, K // group, 64), dtype=torch.float16, device=W.device)
     _check(lib().milo_pack(_ptr(W), N, K, group, _ptr(Q), _ptr(s), _ptr(z), _ptr(dev_status),
                            _stream()), "milo_pack")
     return Q, s, z
 
 
-def milo_unpack(Q: torch.Tensor, K: int) -> torch.Tensor:
+def milo_packed_bytes(N: int, K: int) -> tuple:
+    """(bytes of Q, bytes of each of scale and zero) for a weight [N, K]."""
+    qb, gb = C.c_size_t(), C.c_size_t()
+    _check(lib().milo_packed_bytes(N, K, C.byref(qb), C.byref(gb)), "milo_packed_bytes")
+    return qb.value, gb.value
+
+
+def milo_unpack(Q: torch.Tensor, N: int, K: int) -> torch.Tensor:
+    """Codes u8 [N, K] of packed words Q (device layout)."""
     _cuda(Q, "Q")
-    N = Q.shape[0]
     codes = torch.empty((N, K), dtype=torch.uint8, device=Q.device)
     _check(lib().milo_unpack(_ptr(Q), N, K, _ptr(codes), _stream()), "milo_unpack")
     return codes
@@ -199,20 +212,20 @@ def milo_route(logits: torch.Tensor | None, k: int, renorm: bool, E: int | None 
 # ---------------------------------------------------------------------------
 
 class QWeight:
-    """A packed projection on the device: Q, scale, zero and the compensator U [N, r], V [r, K]."""
+    """A packed projection W [N, K] on the device: Q, scale, zero (device layout of
+    milo.h) and the compensator U [N, r], V [r, K]."""
 
-    def __init__(self, Q, scale, zero, U=None, V=None):
+    def __init__(self, Q, scale, zero, N: int, K: int, U=None, V=None):
         self.Q, self.scale, self.zero = Q, scale, zero
+        self.N, self.K = int(N), int(K)
         self.rank = 0 if U is None or U.numel() == 0 else int(U.shape[1])
         self.U = U if self.rank else None
         self.V = V if self.rank else None
-        self.N = Q.shape[0]
-        self.K = Q.shape[1] * 32 // 3
 
     @classmethod
     def quantize(cls, W: torch.Tensor, U=None, V=None, dev_status=None):
         Q, s, z = milo_pack(W, dev_status=dev_status)
-        return cls(Q, s, z, U, V)
+        return cls(Q, s, z, W.shape[0], W.shape[1], U, V)
 
     def cstruct(self) -> milo_qweight:
         return milo_qweight(self.Q.data_ptr(), self.scale.data_ptr(), self.zero.data_ptr(),

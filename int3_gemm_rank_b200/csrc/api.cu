@@ -1,5 +1,5 @@
-// api.cu -- host side of libmilo: argument validation, device tables (TMA
-// tensor maps), workspace layout and the launch sequence of the forward.
+// api.cu -- host side of libmilo: argument validation, device tables,
+// workspace layout and the launch sequence of the forward.
 //
 // The sequence for one MoE layer ("MiLo: Efficient Quantized MoE Inference
 // with Mixture of Low-Rank Compensators": routed experts, each a quantised
@@ -27,49 +27,6 @@ static thread_local std::string g_last_error;
 void clear_error() { g_last_error.clear(); }
 void set_error(const std::string& msg) { g_last_error = msg; }
 
-// ---------------------------------------------------------------------------
-// tensor maps (driver entry point fetched through the runtime; no -lcuda)
-// ---------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-// 2-D row-major tensor [rows, cols] of `esize`-byte elements with row pitch
-// `pitch` bytes; box {bcols, brows}.
-static milo_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize,
-                            uint64_t cols, uint64_t rows, uint64_t pitch, uint32_t bcols,
-                            uint32_t brows, const char* what,
-                            CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return fail(MILO_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {pitch};
-    cuuint32_t box[2] = {bcols, brows};
-    cuuint32_t estr[2] = {1, 1};
-    (void)esize;
-    CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS)
-        return fail(MILO_ERR_INVALID_ARG, std::string("tensor map encoding failed for ") + what +
-                                              " (code " + std::to_string(static_cast<int>(r)) + ")");
-    return MILO_OK;
-}
-
 // Measurement hook (milo_set_profile_events).
 static cudaEvent_t g_prof[4] = {nullptr, nullptr, nullptr, nullptr};
 static int g_prof_n = 0;
@@ -87,8 +44,7 @@ static int sm_count() {
 // ---------------------------------------------------------------------------
 // tables
 // ---------------------------------------------------------------------------
-static milo_status fill_proj(ProjDev* d, const milo_qweight& w, int N, int K, int tile_rows,
-                             const char* what) {
+static milo_status fill_proj(ProjDev* d, const milo_qweight& w, int N, int K, const char* what) {
     memset(d, 0, sizeof(*d));
     if (!w.q || !w.scale || !w.zero)
         return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": NULL weight pointer");
@@ -100,17 +56,6 @@ static milo_status fill_proj(ProjDev* d, const milo_qweight& w, int N, int K, in
     if (!aligned(w.q, 16) || !aligned(w.scale, 16) || !aligned(w.zero, 16) ||
         (w.rank > 0 && (!aligned(w.U, 16) || !aligned(w.V, 16))))
         return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": pointers must be 16-byte aligned");
-    const int G = K / MILO_GROUP;
-    milo_status s;
-    if ((s = make_map(&d->q_map, w.q, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 3 * K / 32, N,
-                      static_cast<uint64_t>(3 * K / 32) * 4, 12, tile_rows, what)) != MILO_OK) return s;
-    if ((s = make_map(&d->s_map, w.scale, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, N, G,
-                      static_cast<uint64_t>(N) * 2, tile_rows, 4, what)) != MILO_OK) return s;
-    if ((s = make_map(&d->z_map, w.zero, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, N, G,
-                      static_cast<uint64_t>(N) * 2, tile_rows, 4, what)) != MILO_OK) return s;
-    if (w.rank > 0 &&
-        (s = make_map(&d->u_map, w.U, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w.rank, N,
-                      static_cast<uint64_t>(w.rank) * 2, w.rank, tile_rows, what)) != MILO_OK) return s;
     d->q = w.q;
     d->scale = w.scale;
     d->zero = w.zero;
@@ -119,7 +64,6 @@ static milo_status fill_proj(ProjDev* d, const milo_qweight& w, int N, int K, in
     d->rank = w.rank;
     d->N = N;
     d->K = K;
-    d->tile_rows = tile_rows;
     return MILO_OK;
 }
 
@@ -150,8 +94,12 @@ struct Carve {
     }
 };
 
-static int gpad_of(int K) { return static_cast<int>(round_up(K / MILO_GROUP, 4)); }
-static size_t frag_row_bytes(int K) { return static_cast<size_t>(K / 128) * 288; }
+// Prepared activations and group sums of R rows: chunk-major (K chunks of 256).
+static int chunks_of(int K) { return (K + kChunkK - 1) / kChunkK; }
+static size_t frag_bytes(int K, int R) {
+    return static_cast<size_t>(chunks_of(K)) * R * kFragRowHalves * 2;
+}
+static size_t gsum_bytes(int K, int R) { return static_cast<size_t>(chunks_of(K)) * R * 16; }
 
 struct LorcPlan {
     int splits, row_groups;
@@ -212,8 +160,8 @@ static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
     w.grp = c.take(static_cast<size_t>(n_exp) * 8);
     w.rows = c.take(static_cast<size_t>(w.R) * 4);
     w.inv = c.take(static_cast<size_t>(w.R) * 4);
-    w.frag = c.take(static_cast<size_t>(w.R) * frag_row_bytes(lin->K));
-    w.gsum = c.take(static_cast<size_t>(w.R) * gpad_of(lin->K) * 4);
+    w.frag = c.take(frag_bytes(lin->K, w.R));
+    w.gsum = c.take(gsum_bytes(lin->K, w.R));
     w.t = c.take(static_cast<size_t>(w.R) * w.tcols * 2);
     w.lp = lorc_plan(n_exp, 1, lin->K, std::max(1LL, static_cast<long long>(w.R) / std::max<long long>(1, groups)));
     w.tpart = c.take(static_cast<size_t>(w.lp.splits) * w.R * w.tcols * 4);
@@ -242,12 +190,12 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
     w.tc2 = std::max(8, L->max_rank);
     w.grp = c.take(static_cast<size_t>(n_exp) * 8);
     w.rows = c.take(static_cast<size_t>(w.R) * 4);
-    w.xfrag = c.take(static_cast<size_t>(w.R) * frag_row_bytes(H));
-    w.xg = c.take(static_cast<size_t>(w.R) * gpad_of(H) * 4);
+    w.xfrag = c.take(frag_bytes(H, w.R));
+    w.xg = c.take(gsum_bytes(H, w.R));
     w.t13 = c.take(static_cast<size_t>(w.R) * w.tc13 * 2);
     w.h = c.take(static_cast<size_t>(w.R) * I * 2);
-    w.hfrag = c.take(static_cast<size_t>(w.R) * frag_row_bytes(I));
-    w.hg = c.take(static_cast<size_t>(w.R) * gpad_of(I) * 4);
+    w.hfrag = c.take(frag_bytes(I, w.R));
+    w.hg = c.take(gsum_bytes(I, w.R));
     w.t2 = c.take(static_cast<size_t>(w.R) * w.tc2 * 2);
     const long long rows_per_exp = std::max(1LL, static_cast<long long>(w.R) / std::max<long long>(1, groups));
     w.lp13 = lorc_plan(n_exp, 2, H, rows_per_exp);
@@ -262,77 +210,22 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
 // ---------------------------------------------------------------------------
 // launch helpers
 // ---------------------------------------------------------------------------
-static milo_status act_maps(GemvParams& g, void* frag, void* gsum, void* t, int R, int K, int tcols,
-                            bool has_t) {
-    milo_status s;
-    const int SB = K / 128;
-    const int Rm = std::max(R, 1);
-    if ((s = make_map(&g.x_map, frag, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<uint64_t>(SB) * 144, Rm,
-                      frag_row_bytes(K), 144, kTokTile, "activations")) != MILO_OK) return s;
-    if ((s = make_map(&g.g_map, gsum, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, gpad_of(K), Rm,
-                      static_cast<uint64_t>(gpad_of(K)) * 4, 4, kTokTile, "group sums")) != MILO_OK) return s;
-    if (has_t) {
-        if ((s = make_map(&g.t_map, t, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, tcols, Rm,
-                          static_cast<uint64_t>(tcols) * 2, tcols, kTokTile, "compensator rows")) != MILO_OK)
-            return s;
-    } else {
-        memset(&g.t_map, 0, sizeof(g.t_map));
-    }
-    return MILO_OK;
+static void act_ptrs(GemvParams& g, void* frag, void* gsum, void* t, int R, int K, int tcols, bool has_t) {
+    g.x = static_cast<const uint16_t*>(frag);
+    g.gsum = static_cast<const float*>(gsum);
+    g.t = has_t ? static_cast<const uint16_t*>(t) : nullptr;
+    g.R = R;
+    g.K = K;
+    g.SB = K / 128;
+    g.G = K / MILO_GROUP;
+    g.chunks = chunks_of(K);
+    g.has_t = has_t;
+    g.tcols = tcols;
 }
 
 static milo_status run_gemv(GemvParams& g, bool glu, cudaStream_t st, const char* what) {
     const int grid = 3 * sm_count();
     return check_cuda(launch_gemv(g, glu, grid, st), what);
-}
-
-// Which grouped-GEMM kernel runs: the mma.sync one (default) or the
-// tcgen05/TMEM one (MILO_GEMM=tc).  Both give the same results within fp32
-// rounding and are covered by the same parity tests.  At decode sizes (16
-// routed rows per tile) a tcgen05.mma of M=128, K=16 costs about as much to
-// issue as one with N=64, so the warp-level MMA is faster there.
-static bool use_tc() {
-    const char* v = getenv("MILO_GEMM");
-    return v && v[0] == 't';
-}
-
-// Run the grouped GEMM described by g with the tcgen05 kernel: the activation
-// buffer holds the A-column-ordered layout ([R][K] fp16).
-static milo_status run_tc(const GemvParams& g, bool glu, void* acts, void* gsum, void* t,
-                          cudaStream_t st, const char* what) {
-    TcParams p;
-    memset(&p, 0, sizeof(p));
-    milo_status s;
-    const int Rm = std::max(g.R, 1);
-    if ((s = make_map(&p.b_map, acts, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, g.K, Rm,
-                      static_cast<uint64_t>(g.K) * 2, 64, kTokTile, "activations",
-                      CU_TENSOR_MAP_SWIZZLE_128B)) != MILO_OK) return s;
-    if ((s = make_map(&p.g_map, gsum, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, gpad_of(g.K), Rm,
-                      static_cast<uint64_t>(gpad_of(g.K)) * 4, 4, kTokTile, "group sums")) != MILO_OK)
-        return s;
-    if (g.has_t &&
-        (s = make_map(&p.t_map, t, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, g.tcols, Rm,
-                      static_cast<uint64_t>(g.tcols) * 2, 64, kTokTile, "compensator rows",
-                      CU_TENSOR_MAP_SWIZZLE_128B)) != MILO_OK) return s;
-    p.table = g.table;
-    p.grp = g.grp;
-    p.y_part = g.y_part;
-    p.h = g.h;
-    p.dev_status = g.dev_status;
-    p.stride = g.stride;
-    p.proj_a = g.proj_a;
-    p.proj_b = g.proj_b;
-    p.n_exp = g.n_exp;
-    p.N = g.N;
-    p.K = g.K;
-    p.R = g.R;
-    p.splits = g.splits;
-    p.chunks = g.chunks;
-    p.cps = g.cps;
-    p.has_t = g.has_t;
-    p.tcols = g.tcols;
-    p.t_col_b = g.t_col_b;
-    return check_cuda(launch_tc_gemm(p, glu, 2 * sm_count(), st), what);
 }
 
 }  // namespace milo
@@ -386,7 +279,7 @@ extern "C" milo_status milo_linear_prepare(milo_linear* lin, const milo_qweight*
     std::vector<ProjDev> t(lin->n_experts);
     int rmax = 0;
     for (int e = 0; e < lin->n_experts; ++e) {
-        if ((s = fill_proj(&t[e], weights[e], lin->N, lin->K, kRowsPlain, "milo_linear_prepare")) != MILO_OK)
+        if ((s = fill_proj(&t[e], weights[e], lin->N, lin->K, "milo_linear_prepare")) != MILO_OK)
             return s;
         rmax = std::max(rmax, weights[e].rank);
     }
@@ -413,9 +306,9 @@ extern "C" milo_status milo_layer_prepare(milo_moe_layer* L, const milo_expert* 
     std::vector<ProjDev> t(3 * static_cast<size_t>(n_exp));
     int rmax = 0;
     for (int e = 0; e < n_exp; ++e) {
-        if ((s = fill_proj(&t[3 * e + 0], experts[e].w1, L->inter, L->hidden, kRowsGlu, "w1")) != MILO_OK) return s;
-        if ((s = fill_proj(&t[3 * e + 1], experts[e].w3, L->inter, L->hidden, kRowsGlu, "w3")) != MILO_OK) return s;
-        if ((s = fill_proj(&t[3 * e + 2], experts[e].w2, L->hidden, L->inter, kRowsPlain, "w2")) != MILO_OK) return s;
+        if ((s = fill_proj(&t[3 * e + 0], experts[e].w1, L->inter, L->hidden, "w1")) != MILO_OK) return s;
+        if ((s = fill_proj(&t[3 * e + 1], experts[e].w3, L->inter, L->hidden, "w3")) != MILO_OK) return s;
+        if ((s = fill_proj(&t[3 * e + 2], experts[e].w2, L->hidden, L->inter, "w2")) != MILO_OK) return s;
         rmax = std::max({rmax, experts[e].w1.rank, experts[e].w3.rank, experts[e].w2.rank});
     }
     if ((s = upload(device_table, table_bytes, t)) != MILO_OK) return s;
@@ -466,11 +359,9 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     int32_t* rows = reinterpret_cast<int32_t*>(base + w.rows);
     int32_t* inv = reinterpret_cast<int32_t*>(base + w.inv);
 
-    const bool tc = use_tc();
     PrepParams pp{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.frag),
-                  reinterpret_cast<float*>(base + w.gsum), dev_status, w.R, lin->K, gpad_of(lin->K),
-                  x_dt == MILO_BF16, tc ? 1 : 0, 1, expert_offsets, perm, grp, inv, T, k, lin->n_experts, 0,
-                  w.R};
+                  reinterpret_cast<float*>(base + w.gsum), dev_status, w.R, lin->K, x_dt == MILO_BF16, 1,
+                  expert_offsets, perm, grp, inv, T, k, lin->n_experts, 0, w.R};
     milo_status s = check_cuda(launch_prep(pp, st), "prep");
     if (s != MILO_OK) return s;
 
@@ -486,8 +377,7 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
 
     GemvParams g;
     memset(&g, 0, sizeof(g));
-    if (!tc && (s = act_maps(g, base + w.frag, base + w.gsum, base + w.t, w.R, lin->K, w.tcols, has_t)) != MILO_OK)
-        return s;
+    act_ptrs(g, base + w.frag, base + w.gsum, base + w.t, w.R, lin->K, w.tcols, has_t);
     g.table = table;
     g.grp = grp;
     g.y_part = reinterpret_cast<float*>(base + w.part);
@@ -497,17 +387,10 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     g.proj_b = 0;
     g.n_exp = lin->n_experts;
     g.N = lin->N;
-    g.K = lin->K;
-    g.R = w.R;
-    g.chunks = (lin->K + kChunkK - 1) / kChunkK;
     g.splits = w.splits;
     g.cps = (g.chunks + w.splits - 1) / w.splits;
-    g.has_t = has_t;
-    g.tcols = w.tcols;
     prof_record(0, st);
-    if (tc) s = run_tc(g, false, base + w.frag, base + w.gsum, base + w.t, st, "tc gemm");
-    else s = run_gemv(g, false, st, "gemv");
-    if (s != MILO_OK) return s;
+    if ((s = run_gemv(g, false, st, "gemv")) != MILO_OK) return s;
     prof_record(1, st);
 
     CombineParams cp{reinterpret_cast<const float*>(base + w.part), inv, nullptr, y, dev_status,
@@ -542,11 +425,9 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     const bool has_t = L->max_rank > 0;
     milo_status s;
 
-    const bool tc = use_tc();
     PrepParams px{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.xfrag),
-                  reinterpret_cast<float*>(base + w.xg), dev_status, w.R, H, gpad_of(H), x_dt == MILO_BF16,
-                  tc ? 1 : 0, 1, expert_offsets, perm, grp, nullptr, T, L->top_k, L->n_routed, L->n_shared,
-                  w.R_routed};
+                  reinterpret_cast<float*>(base + w.xg), dev_status, w.R, H, x_dt == MILO_BF16, 1,
+                  expert_offsets, perm, grp, nullptr, T, L->top_k, L->n_routed, L->n_shared, w.R_routed};
     if ((s = check_cuda(launch_prep(px, st), "prep x")) != MILO_OK) return s;
     if (has_t) {
         LorcParams lp{static_cast<const uint16_t*>(x), rows, table, grp,
@@ -558,8 +439,7 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
 
     GemvParams g1;
     memset(&g1, 0, sizeof(g1));
-    if (!tc && (s = act_maps(g1, base + w.xfrag, base + w.xg, base + w.t13, w.R, H, w.tc13, has_t)) != MILO_OK)
-        return s;
+    act_ptrs(g1, base + w.xfrag, base + w.xg, base + w.t13, w.R, H, w.tc13, has_t);
     g1.table = table;
     g1.grp = grp;
     g1.h = reinterpret_cast<uint16_t*>(base + w.h);
@@ -569,24 +449,16 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     g1.proj_b = 1;
     g1.n_exp = n_exp;
     g1.N = I;
-    g1.K = H;
-    g1.R = w.R;
-    g1.chunks = (H + kChunkK - 1) / kChunkK;
     g1.splits = 1;
     g1.cps = g1.chunks;
-    g1.has_t = has_t;
-    g1.tcols = w.tc13;
     g1.t_col_b = L->max_rank;
     prof_record(0, st);
-    if (tc) s = run_tc(g1, true, base + w.xfrag, base + w.xg, base + w.t13, st, "tc gemm w1|w3");
-    else s = run_gemv(g1, true, st, "gemv w1|w3");
-    if (s != MILO_OK) return s;
+    if ((s = run_gemv(g1, true, st, "gemv w1|w3")) != MILO_OK) return s;
     prof_record(1, st);
 
     PrepParams ph{reinterpret_cast<const uint16_t*>(base + w.h), nullptr,
                   reinterpret_cast<uint16_t*>(base + w.hfrag), reinterpret_cast<float*>(base + w.hg),
-                  dev_status, w.R, I, gpad_of(I), 0, tc ? 1 : 0, 0, nullptr, nullptr, nullptr, nullptr, 0, 0, 0,
-                  0, 0};
+                  dev_status, w.R, I, 0, 0, nullptr, nullptr, nullptr, nullptr, 0, 0, 0, 0, 0};
     if ((s = check_cuda(launch_prep(ph, st), "prep h")) != MILO_OK) return s;
     if (has_t) {
         LorcParams lp{reinterpret_cast<const uint16_t*>(base + w.h), nullptr, table, grp,
@@ -597,8 +469,7 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
 
     GemvParams g2;
     memset(&g2, 0, sizeof(g2));
-    if (!tc && (s = act_maps(g2, base + w.hfrag, base + w.hg, base + w.t2, w.R, I, w.tc2, has_t)) != MILO_OK)
-        return s;
+    act_ptrs(g2, base + w.hfrag, base + w.hg, base + w.t2, w.R, I, w.tc2, has_t);
     g2.table = table;
     g2.grp = grp;
     g2.y_part = reinterpret_cast<float*>(base + w.part);
@@ -608,17 +479,10 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     g2.proj_b = 2;
     g2.n_exp = n_exp;
     g2.N = H;
-    g2.K = I;
-    g2.R = w.R;
-    g2.chunks = (I + kChunkK - 1) / kChunkK;
     g2.splits = w.splits;
     g2.cps = (g2.chunks + w.splits - 1) / w.splits;
-    g2.has_t = has_t;
-    g2.tcols = w.tc2;
     prof_record(2, st);
-    if (tc) s = run_tc(g2, false, base + w.hfrag, base + w.hg, base + w.t2, st, "tc gemm w2");
-    else s = run_gemv(g2, false, st, "gemv w2");
-    if (s != MILO_OK) return s;
+    if ((s = run_gemv(g2, false, st, "gemv w2")) != MILO_OK) return s;
     prof_record(3, st);
 
     CombineParams cp{reinterpret_cast<const float*>(base + w.part), inv_perm, topk_w, y, dev_status,

@@ -132,38 +132,23 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
         s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
         s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 2);
         if (!active) continue;
+        // chunk-major layout: the 16-row tile of one K chunk is one contiguous block
+        const size_t crow = static_cast<size_t>(sb >> 1) * p.R + row;
         if (c == 0) {
-            p.gsum[static_cast<size_t>(row) * p.gpad + 2 * sb] = s0;
-            p.gsum[static_cast<size_t>(row) * p.gpad + 2 * sb + 1] = s1;
+            p.gsum[crow * 4 + 2 * (sb & 1)] = s0;
+            p.gsum[crow * 4 + 2 * (sb & 1) + 1] = s1;
         }
-        if (p.layout == 0) {
-            // mma.sync: per super-block, step-major, lane-in-quad c, 4 fp16 each
-            uint2* out = reinterpret_cast<uint2*>(p.frag + (static_cast<size_t>(row) * SB + sb) * kFragHalvesPerSB) + c;
-            out[0 * 4] = frag_step<0>(x);
-            out[1 * 4] = frag_step<1>(x);
-            out[2 * 4] = frag_step<2>(x);
-            out[3 * 4] = frag_step<3>(x);
-            out[4 * 4] = frag_step<4>(x);
-            out[5 * 4] = frag_step<5>(x);
-            out[6 * 4] = frag_step<6>(x);
-            out[7 * 4] = frag_step<7>(x);
-            out[8 * 4] = make_uint2(0u, 0u);      // padding (bank spread)
-        } else {
-            // tcgen05: K slots in the order of the A columns (unit c's first-group
-            // registers at columns 8c..8c+7, its second-group ones at 32+8c..)
-            uint4* o1 = reinterpret_cast<uint4*>(p.frag + static_cast<size_t>(row) * p.K + 128 * sb + 16 * c);
-            uint4* o2 = reinterpret_cast<uint4*>(p.frag + static_cast<size_t>(row) * p.K + 128 * sb + 64 + 16 * c);
-            const uint2 f0 = frag_step<0>(x), f1 = frag_step<1>(x), f2 = frag_step<2>(x), f3 = frag_step<3>(x);
-            const uint2 f4 = frag_step<4>(x), f5 = frag_step<5>(x), f6 = frag_step<6>(x), f7 = frag_step<7>(x);
-            o1[0] = make_uint4(f0.x, f0.y, f1.x, f1.y);
-            o1[1] = make_uint4(f2.x, f2.y, f3.x, f3.y);
-            o2[0] = make_uint4(f4.x, f4.y, f5.x, f5.y);
-            o2[1] = make_uint4(f6.x, f6.y, f7.x, f7.y);
-        }
+        // per super-block: step-major, lane-in-quad c, 4 fp16 each
+        uint2* out = reinterpret_cast<uint2*>(p.frag + crow * kFragRowHalves + (sb & 1) * kFragHalvesPerSB) + c;
+        out[0 * 4] = frag_step<0>(x);
+        out[1 * 4] = frag_step<1>(x);
+        out[2 * 4] = frag_step<2>(x);
+        out[3 * 4] = frag_step<3>(x);
+        out[4 * 4] = frag_step<4>(x);
+        out[5 * 4] = frag_step<5>(x);
+        out[6 * 4] = frag_step<6>(x);
+        out[7 * 4] = frag_step<7>(x);
     }
-    if (blockIdx.y == 0)
-        for (int j = 2 * SB + threadIdx.x; j < p.gpad; j += blockDim.x)
-            p.gsum[static_cast<size_t>(row) * p.gpad + j] = 0.0f;
     flag(p.dev_status, st);
 }
 

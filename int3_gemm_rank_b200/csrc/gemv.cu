@@ -11,10 +11,13 @@
 //     point folded into the kernel.
 //
 // B200 design (not a translation of the page's kernel):
-//   - One producer warp streams each CTA's weight tile with 2-D TMA loads
-//     (packed codes, scales, zeros) plus the prepared activation fragments and
-//     per-group activation sums into a 3-stage shared-memory ring guarded by
-//     mbarriers.  Weights are read from HBM exactly once per token tile.
+//   - One producer thread streams each CTA's weight tile into a 3-stage
+//     shared-memory ring guarded by mbarriers.  The packed weights are stored
+//     in 64-row tiles (milo.h), so a K chunk of a tile (codes, scales, zeros)
+//     is a handful of contiguous blocks, each fetched by one 1-D bulk copy of
+//     the TMA engine; the prepared activations and group sums of the item's
+//     routed rows are contiguous too.  Weights are read from HBM exactly once
+//     per token tile, with an evict-first L2 policy.
 //   - Four consumer warps each own 32 weight rows.  A lane reads its 3-word
 //     unit of two rows and extracts code pairs with one LOP3 each (plus one
 //     shift per word): the masked fp16 pattern already is code * 8^i * 2^-24,
@@ -27,6 +30,8 @@
 //     A = U rows (fp16), B = t = x V^T (fp16, computed beforehand per expert).
 //   - Epilogue: SwiGLU h = silu(a) * b in the w1|w3 kernel (both rows live in
 //     the same lane), or fp32 partial sums per K split for the plain one.
+//   - A K chunk is two super-blocks; when K/128 is odd the last chunk has one,
+//     and only the bytes that exist are copied and computed.
 //   - Work items (expert, row tile, K split, 16-row token tile) are enumerated
 //     on the device from the expert offsets, so the host never synchronises;
 //     CTAs are persistent (three per SM) and walk the items round-robin, the
@@ -41,23 +46,23 @@ namespace milo {
 constexpr int kStages = 3;
 constexpr int kConsumerWarps = 4;
 constexpr int kGemvThreads = 32 * (kConsumerWarps + 1);
-// Stage layout (bytes).  Q tiles are [2 super-blocks][rows][12 words]; the
-// GLU kernel keeps w1's 64 rows at kOffQ and w3's at kOffQB.
+// Stage layout (bytes).  Codes: two 64-row tiles, each [2 super-blocks][64
+// rows][12 words] (GLU: w1's tile, then w3's; plain: rows 0-63, then 64-127).
+// Scales/zeros: [4 groups][64 rows] fp16 blocks, GLU: w1 s, w1 z, w3 s, w3 z;
+// plain: s rows 0-63, s rows 64-127, z rows 0-63, z rows 64-127.
 constexpr int kOffQ = 0;
-constexpr int kOffQB = 6144;
-constexpr int kOffS = 12288;       // scale/zero tiles [4 groups][rows] fp16, 2048 B in all
-constexpr int kOffX = 14336;       // activation fragments [2 sb][16 rows][144 fp16]
-constexpr int kOffG = 23552;       // group sums [16 rows][4 groups] f32
-constexpr int kStageBytes = 23808;
+constexpr int kOffQB = 2 * kQTileSBWords * 4;            // 6144
+constexpr int kOffS = 2 * kOffQB;                         // 12288
+constexpr int kOffX = kOffS + 2048;                       // activations [16 rows][272 fp16]
+constexpr int kOffG = kOffX + kTokTile * kFragRowHalves * 2;   // group sums [16 rows][4] f32
+constexpr int kStageBytes = kOffG + kTokTile * 16;
 constexpr int kOffUA = 0, kOffUB = 8192, kOffT = 16384;   // compensator stage
-constexpr int kXBytesSB = kTokTile * kFragHalvesPerSB * 2;  // 4608
 constexpr int kBarOffset = kStages * kStageBytes;
 constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 3 * (MILO_MAX_EXPERTS + 1) * 4 + 16;
 
-static_assert(kOffQB == 2 * kRowsGlu * 48, "Q tile layout");
-static_assert(kOffS == 2 * kRowsPlain * 48, "Q tile layout");
-static_assert(kOffG + kTokTile * 4 * 4 == kStageBytes, "stage layout");
-static_assert(kOffT + kTokTile * 2 * MILO_MAX_RANK * 2 <= kStageBytes, "compensator stage");
+static_assert(kStageBytes % 16 == 0 && kOffX % 16 == 0 && kOffG % 16 == 0, "bulk-copy alignment");
+static_assert(kOffT >= kRowsPlain * MILO_MAX_RANK * 2, "compensator stage: U rows");
+static_assert(kOffT + kTokTile * 2 * MILO_MAX_RANK * 2 <= kStageBytes, "compensator stage: t rows");
 
 struct Item {
     int e, ntile, split, tt;
@@ -93,8 +98,7 @@ __device__ __forceinline__ void code_step(const uint32_t (&wd)[2][2][3], const u
     uint2 b[NT];
 #pragma unroll
     for (int n8 = 0; n8 < NT; ++n8)
-        b[n8] = *reinterpret_cast<const uint2*>(
-            xs + ((n8 * 8 + g) * kFragHalvesPerSB + S * 16 + c * 4) * 2);
+        b[n8] = *reinterpret_cast<const uint2*>(xs + ((n8 * 8 + g) * kFragRowHalves + S * 16 + c * 4) * 2);
 #pragma unroll
     for (int ti = 0; ti < 2; ++ti) {
         const uint32_t a0 = unit_reg<t0, f0>(wd[ti][0], hw[ti][0]);
@@ -109,12 +113,35 @@ __device__ __forceinline__ void code_step(const uint32_t (&wd)[2][2][3], const u
     }
 }
 
+// Per m16 tile ti of a consumer warp: word offset of its 64-row code tile in
+// the stage, first row inside that tile, byte offset of its scales (zeros
+// follow at zdelta).
+template <bool GLU>
+struct TileMap {
+    int q[2], r[2], s[2];
+    static constexpr int zdelta = GLU ? 512 : 1024;
+    __device__ __forceinline__ explicit TileMap(int warp) {
+#pragma unroll
+        for (int ti = 0; ti < 2; ++ti) {
+            if (GLU) {
+                q[ti] = ti * (kOffQB / 4);
+                r[ti] = 16 * warp;
+                s[ti] = kOffS + ti * 1024;
+            } else {
+                const int half = warp >> 1;
+                q[ti] = half * (kOffQB / 4);
+                r[ti] = 32 * (warp & 1) + 16 * ti;
+                s[ti] = kOffS + half * 512;
+            }
+        }
+    }
+};
+
 // acc += s * 2^24 * D_g - s * z * X_g for the scale group `grp` of the stage.
 template <bool GLU, int NT>
 __device__ __forceinline__ void fold_group(float (&acc)[2][2][4], const float (&dz)[2][2][4],
-                                           const uint8_t* st, int grp, const int (&rbase)[2],
+                                           const uint8_t* st, int grp, const TileMap<GLU>& tm,
                                            int g, int c) {
-    constexpr int RA = GLU ? kRowsGlu : kRowsPlain;
     const float* gs = reinterpret_cast<const float*>(st + kOffG);
     float xg[NT][2];
 #pragma unroll
@@ -124,14 +151,14 @@ __device__ __forceinline__ void fold_group(float (&acc)[2][2][4], const float (&
     }
 #pragma unroll
     for (int ti = 0; ti < 2; ++ti) {
-        const __half* S = reinterpret_cast<const __half*>(st + kOffS + (GLU ? ti * 1024 : 0));
-        const __half* Z = S + (GLU ? 256 : 512);
+        const __half* S = reinterpret_cast<const __half*>(st + tm.s[ti]);
+        const __half* Z = reinterpret_cast<const __half*>(st + tm.s[ti] + TileMap<GLU>::zdelta);
         float s24[2], nsz[2];
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
-            const int row = rbase[ti] + g + 8 * rr;
-            const float sv = __half2float(S[grp * RA + row]);
-            const float zv = __half2float(Z[grp * RA + row]);
+            const int row = tm.r[ti] + g + 8 * rr;
+            const float sv = __half2float(S[grp * kTileRows + row]);
+            const float zv = __half2float(Z[grp * kTileRows + row]);
             s24[rr] = sv * 16777216.0f;
             nsz[rr] = -sv * zv;
         }
@@ -147,15 +174,13 @@ __device__ __forceinline__ void fold_group(float (&acc)[2][2][4], const float (&
 }
 
 template <bool GLU, int NT>
-__device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2][2][4], int warp,
-                                              int lane) {
-    constexpr int RA = GLU ? kRowsGlu : kRowsPlain;
+__device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2][2][4], const TileMap<GLU>& tm,
+                                              int nsb, int lane) {
     const int g = lane >> 2, c = lane & 3;
-    const int rbase[2] = {GLU ? 16 * warp : 32 * warp, GLU ? 16 * warp : 32 * warp + 16};
-    const uint32_t* qt[2] = {reinterpret_cast<const uint32_t*>(st + kOffQ),
-                             reinterpret_cast<const uint32_t*>(st + (GLU ? kOffQB : kOffQ))};
+    const uint32_t* qt = reinterpret_cast<const uint32_t*>(st + kOffQ);
 #pragma unroll
     for (int sbl = 0; sbl < 2; ++sbl) {
+        if (sbl == nsb) break;
         uint32_t wd[2][2][3], hw[2][2][3];
 #pragma unroll
         for (int ti = 0; ti < 2; ++ti)
@@ -163,21 +188,21 @@ __device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2]
             for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
                 for (int t = 0; t < 3; ++t) {
-                    wd[ti][rr][t] = qt[ti][(sbl * RA + rbase[ti] + g + 8 * rr) * 12 + 3 * c + t];
+                    wd[ti][rr][t] = qt[tm.q[ti] + sbl * kQTileSBWords + (tm.r[ti] + g + 8 * rr) * 12 + 3 * c + t];
                     hw[ti][rr][t] = wd[ti][rr][t] >> 9;
                 }
-        const uint8_t* xs = st + kOffX + sbl * kXBytesSB;
+        const uint8_t* xs = st + kOffX + sbl * kFragHalvesPerSB * 2;
         float dz[2][2][4];
         code_step<0, NT>(wd, hw, xs, g, c, dz);
         code_step<1, NT>(wd, hw, xs, g, c, dz);
         code_step<2, NT>(wd, hw, xs, g, c, dz);
         code_step<3, NT>(wd, hw, xs, g, c, dz);
-        fold_group<GLU, NT>(acc, dz, st, 2 * sbl, rbase, g, c);
+        fold_group<GLU, NT>(acc, dz, st, 2 * sbl, tm, g, c);
         code_step<4, NT>(wd, hw, xs, g, c, dz);
         code_step<5, NT>(wd, hw, xs, g, c, dz);
         code_step<6, NT>(wd, hw, xs, g, c, dz);
         code_step<7, NT>(wd, hw, xs, g, c, dz);
-        fold_group<GLU, NT>(acc, dz, st, 2 * sbl + 1, rbase, g, c);
+        fold_group<GLU, NT>(acc, dz, st, 2 * sbl + 1, tm, g, c);
     }
 }
 
@@ -219,7 +244,6 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     int* start = reinterpret_cast<int*>(empty + kStages);
     int* cnt = start + (MILO_MAX_EXPERTS + 1);
     int* row0s = cnt + (MILO_MAX_EXPERTS + 1);
-    volatile int* abort_flag = row0s + (MILO_MAX_EXPERTS + 1);
 
     constexpr int RA = GLU ? kRowsGlu : kRowsPlain;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -230,7 +254,6 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
         }
-        *abort_flag = 0;
         fence_barrier_init();
         int run = 0;
         for (int e = 0; e < p.n_exp; ++e) {
@@ -249,75 +272,80 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------------ producer
         if (lane != 0) return;
+        const uint64_t pol = l2_evict_first();
         int stage = 0;
         uint32_t phase = 0;
-        for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+        uint32_t filled = 0, fph = 0;     // per stage: has a fill, parity of its last fill
+        bool fail = false;
+        for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
             const Item w = decode_item(it, start, cnt, p.n_exp, p.splits);
             const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
             const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
             const int n0 = w.ntile * RA;
+            const int tile0 = n0 / kTileRows;
+            const int ntl = GLU ? 2 : min(2, (p.N - n0 + kTileRows - 1) / kTileRows);
             const int row0 = row0s[w.e] + w.tt * kTokTile;
+            const int ntok = min(kTokTile, cnt[w.e] - w.tt * kTokTile);
             const int c0 = w.split * p.cps;
             const int c1 = min(p.chunks, c0 + p.cps);
-            tmap_acquire(&pa->q_map);
-            tmap_acquire(&pa->s_map);
-            tmap_acquire(&pa->z_map);
-            if (GLU) {
-                tmap_acquire(&pb->q_map);
-                tmap_acquire(&pb->s_map);
-                tmap_acquire(&pb->z_map);
-            }
             for (int ch = c0; ch < c1; ++ch) {
                 if (!mbar_wait(&empty[stage], phase ^ 1)) {
-                    flag(p.dev_status, MILO_DEV_TIMEOUT);
-                    *abort_flag = 1;
-                    return;
+                    fail = true;
+                    break;
                 }
                 uint8_t* st = smem + stage * kStageBytes;
                 uint64_t* fb = &full[stage];
-                mbar_arrive_expect_tx(fb, kStageBytes);
+                filled |= 1u << stage;
+                fph = (fph & ~(1u << stage)) | (phase << stage);
+                const int nsb = min(2, p.SB - 2 * ch);
+                const uint32_t qb = nsb * kQTileSBWords * 4;        // codes of one tile
+                const uint32_t gb = nsb * 2 * kTileRows * 2;         // scales (zeros) of one tile
+                const uint32_t xb = ntok * kFragRowHalves * 2;
+                const uint32_t tb = ntok * 16;
+                mbar_arrive_expect_tx(fb, ntl * (qb + 2 * gb) + xb + tb);
 #pragma unroll
-                for (int sbl = 0; sbl < 2; ++sbl) {
-                    const int sb = 2 * ch + sbl;
-                    tma_load_2d(st + kOffQ + sbl * RA * 48, &pa->q_map, fb, 12 * sb, n0);
-                    if (GLU) tma_load_2d(st + kOffQB + sbl * RA * 48, &pb->q_map, fb, 12 * sb, n0);
-                    tma_load_2d(st + kOffX + sbl * kXBytesSB, &p.x_map, fb, kFragHalvesPerSB * sb, row0);
+                for (int h = 0; h < 2; ++h) {
+                    if (h == ntl) break;
+                    const ProjDev* pj = (GLU && h == 1) ? pb : pa;
+                    const int tile = GLU ? tile0 : tile0 + h;
+                    bulk_load_hint(st + kOffQ + h * kOffQB,
+                                   pj->q + (static_cast<size_t>(tile) * p.SB + 2 * ch) * kQTileSBWords, qb, fb, pol);
+                    const size_t go = (static_cast<size_t>(tile) * p.G + 4 * ch) * kTileRows;
+                    // GLU: [s a | z a | s b | z b]; plain: [s t0 | s t1 | z t0 | z t1]
+                    const int so = GLU ? kOffS + h * 1024 : kOffS + h * 512;
+                    const int zo = GLU ? so + 512 : so + 1024;
+                    bulk_load_hint(st + so, pj->scale + go, gb, fb, pol);
+                    bulk_load_hint(st + zo, pj->zero + go, gb, fb, pol);
                 }
-                if (GLU) {
-                    tma_load_2d(st + kOffS, &pa->s_map, fb, n0, 4 * ch);
-                    tma_load_2d(st + kOffS + 512, &pa->z_map, fb, n0, 4 * ch);
-                    tma_load_2d(st + kOffS + 1024, &pb->s_map, fb, n0, 4 * ch);
-                    tma_load_2d(st + kOffS + 1536, &pb->z_map, fb, n0, 4 * ch);
-                } else {
-                    tma_load_2d(st + kOffS, &pa->s_map, fb, n0, 4 * ch);
-                    tma_load_2d(st + kOffS + 1024, &pa->z_map, fb, n0, 4 * ch);
-                }
-                tma_load_2d(st + kOffG, &p.g_map, fb, 4 * ch, row0);
+                const size_t xr = static_cast<size_t>(ch) * p.R + row0;
+                bulk_load(st + kOffX, p.x + xr * kFragRowHalves, xb, fb);
+                bulk_load(st + kOffG, p.gsum + xr * 4, tb, fb);
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
             }
             const int ra = pa->rank, rb = GLU ? pb->rank : 0;
-            if (w.split == 0 && p.has_t && (ra > 0 || rb > 0)) {
+            if (!fail && w.split == 0 && p.has_t && (ra > 0 || rb > 0)) {
                 if (!mbar_wait(&empty[stage], phase ^ 1)) {
-                    flag(p.dev_status, MILO_DEV_TIMEOUT);
-                    *abort_flag = 1;
-                    return;
+                    fail = true;
+                    break;
                 }
                 uint8_t* st = smem + stage * kStageBytes;
                 uint64_t* fb = &full[stage];
-                const uint32_t bytes = ra * RA * 2 + (GLU ? rb * RA * 2 : 0) + p.tcols * kTokTile * 2;
-                mbar_arrive_expect_tx(fb, bytes);
-                if (ra > 0) {
-                    tmap_acquire(&pa->u_map);
-                    tma_load_2d(st + kOffUA, &pa->u_map, fb, 0, n0);
-                }
-                if (GLU && rb > 0) {
-                    tmap_acquire(&pb->u_map);
-                    tma_load_2d(st + kOffUB, &pb->u_map, fb, 0, n0);
-                }
-                tma_load_2d(st + kOffT, &p.t_map, fb, 0, row0);
+                filled |= 1u << stage;
+                fph = (fph & ~(1u << stage)) | (phase << stage);
+                const int urows = min(RA, p.N - n0);
+                const uint32_t ua = urows * ra * 2, ub = urows * rb * 2;
+                const uint32_t tb = ntok * p.tcols * 2;
+                mbar_arrive_expect_tx(fb, ua + ub + tb);
+                if (ua) bulk_load_hint(st + kOffUA, pa->U + static_cast<size_t>(n0) * ra, ua, fb, pol);
+                if (ub) bulk_load_hint(st + kOffUB, pb->U + static_cast<size_t>(n0) * rb, ub, fb, pol);
+                bulk_load(st + kOffT, p.t + static_cast<size_t>(row0) * p.tcols, tb, fb);
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
             }
         }
+        // No copy may still be landing in shared memory when the CTA leaves.
+        for (int s2 = 0; s2 < kStages; ++s2)
+            if (((filled >> s2) & 1u) && !mbar_wait(&full[s2], (fph >> s2) & 1u)) fail = true;
+        if (fail) flag(p.dev_status, MILO_DEV_TIMEOUT);
         return;
     }
 
@@ -325,6 +353,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     int stage = 0;
     uint32_t phase = 0;
     const int g = lane >> 2, c = lane & 3;
+    const TileMap<GLU> tm(warp);
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
         const Item w = decode_item(it, start, cnt, p.n_exp, p.splits);
         const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
@@ -345,12 +374,12 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         for (int ch = c0; ch < c1; ++ch) {
             if (!mbar_wait(&full[stage], phase)) {
                 flag(p.dev_status, MILO_DEV_TIMEOUT);
-                *abort_flag = 1;
                 return;
             }
             const uint8_t* st = smem + stage * kStageBytes;
-            if (ntok > 8) chunk_compute<GLU, 2>(st, acc, warp, lane);
-            else chunk_compute<GLU, 1>(st, acc, warp, lane);
+            const int nsb = min(2, p.SB - 2 * ch);
+            if (ntok > 8) chunk_compute<GLU, 2>(st, acc, tm, nsb, lane);
+            else chunk_compute<GLU, 1>(st, acc, tm, nsb, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
             if (++stage == kStages) { stage = 0; phase ^= 1; }
@@ -359,7 +388,6 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         if (w.split == 0 && p.has_t && (ra > 0 || rb > 0)) {
             if (!mbar_wait(&full[stage], phase)) {
                 flag(p.dev_status, MILO_DEV_TIMEOUT);
-                *abort_flag = 1;
                 return;
             }
             const uint8_t* st = smem + stage * kStageBytes;
@@ -381,7 +409,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                     const int tok = n8 * 8 + 2 * c + (i & 1);
                     if (tok < ntok && f < p.N) {
                         const float a = acc[0][n8][i], b = acc[1][n8][i];
-                        const float hv = a / (1.0f + expf(-a)) * b;
+                        const float hv = __fdividef(a, 1.0f + __expf(-a)) * b;
                         const __half hh = __float2half_rn(hv);
                         if (!isfinite(hv)) st |= MILO_DEV_NONFINITE;
                         else if (__hisinf(hh)) st |= MILO_DEV_FP16_RANGE;

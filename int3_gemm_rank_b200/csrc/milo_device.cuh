@@ -101,10 +101,6 @@ __host__ __device__ constexpr int field_shift(int f) {
 __host__ __device__ constexpr float act_scale(int f) {
     return f == 0 || f == 3 ? 1.0f : f == 1 || f == 4 ? 0.125f : 0.015625f;
 }
-// Prepared activations: per row and super-block, 8 steps x 4 lanes-in-quad
-// (c) x 4 fp16, then 16 fp16 of padding so that rows of a 16-row tile fall on
-// different shared-memory banks: 144 fp16 (288 bytes).
-constexpr int kFragHalvesPerSB = 144;
 
 // ---------------------------------------------------------------------------
 // PTX: mbarrier
@@ -153,22 +149,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------------------
-// PTX: TMA (no multicast anywhere in this library)
+// PTX: bulk copies (TMA engine, 1-D; no multicast anywhere in this library)
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ void tmap_acquire(const CUtensorMap* map) {
-    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;"
-                 ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+// L2 policy for data read once per launch (packed weights): evict first, so
+// that activations and partial sums stay resident.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
 }
 
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t x, int32_t y) {
+// Copy `bytes` contiguous bytes global -> this CTA's shared memory; the
+// mbarrier's transaction count receives them.  Both addresses 16-byte
+// aligned, `bytes` a positive multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
-          "r"(x), "r"(y)
-        : "memory");
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                               uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy) : "memory");
 }
 
 // ---------------------------------------------------------------------------

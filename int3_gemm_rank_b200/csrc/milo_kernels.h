@@ -16,32 +16,40 @@ constexpr int kRowsGlu = 64;       // output features per CTA, w1|w3 + SwiGLU (1
 constexpr int kTokTile = 16;       // routed rows per work item (two n8 MMA tiles)
 constexpr int kChunkK = 256;       // K per pipeline stage (two 128-code super-blocks)
 
-// One projection in the device table.  The tensor maps are encoded on the
-// host at prepare time; the kernels read them from global memory.
-struct alignas(64) ProjDev {
-    CUtensorMap q_map;   // Q u32 [N, 3K/32], box {12 words, tile rows}
-    CUtensorMap s_map;   // scale fp16 [K/64, N], box {tile rows, 4 groups}
-    CUtensorMap z_map;   // zero  fp16 [K/64, N], box {tile rows, 4 groups}
-    CUtensorMap u_map;   // U fp16 [N, r], box {r, tile rows}; unused when rank == 0
-    const uint32_t* q;
-    const uint16_t* scale;
-    const uint16_t* zero;
-    const uint16_t* U;
-    const uint16_t* V;
-    int32_t rank, N, K, tile_rows;
+// Prepared activations: per row and K chunk (two super-blocks), for each
+// super-block 8 MMA steps x 4 lanes-in-quad x 4 fp16, then 16 fp16 of padding
+// so that the rows of a 16-row tile fall on different shared-memory banks
+// (row pitch 136 words, 8 mod 32): 272 fp16 (544 bytes).
+constexpr int kFragHalvesPerSB = 128;
+constexpr int kFragRowHalves = 2 * kFragHalvesPerSB + 16;
+
+// Rows of the packed weights are grouped in tiles of 64 (milo.h): a tile's
+// words for one super-block, and its scales (zeros) for one group, are
+// contiguous, so a K chunk of a tile arrives with one bulk copy per tensor.
+constexpr int kTileRows = 64;
+constexpr int kQTileSBWords = kTileRows * 12;       // one tile, one super-block: 3072 bytes
+
+// One projection in the device table (device pointers and shape).
+struct alignas(16) ProjDev {
+    const uint32_t* q;          // [ceil(N/64)][K/128][64][12] words
+    const uint16_t* scale;      // [ceil(N/64)][K/64][64] fp16
+    const uint16_t* zero;       // [ceil(N/64)][K/64][64] fp16
+    const uint16_t* U;          // [N][rank] fp16, NULL when rank == 0
+    const uint16_t* V;          // [rank][K] fp16, NULL when rank == 0
+    int32_t rank, N, K, pad;
 };
 
 struct GemvParams {
-    CUtensorMap x_map;          // prepared activations [R, SB*144] fp16, box {144, 16}
-    CUtensorMap g_map;          // group sums [R, Gpad] f32, box {4, 16}
-    CUtensorMap t_map;          // LoRC down-projection [R, tcols] fp16, box {tcols, 16}
+    const uint16_t* x;          // prepared activations [chunks][R][kFragRowHalves] fp16
+    const float* gsum;          // group sums [chunks][R][4] f32
+    const uint16_t* t;          // LoRC down-projection [R][tcols] fp16
     const ProjDev* table;       // device table
     const int32_t* grp;         // [n_exp][2]: first row, row count of each group (expert)
     float* y_part;              // plain: [splits][R][N] f32 partial sums
     uint16_t* h;                // SwiGLU: [R][N] fp16
     int32_t* dev_status;
     int stride, proj_a, proj_b; // table entries per expert; entry of A (w1 / the projection), B (w3)
-    int n_exp, N, K, R;
+    int n_exp, N, K, R, SB, G;  // G = K / 64 groups
     int splits, chunks, cps;    // split-K count, K chunks, chunks per split
     int has_t, tcols, t_col_b;  // LoRC activations present; row width; first column of w3's
 };
@@ -50,11 +58,10 @@ struct PrepParams {
     const uint16_t* src;        // [*, K] bf16/fp16 (or fp16 h)
     int32_t* row_src;           // row p -> source row; built here when `rows` is set, else
                                 // read (NULL: identity); -1 = zero row
-    uint16_t* frag;             // [R, SB*144] fp16
-    float* gsum;                // [R, Gpad] f32
+    uint16_t* frag;             // [chunks][R][kFragRowHalves] fp16, chunks = ceil(K/256)
+    float* gsum;                // [chunks][R][4] f32
     int32_t* dev_status;
-    int R, K, gpad, src_bf16;
-    int layout;                 // 0: mma.sync fragments [R][K/128][144]; 1: tcgen05 A-column order [R][K]
+    int R, K, src_bf16;
     // Row bookkeeping (first preparation of a call only): routed rows come from
     // the router's offsets/perm, the n_shared*T shared-expert rows follow them.
     int rows;                   // 1: build grp / row_src / inv from offsets and perm
@@ -88,24 +95,6 @@ struct CombineParams {
     int per_slot;               // 1: y row per flat slot (grouped linear), 0: per token
 };
 
-// Parameters of the tcgen05 grouped GEMM (gemm_tc.cu).
-struct TcParams {
-    CUtensorMap b_map;          // activations in A-column order [R, K] fp16, box {64, 16}, 128B swizzle
-    CUtensorMap g_map;          // group sums [R, Gpad] f32, box {4, 16}
-    CUtensorMap t_map;          // compensator activations [R, tcols] fp16, box {64, 16}, 128B swizzle
-    const ProjDev* table;
-    const int32_t* grp;
-    float* y_part;
-    uint16_t* h;
-    int32_t* dev_status;
-    int stride, proj_a, proj_b;
-    int n_exp, N, K, R;
-    int splits, chunks, cps;
-    int has_t, tcols, t_col_b;
-};
-
-size_t tc_smem_bytes();
-cudaError_t launch_tc_gemm(const TcParams& p, bool glu, int grid, cudaStream_t s);
 size_t gemv_smem_bytes(bool glu);
 cudaError_t launch_gemv(const GemvParams& p, bool glu, int grid, cudaStream_t s);
 cudaError_t launch_prep(const PrepParams& p, cudaStream_t s);

@@ -59,6 +59,8 @@ def lib():
         L.milo_ref_pack.argtypes = [vp, i, i, vp]; L.milo_ref_pack.restype = None
         L.milo_ref_unpack.argtypes = [vp, i, i, vp]; L.milo_ref_unpack.restype = None
         L.milo_ref_code_bit.argtypes = [i, i, C.POINTER(i), C.POINTER(i)]
+        L.milo_ref_tile_words.argtypes = [vp, i, i, vp]; L.milo_ref_tile_words.restype = None
+        L.milo_ref_tile_groups.argtypes = [vp, i, i, vp]; L.milo_ref_tile_groups.restype = None
         L.milo_ref_dequant.argtypes = [vp, vp, vp, i, i, i, vp]; L.milo_ref_dequant.restype = None
         L.milo_ref_group.argtypes = [vp, i, i, i, vp, vp, vp]; L.milo_ref_group.restype = i
         L.milo_ref_route.argtypes = [vp, i, i, i, i, vp, vp, vp, vp, vp]; L.milo_ref_route.restype = i
@@ -118,6 +120,25 @@ def unpack(Q: np.ndarray, K: int) -> np.ndarray:
     q = np.zeros((N, K), np.uint8)
     lib().milo_ref_unpack(_p(Q), N, K, _p(q))
     return q
+
+
+def tile_words(Q: np.ndarray, K: int) -> np.ndarray:
+    """Row-major packed words [N, 3K/32] -> the device layout [ceil(N/64), K/128, 64, 12]."""
+    Q = _c(Q, np.uint32)
+    N = Q.shape[0]
+    NT = (N + 63) // 64
+    Qt = np.zeros((NT, K // 128, 64, 12), np.uint32)
+    lib().milo_ref_tile_words(_p(Q), N, K, _p(Qt))
+    return Qt
+
+
+def tile_groups(A: np.ndarray) -> np.ndarray:
+    """Group-major [G, N] (scale or zero) -> the device layout [ceil(N/64), G, 64]."""
+    A = _c(A, np.uint16)
+    G, N = A.shape
+    At = np.zeros(((N + 63) // 64, G, 64), np.uint16)
+    lib().milo_ref_tile_groups(_p(A), N, G, _p(At))
+    return At
 
 
 def code_bit(k: int, beta: int):

@@ -214,6 +214,33 @@ void milo_ref_unpack(const uint32_t* Q, int N, int K, uint8_t* q) {
         }
 }
 
+/*
+ * Device layout of the packed tensors.  The GPU kernels fetch the words of 64
+ * rows for one or two super-blocks as one contiguous block, so the device
+ * buffers group rows in tiles of 64 (the last tile padded with zero rows):
+ *     Qt[((n / 64) * SB + b) * 768 + (n % 64) * 12 + j] = Q[n, 12 b + j]
+ *     At[((n / 64) * G + g) * 64 + (n % 64)]           = A[g, n]
+ * (SB = K / 128 super-blocks, G = K / 64 groups; A is a scale or zero array
+ * [G, N]).  These are relayouts only, used to compare with the device packer.
+ */
+void milo_ref_tile_words(const uint32_t* Q, int N, int K, uint32_t* Qt) {
+    int SB = K / 128, W = 3 * K / 32, NT = (N + 63) / 64;
+    memset(Qt, 0, sizeof(uint32_t) * (size_t)NT * 64 * W);
+    for (int n = 0; n < N; ++n)
+        for (int b = 0; b < SB; ++b)
+            for (int j = 0; j < 12; ++j)
+                Qt[((size_t)(n / 64) * SB + b) * 768 + (size_t)(n % 64) * 12 + j] =
+                    Q[(size_t)n * W + 12 * b + j];
+}
+
+void milo_ref_tile_groups(const uint16_t* A, int N, int G, uint16_t* At) {
+    int NT = (N + 63) / 64;
+    memset(At, 0, sizeof(uint16_t) * (size_t)NT * 64 * G);
+    for (int g = 0; g < G; ++g)
+        for (int n = 0; n < N; ++n)
+            At[((size_t)(n / 64) * G + g) * 64 + (n % 64)] = A[(size_t)g * N + n];
+}
+
 /* w_hat[n, k] = (q - z) * s in fp64. */
 void milo_ref_dequant(const uint8_t* q, const uint16_t* scale, const uint16_t* zero,
                       int N, int K, int group, double* w_hat) {

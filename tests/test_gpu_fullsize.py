@@ -35,10 +35,6 @@ def milo():
     return m
 
 
-@pytest.fixture(params=["tc", "mma"])
-def gemm_path(request, monkeypatch):
-    monkeypatch.setenv("MILO_GEMM", request.param)
-    return request.param
 
 
 def _gpu_proj(milo, P):
@@ -73,7 +69,7 @@ def _route(milo, wk):
     return r, ids, w, inv
 
 
-def test_single_expert_decode_full(milo, gemm_path):
+def test_single_expert_decode_full(milo):
     x, P = wl.single()
     lin = milo.GroupedLinear([_gpu_proj(milo, P)])
     r = milo.milo_route(None, 1, False, E=1, ids=to_dev(np.zeros((1, 1), np.int32)))
@@ -105,11 +101,11 @@ def _layer_full(milo, wk):
     assert herr <= REL_TOL, herr
 
 
-def test_mixtral_decode_layer_full(milo, gemm_path):
+def test_mixtral_decode_layer_full(milo):
     _layer_full(milo, wl.mixtral())
 
 
-def test_deepseek_decode_layer_full(milo, gemm_path):
+def test_deepseek_decode_layer_full(milo):
     _layer_full(milo, wl.deepseek())
 
 

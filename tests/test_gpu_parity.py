@@ -28,11 +28,6 @@ def milo():
     return m
 
 
-@pytest.fixture(params=["tc", "mma"])
-def gemm_path(request, monkeypatch):
-    """Run a test with the tcgen05 grouped GEMM (default) and with the mma.sync one."""
-    monkeypatch.setenv("MILO_GEMM", request.param)
-    return request.param
 
 
 def _status(st):
@@ -44,16 +39,16 @@ def _status(st):
 # packing and extraction
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("N,K", [(1, 128), (48, 384), (208, 1024), (1024, 1024), (16, 14336)])
+@pytest.mark.parametrize("N,K", [(1, 128), (48, 384), (208, 1024), (1024, 1024), (16, 14336), (130, 1408)])
 def test_pack_bit_exact(milo, N, K):
     W = wl.gen_weight(np.random.default_rng(N * 7 + K), N, K)
     st = milo.new_status()
     Q, s, z = milo.milo_pack(f16_dev(W), dev_status=st)
     q_ref, s_ref, z_ref, st_ref = oracle.quantize(W)
     assert _status(st) == st_ref == 0
-    assert np.array_equal(Q.cpu().numpy().view(np.uint32), oracle.pack(q_ref))
-    assert np.array_equal(s.cpu().numpy().view(np.uint16), s_ref)
-    assert np.array_equal(z.cpu().numpy().view(np.uint16), z_ref)
+    assert np.array_equal(Q.cpu().numpy().view(np.uint32), oracle.tile_words(oracle.pack(q_ref), K))
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), oracle.tile_groups(s_ref))
+    assert np.array_equal(z.cpu().numpy().view(np.uint16), oracle.tile_groups(z_ref))
 
 
 def test_pack_degenerate_and_signed_zero_groups(milo):
@@ -65,9 +60,9 @@ def test_pack_degenerate_and_signed_zero_groups(milo):
     Wb = W.astype(np.float16).view(np.uint16)
     Q, s, z = milo.milo_pack(f16_dev(Wb))
     q_ref, s_ref, z_ref, _ = oracle.quantize(Wb)
-    assert np.array_equal(Q.cpu().numpy().view(np.uint32), oracle.pack(q_ref))
-    assert np.array_equal(s.cpu().numpy().view(np.uint16), s_ref)
-    assert np.array_equal(z.cpu().numpy().view(np.uint16), z_ref)
+    assert np.array_equal(Q.cpu().numpy().view(np.uint32), oracle.tile_words(oracle.pack(q_ref), 128))
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), oracle.tile_groups(s_ref))
+    assert np.array_equal(z.cpu().numpy().view(np.uint16), oracle.tile_groups(z_ref))
 
 
 def test_pack_flags_nonfinite(milo):
@@ -81,8 +76,8 @@ def test_pack_flags_nonfinite(milo):
 @pytest.mark.parametrize("N,K", [(3, 128), (64, 1408), (5, 4096)])
 def test_unpack_bit_exact(milo, N, K):
     q = np.random.default_rng(N + K).integers(0, 8, (N, K), dtype=np.uint8)
-    Q = oracle.pack(q)
-    codes = milo.milo_unpack(to_dev(Q.view(np.int32)), K)
+    Q = oracle.tile_words(oracle.pack(q), K)
+    codes = milo.milo_unpack(to_dev(Q.view(np.int32)), N, K)
     assert np.array_equal(codes.cpu().numpy(), q)
 
 
@@ -172,14 +167,14 @@ def _linear_check(milo, projs, x_bits, x_dt, ids, k, out_dtypes=(torch.float32,)
     return err
 
 
-def test_linear_single_expert_decode_rank16(milo, gemm_path):
+def test_linear_single_expert_decode_rank16(milo):
     """1 token, W 1024x1024 with outliers, rank-16 compensator."""
     x, P = wl.single(seed_workload="t_single")
     _linear_check(milo, [P], x, "f16", np.zeros((1, 1), np.int32), 1,
                   (torch.float32, torch.float16, torch.bfloat16))
 
 
-def test_linear_ragged_rows_multi_token_tiles(milo, gemm_path):
+def test_linear_ragged_rows_multi_token_tiles(milo):
     """N = 208 (ragged last row tile), K = 384 (half-empty last K chunk),
     experts of rank 0 / 8 / 24, 53 tokens over 3 experts (one expert > 16 rows)."""
     projs = [wl.make_projection("t_rag", "w", e, 208, 384, r) for e, r in enumerate((0, 8, 24))]
@@ -188,20 +183,20 @@ def test_linear_ragged_rows_multi_token_tiles(milo, gemm_path):
     _linear_check(milo, projs, x, "bf16", ids, 1, (torch.float32, torch.float16))
 
 
-def test_linear_top2_slots_and_idle_experts(milo, gemm_path):
+def test_linear_top2_slots_and_idle_experts(milo):
     projs = [wl.make_projection("t_k2", "w", e, 256, 512, 16 * (e % 3)) for e in range(6)]
     x = wl.gen_activations(np.random.default_rng(10), 3, 512, "f16")
     ids = np.array([[4, 1], [1, 0], [4, 5]], np.int32)   # experts 2, 3 idle
     _linear_check(milo, projs, x, "f16", ids, 2)
 
 
-def test_linear_all_rows_one_expert(milo, gemm_path):
+def test_linear_all_rows_one_expert(milo):
     projs = [wl.make_projection("t_one", "w", e, 128, 256, 8) for e in range(4)]
     x = wl.gen_activations(np.random.default_rng(11), 70, 256, "bf16")
     _linear_check(milo, projs, x, "bf16", np.full((70, 1), 2, np.int32), 1)
 
 
-def test_linear_bad_ids_dropped_and_zero(milo, gemm_path):
+def test_linear_bad_ids_dropped_and_zero(milo):
     projs = [wl.make_projection("t_bad", "w", e, 128, 256, 0) for e in range(2)]
     lin, ref = _linear_pair(milo, projs)
     x_bits = wl.gen_activations(np.random.default_rng(12), 3, 256, "f16")
@@ -283,18 +278,18 @@ def run_layer_parity(milo, wk, check_h=True, out_dtypes=(torch.float32,)):
     return err
 
 
-def test_moe_small_shared_expert(milo, gemm_path):
+def test_moe_small_shared_expert(milo):
     wk = wl.small_moe("t_moe1", T=5, hidden=256, inter=384, n_routed=4, n_shared=1, top_k=2)
     run_layer_parity(milo, wk, out_dtypes=(torch.float32, torch.bfloat16, torch.float16))
 
 
-def test_moe_small_no_compensator_full_softmax(milo, gemm_path):
+def test_moe_small_no_compensator_full_softmax(milo):
     wk = wl.small_moe("t_moe2", T=19, hidden=384, inter=256, n_routed=6, n_shared=0, top_k=3,
                       renorm=False, rank_choices=(0,), x_dtype="f16")
     run_layer_parity(milo, wk)
 
 
-def test_moe_small_many_tokens_per_expert(milo, gemm_path):
+def test_moe_small_many_tokens_per_expert(milo):
     wk = wl.small_moe("t_moe3", T=90, hidden=256, inter=512, n_routed=3, n_shared=2, top_k=1,
                       rank_choices=(8, 64))
     run_layer_parity(milo, wk)

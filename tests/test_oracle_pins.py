@@ -130,6 +130,26 @@ def test_unpack_roundtrip_exhaustive_one_hot_and_random():
     assert np.array_equal(oracle.unpack(oracle.pack(q), q.shape[1]), q)
 
 
+def test_device_tiling_matches_reshape():
+    """The device layout of the packed words and of the group arrays: 64-row
+    tiles, super-block (group) major inside a tile, zero rows padding the last
+    tile.  Checked against a numpy reshape/transpose of the padded arrays for
+    N that is and is not a multiple of 64."""
+    rng = np.random.default_rng(11)
+    for N, K in ((64, 128), (100, 384), (16, 256), (130, 128)):
+        Q = rng.integers(0, 2 ** 32, (N, 3 * K // 32), dtype=np.uint64).astype(np.uint32)
+        NT = (N + 63) // 64
+        pad = np.zeros((NT * 64, 3 * K // 32), np.uint32)
+        pad[:N] = Q
+        want = pad.reshape(NT, 64, K // 128, 12).transpose(0, 2, 1, 3)
+        assert np.array_equal(oracle.tile_words(Q, K), want)
+        A = rng.integers(0, 2 ** 16, (K // 64, N), dtype=np.uint32).astype(np.uint16)
+        padA = np.zeros((K // 64, NT * 64), np.uint16)
+        padA[:, :N] = A
+        wantA = padA.reshape(K // 64, NT, 64).transpose(1, 0, 2)
+        assert np.array_equal(oracle.tile_groups(A), wantA)
+
+
 def test_unit_codes_share_one_group_per_pair():
     """Each 16-bit half-pair (bits [3i,3i+3) and [16+3i,..)) of a word carries two
     codes of the same scale group; the spare bits of a unit belong to one group."""
