@@ -93,18 +93,20 @@ MILO_API int32_t milo_version(void);
  *     bits [3i, 3i+3) = u_{10t+2i},   bits [16+3i, 16+3i+3) = u_{10t+2i+1},
  * bit 15 = bit t of u_30, bit 31 = bit t of u_31.
  *
- * Device layout: rows are grouped in tiles of 64 (the last tile padded with
- * zero rows, Npad = 64 * ceil(N/64)), so that the kernels fetch the words of
- * a tile for one K chunk, and its scales and zeros, as contiguous blocks:
- *     Q     u32  [Npad/64][K/128][64][12]:  Q[n/64][b][n%64][j] = word 12b+j of row n
- *     scale fp16 [Npad/64][K/64][64]:       scale[n/64][g][n%64] = s of row n, group g
- *     zero  fp16 [Npad/64][K/64][64]        (same layout)
- * Dequantisation: w_hat[n, k] = (q[n, k] - z[n, k/64]) * s[n, k/64].
- * milo_packed_bytes gives the buffer sizes.
+ * Device layout: one blob per weight.  Rows are grouped in tiles of 64 (the
+ * last tile padded with zero rows), K in chunks of two super-blocks (the last
+ * chunk holds one when K/128 is odd).  The (tile t, chunk c) block starts at
+ * byte (t * K/128 + 2c) * 3584 and holds, for its nsb super-blocks b,
+ *     the words u32 [64 rows][12]      (word j of row 64t+r = word 12b+j above)
+ * then, for its 2*nsb groups g,
+ *     s fp16 [64 rows], z fp16 [64 rows]
+ * so that the kernels fetch a tile's chunk -- codes, scales and zeros -- with
+ * one copy.  Dequantisation: w_hat[n, k] = (q[n, k] - z[n, k/64]) * s[n, k/64].
+ * The blob has ceil(N/64) * (K/128) * 3584 bytes (milo_packed_bytes).
  */
 
-/* Bytes of Q and of each of scale, zero for a weight [N, K] (K % 128 == 0). */
-MILO_API milo_status milo_packed_bytes(int32_t N, int32_t K, size_t* q_bytes, size_t* group_bytes);
+/* Bytes of the packed blob of a weight [N, K] (K % 128 == 0). */
+MILO_API milo_status milo_packed_bytes(int32_t N, int32_t K, size_t* bytes);
 
 /*
  * milo_pack -- quantise W fp16 [N, K] (row-major) to int3 and pack it.
@@ -113,22 +115,21 @@ MILO_API milo_status milo_packed_bytes(int32_t N, int32_t K, size_t* q_bytes, si
  *     s = fp16((max - min) / 7)   (s := 1 when it rounds to 0)
  *     z = fp16(-min / s)
  *     q = clamp(rint(w / s + z), 0, 7)    (fp32, ties to even, no FMA)
- * Writes Q, scale and zero in the device layout above, padding rows included
- * (sizes from milo_packed_bytes; Q 16-byte aligned).
+ * Writes the blob in the device layout above, padding rows included (size
+ * from milo_packed_bytes; 16-byte aligned).
  * Errors: group != 64 or K % 128 != 0 -> UNSUPPORTED_SHAPE; N, K <= 0 or NULL
  * pointers -> INVALID_ARG.  Device: NONFINITE for NaN/Inf weights, FP16_RANGE
  * when s or z overflows fp16.  dev_status may be NULL.
  */
-MILO_API milo_status milo_pack(const uint16_t* W, int32_t N, int32_t K, int32_t group,
-                      uint32_t* Q, uint16_t* scale, uint16_t* zero,
+MILO_API milo_status milo_pack(const uint16_t* W, int32_t N, int32_t K, int32_t group, void* packed,
                       int32_t* dev_status, void* stream);
 
 /*
- * milo_unpack -- extract the codes of Q (device layout above) into codes
- * u8 [N, K] row-major, with the same register-level field extraction the GEMM
- * kernels use.
+ * milo_unpack -- extract the codes of a packed blob (device layout above)
+ * into codes u8 [N, K] row-major, with the same register-level field
+ * extraction the GEMM kernels use.
  */
-MILO_API milo_status milo_unpack(const uint32_t* Q, int32_t N, int32_t K, uint8_t* codes,
+MILO_API milo_status milo_unpack(const void* packed, int32_t N, int32_t K, uint8_t* codes,
                         void* stream);
 
 /* ------------------------------------------------------------------------ */
@@ -164,9 +165,7 @@ MILO_API milo_status milo_route(const uint16_t* logits, int32_t T, int32_t E, in
  * holding device pointers).  U fp16 [N, r] and V fp16 [r, K] row-major; both
  * may be NULL when rank == 0.  rank is a multiple of 8, at most MILO_MAX_RANK. */
 typedef struct milo_qweight {
-    const uint32_t* q;
-    const uint16_t* scale;
-    const uint16_t* zero;
+    const void* packed;     /* blob written by milo_pack */
     const uint16_t* U;
     const uint16_t* V;
     int32_t rank;

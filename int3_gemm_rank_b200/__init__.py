@@ -41,8 +41,7 @@ class MiloError(RuntimeError):
 
 
 class milo_qweight(C.Structure):
-    _fields_ = [("q", C.c_void_p), ("scale", C.c_void_p), ("zero", C.c_void_p),
-                ("U", C.c_void_p), ("V", C.c_void_p), ("rank", C.c_int32)]
+    _fields_ = [("packed", C.c_void_p), ("U", C.c_void_p), ("V", C.c_void_p), ("rank", C.c_int32)]
 
 
 class milo_expert(C.Structure):
@@ -75,9 +74,9 @@ def lib() -> C.CDLL:
         L.milo_status_str.argtypes = [C.c_int]; L.milo_status_str.restype = C.c_char_p
         L.milo_last_error.argtypes = []; L.milo_last_error.restype = C.c_char_p
         L.milo_version.argtypes = []; L.milo_version.restype = i32
-        L.milo_pack.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp]; L.milo_pack.restype = C.c_int
+        L.milo_pack.argtypes = [vp, i32, i32, i32, vp, vp, vp]; L.milo_pack.restype = C.c_int
         L.milo_unpack.argtypes = [vp, i32, i32, vp, vp]; L.milo_unpack.restype = C.c_int
-        L.milo_packed_bytes.argtypes = [i32, i32, C.POINTER(sz), C.POINTER(sz)]
+        L.milo_packed_bytes.argtypes = [i32, i32, C.POINTER(sz)]
         L.milo_packed_bytes.restype = C.c_int
         L.milo_route.argtypes = [vp, i32, i32, i32, u32, vp, vp, vp, vp, vp, vp, vp]
         L.milo_route.restype = C.c_int
@@ -148,34 +147,28 @@ def new_status(device=None) -> torch.Tensor:
 # packing
 # ---------------------------------------------------------------------------
 
-def milo_pack(W: torch.Tensor, group: int = MILO_GROUP, dev_status: torch.Tensor | None = None):
-    """Quantise W fp16 [N, K] to int3 and pack it in the device layout of milo.h.
+def milo_packed_bytes(N: int, K: int) -> int:
+    """Bytes of the packed blob of a weight [N, K]."""
+    nb = C.c_size_t()
+    _check(lib().milo_packed_bytes(N, K, C.byref(nb)), "milo_packed_bytes")
+    return nb.value
 
-    Returns (Q int32 [Npad/64, K/128, 64, 12], scale, zero fp16 [Npad/64, K/64, 64]),
-    Npad = 64 * ceil(N / 64)."""
+
+def milo_pack(W: torch.Tensor, group: int = MILO_GROUP, dev_status: torch.Tensor | None = None):
+    """Quantise W fp16 [N, K] to int3 and pack it: the device blob (uint8 tensor) of milo.h."""
     _cuda(W, "W")
     N, K = W.shape
-    NT = (N + 63) // 64
-    Q = torch.empty((NT, K // 128, 64, 12), dtype=torch.int32, device=W.device)
-    s = torch.empty((NT, K // group, 64), dtype=torch.float16, device=W.device)
-    z = torch.empty((NT, K // group, 64), dtype=torch.float16, device=W.device)
-    _check(lib().milo_pack(_ptr(W), N, K, group, _ptr(Q), _ptr(s), _ptr(z), _ptr(dev_status),
-                           _stream()), "milo_pack")
-    return Q, s, z
+    nbytes = milo_packed_bytes(N, K) if K > 0 and K % 128 == 0 and N > 0 else 16
+    blob = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    _check(lib().milo_pack(_ptr(W), N, K, group, _ptr(blob), _ptr(dev_status), _stream()), "milo_pack")
+    return blob
 
 
-def milo_packed_bytes(N: int, K: int) -> tuple:
-    """(bytes of Q, bytes of each of scale and zero) for a weight [N, K]."""
-    qb, gb = C.c_size_t(), C.c_size_t()
-    _check(lib().milo_packed_bytes(N, K, C.byref(qb), C.byref(gb)), "milo_packed_bytes")
-    return qb.value, gb.value
-
-
-def milo_unpack(Q: torch.Tensor, N: int, K: int) -> torch.Tensor:
-    """Codes u8 [N, K] of packed words Q (device layout)."""
-    _cuda(Q, "Q")
-    codes = torch.empty((N, K), dtype=torch.uint8, device=Q.device)
-    _check(lib().milo_unpack(_ptr(Q), N, K, _ptr(codes), _stream()), "milo_unpack")
+def milo_unpack(packed: torch.Tensor, N: int, K: int) -> torch.Tensor:
+    """Codes u8 [N, K] of a packed blob."""
+    _cuda(packed, "packed")
+    codes = torch.empty((N, K), dtype=torch.uint8, device=packed.device)
+    _check(lib().milo_unpack(_ptr(packed), N, K, _ptr(codes), _stream()), "milo_unpack")
     return codes
 
 
@@ -212,11 +205,11 @@ def milo_route(logits: torch.Tensor | None, k: int, renorm: bool, E: int | None 
 # ---------------------------------------------------------------------------
 
 class QWeight:
-    """A packed projection W [N, K] on the device: Q, scale, zero (device layout of
-    milo.h) and the compensator U [N, r], V [r, K]."""
+    """A packed projection W [N, K] on the device: the blob of milo.h (codes,
+    scales, zeros) and the compensator U [N, r], V [r, K]."""
 
-    def __init__(self, Q, scale, zero, N: int, K: int, U=None, V=None):
-        self.Q, self.scale, self.zero = Q, scale, zero
+    def __init__(self, packed, N: int, K: int, U=None, V=None):
+        self.packed = packed
         self.N, self.K = int(N), int(K)
         self.rank = 0 if U is None or U.numel() == 0 else int(U.shape[1])
         self.U = U if self.rank else None
@@ -224,12 +217,10 @@ class QWeight:
 
     @classmethod
     def quantize(cls, W: torch.Tensor, U=None, V=None, dev_status=None):
-        Q, s, z = milo_pack(W, dev_status=dev_status)
-        return cls(Q, s, z, W.shape[0], W.shape[1], U, V)
+        return cls(milo_pack(W, dev_status=dev_status), W.shape[0], W.shape[1], U, V)
 
     def cstruct(self) -> milo_qweight:
-        return milo_qweight(self.Q.data_ptr(), self.scale.data_ptr(), self.zero.data_ptr(),
-                            self.U.data_ptr() if self.rank else None,
+        return milo_qweight(self.packed.data_ptr(), self.U.data_ptr() if self.rank else None,
                             self.V.data_ptr() if self.rank else None, self.rank)
 
 

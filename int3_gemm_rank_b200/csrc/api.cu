@@ -46,19 +46,15 @@ static int sm_count() {
 // ---------------------------------------------------------------------------
 static milo_status fill_proj(ProjDev* d, const milo_qweight& w, int N, int K, const char* what) {
     memset(d, 0, sizeof(*d));
-    if (!w.q || !w.scale || !w.zero)
-        return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": NULL weight pointer");
+    if (!w.packed) return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": NULL packed weight");
     if (w.rank < 0 || w.rank % 8 || w.rank > MILO_MAX_RANK)
         return fail(MILO_ERR_UNSUPPORTED_SHAPE,
                     std::string(what) + ": rank must be a multiple of 8 in [0, 64]");
     if (w.rank > 0 && (!w.U || !w.V))
         return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": U and V are required when rank > 0");
-    if (!aligned(w.q, 16) || !aligned(w.scale, 16) || !aligned(w.zero, 16) ||
-        (w.rank > 0 && (!aligned(w.U, 16) || !aligned(w.V, 16))))
+    if (!aligned(w.packed, 16) || (w.rank > 0 && (!aligned(w.U, 16) || !aligned(w.V, 16))))
         return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": pointers must be 16-byte aligned");
-    d->q = w.q;
-    d->scale = w.scale;
-    d->zero = w.zero;
+    d->packed = static_cast<const uint8_t*>(w.packed);
     d->U = w.rank > 0 ? w.U : nullptr;
     d->V = w.rank > 0 ? w.V : nullptr;
     d->rank = w.rank;
@@ -99,14 +95,13 @@ static int chunks_of(int K) { return (K + kChunkK - 1) / kChunkK; }
 static size_t frag_bytes(int K, int R) {
     return static_cast<size_t>(chunks_of(K)) * R * kFragRowHalves * 2;
 }
-static size_t gsum_bytes(int K, int R) { return static_cast<size_t>(chunks_of(K)) * R * 16; }
 
 struct LorcPlan {
     int splits, row_groups;
 };
 
 struct LinearWs {
-    size_t grp, rows, inv, frag, gsum, t, tpart, part, total;
+    size_t grp, rows, inv, frag, t, tpart, part, total;
     int R, splits, tcols;
     LorcPlan lp;
 };
@@ -161,7 +156,6 @@ static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
     w.rows = c.take(static_cast<size_t>(w.R) * 4);
     w.inv = c.take(static_cast<size_t>(w.R) * 4);
     w.frag = c.take(frag_bytes(lin->K, w.R));
-    w.gsum = c.take(gsum_bytes(lin->K, w.R));
     w.t = c.take(static_cast<size_t>(w.R) * w.tcols * 2);
     w.lp = lorc_plan(n_exp, 1, lin->K, std::max(1LL, static_cast<long long>(w.R) / std::max<long long>(1, groups)));
     w.tpart = c.take(static_cast<size_t>(w.lp.splits) * w.R * w.tcols * 4);
@@ -171,7 +165,7 @@ static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
 }
 
 struct MoeWs {
-    size_t grp, rows, xfrag, xg, t13, h, hfrag, hg, t2, tpart, part, total;
+    size_t grp, rows, xfrag, t13, h, hfrag, t2, tpart, part, total;
     int R, R_routed, splits, tc13, tc2;
     LorcPlan lp13, lp2;
 };
@@ -191,11 +185,9 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
     w.grp = c.take(static_cast<size_t>(n_exp) * 8);
     w.rows = c.take(static_cast<size_t>(w.R) * 4);
     w.xfrag = c.take(frag_bytes(H, w.R));
-    w.xg = c.take(gsum_bytes(H, w.R));
     w.t13 = c.take(static_cast<size_t>(w.R) * w.tc13 * 2);
     w.h = c.take(static_cast<size_t>(w.R) * I * 2);
     w.hfrag = c.take(frag_bytes(I, w.R));
-    w.hg = c.take(gsum_bytes(I, w.R));
     w.t2 = c.take(static_cast<size_t>(w.R) * w.tc2 * 2);
     const long long rows_per_exp = std::max(1LL, static_cast<long long>(w.R) / std::max<long long>(1, groups));
     w.lp13 = lorc_plan(n_exp, 2, H, rows_per_exp);
@@ -210,9 +202,8 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
 // ---------------------------------------------------------------------------
 // launch helpers
 // ---------------------------------------------------------------------------
-static void act_ptrs(GemvParams& g, void* frag, void* gsum, void* t, int R, int K, int tcols, bool has_t) {
+static void act_ptrs(GemvParams& g, void* frag, void* t, int R, int K, int tcols, bool has_t) {
     g.x = static_cast<const uint16_t*>(frag);
-    g.gsum = static_cast<const float*>(gsum);
     g.t = has_t ? static_cast<const uint16_t*>(t) : nullptr;
     g.R = R;
     g.K = K;
@@ -360,7 +351,7 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     int32_t* inv = reinterpret_cast<int32_t*>(base + w.inv);
 
     PrepParams pp{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.frag),
-                  reinterpret_cast<float*>(base + w.gsum), dev_status, w.R, lin->K, x_dt == MILO_BF16, 1,
+                  dev_status, w.R, lin->K, x_dt == MILO_BF16, 1,
                   expert_offsets, perm, grp, inv, T, k, lin->n_experts, 0, w.R};
     milo_status s = check_cuda(launch_prep(pp, st), "prep");
     if (s != MILO_OK) return s;
@@ -377,7 +368,7 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
 
     GemvParams g;
     memset(&g, 0, sizeof(g));
-    act_ptrs(g, base + w.frag, base + w.gsum, base + w.t, w.R, lin->K, w.tcols, has_t);
+    act_ptrs(g, base + w.frag, base + w.t, w.R, lin->K, w.tcols, has_t);
     g.table = table;
     g.grp = grp;
     g.y_part = reinterpret_cast<float*>(base + w.part);
@@ -426,7 +417,7 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     milo_status s;
 
     PrepParams px{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.xfrag),
-                  reinterpret_cast<float*>(base + w.xg), dev_status, w.R, H, x_dt == MILO_BF16, 1,
+                  dev_status, w.R, H, x_dt == MILO_BF16, 1,
                   expert_offsets, perm, grp, nullptr, T, L->top_k, L->n_routed, L->n_shared, w.R_routed};
     if ((s = check_cuda(launch_prep(px, st), "prep x")) != MILO_OK) return s;
     if (has_t) {
@@ -439,7 +430,7 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
 
     GemvParams g1;
     memset(&g1, 0, sizeof(g1));
-    act_ptrs(g1, base + w.xfrag, base + w.xg, base + w.t13, w.R, H, w.tc13, has_t);
+    act_ptrs(g1, base + w.xfrag, base + w.t13, w.R, H, w.tc13, has_t);
     g1.table = table;
     g1.grp = grp;
     g1.h = reinterpret_cast<uint16_t*>(base + w.h);
@@ -457,8 +448,8 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     prof_record(1, st);
 
     PrepParams ph{reinterpret_cast<const uint16_t*>(base + w.h), nullptr,
-                  reinterpret_cast<uint16_t*>(base + w.hfrag), reinterpret_cast<float*>(base + w.hg),
-                  dev_status, w.R, I, 0, 0, nullptr, nullptr, nullptr, nullptr, 0, 0, 0, 0, 0};
+                  reinterpret_cast<uint16_t*>(base + w.hfrag), dev_status, w.R, I, 0, 0, nullptr, nullptr,
+                  nullptr, nullptr, 0, 0, 0, 0, 0};
     if ((s = check_cuda(launch_prep(ph, st), "prep h")) != MILO_OK) return s;
     if (has_t) {
         LorcParams lp{reinterpret_cast<const uint16_t*>(base + w.h), nullptr, table, grp,
@@ -469,7 +460,7 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
 
     GemvParams g2;
     memset(&g2, 0, sizeof(g2));
-    act_ptrs(g2, base + w.hfrag, base + w.hg, base + w.t2, w.R, I, w.tc2, has_t);
+    act_ptrs(g2, base + w.hfrag, base + w.t2, w.R, I, w.tc2, has_t);
     g2.table = table;
     g2.grp = grp;
     g2.y_part = reinterpret_cast<float*>(base + w.part);

@@ -132,11 +132,13 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
         s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
         s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 2);
         if (!active) continue;
-        // chunk-major layout: the 16-row tile of one K chunk is one contiguous block
+        // chunk-major layout: the 16-row tile of one K chunk is one contiguous
+        // block; the chunk's four group sums sit in the row's padding
         const size_t crow = static_cast<size_t>(sb >> 1) * p.R + row;
         if (c == 0) {
-            p.gsum[crow * 4 + 2 * (sb & 1)] = s0;
-            p.gsum[crow * 4 + 2 * (sb & 1) + 1] = s1;
+            float* gs = reinterpret_cast<float*>(p.frag + crow * kFragRowHalves + kGsumHalf);
+            gs[2 * (sb & 1)] = s0;
+            gs[2 * (sb & 1) + 1] = s1;
         }
         // per super-block: step-major, lane-in-quad c, 4 fp16 each
         uint2* out = reinterpret_cast<uint2*>(p.frag + crow * kFragRowHalves + (sb & 1) * kFragHalvesPerSB) + c;

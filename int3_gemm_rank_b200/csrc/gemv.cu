@@ -13,11 +13,13 @@
 // B200 design (not a translation of the page's kernel):
 //   - One producer thread streams each CTA's weight tile into a 3-stage
 //     shared-memory ring guarded by mbarriers.  The packed weights are stored
-//     in 64-row tiles (milo.h), so a K chunk of a tile (codes, scales, zeros)
-//     is a handful of contiguous blocks, each fetched by one 1-D bulk copy of
-//     the TMA engine; the prepared activations and group sums of the item's
-//     routed rows are contiguous too.  Weights are read from HBM exactly once
-//     per token tile, with an evict-first L2 policy.
+//     as (64-row tile, K chunk) blocks holding codes, scales and zeros
+//     (milo.h), and the prepared activations of the item's routed rows (group
+//     sums in the row padding) are contiguous too, so a stage is two or three
+//     1-D bulk copies of the TMA engine.  Each copy instruction costs the
+//     issuing thread about the same whatever its size, so the layout keeps
+//     their number minimal.  Weights are read from HBM exactly once per token
+//     tile, with an evict-first L2 policy.
 //   - Four consumer warps each own 32 weight rows.  A lane reads its 3-word
 //     unit of two rows and extracts code pairs with one LOP3 each (plus one
 //     shift per word): the masked fp16 pattern already is code * 8^i * 2^-24,
@@ -46,21 +48,19 @@ namespace milo {
 constexpr int kStages = 3;
 constexpr int kConsumerWarps = 4;
 constexpr int kGemvThreads = 32 * (kConsumerWarps + 1);
-// Stage layout (bytes).  Codes: two 64-row tiles, each [2 super-blocks][64
-// rows][12 words] (GLU: w1's tile, then w3's; plain: rows 0-63, then 64-127).
-// Scales/zeros: [4 groups][64 rows] fp16 blocks, GLU: w1 s, w1 z, w3 s, w3 z;
-// plain: s rows 0-63, s rows 64-127, z rows 0-63, z rows 64-127.
+// Stage layout (bytes).  Two weight regions of kTileBlk bytes, each one
+// (tile, chunk) block of the packed blob: codes [nsb][64 rows][12 words], then
+// per group [64 scales][64 zeros] (GLU: w1's tile, then w3's; plain: rows
+// 0-63, then 64-127).  Then the activations [16 rows][272 fp16].
+constexpr int kTileBlk = 2 * kBlockSB;                    // 7168
 constexpr int kOffQ = 0;
-constexpr int kOffQB = 2 * kQTileSBWords * 4;            // 6144
-constexpr int kOffS = 2 * kOffQB;                         // 12288
-constexpr int kOffX = kOffS + 2048;                       // activations [16 rows][272 fp16]
-constexpr int kOffG = kOffX + kTokTile * kFragRowHalves * 2;   // group sums [16 rows][4] f32
-constexpr int kStageBytes = kOffG + kTokTile * 16;
+constexpr int kOffX = 2 * kTileBlk;                       // 14336
+constexpr int kStageBytes = kOffX + kTokTile * kFragRowHalves * 2;
 constexpr int kOffUA = 0, kOffUB = 8192, kOffT = 16384;   // compensator stage
 constexpr int kBarOffset = kStages * kStageBytes;
 constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 3 * (MILO_MAX_EXPERTS + 1) * 4 + 16;
 
-static_assert(kStageBytes % 16 == 0 && kOffX % 16 == 0 && kOffG % 16 == 0, "bulk-copy alignment");
+static_assert(kStageBytes % 16 == 0 && kOffX % 16 == 0 && kTileBlk % 16 == 0, "bulk-copy alignment");
 static_assert(kOffT >= kRowsPlain * MILO_MAX_RANK * 2, "compensator stage: U rows");
 static_assert(kOffT + kTokTile * 2 * MILO_MAX_RANK * 2 <= kStageBytes, "compensator stage: t rows");
 
@@ -113,52 +113,48 @@ __device__ __forceinline__ void code_step(const uint32_t (&wd)[2][2][3], const u
     }
 }
 
-// Per m16 tile ti of a consumer warp: word offset of its 64-row code tile in
-// the stage, first row inside that tile, byte offset of its scales (zeros
-// follow at zdelta).
+// Per m16 tile ti of a consumer warp: byte offset of its weight region in the
+// stage and its first row inside the 64-row tile.
 template <bool GLU>
 struct TileMap {
-    int q[2], r[2], s[2];
-    static constexpr int zdelta = GLU ? 512 : 1024;
+    int reg[2], r[2];
     __device__ __forceinline__ explicit TileMap(int warp) {
 #pragma unroll
         for (int ti = 0; ti < 2; ++ti) {
             if (GLU) {
-                q[ti] = ti * (kOffQB / 4);
+                reg[ti] = ti * kTileBlk;
                 r[ti] = 16 * warp;
-                s[ti] = kOffS + ti * 1024;
             } else {
-                const int half = warp >> 1;
-                q[ti] = half * (kOffQB / 4);
+                reg[ti] = (warp >> 1) * kTileBlk;
                 r[ti] = 32 * (warp & 1) + 16 * ti;
-                s[ti] = kOffS + half * 512;
             }
         }
     }
 };
 
-// acc += s * 2^24 * D_g - s * z * X_g for the scale group `grp` of the stage.
-template <bool GLU, int NT>
+// acc += s * 2^24 * D_g - s * z * X_g for group `grp` (0..3) of the chunk;
+// the scales of the chunk's groups start nsb * 3072 bytes into each region.
+template <int NT>
 __device__ __forceinline__ void fold_group(float (&acc)[2][2][4], const float (&dz)[2][2][4],
-                                           const uint8_t* st, int grp, const TileMap<GLU>& tm,
-                                           int g, int c) {
-    const float* gs = reinterpret_cast<const float*>(st + kOffG);
+                                           const uint8_t* st, int grp, const int (&reg)[2],
+                                           const int (&rbase)[2], int nsb, int g, int c) {
     float xg[NT][2];
 #pragma unroll
-    for (int n8 = 0; n8 < NT; ++n8) {
-        xg[n8][0] = gs[(n8 * 8 + 2 * c) * 4 + grp];
-        xg[n8][1] = gs[(n8 * 8 + 2 * c + 1) * 4 + grp];
-    }
+    for (int n8 = 0; n8 < NT; ++n8)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int tok = n8 * 8 + 2 * c + j;
+            xg[n8][j] = reinterpret_cast<const float*>(st + kOffX + (tok * kFragRowHalves + kGsumHalf) * 2)[grp];
+        }
 #pragma unroll
     for (int ti = 0; ti < 2; ++ti) {
-        const __half* S = reinterpret_cast<const __half*>(st + tm.s[ti]);
-        const __half* Z = reinterpret_cast<const __half*>(st + tm.s[ti] + TileMap<GLU>::zdelta);
+        const __half* S = reinterpret_cast<const __half*>(st + reg[ti] + nsb * kQTileSBWords * 4 + grp * kGroupBytes);
         float s24[2], nsz[2];
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
-            const int row = tm.r[ti] + g + 8 * rr;
-            const float sv = __half2float(S[grp * kTileRows + row]);
-            const float zv = __half2float(Z[grp * kTileRows + row]);
+            const int row = rbase[ti] + g + 8 * rr;
+            const float sv = __half2float(S[row]);
+            const float zv = __half2float(S[kTileRows + row]);
             s24[rr] = sv * 16777216.0f;
             nsz[rr] = -sv * zv;
         }
@@ -177,32 +173,33 @@ template <bool GLU, int NT>
 __device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2][2][4], const TileMap<GLU>& tm,
                                               int nsb, int lane) {
     const int g = lane >> 2, c = lane & 3;
-    const uint32_t* qt = reinterpret_cast<const uint32_t*>(st + kOffQ);
 #pragma unroll
     for (int sbl = 0; sbl < 2; ++sbl) {
         if (sbl == nsb) break;
         uint32_t wd[2][2][3], hw[2][2][3];
 #pragma unroll
-        for (int ti = 0; ti < 2; ++ti)
+        for (int ti = 0; ti < 2; ++ti) {
+            const uint32_t* qt = reinterpret_cast<const uint32_t*>(st + tm.reg[ti]) + sbl * kQTileSBWords;
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
                 for (int t = 0; t < 3; ++t) {
-                    wd[ti][rr][t] = qt[tm.q[ti] + sbl * kQTileSBWords + (tm.r[ti] + g + 8 * rr) * 12 + 3 * c + t];
+                    wd[ti][rr][t] = qt[(tm.r[ti] + g + 8 * rr) * 12 + 3 * c + t];
                     hw[ti][rr][t] = wd[ti][rr][t] >> 9;
                 }
+        }
         const uint8_t* xs = st + kOffX + sbl * kFragHalvesPerSB * 2;
         float dz[2][2][4];
         code_step<0, NT>(wd, hw, xs, g, c, dz);
         code_step<1, NT>(wd, hw, xs, g, c, dz);
         code_step<2, NT>(wd, hw, xs, g, c, dz);
         code_step<3, NT>(wd, hw, xs, g, c, dz);
-        fold_group<GLU, NT>(acc, dz, st, 2 * sbl, tm, g, c);
+        fold_group<NT>(acc, dz, st, 2 * sbl, tm.reg, tm.r, nsb, g, c);
         code_step<4, NT>(wd, hw, xs, g, c, dz);
         code_step<5, NT>(wd, hw, xs, g, c, dz);
         code_step<6, NT>(wd, hw, xs, g, c, dz);
         code_step<7, NT>(wd, hw, xs, g, c, dz);
-        fold_group<GLU, NT>(acc, dz, st, 2 * sbl + 1, tm, g, c);
+        fold_group<NT>(acc, dz, st, 2 * sbl + 1, tm.reg, tm.r, nsb, g, c);
     }
 }
 
@@ -298,28 +295,17 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 filled |= 1u << stage;
                 fph = (fph & ~(1u << stage)) | (phase << stage);
                 const int nsb = min(2, p.SB - 2 * ch);
-                const uint32_t qb = nsb * kQTileSBWords * 4;        // codes of one tile
-                const uint32_t gb = nsb * 2 * kTileRows * 2;         // scales (zeros) of one tile
+                const uint32_t wb = nsb * kBlockSB;                  // one tile's block
                 const uint32_t xb = ntok * kFragRowHalves * 2;
-                const uint32_t tb = ntok * 16;
-                mbar_arrive_expect_tx(fb, ntl * (qb + 2 * gb) + xb + tb);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    if (h == ntl) break;
-                    const ProjDev* pj = (GLU && h == 1) ? pb : pa;
-                    const int tile = GLU ? tile0 : tile0 + h;
-                    bulk_load_hint(st + kOffQ + h * kOffQB,
-                                   pj->q + (static_cast<size_t>(tile) * p.SB + 2 * ch) * kQTileSBWords, qb, fb, pol);
-                    const size_t go = (static_cast<size_t>(tile) * p.G + 4 * ch) * kTileRows;
-                    // GLU: [s a | z a | s b | z b]; plain: [s t0 | s t1 | z t0 | z t1]
-                    const int so = GLU ? kOffS + h * 1024 : kOffS + h * 512;
-                    const int zo = GLU ? so + 512 : so + 1024;
-                    bulk_load_hint(st + so, pj->scale + go, gb, fb, pol);
-                    bulk_load_hint(st + zo, pj->zero + go, gb, fb, pol);
-                }
-                const size_t xr = static_cast<size_t>(ch) * p.R + row0;
-                bulk_load(st + kOffX, p.x + xr * kFragRowHalves, xb, fb);
-                bulk_load(st + kOffG, p.gsum + xr * 4, tb, fb);
+                mbar_arrive_expect_tx(fb, ntl * wb + xb);
+                bulk_load_hint(st + kOffQ, pa->packed + (static_cast<size_t>(tile0) * p.SB + 2 * ch) * kBlockSB,
+                               wb, fb, pol);
+                if (ntl == 2)
+                    bulk_load_hint(st + kOffQ + kTileBlk,
+                                   (GLU ? pb->packed + (static_cast<size_t>(tile0) * p.SB + 2 * ch) * kBlockSB
+                                        : pa->packed + (static_cast<size_t>(tile0 + 1) * p.SB + 2 * ch) * kBlockSB),
+                                   wb, fb, pol);
+                bulk_load(st + kOffX, p.x + (static_cast<size_t>(ch) * p.R + row0) * kFragRowHalves, xb, fb);
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
             }
             const int ra = pa->rank, rb = GLU ? pb->rank : 0;

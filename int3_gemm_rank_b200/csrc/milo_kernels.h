@@ -20,20 +20,23 @@ constexpr int kChunkK = 256;       // K per pipeline stage (two 128-code super-b
 // super-block 8 MMA steps x 4 lanes-in-quad x 4 fp16, then 16 fp16 of padding
 // so that the rows of a 16-row tile fall on different shared-memory banks
 // (row pitch 136 words, 8 mod 32): 272 fp16 (544 bytes).
+// The first 8 padding fp16 hold the chunk's four group sums (f32).
 constexpr int kFragHalvesPerSB = 128;
 constexpr int kFragRowHalves = 2 * kFragHalvesPerSB + 16;
+constexpr int kGsumHalf = 2 * kFragHalvesPerSB;
 
-// Rows of the packed weights are grouped in tiles of 64 (milo.h): a tile's
-// words for one super-block, and its scales (zeros) for one group, are
-// contiguous, so a K chunk of a tile arrives with one bulk copy per tensor.
+// Packed weights (milo.h): rows in tiles of 64, K in chunks of two
+// super-blocks; each (tile, chunk) block -- the codes of its super-blocks, then
+// per group 64 scales and 64 zeros -- is contiguous, so one bulk copy brings a
+// tile's chunk.  kBlockSB bytes per tile and super-block.
 constexpr int kTileRows = 64;
-constexpr int kQTileSBWords = kTileRows * 12;       // one tile, one super-block: 3072 bytes
+constexpr int kQTileSBWords = kTileRows * 12;       // codes of one tile, one super-block: 3072 bytes
+constexpr int kGroupBytes = kTileRows * 2 * 2;      // scales and zeros of one tile, one group: 256 bytes
+constexpr int kBlockSB = kQTileSBWords * 4 + 2 * kGroupBytes;   // 3584
 
 // One projection in the device table (device pointers and shape).
-struct alignas(16) ProjDev {
-    const uint32_t* q;          // [ceil(N/64)][K/128][64][12] words
-    const uint16_t* scale;      // [ceil(N/64)][K/64][64] fp16
-    const uint16_t* zero;       // [ceil(N/64)][K/64][64] fp16
+struct alignas(64) ProjDev {
+    const uint8_t* packed;      // blob of ceil(N/64) * (K/128) * kBlockSB bytes
     const uint16_t* U;          // [N][rank] fp16, NULL when rank == 0
     const uint16_t* V;          // [rank][K] fp16, NULL when rank == 0
     int32_t rank, N, K, pad;
@@ -41,7 +44,7 @@ struct alignas(16) ProjDev {
 
 struct GemvParams {
     const uint16_t* x;          // prepared activations [chunks][R][kFragRowHalves] fp16
-    const float* gsum;          // group sums [chunks][R][4] f32
+                                // (group sums in each row's padding, see kGsumHalf)
     const uint16_t* t;          // LoRC down-projection [R][tcols] fp16
     const ProjDev* table;       // device table
     const int32_t* grp;         // [n_exp][2]: first row, row count of each group (expert)
@@ -59,7 +62,6 @@ struct PrepParams {
     int32_t* row_src;           // row p -> source row; built here when `rows` is set, else
                                 // read (NULL: identity); -1 = zero row
     uint16_t* frag;             // [chunks][R][kFragRowHalves] fp16, chunks = ceil(K/256)
-    float* gsum;                // [chunks][R][4] f32
     int32_t* dev_status;
     int R, K, src_bf16;
     // Row bookkeeping (first preparation of a call only): routed rows come from

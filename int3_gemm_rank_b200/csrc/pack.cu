@@ -9,36 +9,43 @@
 
 #include "milo_device.cuh"
 #include "milo_host.h"
+#include "milo_kernels.h"
 
 namespace milo {
 
-// Device layout (milo.h): rows in tiles of 64, the last tile padded with zero
-// rows; within a tile, super-block (group) major.
-__device__ __forceinline__ size_t q_tiled(int n, int b, int SB) {
-    return (static_cast<size_t>(n / 64) * SB + b) * 768 + static_cast<size_t>(n % 64) * 12;
+// Device blob (milo.h): 64-row tiles, K chunks of two super-blocks, each
+// (tile, chunk) block = the words of its super-blocks, then per group the 64
+// scales and the 64 zeros.  Byte offsets of row n's words for super-block b
+// and of its scale for group j (its zero follows 128 bytes later).
+__device__ __forceinline__ size_t blob_words(int n, int b, int SB) {
+    const int c = b >> 1;
+    return (static_cast<size_t>(n / 64) * SB + 2 * c) * kBlockSB + ((b & 1) * 64 + (n % 64)) * 48;
 }
-__device__ __forceinline__ size_t g_tiled(int n, int j, int G) {
-    return (static_cast<size_t>(n / 64) * G + j) * 64 + (n % 64);
+__device__ __forceinline__ size_t blob_group(int n, int j, int SB) {
+    const int c = j >> 2, nsb = min(2, SB - 2 * c);
+    return (static_cast<size_t>(n / 64) * SB + 2 * c) * kBlockSB + nsb * 3072 + (j & 3) * 256 + (n % 64) * 2;
 }
 
 // One thread per (row, 128-code super-block): two scale groups.  Rows N..
 // of the last tile get zero words, scales and zeros.
 __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ W, int N, int K,
-                                                   uint32_t* __restrict__ Q,
-                                                   uint16_t* __restrict__ scale,
-                                                   uint16_t* __restrict__ zero,
+                                                   uint8_t* __restrict__ blob,
                                                    int32_t* __restrict__ dev_status) {
-    const int SB = K / 128, G = K / 64;
+    const int SB = K / 128;
     const int Npad = (N + 63) / 64 * 64;
     const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (gid >= static_cast<long long>(Npad) * SB) return;
     const int n = static_cast<int>(gid / SB);
     const int b = static_cast<int>(gid % SB);
+    uint16_t* sz = reinterpret_cast<uint16_t*>(blob);
     if (n >= N) {
-        uint4* dst = reinterpret_cast<uint4*>(Q + q_tiled(n, b, SB));
+        uint4* dst = reinterpret_cast<uint4*>(blob + blob_words(n, b, SB));
         dst[0] = dst[1] = dst[2] = make_uint4(0u, 0u, 0u, 0u);
-        scale[g_tiled(n, 2 * b, G)] = scale[g_tiled(n, 2 * b + 1, G)] = 0;
-        zero[g_tiled(n, 2 * b, G)] = zero[g_tiled(n, 2 * b + 1, G)] = 0;
+        for (int g = 0; g < 2; ++g) {
+            const size_t o = blob_group(n, 2 * b + g, SB) / 2;
+            sz[o] = 0;
+            sz[o + 64] = 0;
+        }
         return;
     }
     const uint16_t* w = W + static_cast<size_t>(n) * K + static_cast<size_t>(b) * 128;
@@ -61,9 +68,9 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
         const __half zh = __float2half_rn(__fdiv_rn(-mn, s));
         const float z = __half2float(zh);
         if (!isfinite(s) || !isfinite(z)) st |= MILO_DEV_FP16_RANGE;
-        const int j = 2 * b + g;
-        scale[g_tiled(n, j, G)] = __half_as_ushort(sh);
-        zero[g_tiled(n, j, G)] = __half_as_ushort(zh);
+        const size_t o = blob_group(n, 2 * b + g, SB) / 2;
+        sz[o] = __half_as_ushort(sh);
+        sz[o + 64] = __half_as_ushort(zh);
         for (int i = 0; i < 64; ++i) {
             const float v = __fadd_rn(__fdiv_rn(__half2float(__ushort_as_half(w[64 * g + i])), s), z);
             float r = rintf(v);
@@ -90,7 +97,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
         for (int t = 0; t < 3; ++t)
             words[3 * c + t] |= (((u30 >> t) & 1u) << 15) | (((u31 >> t) & 1u) << 31);
     }
-    uint4* dst = reinterpret_cast<uint4*>(Q + q_tiled(n, b, SB));
+    uint4* dst = reinterpret_cast<uint4*>(blob + blob_words(n, b, SB));
     dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
     dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
     dst[2] = make_uint4(words[8], words[9], words[10], words[11]);
@@ -118,7 +125,7 @@ __device__ __forceinline__ void unpack_step(const uint32_t (&w)[3], const uint32
     unpack_reg<S, 1>(w, hw, u);
 }
 
-__global__ void __launch_bounds__(128) unpack_kernel(const uint32_t* __restrict__ Q, int N, int K,
+__global__ void __launch_bounds__(128) unpack_kernel(const uint8_t* __restrict__ blob, int N, int K,
                                                      uint8_t* __restrict__ codes) {
     const int SB = K / 128;
     const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -126,7 +133,7 @@ __global__ void __launch_bounds__(128) unpack_kernel(const uint32_t* __restrict_
     const int c = static_cast<int>(gid % 4);
     const long long nb = gid / 4;
     const int n = static_cast<int>(nb / SB), b = static_cast<int>(nb % SB);
-    const uint32_t* src = Q + q_tiled(n, b, SB) + 3 * c;
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(blob + blob_words(n, b, SB)) + 3 * c;
     const uint32_t w[3] = {src[0], src[1], src[2]};
     const uint32_t hw[3] = {w[0] >> 9, w[1] >> 9, w[2] >> 9};
     uint8_t u[32];
@@ -149,50 +156,43 @@ __global__ void __launch_bounds__(128) unpack_kernel(const uint32_t* __restrict_
 
 using namespace milo;
 
-extern "C" milo_status milo_pack(const uint16_t* W, int32_t N, int32_t K, int32_t group,
-                                 uint32_t* Q, uint16_t* scale, uint16_t* zero,
+extern "C" milo_status milo_pack(const uint16_t* W, int32_t N, int32_t K, int32_t group, void* packed,
                                  int32_t* dev_status, void* stream) {
     clear_error();
     if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, "milo_pack: N and K must be positive");
     if (group != MILO_GROUP) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_pack: group must be 64");
     if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_pack: K must be a multiple of 128");
-    if (!W || !Q || !scale || !zero) return fail(MILO_ERR_INVALID_ARG, "milo_pack: NULL pointer");
-    if (!aligned(Q, 16) || !aligned(W, 2))
-        return fail(MILO_ERR_INVALID_ARG, "milo_pack: Q must be 16-byte aligned");
-    if (!aligned(scale, 2) || !aligned(zero, 2))
-        return fail(MILO_ERR_INVALID_ARG, "milo_pack: scale and zero must be 2-byte aligned");
+    if (!W || !packed) return fail(MILO_ERR_INVALID_ARG, "milo_pack: NULL pointer");
+    if (!aligned(packed, 16) || !aligned(W, 2))
+        return fail(MILO_ERR_INVALID_ARG, "milo_pack: the packed buffer must be 16-byte aligned");
     const long long threads = static_cast<long long>((N + 63) / 64 * 64) * (K / 128);
     const int block = 128;
     const long long grid = (threads + block - 1) / block;
     if (grid > 0x7FFFFFFFLL) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_pack: too large");
     pack_kernel<<<static_cast<unsigned>(grid), block, 0, static_cast<cudaStream_t>(stream)>>>(
-        W, N, K, Q, scale, zero, dev_status);
+        W, N, K, static_cast<uint8_t*>(packed), dev_status);
     return check_launch("milo_pack");
 }
 
-extern "C" milo_status milo_unpack(const uint32_t* Q, int32_t N, int32_t K, uint8_t* codes,
-                                   void* stream) {
+extern "C" milo_status milo_unpack(const void* packed, int32_t N, int32_t K, uint8_t* codes, void* stream) {
     clear_error();
-    if (!Q || !codes) return fail(MILO_ERR_INVALID_ARG, "milo_unpack: NULL pointer");
+    if (!packed || !codes) return fail(MILO_ERR_INVALID_ARG, "milo_unpack: NULL pointer");
     if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, "milo_unpack: N and K must be positive");
     if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_unpack: K must be a multiple of 128");
-    if (!aligned(Q, 4)) return fail(MILO_ERR_INVALID_ARG, "milo_unpack: Q must be 4-byte aligned");
+    if (!aligned(packed, 4)) return fail(MILO_ERR_INVALID_ARG, "milo_unpack: the packed buffer must be 4-byte aligned");
     const long long threads = static_cast<long long>(N) * (K / 128) * 4;
     const int block = 128;
     const long long grid = (threads + block - 1) / block;
     if (grid > 0x7FFFFFFFLL) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_unpack: too large");
     unpack_kernel<<<static_cast<unsigned>(grid), block, 0, static_cast<cudaStream_t>(stream)>>>(
-        Q, N, K, codes);
+        static_cast<const uint8_t*>(packed), N, K, codes);
     return check_launch("milo_unpack");
 }
 
-extern "C" milo_status milo_packed_bytes(int32_t N, int32_t K, size_t* q_bytes, size_t* group_bytes) {
+extern "C" milo_status milo_packed_bytes(int32_t N, int32_t K, size_t* bytes) {
     clear_error();
-    if (N <= 0 || K <= 0 || !q_bytes || !group_bytes)
-        return fail(MILO_ERR_INVALID_ARG, "milo_packed_bytes: bad argument");
+    if (N <= 0 || K <= 0 || !bytes) return fail(MILO_ERR_INVALID_ARG, "milo_packed_bytes: bad argument");
     if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_packed_bytes: K must be a multiple of 128");
-    const size_t rows = static_cast<size_t>(N + 63) / 64 * 64;
-    *q_bytes = rows * (3 * static_cast<size_t>(K) / 32) * 4;
-    *group_bytes = rows * (static_cast<size_t>(K) / 64) * 2;
+    *bytes = static_cast<size_t>((N + 63) / 64) * (K / 128) * kBlockSB;
     return MILO_OK;
 }

@@ -59,8 +59,7 @@ def lib():
         L.milo_ref_pack.argtypes = [vp, i, i, vp]; L.milo_ref_pack.restype = None
         L.milo_ref_unpack.argtypes = [vp, i, i, vp]; L.milo_ref_unpack.restype = None
         L.milo_ref_code_bit.argtypes = [i, i, C.POINTER(i), C.POINTER(i)]
-        L.milo_ref_tile_words.argtypes = [vp, i, i, vp]; L.milo_ref_tile_words.restype = None
-        L.milo_ref_tile_groups.argtypes = [vp, i, i, vp]; L.milo_ref_tile_groups.restype = None
+        L.milo_ref_tile_pack.argtypes = [vp, vp, vp, i, i, vp]; L.milo_ref_tile_pack.restype = None
         L.milo_ref_dequant.argtypes = [vp, vp, vp, i, i, i, vp]; L.milo_ref_dequant.restype = None
         L.milo_ref_group.argtypes = [vp, i, i, i, vp, vp, vp]; L.milo_ref_group.restype = i
         L.milo_ref_route.argtypes = [vp, i, i, i, i, vp, vp, vp, vp, vp]; L.milo_ref_route.restype = i
@@ -122,23 +121,14 @@ def unpack(Q: np.ndarray, K: int) -> np.ndarray:
     return q
 
 
-def tile_words(Q: np.ndarray, K: int) -> np.ndarray:
-    """Row-major packed words [N, 3K/32] -> the device layout [ceil(N/64), K/128, 64, 12]."""
-    Q = _c(Q, np.uint32)
+def tile_pack(Q: np.ndarray, scale: np.ndarray, zero: np.ndarray, K: int) -> np.ndarray:
+    """Row-major words [N, 3K/32] and group-major scale, zero [K/64, N] -> the device
+    blob (u8, ceil(N/64) * K/128 * 3584 bytes)."""
+    Q = _c(Q, np.uint32); s = _c(scale, np.uint16); z = _c(zero, np.uint16)
     N = Q.shape[0]
-    NT = (N + 63) // 64
-    Qt = np.zeros((NT, K // 128, 64, 12), np.uint32)
-    lib().milo_ref_tile_words(_p(Q), N, K, _p(Qt))
-    return Qt
-
-
-def tile_groups(A: np.ndarray) -> np.ndarray:
-    """Group-major [G, N] (scale or zero) -> the device layout [ceil(N/64), G, 64]."""
-    A = _c(A, np.uint16)
-    G, N = A.shape
-    At = np.zeros(((N + 63) // 64, G, 64), np.uint16)
-    lib().milo_ref_tile_groups(_p(A), N, G, _p(At))
-    return At
+    blob = np.zeros(((N + 63) // 64) * (K // 128) * 3584, np.uint8)
+    lib().milo_ref_tile_pack(_p(Q), _p(s), _p(z), N, K, _p(blob))
+    return blob
 
 
 def code_bit(k: int, beta: int):

@@ -215,30 +215,41 @@ void milo_ref_unpack(const uint32_t* Q, int N, int K, uint8_t* q) {
 }
 
 /*
- * Device layout of the packed tensors.  The GPU kernels fetch the words of 64
- * rows for one or two super-blocks as one contiguous block, so the device
- * buffers group rows in tiles of 64 (the last tile padded with zero rows):
- *     Qt[((n / 64) * SB + b) * 768 + (n % 64) * 12 + j] = Q[n, 12 b + j]
- *     At[((n / 64) * G + g) * 64 + (n % 64)]           = A[g, n]
- * (SB = K / 128 super-blocks, G = K / 64 groups; A is a scale or zero array
- * [G, N]).  These are relayouts only, used to compare with the device packer.
+ * Device layout of a packed weight: one byte blob.  Rows are grouped in tiles
+ * of 64 (the last tile padded with zero rows), K in chunks of two super-blocks
+ * (the last chunk has one when K/128 is odd), and each (tile, chunk) block is
+ * contiguous, so the GPU kernels fetch it with a single copy:
+ *     block(t, c) at byte (t * SB + 2 * c) * 3584, holding for its nsb
+ *     super-blocks b (in order) the words  [64 rows][12]        (nsb * 3072 B)
+ *     then for its 2 * nsb groups g (in order)  [64 s fp16][64 z fp16]  (256 B each)
+ * Word j of row n, super-block b, is Q[n, 12 b + j]; s and z of row n, group
+ * g are scale[g, n] and zero[g, n].  This is a relayout only, used to compare
+ * with the device packer.
  */
-void milo_ref_tile_words(const uint32_t* Q, int N, int K, uint32_t* Qt) {
-    int SB = K / 128, W = 3 * K / 32, NT = (N + 63) / 64;
-    memset(Qt, 0, sizeof(uint32_t) * (size_t)NT * 64 * W);
-    for (int n = 0; n < N; ++n)
-        for (int b = 0; b < SB; ++b)
-            for (int j = 0; j < 12; ++j)
-                Qt[((size_t)(n / 64) * SB + b) * 768 + (size_t)(n % 64) * 12 + j] =
-                    Q[(size_t)n * W + 12 * b + j];
-}
-
-void milo_ref_tile_groups(const uint16_t* A, int N, int G, uint16_t* At) {
-    int NT = (N + 63) / 64;
-    memset(At, 0, sizeof(uint16_t) * (size_t)NT * 64 * G);
-    for (int g = 0; g < G; ++g)
-        for (int n = 0; n < N; ++n)
-            At[((size_t)(n / 64) * G + g) * 64 + (n % 64)] = A[(size_t)g * N + n];
+void milo_ref_tile_pack(const uint32_t* Q, const uint16_t* scale, const uint16_t* zero,
+                        int N, int K, uint8_t* blob) {
+    int SB = K / 128, G = K / 64, W = 3 * K / 32, NT = (N + 63) / 64;
+    memset(blob, 0, (size_t)NT * SB * 3584);
+    for (int t = 0; t < NT; ++t)
+        for (int c = 0; 2 * c < SB; ++c) {
+            int nsb = SB - 2 * c < 2 ? SB - 2 * c : 2;
+            uint8_t* base = blob + ((size_t)t * SB + 2 * c) * 3584;
+            uint32_t* words = (uint32_t*)base;
+            uint16_t* groups = (uint16_t*)(base + (size_t)nsb * 3072);
+            for (int r = 0; r < 64; ++r) {
+                int n = 64 * t + r;
+                if (n >= N) continue;
+                for (int i = 0; i < nsb; ++i)
+                    for (int j = 0; j < 12; ++j)
+                        words[(i * 64 + r) * 12 + j] = Q[(size_t)n * W + 12 * (2 * c + i) + j];
+                for (int i = 0; i < 2 * nsb; ++i) {
+                    int g = 4 * c + i;
+                    groups[i * 128 + r] = scale[(size_t)g * N + n];
+                    groups[i * 128 + 64 + r] = zero[(size_t)g * N + n];
+                }
+            }
+            (void)G;
+        }
 }
 
 /* w_hat[n, k] = (q - z) * s in fp64. */

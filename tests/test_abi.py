@@ -47,12 +47,12 @@ def test_host_validation_rejects_before_launch(milo):
     L = milo.lib()
     fake = C.c_void_p(0x1000)
     # group != 64
-    assert L.milo_pack(fake, 16, 128, 32, fake, fake, fake, None, None) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    assert L.milo_pack(fake, 16, 128, 32, fake, None, None) == milo.MILO_ERR_UNSUPPORTED_SHAPE
     # K not a multiple of 128
-    assert L.milo_pack(fake, 16, 100, 64, fake, fake, fake, None, None) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    assert L.milo_pack(fake, 16, 100, 64, fake, None, None) == milo.MILO_ERR_UNSUPPORTED_SHAPE
     assert b"multiple of 128" in L.milo_last_error()
     # NULL pointers
-    assert L.milo_pack(None, 16, 128, 64, fake, fake, fake, None, None) == milo.MILO_ERR_INVALID_ARG
+    assert L.milo_pack(None, 16, 128, 64, fake, None, None) == milo.MILO_ERR_INVALID_ARG
     # router limits
     assert L.milo_route(fake, 4, 300, 2, 0, fake, fake, fake, fake, fake, None, None) == \
         milo.MILO_ERR_UNSUPPORTED_SHAPE
@@ -67,12 +67,12 @@ def test_prepare_validates_shapes_and_ranks(milo):
     nb = C.c_size_t()
     assert L.milo_table_bytes(3, C.byref(nb)) == 0 and nb.value % 64 == 0 and nb.value > 0
     fake = 0x10000
-    w = milo.milo_qweight(fake, fake, fake, None, None, 12)   # rank not a multiple of 8
+    w = milo.milo_qweight(fake, None, None, 12)   # rank not a multiple of 8
     lin = milo.milo_linear(64, 128, 1, 64, 0, None)
     assert L.milo_linear_prepare(C.byref(lin), C.byref(w), C.c_void_p(fake), 1 << 20) == \
         milo.MILO_ERR_UNSUPPORTED_SHAPE
     lin = milo.milo_linear(64, 200, 1, 64, 0, None)            # K % 128
-    w = milo.milo_qweight(fake, fake, fake, None, None, 0)
+    w = milo.milo_qweight(fake, None, None, 0)
     assert L.milo_linear_prepare(C.byref(lin), C.byref(w), C.c_void_p(fake), 1 << 20) == \
         milo.MILO_ERR_UNSUPPORTED_SHAPE
     lin = milo.milo_linear(64, 128, 1, 32, 0, None)            # group

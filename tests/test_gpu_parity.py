@@ -43,12 +43,10 @@ def _status(st):
 def test_pack_bit_exact(milo, N, K):
     W = wl.gen_weight(np.random.default_rng(N * 7 + K), N, K)
     st = milo.new_status()
-    Q, s, z = milo.milo_pack(f16_dev(W), dev_status=st)
+    blob = milo.milo_pack(f16_dev(W), dev_status=st)
     q_ref, s_ref, z_ref, st_ref = oracle.quantize(W)
     assert _status(st) == st_ref == 0
-    assert np.array_equal(Q.cpu().numpy().view(np.uint32), oracle.tile_words(oracle.pack(q_ref), K))
-    assert np.array_equal(s.cpu().numpy().view(np.uint16), oracle.tile_groups(s_ref))
-    assert np.array_equal(z.cpu().numpy().view(np.uint16), oracle.tile_groups(z_ref))
+    assert np.array_equal(blob.cpu().numpy(), oracle.tile_pack(oracle.pack(q_ref), s_ref, z_ref, K))
 
 
 def test_pack_degenerate_and_signed_zero_groups(milo):
@@ -58,11 +56,9 @@ def test_pack_degenerate_and_signed_zero_groups(milo):
     W[2] = np.linspace(-1e-7, 1e-7, 128)         # subnormal-range values
     W[3, :9] = [0, 7, 0.5, 1.5, 2.5, 3.5, 4.5, 5.5, 6.5]   # ties to even
     Wb = W.astype(np.float16).view(np.uint16)
-    Q, s, z = milo.milo_pack(f16_dev(Wb))
+    blob = milo.milo_pack(f16_dev(Wb))
     q_ref, s_ref, z_ref, _ = oracle.quantize(Wb)
-    assert np.array_equal(Q.cpu().numpy().view(np.uint32), oracle.tile_words(oracle.pack(q_ref), 128))
-    assert np.array_equal(s.cpu().numpy().view(np.uint16), oracle.tile_groups(s_ref))
-    assert np.array_equal(z.cpu().numpy().view(np.uint16), oracle.tile_groups(z_ref))
+    assert np.array_equal(blob.cpu().numpy(), oracle.tile_pack(oracle.pack(q_ref), s_ref, z_ref, 128))
 
 
 def test_pack_flags_nonfinite(milo):
@@ -76,8 +72,9 @@ def test_pack_flags_nonfinite(milo):
 @pytest.mark.parametrize("N,K", [(3, 128), (64, 1408), (5, 4096)])
 def test_unpack_bit_exact(milo, N, K):
     q = np.random.default_rng(N + K).integers(0, 8, (N, K), dtype=np.uint8)
-    Q = oracle.tile_words(oracle.pack(q), K)
-    codes = milo.milo_unpack(to_dev(Q.view(np.int32)), N, K)
+    G = K // 64
+    blob = oracle.tile_pack(oracle.pack(q), np.zeros((G, N), np.uint16), np.zeros((G, N), np.uint16), K)
+    codes = milo.milo_unpack(to_dev(blob), N, K)
     assert np.array_equal(codes.cpu().numpy(), q)
 
 

@@ -130,24 +130,34 @@ def test_unpack_roundtrip_exhaustive_one_hot_and_random():
     assert np.array_equal(oracle.unpack(oracle.pack(q), q.shape[1]), q)
 
 
-def test_device_tiling_matches_reshape():
-    """The device layout of the packed words and of the group arrays: 64-row
-    tiles, super-block (group) major inside a tile, zero rows padding the last
-    tile.  Checked against a numpy reshape/transpose of the padded arrays for
-    N that is and is not a multiple of 64."""
+def test_device_blob_matches_reshape():
+    """The device blob of a packed weight: 64-row tiles (zero rows pad the last),
+    K chunks of two super-blocks (one in the last chunk when K/128 is odd), each
+    (tile, chunk) block = the tile's words super-block major, then per group the
+    64 scales and the 64 zeros.  Checked against numpy reshapes/transposes of the
+    padded arrays, for N that is and is not a multiple of 64 and for even and odd
+    K/128."""
     rng = np.random.default_rng(11)
-    for N, K in ((64, 128), (100, 384), (16, 256), (130, 128)):
+    for N, K in ((64, 256), (100, 384), (16, 128), (130, 640)):
+        SB, G, NT = K // 128, K // 64, (N + 63) // 64
         Q = rng.integers(0, 2 ** 32, (N, 3 * K // 32), dtype=np.uint64).astype(np.uint32)
-        NT = (N + 63) // 64
-        pad = np.zeros((NT * 64, 3 * K // 32), np.uint32)
-        pad[:N] = Q
-        want = pad.reshape(NT, 64, K // 128, 12).transpose(0, 2, 1, 3)
-        assert np.array_equal(oracle.tile_words(Q, K), want)
-        A = rng.integers(0, 2 ** 16, (K // 64, N), dtype=np.uint32).astype(np.uint16)
-        padA = np.zeros((K // 64, NT * 64), np.uint16)
-        padA[:, :N] = A
-        wantA = padA.reshape(K // 64, NT, 64).transpose(1, 0, 2)
-        assert np.array_equal(oracle.tile_groups(A), wantA)
+        sc = rng.integers(0, 2 ** 16, (G, N), dtype=np.uint32).astype(np.uint16)
+        ze = rng.integers(0, 2 ** 16, (G, N), dtype=np.uint32).astype(np.uint16)
+        Qp = np.zeros((NT * 64, 3 * K // 32), np.uint32); Qp[:N] = Q
+        sp = np.zeros((G, NT * 64), np.uint16); sp[:, :N] = sc
+        zp = np.zeros((G, NT * 64), np.uint16); zp[:, :N] = ze
+        words = Qp.reshape(NT, 64, SB, 12).transpose(0, 2, 1, 3)          # [t][b][r][j]
+        groups = np.stack([sp.reshape(G, NT, 64), zp.reshape(G, NT, 64)], axis=2)   # [g][t][s|z][r]
+        groups = groups.transpose(1, 0, 2, 3)                                # [t][g][s|z][r]
+        parts = []
+        for t in range(NT):
+            for c in range(0, SB, 2):
+                nsb = min(2, SB - c)
+                parts.append(words[t, c:c + nsb].reshape(-1).view(np.uint8))
+                parts.append(groups[t, 2 * c:2 * c + 2 * nsb].reshape(-1).view(np.uint8))
+        want = np.concatenate(parts)
+        assert want.size == NT * SB * 3584
+        assert np.array_equal(oracle.tile_pack(Q, sc, ze, K), want)
 
 
 def test_unit_codes_share_one_group_per_pair():
