@@ -13,6 +13,7 @@
 #include <cuda_runtime.h>
 
 #include "milo_device.cuh"
+#include "milo_host.h"
 #include "milo_kernels.h"
 
 namespace milo {
@@ -88,6 +89,8 @@ __device__ __forceinline__ int row_source(const PrepParams& p, int row, int32_t&
 }
 
 __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
+    grid_dep_launch();
+    grid_dep_wait();
     const int row = blockIdx.x;
     const int SB = p.K / 128;
     int32_t st = 0;
@@ -158,8 +161,7 @@ cudaError_t launch_prep(const PrepParams& p, cudaStream_t s) {
     if (p.R <= 0) return cudaSuccess;
     // 32 super-blocks per block; enough blocks per row to fill the GPU at decode sizes
     const int chunks = (p.K / 128 * 4 + 127) / 128;
-    prep_kernel<<<dim3(p.R, chunks), 128, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(prep_kernel, dim3(p.R, chunks), dim3(128), 0, s, p);
 }
 
 // ---------------------------------------------------------------------------
@@ -182,6 +184,8 @@ constexpr int kLorcChunk = 256;             // K staged per step (per block)
 constexpr int kLorcPitch = kLorcChunk + 8;  // fp16; rows fall on different banks
 
 __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
+    grid_dep_launch();
+    grid_dep_wait();
     __shared__ __align__(16) uint16_t xs[16][kLorcPitch];
     __shared__ __align__(16) uint16_t vs[16][kLorcPitch];
     __shared__ float part[4][16][17];
@@ -288,6 +292,8 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
 }
 
 __global__ void __launch_bounds__(256) lorc_reduce_kernel(const LorcParams p) {
+    grid_dep_launch();
+    grid_dep_wait();
     const size_t n = static_cast<size_t>(p.R) * p.tcols;
     const size_t stride = n;
     for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
@@ -308,14 +314,13 @@ cudaError_t launch_lorc(const LorcParams& p, cudaStream_t s) {
     const int nproj = p.proj_b >= 0 ? 2 : 1;
     const long long blocks = static_cast<long long>(p.n_exp) * nproj * kLorcRankBlocks * p.splits;
     if (blocks <= 0 || p.R <= 0) return cudaSuccess;
-    lorc_partial_kernel<<<dim3(static_cast<unsigned>(blocks), p.row_groups), 128, 0, s>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(lorc_partial_kernel, dim3(static_cast<unsigned>(blocks), p.row_groups), dim3(128),
+                               0, s, p);
     if (e != cudaSuccess) return e;
     const long long n = static_cast<long long>(p.R) * p.tcols;
     long long rb = (n + 255) / 256;
     if (rb > 2048) rb = 2048;
-    lorc_reduce_kernel<<<static_cast<unsigned>(rb), 256, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(lorc_reduce_kernel, dim3(static_cast<unsigned>(rb)), dim3(256), 0, s, p);
 }
 
 // ---------------------------------------------------------------------------
@@ -333,6 +338,8 @@ __device__ __forceinline__ float4 row_sum(const float* part, int splits, size_t 
 }
 
 __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
+    grid_dep_launch();
+    grid_dep_wait();
     const int H4 = p.H / 4;
     const int rows_out = p.per_slot ? p.T * p.k : p.T;
     const long long total = static_cast<long long>(rows_out) * H4;
@@ -388,8 +395,7 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t s) {
     if (total <= 0) return cudaSuccess;
     long long blocks = (total + 255) / 256;
     if (blocks > 4096) blocks = 4096;
-    combine_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, p);
 }
 
 }  // namespace milo

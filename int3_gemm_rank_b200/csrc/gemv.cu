@@ -41,6 +41,7 @@
 #include <cuda_runtime.h>
 
 #include "milo_device.cuh"
+#include "milo_host.h"
 #include "milo_kernels.h"
 
 namespace milo {
@@ -246,12 +247,16 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tiles = (p.N + RA - 1) / RA;
 
+    grid_dep_launch();
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
         }
         fence_barrier_init();
+    }
+    grid_dep_wait();
+    if (threadIdx.x == 0) {
         int run = 0;
         for (int e = 0; e < p.n_exp; ++e) {
             const int r0 = p.grp[2 * e], m = p.grp[2 * e + 1];
@@ -434,9 +439,8 @@ cudaError_t launch_gemv(const GemvParams& p, bool glu, int grid, cudaStream_t s)
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) configured[dev][glu] = true;
     }
-    if (glu) gemv_kernel<true><<<grid, kGemvThreads, kSmemBytes, s>>>(p);
-    else gemv_kernel<false><<<grid, kGemvThreads, kSmemBytes, s>>>(p);
-    return cudaGetLastError();
+    if (glu) return launch_pdl(gemv_kernel<true>, dim3(grid), dim3(kGemvThreads), kSmemBytes, s, p);
+    return launch_pdl(gemv_kernel<false>, dim3(grid), dim3(kGemvThreads), kSmemBytes, s, p);
 }
 
 }  // namespace milo

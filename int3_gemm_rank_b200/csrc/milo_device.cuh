@@ -23,6 +23,20 @@ __device__ __forceinline__ void flag(int32_t* st, int32_t bits) {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch
+// ---------------------------------------------------------------------------
+
+// The kernels of a forward are launched with programmatic stream
+// serialization: a kernel may be scheduled while the previous one drains.
+// grid_dep_wait() returns once the grids it depends on have completed and
+// their writes are visible (at once for a normal launch); every kernel calls
+// it before touching what earlier kernels wrote, so completion stays
+// transitive along the stream.  grid_dep_launch() lets the next kernel start
+// launching.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // conversions
 // ---------------------------------------------------------------------------
 

@@ -29,6 +29,8 @@ route_kernel(const uint16_t* __restrict__ logits, int T, int E, int k, uint32_t 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int F = T * k;
     int32_t st = 0;
+    grid_dep_launch();
+    grid_dep_wait();
 
     // -- top-k per token: insertion into a list kept in descending logit order;
     //    a strictly larger logit is needed to pass an entry, so equal logits
@@ -146,7 +148,8 @@ extern "C" milo_status milo_route(const uint16_t* logits, int32_t T, int32_t E, 
         return fail(MILO_ERR_INVALID_ARG, "milo_route: logits and topk_w are required");
     if (static_cast<long long>(T) * k > 0x3FFFFFFFLL)
         return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_route: T*k too large");
-    route_kernel<<<1, kRouteThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        logits, T, E, k, flags, topk_ids, topk_w, expert_offsets, perm, inv_perm, dev_status);
-    return check_launch("milo_route");
+    return check_cuda(launch_pdl(route_kernel, dim3(1), dim3(kRouteThreads), 0, static_cast<cudaStream_t>(stream),
+                                 logits, T, E, k, flags, topk_ids, topk_w, expert_offsets, perm, inv_perm,
+                                 dev_status),
+                      "milo_route");
 }
