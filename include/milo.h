@@ -98,8 +98,8 @@ MILO_API int32_t milo_version(void);
  * chunk holds one when K/128 is odd).  The (tile t, chunk c) block starts at
  * byte (t * K/128 + 2c) * 3584 and holds, for its nsb super-blocks b,
  *     the words u32 [64 rows][12]      (word j of row 64t+r = word 12b+j above)
- * then, for its 2*nsb groups g,
- *     s fp16 [64 rows], z fp16 [64 rows]
+ * then, for its 2*nsb groups g, 256 bytes: for each 16-row block m (0..3)
+ * and j (0..7) the fp16 quadruple s, z of row 16m+j, s, z of row 16m+j+8
  * so that the kernels fetch a tile's chunk -- codes, scales and zeros -- with
  * one copy.  Dequantisation: w_hat[n, k] = (q[n, k] - z[n, k/64]) * s[n, k/64].
  * The blob has ceil(N/64) * (K/128) * 3584 bytes (milo_packed_bytes).

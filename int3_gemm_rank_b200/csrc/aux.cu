@@ -1,5 +1,5 @@
 // aux.cu -- the kernels around the grouped int3 GEMM:
-//   prep_kernel    activations -> fp16 MMA fragments (power-of-8 factors of the
+//   prep_kernel    activations -> fp16 MMA fragments (power-of-2 factors of the
 //                  int3 field extraction folded in) and per-group sums; the
 //                  first one of a call also does the row bookkeeping (expert
 //                  groups, row -> token) from the router's offsets and perm
@@ -25,7 +25,7 @@ template <int S, int H>
 __device__ __forceinline__ uint32_t frag_pair(const __half (&x)[32]) {
     constexpr int t = sched_word(S, H), f = sched_field(S, H);
     constexpr int m = reg_code(t, f);
-    const __half sc = __float2half_rn(act_scale(f));
+    const __half sc = __float2half_rn(act_scale(t, f));
     const __half lo = __hmul(x[m], sc), hi = __hmul(x[m + 1], sc);
     return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
 }

@@ -22,8 +22,8 @@
 //     tile, with an evict-first L2 policy.
 //   - Four consumer warps each own 32 weight rows.  A lane reads its 3-word
 //     unit of two rows and extracts code pairs with one LOP3 each (plus one
-//     shift per word): the masked fp16 pattern already is code * 8^i * 2^-24,
-//     and the power of 8 is folded into the activations, which are shared by
+//     shift per word): the masked fp16 pattern already is code * 2^e * 2^-24,
+//     and the power of 2 is folded into the activations, which are shared by
 //     all rows.  mma.sync m16n8k16 (A = codes, B = tokens) accumulates
 //     D_g = 2^-24 * sum_k x_k q_k per scale group g; after each group the lane
 //     folds  acc += s * 2^24 * D_g - s * z * sum_k x_k  in fp32.  The zero point
@@ -134,28 +134,23 @@ struct TileMap {
 };
 
 // acc += s * 2^24 * D_g - s * z * X_g for group `grp` (0..3) of the chunk;
-// the scales of the chunk's groups start nsb * 3072 bytes into each region.
+// the scales of the chunk's groups start nsb * 3072 bytes into each region,
+// as (s, z) pairs of rows j and j + 8 of each 16-row block, so one 64-bit
+// load brings the lane's two rows.  xg[n8][j]: X_g of its tokens.
 template <int NT>
 __device__ __forceinline__ void fold_group(float (&acc)[2][2][4], const float (&dz)[2][2][4],
                                            const uint8_t* st, int grp, const int (&reg)[2],
-                                           const int (&rbase)[2], int nsb, int g, int c) {
-    float xg[NT][2];
-#pragma unroll
-    for (int n8 = 0; n8 < NT; ++n8)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int tok = n8 * 8 + 2 * c + j;
-            xg[n8][j] = reinterpret_cast<const float*>(st + kOffX + (tok * kFragRowHalves + kGsumHalf) * 2)[grp];
-        }
+                                           const int (&rbase)[2], int nsb, int g, const float (&xg)[NT][2]) {
 #pragma unroll
     for (int ti = 0; ti < 2; ++ti) {
-        const __half* S = reinterpret_cast<const __half*>(st + reg[ti] + nsb * kQTileSBWords * 4 + grp * kGroupBytes);
+        const uint2 q = *reinterpret_cast<const uint2*>(st + reg[ti] + nsb * kQTileSBWords * 4 + grp * kGroupBytes +
+                                                        ((rbase[ti] >> 4) * 8 + g) * 8);
         float s24[2], nsz[2];
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
-            const int row = rbase[ti] + g + 8 * rr;
-            const float sv = __half2float(S[row]);
-            const float zv = __half2float(S[kTileRows + row]);
+            const uint32_t v = rr ? q.y : q.x;
+            const float sv = __half2float(__ushort_as_half(static_cast<uint16_t>(v & 0xFFFFu)));
+            const float zv = __half2float(__ushort_as_half(static_cast<uint16_t>(v >> 16)));
             s24[rr] = sv * 16777216.0f;
             nsz[rr] = -sv * zv;
         }
@@ -186,21 +181,33 @@ __device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2]
 #pragma unroll
                 for (int t = 0; t < 3; ++t) {
                     wd[ti][rr][t] = qt[(tm.r[ti] + g + 8 * rr) * 12 + 3 * c + t];
-                    hw[ti][rr][t] = wd[ti][rr][t] >> 9;
+                    hw[ti][rr][t] = wd[ti][rr][t] >> word_shift(t);
                 }
         }
         const uint8_t* xs = st + kOffX + sbl * kFragHalvesPerSB * 2;
+        // group sums of this super-block's two groups for the lane's tokens
+        float xa[NT][2], xb[NT][2];
+#pragma unroll
+        for (int n8 = 0; n8 < NT; ++n8)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int tok = n8 * 8 + 2 * c + j;
+                const float2 v = *reinterpret_cast<const float2*>(
+                    st + kOffX + (tok * kFragRowHalves + kGsumHalf) * 2 + sbl * 8);
+                xa[n8][j] = v.x;
+                xb[n8][j] = v.y;
+            }
         float dz[2][2][4];
         code_step<0, NT>(wd, hw, xs, g, c, dz);
         code_step<1, NT>(wd, hw, xs, g, c, dz);
         code_step<2, NT>(wd, hw, xs, g, c, dz);
         code_step<3, NT>(wd, hw, xs, g, c, dz);
-        fold_group<NT>(acc, dz, st, 2 * sbl, tm.reg, tm.r, nsb, g, c);
+        fold_group<NT>(acc, dz, st, 2 * sbl, tm.reg, tm.r, nsb, g, xa);
         code_step<4, NT>(wd, hw, xs, g, c, dz);
         code_step<5, NT>(wd, hw, xs, g, c, dz);
         code_step<6, NT>(wd, hw, xs, g, c, dz);
         code_step<7, NT>(wd, hw, xs, g, c, dz);
-        fold_group<NT>(acc, dz, st, 2 * sbl + 1, tm.reg, tm.r, nsb, g, c);
+        fold_group<NT>(acc, dz, st, 2 * sbl + 1, tm.reg, tm.r, nsb, g, xb);
     }
 }
 
@@ -247,7 +254,6 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tiles = (p.N + RA - 1) / RA;
 
-    grid_dep_launch();
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
@@ -439,8 +445,13 @@ cudaError_t launch_gemv(const GemvParams& p, bool glu, int grid, cudaStream_t s)
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) configured[dev][glu] = true;
     }
-    if (glu) return launch_pdl(gemv_kernel<true>, dim3(grid), dim3(kGemvThreads), kSmemBytes, s, p);
-    return launch_pdl(gemv_kernel<false>, dim3(grid), dim3(kGemvThreads), kSmemBytes, s, p);
+    // A normal launch: the persistent grid starts once the previous kernel has
+    // left every SM, so its CTAs are spread evenly over the SMs (an early,
+    // programmatic launch places them wherever resources free up first, and
+    // the per-SM load of the static item split then goes uneven).
+    if (glu) gemv_kernel<true><<<grid, kGemvThreads, kSmemBytes, s>>>(p);
+    else gemv_kernel<false><<<grid, kGemvThreads, kSmemBytes, s>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace milo

@@ -63,27 +63,33 @@ __device__ __forceinline__ __half to_half(uint16_t bits, bool is_bf16, int32_t& 
 // Masking a field that lies in bits 0..8 of a half leaves an fp16 whose value
 // is code * 8^i * 2^-24 (fields 0, 1, 2: the pattern is an integer below 2^11,
 // and fp16 patterns below 2^11 are that integer times 2^-24).  Fields 3 and 4
-// and the spare bit are brought down by one shift of 9.  So each pair of codes
-// costs one LOP3 (plus one shared shift per word) and the power-of-8 factor is
-// undone on the activation side, where it costs nothing per weight.  The six
-// spare bits of a unit (bit t of u_30 in bit 15 of word t, bit t of u_31 in
-// bit 31) are gathered into bits 6..8 / 22..24 of one more register, i.e.
-// u_30 * 64 and u_31 * 64 in the fp16 halves.
+// and the spare bit of word t are brought down by one shift of 9 - t, so they
+// land t bits higher than fields 0 and 1 do.  Each pair of codes costs one
+// LOP3 (plus one shift per word) and the power-of-2 factor left in the value
+// is undone on the activation side, where it costs nothing per weight.  The
+// six spare bits of a unit (bit t of u_30 in bit 15 of word t, bit t of u_31
+// in bit 31) arrive at bits 6 + t / 22 + t of the shifted words, so three
+// LOP3s gather them into one more register: u_30 * 64 and u_31 * 64 in the
+// fp16 halves.
 constexpr uint32_t kField0 = 0x00070007u;   // bits 0-2   -> code * 1
 constexpr uint32_t kField1 = 0x00380038u;   // bits 3-5   -> code * 8
 constexpr uint32_t kField2 = 0x01C001C0u;   // bits 6-8   -> code * 64
 constexpr uint32_t kSpare = 0x00400040u;    // bit 15 >> 9 -> bit 6 (bit 31 >> 9 -> bit 22)
 
-// Register f (0..5) of a unit; w[] are its three words, hw[] the words >> 9.
-// Fields 0..4 come from word t; register 5 gathers the spare bits.
+// Shift that brings fields 3, 4 and the spare bit of word t down.
+__host__ __device__ constexpr int word_shift(int t) { return 9 - t; }
+
+// Register f (0..5) of a unit; w[] are its three words, hw[t] = w[t] >>
+// word_shift(t).  Fields 0..4 come from word t; register 5 gathers the spare
+// bits.
 template <int T, int F>
 __device__ __forceinline__ uint32_t unit_reg(const uint32_t (&w)[3], const uint32_t (&hw)[3]) {
     if constexpr (F == 0) return w[T] & kField0;
     else if constexpr (F == 1) return w[T] & kField1;
     else if constexpr (F == 2) return w[T] & kField2;
-    else if constexpr (F == 3) return hw[T] & kField0;
-    else if constexpr (F == 4) return hw[T] & kField1;
-    else return (hw[0] & kSpare) + (hw[1] & kSpare) * 2u + (hw[2] & kSpare) * 4u;
+    else if constexpr (F == 3) return hw[T] & (kField0 << T);
+    else if constexpr (F == 4) return hw[T] & (kField1 << T);
+    else return (hw[0] & kSpare) | (hw[1] & (kSpare << 1)) | (hw[2] & (kSpare << 2));
 }
 
 // Register schedule of one 3-word unit over the eight k16 MMA steps of a
@@ -107,13 +113,13 @@ __host__ __device__ constexpr int reg_code(int t, int f) { return f < 5 ? 10 * t
 __host__ __device__ constexpr int unit_k(int c, int m) {
     return m < 16 ? 16 * c + m : 64 + 16 * c + (m - 16);
 }
-// Power of 8 left in the extracted value of field f, and its inverse, which
-// multiplies the activation paired with it.
-__host__ __device__ constexpr int field_shift(int f) {
-    return f == 0 || f == 3 ? 0 : f == 1 || f == 4 ? 3 : 6;
+// Power of 2 left in the extracted value of register (word t, field f), and
+// its inverse, which multiplies the activation paired with it.
+__host__ __device__ constexpr int field_shift(int t, int f) {
+    return f == 0 ? 0 : f == 1 ? 3 : f == 2 ? 6 : f == 3 ? t : f == 4 ? 3 + t : 6;
 }
-__host__ __device__ constexpr float act_scale(int f) {
-    return f == 0 || f == 3 ? 1.0f : f == 1 || f == 4 ? 0.125f : 0.015625f;
+__host__ __device__ constexpr float act_scale(int t, int f) {
+    return 1.0f / static_cast<float>(1 << field_shift(t, f));
 }
 
 // ---------------------------------------------------------------------------

@@ -14,16 +14,18 @@
 namespace milo {
 
 // Device blob (milo.h): 64-row tiles, K chunks of two super-blocks, each
-// (tile, chunk) block = the words of its super-blocks, then per group the 64
-// scales and the 64 zeros.  Byte offsets of row n's words for super-block b
-// and of its scale for group j (its zero follows 128 bytes later).
+// (tile, chunk) block = the words of its super-blocks, then per group the
+// scales and zeros as (s, z) pairs of rows r and r + 8 of each 16-row block.
+// Byte offsets of row n's words for super-block b and of its scale for group
+// j (its zero follows 2 bytes later).
 __device__ __forceinline__ size_t blob_words(int n, int b, int SB) {
     const int c = b >> 1;
     return (static_cast<size_t>(n / 64) * SB + 2 * c) * kBlockSB + ((b & 1) * 64 + (n % 64)) * 48;
 }
 __device__ __forceinline__ size_t blob_group(int n, int j, int SB) {
-    const int c = j >> 2, nsb = min(2, SB - 2 * c);
-    return (static_cast<size_t>(n / 64) * SB + 2 * c) * kBlockSB + nsb * 3072 + (j & 3) * 256 + (n % 64) * 2;
+    const int c = j >> 2, nsb = min(2, SB - 2 * c), r = n % 64;
+    return (static_cast<size_t>(n / 64) * SB + 2 * c) * kBlockSB + nsb * 3072 + (j & 3) * kGroupBytes +
+           (((r >> 4) * 8 + (r & 7)) * 4 + ((r >> 3) & 1) * 2) * 2;
 }
 
 // One thread per (row, 128-code super-block): two scale groups.  Rows N..
@@ -44,7 +46,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
         for (int g = 0; g < 2; ++g) {
             const size_t o = blob_group(n, 2 * b + g, SB) / 2;
             sz[o] = 0;
-            sz[o + 64] = 0;
+            sz[o + 1] = 0;
         }
         return;
     }
@@ -70,7 +72,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
         if (!isfinite(s) || !isfinite(z)) st |= MILO_DEV_FP16_RANGE;
         const size_t o = blob_group(n, 2 * b + g, SB) / 2;
         sz[o] = __half_as_ushort(sh);
-        sz[o + 64] = __half_as_ushort(zh);
+        sz[o + 1] = __half_as_ushort(zh);
         for (int i = 0; i < 64; ++i) {
             const float v = __fadd_rn(__fdiv_rn(__half2float(__ushort_as_half(w[64 * g + i])), s), z);
             float r = rintf(v);
@@ -105,14 +107,14 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
 }
 
 // One thread per (row, super-block, unit): recover the 32 codes of a unit with
-// the register-level extraction of the GEMM (field masks, one shift by 9, the
-// gathered spare register, the eight-step schedule), so that its bit-exact
+// the register-level extraction of the GEMM (field masks, one shift per word,
+// the gathered spare register, the eight-step schedule), so that its bit-exact
 // parity covers that logic.
 template <int S, int H>
 __device__ __forceinline__ void unpack_reg(const uint32_t (&w)[3], const uint32_t (&hw)[3],
                                            uint8_t (&u)[32]) {
     constexpr int t = sched_word(S, H), f = sched_field(S, H);
-    constexpr int m = reg_code(t, f), sh = field_shift(f);
+    constexpr int m = reg_code(t, f), sh = field_shift(t, f);
     const uint32_t r = unit_reg<t, f>(w, hw);
     u[m] = static_cast<uint8_t>((r & 0xFFFFu) >> sh);
     u[m + 1] = static_cast<uint8_t>((r >> 16) >> sh);
@@ -135,7 +137,7 @@ __global__ void __launch_bounds__(128) unpack_kernel(const uint8_t* __restrict__
     const int n = static_cast<int>(nb / SB), b = static_cast<int>(nb % SB);
     const uint32_t* src = reinterpret_cast<const uint32_t*>(blob + blob_words(n, b, SB)) + 3 * c;
     const uint32_t w[3] = {src[0], src[1], src[2]};
-    const uint32_t hw[3] = {w[0] >> 9, w[1] >> 9, w[2] >> 9};
+    const uint32_t hw[3] = {w[0] >> word_shift(0), w[1] >> word_shift(1), w[2] >> word_shift(2)};
     uint8_t u[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) u[i] = 0xFF;   // a code the schedule misses stays 0xFF

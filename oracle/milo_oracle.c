@@ -221,7 +221,9 @@ void milo_ref_unpack(const uint32_t* Q, int N, int K, uint8_t* q) {
  * contiguous, so the GPU kernels fetch it with a single copy:
  *     block(t, c) at byte (t * SB + 2 * c) * 3584, holding for its nsb
  *     super-blocks b (in order) the words  [64 rows][12]        (nsb * 3072 B)
- *     then for its 2 * nsb groups g (in order)  [64 s fp16][64 z fp16]  (256 B each)
+ *     then for its 2 * nsb groups g (in order) 256 bytes: for each 16-row
+ *     block m (0..3) and j (0..7) the fp16 quadruple
+ *         s[16m + j], z[16m + j], s[16m + j + 8], z[16m + j + 8]
  * Word j of row n, super-block b, is Q[n, 12 b + j]; s and z of row n, group
  * g are scale[g, n] and zero[g, n].  This is a relayout only, used to compare
  * with the device packer.
@@ -244,8 +246,9 @@ void milo_ref_tile_pack(const uint32_t* Q, const uint16_t* scale, const uint16_t
                         words[(i * 64 + r) * 12 + j] = Q[(size_t)n * W + 12 * (2 * c + i) + j];
                 for (int i = 0; i < 2 * nsb; ++i) {
                     int g = 4 * c + i;
-                    groups[i * 128 + r] = scale[(size_t)g * N + n];
-                    groups[i * 128 + 64 + r] = zero[(size_t)g * N + n];
+                    int q = i * 128 + ((r / 16) * 8 + r % 8) * 4 + ((r % 16) / 8) * 2;
+                    groups[q] = scale[(size_t)g * N + n];
+                    groups[q + 1] = zero[(size_t)g * N + n];
                 }
             }
             (void)G;

@@ -134,7 +134,8 @@ def test_device_blob_matches_reshape():
     """The device blob of a packed weight: 64-row tiles (zero rows pad the last),
     K chunks of two super-blocks (one in the last chunk when K/128 is odd), each
     (tile, chunk) block = the tile's words super-block major, then per group the
-    64 scales and the 64 zeros.  Checked against numpy reshapes/transposes of the
+    scales and zeros, interleaved as (s, z) of rows j and j + 8 of each 16-row
+    block.  Checked against numpy reshapes/transposes of the
     padded arrays, for N that is and is not a multiple of 64 and for even and odd
     K/128."""
     rng = np.random.default_rng(11)
@@ -147,8 +148,9 @@ def test_device_blob_matches_reshape():
         sp = np.zeros((G, NT * 64), np.uint16); sp[:, :N] = sc
         zp = np.zeros((G, NT * 64), np.uint16); zp[:, :N] = ze
         words = Qp.reshape(NT, 64, SB, 12).transpose(0, 2, 1, 3)          # [t][b][r][j]
-        groups = np.stack([sp.reshape(G, NT, 64), zp.reshape(G, NT, 64)], axis=2)   # [g][t][s|z][r]
-        groups = groups.transpose(1, 0, 2, 3)                                # [t][g][s|z][r]
+        # [g][t][m][hi][j][s|z] with row r = 16m + 8hi + j, stored as [t][g][m][j][hi][s|z]
+        groups = np.stack([sp.reshape(G, NT, 4, 2, 8), zp.reshape(G, NT, 4, 2, 8)], axis=-1)
+        groups = groups.transpose(1, 0, 2, 4, 3, 5)
         parts = []
         for t in range(NT):
             for c in range(0, SB, 2):
