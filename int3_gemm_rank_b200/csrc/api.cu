@@ -126,19 +126,18 @@ static int choose_splits(long long base_items, int chunks) {
     return best;
 }
 
-// K slices and row-tile groups of the compensator down-projection: enough
-// blocks to fill the GPU (about four per SM), K slices dividing K/128.
-static LorcPlan lorc_plan(int n_exp, int nproj, int K, long long rows_per_exp) {
-    const long long target = 8LL * sm_count();
+// K slices and row-tile groups of the compensator down-projection.  A block
+// handles one 16-row tile of one expert for one K slice, so its latency is a
+// couple of staging rounds: slices of about four super-blocks (the last one
+// may be shorter) while the row tiles alone do not fill the GPU, and enough
+// row groups for the largest possible group (max_rows), capped in blocks.
+static LorcPlan lorc_plan(int n_exp, int nproj, int K, long long max_rows) {
     const long long base = static_cast<long long>(n_exp) * nproj * ((MILO_MAX_RANK + 15) / 16);
     const int sb = K / 128;
-    const long long tiles = std::max(1LL, (rows_per_exp + 15) / 16);
+    const long long tiles = std::max(1LL, (max_rows + 15) / 16);
     LorcPlan pl{1, 1};
-    pl.row_groups = static_cast<int>(std::min<long long>(tiles, std::max(1LL, target / std::max(1LL, base))));
-    // K slices only while the row tiles do not fill the GPU (they cost partial sums)
-    const long long want = tiles > 4 ? 1 : std::max(1LL, target / std::max(1LL, base * pl.row_groups));
-    for (int d = 1; d <= sb; ++d)
-        if (sb % d == 0 && d <= want) pl.splits = d;
+    pl.splits = tiles >= 8 ? 1 : std::max(1, (sb + 3) / 4);
+    pl.row_groups = static_cast<int>(std::min<long long>(tiles, std::max(1LL, 65536 / (base * pl.splits))));
     return pl;
 }
 
@@ -157,7 +156,7 @@ static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
     w.inv = c.take(static_cast<size_t>(w.R) * 4);
     w.frag = c.take(frag_bytes(lin->K, w.R));
     w.t = c.take(static_cast<size_t>(w.R) * w.tcols * 2);
-    w.lp = lorc_plan(n_exp, 1, lin->K, std::max(1LL, static_cast<long long>(w.R) / std::max<long long>(1, groups)));
+    w.lp = lorc_plan(n_exp, 1, lin->K, static_cast<long long>(T) * k);   // at most all rows in one expert
     w.tpart = c.take(static_cast<size_t>(w.lp.splits) * w.R * w.tcols * 4);
     w.part = c.take(static_cast<size_t>(w.splits) * w.R * lin->N * 4);
     w.total = c.off;
@@ -189,9 +188,9 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
     w.h = c.take(static_cast<size_t>(w.R) * I * 2);
     w.hfrag = c.take(frag_bytes(I, w.R));
     w.t2 = c.take(static_cast<size_t>(w.R) * w.tc2 * 2);
-    const long long rows_per_exp = std::max(1LL, static_cast<long long>(w.R) / std::max<long long>(1, groups));
-    w.lp13 = lorc_plan(n_exp, 2, H, rows_per_exp);
-    w.lp2 = lorc_plan(n_exp, 1, I, rows_per_exp);
+    // a token meets an expert at most once, and a shared expert sees every token
+    w.lp13 = lorc_plan(n_exp, 2, H, T);
+    w.lp2 = lorc_plan(n_exp, 1, I, T);
     w.tpart = c.take(std::max(static_cast<size_t>(w.lp13.splits) * w.tc13,
                               static_cast<size_t>(w.lp2.splits) * w.tc2) * w.R * 4);
     w.part = c.take(static_cast<size_t>(w.splits) * w.R * H * 4);

@@ -209,8 +209,10 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
     if (m <= 0 || row0 < 0 || row0 + m > p.R) return;
     const int col0 = which == 0 ? 0 : p.t_col_b;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-    const int slice = p.K / p.splits;                 // a multiple of 128
-    const int kbeg = split * slice;
+    // K slice of this block: whole super-blocks, the last slice may be shorter
+    const int slice_sb = (p.K / 128 + p.splits - 1) / p.splits;
+    const int kbeg = min(p.K, split * slice_sb * 128);
+    const int kend = min(p.K, kbeg + slice_sb * 128);
     float* out = p.part + static_cast<size_t>(split) * p.R * p.tcols;
     int32_t st = 0;
     if (j0 >= r) {   // ranks of this block are all past r: zeros only
@@ -229,9 +231,9 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
             src_row[i] = mt + i < m ? (p.row_src ? p.row_src[row0 + mt + i] : row0 + mt + i) : -1;
         }
         float acc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
-        for (int kc = kbeg; kc < kbeg + slice; kc += kLorcChunk) {
-            // this chunk: 256 or, at the end of a slice, 128 (slices are multiples of 128)
-            const int cs = min(kLorcChunk, kbeg + slice - kc);
+        for (int kc = kbeg; kc < kend; kc += kLorcChunk) {
+            // this chunk: 256 or, at the end of a slice, 128 (slices are whole super-blocks)
+            const int cs = min(kLorcChunk, kend - kc);
             const int kw = cs / 4;                    // K per warp: 32 or 64
             __syncthreads();
             // stage x rows and V rows [16][cs] with 16-byte loads
@@ -337,7 +339,7 @@ __device__ __forceinline__ float4 row_sum(const float* part, int splits, size_t 
     return a;
 }
 
-__global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
+__global__ void __launch_bounds__(64) combine_kernel(const CombineParams p) {
     grid_dep_launch();
     grid_dep_wait();
     const int H4 = p.H / 4;
@@ -393,9 +395,11 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t s) {
     const long long rows_out = p.per_slot ? static_cast<long long>(p.T) * p.k : p.T;
     const long long total = rows_out * (p.H / 4);
     if (total <= 0) return cudaSuccess;
-    long long blocks = (total + 255) / 256;
-    if (blocks > 4096) blocks = 4096;
-    return launch_pdl(combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, p);
+    // small blocks: at decode sizes the outputs are few, and spreading them
+    // over more SMs hides the dependent loads (inv_perm, then the partials)
+    long long blocks = (total + 63) / 64;
+    if (blocks > 8192) blocks = 8192;
+    return launch_pdl(combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(64), 0, s, p);
 }
 
 }  // namespace milo

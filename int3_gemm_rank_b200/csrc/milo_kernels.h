@@ -84,7 +84,7 @@ struct LorcParams {
     int32_t* dev_status;
     int stride, proj_a, proj_b; // proj_b < 0: single projection
     int n_exp, K, R, tcols, t_col_b, src_bf16;
-    int splits, row_groups;     // K slices (each a multiple of 128); row-tile strides
+    int splits, row_groups;     // K slices of ceil(K/128 / splits) super-blocks; row-tile strides
 };
 
 struct CombineParams {

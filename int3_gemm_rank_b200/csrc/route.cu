@@ -32,39 +32,67 @@ route_kernel(const uint16_t* __restrict__ logits, int T, int E, int k, uint32_t 
     grid_dep_launch();
     grid_dep_wait();
 
-    // -- top-k per token: insertion into a list kept in descending logit order;
-    //    a strictly larger logit is needed to pass an entry, so equal logits
-    //    keep ascending expert order.
+    // -- top-k per token, one warp per token: the lanes hold the token's
+    //    logits (expert e at lane e % 32, slot e / 32) and k rounds of a warp
+    //    arg-max pick the largest remaining logit, ties to the lower expert id
+    //    (a key orders by value, then by descending id).  NaN counts as -inf
+    //    (and is flagged).  Slot j = j-th pick.
     if (!(flags & MILO_ROUTE_IDS_GIVEN)) {
-        for (int t = tid; t < T; t += kRouteThreads) {
+        constexpr int kSlots = (MILO_MAX_EXPERTS + 31) / 32;
+        for (int t = warp; t < T; t += kRouteWarps) {
             const uint16_t* l = logits + static_cast<size_t>(t) * E;
-            float lv[MILO_MAX_TOPK];
-            int le[MILO_MAX_TOPK];
-            int n = 0;
-            for (int e = 0; e < E; ++e) {
-                const float v = __half2float(__ushort_as_half(l[e]));
-                if (!isfinite(v)) st |= MILO_DEV_NONFINITE;
-                if (n == k && !(v > lv[k - 1])) continue;
-                int pos = n < k ? n : k - 1;
-                while (pos > 0 && v > lv[pos - 1]) {
-                    lv[pos] = lv[pos - 1];
-                    le[pos] = le[pos - 1];
-                    --pos;
+            float v[kSlots];
+            unsigned long long key[kSlots];
+#pragma unroll
+            for (int i = 0; i < kSlots; ++i) {
+                const int e = 32 * i + lane;
+                v[i] = -INFINITY;
+                key[i] = 0ull;   // below every real key: empty or already picked
+                if (e < E) {
+                    float x = __half2float(__ushort_as_half(l[e]));
+                    if (!isfinite(x)) st |= MILO_DEV_NONFINITE;
+                    if (x != x) x = -INFINITY;
+                    v[i] = x;
+                    const uint32_t b = __float_as_uint(x);
+                    const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+                    key[i] = (static_cast<unsigned long long>(ord) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e));
                 }
-                lv[pos] = v;
-                le[pos] = e;
-                if (n < k) ++n;
             }
-            const float m = lv[0];
-            float den = 0.0f;
-            if (flags & MILO_ROUTE_RENORM) {
-                for (int j = 0; j < k; ++j) den += expf(lv[j] - m);
-            } else {
-                for (int e = 0; e < E; ++e) den += expf(__half2float(__ushort_as_half(l[e])) - m);
-            }
+            // lane j keeps pick j (k <= 16 < 32); the renormalising sum runs in slot order
+            int my_e = 0;
+            float my_v = 0.0f, m = 0.0f, den = 0.0f;
             for (int j = 0; j < k; ++j) {
-                ids[static_cast<size_t>(t) * k + j] = le[j];
-                wts[static_cast<size_t>(t) * k + j] = expf(lv[j] - m) / den;
+                unsigned long long best = 0ull;
+#pragma unroll
+                for (int i = 0; i < kSlots; ++i) best = key[i] > best ? key[i] : best;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+                    best = other > best ? other : best;
+                }
+                const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best & 0xFFFFFFFFull));
+                const uint32_t ord = static_cast<uint32_t>(best >> 32);
+                const float val = __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
+                if (j == 0) m = val;
+                if (flags & MILO_ROUTE_RENORM) den += expf(val - m);
+                if (lane == j) {
+                    my_e = e;
+                    my_v = val;
+                }
+#pragma unroll
+                for (int i = 0; i < kSlots; ++i)
+                    if (32 * i + lane == e) key[i] = 0ull;
+            }
+            if (!(flags & MILO_ROUTE_RENORM)) {
+#pragma unroll
+                for (int i = 0; i < kSlots; ++i)
+                    if (32 * i + lane < E) den += expf(v[i] - m);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xFFFFFFFFu, den, o);
+            }
+            if (lane < k) {
+                ids[static_cast<size_t>(t) * k + lane] = my_e;
+                wts[static_cast<size_t>(t) * k + lane] = expf(my_v - m) / den;
             }
         }
     }
