@@ -123,7 +123,9 @@ static int choose_splits(long long base_items, int chunks) {
         eff -= 0.004 * (s - 1);                           // partial-sum traffic
         if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
     }
-    return best;
+    // with ceil(chunks / best) chunks per split, every split must get one
+    const int cps = (chunks + best - 1) / best;
+    return (chunks + cps - 1) / cps;
 }
 
 // K slices and row-tile groups of the compensator down-projection.  A block

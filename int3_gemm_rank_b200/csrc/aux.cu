@@ -12,6 +12,8 @@
 // GEMM and (x V^T) U^T; the MoE layer combines the routed experts' outputs.
 #include <cuda_runtime.h>
 
+#include <climits>
+
 #include "milo_device.cuh"
 #include "milo_host.h"
 #include "milo_kernels.h"
@@ -38,31 +40,46 @@ __device__ __forceinline__ uint2 frag_step(const __half (&x)[32]) {
 // Expert groups (first row, count), clamped into a non-decreasing sequence
 // within [0, T*k]; shared experts follow the routed rows.  Block (0, 0) only.
 __device__ void build_groups(const PrepParams& p, int32_t& st) {
+    // ok_off[e] = max(ok_off[e-1], min(offsets[e], F)), ok_off[0] = 0: a
+    // running maximum, so warp 0 scans it 32 experts at a time after all
+    // threads have loaded the offsets.
     __shared__ int ok_off[MILO_MAX_EXPERTS + 1];
     const int F = p.T * p.k;
-    if (threadIdx.x == 0) {
-        int prev = 0;
-        for (int e = 0; e <= p.E; ++e) {
-            int o = p.offsets[e];
-            if (e == 0 && o != 0) st |= MILO_DEV_BAD_EXPERT_ID;
-            if (o < prev || o > F) {
-                st |= MILO_DEV_BAD_EXPERT_ID;
-                o = o < prev ? prev : F;
+    const int lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e <= p.E; e += blockDim.x) ok_off[e] = p.offsets[e];
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        int run = 0;
+        for (int base = 0; base <= p.E; base += 32) {
+            const int e = base + lane;
+            const int o = e <= p.E ? ok_off[e] : 0;
+            int incl = e == 0 ? 0 : (e <= p.E ? min(o, F) : INT_MIN);
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+                if (lane >= d) incl = max(incl, y);
             }
-            ok_off[e] = e == 0 ? 0 : o;
-            prev = ok_off[e];
-        }
-        for (int e = 0; e < p.E; ++e) {
-            p.grp[2 * e] = ok_off[e];
-            p.grp[2 * e + 1] = ok_off[e + 1] - ok_off[e];
-        }
-        for (int s = 0; s < p.S; ++s) {
-            p.grp[2 * (p.E + s)] = p.R_routed + s * p.T;
-            p.grp[2 * (p.E + s) + 1] = p.T;
+            incl = max(incl, run);
+            const int up = __shfl_up_sync(0xFFFFFFFFu, incl, 1);   // every lane takes part
+            const int prev = lane == 0 ? run : up;
+            if (e <= p.E) {
+                if ((e == 0 && o != 0) || o > F || (e > 0 && o < prev)) st |= MILO_DEV_BAD_EXPERT_ID;
+            }
+            __syncwarp();
+            if (e <= p.E) ok_off[e] = incl;
+            run = __shfl_sync(0xFFFFFFFFu, incl, 31);
         }
     }
+    __syncthreads();
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+        p.grp[2 * e] = ok_off[e];
+        p.grp[2 * e + 1] = ok_off[e + 1] - ok_off[e];
+    }
+    for (int s = threadIdx.x; s < p.S; s += blockDim.x) {
+        p.grp[2 * (p.E + s)] = p.R_routed + s * p.T;
+        p.grp[2 * (p.E + s) + 1] = p.T;
+    }
     if (p.inv) {
-        __syncthreads();
         for (int f = threadIdx.x; f < F; f += blockDim.x) p.inv[f] = -1;
         __syncthreads();
         const int used = ok_off[p.E];

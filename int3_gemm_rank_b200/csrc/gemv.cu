@@ -38,6 +38,8 @@
 //     on the device from the expert offsets, so the host never synchronises;
 //     CTAs are persistent (three per SM) and walk the items round-robin, the
 //     token tiles of one weight tile being adjacent so that they share L2.
+//     The consumers learn each item from a header the producer writes into
+//     the item's first stage.
 #include <cuda_runtime.h>
 
 #include "milo_device.cuh"
@@ -59,7 +61,7 @@ constexpr int kOffX = 2 * kTileBlk;                       // 14336
 constexpr int kStageBytes = kOffX + kTokTile * kFragRowHalves * 2;
 constexpr int kOffUA = 0, kOffUB = 8192, kOffT = 16384;   // compensator stage
 constexpr int kBarOffset = kStages * kStageBytes;
-constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 3 * (MILO_MAX_EXPERTS + 1) * 4 + 16;
+constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 3 * (MILO_MAX_EXPERTS + 1) * 4 + kStages * 4 + 16;
 
 static_assert(kStageBytes % 16 == 0 && kOffX % 16 == 0 && kTileBlk % 16 == 0, "bulk-copy alignment");
 static_assert(kOffT >= kRowsPlain * MILO_MAX_RANK * 2, "compensator stage: U rows");
@@ -249,6 +251,8 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     int* start = reinterpret_cast<int*>(empty + kStages);
     int* cnt = start + (MILO_MAX_EXPERTS + 1);
     int* row0s = cnt + (MILO_MAX_EXPERTS + 1);
+    // header of each stage: the work item whose first stage it is (-1: no more items)
+    volatile int* stage_item = row0s + (MILO_MAX_EXPERTS + 1);
 
     constexpr int RA = GLU ? kRowsGlu : kRowsPlain;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -262,17 +266,31 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         fence_barrier_init();
     }
     grid_dep_wait();
-    if (threadIdx.x == 0) {
+    // Item table from the expert groups: all threads load groups (independent
+    // global loads), then warp 0 scans the per-expert item counts.
+    for (int e = threadIdx.x; e < p.n_exp; e += blockDim.x) {
+        const int r0 = p.grp[2 * e], m = p.grp[2 * e + 1];
+        const bool ok = m > 0 && r0 >= 0 && r0 + m <= p.R;
+        cnt[e] = ok ? m : 0;
+        row0s[e] = r0;
+    }
+    __syncthreads();
+    if (warp == 0) {
         int run = 0;
-        for (int e = 0; e < p.n_exp; ++e) {
-            const int r0 = p.grp[2 * e], m = p.grp[2 * e + 1];
-            const bool ok = m > 0 && r0 >= 0 && r0 + m <= p.R;
-            start[e] = run;
-            cnt[e] = ok ? m : 0;
-            row0s[e] = r0;
-            if (ok) run += ((m + kTokTile - 1) / kTokTile) * n_tiles * p.splits;
+        for (int base = 0; base < p.n_exp; base += 32) {
+            const int e = base + lane;
+            const int m = e < p.n_exp ? cnt[e] : 0;
+            const int items = m > 0 ? ((m + kTokTile - 1) / kTokTile) * n_tiles * p.splits : 0;
+            int incl = items;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (e < p.n_exp) start[e] = run + incl - items;
+            run += __shfl_sync(0xFFFFFFFFu, incl, 31);
         }
-        start[p.n_exp] = run;
+        if (lane == 0) start[p.n_exp] = run;
     }
     __syncthreads();
     const int n_items = start[p.n_exp];
@@ -285,7 +303,15 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         uint32_t phase = 0;
         uint32_t filled = 0, fph = 0;     // per stage: has a fill, parity of its last fill
         bool fail = false;
-        for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
+        // Items are taken round-robin (item b, b + gridDim.x, ...).  A global
+        // work queue balanced the skewed DeepSeekMoE-shaped layer no better
+        // and cost the Mixtral-shaped one 15 %; the static split is kept.
+        int next = blockIdx.x;
+        for (;;) {
+            const int it = next;
+            if (it < 0 || it >= n_items) break;
+            next += gridDim.x;
+            bool header = false;      // the item's first stage has been filled
             const Item w = decode_item(it, start, cnt, p.n_exp, p.splits);
             const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
             const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
@@ -305,6 +331,10 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 uint64_t* fb = &full[stage];
                 filled |= 1u << stage;
                 fph = (fph & ~(1u << stage)) | (phase << stage);
+                if (!header) {
+                    stage_item[stage] = it;
+                    header = true;
+                }
                 const int nsb = min(2, p.SB - 2 * ch);
                 const uint32_t wb = nsb * kBlockSB;                  // one tile's block
                 const uint32_t xb = ntok * kFragRowHalves * 2;
@@ -329,6 +359,10 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 uint64_t* fb = &full[stage];
                 filled |= 1u << stage;
                 fph = (fph & ~(1u << stage)) | (phase << stage);
+                if (!header) {
+                    stage_item[stage] = it;
+                    header = true;
+                }
                 const int urows = min(RA, p.N - n0);
                 const uint32_t ua = urows * ra * 2, ub = urows * rb * 2;
                 const uint32_t tb = ntok * p.tcols * 2;
@@ -337,6 +371,29 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 if (ub) bulk_load_hint(st + kOffUB, pb->U + static_cast<size_t>(n0) * rb, ub, fb, pol);
                 bulk_load(st + kOffT, p.t + static_cast<size_t>(row0) * p.tcols, tb, fb);
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
+            }
+            if (!fail && !header) {   // an item with no stage of its own: a header-only stage
+                if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                    fail = true;
+                    break;
+                }
+                filled |= 1u << stage;
+                fph = (fph & ~(1u << stage)) | (phase << stage);
+                stage_item[stage] = it;
+                mbar_arrive(&full[stage]);
+                if (++stage == kStages) { stage = 0; phase ^= 1; }
+            }
+            if (fail) break;
+        }
+        // end of the queue for this CTA's consumers
+        if (!fail) {
+            if (mbar_wait(&empty[stage], phase ^ 1)) {
+                filled |= 1u << stage;
+                fph = (fph & ~(1u << stage)) | (phase << stage);
+                stage_item[stage] = -1;
+                mbar_arrive(&full[stage]);
+            } else {
+                fail = true;
             }
         }
         // No copy may still be landing in shared memory when the CTA leaves.
@@ -351,7 +408,15 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     uint32_t phase = 0;
     const int g = lane >> 2, c = lane & 3;
     const TileMap<GLU> tm(warp);
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+    for (;;) {
+        // the item's first stage carries its index in the stage header
+        if (!warp_wait(&full[stage], phase)) {
+            flag(p.dev_status, MILO_DEV_TIMEOUT);
+            return;
+        }
+        const int it = stage_item[stage];
+        if (it < 0) break;
+        bool waited = true;       // the next stage's barrier has been passed already
         const Item w = decode_item(it, start, cnt, p.n_exp, p.splits);
         const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
         const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
@@ -369,10 +434,11 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 for (int i = 0; i < 4; ++i) acc[a][b][i] = 0.0f;
 
         for (int ch = c0; ch < c1; ++ch) {
-            if (!mbar_wait(&full[stage], phase)) {
+            if (!waited && !warp_wait(&full[stage], phase)) {
                 flag(p.dev_status, MILO_DEV_TIMEOUT);
                 return;
             }
+            waited = false;
             const uint8_t* st = smem + stage * kStageBytes;
             const int nsb = min(2, p.SB - 2 * ch);
             if (ntok > 8) chunk_compute<GLU, 2>(st, acc, tm, nsb, lane);
@@ -383,13 +449,19 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         }
         const int ra = pa->rank, rb = GLU ? pb->rank : 0;
         if (w.split == 0 && p.has_t && (ra > 0 || rb > 0)) {
-            if (!mbar_wait(&full[stage], phase)) {
+            if (!waited && !warp_wait(&full[stage], phase)) {
                 flag(p.dev_status, MILO_DEV_TIMEOUT);
                 return;
             }
+            waited = false;
             const uint8_t* st = smem + stage * kStageBytes;
             if (ntok > 8) lorc_compute<GLU, 2>(st, acc, warp, lane, ra, rb, p.tcols, p.t_col_b);
             else lorc_compute<GLU, 1>(st, acc, warp, lane, ra, rb, p.tcols, p.t_col_b);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+        if (waited) {   // a header-only stage: release it
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
             if (++stage == kStages) { stage = 0; phase ^= 1; }

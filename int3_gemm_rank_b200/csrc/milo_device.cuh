@@ -1,6 +1,6 @@
 // milo_device.cuh -- device helpers shared by the sm_100a kernels of libmilo.
 //
-// PTX wrappers (mbarrier, TMA bulk-tensor loads, mma.sync), the int3 field
+// PTX wrappers (mbarrier, 1-D bulk copies, mma.sync), the int3 field
 // extraction of the packing format and its register schedule, and small
 // conversions.  Nothing here is shared with the CPU oracle.
 #pragma once
@@ -158,14 +158,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: each try_wait suspends for a hardware-chosen interval, so the
-// limit below amounts to well over a second before the wait gives up.
-constexpr uint32_t kWaitLimit = 1u << 24;
+// Bounded wait: gives up after about two seconds of SM clock (the caller then
+// flags MILO_DEV_TIMEOUT and unwinds), however long each try_wait suspends.
+constexpr long long kWaitCycles = 4000000000LL;
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-    return false;
+        if (clock64() - t0 > kWaitCycles) return false;
+    }
+}
+
+// The same, decided for the whole warp: every lane returns the same answer,
+// so the warp never splits on a timeout ahead of a warp-collective step.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+    return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity));
 }
 
 // ---------------------------------------------------------------------------
