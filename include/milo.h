@@ -94,14 +94,14 @@ MILO_API int32_t milo_version(void);
  * bit 15 = bit t of u_30, bit 31 = bit t of u_31.
  *
  * Device layout: one blob per weight.  Rows are grouped in tiles of 64 (the
- * last tile padded with zero rows), K in chunks of two super-blocks (the last
- * chunk holds one when K/128 is odd).  The (tile t, chunk c) block starts at
- * byte (t * K/128 + 2c) * 3584 and holds, for its nsb super-blocks b,
+ * last tile padded with zero rows).  The (tile t, super-block b) block starts
+ * at byte (t * K/128 + b) * 3584 and holds
  *     the words u32 [64 rows][12]      (word j of row 64t+r = word 12b+j above)
- * then, for its 2*nsb groups g, 256 bytes: for each 16-row block m (0..3)
- * and j (0..7) the fp16 quadruple s, z of row 16m+j, s, z of row 16m+j+8
- * so that the kernels fetch a tile's chunk -- codes, scales and zeros -- with
- * one copy.  Dequantisation: w_hat[n, k] = (q[n, k] - z[n, k/64]) * s[n, k/64].
+ * then, for groups 2b and 2b+1, 256 bytes each: for each 16-row block m
+ * (0..3) and j (0..7) the fp16 quadruple s, z of row 16m+j, s, z of row 16m+j+8
+ * so that the kernels fetch one or more consecutive super-blocks of a tile --
+ * codes, scales and zeros -- with one copy.
+ * Dequantisation: w_hat[n, k] = (q[n, k] - z[n, k/64]) * s[n, k/64].
  * The blob has ceil(N/64) * (K/128) * 3584 bytes (milo_packed_bytes).
  */
 

@@ -51,10 +51,11 @@ namespace milo {
 constexpr int kStages = 3;
 constexpr int kConsumerWarps = 4;
 constexpr int kGemvThreads = 32 * (kConsumerWarps + 1);
-// Stage layout (bytes).  Two weight regions of kTileBlk bytes, each one
-// (tile, chunk) block of the packed blob: codes [nsb][64 rows][12 words], then
-// per group [64 scales][64 zeros] (GLU: w1's tile, then w3's; plain: rows
-// 0-63, then 64-127).  Then the activations [16 rows][272 fp16].
+// Stage layout (bytes).  Two weight regions of kTileBlk bytes, each the nsb
+// (tile, super-block) blocks of the packed blob: per super-block the codes
+// [64 rows][12 words], then its two groups' (s, z) pairs (GLU: w1's tile,
+// then w3's; plain: rows 0-63, then 64-127).  Then the activations
+// [16 rows][272 fp16].
 constexpr int kTileBlk = 2 * kBlockSB;                    // 7168
 constexpr int kOffQ = 0;
 constexpr int kOffX = 2 * kTileBlk;                       // 14336
@@ -136,17 +137,17 @@ struct TileMap {
 };
 
 // acc += s * 2^24 * D_g - s * z * X_g for group `grp` (0..3) of the chunk;
-// the scales of the chunk's groups start nsb * 3072 bytes into each region,
-// as (s, z) pairs of rows j and j + 8 of each 16-row block, so one 64-bit
-// load brings the lane's two rows.  xg[n8][j]: X_g of its tokens.
+// super-block grp / 2's scales follow its codes, as (s, z) pairs of rows j and
+// j + 8 of each 16-row block, so one 64-bit load brings the lane's two rows.
+// xg[n8][j]: X_g of its tokens.
 template <int NT>
 __device__ __forceinline__ void fold_group(float (&acc)[2][2][4], const float (&dz)[2][2][4],
                                            const uint8_t* st, int grp, const int (&reg)[2],
-                                           const int (&rbase)[2], int nsb, int g, const float (&xg)[NT][2]) {
+                                           const int (&rbase)[2], int g, const float (&xg)[NT][2]) {
 #pragma unroll
     for (int ti = 0; ti < 2; ++ti) {
-        const uint2 q = *reinterpret_cast<const uint2*>(st + reg[ti] + nsb * kQTileSBWords * 4 + grp * kGroupBytes +
-                                                        ((rbase[ti] >> 4) * 8 + g) * 8);
+        const uint2 q = *reinterpret_cast<const uint2*>(st + reg[ti] + (grp >> 1) * kBlockSB + kQTileSBWords * 4 +
+                                                        (grp & 1) * kGroupBytes + ((rbase[ti] >> 4) * 8 + g) * 8);
         float s24[2], nsz[2];
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
@@ -177,7 +178,7 @@ __device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2]
         uint32_t wd[2][2][3], hw[2][2][3];
 #pragma unroll
         for (int ti = 0; ti < 2; ++ti) {
-            const uint32_t* qt = reinterpret_cast<const uint32_t*>(st + tm.reg[ti]) + sbl * kQTileSBWords;
+            const uint32_t* qt = reinterpret_cast<const uint32_t*>(st + tm.reg[ti] + sbl * kBlockSB);
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
@@ -204,12 +205,12 @@ __device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2]
         code_step<1, NT>(wd, hw, xs, g, c, dz);
         code_step<2, NT>(wd, hw, xs, g, c, dz);
         code_step<3, NT>(wd, hw, xs, g, c, dz);
-        fold_group<NT>(acc, dz, st, 2 * sbl, tm.reg, tm.r, nsb, g, xa);
+        fold_group<NT>(acc, dz, st, 2 * sbl, tm.reg, tm.r, g, xa);
         code_step<4, NT>(wd, hw, xs, g, c, dz);
         code_step<5, NT>(wd, hw, xs, g, c, dz);
         code_step<6, NT>(wd, hw, xs, g, c, dz);
         code_step<7, NT>(wd, hw, xs, g, c, dz);
-        fold_group<NT>(acc, dz, st, 2 * sbl + 1, tm.reg, tm.r, nsb, g, xb);
+        fold_group<NT>(acc, dz, st, 2 * sbl + 1, tm.reg, tm.r, g, xb);
     }
 }
 

@@ -25,10 +25,10 @@ constexpr int kFragHalvesPerSB = 128;
 constexpr int kFragRowHalves = 2 * kFragHalvesPerSB + 16;
 constexpr int kGsumHalf = 2 * kFragHalvesPerSB;
 
-// Packed weights (milo.h): rows in tiles of 64, K in chunks of two
-// super-blocks; each (tile, chunk) block -- the codes of its super-blocks, then
-// per group 64 scales and 64 zeros -- is contiguous, so one bulk copy brings a
-// tile's chunk.  kBlockSB bytes per tile and super-block.
+// Packed weights (milo.h): rows in tiles of 64; each (tile, super-block)
+// block -- the codes, then the two groups' scales and zeros -- is contiguous,
+// and consecutive super-blocks of a tile are adjacent, so one bulk copy brings
+// a tile's K chunk.  kBlockSB bytes per tile and super-block.
 constexpr int kTileRows = 64;
 constexpr int kQTileSBWords = kTileRows * 12;       // codes of one tile, one super-block: 3072 bytes
 constexpr int kGroupBytes = kTileRows * 2 * 2;      // scales and zeros of one tile, one group: 256 bytes

@@ -13,18 +13,17 @@
 
 namespace milo {
 
-// Device blob (milo.h): 64-row tiles, K chunks of two super-blocks, each
-// (tile, chunk) block = the words of its super-blocks, then per group the
-// scales and zeros as (s, z) pairs of rows r and r + 8 of each 16-row block.
-// Byte offsets of row n's words for super-block b and of its scale for group
-// j (its zero follows 2 bytes later).
+// Device blob (milo.h): one block per (64-row tile, super-block) = the tile's
+// words for the super-block, then its two groups' scales and zeros as (s, z)
+// pairs of rows r and r + 8 of each 16-row block.  Byte offsets of row n's
+// words for super-block b and of its scale for group j (its zero follows 2
+// bytes later).
 __device__ __forceinline__ size_t blob_words(int n, int b, int SB) {
-    const int c = b >> 1;
-    return (static_cast<size_t>(n / 64) * SB + 2 * c) * kBlockSB + ((b & 1) * 64 + (n % 64)) * 48;
+    return (static_cast<size_t>(n / 64) * SB + b) * kBlockSB + (n % 64) * 48;
 }
 __device__ __forceinline__ size_t blob_group(int n, int j, int SB) {
-    const int c = j >> 2, nsb = min(2, SB - 2 * c), r = n % 64;
-    return (static_cast<size_t>(n / 64) * SB + 2 * c) * kBlockSB + nsb * 3072 + (j & 3) * kGroupBytes +
+    const int r = n % 64;
+    return (static_cast<size_t>(n / 64) * SB + (j >> 1)) * kBlockSB + kQTileSBWords * 4 + (j & 1) * kGroupBytes +
            (((r >> 4) * 8 + (r & 7)) * 4 + ((r >> 3) & 1) * 2) * 2;
 }
 

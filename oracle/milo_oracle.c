@@ -216,42 +216,37 @@ void milo_ref_unpack(const uint32_t* Q, int N, int K, uint8_t* q) {
 
 /*
  * Device layout of a packed weight: one byte blob.  Rows are grouped in tiles
- * of 64 (the last tile padded with zero rows), K in chunks of two super-blocks
- * (the last chunk has one when K/128 is odd), and each (tile, chunk) block is
- * contiguous, so the GPU kernels fetch it with a single copy:
- *     block(t, c) at byte (t * SB + 2 * c) * 3584, holding for its nsb
- *     super-blocks b (in order) the words  [64 rows][12]        (nsb * 3072 B)
- *     then for its 2 * nsb groups g (in order) 256 bytes: for each 16-row
- *     block m (0..3) and j (0..7) the fp16 quadruple
+ * of 64 (the last tile padded with zero rows); the block of (tile t,
+ * super-block b) is contiguous, at byte (t * SB + b) * 3584, and holds
+ *     the words of the tile's rows  [64 rows][12]               (3072 B)
+ *     then for the super-block's groups 2b and 2b + 1, 256 bytes each: for
+ *     each 16-row block m (0..3) and j (0..7) the fp16 quadruple
  *         s[16m + j], z[16m + j], s[16m + j + 8], z[16m + j + 8]
- * Word j of row n, super-block b, is Q[n, 12 b + j]; s and z of row n, group
- * g are scale[g, n] and zero[g, n].  This is a relayout only, used to compare
- * with the device packer.
+ * so the GPU kernels fetch one or two super-blocks of a tile -- codes, scales
+ * and zeros -- with a single copy.  Word j of row n, super-block b, is
+ * Q[n, 12 b + j]; s and z of row n, group g are scale[g, n] and zero[g, n].
+ * This is a relayout only, used to compare with the device packer.
  */
 void milo_ref_tile_pack(const uint32_t* Q, const uint16_t* scale, const uint16_t* zero,
                         int N, int K, uint8_t* blob) {
-    int SB = K / 128, G = K / 64, W = 3 * K / 32, NT = (N + 63) / 64;
+    int SB = K / 128, W = 3 * K / 32, NT = (N + 63) / 64;
     memset(blob, 0, (size_t)NT * SB * 3584);
     for (int t = 0; t < NT; ++t)
-        for (int c = 0; 2 * c < SB; ++c) {
-            int nsb = SB - 2 * c < 2 ? SB - 2 * c : 2;
-            uint8_t* base = blob + ((size_t)t * SB + 2 * c) * 3584;
+        for (int b = 0; b < SB; ++b) {
+            uint8_t* base = blob + ((size_t)t * SB + b) * 3584;
             uint32_t* words = (uint32_t*)base;
-            uint16_t* groups = (uint16_t*)(base + (size_t)nsb * 3072);
+            uint16_t* groups = (uint16_t*)(base + 3072);
             for (int r = 0; r < 64; ++r) {
                 int n = 64 * t + r;
                 if (n >= N) continue;
-                for (int i = 0; i < nsb; ++i)
-                    for (int j = 0; j < 12; ++j)
-                        words[(i * 64 + r) * 12 + j] = Q[(size_t)n * W + 12 * (2 * c + i) + j];
-                for (int i = 0; i < 2 * nsb; ++i) {
-                    int g = 4 * c + i;
+                for (int j = 0; j < 12; ++j) words[r * 12 + j] = Q[(size_t)n * W + 12 * b + j];
+                for (int i = 0; i < 2; ++i) {
+                    int g = 2 * b + i;
                     int q = i * 128 + ((r / 16) * 8 + r % 8) * 4 + ((r % 16) / 8) * 2;
                     groups[q] = scale[(size_t)g * N + n];
                     groups[q + 1] = zero[(size_t)g * N + n];
                 }
             }
-            (void)G;
         }
 }
 

@@ -132,10 +132,9 @@ def test_unpack_roundtrip_exhaustive_one_hot_and_random():
 
 def test_device_blob_matches_reshape():
     """The device blob of a packed weight: 64-row tiles (zero rows pad the last),
-    K chunks of two super-blocks (one in the last chunk when K/128 is odd), each
-    (tile, chunk) block = the tile's words super-block major, then per group the
-    scales and zeros, interleaved as (s, z) of rows j and j + 8 of each 16-row
-    block.  Checked against numpy reshapes/transposes of the
+    one block per (tile, super-block) = the tile's words for the super-block,
+    then its two groups' scales and zeros, interleaved as (s, z) of rows j and
+    j + 8 of each 16-row block.  Checked against numpy reshapes/transposes of the
     padded arrays, for N that is and is not a multiple of 64 and for even and odd
     K/128."""
     rng = np.random.default_rng(11)
@@ -153,10 +152,9 @@ def test_device_blob_matches_reshape():
         groups = groups.transpose(1, 0, 2, 4, 3, 5)
         parts = []
         for t in range(NT):
-            for c in range(0, SB, 2):
-                nsb = min(2, SB - c)
-                parts.append(words[t, c:c + nsb].reshape(-1).view(np.uint8))
-                parts.append(groups[t, 2 * c:2 * c + 2 * nsb].reshape(-1).view(np.uint8))
+            for b in range(SB):
+                parts.append(words[t, b].reshape(-1).view(np.uint8))
+                parts.append(groups[t, 2 * b:2 * b + 2].reshape(-1).view(np.uint8))
         want = np.concatenate(parts)
         assert want.size == NT * SB * 3584
         assert np.array_equal(oracle.tile_pack(Q, sc, ze, K), want)
