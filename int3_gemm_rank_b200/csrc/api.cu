@@ -27,6 +27,46 @@ static thread_local std::string g_last_error;
 void clear_error() { g_last_error.clear(); }
 void set_error(const std::string& msg) { g_last_error = msg; }
 
+// ---------------------------------------------------------------------------
+// tensor maps of the tcgen05 GEMM (driver entry point fetched through the
+// runtime; no -lcuda)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [rows, cols] with row pitch `pitch` bytes; box {bcols, brows}.
+static milo_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols,
+                            uint64_t rows, uint64_t pitch, uint32_t bcols, uint32_t brows, const char* what,
+                            CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(MILO_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {pitch};
+    cuuint32_t box[2] = {bcols, brows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(MILO_ERR_INVALID_ARG, std::string("tensor map encoding failed for ") + what + " (code " +
+                                              std::to_string(static_cast<int>(r)) + ")");
+    return MILO_OK;
+}
+
 // Measurement hook (milo_set_profile_events).
 static cudaEvent_t g_prof[4] = {nullptr, nullptr, nullptr, nullptr};
 static int g_prof_n = 0;
@@ -93,15 +133,18 @@ struct Carve {
 // Prepared activations and group sums of R rows: chunk-major (K chunks of 256).
 static int chunks_of(int K) { return (K + kChunkK - 1) / kChunkK; }
 static size_t frag_bytes(int K, int R) {
+    // the mma.sync layout; the tcgen05 layout [R][K] fp16 is never larger
     return static_cast<size_t>(chunks_of(K)) * R * kFragRowHalves * 2;
 }
+// group sums of the tcgen05 path: [R][4 * chunks] f32
+static size_t gsum_bytes(int K, int R) { return static_cast<size_t>(chunks_of(K)) * R * 16; }
 
 struct LorcPlan {
     int splits, row_groups;
 };
 
 struct LinearWs {
-    size_t grp, rows, inv, frag, t, tpart, part, total;
+    size_t grp, rows, inv, frag, gsum, t, tpart, part, total;
     int R, splits, tcols;
     LorcPlan lp;
 };
@@ -157,6 +200,7 @@ static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
     w.rows = c.take(static_cast<size_t>(w.R) * 4);
     w.inv = c.take(static_cast<size_t>(w.R) * 4);
     w.frag = c.take(frag_bytes(lin->K, w.R));
+    w.gsum = c.take(gsum_bytes(lin->K, w.R));
     w.t = c.take(static_cast<size_t>(w.R) * w.tcols * 2);
     w.lp = lorc_plan(n_exp, 1, lin->K, static_cast<long long>(T) * k);   // at most all rows in one expert
     w.tpart = c.take(static_cast<size_t>(w.lp.splits) * w.R * w.tcols * 4);
@@ -166,7 +210,7 @@ static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
 }
 
 struct MoeWs {
-    size_t grp, rows, xfrag, t13, h, hfrag, t2, tpart, part, total;
+    size_t grp, rows, xfrag, xg, t13, h, hfrag, hg, t2, tpart, part, total;
     int R, R_routed, splits, tc13, tc2;
     LorcPlan lp13, lp2;
 };
@@ -186,9 +230,11 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
     w.grp = c.take(static_cast<size_t>(n_exp) * 8);
     w.rows = c.take(static_cast<size_t>(w.R) * 4);
     w.xfrag = c.take(frag_bytes(H, w.R));
+    w.xg = c.take(gsum_bytes(H, w.R));
     w.t13 = c.take(static_cast<size_t>(w.R) * w.tc13 * 2);
     w.h = c.take(static_cast<size_t>(w.R) * I * 2);
     w.hfrag = c.take(frag_bytes(I, w.R));
+    w.hg = c.take(gsum_bytes(I, w.R));
     w.t2 = c.take(static_cast<size_t>(w.R) * w.tc2 * 2);
     // a token meets an expert at most once, and a shared expert sees every token
     w.lp13 = lorc_plan(n_exp, 2, H, T);
@@ -218,6 +264,56 @@ static void act_ptrs(GemvParams& g, void* frag, void* t, int R, int K, int tcols
 static milo_status run_gemv(GemvParams& g, bool glu, cudaStream_t st, const char* what) {
     const int grid = 3 * sm_count();
     return check_cuda(launch_gemv(g, glu, grid, st), what);
+}
+
+// Which grouped GEMM runs.  The mma.sync kernel suits a few routed rows per
+// expert (decode): a tcgen05.mma of N = 16 costs as much to issue as one of
+// N = 64.  With many rows per expert (prefill) the weights are reused across
+// 128-row tiles and the tcgen05 kernel takes over.  MILO_GEMM=mma|tc forces
+// one (both give the same results within fp32 rounding).
+static bool use_tc(long long routed_rows, int n_routed) {
+    const char* v = getenv("MILO_GEMM");
+    if (v && v[0] == 't') return true;
+    if (v && v[0] == 'm') return false;
+    return routed_rows >= 64LL * std::max(1, n_routed);
+}
+
+// The grouped GEMM described by g on the tcgen05 kernel: activations in
+// A-column order [R][K] fp16 with group sums [R][4 * chunks] f32.
+static milo_status run_tc(const GemvParams& g, bool glu, void* xcol, void* gsum, cudaStream_t st,
+                          const char* what) {
+    TcParams p;
+    memset(&p, 0, sizeof(p));
+    milo_status s;
+    const int Rm = std::max(g.R, 1);
+    const int chunks = chunks_of(g.K);
+    if ((s = make_map(&p.b_map, xcol, CU_TENSOR_MAP_DATA_TYPE_UINT16, g.K, Rm, static_cast<uint64_t>(g.K) * 2, 64,
+                      128, "activations", CU_TENSOR_MAP_SWIZZLE_128B)) != MILO_OK)
+        return s;
+    if ((s = make_map(&p.g_map, gsum, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4 * chunks, Rm,
+                      static_cast<uint64_t>(chunks) * 16, 4, 128, "group sums")) != MILO_OK)
+        return s;
+    if (g.has_t && (s = make_map(&p.t_map, g.t, CU_TENSOR_MAP_DATA_TYPE_UINT16, g.tcols, Rm,
+                                 static_cast<uint64_t>(g.tcols) * 2, 64, 128, "compensator rows",
+                                 CU_TENSOR_MAP_SWIZZLE_128B)) != MILO_OK)
+        return s;
+    p.table = g.table;
+    p.grp = g.grp;
+    p.y_part = g.y_part;
+    p.h = g.h;
+    p.dev_status = g.dev_status;
+    p.stride = g.stride;
+    p.proj_a = g.proj_a;
+    p.proj_b = g.proj_b;
+    p.n_exp = g.n_exp;
+    p.N = g.N;
+    p.K = g.K;
+    p.R = g.R;
+    p.SB = g.K / 128;
+    p.has_t = g.has_t;
+    p.tcols = g.tcols;
+    p.t_col_b = g.t_col_b;
+    return check_cuda(launch_tc_gemm(p, glu, sm_count(), st), what);
 }
 
 }  // namespace milo
@@ -351,9 +447,10 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     int32_t* rows = reinterpret_cast<int32_t*>(base + w.rows);
     int32_t* inv = reinterpret_cast<int32_t*>(base + w.inv);
 
+    const bool tc = use_tc(static_cast<long long>(T) * k, lin->n_experts);
     PrepParams pp{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.frag),
-                  dev_status, w.R, lin->K, x_dt == MILO_BF16, 1,
-                  expert_offsets, perm, grp, inv, T, k, lin->n_experts, 0, w.R};
+                  reinterpret_cast<float*>(base + w.gsum), tc ? 1 : 0, dev_status, w.R, lin->K, x_dt == MILO_BF16,
+                  1, expert_offsets, perm, grp, inv, T, k, lin->n_experts, 0, w.R};
     milo_status s = check_cuda(launch_prep(pp, st), "prep");
     if (s != MILO_OK) return s;
 
@@ -379,14 +476,17 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     g.proj_b = 0;
     g.n_exp = lin->n_experts;
     g.N = lin->N;
-    g.splits = w.splits;
-    g.cps = (g.chunks + w.splits - 1) / w.splits;
+    const int splits = tc ? 1 : w.splits;   // the tcgen05 kernel does not split K
+    g.splits = splits;
+    g.cps = (g.chunks + splits - 1) / splits;
     prof_record(0, st);
-    if ((s = run_gemv(g, false, st, "gemv")) != MILO_OK) return s;
+    if (tc) s = run_tc(g, false, base + w.frag, base + w.gsum, st, "tc gemm");
+    else s = run_gemv(g, false, st, "gemv");
+    if (s != MILO_OK) return s;
     prof_record(1, st);
 
     CombineParams cp{reinterpret_cast<const float*>(base + w.part), inv, nullptr, y, dev_status,
-                     T, k, 0, lin->N, w.R, w.splits, w.R, static_cast<int>(y_dt), 1};
+                     T, k, 0, lin->N, w.R, splits, w.R, static_cast<int>(y_dt), 1};
     return check_cuda(launch_combine(cp, st), "combine");
 }
 
@@ -417,8 +517,9 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     const bool has_t = L->max_rank > 0;
     milo_status s;
 
+    const bool tc = use_tc(w.R_routed, L->n_routed);
     PrepParams px{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.xfrag),
-                  dev_status, w.R, H, x_dt == MILO_BF16, 1,
+                  reinterpret_cast<float*>(base + w.xg), tc ? 1 : 0, dev_status, w.R, H, x_dt == MILO_BF16, 1,
                   expert_offsets, perm, grp, nullptr, T, L->top_k, L->n_routed, L->n_shared, w.R_routed};
     if ((s = check_cuda(launch_prep(px, st), "prep x")) != MILO_OK) return s;
     if (has_t) {
@@ -445,12 +546,14 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     g1.cps = g1.chunks;
     g1.t_col_b = L->max_rank;
     prof_record(0, st);
-    if ((s = run_gemv(g1, true, st, "gemv w1|w3")) != MILO_OK) return s;
+    if (tc) s = run_tc(g1, true, base + w.xfrag, base + w.xg, st, "tc gemm w1|w3");
+    else s = run_gemv(g1, true, st, "gemv w1|w3");
+    if (s != MILO_OK) return s;
     prof_record(1, st);
 
     PrepParams ph{reinterpret_cast<const uint16_t*>(base + w.h), nullptr,
-                  reinterpret_cast<uint16_t*>(base + w.hfrag), dev_status, w.R, I, 0, 0, nullptr, nullptr,
-                  nullptr, nullptr, 0, 0, 0, 0, 0};
+                  reinterpret_cast<uint16_t*>(base + w.hfrag), reinterpret_cast<float*>(base + w.hg), tc ? 1 : 0,
+                  dev_status, w.R, I, 0, 0, nullptr, nullptr, nullptr, nullptr, 0, 0, 0, 0, 0};
     if ((s = check_cuda(launch_prep(ph, st), "prep h")) != MILO_OK) return s;
     if (has_t) {
         LorcParams lp{reinterpret_cast<const uint16_t*>(base + w.h), nullptr, table, grp,
@@ -471,13 +574,16 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     g2.proj_b = 2;
     g2.n_exp = n_exp;
     g2.N = H;
-    g2.splits = w.splits;
-    g2.cps = (g2.chunks + w.splits - 1) / w.splits;
+    const int splits = tc ? 1 : w.splits;   // the tcgen05 kernel does not split K
+    g2.splits = splits;
+    g2.cps = (g2.chunks + splits - 1) / splits;
     prof_record(2, st);
-    if ((s = run_gemv(g2, false, st, "gemv w2")) != MILO_OK) return s;
+    if (tc) s = run_tc(g2, false, base + w.hfrag, base + w.hg, st, "tc gemm w2");
+    else s = run_gemv(g2, false, st, "gemv w2");
+    if (s != MILO_OK) return s;
     prof_record(3, st);
 
     CombineParams cp{reinterpret_cast<const float*>(base + w.part), inv_perm, topk_w, y, dev_status,
-                     T, L->top_k, L->n_shared, H, w.R, w.splits, w.R_routed, static_cast<int>(y_dt), 0};
+                     T, L->top_k, L->n_shared, H, w.R, splits, w.R_routed, static_cast<int>(y_dt), 0};
     return check_cuda(launch_combine(cp, st), "combine");
 }

@@ -152,6 +152,25 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
         s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
         s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 2);
         if (!active) continue;
+        if (p.layout == 1) {
+            // tcgen05 GEMM: [R][K] with the K slots of each super-block in the
+            // order of the A columns (unit c's first-group registers at columns
+            // 8c..8c+7, its second-group ones at 32+8c..), group sums [R][4*chunks]
+            uint4* o1 = reinterpret_cast<uint4*>(p.frag + static_cast<size_t>(row) * p.K + 128 * sb + 16 * c);
+            uint4* o2 = reinterpret_cast<uint4*>(p.frag + static_cast<size_t>(row) * p.K + 128 * sb + 64 + 16 * c);
+            const uint2 f0 = frag_step<0>(x), f1 = frag_step<1>(x), f2 = frag_step<2>(x), f3 = frag_step<3>(x);
+            const uint2 f4 = frag_step<4>(x), f5 = frag_step<5>(x), f6 = frag_step<6>(x), f7 = frag_step<7>(x);
+            o1[0] = make_uint4(f0.x, f0.y, f1.x, f1.y);
+            o1[1] = make_uint4(f2.x, f2.y, f3.x, f3.y);
+            o2[0] = make_uint4(f4.x, f4.y, f5.x, f5.y);
+            o2[1] = make_uint4(f6.x, f6.y, f7.x, f7.y);
+            if (c == 0) {
+                const size_t gp = static_cast<size_t>(row) * 4 * ((SB + 1) / 2) + 2 * sb;
+                p.gsum[gp] = s0;
+                p.gsum[gp + 1] = s1;
+            }
+            continue;
+        }
         // chunk-major layout: the 16-row tile of one K chunk is one contiguous
         // block; the chunk's four group sums sit in the row's padding
         const size_t crow = static_cast<size_t>(sb >> 1) * p.R + row;

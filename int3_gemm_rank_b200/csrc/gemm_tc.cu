@@ -1,0 +1,618 @@
+// gemm_tc.cu -- grouped int3 x fp16 GEMM with the low-rank compensator on the
+// 5th-generation tensor cores (tcgen05, TMEM), for experts with many routed
+// rows (prefill, large batches) (sm_100a).
+//
+// "MiLo: Efficient Quantized MoE Inference with Mixture of Low-Rank
+// Compensators": W_out = W_quant + U V ("MiLo Algorithm"), an int3 x FP16 GEMM
+// with dequantisation and the asymmetric zero point fused in ("MiLo Kernel").
+//
+// Design (B200):
+//   - A work item is (expert, 128 weight rows, 128 routed rows); a stage is
+//     one 128-code super-block.  The producer warp brings the activations
+//     (2-D TMA, 128-byte swizzle: the K-major B operand), the two 64-row
+//     blob blocks (1-D bulk copies: codes, scales, zeros) and the group sums.
+//   - Four extraction warps (one thread per weight row) turn the row's 32
+//     code pairs into exact fp16 patterns code * 2^e * 2^-24 (one LOP3 per
+//     pair, the 2^e folded into the activations) and store them to TMEM: the
+//     A operand.
+//   - One thread of the MMA warp issues tcgen05.mma M=128, N=128, K=16 with A
+//     from TMEM and B from shared memory, per 64-code scale group into its own
+//     TMEM accumulator D_g (double-buffered).
+//   - Eight fold warps (two per weight row: 64 routed rows and 64 fp32
+//     accumulators each) read D_g and fold acc += s * 2^24 * D_g - s * z * X_g
+//     (packed FFMA2),
+//     so the zero point and the scale cost nothing per weight and the result
+//     is exact to fp32 rounding.  The group sums X_g of a stage are transposed
+//     once in shared memory so that each fold thread reads them four at a time.
+//   - The compensator is one more stage: A = U rows, B = t = x V^T.
+//   - Epilogue: SwiGLU through a shared-memory exchange (w3 rows hand b to the
+//     w1 rows), or the fp32 output rows.
+//   - Every wait is bounded; on a timeout the kernel flags MILO_DEV_TIMEOUT,
+//     drains its copies and MMAs and frees TMEM before leaving.
+#include <cuda_runtime.h>
+
+#include "milo_device.cuh"
+#include "milo_host.h"
+#include "milo_kernels.h"
+#include "milo_tc.cuh"
+
+namespace milo {
+
+constexpr int kTcTok = 128;                 // routed rows per item (MMA N)
+constexpr int kTcRows = 128;                // weight rows per item (MMA M)
+constexpr int kTcStages = 4;
+constexpr int kTcStage = 49152;             // bytes per stage (multiple of 1024)
+constexpr int kTcOffB = 0;                  // activations: 2 swizzled atoms [128 rows][128 B]
+constexpr int kTcAtom = kTcTok * 128;       // 16384
+constexpr int kTcOffW = 2 * kTcAtom;        // two blob blocks (rows 0-63, 64-127)
+constexpr int kTcOffG = kTcOffW + 2 * kBlockSB;   // group sums [128 rows][4] f32
+constexpr int kTcStageTx = 2 * kTcAtom + kTcTok * 16;   // plus the blob blocks
+constexpr int kTcOffUA = kTcOffW;           // compensator stage: U rows of w1 (or 128 rows)
+constexpr int kTcOffUB = kTcOffW + 64 * MILO_MAX_RANK * 2;   // U rows of w3
+constexpr int kTcXT = kTcStages * kTcStage;             // transposed group sums [stage][2][128] f32
+constexpr int kTcXch = kTcXT + kTcStages * 2 * kTcTok * 4;   // SwiGLU exchange [64 rows][64 tokens] f32
+constexpr int kTcBar = kTcXch + 64 * 64 * 4;
+constexpr int kTcNumBars = 3 * kTcStages + 2 * 2 + 2 * 2 + 1 + 4;   // + xready[stage], done, xfull[2], xempty[2]
+constexpr int kTcTab = kTcBar + 8 * kTcNumBars + 16;
+constexpr int kTcSmemUsed = kTcTab + 3 * (MILO_MAX_EXPERTS + 1) * 4;
+constexpr int kTcSmemBytes = kTcSmemUsed + 1024;        // slack to align the base to 1024 B
+constexpr int kTcFoldWarps = 8;             // two per TMEM lane quarter, 64 routed rows each
+constexpr int kTcThreads = 32 * (2 + 4 + kTcFoldWarps);   // producer, MMA, extraction, fold
+constexpr uint32_t kTcTmemCols = 512;       // A: 2 x 64 columns, D: 2 x 128 columns
+constexpr int kTcACol = 0, kTcDCol = 128;
+
+static_assert(kTcOffG + kTcTok * 16 <= kTcStage, "stage layout");
+static_assert(kTcOffUB + 64 * MILO_MAX_RANK * 2 <= kTcStage, "compensator stage: U rows");
+static_assert(kTcOffUA + kTcRows * MILO_MAX_RANK * 2 <= kTcStage, "compensator stage: plain U rows");
+static_assert(kTcSmemBytes <= 227 * 1024, "shared memory");
+
+struct TcItem {
+    int e, ntile, tt;
+};
+
+__device__ __forceinline__ TcItem tc_decode(int it, const int* start, const int* cnt, int n_exp) {
+    int lo = 0, hi = n_exp - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (start[mid] <= it) lo = mid;
+        else hi = mid - 1;
+    }
+    TcItem r;
+    r.e = lo;
+    const int local = it - start[lo];
+    const int tte = (cnt[lo] + kTcTok - 1) / kTcTok;
+    r.tt = local % tte;
+    r.ntile = local / tte;
+    return r;
+}
+
+// Register R (0..15) of unit C goes to A column 32 * (R / 8) + 8 * C + R % 8:
+// the first scale group's registers fill columns 0..31, the second's 32..63
+// (R = 2 * step + half of the eight-step register schedule).
+template <int C, int R>
+__device__ __forceinline__ void tc_unit_reg(const uint32_t (&w)[3], const uint32_t (&hw)[3], uint32_t (&a)[64]) {
+    constexpr int s = R / 2, hh = R % 2;
+    a[32 * (R / 8) + 8 * C + (R % 8)] = unit_reg<sched_word(s, hh), sched_field(s, hh)>(w, hw);
+}
+
+template <int C>
+__device__ __forceinline__ void tc_unit(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t (&a)[64]) {
+    const uint32_t w[3] = {w0, w1, w2};
+    const uint32_t hw[3] = {w0 >> word_shift(0), w1 >> word_shift(1), w2 >> word_shift(2)};
+    tc_unit_reg<C, 0>(w, hw, a);
+    tc_unit_reg<C, 1>(w, hw, a);
+    tc_unit_reg<C, 2>(w, hw, a);
+    tc_unit_reg<C, 3>(w, hw, a);
+    tc_unit_reg<C, 4>(w, hw, a);
+    tc_unit_reg<C, 5>(w, hw, a);
+    tc_unit_reg<C, 6>(w, hw, a);
+    tc_unit_reg<C, 7>(w, hw, a);
+    tc_unit_reg<C, 8>(w, hw, a);
+    tc_unit_reg<C, 9>(w, hw, a);
+    tc_unit_reg<C, 10>(w, hw, a);
+    tc_unit_reg<C, 11>(w, hw, a);
+    tc_unit_reg<C, 12>(w, hw, a);
+    tc_unit_reg<C, 13>(w, hw, a);
+    tc_unit_reg<C, 14>(w, hw, a);
+    tc_unit_reg<C, 15>(w, hw, a);
+}
+
+template <bool GLU>
+__global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTcBar);
+    uint64_t* empty = full + kTcStages;
+    uint64_t* afull = empty + kTcStages;
+    uint64_t* aempty = afull + 2;
+    uint64_t* dfull = aempty + 2;
+    uint64_t* dempty = dfull + 2;
+    uint64_t* done_bar = dempty + 2;
+    uint64_t* xfull = done_bar + 1;      // [2] SwiGLU exchange, per round: w3 rows -> w1 rows
+    uint64_t* xempty = xfull + 2;        // [2]
+    uint64_t* xready = xempty + 2;       // [kTcStages]: a stage's group sums are transposed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xready + kTcStages);
+    int* start = reinterpret_cast<int*>(smem + kTcTab);
+    int* cnt = start + (MILO_MAX_EXPERTS + 1);
+    int* row0s = cnt + (MILO_MAX_EXPERTS + 1);
+    float* xt = reinterpret_cast<float*>(smem + kTcXT);
+    float* xch = reinterpret_cast<float*>(smem + kTcXch);
+
+    constexpr int RA = GLU ? kRowsGlu : kRowsPlain;   // output features per item
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles = (p.N + RA - 1) / RA;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1 + 4 + kTcFoldWarps);   // MMA commit, extraction warps, fold warps
+            mbar_init(&xready[s], kTcFoldWarps);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&afull[b], 4);
+            mbar_init(&aempty[b], 1);
+            mbar_init(&dfull[b], 1);
+            mbar_init(&dempty[b], kTcFoldWarps);
+        }
+        mbar_init(done_bar, 1);
+        for (int rd = 0; rd < 2; ++rd) {
+            mbar_init(&xfull[rd], 2);    // the two w3 fold warps of the round
+            mbar_init(&xempty[rd], 2);   // the two w1 fold warps of the round
+        }
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, kTcTmemCols);
+    grid_dep_wait();
+    // item table: all threads load the expert groups, warp 0 scans the item counts
+    for (int e = threadIdx.x; e < p.n_exp; e += blockDim.x) {
+        const int r0 = p.grp[2 * e], m = p.grp[2 * e + 1];
+        const bool ok = m > 0 && r0 >= 0 && r0 + m <= p.R;
+        cnt[e] = ok ? m : 0;
+        row0s[e] = r0;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int run = 0;
+        for (int base = 0; base < p.n_exp; base += 32) {
+            const int e = base + lane;
+            const int m = e < p.n_exp ? cnt[e] : 0;
+            const int items = m > 0 ? ((m + kTcTok - 1) / kTcTok) * n_tiles : 0;
+            int incl = items;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (e < p.n_exp) start[e] = run + incl - items;
+            run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0) start[p.n_exp] = run;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const int n_items = start[p.n_exp];
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint64_t pol = l2_evict_first();
+            int stage = 0;
+            uint32_t phase = 0, filled = 0, fph = 0;
+            bool fail = false;
+            for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
+                const TcItem w = tc_decode(it, start, cnt, p.n_exp);
+                const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
+                const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
+                const int n0 = w.ntile * RA;
+                const int tile0 = n0 / kTileRows;
+                const int ntl = GLU ? 2 : min(2, (p.N - n0 + kTileRows - 1) / kTileRows);
+                const int row0 = row0s[w.e] + w.tt * kTcTok;
+                for (int b = 0; b < p.SB; ++b) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                        fail = true;
+                        break;
+                    }
+                    uint8_t* st = smem + stage * kTcStage;
+                    uint64_t* fb = &full[stage];
+                    filled |= 1u << stage;
+                    fph = (fph & ~(1u << stage)) | (phase << stage);
+                    mbar_arrive_expect_tx(fb, kTcStageTx + ntl * kBlockSB);
+                    tma_load_2d(st + kTcOffB, &p.b_map, fb, 128 * b, row0);
+                    tma_load_2d(st + kTcOffB + kTcAtom, &p.b_map, fb, 128 * b + 64, row0);
+                    bulk_load_hint(st + kTcOffW, pa->packed + (static_cast<size_t>(tile0) * p.SB + b) * kBlockSB,
+                                   kBlockSB, fb, pol);
+                    if (ntl == 2)
+                        bulk_load_hint(st + kTcOffW + kBlockSB,
+                                       GLU ? pb->packed + (static_cast<size_t>(tile0) * p.SB + b) * kBlockSB
+                                           : pa->packed + (static_cast<size_t>(tile0 + 1) * p.SB + b) * kBlockSB,
+                                       kBlockSB, fb, pol);
+                    tma_load_2d(st + kTcOffG, &p.g_map, fb, 4 * (b >> 1), row0);
+                    if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+                }
+                if (fail) break;
+                const int ra = pa->rank, rb = GLU ? pb->rank : 0;
+                if (p.has_t && (ra > 0 || rb > 0)) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                        fail = true;
+                        break;
+                    }
+                    uint8_t* st = smem + stage * kTcStage;
+                    uint64_t* fb = &full[stage];
+                    filled |= 1u << stage;
+                    fph = (fph & ~(1u << stage)) | (phase << stage);
+                    const int nbox = (p.tcols + 63) / 64;
+                    const int urows = min(RA, p.N - n0);
+                    const uint32_t ua = urows * ra * 2, ub = urows * rb * 2;
+                    mbar_arrive_expect_tx(fb, nbox * kTcAtom + ua + ub);
+                    for (int j = 0; j < nbox; ++j) tma_load_2d(st + kTcOffB + j * kTcAtom, &p.t_map, fb, 64 * j, row0);
+                    if (ua) bulk_load_hint(st + kTcOffUA, pa->U + static_cast<size_t>(n0) * ra, ua, fb, pol);
+                    if (ub) bulk_load_hint(st + kTcOffUB, pb->U + static_cast<size_t>(n0) * rb, ub, fb, pol);
+                    if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            // no copy may still be landing in shared memory when the CTA leaves
+            for (int s2 = 0; s2 < kTcStages; ++s2)
+                if (((filled >> s2) & 1u) && !mbar_wait(&full[s2], (fph >> s2) & 1u)) fail = true;
+            if (fail) flag(p.dev_status, MILO_DEV_TIMEOUT);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = f16_idesc(kTcRows, kTcTok);
+            int stage = 0, ab = 0, db = 0;
+            uint32_t phase = 0, aph = 0, dph = 0;
+            bool fail = false;
+            for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
+                const TcItem w = tc_decode(it, start, cnt, p.n_exp);
+                const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
+                const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
+                for (int b = 0; b < p.SB && !fail; ++b) {
+                    if (!mbar_wait(&full[stage], phase) || !mbar_wait(&afull[ab], aph)) {
+                        fail = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sb_addr = smem_u32(smem + stage * kTcStage) + kTcOffB;
+                    for (int h = 0; h < 2; ++h) {
+                        if (!mbar_wait(&dempty[db], dph ^ 1)) {
+                            fail = true;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t d_addr = tbase + kTcDCol + kTcTok * db;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            tc_mma_ts(d_addr, tbase + kTcACol + 64 * ab + 32 * h + 8 * q,
+                                      sw128_kmajor_desc(sb_addr + h * kTcAtom + 32 * q), idesc, q > 0 ? 1u : 0u);
+                        tc_commit(&dfull[db]);
+                        if (++db == 2) { db = 0; dph ^= 1; }
+                    }
+                    if (fail) break;
+                    tc_commit(&aempty[ab]);
+                    if (++ab == 2) { ab = 0; aph ^= 1; }
+                    tc_commit(&empty[stage]);
+                    if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+                }
+                if (fail) break;
+                const int ra = pa->rank, rb = GLU ? pb->rank : 0;
+                if (p.has_t && (ra > 0 || rb > 0)) {
+                    if (!mbar_wait(&full[stage], phase) || !mbar_wait(&afull[ab], aph) ||
+                        !mbar_wait(&dempty[db], dph ^ 1)) {
+                        fail = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t t_addr = smem_u32(smem + stage * kTcStage) + kTcOffB;
+                    const uint32_t d_addr = tbase + kTcDCol + kTcTok * db;
+                    const int steps = (p.tcols + 15) / 16;
+                    for (int q = 0; q < steps; ++q)
+                        tc_mma_ts(d_addr, tbase + kTcACol + 64 * ab + 8 * q,
+                                  sw128_kmajor_desc(t_addr + (q / 4) * kTcAtom + (q % 4) * 32), idesc,
+                                  q > 0 ? 1u : 0u);
+                    tc_commit(&dfull[db]);
+                    if (++db == 2) { db = 0; dph ^= 1; }
+                    tc_commit(&aempty[ab]);
+                    if (++ab == 2) { ab = 0; aph ^= 1; }
+                    tc_commit(&empty[stage]);
+                    if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (fail) flag(p.dev_status, MILO_DEV_TIMEOUT);
+            // every issued MMA has completed before TMEM is released
+            tc_commit(done_bar);
+            if (!mbar_wait(done_bar, 0)) flag(p.dev_status, MILO_DEV_TIMEOUT);
+        }
+    } else if (warp < 6) {
+        // ---------------------------------------------------------------- extraction (A operand)
+        const int quarter = warp & 3;
+        const int row = 32 * quarter + lane;               // TMEM lane = weight row of the item
+        const uint32_t lane_base = tbase + (static_cast<uint32_t>(32 * quarter) << 16);
+        const int half = row >> 6, r64 = row & 63;
+        int stage = 0, ab = 0;
+        uint32_t phase = 0, aph = 0;
+        bool fail = false;
+        for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
+            const TcItem w = tc_decode(it, start, cnt, p.n_exp);
+            const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
+            const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
+            for (int b = 0; b < p.SB; ++b) {
+                if (!warp_wait(&full[stage], phase)) {
+                    fail = true;
+                    break;
+                }
+                const uint8_t* st = smem + stage * kTcStage;
+                const uint4* qv = reinterpret_cast<const uint4*>(st + kTcOffW + half * kBlockSB + r64 * 48);
+                const uint4 v0 = qv[0], v1 = qv[1], v2 = qv[2];
+                uint32_t a[64];
+                tc_unit<0>(v0.x, v0.y, v0.z, a);
+                tc_unit<1>(v0.w, v1.x, v1.y, a);
+                tc_unit<2>(v1.z, v1.w, v2.x, a);
+                tc_unit<3>(v2.y, v2.z, v2.w, a);
+                if (!warp_wait(&aempty[ab], aph ^ 1)) {
+                    fail = true;
+                    break;
+                }
+                tc_fence_after();
+                tc_st64(lane_base + kTcACol + 64 * ab, a);
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&afull[ab]);
+                    mbar_arrive(&empty[stage]);
+                }
+                if (++ab == 2) { ab = 0; aph ^= 1; }
+                if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+            }
+            if (fail) break;
+            const int ra = pa->rank, rb = GLU ? pb->rank : 0;
+            if (p.has_t && (ra > 0 || rb > 0)) {
+                if (!warp_wait(&full[stage], phase)) {
+                    fail = true;
+                    break;
+                }
+                // this row's U values at the K slots of its projection's t columns
+                const uint8_t* st = smem + stage * kTcStage;
+                const uint16_t* src;
+                int lo, r;
+                if (GLU && row >= 64) {
+                    src = reinterpret_cast<const uint16_t*>(st + kTcOffUB) + (row - 64) * rb;
+                    lo = p.t_col_b;
+                    r = rb;
+                } else {
+                    src = reinterpret_cast<const uint16_t*>(st + kTcOffUA) + row * ra;
+                    lo = 0;
+                    r = ra;
+                }
+                uint32_t a[64];
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    const int slot = 2 * j;
+                    a[j] = (slot >= lo && slot < lo + r) ? *reinterpret_cast<const uint32_t*>(src + (slot - lo)) : 0u;
+                }
+                if (!warp_wait(&aempty[ab], aph ^ 1)) {
+                    fail = true;
+                    break;
+                }
+                tc_fence_after();
+                tc_st64(lane_base + kTcACol + 64 * ab, a);
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&afull[ab]);
+                    mbar_arrive(&empty[stage]);
+                }
+                if (++ab == 2) { ab = 0; aph ^= 1; }
+                if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+            }
+        }
+        if (fail && lane == 0) flag(p.dev_status, MILO_DEV_TIMEOUT);
+    } else {
+        // ---------------------------------------------------------------- fold + epilogue
+        const int quarter = warp & 3;
+        const int th = (warp - 6) >> 2;                    // routed rows 64 * th .. 64 * th + 63
+        const int row = 32 * quarter + lane;
+        const uint32_t lane_base = tbase + (static_cast<uint32_t>(32 * quarter) << 16);
+        const int tix = threadIdx.x - 192;                 // 0..255: one group sum to transpose
+        const int half = row >> 6, r64 = row & 63;
+        // byte offset of this row's (s, z) pair inside a group's 256 bytes
+        const int pair_off = (((r64 >> 4) * 8 + (r64 & 7)) * 4 + ((r64 >> 3) & 1) * 2) * 2;
+        int stage = 0, db = 0;
+        uint32_t phase = 0, dph = 0;
+        uint32_t xi = 0;        // items done: the exchange barriers complete one phase per item
+        uint32_t xrph = 0;      // per stage slot: parity of xready (used on code stages only)
+        bool fail = false;
+        int32_t st_bits = 0;
+        for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
+            const TcItem w = tc_decode(it, start, cnt, p.n_exp);
+            const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
+            const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
+            const int n0 = w.ntile * RA;
+            const int row0 = row0s[w.e] + w.tt * kTcTok;
+            const int ntok = min(kTcTok, cnt[w.e] - w.tt * kTcTok);
+            float2 acc[32];      // routed rows 64 * th + 2i, +1
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
+
+            for (int b = 0; b < p.SB; ++b) {
+                if (!warp_wait(&full[stage], phase)) {
+                    fail = true;
+                    break;
+                }
+                const uint8_t* st = smem + stage * kTcStage;
+                // transpose the super-block's two group sums: [row][4] -> [group][row]
+                float* X = xt + stage * 2 * kTcTok;
+                {
+                    const float* G = reinterpret_cast<const float*>(st + kTcOffG);
+                    const int tok = tix & (kTcTok - 1), gi = tix >> 7;
+                    X[gi * kTcTok + tok] = G[tok * 4 + 2 * (b & 1) + gi];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&xready[stage]);
+                    if (!warp_wait(&xready[stage], (xrph >> stage) & 1u)) {
+                        fail = true;
+                        break;
+                    }
+                    xrph ^= 1u << stage;
+                }
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t szv = *reinterpret_cast<const uint32_t*>(
+                        st + kTcOffW + half * kBlockSB + kQTileSBWords * 4 + h * kGroupBytes + pair_off);
+                    const float sv = __half2float(__ushort_as_half(static_cast<uint16_t>(szv & 0xFFFFu)));
+                    const float zv = __half2float(__ushort_as_half(static_cast<uint16_t>(szv >> 16)));
+                    const float s24 = sv * 16777216.0f, nsz = -sv * zv;
+                    if (!warp_wait(&dfull[db], dph)) {
+                        fail = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float2 s2 = make_float2(s24, s24), z2 = make_float2(nsz, nsz);
+                    const float4* Xh = reinterpret_cast<const float4*>(X + h * kTcTok + 64 * th);
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        uint32_t d[32];
+                        tc_ld<32>(lane_base + kTcDCol + kTcTok * db + 64 * th + 32 * j, d);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 xv = Xh[8 * j + i];
+                            float2& a0 = acc[16 * j + 2 * i];
+                            float2& a1 = acc[16 * j + 2 * i + 1];
+                            a0 = __ffma2_rn(s2, make_float2(__uint_as_float(d[4 * i]), __uint_as_float(d[4 * i + 1])), a0);
+                            a0 = __ffma2_rn(z2, make_float2(xv.x, xv.y), a0);
+                            a1 = __ffma2_rn(s2, make_float2(__uint_as_float(d[4 * i + 2]), __uint_as_float(d[4 * i + 3])), a1);
+                            a1 = __ffma2_rn(z2, make_float2(xv.z, xv.w), a1);
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&dempty[db]);
+                    if (++db == 2) { db = 0; dph ^= 1; }
+                }
+                if (fail) break;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
+                if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+            }
+            if (fail) break;
+            const int ra = pa->rank, rb = GLU ? pb->rank : 0;
+            if (p.has_t && (ra > 0 || rb > 0)) {
+                // the compensator stage holds nothing this warp reads: release it once filled
+                if (!warp_wait(&full[stage], phase)) {
+                    fail = true;
+                    break;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
+                if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+                if (!warp_wait(&dfull[db], dph)) {
+                    fail = true;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    uint32_t d[32];
+                    tc_ld<32>(lane_base + kTcDCol + kTcTok * db + 64 * th + 32 * j, d);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        acc[16 * j + i].x += __uint_as_float(d[2 * i]);
+                        acc[16 * j + i].y += __uint_as_float(d[2 * i + 1]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dempty[db]);
+                if (++db == 2) { db = 0; dph ^= 1; }
+            }
+
+            // ------------------------------------------------------------ epilogue
+            if constexpr (GLU) {
+                // rows 64..127 (w3) hand b to rows 0..63 (w1) through one buffer,
+                // round 0 for the warps with th == 0, then round 1.  Each round
+                // has its own barrier pair completing one phase per item; a w3
+                // warp first waits until the buffer's previous reader is done
+                // (round 1 of the previous item, or round 0 of this one).
+                if (row >= 64) {
+                    const bool ok = th == 0 ? warp_wait(&xempty[1], (xi + 1) & 1u) : warp_wait(&xempty[0], xi & 1u);
+                    if (!ok) {
+                        fail = true;
+                        break;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        xch[(2 * i) * 64 + (row - 64)] = acc[i].x;
+                        xch[(2 * i + 1) * 64 + (row - 64)] = acc[i].y;
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&xfull[th]);
+                } else {
+                    if (!warp_wait(&xfull[th], xi & 1u)) {
+                        fail = true;
+                        break;
+                    }
+                    const int f = n0 + row;
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        const int t = 64 * th + i;
+                        const float bv = xch[i * 64 + row];
+                        const float av = (i & 1) ? acc[i >> 1].y : acc[i >> 1].x;
+                        if (t < ntok && f < p.N) {
+                            const float hv = __fdividef(av, 1.0f + __expf(-av)) * bv;
+                            const __half hh = __float2half_rn(hv);
+                            if (!isfinite(hv)) st_bits |= MILO_DEV_NONFINITE;
+                            else if (__hisinf(hh)) st_bits |= MILO_DEV_FP16_RANGE;
+                            p.h[static_cast<size_t>(row0 + t) * p.N + f] = __half_as_ushort(hh);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&xempty[th]);
+                }
+                ++xi;
+            } else {
+                const int n = n0 + row;
+                if (n < p.N) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        const int t = 64 * th + i;
+                        if (t < ntok)
+                            p.y_part[static_cast<size_t>(row0 + t) * p.N + n] = (i & 1) ? acc[i >> 1].y : acc[i >> 1].x;
+                    }
+                }
+            }
+        }
+        if (fail) st_bits |= MILO_DEV_TIMEOUT;
+        flag(p.dev_status, st_bits);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, kTcTmemCols);
+    }
+}
+
+size_t tc_smem_bytes() { return kTcSmemBytes; }
+
+cudaError_t launch_tc_gemm(const TcParams& p, bool glu, int grid, cudaStream_t s) {
+    static bool configured[64][2] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !configured[dev][glu]) {
+        e = glu ? cudaFuncSetAttribute(tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes)
+                : cudaFuncSetAttribute(tc_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev][glu] = true;
+    }
+    // normal stream ordering, like the other persistent GEMM
+    if (glu) tc_gemm_kernel<true><<<grid, kTcThreads, kTcSmemBytes, s>>>(p);
+    else tc_gemm_kernel<false><<<grid, kTcThreads, kTcSmemBytes, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace milo

@@ -57,11 +57,31 @@ struct GemvParams {
     int has_t, tcols, t_col_b;  // LoRC activations present; row width; first column of w3's
 };
 
+// Parameters of the tcgen05 grouped GEMM for large per-expert row counts
+// (gemm_tc.cu).  Activations in MMA column order [R][K] fp16 and their group
+// sums [R][4 * chunks] f32 arrive by 2-D TMA; weights as blob blocks.
+struct TcParams {
+    CUtensorMap b_map;          // activations [R][K] fp16, box {64, 128}, 128-byte swizzle
+    CUtensorMap g_map;          // group sums [R][4 * chunks] f32, box {4, 128}
+    CUtensorMap t_map;          // LoRC down-projection [R][tcols] fp16, box {64, 128}, 128-byte swizzle
+    const ProjDev* table;
+    const int32_t* grp;
+    float* y_part;              // plain: [R][N] f32
+    uint16_t* h;                // SwiGLU: [R][N] fp16
+    int32_t* dev_status;
+    int stride, proj_a, proj_b;
+    int n_exp, N, K, R, SB;
+    int has_t, tcols, t_col_b;
+};
+
 struct PrepParams {
     const uint16_t* src;        // [*, K] bf16/fp16 (or fp16 h)
     int32_t* row_src;           // row p -> source row; built here when `rows` is set, else
                                 // read (NULL: identity); -1 = zero row
-    uint16_t* frag;             // [chunks][R][kFragRowHalves] fp16, chunks = ceil(K/256)
+    uint16_t* frag;             // layout 0: [chunks][R][kFragRowHalves] fp16, chunks = ceil(K/256);
+                                // layout 1: [R][K] fp16 in tcgen05 A-column order
+    float* gsum;                // layout 1: group sums [R][4 * chunks] f32
+    int layout;
     int32_t* dev_status;
     int R, K, src_bf16;
     // Row bookkeeping (first preparation of a call only): routed rows come from
@@ -97,6 +117,8 @@ struct CombineParams {
     int per_slot;               // 1: y row per flat slot (grouped linear), 0: per token
 };
 
+size_t tc_smem_bytes();
+cudaError_t launch_tc_gemm(const TcParams& p, bool glu, int grid, cudaStream_t s);
 size_t gemv_smem_bytes(bool glu);
 cudaError_t launch_gemv(const GemvParams& p, bool glu, int grid, cudaStream_t s);
 cudaError_t launch_prep(const PrepParams& p, cudaStream_t s);

@@ -30,6 +30,14 @@ def milo():
 
 
 
+@pytest.fixture(params=["mma", "tc"])
+def gemm_path(request, monkeypatch):
+    """Run a test on the mma.sync grouped GEMM (chosen for few rows per expert)
+    and on the tcgen05 one (chosen for many)."""
+    monkeypatch.setenv("MILO_GEMM", request.param)
+    return request.param
+
+
 def _status(st):
     torch.cuda.synchronize()
     return int(st.item())
@@ -164,14 +172,14 @@ def _linear_check(milo, projs, x_bits, x_dt, ids, k, out_dtypes=(torch.float32,)
     return err
 
 
-def test_linear_single_expert_decode_rank16(milo):
+def test_linear_single_expert_decode_rank16(milo, gemm_path):
     """1 token, W 1024x1024 with outliers, rank-16 compensator."""
     x, P = wl.single(seed_workload="t_single")
     _linear_check(milo, [P], x, "f16", np.zeros((1, 1), np.int32), 1,
                   (torch.float32, torch.float16, torch.bfloat16))
 
 
-def test_linear_ragged_rows_multi_token_tiles(milo):
+def test_linear_ragged_rows_multi_token_tiles(milo, gemm_path):
     """N = 208 (ragged last row tile), K = 384 (half-empty last K chunk),
     experts of rank 0 / 8 / 24, 53 tokens over 3 experts (one expert > 16 rows)."""
     projs = [wl.make_projection("t_rag", "w", e, 208, 384, r) for e, r in enumerate((0, 8, 24))]
@@ -180,20 +188,30 @@ def test_linear_ragged_rows_multi_token_tiles(milo):
     _linear_check(milo, projs, x, "bf16", ids, 1, (torch.float32, torch.float16))
 
 
-def test_linear_top2_slots_and_idle_experts(milo):
+def test_linear_top2_slots_and_idle_experts(milo, gemm_path):
     projs = [wl.make_projection("t_k2", "w", e, 256, 512, 16 * (e % 3)) for e in range(6)]
     x = wl.gen_activations(np.random.default_rng(10), 3, 512, "f16")
     ids = np.array([[4, 1], [1, 0], [4, 5]], np.int32)   # experts 2, 3 idle
     _linear_check(milo, projs, x, "f16", ids, 2)
 
 
-def test_linear_all_rows_one_expert(milo):
+def test_linear_all_rows_one_expert(milo, gemm_path):
     projs = [wl.make_projection("t_one", "w", e, 128, 256, 8) for e in range(4)]
     x = wl.gen_activations(np.random.default_rng(11), 70, 256, "bf16")
     _linear_check(milo, projs, x, "bf16", np.full((70, 1), 2, np.int32), 1)
 
 
-def test_linear_bad_ids_dropped_and_zero(milo):
+def test_linear_many_rows_per_expert(milo, gemm_path):
+    """300 rows over 2 experts (several 128-row tiles and a ragged one), N = 192
+    (one and a half 128-row weight tiles), K = 640 (odd number of super-blocks),
+    ranks 8 and 40."""
+    projs = [wl.make_projection("t_many", "w", e, 192, 640, r) for e, r in enumerate((8, 40))]
+    x = wl.gen_activations(np.random.default_rng(13), 300, 640, "bf16")
+    ids = np.random.default_rng(14).choice(2, size=(300, 1), p=[0.55, 0.45]).astype(np.int32)
+    _linear_check(milo, projs, x, "bf16", ids, 1, (torch.float32, torch.float16))
+
+
+def test_linear_bad_ids_dropped_and_zero(milo, gemm_path):
     projs = [wl.make_projection("t_bad", "w", e, 128, 256, 0) for e in range(2)]
     lin, ref = _linear_pair(milo, projs)
     x_bits = wl.gen_activations(np.random.default_rng(12), 3, 256, "f16")
@@ -275,18 +293,18 @@ def run_layer_parity(milo, wk, check_h=True, out_dtypes=(torch.float32,)):
     return err
 
 
-def test_moe_small_shared_expert(milo):
+def test_moe_small_shared_expert(milo, gemm_path):
     wk = wl.small_moe("t_moe1", T=5, hidden=256, inter=384, n_routed=4, n_shared=1, top_k=2)
     run_layer_parity(milo, wk, out_dtypes=(torch.float32, torch.bfloat16, torch.float16))
 
 
-def test_moe_small_no_compensator_full_softmax(milo):
+def test_moe_small_no_compensator_full_softmax(milo, gemm_path):
     wk = wl.small_moe("t_moe2", T=19, hidden=384, inter=256, n_routed=6, n_shared=0, top_k=3,
                       renorm=False, rank_choices=(0,), x_dtype="f16")
     run_layer_parity(milo, wk)
 
 
-def test_moe_small_many_tokens_per_expert(milo):
+def test_moe_small_many_tokens_per_expert(milo, gemm_path):
     wk = wl.small_moe("t_moe3", T=90, hidden=256, inter=512, n_routed=3, n_shared=2, top_k=1,
                       rank_choices=(8, 64))
     run_layer_parity(milo, wk)
