@@ -17,13 +17,13 @@
 //     A operand.
 //   - One thread of the MMA warp issues tcgen05.mma M=128, N=128, K=16 with A
 //     from TMEM and B from shared memory, per 64-code scale group into its own
-//     TMEM accumulator D_g (double-buffered).
+//     TMEM accumulator D_g (three in flight).
 //   - Eight fold warps (two per weight row: 64 routed rows and 64 fp32
 //     accumulators each) read D_g and fold acc += s * 2^24 * D_g - s * z * X_g
 //     (packed FFMA2),
 //     so the zero point and the scale cost nothing per weight and the result
-//     is exact to fp32 rounding.  The group sums X_g of a stage are transposed
-//     once in shared memory so that each fold thread reads them four at a time.
+//     is exact to fp32 rounding.  Each fold warp transposes its rows' group sums
+//     X_g of a stage in shared memory so that its threads read them four at a time.
 //   - The compensator is one more stage: A = U rows, B = t = x V^T.
 //   - Epilogue: SwiGLU through a shared-memory exchange (w3 rows hand b to the
 //     w1 rows), or the fp32 output rows.
@@ -41,6 +41,7 @@ namespace milo {
 constexpr int kTcTok = 128;                 // routed rows per item (MMA N)
 constexpr int kTcRows = 128;                // weight rows per item (MMA M)
 constexpr int kTcStages = 4;
+constexpr int kTcFoldWarpsX = 8;            // fold warps (each keeps its own transposed group sums)
 constexpr int kTcStage = 49152;             // bytes per stage (multiple of 1024)
 constexpr int kTcOffB = 0;                  // activations: 2 swizzled atoms [128 rows][128 B]
 constexpr int kTcAtom = kTcTok * 128;       // 16384
@@ -49,22 +50,24 @@ constexpr int kTcOffG = kTcOffW + 2 * kBlockSB;   // group sums [128 rows][4] f3
 constexpr int kTcStageTx = 2 * kTcAtom + kTcTok * 16;   // plus the blob blocks
 constexpr int kTcOffUA = kTcOffW;           // compensator stage: U rows of w1 (or 128 rows)
 constexpr int kTcOffUB = kTcOffW + 64 * MILO_MAX_RANK * 2;   // U rows of w3
-constexpr int kTcXT = kTcStages * kTcStage;             // transposed group sums [stage][2][128] f32
-constexpr int kTcXch = kTcXT + kTcStages * 2 * kTcTok * 4;   // SwiGLU exchange [64 rows][64 tokens] f32
+constexpr int kTcXT = kTcStages * kTcStage;             // per fold warp: group sums [2][64 rows] f32
+constexpr int kTcXch = kTcXT + kTcFoldWarpsX * 2 * 64 * 4;   // SwiGLU exchange [64 rows][64 tokens] f32
 constexpr int kTcBar = kTcXch + 64 * 64 * 4;
-constexpr int kTcNumBars = 3 * kTcStages + 2 * 2 + 2 * 2 + 1 + 4;   // + xready[stage], done, xfull[2], xempty[2]
+constexpr int kTcDBufs = 3;                // TMEM accumulators D_g in flight between MMA and fold
+constexpr int kTcNumBars = 2 * kTcStages + 2 * 2 + 2 * kTcDBufs + 1 + 4;   // + done, xfull[2], xempty[2]
 constexpr int kTcTab = kTcBar + 8 * kTcNumBars + 16;
 constexpr int kTcSmemUsed = kTcTab + 3 * (MILO_MAX_EXPERTS + 1) * 4;
 constexpr int kTcSmemBytes = kTcSmemUsed + 1024;        // slack to align the base to 1024 B
-constexpr int kTcFoldWarps = 8;             // two per TMEM lane quarter, 64 routed rows each
+constexpr int kTcFoldWarps = kTcFoldWarpsX;   // two per TMEM lane quarter, 64 routed rows each
 constexpr int kTcThreads = 32 * (2 + 4 + kTcFoldWarps);   // producer, MMA, extraction, fold
-constexpr uint32_t kTcTmemCols = 512;       // A: 2 x 64 columns, D: 2 x 128 columns
+constexpr uint32_t kTcTmemCols = 512;       // A: 2 x 64 columns, D: 3 x 128 columns
 constexpr int kTcACol = 0, kTcDCol = 128;
 
 static_assert(kTcOffG + kTcTok * 16 <= kTcStage, "stage layout");
 static_assert(kTcOffUB + 64 * MILO_MAX_RANK * 2 <= kTcStage, "compensator stage: U rows");
 static_assert(kTcOffUA + kTcRows * MILO_MAX_RANK * 2 <= kTcStage, "compensator stage: plain U rows");
 static_assert(kTcSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kTcDCol + kTcDBufs * kTcTok <= static_cast<int>(kTcTmemCols), "TMEM columns");
 
 struct TcItem {
     int e, ntile, tt;
@@ -126,12 +129,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     uint64_t* afull = empty + kTcStages;
     uint64_t* aempty = afull + 2;
     uint64_t* dfull = aempty + 2;
-    uint64_t* dempty = dfull + 2;
-    uint64_t* done_bar = dempty + 2;
+    uint64_t* dempty = dfull + kTcDBufs;
+    uint64_t* done_bar = dempty + kTcDBufs;
     uint64_t* xfull = done_bar + 1;      // [2] SwiGLU exchange, per round: w3 rows -> w1 rows
     uint64_t* xempty = xfull + 2;        // [2]
-    uint64_t* xready = xempty + 2;       // [kTcStages]: a stage's group sums are transposed
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xready + kTcStages);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + 2);
     int* start = reinterpret_cast<int*>(smem + kTcTab);
     int* cnt = start + (MILO_MAX_EXPERTS + 1);
     int* row0s = cnt + (MILO_MAX_EXPERTS + 1);
@@ -146,11 +148,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         for (int s = 0; s < kTcStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1 + 4 + kTcFoldWarps);   // MMA commit, extraction warps, fold warps
-            mbar_init(&xready[s], kTcFoldWarps);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&afull[b], 4);
             mbar_init(&aempty[b], 1);
+        }
+        for (int b = 0; b < kTcDBufs; ++b) {
             mbar_init(&dfull[b], 1);
             mbar_init(&dempty[b], kTcFoldWarps);
         }
@@ -287,7 +290,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                             tc_mma_ts(d_addr, tbase + kTcACol + 64 * ab + 32 * h + 8 * q,
                                       sw128_kmajor_desc(sb_addr + h * kTcAtom + 32 * q), idesc, q > 0 ? 1u : 0u);
                         tc_commit(&dfull[db]);
-                        if (++db == 2) { db = 0; dph ^= 1; }
+                        if (++db == kTcDBufs) { db = 0; dph ^= 1; }
                     }
                     if (fail) break;
                     tc_commit(&aempty[ab]);
@@ -312,7 +315,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                                   sw128_kmajor_desc(t_addr + (q / 4) * kTcAtom + (q % 4) * 32), idesc,
                                   q > 0 ? 1u : 0u);
                     tc_commit(&dfull[db]);
-                    if (++db == 2) { db = 0; dph ^= 1; }
+                    if (++db == kTcDBufs) { db = 0; dph ^= 1; }
                     tc_commit(&aempty[ab]);
                     if (++ab == 2) { ab = 0; aph ^= 1; }
                     tc_commit(&empty[stage]);
@@ -416,14 +419,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const int th = (warp - 6) >> 2;                    // routed rows 64 * th .. 64 * th + 63
         const int row = 32 * quarter + lane;
         const uint32_t lane_base = tbase + (static_cast<uint32_t>(32 * quarter) << 16);
-        const int tix = threadIdx.x - 192;                 // 0..255: one group sum to transpose
         const int half = row >> 6, r64 = row & 63;
         // byte offset of this row's (s, z) pair inside a group's 256 bytes
         const int pair_off = (((r64 >> 4) * 8 + (r64 & 7)) * 4 + ((r64 >> 3) & 1) * 2) * 2;
         int stage = 0, db = 0;
         uint32_t phase = 0, dph = 0;
         uint32_t xi = 0;        // items done: the exchange barriers complete one phase per item
-        uint32_t xrph = 0;      // per stage slot: parity of xready (used on code stages only)
         bool fail = false;
         int32_t st_bits = 0;
         for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
@@ -443,19 +444,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     break;
                 }
                 const uint8_t* st = smem + stage * kTcStage;
-                // transpose the super-block's two group sums: [row][4] -> [group][row]
-                float* X = xt + stage * 2 * kTcTok;
+                // this warp's copy of the super-block's two group sums for its 64
+                // routed rows: [row][4] -> [group][row]
+                float* X = xt + (warp - 6) * 2 * 64;
                 {
                     const float* G = reinterpret_cast<const float*>(st + kTcOffG);
-                    const int tok = tix & (kTcTok - 1), gi = tix >> 7;
-                    X[gi * kTcTok + tok] = G[tok * 4 + 2 * (b & 1) + gi];
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&xready[stage]);
-                    if (!warp_wait(&xready[stage], (xrph >> stage) & 1u)) {
-                        fail = true;
-                        break;
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int tl = 2 * lane + u;
+                        const float2 gv = *reinterpret_cast<const float2*>(G + (64 * th + tl) * 4 + 2 * (b & 1));
+                        X[tl] = gv.x;
+                        X[64 + tl] = gv.y;
                     }
-                    xrph ^= 1u << stage;
+                    __syncwarp();
                 }
                 for (int h = 0; h < 2; ++h) {
                     const uint32_t szv = *reinterpret_cast<const uint32_t*>(
@@ -469,7 +470,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     }
                     tc_fence_after();
                     const float2 s2 = make_float2(s24, s24), z2 = make_float2(nsz, nsz);
-                    const float4* Xh = reinterpret_cast<const float4*>(X + h * kTcTok + 64 * th);
+                    const float4* Xh = reinterpret_cast<const float4*>(X + h * 64);
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         uint32_t d[32];
@@ -489,10 +490,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&dempty[db]);
-                    if (++db == 2) { db = 0; dph ^= 1; }
+                    if (++db == kTcDBufs) { db = 0; dph ^= 1; }
                 }
                 if (fail) break;
-                __syncwarp();
+                __syncwarp();      // the warp's group-sum copy is rewritten next stage
                 if (lane == 0) mbar_arrive(&empty[stage]);
                 if (++stage == kTcStages) { stage = 0; phase ^= 1; }
             }
@@ -526,7 +527,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&dempty[db]);
-                if (++db == 2) { db = 0; dph ^= 1; }
+                if (++db == kTcDBufs) { db = 0; dph ^= 1; }
             }
 
             // ------------------------------------------------------------ epilogue
