@@ -136,8 +136,9 @@ static size_t frag_bytes(int K, int R) {
     // the mma.sync layout; the tcgen05 layout [R][K] fp16 is never larger
     return static_cast<size_t>(chunks_of(K)) * R * kFragRowHalves * 2;
 }
-// group sums of the tcgen05 path: [R][4 * chunks] f32
-static size_t gsum_bytes(int K, int R) { return static_cast<size_t>(chunks_of(K)) * R * 16; }
+// zero-point operand of the tcgen05 path: per row and pair of super-blocks,
+// the four group sums as fp16 (hi, lo, hi, lo): [R][chunks][16] fp16
+static size_t gsum_bytes(int K, int R) { return static_cast<size_t>(chunks_of(K)) * R * 32; }
 
 struct LorcPlan {
     int splits, row_groups;
@@ -279,7 +280,7 @@ static bool use_tc(long long routed_rows, int n_routed) {
 }
 
 // The grouped GEMM described by g on the tcgen05 kernel: activations in
-// A-column order [R][K] fp16 with group sums [R][4 * chunks] f32.
+// A-column order [R][K] fp16 with the zero-point operand [R][chunks][16] fp16.
 static milo_status run_tc(const GemvParams& g, bool glu, void* xcol, void* gsum, cudaStream_t st,
                           const char* what) {
     TcParams p;
@@ -290,8 +291,9 @@ static milo_status run_tc(const GemvParams& g, bool glu, void* xcol, void* gsum,
     if ((s = make_map(&p.b_map, xcol, CU_TENSOR_MAP_DATA_TYPE_UINT16, g.K, Rm, static_cast<uint64_t>(g.K) * 2, 64,
                       128, "activations", CU_TENSOR_MAP_SWIZZLE_128B)) != MILO_OK)
         return s;
-    if ((s = make_map(&p.g_map, gsum, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4 * chunks, Rm,
-                      static_cast<uint64_t>(chunks) * 16, 4, 128, "group sums")) != MILO_OK)
+    if ((s = make_map(&p.z_map, gsum, CU_TENSOR_MAP_DATA_TYPE_UINT16, 16 * chunks, Rm,
+                      static_cast<uint64_t>(chunks) * 32, 16, 128, "group sums",
+                      CU_TENSOR_MAP_SWIZZLE_32B)) != MILO_OK)
         return s;
     if (g.has_t && (s = make_map(&p.t_map, g.t, CU_TENSOR_MAP_DATA_TYPE_UINT16, g.tcols, Rm,
                                  static_cast<uint64_t>(g.tcols) * 2, 64, 128, "compensator rows",
@@ -449,7 +451,7 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
 
     const bool tc = use_tc(static_cast<long long>(T) * k, lin->n_experts);
     PrepParams pp{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.frag),
-                  reinterpret_cast<float*>(base + w.gsum), tc ? 1 : 0, dev_status, w.R, lin->K, x_dt == MILO_BF16,
+                  reinterpret_cast<uint16_t*>(base + w.gsum), tc ? 1 : 0, dev_status, w.R, lin->K, x_dt == MILO_BF16,
                   1, expert_offsets, perm, grp, inv, T, k, lin->n_experts, 0, w.R};
     milo_status s = check_cuda(launch_prep(pp, st), "prep");
     if (s != MILO_OK) return s;
@@ -519,7 +521,7 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
 
     const bool tc = use_tc(w.R_routed, L->n_routed);
     PrepParams px{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.xfrag),
-                  reinterpret_cast<float*>(base + w.xg), tc ? 1 : 0, dev_status, w.R, H, x_dt == MILO_BF16, 1,
+                  reinterpret_cast<uint16_t*>(base + w.xg), tc ? 1 : 0, dev_status, w.R, H, x_dt == MILO_BF16, 1,
                   expert_offsets, perm, grp, nullptr, T, L->top_k, L->n_routed, L->n_shared, w.R_routed};
     if ((s = check_cuda(launch_prep(px, st), "prep x")) != MILO_OK) return s;
     if (has_t) {
@@ -552,7 +554,7 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     prof_record(1, st);
 
     PrepParams ph{reinterpret_cast<const uint16_t*>(base + w.h), nullptr,
-                  reinterpret_cast<uint16_t*>(base + w.hfrag), reinterpret_cast<float*>(base + w.hg), tc ? 1 : 0,
+                  reinterpret_cast<uint16_t*>(base + w.hfrag), reinterpret_cast<uint16_t*>(base + w.hg), tc ? 1 : 0,
                   dev_status, w.R, I, 0, 0, nullptr, nullptr, nullptr, nullptr, 0, 0, 0, 0, 0};
     if ((s = check_cuda(launch_prep(ph, st), "prep h")) != MILO_OK) return s;
     if (has_t) {

@@ -165,9 +165,22 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
             o2[0] = make_uint4(f4.x, f4.y, f5.x, f5.y);
             o2[1] = make_uint4(f6.x, f6.y, f7.x, f7.y);
             if (c == 0) {
-                const size_t gp = static_cast<size_t>(row) * 4 * ((SB + 1) / 2) + 2 * sb;
-                p.gsum[gp] = s0;
-                p.gsum[gp + 1] = s1;
+                // the two group sums split exactly enough into fp16 hi + lo
+                // (2^-22 relative), slots (hi, lo, hi, lo) per group; a pair of
+                // super-blocks shares 16 slots, the odd tail's second half is 0
+                uint32_t v[4];
+                const float gs[2] = {s0, s1};
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    const __half hi = __float2half_rn(gs[g]);
+                    const __half lo = __float2half_rn(gs[g] - __half2float(hi));
+                    if (__hisinf(hi)) st |= MILO_DEV_FP16_RANGE;
+                    v[2 * g] = v[2 * g + 1] =
+                        static_cast<uint32_t>(__half_as_ushort(hi)) | (static_cast<uint32_t>(__half_as_ushort(lo)) << 16);
+                }
+                uint4* zp = reinterpret_cast<uint4*>(p.gsum + (static_cast<size_t>(row) * ((SB + 1) / 2) + (sb >> 1)) * 16);
+                zp[sb & 1] = make_uint4(v[0], v[1], v[2], v[3]);
+                if (sb == SB - 1 && !(sb & 1)) zp[1] = make_uint4(0u, 0u, 0u, 0u);
             }
             continue;
         }

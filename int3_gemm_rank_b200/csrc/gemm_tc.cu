@@ -10,20 +10,23 @@
 //   - A work item is (expert, 128 weight rows, 128 routed rows); a stage is
 //     one 128-code super-block.  The producer warp brings the activations
 //     (2-D TMA, 128-byte swizzle: the K-major B operand), the two 64-row
-//     blob blocks (1-D bulk copies: codes, scales, zeros) and the group sums.
+//     blob blocks (1-D bulk copies: codes, scales, zeros) and, on the second
+//     stage of each super-block pair, the pair's group-sum tile.
 //   - Four extraction warps (one thread per weight row) turn the row's 32
 //     code pairs into exact fp16 patterns code * 2^e * 2^-24 (one LOP3 per
 //     pair, the 2^e folded into the activations) and store them to TMEM: the
-//     A operand.
+//     A operand.  They also write -s_g * z_g of the row's groups, split into
+//     fp16 hi + lo, to shared memory (32-byte swizzle).
 //   - One thread of the MMA warp issues tcgen05.mma M=128, N=128, K=16 with A
 //     from TMEM and B from shared memory, per 64-code scale group into its own
-//     TMEM accumulator D_g (three in flight).
+//     TMEM accumulator D_g (double-buffered), and once per super-block pair a
+//     zero-point step Z += (-s z)_hi,lo x (X_g)_hi,lo over the pair's four
+//     groups (four K slots each: the four hi/lo cross products).
 //   - Eight fold warps (two per weight row: 64 routed rows and 64 fp32
-//     accumulators each) read D_g and fold acc += s * 2^24 * D_g - s * z * X_g
-//     (packed FFMA2),
-//     so the zero point and the scale cost nothing per weight and the result
-//     is exact to fp32 rounding.  Each fold warp transposes its rows' group sums
-//     X_g of a stage in shared memory so that its threads read them four at a time.
+//     accumulators each) read D_g and fold acc += s * 2^24 * D_g (packed
+//     FFMA2), then add Z once per item, so the scale and the zero point cost
+//     no per-weight work; -s z splits exactly, X_g to 2^-22 relative, and
+//     the rest is fp32 accumulation.
 //   - The compensator is one more stage: A = U rows, B = t = x V^T.
 //   - Epilogue: SwiGLU through a shared-memory exchange (w3 rows hand b to the
 //     w1 rows), or the fp32 output rows.
@@ -41,33 +44,37 @@ namespace milo {
 constexpr int kTcTok = 128;                 // routed rows per item (MMA N)
 constexpr int kTcRows = 128;                // weight rows per item (MMA M)
 constexpr int kTcStages = 4;
-constexpr int kTcFoldWarpsX = 8;            // fold warps (each keeps its own transposed group sums)
 constexpr int kTcStage = 49152;             // bytes per stage (multiple of 1024)
 constexpr int kTcOffB = 0;                  // activations: 2 swizzled atoms [128 rows][128 B]
 constexpr int kTcAtom = kTcTok * 128;       // 16384
 constexpr int kTcOffW = 2 * kTcAtom;        // two blob blocks (rows 0-63, 64-127)
-constexpr int kTcOffG = kTcOffW + 2 * kBlockSB;   // group sums [128 rows][4] f32
-constexpr int kTcStageTx = 2 * kTcAtom + kTcTok * 16;   // plus the blob blocks
+// zero-point step, once per pair of super-blocks (four groups, four K slots
+// each): B = group sums X_g as fp16 hi, lo (routed rows), A = -s*z as fp16
+// hi, lo (weight rows); both [128 rows][32 B] with the 32-byte swizzle
+constexpr int kTcOffZB = 40960;
+constexpr int kTcOffZA = 45056;
+constexpr int kTcZTile = kTcTok * 32;
+constexpr int kTcStageTx = 2 * kTcAtom;     // plus the blob blocks (and the B_z tile)
 constexpr int kTcOffUA = kTcOffW;           // compensator stage: U rows of w1 (or 128 rows)
 constexpr int kTcOffUB = kTcOffW + 64 * MILO_MAX_RANK * 2;   // U rows of w3
-constexpr int kTcXT = kTcStages * kTcStage;             // per fold warp: group sums [2][64 rows] f32
-constexpr int kTcXch = kTcXT + kTcFoldWarpsX * 2 * 64 * 4;   // SwiGLU exchange [64 rows][64 tokens] f32
+constexpr int kTcXch = kTcStages * kTcStage;             // SwiGLU exchange [64 rows][64 tokens] f32
 constexpr int kTcBar = kTcXch + 64 * 64 * 4;
-constexpr int kTcDBufs = 3;                // TMEM accumulators D_g in flight between MMA and fold
-constexpr int kTcNumBars = 2 * kTcStages + 2 * 2 + 2 * kTcDBufs + 1 + 4;   // + done, xfull[2], xempty[2]
+constexpr int kTcDBufs = 2;                // TMEM accumulators D_g in flight between MMA and fold
+constexpr int kTcNumBars = 2 * kTcStages + 2 * 2 + 2 * kTcDBufs + 1 + 4 + 1;   // + done, xfull[2], xempty[2], zempty
 constexpr int kTcTab = kTcBar + 8 * kTcNumBars + 16;
 constexpr int kTcSmemUsed = kTcTab + 3 * (MILO_MAX_EXPERTS + 1) * 4;
 constexpr int kTcSmemBytes = kTcSmemUsed + 1024;        // slack to align the base to 1024 B
-constexpr int kTcFoldWarps = kTcFoldWarpsX;   // two per TMEM lane quarter, 64 routed rows each
+constexpr int kTcFoldWarps = 8;             // two per TMEM lane quarter, 64 routed rows each
 constexpr int kTcThreads = 32 * (2 + 4 + kTcFoldWarps);   // producer, MMA, extraction, fold
-constexpr uint32_t kTcTmemCols = 512;       // A: 2 x 64 columns, D: 3 x 128 columns
-constexpr int kTcACol = 0, kTcDCol = 128;
+constexpr uint32_t kTcTmemCols = 512;       // A: 2 x 64 columns, D_g: 2 x 128, Z: 128
+constexpr int kTcACol = 0, kTcDCol = 128, kTcZCol = kTcDCol + kTcDBufs * kTcTok;
 
-static_assert(kTcOffG + kTcTok * 16 <= kTcStage, "stage layout");
+static_assert(kTcOffW + 2 * kBlockSB <= kTcOffZB && kTcOffZB + kTcZTile <= kTcOffZA, "stage layout");
+static_assert(kTcOffZA + kTcZTile <= kTcStage && kTcOffZB % 1024 == 0 && kTcOffZA % 1024 == 0, "stage layout");
 static_assert(kTcOffUB + 64 * MILO_MAX_RANK * 2 <= kTcStage, "compensator stage: U rows");
 static_assert(kTcOffUA + kTcRows * MILO_MAX_RANK * 2 <= kTcStage, "compensator stage: plain U rows");
 static_assert(kTcSmemBytes <= 227 * 1024, "shared memory");
-static_assert(kTcDCol + kTcDBufs * kTcTok <= static_cast<int>(kTcTmemCols), "TMEM columns");
+static_assert(kTcZCol + kTcTok <= static_cast<int>(kTcTmemCols), "TMEM columns");
 
 struct TcItem {
     int e, ntile, tt;
@@ -133,11 +140,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     uint64_t* done_bar = dempty + kTcDBufs;
     uint64_t* xfull = done_bar + 1;      // [2] SwiGLU exchange, per round: w3 rows -> w1 rows
     uint64_t* xempty = xfull + 2;        // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + 2);
+    uint64_t* zempty = xempty + 2;       // the fold warps have read the item's Z accumulator
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(zempty + 1);
     int* start = reinterpret_cast<int*>(smem + kTcTab);
     int* cnt = start + (MILO_MAX_EXPERTS + 1);
     int* row0s = cnt + (MILO_MAX_EXPERTS + 1);
-    float* xt = reinterpret_cast<float*>(smem + kTcXT);
     float* xch = reinterpret_cast<float*>(smem + kTcXch);
 
     constexpr int RA = GLU ? kRowsGlu : kRowsPlain;   // output features per item
@@ -158,6 +165,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             mbar_init(&dempty[b], kTcFoldWarps);
         }
         mbar_init(done_bar, 1);
+        mbar_init(zempty, kTcFoldWarps);
         for (int rd = 0; rd < 2; ++rd) {
             mbar_init(&xfull[rd], 2);    // the two w3 fold warps of the round
             mbar_init(&xempty[rd], 2);   // the two w1 fold warps of the round
@@ -221,7 +229,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     uint64_t* fb = &full[stage];
                     filled |= 1u << stage;
                     fph = (fph & ~(1u << stage)) | (phase << stage);
-                    mbar_arrive_expect_tx(fb, kTcStageTx + ntl * kBlockSB);
+                    const bool zs = (b & 1) || b == p.SB - 1;    // last stage of a super-block pair
+                    mbar_arrive_expect_tx(fb, kTcStageTx + ntl * kBlockSB + (zs ? kTcZTile : 0));
                     tma_load_2d(st + kTcOffB, &p.b_map, fb, 128 * b, row0);
                     tma_load_2d(st + kTcOffB + kTcAtom, &p.b_map, fb, 128 * b + 64, row0);
                     bulk_load_hint(st + kTcOffW, pa->packed + (static_cast<size_t>(tile0) * p.SB + b) * kBlockSB,
@@ -231,7 +240,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                                        GLU ? pb->packed + (static_cast<size_t>(tile0) * p.SB + b) * kBlockSB
                                            : pa->packed + (static_cast<size_t>(tile0 + 1) * p.SB + b) * kBlockSB,
                                        kBlockSB, fb, pol);
-                    tma_load_2d(st + kTcOffG, &p.g_map, fb, 4 * (b >> 1), row0);
+                    if (zs) tma_load_2d(st + kTcOffZB, &p.z_map, fb, 16 * (b >> 1), row0);
                     if (++stage == kTcStages) { stage = 0; phase ^= 1; }
                 }
                 if (fail) break;
@@ -265,7 +274,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         if (lane == 0) {
             const uint32_t idesc = f16_idesc(kTcRows, kTcTok);
             int stage = 0, ab = 0, db = 0;
-            uint32_t phase = 0, aph = 0, dph = 0;
+            uint32_t phase = 0, aph = 0, dph = 0, zph = 0;
             bool fail = false;
             for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
                 const TcItem w = tc_decode(it, start, cnt, p.n_exp);
@@ -278,6 +287,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     }
                     tc_fence_after();
                     const uint32_t sb_addr = smem_u32(smem + stage * kTcStage) + kTcOffB;
+                    const bool zs = (b & 1) || b == p.SB - 1;
                     for (int h = 0; h < 2; ++h) {
                         if (!mbar_wait(&dempty[db], dph ^ 1)) {
                             fail = true;
@@ -289,6 +299,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         for (int q = 0; q < 4; ++q)
                             tc_mma_ts(d_addr, tbase + kTcACol + 64 * ab + 32 * h + 8 * q,
                                       sw128_kmajor_desc(sb_addr + h * kTcAtom + 32 * q), idesc, q > 0 ? 1u : 0u);
+                        if (h == 1 && zs) {
+                            // zero-point step of the pair into Z; the first one of an
+                            // item waits until the fold has read the previous item's Z.
+                            // Committed with this group's D_g, so a fold warp that saw
+                            // the item's last D_g may read Z.
+                            if (b < 2) {
+                                if (!mbar_wait(zempty, zph ^ 1)) {
+                                    fail = true;
+                                    break;
+                                }
+                                zph ^= 1;
+                                tc_fence_after();
+                            }
+                            tc_mma_ss(tbase + kTcZCol, sw32_kmajor_desc(sb_addr - kTcOffB + kTcOffZA),
+                                      sw32_kmajor_desc(sb_addr - kTcOffB + kTcOffZB), idesc, b >= 2 ? 1u : 0u);
+                        }
                         tc_commit(&dfull[db]);
                         if (++db == kTcDBufs) { db = 0; dph ^= 1; }
                     }
@@ -333,9 +359,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const int row = 32 * quarter + lane;               // TMEM lane = weight row of the item
         const uint32_t lane_base = tbase + (static_cast<uint32_t>(32 * quarter) << 16);
         const int half = row >> 6, r64 = row & 63;
+        // byte offset of this row's (s, z) pair inside a group's 256 bytes
+        const int pair_off = (((r64 >> 4) * 8 + (r64 & 7)) * 4 + ((r64 >> 3) & 1) * 2) * 2;
         int stage = 0, ab = 0;
         uint32_t phase = 0, aph = 0;
         bool fail = false;
+        int32_t st_bits = 0;
+        uint4 zprev = make_uint4(0u, 0u, 0u, 0u);   // A_z slots of the pair's first super-block
         for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
             const TcItem w = tc_decode(it, start, cnt, p.n_exp);
             const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
@@ -353,6 +383,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 tc_unit<1>(v0.w, v1.x, v1.y, a);
                 tc_unit<2>(v1.z, v1.w, v2.x, a);
                 tc_unit<3>(v2.y, v2.z, v2.w, a);
+                // -s*z of the two groups, split exactly into fp16 hi + lo, in the
+                // K slots (hi, hi, lo, lo) that meet (X hi, X lo, X hi, X lo)
+                uint32_t zw[4];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t szv = *reinterpret_cast<const uint32_t*>(
+                        st + kTcOffW + half * kBlockSB + kQTileSBWords * 4 + h * kGroupBytes + pair_off);
+                    const float c = -__half2float(__ushort_as_half(static_cast<uint16_t>(szv & 0xFFFFu))) *
+                                    __half2float(__ushort_as_half(static_cast<uint16_t>(szv >> 16)));
+                    const __half hi = __float2half_rn(c);
+                    const __half lo = __float2half_rn(c - __half2float(hi));
+                    if (__hisinf(hi)) st_bits |= MILO_DEV_FP16_RANGE;
+                    zw[2 * h] = static_cast<uint32_t>(__half_as_ushort(hi)) * 0x10001u;
+                    zw[2 * h + 1] = static_cast<uint32_t>(__half_as_ushort(lo)) * 0x10001u;
+                }
+                const bool zs = (b & 1) || b == p.SB - 1;
+                if (zs) {
+                    uint8_t* za = smem + stage * kTcStage + kTcOffZA;
+                    const uint4 cur = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+                    const bool second = b & 1;
+                    *reinterpret_cast<uint4*>(za + sw32_offset(row, 0)) = second ? zprev : cur;
+                    *reinterpret_cast<uint4*>(za + sw32_offset(row, 1)) = second ? cur : make_uint4(0u, 0u, 0u, 0u);
+                    fence_proxy_async_smem();
+                } else {
+                    zprev = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+                }
                 if (!warp_wait(&aempty[ab], aph ^ 1)) {
                     fail = true;
                     break;
@@ -412,7 +468,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 if (++stage == kTcStages) { stage = 0; phase ^= 1; }
             }
         }
-        if (fail && lane == 0) flag(p.dev_status, MILO_DEV_TIMEOUT);
+        if (fail) st_bits |= MILO_DEV_TIMEOUT;
+        flag(p.dev_status, st_bits);
     } else {
         // ---------------------------------------------------------------- fold + epilogue
         const int quarter = warp & 3;
@@ -444,48 +501,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     break;
                 }
                 const uint8_t* st = smem + stage * kTcStage;
-                // this warp's copy of the super-block's two group sums for its 64
-                // routed rows: [row][4] -> [group][row]
-                float* X = xt + (warp - 6) * 2 * 64;
-                {
-                    const float* G = reinterpret_cast<const float*>(st + kTcOffG);
+                float s24[2];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int tl = 2 * lane + u;
-                        const float2 gv = *reinterpret_cast<const float2*>(G + (64 * th + tl) * 4 + 2 * (b & 1));
-                        X[tl] = gv.x;
-                        X[64 + tl] = gv.y;
-                    }
-                    __syncwarp();
-                }
+                for (int h = 0; h < 2; ++h)
+                    s24[h] = 16777216.0f * __half2float(*reinterpret_cast<const __half*>(
+                                               st + kTcOffW + half * kBlockSB + kQTileSBWords * 4 + h * kGroupBytes +
+                                               pair_off));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
+                if (++stage == kTcStages) { stage = 0; phase ^= 1; }
                 for (int h = 0; h < 2; ++h) {
-                    const uint32_t szv = *reinterpret_cast<const uint32_t*>(
-                        st + kTcOffW + half * kBlockSB + kQTileSBWords * 4 + h * kGroupBytes + pair_off);
-                    const float sv = __half2float(__ushort_as_half(static_cast<uint16_t>(szv & 0xFFFFu)));
-                    const float zv = __half2float(__ushort_as_half(static_cast<uint16_t>(szv >> 16)));
-                    const float s24 = sv * 16777216.0f, nsz = -sv * zv;
                     if (!warp_wait(&dfull[db], dph)) {
                         fail = true;
                         break;
                     }
                     tc_fence_after();
-                    const float2 s2 = make_float2(s24, s24), z2 = make_float2(nsz, nsz);
-                    const float4* Xh = reinterpret_cast<const float4*>(X + h * 64);
+                    const float2 s2 = make_float2(s24[h], s24[h]);
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         uint32_t d[32];
                         tc_ld<32>(lane_base + kTcDCol + kTcTok * db + 64 * th + 32 * j, d);
                         tc_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float4 xv = Xh[8 * j + i];
-                            float2& a0 = acc[16 * j + 2 * i];
-                            float2& a1 = acc[16 * j + 2 * i + 1];
-                            a0 = __ffma2_rn(s2, make_float2(__uint_as_float(d[4 * i]), __uint_as_float(d[4 * i + 1])), a0);
-                            a0 = __ffma2_rn(z2, make_float2(xv.x, xv.y), a0);
-                            a1 = __ffma2_rn(s2, make_float2(__uint_as_float(d[4 * i + 2]), __uint_as_float(d[4 * i + 3])), a1);
-                            a1 = __ffma2_rn(z2, make_float2(xv.z, xv.w), a1);
-                        }
+                        for (int i = 0; i < 16; ++i)
+                            acc[16 * j + i] = __ffma2_rn(
+                                s2, make_float2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])), acc[16 * j + i]);
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -493,11 +533,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     if (++db == kTcDBufs) { db = 0; dph ^= 1; }
                 }
                 if (fail) break;
-                __syncwarp();      // the warp's group-sum copy is rewritten next stage
-                if (lane == 0) mbar_arrive(&empty[stage]);
-                if (++stage == kTcStages) { stage = 0; phase ^= 1; }
             }
             if (fail) break;
+            // the zero-point sums Z = sum_g (-s_g z_g) X_g: the last D_g's commit
+            // covered the item's last zero-point step
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                uint32_t d[32];
+                tc_ld<32>(lane_base + kTcZCol + 64 * th + 32 * j, d);
+                tc_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    acc[16 * j + i].x += __uint_as_float(d[2 * i]);
+                    acc[16 * j + i].y += __uint_as_float(d[2 * i + 1]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(zempty);
             const int ra = pa->rank, rb = GLU ? pb->rank : 0;
             if (p.has_t && (ra > 0 || rb > 0)) {
                 // the compensator stage holds nothing this warp reads: release it once filled

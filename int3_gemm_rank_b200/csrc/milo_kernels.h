@@ -62,7 +62,7 @@ struct GemvParams {
 // sums [R][4 * chunks] f32 arrive by 2-D TMA; weights as blob blocks.
 struct TcParams {
     CUtensorMap b_map;          // activations [R][K] fp16, box {64, 128}, 128-byte swizzle
-    CUtensorMap g_map;          // group sums [R][4 * chunks] f32, box {4, 128}
+    CUtensorMap z_map;          // group sums [R][chunks][16] fp16 (hi, lo, hi, lo per group), box {16, 128}
     CUtensorMap t_map;          // LoRC down-projection [R][tcols] fp16, box {64, 128}, 128-byte swizzle
     const ProjDev* table;
     const int32_t* grp;
@@ -80,7 +80,7 @@ struct PrepParams {
                                 // read (NULL: identity); -1 = zero row
     uint16_t* frag;             // layout 0: [chunks][R][kFragRowHalves] fp16, chunks = ceil(K/256);
                                 // layout 1: [R][K] fp16 in tcgen05 A-column order
-    float* gsum;                // layout 1: group sums [R][4 * chunks] f32
+    uint16_t* gsum;             // layout 1: group sums [R][chunks][16] fp16: per group (hi, lo, hi, lo)
     int layout;
     int32_t* dev_status;
     int R, K, src_bf16;

@@ -103,6 +103,24 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
     return d;
 }
 
+// The same for a K-major tile with 32-byte rows and the 32-byte swizzle
+// (16-byte halves of a row exchanged on rows 4..7 of each 8-row group): one
+// k16 step of 128 rows, 8-row groups 256 bytes apart.
+__device__ __forceinline__ uint64_t sw32_kmajor_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1) << 16;
+    d |= static_cast<uint64_t>(256 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(6) << 61;                     // 32-byte swizzle
+    return d;
+}
+
+// Byte offset of 16-byte half H (0, 1) of row R inside such a tile.
+__host__ __device__ constexpr int sw32_offset(int r, int h) {
+    return (r >> 3) * 256 + (r & 7) * 32 + ((h ^ ((r >> 2) & 1)) << 4);
+}
+
 // Instruction descriptor: D f32, A and B f16, both K-major, M x N.
 __host__ __device__ constexpr uint32_t f16_idesc(int M, int N) {
     return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
@@ -118,6 +136,20 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_addr, uint32_t a_addr, uint
 }
 
 // Named barrier among `count` threads (a subset of the CTA).
+// D[tmem] (+)= A[smem] * B[smem]^T, one k16 step; issued by one thread.
+__device__ __forceinline__ void tc_mma_ss(uint32_t d_addr, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_addr), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// Generic-proxy writes to shared memory made visible to the tensor core (async proxy).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
