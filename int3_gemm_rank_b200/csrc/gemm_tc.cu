@@ -207,7 +207,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
-        if (lane == 0) {
+        // the whole warp runs the loop; one elected lane issues the copies
+        {
             const uint64_t pol = l2_evict_first();
             int stage = 0;
             uint32_t phase = 0, filled = 0, fph = 0;
@@ -221,7 +222,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 const int ntl = GLU ? 2 : min(2, (p.N - n0 + kTileRows - 1) / kTileRows);
                 const int row0 = row0s[w.e] + w.tt * kTcTok;
                 for (int b = 0; b < p.SB; ++b) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                    if (!warp_wait(&empty[stage], phase ^ 1)) {
                         fail = true;
                         break;
                     }
@@ -230,23 +231,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     filled |= 1u << stage;
                     fph = (fph & ~(1u << stage)) | (phase << stage);
                     const bool zs = (b & 1) || b == p.SB - 1;    // last stage of a super-block pair
-                    mbar_arrive_expect_tx(fb, kTcStageTx + ntl * kBlockSB + (zs ? kTcZTile : 0));
-                    tma_load_2d(st + kTcOffB, &p.b_map, fb, 128 * b, row0);
-                    tma_load_2d(st + kTcOffB + kTcAtom, &p.b_map, fb, 128 * b + 64, row0);
-                    bulk_load_hint(st + kTcOffW, pa->packed + (static_cast<size_t>(tile0) * p.SB + b) * kBlockSB,
-                                   kBlockSB, fb, pol);
-                    if (ntl == 2)
-                        bulk_load_hint(st + kTcOffW + kBlockSB,
-                                       GLU ? pb->packed + (static_cast<size_t>(tile0) * p.SB + b) * kBlockSB
-                                           : pa->packed + (static_cast<size_t>(tile0 + 1) * p.SB + b) * kBlockSB,
-                                       kBlockSB, fb, pol);
-                    if (zs) tma_load_2d(st + kTcOffZB, &p.z_map, fb, 16 * (b >> 1), row0);
+                    const uint8_t* w0 = pa->packed + (static_cast<size_t>(tile0) * p.SB + b) * kBlockSB;
+                    const uint8_t* w1 = GLU ? pb->packed + (static_cast<size_t>(tile0) * p.SB + b) * kBlockSB
+                                            : w0 + static_cast<size_t>(p.SB) * kBlockSB;
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(fb, kTcStageTx + ntl * kBlockSB + (zs ? kTcZTile : 0));
+                        tma_load_2d(st + kTcOffB, &p.b_map, fb, 128 * b, row0);
+                        tma_load_2d(st + kTcOffB + kTcAtom, &p.b_map, fb, 128 * b + 64, row0);
+                        bulk_load_hint(st + kTcOffW, w0, kBlockSB, fb, pol);
+                        if (ntl == 2) bulk_load_hint(st + kTcOffW + kBlockSB, w1, kBlockSB, fb, pol);
+                        if (zs) tma_load_2d(st + kTcOffZB, &p.z_map, fb, 16 * (b >> 1), row0);
+                    }
+                    __syncwarp();
                     if (++stage == kTcStages) { stage = 0; phase ^= 1; }
                 }
                 if (fail) break;
                 const int ra = pa->rank, rb = GLU ? pb->rank : 0;
                 if (p.has_t && (ra > 0 || rb > 0)) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                    if (!warp_wait(&empty[stage], phase ^ 1)) {
                         fail = true;
                         break;
                     }
@@ -257,21 +259,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     const int nbox = (p.tcols + 63) / 64;
                     const int urows = min(RA, p.N - n0);
                     const uint32_t ua = urows * ra * 2, ub = urows * rb * 2;
-                    mbar_arrive_expect_tx(fb, nbox * kTcAtom + ua + ub);
-                    for (int j = 0; j < nbox; ++j) tma_load_2d(st + kTcOffB + j * kTcAtom, &p.t_map, fb, 64 * j, row0);
-                    if (ua) bulk_load_hint(st + kTcOffUA, pa->U + static_cast<size_t>(n0) * ra, ua, fb, pol);
-                    if (ub) bulk_load_hint(st + kTcOffUB, pb->U + static_cast<size_t>(n0) * rb, ub, fb, pol);
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(fb, nbox * kTcAtom + ua + ub);
+                        for (int j = 0; j < nbox; ++j)
+                            tma_load_2d(st + kTcOffB + j * kTcAtom, &p.t_map, fb, 64 * j, row0);
+                        if (ua) bulk_load_hint(st + kTcOffUA, pa->U + static_cast<size_t>(n0) * ra, ua, fb, pol);
+                        if (ub) bulk_load_hint(st + kTcOffUB, pb->U + static_cast<size_t>(n0) * rb, ub, fb, pol);
+                    }
+                    __syncwarp();
                     if (++stage == kTcStages) { stage = 0; phase ^= 1; }
                 }
             }
             // no copy may still be landing in shared memory when the CTA leaves
             for (int s2 = 0; s2 < kTcStages; ++s2)
-                if (((filled >> s2) & 1u) && !mbar_wait(&full[s2], (fph >> s2) & 1u)) fail = true;
-            if (fail) flag(p.dev_status, MILO_DEV_TIMEOUT);
+                if (((filled >> s2) & 1u) && !warp_wait(&full[s2], (fph >> s2) & 1u)) fail = true;
+            if (fail && lane == 0) flag(p.dev_status, MILO_DEV_TIMEOUT);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // the whole warp runs the loop (uniform operands); one lane issues
+        {
             const uint32_t idesc = f16_idesc(kTcRows, kTcTok);
             int stage = 0, ab = 0, db = 0;
             uint32_t phase = 0, aph = 0, dph = 0, zph = 0;
@@ -281,7 +288,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
                 const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
                 for (int b = 0; b < p.SB && !fail; ++b) {
-                    if (!mbar_wait(&full[stage], phase) || !mbar_wait(&afull[ab], aph)) {
+                    if (!warp_wait(&full[stage], phase) || !warp_wait(&afull[ab], aph)) {
                         fail = true;
                         break;
                     }
@@ -289,7 +296,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     const uint32_t sb_addr = smem_u32(smem + stage * kTcStage) + kTcOffB;
                     const bool zs = (b & 1) || b == p.SB - 1;
                     for (int h = 0; h < 2; ++h) {
-                        if (!mbar_wait(&dempty[db], dph ^ 1)) {
+                        if (!warp_wait(&dempty[db], dph ^ 1)) {
                             fail = true;
                             break;
                         }
@@ -305,7 +312,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                             // Committed with this group's D_g, so a fold warp that saw
                             // the item's last D_g may read Z.
                             if (b < 2) {
-                                if (!mbar_wait(zempty, zph ^ 1)) {
+                                if (!warp_wait(zempty, zph ^ 1)) {
                                     fail = true;
                                     break;
                                 }
@@ -327,8 +334,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 if (fail) break;
                 const int ra = pa->rank, rb = GLU ? pb->rank : 0;
                 if (p.has_t && (ra > 0 || rb > 0)) {
-                    if (!mbar_wait(&full[stage], phase) || !mbar_wait(&afull[ab], aph) ||
-                        !mbar_wait(&dempty[db], dph ^ 1)) {
+                    if (!warp_wait(&full[stage], phase) || !warp_wait(&afull[ab], aph) ||
+                        !warp_wait(&dempty[db], dph ^ 1)) {
                         fail = true;
                         break;
                     }
@@ -348,10 +355,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     if (++stage == kTcStages) { stage = 0; phase ^= 1; }
                 }
             }
-            if (fail) flag(p.dev_status, MILO_DEV_TIMEOUT);
+            if (fail && lane == 0) flag(p.dev_status, MILO_DEV_TIMEOUT);
             // every issued MMA has completed before TMEM is released
             tc_commit(done_bar);
-            if (!mbar_wait(done_bar, 0)) flag(p.dev_status, MILO_DEV_TIMEOUT);
+            if (!warp_wait(done_bar, 0) && lane == 0) flag(p.dev_status, MILO_DEV_TIMEOUT);
         }
     } else if (warp < 6) {
         // ---------------------------------------------------------------- extraction (A operand)

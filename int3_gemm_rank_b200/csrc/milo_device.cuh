@@ -171,6 +171,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// True in one lane of a converged warp (the same lane every time).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t e;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(e));
+    return e != 0;
+}
+
 // The same, decided for the whole warp: every lane returns the same answer,
 // so the warp never splits on a timeout ahead of a warp-collective step.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {

@@ -126,22 +126,30 @@ __host__ __device__ constexpr uint32_t f16_idesc(int M, int N) {
     return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T, one k16 step; issued by one thread.
+// The MMA helpers below are called by all 32 lanes of the issuing warp with
+// warp-uniform operands, and one lane chosen by elect.sync issues the
+// instruction.  (Issued from a divergent single-lane branch, the operands
+// live in per-thread registers and every tcgen05.mma costs about three times
+// the tensor core's own 64 cycles for M = 128, N = 128, K = 16.)
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, one k16 step.
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_addr, uint32_t a_addr, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
         ::"r"(d_addr), "r"(a_addr), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
 // Named barrier among `count` threads (a subset of the CTA).
-// D[tmem] (+)= A[smem] * B[smem]^T, one k16 step; issued by one thread.
+// D[tmem] (+)= A[smem] * B[smem]^T, one k16 step.
 __device__ __forceinline__ void tc_mma_ss(uint32_t d_addr, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d_addr), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
@@ -154,10 +162,11 @@ __device__ __forceinline__ void named_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// The mbarrier receives one arrival when every MMA this thread issued so far
-// has completed.
+// The mbarrier receives one arrival when every MMA the elected lane issued
+// so far has completed (elect.sync picks the same lane every time).
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
                  ::"r"(smem_u32(bar)) : "memory");
 }
 
