@@ -289,14 +289,14 @@ static milo_status run_tc(const GemvParams& g, bool glu, void* xcol, void* gsum,
     const int Rm = std::max(g.R, 1);
     const int chunks = chunks_of(g.K);
     if ((s = make_map(&p.b_map, xcol, CU_TENSOR_MAP_DATA_TYPE_UINT16, g.K, Rm, static_cast<uint64_t>(g.K) * 2, 64,
-                      128, "activations", CU_TENSOR_MAP_SWIZZLE_128B)) != MILO_OK)
+                      kTcTokens, "activations", CU_TENSOR_MAP_SWIZZLE_128B)) != MILO_OK)
         return s;
     if ((s = make_map(&p.z_map, gsum, CU_TENSOR_MAP_DATA_TYPE_UINT16, 16 * chunks, Rm,
-                      static_cast<uint64_t>(chunks) * 32, 16, 128, "group sums",
+                      static_cast<uint64_t>(chunks) * 32, 16, kTcTokens, "group sums",
                       CU_TENSOR_MAP_SWIZZLE_32B)) != MILO_OK)
         return s;
     if (g.has_t && (s = make_map(&p.t_map, g.t, CU_TENSOR_MAP_DATA_TYPE_UINT16, g.tcols, Rm,
-                                 static_cast<uint64_t>(g.tcols) * 2, 64, 128, "compensator rows",
+                                 static_cast<uint64_t>(g.tcols) * 2, 64, kTcTokens, "compensator rows",
                                  CU_TENSOR_MAP_SWIZZLE_128B)) != MILO_OK)
         return s;
     p.table = g.table;

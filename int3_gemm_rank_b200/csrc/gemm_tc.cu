@@ -7,7 +7,7 @@
 // with dequantisation and the asymmetric zero point fused in ("MiLo Kernel").
 //
 // Design (B200):
-//   - A work item is (expert, 128 weight rows, 128 routed rows); a stage is
+//   - A work item is (expert, 128 weight rows, kTcTok routed rows); a stage is
 //     one 128-code super-block.  The producer warp brings the activations
 //     (2-D TMA, 128-byte swizzle: the K-major B operand), the two 64-row
 //     blob blocks (1-D bulk copies: codes, scales, zeros) and, on the second
@@ -17,19 +17,20 @@
 //     pair, the 2^e folded into the activations) and store them to TMEM: the
 //     A operand.  They also write -s_g * z_g of the row's groups, split into
 //     fp16 hi + lo, to shared memory (32-byte swizzle).
-//   - One thread of the MMA warp issues tcgen05.mma M=128, N=128, K=16 with A
-//     from TMEM and B from shared memory, per 64-code scale group into its own
-//     TMEM accumulator D_g (double-buffered), and once per super-block pair a
+//   - The MMA warp issues tcgen05.mma M=128, N=kTcTok, K=16 (one elected lane)
+//     with A from TMEM and B from shared memory, per 64-code scale group into
+//     its own TMEM accumulator D_g (several in flight), and once per pair a
 //     zero-point step Z += (-s z)_hi,lo x (X_g)_hi,lo over the pair's four
 //     groups (four K slots each: the four hi/lo cross products).
-//   - Eight fold warps (two per weight row: 64 routed rows and 64 fp32
+//   - Eight fold warps (two per weight row: kTcTok / 2 routed rows and fp32
 //     accumulators each) read D_g and fold acc += s * 2^24 * D_g (packed
 //     FFMA2), then add Z once per item, so the scale and the zero point cost
 //     no per-weight work; -s z splits exactly, X_g to 2^-22 relative, and
 //     the rest is fp32 accumulation.
 //   - The compensator is one more stage: A = U rows, B = t = x V^T.
-//   - Epilogue: SwiGLU through a shared-memory exchange (w3 rows hand b to the
-//     w1 rows), or the fp32 output rows.
+//   - Epilogue: SwiGLU through a shared-memory exchange between the w1 and w3
+//     rows of each output feature (each side finishes half the tokens), or
+//     the fp32 output rows.
 //   - Every wait is bounded; on a timeout the kernel flags MILO_DEV_TIMEOUT,
 //     drains its copies and MMAs and frees TMEM before leaving.
 #include <cuda_runtime.h>
@@ -41,36 +42,43 @@
 
 namespace milo {
 
-constexpr int kTcTok = 128;                 // routed rows per item (MMA N)
+constexpr int kTcTok = kTcTokens;           // routed rows per item (MMA N)
+constexpr int kTcHalf = kTcTok / 2;         // routed rows per fold warp
 constexpr int kTcRows = 128;                // weight rows per item (MMA M)
-constexpr int kTcStages = 4;
-constexpr int kTcStage = 49152;             // bytes per stage (multiple of 1024)
-constexpr int kTcOffB = 0;                  // activations: 2 swizzled atoms [128 rows][128 B]
-constexpr int kTcAtom = kTcTok * 128;       // 16384
+constexpr int kTcAlign(int b) { return (b + 1023) / 1024 * 1024; }
+constexpr int kTcOffB = 0;                  // activations: 2 swizzled atoms [kTcTok rows][128 B]
+constexpr int kTcAtom = kTcTok * 128;
 constexpr int kTcOffW = 2 * kTcAtom;        // two blob blocks (rows 0-63, 64-127)
 // zero-point step, once per pair of super-blocks (four groups, four K slots
-// each): B = group sums X_g as fp16 hi, lo (routed rows), A = -s*z as fp16
-// hi, lo (weight rows); both [128 rows][32 B] with the 32-byte swizzle
-constexpr int kTcOffZB = 40960;
-constexpr int kTcOffZA = 45056;
+// each): B = group sums X_g as fp16 hi, lo [kTcTok routed rows][32 B], A =
+// -s*z as fp16 hi, lo [128 weight rows][32 B], both with the 32-byte swizzle
+constexpr int kTcOffZB = kTcAlign(kTcOffW + 2 * kBlockSB);
 constexpr int kTcZTile = kTcTok * 32;
+constexpr int kTcOffZA = kTcAlign(kTcOffZB + kTcZTile);
+constexpr int kTcZATile = kTcRows * 32;
 constexpr int kTcStageTx = 2 * kTcAtom;     // plus the blob blocks (and the B_z tile)
 constexpr int kTcOffUA = kTcOffW;           // compensator stage: U rows of w1 (or 128 rows)
 constexpr int kTcOffUB = kTcOffW + 64 * MILO_MAX_RANK * 2;   // U rows of w3
-constexpr int kTcXch = kTcStages * kTcStage;             // SwiGLU exchange [64 rows][64 tokens] f32
-constexpr int kTcBar = kTcXch + 64 * 64 * 4;
-constexpr int kTcDBufs = 2;                // TMEM accumulators D_g in flight between MMA and fold
+constexpr int kTcMax(int a, int b) { return a > b ? a : b; }
+constexpr int kTcStage = kTcAlign(kTcMax(kTcOffZA + kTcZATile, kTcOffUA + kTcRows * MILO_MAX_RANK * 2));   // bytes per stage
+constexpr int kTcStages = kTcTok == 128 ? 3 : 4;
+constexpr int kTcXch = kTcStages * kTcStage;             // SwiGLU exchange, per token half: [48 tokens][64 rows] f32
+constexpr int kTcXchHalf = kTcHalf * 64;                  // floats per half
+constexpr int kTcBar = kTcXch + 2 * kTcXchHalf * 4;
+constexpr int kTcDBufs = (512 - 128 - kTcTok) / kTcTok;   // TMEM accumulators D_g in flight between MMA and fold
 constexpr int kTcNumBars = 2 * kTcStages + 2 * 2 + 2 * kTcDBufs + 1 + 4 + 1;   // + done, xfull[2], xempty[2], zempty
 constexpr int kTcTab = kTcBar + 8 * kTcNumBars + 16;
 constexpr int kTcSmemUsed = kTcTab + 3 * (MILO_MAX_EXPERTS + 1) * 4;
 constexpr int kTcSmemBytes = kTcSmemUsed + 1024;        // slack to align the base to 1024 B
-constexpr int kTcFoldWarps = 8;             // two per TMEM lane quarter, 64 routed rows each
+constexpr int kTcFoldWarps = 8;             // two per TMEM lane quarter, kTcHalf routed rows each
 constexpr int kTcThreads = 32 * (2 + 4 + kTcFoldWarps);   // producer, MMA, extraction, fold
-constexpr uint32_t kTcTmemCols = 512;       // A: 2 x 64 columns, D_g: 2 x 128, Z: 128
+constexpr uint32_t kTcTmemCols = 512;       // A: 2 x 64 columns, D_g: kTcDBufs x kTcTok, Z: kTcTok
 constexpr int kTcACol = 0, kTcDCol = 128, kTcZCol = kTcDCol + kTcDBufs * kTcTok;
 
 static_assert(kTcOffW + 2 * kBlockSB <= kTcOffZB && kTcOffZB + kTcZTile <= kTcOffZA, "stage layout");
-static_assert(kTcOffZA + kTcZTile <= kTcStage && kTcOffZB % 1024 == 0 && kTcOffZA % 1024 == 0, "stage layout");
+static_assert(kTcOffZA + kTcZATile <= kTcStage && kTcOffZB % 1024 == 0 && kTcOffZA % 1024 == 0, "stage layout");
+static_assert(kTcAtom % 1024 == 0 && kTcTok % 32 == 0 && kTcHalf % 16 == 0, "tile shapes");
+static_assert(kTcDCol % 32 == 0 && kTcTok % 32 == 0 && kTcZCol % 32 == 0, "accumulator columns");
 static_assert(kTcOffUB + 64 * MILO_MAX_RANK * 2 <= kTcStage, "compensator stage: U rows");
 static_assert(kTcOffUA + kTcRows * MILO_MAX_RANK * 2 <= kTcStage, "compensator stage: plain U rows");
 static_assert(kTcSmemBytes <= 227 * 1024, "shared memory");
@@ -127,6 +135,24 @@ __device__ __forceinline__ void tc_unit(uint32_t w0, uint32_t w1, uint32_t w2, u
     tc_unit_reg<C, 15>(w, hw, a);
 }
 
+// A fold warp reads its kTcHalf accumulator columns in chunks of kTcChunk
+// (48: three x16 loads in flight; 32: one x32 load), the caller waiting with
+// tc_wait_ld.
+constexpr int kTcChunk = kTcHalf % 32 == 0 ? 32 : 48;
+constexpr int kTcChunks = kTcHalf / kTcChunk;
+static_assert(kTcHalf % kTcChunk == 0, "fold chunks");
+
+template <int C>
+__device__ __forceinline__ void tc_ld_chunk(uint32_t taddr, uint32_t (&d)[C]) {
+    if constexpr (C == 32) {
+        tc_ld<32>(taddr, d);
+    } else {
+        tc_ld<16>(taddr, reinterpret_cast<uint32_t(&)[16]>(d[0]));
+        tc_ld<16>(taddr + 16, reinterpret_cast<uint32_t(&)[16]>(d[16]));
+        tc_ld<16>(taddr + 32, reinterpret_cast<uint32_t(&)[16]>(d[32]));
+    }
+}
+
 template <bool GLU>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -138,7 +164,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     uint64_t* dfull = aempty + 2;
     uint64_t* dempty = dfull + kTcDBufs;
     uint64_t* done_bar = dempty + kTcDBufs;
-    uint64_t* xfull = done_bar + 1;      // [2] SwiGLU exchange, per round: w3 rows -> w1 rows
+    uint64_t* xfull = done_bar + 1;      // [2] SwiGLU exchange, per token half: w3 rows -> w1 rows
     uint64_t* xempty = xfull + 2;        // [2]
     uint64_t* zempty = xempty + 2;       // the fold warps have read the item's Z accumulator
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(zempty + 1);
@@ -167,8 +193,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         mbar_init(done_bar, 1);
         mbar_init(zempty, kTcFoldWarps);
         for (int rd = 0; rd < 2; ++rd) {
-            mbar_init(&xfull[rd], 2);    // the two w3 fold warps of the round
-            mbar_init(&xempty[rd], 2);   // the two w1 fold warps of the round
+            mbar_init(&xfull[rd], 4);    // the four fold warps of the token half
+            mbar_init(&xempty[rd], 4);
         }
         fence_barrier_init();
     }
@@ -377,6 +403,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             const TcItem w = tc_decode(it, start, cnt, p.n_exp);
             const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
             const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
+            // a plain item's second 64-row block is not loaded when the tile
+            // ends first: those rows compute garbage that is never stored
+            const bool live = GLU || w.ntile * RA + 64 * half < p.N;
             for (int b = 0; b < p.SB; ++b) {
                 if (!warp_wait(&full[stage], phase)) {
                     fail = true;
@@ -397,8 +426,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 for (int h = 0; h < 2; ++h) {
                     const uint32_t szv = *reinterpret_cast<const uint32_t*>(
                         st + kTcOffW + half * kBlockSB + kQTileSBWords * 4 + h * kGroupBytes + pair_off);
-                    const float c = -__half2float(__ushort_as_half(static_cast<uint16_t>(szv & 0xFFFFu))) *
-                                    __half2float(__ushort_as_half(static_cast<uint16_t>(szv >> 16)));
+                    const float c = live ? -__half2float(__ushort_as_half(static_cast<uint16_t>(szv & 0xFFFFu))) *
+                                               __half2float(__ushort_as_half(static_cast<uint16_t>(szv >> 16)))
+                                         : 0.0f;
                     const __half hi = __float2half_rn(c);
                     const __half lo = __float2half_rn(c - __half2float(hi));
                     if (__hisinf(hi)) st_bits |= MILO_DEV_FP16_RANGE;
@@ -480,7 +510,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     } else {
         // ---------------------------------------------------------------- fold + epilogue
         const int quarter = warp & 3;
-        const int th = (warp - 6) >> 2;                    // routed rows 64 * th .. 64 * th + 63
+        const int th = (warp - 6) >> 2;                    // routed rows 48 * th .. 48 * th + 47
         const int row = 32 * quarter + lane;
         const uint32_t lane_base = tbase + (static_cast<uint32_t>(32 * quarter) << 16);
         const int half = row >> 6, r64 = row & 63;
@@ -498,9 +528,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             const int n0 = w.ntile * RA;
             const int row0 = row0s[w.e] + w.tt * kTcTok;
             const int ntok = min(kTcTok, cnt[w.e] - w.tt * kTcTok);
-            float2 acc[32];      // routed rows 64 * th + 2i, +1
+            float2 acc[kTcHalf / 2];      // routed rows kTcHalf * th + 2i, +1
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
+            for (int i = 0; i < kTcHalf / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
 
             for (int b = 0; b < p.SB; ++b) {
                 if (!warp_wait(&full[stage], phase)) {
@@ -524,19 +554,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     }
                     tc_fence_after();
                     const float2 s2 = make_float2(s24[h], s24[h]);
+                    const uint32_t dcol = lane_base + kTcDCol + kTcTok * db + kTcHalf * th;
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        uint32_t d[32];
-                        tc_ld<32>(lane_base + kTcDCol + kTcTok * db + 64 * th + 32 * j, d);
+                    for (int j = 0; j < kTcChunks; ++j) {
+                        uint32_t d[kTcChunk];
+                        tc_ld_chunk(dcol + kTcChunk * j, d);
                         tc_wait_ld();
+                        if (j == kTcChunks - 1) {
+                            // the last values are in registers: hand the buffer back first
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&dempty[db]);
+                        }
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            acc[16 * j + i] = __ffma2_rn(
-                                s2, make_float2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])), acc[16 * j + i]);
+                        for (int i = 0; i < kTcChunk / 2; ++i)
+                            acc[kTcChunk / 2 * j + i] = __ffma2_rn(
+                                s2, make_float2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])),
+                                acc[kTcChunk / 2 * j + i]);
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&dempty[db]);
                     if (++db == kTcDBufs) { db = 0; dph ^= 1; }
                 }
                 if (fail) break;
@@ -545,14 +580,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             // the zero-point sums Z = sum_g (-s_g z_g) X_g: the last D_g's commit
             // covered the item's last zero-point step
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                uint32_t d[32];
-                tc_ld<32>(lane_base + kTcZCol + 64 * th + 32 * j, d);
+            for (int j = 0; j < kTcChunks; ++j) {
+                uint32_t d[kTcChunk];
+                tc_ld_chunk(lane_base + kTcZCol + kTcHalf * th + kTcChunk * j, d);
                 tc_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    acc[16 * j + i].x += __uint_as_float(d[2 * i]);
-                    acc[16 * j + i].y += __uint_as_float(d[2 * i + 1]);
+                for (int i = 0; i < kTcChunk / 2; ++i) {
+                    acc[kTcChunk / 2 * j + i].x += __uint_as_float(d[2 * i]);
+                    acc[kTcChunk / 2 * j + i].y += __uint_as_float(d[2 * i + 1]);
                 }
             }
             tc_fence_before();
@@ -574,14 +609,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 }
                 tc_fence_after();
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    uint32_t d[32];
-                    tc_ld<32>(lane_base + kTcDCol + kTcTok * db + 64 * th + 32 * j, d);
+                for (int j = 0; j < kTcChunks; ++j) {
+                    uint32_t d[kTcChunk];
+                    tc_ld_chunk(lane_base + kTcDCol + kTcTok * db + kTcHalf * th + kTcChunk * j, d);
                     tc_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        acc[16 * j + i].x += __uint_as_float(d[2 * i]);
-                        acc[16 * j + i].y += __uint_as_float(d[2 * i + 1]);
+                    for (int i = 0; i < kTcChunk / 2; ++i) {
+                        acc[kTcChunk / 2 * j + i].x += __uint_as_float(d[2 * i]);
+                        acc[kTcChunk / 2 * j + i].y += __uint_as_float(d[2 * i + 1]);
                     }
                 }
                 tc_fence_before();
@@ -592,35 +627,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 
             // ------------------------------------------------------------ epilogue
             if constexpr (GLU) {
-                // rows 64..127 (w3) hand b to rows 0..63 (w1) through one buffer,
-                // round 0 for the warps with th == 0, then round 1.  Each round
-                // has its own barrier pair completing one phase per item; a w3
-                // warp first waits until the buffer's previous reader is done
-                // (round 1 of the previous item, or round 0 of this one).
-                if (row >= 64) {
-                    const bool ok = th == 0 ? warp_wait(&xempty[1], (xi + 1) & 1u) : warp_wait(&xempty[0], xi & 1u);
-                    if (!ok) {
-                        fail = true;
-                        break;
-                    }
+                // SwiGLU h = silu(a) * b for output feature n0 + c: a is in TMEM
+                // lane c (w1 row), b in lane 64 + c (w3 row), different warps.  Per
+                // token half th the four warps of the half swap through their own
+                // buffer [48 tokens][64 columns]: the w3 warps post b of the
+                // first 24 tokens, the w1 warps a of the last 24, then each side
+                // finishes its 24 tokens.  xfull / xempty (four arrivals) complete
+                // one phase per item.
+                const bool is_w1 = row < 64;
+                const int c = row & 63;
+                float* R = xch + th * kTcXchHalf;
+                if (!warp_wait(&xempty[th], (xi + 1) & 1u)) {
+                    fail = true;
+                    break;
+                }
+                const int post0 = is_w1 ? kTcHalf / 2 : 0;     // tokens this side posts
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        xch[(2 * i) * 64 + (row - 64)] = acc[i].x;
-                        xch[(2 * i + 1) * 64 + (row - 64)] = acc[i].y;
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&xfull[th]);
-                } else {
-                    if (!warp_wait(&xfull[th], xi & 1u)) {
-                        fail = true;
-                        break;
-                    }
-                    const int f = n0 + row;
+                for (int i = 0; i < kTcHalf / 4; ++i) {
+                    const float2 v = is_w1 ? acc[kTcHalf / 4 + i] : acc[i];
+                    R[(post0 + 2 * i) * 64 + c] = v.x;
+                    R[(post0 + 2 * i + 1) * 64 + c] = v.y;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xfull[th]);
+                if (!warp_wait(&xfull[th], xi & 1u)) {
+                    fail = true;
+                    break;
+                }
+                const int own0 = is_w1 ? 0 : kTcHalf / 2;       // tokens this side finishes
+                const int f = n0 + c;
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        const int t = 64 * th + i;
-                        const float bv = xch[i * 64 + row];
-                        const float av = (i & 1) ? acc[i >> 1].y : acc[i >> 1].x;
+                for (int i = 0; i < kTcHalf / 4; ++i) {
+                    const float2 mine = is_w1 ? acc[i] : acc[kTcHalf / 4 + i];   // tokens own0 + 2i, +1
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int tl = own0 + 2 * i + u;
+                        const float other = R[tl * 64 + c];
+                        const float own = u ? mine.y : mine.x;
+                        const float av = is_w1 ? own : other;
+                        const float bv = is_w1 ? other : own;
+                        const int t = kTcHalf * th + tl;
                         if (t < ntok && f < p.N) {
                             const float hv = __fdividef(av, 1.0f + __expf(-av)) * bv;
                             const __half hh = __float2half_rn(hv);
@@ -629,16 +675,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                             p.h[static_cast<size_t>(row0 + t) * p.N + f] = __half_as_ushort(hh);
                         }
                     }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&xempty[th]);
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xempty[th]);
                 ++xi;
             } else {
                 const int n = n0 + row;
                 if (n < p.N) {
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        const int t = 64 * th + i;
+                    for (int i = 0; i < kTcHalf; ++i) {
+                        const int t = kTcHalf * th + i;
                         if (t < ntok)
                             p.y_part[static_cast<size_t>(row0 + t) * p.N + n] = (i & 1) ? acc[i >> 1].y : acc[i >> 1].x;
                     }

@@ -33,6 +33,7 @@ constexpr int kTileRows = 64;
 constexpr int kQTileSBWords = kTileRows * 12;       // codes of one tile, one super-block: 3072 bytes
 constexpr int kGroupBytes = kTileRows * 2 * 2;      // scales and zeros of one tile, one group: 256 bytes
 constexpr int kBlockSB = kQTileSBWords * 4 + 2 * kGroupBytes;   // 3584
+constexpr int kTcTokens = 128;               // routed rows per tcgen05 work item (the TMA box height)
 
 // One projection in the device table (device pointers and shape).
 struct alignas(64) ProjDev {
