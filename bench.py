@@ -203,29 +203,56 @@ def layer_bytes(wk, counts) -> dict:
     w2_kernel = w2["weights"] + w2["lorc_u"] + act_h + rows * H * 4
     step = (glu["weights"] + glu["lorc_u"] + glu["lorc_v"] + w2["weights"] + w2["lorc_u"] + w2["lorc_v"]
             + wk.T * H * 2 + act_x + 2 * act_h + wk.T * H * 2)
+    # tensor work of the two GEMM launches: the int3 contraction plus the
+    # compensator's up-projection t U^T (the down-projection x V^T runs
+    # in its own kernel)
+    r_glu = sum(int(counts[e]) * (wk.experts[e]["w1"].rank + wk.experts[e]["w3"].rank)
+                for e in range(wk.n_routed) if counts[e] > 0)
+    r_glu += sum(wk.T * (wk.experts[e]["w1"].rank + wk.experts[e]["w3"].rank)
+                 for e in range(wk.n_routed, wk.n_experts))
+    r_w2 = sum(int(counts[e]) * wk.experts[e]["w2"].rank for e in range(wk.n_routed) if counts[e] > 0)
+    r_w2 += sum(wk.T * wk.experts[e]["w2"].rank for e in range(wk.n_routed, wk.n_experts))
+    glu_flops = 2 * rows * (2 * I) * H + 2 * r_glu * I
+    w2_flops = 2 * rows * H * I + 2 * r_w2 * H
     return {"glu_kernel": glu_kernel, "w2_kernel": w2_kernel, "step": step,
-            "weights_only": glu["weights"] + w2["weights"], "active_experts": len(active), "rows": rows}
+            "weights_only": glu["weights"] + w2["weights"], "active_experts": len(active), "rows": rows,
+            "glu_flops": glu_flops, "w2_flops": w2_flops,
+            "routed_rows": int(sum(counts[:wk.n_routed])), "n_routed": wk.n_routed}
+
+
+def uses_tensor_path(bytes_) -> bool:
+    """The library's choice of grouped GEMM: the tcgen05 kernel once the
+    routed rows reach 64 per routed expert on average (MILO_GEMM=mma|tc
+    overrides it), else the mma.sync kernel."""
+    forced = os.environ.get("MILO_GEMM", "")
+    if forced in ("mma", "tc"):
+        return forced == "tc"
+    return bytes_["routed_rows"] >= 64 * bytes_["n_routed"]
 
 
 def peaks() -> dict:
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]), "source": "measured"}
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
     except (OSError, KeyError, ValueError):
-        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(tensor: bool = False) -> str:
+    """Hash of the sources the profiled GEMM kernel is built from."""
     h = hashlib.sha256()
-    for rel in ("int3_gemm_rank_b200/csrc/gemv.cu", "int3_gemm_rank_b200/csrc/milo_device.cuh",
-                "int3_gemm_rank_b200/csrc/milo_kernels.h"):
+    files = ("int3_gemm_rank_b200/csrc/gemm_tc.cu", "int3_gemm_rank_b200/csrc/milo_tc.cuh") if tensor else \
+        ("int3_gemm_rank_b200/csrc/gemv.cu",)
+    for rel in files + ("int3_gemm_rank_b200/csrc/milo_device.cuh", "int3_gemm_rank_b200/csrc/milo_kernels.h"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(name: str):
+def profiled_traffic(name: str, tensor: bool = False):
     """DRAM bytes per launch of the GEMM kernel from the committed ncu summary,
     or None when the summary is missing or the kernel source changed since."""
     path = os.path.join(ROOT, "profiles", name)
@@ -236,7 +263,7 @@ def profiled_traffic(name: str):
                 if ":" in line and line.startswith("- "):
                     k, v = line[2:].split(":", 1)
                     kv[k.strip()] = v.strip()
-        if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+        if kv.get("kernel_source_sha256_16") != kernel_source_hash(tensor):
             return None
         return float(kv["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
@@ -400,7 +427,7 @@ def run_milo(args):
     # route, prep x, lorc w1|w3 (partial + reduce), gemm w1|w3, prep h, lorc w2 (partial + reduce),
     # gemm w2, combine; the compensator launches drop out when no expert has one
     has_lorc = any(wk.experts[e][n].rank for e in range(wk.n_experts) for n in ("w1", "w3", "w2"))
-    launches_per_step = 10 if has_lorc else 6
+    launches_per_step = 8 if has_lorc else 6
 
     # --- correctness gate on the bench configuration itself
     step(x, logits)
@@ -494,6 +521,31 @@ def run_e2e(args, torch, step, x, logits, y, out_dt, T, wk, dev, stream, world):
     return e2e_value, e2e_ms
 
 
+def roofline(args, pk, bytes_, glu_ms, glu_gbs) -> dict:
+    """Roofline of the dominant kernel, the w1|w3 grouped GEMM: HBM-bound on
+    the mma.sync path (decode), tensor-bound on the tcgen05 path (prefill),
+    where the fp16 dense peak equals the measured bf16 one (same rate)."""
+    if uses_tensor_path(bytes_):
+        tf = bytes_["glu_flops"] / (glu_ms / 1e3) / 1e12
+        peak = pk["bf16_tflops"]
+        return {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                "frac_of_sustained": tf / pk["bf16_tflops_sustained"],
+                "traffic": profiled_traffic("tc_gemm_glu_prefill.md", tensor=True)
+                if args.workload == "prefill" and args.tokens is None else None,
+                "kernel": "tc_gemm_kernel<true> (w1|w3 grouped int3 GEMM on tcgen05 + compensator + SwiGLU)",
+                "algorithmic_flops_per_launch": bytes_["glu_flops"], "ms_per_launch": glu_ms,
+                "peak_source": "measured cuBLAS bf16 GEMM, burst (MEASURED_PEAKS.json bf16_tflops); "
+                               "fp16 runs at the bf16 rate" if pk["source"] == "measured"
+                else "fallback 1590 TFLOP/s"}
+    return {"bound": "hbm", "achieved": glu_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": glu_gbs / pk["hbm_gbs"], "traffic": profiled_traffic("gemv_glu_mixtral_decode.md")
+            if args.workload == "mixtral" and args.tokens is None else None,
+            "kernel": "gemv_kernel<true> (w1|w3 grouped int3 GEMM + compensator + SwiGLU)",
+            "algorithmic_bytes_per_launch": bytes_["glu_kernel"], "ms_per_launch": glu_ms,
+            "peak_source": f"{pk['source']} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+            if pk["source"] == "measured" else "fallback 6650 GB/s"}
+
+
 def finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, logits, y, e2e_value,
            launches_per_step, clocks):
     pk = peaks()
@@ -508,18 +560,14 @@ def finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, l
                    "l2": f"inputs larger than L2: {bytes_['weights_only'] / 1e6:.0f} MB of packed weights "
                          f"streamed per step vs {L2_BYTES / 1e6:.0f} MB L2; no flush",
                    "parallelism": f"replica per GPU x{world}", "active_experts": bytes_["active_experts"]},
-        "roofline": {"bound": "hbm", "achieved": glu_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": glu_gbs / pk["hbm_gbs"], "traffic": profiled_traffic("gemv_glu_mixtral_decode.md")
-                     if args.workload == "mixtral" else None,
-                     "kernel": "gemv_kernel<true> (w1|w3 grouped int3 GEMM + compensator + SwiGLU)",
-                     "algorithmic_bytes_per_launch": bytes_["glu_kernel"], "ms_per_launch": glu_ms,
-                     "peak_source": f"{pk['source']} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
-                     if pk["source"] == "measured" else "fallback 6650 GB/s"},
+        "roofline": roofline(args, pk, bytes_, glu_ms, glu_gbs),
         "layer_hbm": {"bytes_per_step": bytes_["step"], "achieved_gbs": step_gbs,
                       "frac": step_gbs / pk["hbm_gbs"]},
         "kernels": {"gemm_w1w3_ms": glu_ms, "gemm_w2_ms": w2_ms,
                     "gemm_w2_gbs": bytes_["w2_kernel"] / (w2_ms / 1e3) / 1e9,
-                    "gemm_w1w3_gbs": glu_gbs},
+                    "gemm_w1w3_gbs": glu_gbs,
+                    "gemm_w1w3_tflops": bytes_["glu_flops"] / (glu_ms / 1e3) / 1e12,
+                    "gemm_w2_tflops": bytes_["w2_flops"] / (w2_ms / 1e3) / 1e12},
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": x.numel() * x.element_size() + logits.numel() * logits.element_size(),
                 "d2h_bytes_per_step": y.numel() * y.element_size()},

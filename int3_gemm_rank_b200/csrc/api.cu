@@ -144,8 +144,11 @@ struct LorcPlan {
     int splits, row_groups;
 };
 
+// slice counters of the compensator kernel: (expert, projection, 16-rank block, row group <= 8)
+static int lorc_counters(int n_exp) { return n_exp * 2 * ((MILO_MAX_RANK + 15) / 16) * 8; }
+
 struct LinearWs {
-    size_t grp, rows, inv, frag, gsum, t, tpart, part, total;
+    size_t grp, rows, inv, frag, gsum, t, tpart, done, part, total;
     int R, splits, tcols;
     LorcPlan lp;
 };
@@ -184,6 +187,7 @@ static LorcPlan lorc_plan(int n_exp, int nproj, int K, long long max_rows) {
     LorcPlan pl{1, 1};
     pl.splits = tiles >= 8 ? 1 : std::max(1, (sb + 3) / 4);
     pl.row_groups = static_cast<int>(std::min<long long>(tiles, std::max(1LL, 65536 / (base * pl.splits))));
+    if (pl.splits > 1) pl.row_groups = std::min(pl.row_groups, 8);   // the slice counters cover 8 row groups
     return pl;
 }
 
@@ -205,13 +209,14 @@ static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
     w.t = c.take(static_cast<size_t>(w.R) * w.tcols * 2);
     w.lp = lorc_plan(n_exp, 1, lin->K, static_cast<long long>(T) * k);   // at most all rows in one expert
     w.tpart = c.take(static_cast<size_t>(w.lp.splits) * w.R * w.tcols * 4);
+    w.done = c.take(static_cast<size_t>(lorc_counters(n_exp)) * 4);
     w.part = c.take(static_cast<size_t>(w.splits) * w.R * lin->N * 4);
     w.total = c.off;
     return w;
 }
 
 struct MoeWs {
-    size_t grp, rows, xfrag, xg, t13, h, hfrag, hg, t2, tpart, part, total;
+    size_t grp, rows, xfrag, xg, t13, h, hfrag, hg, t2, tpart, done, part, total;
     int R, R_routed, splits, tc13, tc2;
     LorcPlan lp13, lp2;
 };
@@ -242,6 +247,7 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
     w.lp2 = lorc_plan(n_exp, 1, I, T);
     w.tpart = c.take(std::max(static_cast<size_t>(w.lp13.splits) * w.tc13,
                               static_cast<size_t>(w.lp2.splits) * w.tc2) * w.R * 4);
+    w.done = c.take(static_cast<size_t>(lorc_counters(n_exp)) * 4);
     w.part = c.take(static_cast<size_t>(w.splits) * w.R * H * 4);
     w.total = c.off;
     return w;
@@ -452,7 +458,8 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     const bool tc = use_tc(static_cast<long long>(T) * k, lin->n_experts);
     PrepParams pp{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.frag),
                   reinterpret_cast<uint16_t*>(base + w.gsum), tc ? 1 : 0, dev_status, w.R, lin->K, x_dt == MILO_BF16,
-                  1, expert_offsets, perm, grp, inv, T, k, lin->n_experts, 0, w.R};
+                  1, expert_offsets, perm, grp, inv, T, k, lin->n_experts, 0, w.R,
+                  reinterpret_cast<int32_t*>(base + w.done), lorc_counters(lin->n_experts)};
     milo_status s = check_cuda(launch_prep(pp, st), "prep");
     if (s != MILO_OK) return s;
 
@@ -461,7 +468,7 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     if (has_t) {
         LorcParams lp{static_cast<const uint16_t*>(x), rows, table, grp,
                       reinterpret_cast<uint16_t*>(base + w.t), reinterpret_cast<float*>(base + w.tpart),
-                      dev_status, 1, 0, -1, lin->n_experts, lin->K, w.R, w.tcols, 0, x_dt == MILO_BF16,
+                      reinterpret_cast<int32_t*>(base + w.done), dev_status, 1, 0, -1, lin->n_experts, lin->K, w.R, w.tcols, 0, x_dt == MILO_BF16,
                       w.lp.splits, w.lp.row_groups};
         if ((s = check_cuda(launch_lorc(lp, st), "lorc")) != MILO_OK) return s;
     }
@@ -522,12 +529,13 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     const bool tc = use_tc(w.R_routed, L->n_routed);
     PrepParams px{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.xfrag),
                   reinterpret_cast<uint16_t*>(base + w.xg), tc ? 1 : 0, dev_status, w.R, H, x_dt == MILO_BF16, 1,
-                  expert_offsets, perm, grp, nullptr, T, L->top_k, L->n_routed, L->n_shared, w.R_routed};
+                  expert_offsets, perm, grp, nullptr, T, L->top_k, L->n_routed, L->n_shared, w.R_routed,
+                  reinterpret_cast<int32_t*>(base + w.done), lorc_counters(n_exp)};
     if ((s = check_cuda(launch_prep(px, st), "prep x")) != MILO_OK) return s;
     if (has_t) {
         LorcParams lp{static_cast<const uint16_t*>(x), rows, table, grp,
                       reinterpret_cast<uint16_t*>(base + w.t13), reinterpret_cast<float*>(base + w.tpart),
-                      dev_status, 3, 0, 1, n_exp, H, w.R, w.tc13, L->max_rank, x_dt == MILO_BF16,
+                      reinterpret_cast<int32_t*>(base + w.done), dev_status, 3, 0, 1, n_exp, H, w.R, w.tc13, L->max_rank, x_dt == MILO_BF16,
                       w.lp13.splits, w.lp13.row_groups};
         if ((s = check_cuda(launch_lorc(lp, st), "lorc w1|w3")) != MILO_OK) return s;
     }
@@ -560,7 +568,7 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     if (has_t) {
         LorcParams lp{reinterpret_cast<const uint16_t*>(base + w.h), nullptr, table, grp,
                       reinterpret_cast<uint16_t*>(base + w.t2), reinterpret_cast<float*>(base + w.tpart),
-                      dev_status, 3, 2, -1, n_exp, I, w.R, w.tc2, 0, 0, w.lp2.splits, w.lp2.row_groups};
+                      reinterpret_cast<int32_t*>(base + w.done), dev_status, 3, 2, -1, n_exp, I, w.R, w.tc2, 0, 0, w.lp2.splits, w.lp2.row_groups};
         if ((s = check_cuda(launch_lorc(lp, st), "lorc w2")) != MILO_OK) return s;
     }
 

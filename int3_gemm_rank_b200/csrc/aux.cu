@@ -111,6 +111,10 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     const int row = blockIdx.x;
     const int SB = p.K / 128;
     int32_t st = 0;
+    if (p.zero) {
+        const int nb = gridDim.x * gridDim.y, b = blockIdx.x * gridDim.y + blockIdx.y;
+        for (int i = b * blockDim.x + threadIdx.x; i < p.nzero; i += nb * blockDim.x) p.zero[i] = 0;
+    }
     int src;
     if (p.rows) {
         if (blockIdx.x == 0 && blockIdx.y == 0) build_groups(p, st);
@@ -215,11 +219,12 @@ cudaError_t launch_prep(const PrepParams& p, cudaStream_t s) {
 
 // ---------------------------------------------------------------------------
 // lorc: t[p, col0 + j] = sum_k x[p, k] V[j, k] for the rows of each expert.
-// Pass 1 (lorc_partial_kernel): one block per (expert, projection, 16-rank
-// block, K slice, row-tile group); its four warps split the K slice and their
-// 16x16 tiles are added in a fixed order into part[slice].  Pass 2
-// (lorc_reduce_kernel) adds the slices in order and rounds to fp16.  Both
-// orders are fixed, so the result does not depend on scheduling.
+// One block per (expert, projection, 16-rank block, K slice, row-tile group);
+// its four warps split the K slice and their 16x16 tiles are added in a fixed
+// order into part[slice].  The block that finishes a (expert, projection,
+// rank block, row group) last adds the slices in order and rounds to fp16
+// (a counter per tile says which block that is).  Both orders are fixed, so
+// the result does not depend on scheduling.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t load_x_pair(const uint16_t* row, int k, bool bf16, int32_t& st) {
     const uint32_t w = *reinterpret_cast<const uint32_t*>(row + k);
@@ -264,15 +269,17 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
     const int kend = min(p.K, kbeg + slice_sb * 128);
     float* out = p.part + static_cast<size_t>(split) * p.R * p.tcols;
     int32_t st = 0;
-    if (j0 >= r) {   // ranks of this block are all past r: zeros only
-        for (int mt = 16 * blockIdx.y; mt < m; mt += 16 * p.row_groups)
-            for (int idx = threadIdx.x; idx < 256; idx += blockDim.x) {
-                const int rr = idx / 16, jj = idx % 16;
-                if (mt + rr < m && j0 + jj < span)
-                    out[static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j0 + jj] = 0.0f;
-            }
+    if (j0 >= r) {   // ranks of this block are all past r: zeros only, from the first slice
+        if (split == 0)
+            for (int mt = 16 * blockIdx.y; mt < m; mt += 16 * p.row_groups)
+                for (int idx = threadIdx.x; idx < 256; idx += blockDim.x) {
+                    const int rr = idx / 16, jj = idx % 16;
+                    if (mt + rr < m && j0 + jj < span)
+                        p.t[static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j0 + jj] = 0;
+                }
         return;
     }
+    const bool single = p.splits == 1;
     for (int mt = 16 * blockIdx.y; mt < m; mt += 16 * p.row_groups) {
         __syncthreads();
         if (threadIdx.x < 16) {
@@ -335,43 +342,43 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
         for (int idx = threadIdx.x; idx < 256; idx += blockDim.x) {
             const int rr = idx / 16, jj = idx % 16;
             const float v = ((part[0][rr][jj] + part[1][rr][jj]) + part[2][rr][jj]) + part[3][rr][jj];
-            if (mt + rr < m && j0 + jj < span)
-                out[static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j0 + jj] = j0 + jj < r ? v : 0.0f;
+            if (mt + rr < m && j0 + jj < span) {
+                const size_t o = static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j0 + jj;
+                if (single) p.t[o] = __half_as_ushort(__float2half_rn(j0 + jj < r ? v : 0.0f));
+                else out[o] = j0 + jj < r ? v : 0.0f;
+            }
         }
     }
     flag(p.dev_status, st);
-}
-
-__global__ void __launch_bounds__(256) lorc_reduce_kernel(const LorcParams p) {
-    grid_dep_launch();
-    grid_dep_wait();
-    const size_t n = static_cast<size_t>(p.R) * p.tcols;
-    const size_t stride = n;
-    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        // eight running sums (slices s, s+8, ...) so the loads overlap, added in a fixed order
-        float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        int s = 0;
-        for (; s + 8 <= p.splits; s += 8)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) a[j] += p.part[(s + j) * stride + i];
-        for (int j = 0; s + j < p.splits; ++j) a[j] += p.part[(s + j) * stride + i];
-        const float v = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
-        p.t[i] = __half_as_ushort(__float2half_rn(v));
-    }
+    if (single) return;
+    // the last block of this tile to finish adds the slices in order
+    __shared__ int last;
+    __threadfence();
+    __syncthreads();
+    int32_t* ctr = p.done + ((e * nproj + which) * kLorcRankBlocks + rblk) * p.row_groups + blockIdx.y;
+    if (threadIdx.x == 0) last = atomicAdd(ctr, 1) == p.splits - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    const size_t slice = static_cast<size_t>(p.R) * p.tcols;
+    for (int mt = 16 * blockIdx.y; mt < m; mt += 16 * p.row_groups)
+        for (int idx = threadIdx.x; idx < 256; idx += blockDim.x) {
+            const int rr = idx / 16, jj = idx % 16;
+            if (mt + rr < m && j0 + jj < span) {
+                const size_t o = static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j0 + jj;
+                float v = 0.0f;
+                for (int sp = 0; sp < p.splits; ++sp) v += __ldcg(p.part + sp * slice + o);
+                p.t[o] = __half_as_ushort(__float2half_rn(v));
+            }
+        }
+    if (threadIdx.x == 0) *ctr = 0;   // ready for the next launch
 }
 
 cudaError_t launch_lorc(const LorcParams& p, cudaStream_t s) {
     const int nproj = p.proj_b >= 0 ? 2 : 1;
     const long long blocks = static_cast<long long>(p.n_exp) * nproj * kLorcRankBlocks * p.splits;
     if (blocks <= 0 || p.R <= 0) return cudaSuccess;
-    cudaError_t e = launch_pdl(lorc_partial_kernel, dim3(static_cast<unsigned>(blocks), p.row_groups), dim3(128),
-                               0, s, p);
-    if (e != cudaSuccess) return e;
-    const long long n = static_cast<long long>(p.R) * p.tcols;
-    long long rb = (n + 255) / 256;
-    if (rb > 2048) rb = 2048;
-    return launch_pdl(lorc_reduce_kernel, dim3(static_cast<unsigned>(rb)), dim3(256), 0, s, p);
+    return launch_pdl(lorc_partial_kernel, dim3(static_cast<unsigned>(blocks), p.row_groups), dim3(128), 0, s, p);
 }
 
 // ---------------------------------------------------------------------------

@@ -93,6 +93,8 @@ struct PrepParams {
     int32_t* grp;               // [E+S][2]: first row, row count
     int32_t* inv;               // optional [T*k] inverse of perm (-1 = dropped)
     int T, k, E, S, R_routed;
+    int32_t* zero;              // optional: `nzero` ints set to 0 (the compensator's slice counters)
+    int nzero;
 };
 
 struct LorcParams {
@@ -102,11 +104,16 @@ struct LorcParams {
     const int32_t* grp;         // [n_exp][2]
     uint16_t* t;                // [R, tcols] fp16
     float* part;                // [splits][R][tcols] f32 partial sums over K slices
+    int32_t* done;              // per (expert, projection, rank block, row group): slices finished; 0 on entry
     int32_t* dev_status;
     int stride, proj_a, proj_b; // proj_b < 0: single projection
     int n_exp, K, R, tcols, t_col_b, src_bf16;
     int splits, row_groups;     // K slices of ceil(K/128 / splits) super-blocks; row-tile strides
 };
+
+// Counters lorc_partial_kernel needs when it splits K (then at most 8 row
+// groups); zeroed by prep_kernel and left at zero.
+constexpr int kLorcCounters = MILO_MAX_EXPERTS * 2 * ((MILO_MAX_RANK + 15) / 16) * 8;
 
 struct CombineParams {
     const float* y_part;        // [splits][R][H]
