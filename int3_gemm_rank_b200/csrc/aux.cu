@@ -374,10 +374,124 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
     if (threadIdx.x == 0) *ctr = 0;   // ready for the next launch
 }
 
+// Many rows per expert (no K split): one block per (expert, projection, 64-row
+// tile) computes all 64 ranks over the whole K, so a V row is read once per 64
+// rows instead of once per 16.  Four warps take 16 rows each; K advances 64 at
+// a time through shared memory, the next chunk's loads in flight (registers)
+// while the current one is multiplied.  One fixed order: deterministic.
+constexpr int kLtRows = 64, kLtK = 64, kLtPitch = kLtK + 8;   // fp16 pitch: rows on different banks
+
+__global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
+    grid_dep_launch();
+    grid_dep_wait();
+    __shared__ __align__(16) uint16_t xs[kLtRows][kLtPitch];
+    __shared__ __align__(16) uint16_t vs[MILO_MAX_RANK][kLtPitch];
+    __shared__ int src_row[kLtRows];
+    const int nproj = p.proj_b >= 0 ? 2 : 1;
+    const int which = blockIdx.x % nproj, e = blockIdx.x / nproj;
+    const ProjDev* P = p.table + e * p.stride + (which == 0 ? p.proj_a : p.proj_b);
+    const int r = P->rank;
+    const int span = p.proj_b >= 0 ? p.t_col_b : p.tcols;
+    const int col0 = which == 0 ? 0 : p.t_col_b;
+    const int row0 = p.grp[2 * e], m = p.grp[2 * e + 1];
+    if (m <= 0 || row0 < 0 || row0 + m > p.R) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+    const int nr8 = (r + 7) / 8;                      // n8 rank tiles that hold ranks < r
+    int32_t st = 0;
+    for (int mt = kLtRows * blockIdx.y; mt < m; mt += kLtRows * gridDim.y) {
+        if (r == 0) {
+            for (int idx = threadIdx.x; idx < kLtRows * span; idx += blockDim.x) {
+                const int rr = idx / span, jj = idx % span;
+                if (mt + rr < m) p.t[static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + jj] = 0;
+            }
+            continue;
+        }
+        __syncthreads();
+        if (threadIdx.x < kLtRows) {
+            const int i = threadIdx.x;
+            src_row[i] = mt + i < m ? (p.row_src ? p.row_src[row0 + mt + i] : row0 + mt + i) : -1;
+        }
+        __syncthreads();
+        // this thread's share of a chunk: x rows (4 x 16 B) and V rows (4 x 16 B)
+        uint4 xr[4], vr[4];
+        auto fetch = [&](int kc) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int i = threadIdx.x + 128 * q;       // 0..511: row i / 8, 16-byte piece i % 8
+                const int rr = i >> 3, pc = i & 7;
+                const int sr = src_row[rr];
+                xr[q] = sr >= 0 ? *reinterpret_cast<const uint4*>(p.src + static_cast<size_t>(sr) * p.K + kc + 8 * pc)
+                                : make_uint4(0u, 0u, 0u, 0u);
+                vr[q] = rr < r ? *reinterpret_cast<const uint4*>(P->V + static_cast<size_t>(rr) * p.K + kc + 8 * pc)
+                               : make_uint4(0u, 0u, 0u, 0u);
+            }
+        };
+        float acc[8][4];
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[n][i] = 0.0f;
+        fetch(0);
+        for (int kc = 0; kc < p.K; kc += kLtK) {
+            __syncthreads();     // the previous chunk's multiplies are done
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int i = threadIdx.x + 128 * q;
+                const int rr = i >> 3, pc = i & 7;
+                uint32_t w[4] = {xr[q].x, xr[q].y, xr[q].z, xr[q].w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const __half lo = to_half(static_cast<uint16_t>(w[u] & 0xFFFFu), p.src_bf16, st);
+                    const __half hi = to_half(static_cast<uint16_t>(w[u] >> 16), p.src_bf16, st);
+                    w[u] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+                }
+                *reinterpret_cast<uint4*>(&xs[rr][8 * pc]) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4*>(&vs[rr][8 * pc]) = vr[q];
+            }
+            __syncthreads();
+            if (kc + kLtK < p.K) fetch(kc + kLtK);
+#pragma unroll
+            for (int k16 = 0; k16 < kLtK; k16 += 16) {
+                const int kk = k16 + 2 * c;
+                const int ra = 16 * warp + g;
+                const uint32_t a0 = *reinterpret_cast<const uint32_t*>(&xs[ra][kk]);
+                const uint32_t a1 = *reinterpret_cast<const uint32_t*>(&xs[ra + 8][kk]);
+                const uint32_t a2 = *reinterpret_cast<const uint32_t*>(&xs[ra][kk + 8]);
+                const uint32_t a3 = *reinterpret_cast<const uint32_t*>(&xs[ra + 8][kk + 8]);
+#pragma unroll
+                for (int n = 0; n < 8; ++n) {
+                    if (n < nr8) {
+                        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&vs[8 * n + g][kk]);
+                        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&vs[8 * n + g][kk + 8]);
+                        mma16816(acc[n], a0, a1, a2, a3, b0, b1);
+                    }
+                }
+            }
+        }
+        // acc[n][i]: row 16 * warp + g + 8 * (i >> 1), rank 8n + 2c + (i & 1)
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int rr = 16 * warp + g + 8 * (i >> 1), j = 8 * n + 2 * c + (i & 1);
+                if (mt + rr < m && j < span)
+                    p.t[static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j] =
+                        __half_as_ushort(__float2half_rn(j < r ? acc[n][i] : 0.0f));
+            }
+    }
+    flag(p.dev_status, st);
+}
+
 cudaError_t launch_lorc(const LorcParams& p, cudaStream_t s) {
     const int nproj = p.proj_b >= 0 ? 2 : 1;
+    if (p.n_exp <= 0 || p.R <= 0) return cudaSuccess;
+    if (p.splits == 1 && p.row_groups >= 8) {
+        // many rows: 64-row tiles, each block striding over its expert's tiles
+        const int tiles = (p.R + kLtRows - 1) / kLtRows;
+        return launch_pdl(lorc_tile_kernel, dim3(static_cast<unsigned>(p.n_exp * nproj), std::min(tiles, 64)),
+                          dim3(128), 0, s, p);
+    }
     const long long blocks = static_cast<long long>(p.n_exp) * nproj * kLorcRankBlocks * p.splits;
-    if (blocks <= 0 || p.R <= 0) return cudaSuccess;
     return launch_pdl(lorc_partial_kernel, dim3(static_cast<unsigned>(blocks), p.row_groups), dim3(128), 0, s, p);
 }
 
