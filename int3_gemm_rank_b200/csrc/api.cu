@@ -321,6 +321,11 @@ static milo_status run_tc(const GemvParams& g, bool glu, void* xcol, void* gsum,
     p.has_t = g.has_t;
     p.tcols = g.tcols;
     p.t_col_b = g.t_col_b;
+    // keep the larger of an expert's routed activations and its weights hot
+    // in L2: when the rows outweigh the weights, sweep the weight tiles fastest
+    const double act_bytes = static_cast<double>(g.R) / std::max(1, g.n_exp) * g.K * 2.0;
+    const double w_bytes = static_cast<double>(g.N) * (glu ? 2 : 1) * g.K * 7.0 / 16.0;
+    p.ntile_fast = act_bytes > w_bytes ? 1 : 0;
     return check_cuda(launch_tc_gemm(p, glu, sm_count(), st), what);
 }
 

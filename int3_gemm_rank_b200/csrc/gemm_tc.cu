@@ -88,7 +88,8 @@ struct TcItem {
     int e, ntile, tt;
 };
 
-__device__ __forceinline__ TcItem tc_decode(int it, const int* start, const int* cnt, int n_exp) {
+__device__ __forceinline__ TcItem tc_decode(int it, const int* start, const int* cnt, int n_exp, int n_tiles,
+                                           int ntile_fast) {
     int lo = 0, hi = n_exp - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -99,8 +100,13 @@ __device__ __forceinline__ TcItem tc_decode(int it, const int* start, const int*
     r.e = lo;
     const int local = it - start[lo];
     const int tte = (cnt[lo] + kTcTok - 1) / kTcTok;
-    r.tt = local % tte;
-    r.ntile = local / tte;
+    if (ntile_fast) {
+        r.ntile = local % n_tiles;
+        r.tt = local / n_tiles;
+    } else {
+        r.tt = local % tte;
+        r.ntile = local / tte;
+    }
     return r;
 }
 
@@ -240,7 +246,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             uint32_t phase = 0, filled = 0, fph = 0;
             bool fail = false;
             for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
-                const TcItem w = tc_decode(it, start, cnt, p.n_exp);
+                const TcItem w = tc_decode(it, start, cnt, p.n_exp, n_tiles, p.ntile_fast);
                 const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
                 const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
                 const int n0 = w.ntile * RA;
@@ -310,7 +316,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             uint32_t phase = 0, aph = 0, dph = 0, zph = 0;
             bool fail = false;
             for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
-                const TcItem w = tc_decode(it, start, cnt, p.n_exp);
+                const TcItem w = tc_decode(it, start, cnt, p.n_exp, n_tiles, p.ntile_fast);
                 const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
                 const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
                 for (int b = 0; b < p.SB && !fail; ++b) {
@@ -400,7 +406,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         int32_t st_bits = 0;
         uint4 zprev = make_uint4(0u, 0u, 0u, 0u);   // A_z slots of the pair's first super-block
         for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
-            const TcItem w = tc_decode(it, start, cnt, p.n_exp);
+            const TcItem w = tc_decode(it, start, cnt, p.n_exp, n_tiles, p.ntile_fast);
             const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
             const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
             // a plain item's second 64-row block is not loaded when the tile
@@ -522,7 +528,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         bool fail = false;
         int32_t st_bits = 0;
         for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
-            const TcItem w = tc_decode(it, start, cnt, p.n_exp);
+            const TcItem w = tc_decode(it, start, cnt, p.n_exp, n_tiles, p.ntile_fast);
             const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
             const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
             const int n0 = w.ntile * RA;

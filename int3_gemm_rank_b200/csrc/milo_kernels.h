@@ -62,9 +62,9 @@ struct GemvParams {
 // (gemm_tc.cu).  Activations in MMA column order [R][K] fp16 and their group
 // sums [R][4 * chunks] f32 arrive by 2-D TMA; weights as blob blocks.
 struct TcParams {
-    CUtensorMap b_map;          // activations [R][K] fp16, box {64, 128}, 128-byte swizzle
-    CUtensorMap z_map;          // group sums [R][chunks][16] fp16 (hi, lo, hi, lo per group), box {16, 128}
-    CUtensorMap t_map;          // LoRC down-projection [R][tcols] fp16, box {64, 128}, 128-byte swizzle
+    CUtensorMap b_map;          // activations [R][K] fp16, box {64, kTcTokens}, 128-byte swizzle
+    CUtensorMap z_map;          // group sums [R][chunks][16] fp16 (hi, lo, hi, lo per group), box {16, kTcTokens}
+    CUtensorMap t_map;          // LoRC down-projection [R][tcols] fp16, box {64, kTcTokens}, 128-byte swizzle
     const ProjDev* table;
     const int32_t* grp;
     float* y_part;              // plain: [R][N] f32
@@ -73,6 +73,8 @@ struct TcParams {
     int stride, proj_a, proj_b;
     int n_exp, N, K, R, SB;
     int has_t, tcols, t_col_b;
+    int ntile_fast;             // item order inside an expert: 1 = weight tiles fastest (routed-row tile
+                                // stays hot in L2), 0 = routed-row tiles fastest (weight tile stays hot)
 };
 
 struct PrepParams {
