@@ -298,7 +298,9 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------------ producer
-        if (lane != 0) return;
+        // The whole warp runs the loop (warp-uniform operands); one elected
+        // lane issues the copies: issued from a divergent single-lane branch a
+        // bulk copy costs the thread about 200 cycles.
         const uint64_t pol = l2_evict_first();
         int stage = 0;
         uint32_t phase = 0;
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             const int c0 = w.split * p.cps;
             const int c1 = min(p.chunks, c0 + p.cps);
             for (int ch = c0; ch < c1; ++ch) {
-                if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                if (!warp_wait(&empty[stage], phase ^ 1)) {
                     fail = true;
                     break;
                 }
@@ -332,27 +334,27 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 uint64_t* fb = &full[stage];
                 filled |= 1u << stage;
                 fph = (fph & ~(1u << stage)) | (phase << stage);
-                if (!header) {
-                    stage_item[stage] = it;
-                    header = true;
-                }
                 const int nsb = min(2, p.SB - 2 * ch);
                 const uint32_t wb = nsb * kBlockSB;                  // one tile's block
                 const uint32_t xb = ntok * kFragRowHalves * 2;
-                mbar_arrive_expect_tx(fb, ntl * wb + xb);
-                bulk_load_hint(st + kOffQ, pa->packed + (static_cast<size_t>(tile0) * p.SB + 2 * ch) * kBlockSB,
-                               wb, fb, pol);
-                if (ntl == 2)
-                    bulk_load_hint(st + kOffQ + kTileBlk,
-                                   (GLU ? pb->packed + (static_cast<size_t>(tile0) * p.SB + 2 * ch) * kBlockSB
-                                        : pa->packed + (static_cast<size_t>(tile0 + 1) * p.SB + 2 * ch) * kBlockSB),
-                                   wb, fb, pol);
-                bulk_load(st + kOffX, p.x + (static_cast<size_t>(ch) * p.R + row0) * kFragRowHalves, xb, fb);
+                const uint8_t* w0 = pa->packed + (static_cast<size_t>(tile0) * p.SB + 2 * ch) * kBlockSB;
+                const uint8_t* w1 = GLU ? pb->packed + (static_cast<size_t>(tile0) * p.SB + 2 * ch) * kBlockSB
+                                        : w0 + static_cast<size_t>(p.SB) * kBlockSB;
+                const uint16_t* xsrc = p.x + (static_cast<size_t>(ch) * p.R + row0) * kFragRowHalves;
+                if (elect_one()) {
+                    if (!header) stage_item[stage] = it;
+                    mbar_arrive_expect_tx(fb, ntl * wb + xb);
+                    bulk_load_hint(st + kOffQ, w0, wb, fb, pol);
+                    if (ntl == 2) bulk_load_hint(st + kOffQ + kTileBlk, w1, wb, fb, pol);
+                    bulk_load(st + kOffX, xsrc, xb, fb);
+                }
+                __syncwarp();
+                header = true;
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
             }
             const int ra = pa->rank, rb = GLU ? pb->rank : 0;
             if (!fail && w.split == 0 && p.has_t && (ra > 0 || rb > 0)) {
-                if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                if (!warp_wait(&empty[stage], phase ^ 1)) {
                     fail = true;
                     break;
                 }
@@ -360,47 +362,54 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 uint64_t* fb = &full[stage];
                 filled |= 1u << stage;
                 fph = (fph & ~(1u << stage)) | (phase << stage);
-                if (!header) {
-                    stage_item[stage] = it;
-                    header = true;
-                }
                 const int urows = min(RA, p.N - n0);
                 const uint32_t ua = urows * ra * 2, ub = urows * rb * 2;
                 const uint32_t tb = ntok * p.tcols * 2;
-                mbar_arrive_expect_tx(fb, ua + ub + tb);
-                if (ua) bulk_load_hint(st + kOffUA, pa->U + static_cast<size_t>(n0) * ra, ua, fb, pol);
-                if (ub) bulk_load_hint(st + kOffUB, pb->U + static_cast<size_t>(n0) * rb, ub, fb, pol);
-                bulk_load(st + kOffT, p.t + static_cast<size_t>(row0) * p.tcols, tb, fb);
+                if (elect_one()) {
+                    if (!header) stage_item[stage] = it;
+                    mbar_arrive_expect_tx(fb, ua + ub + tb);
+                    if (ua) bulk_load_hint(st + kOffUA, pa->U + static_cast<size_t>(n0) * ra, ua, fb, pol);
+                    if (ub) bulk_load_hint(st + kOffUB, pb->U + static_cast<size_t>(n0) * rb, ub, fb, pol);
+                    bulk_load(st + kOffT, p.t + static_cast<size_t>(row0) * p.tcols, tb, fb);
+                }
+                __syncwarp();
+                header = true;
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
             }
             if (!fail && !header) {   // an item with no stage of its own: a header-only stage
-                if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                if (!warp_wait(&empty[stage], phase ^ 1)) {
                     fail = true;
                     break;
                 }
                 filled |= 1u << stage;
                 fph = (fph & ~(1u << stage)) | (phase << stage);
-                stage_item[stage] = it;
-                mbar_arrive(&full[stage]);
+                if (elect_one()) {
+                    stage_item[stage] = it;
+                    mbar_arrive(&full[stage]);
+                }
+                __syncwarp();
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
             }
             if (fail) break;
         }
         // end of the queue for this CTA's consumers
         if (!fail) {
-            if (mbar_wait(&empty[stage], phase ^ 1)) {
+            if (warp_wait(&empty[stage], phase ^ 1)) {
                 filled |= 1u << stage;
                 fph = (fph & ~(1u << stage)) | (phase << stage);
-                stage_item[stage] = -1;
-                mbar_arrive(&full[stage]);
+                if (elect_one()) {
+                    stage_item[stage] = -1;
+                    mbar_arrive(&full[stage]);
+                }
+                __syncwarp();
             } else {
                 fail = true;
             }
         }
         // No copy may still be landing in shared memory when the CTA leaves.
         for (int s2 = 0; s2 < kStages; ++s2)
-            if (((filled >> s2) & 1u) && !mbar_wait(&full[s2], (fph >> s2) & 1u)) fail = true;
-        if (fail) flag(p.dev_status, MILO_DEV_TIMEOUT);
+            if (((filled >> s2) & 1u) && !warp_wait(&full[s2], (fph >> s2) & 1u)) fail = true;
+        if (fail && lane == 0) flag(p.dev_status, MILO_DEV_TIMEOUT);
         return;
     }
 
