@@ -416,10 +416,11 @@ def run_milo(args):
     sp = C.c_void_p(stream.cuda_stream)
 
     def step(xin, lin):
+        cur = C.c_void_p(torch.cuda.current_stream(dev).cuda_stream)   # the capture stream while capturing
         s = L.milo_route(C.c_void_p(lin.data_ptr()), T, E, k, flags, C.c_void_p(ids.data_ptr()),
                          C.c_void_p(wts.data_ptr()), C.c_void_p(off.data_ptr()),
                          C.c_void_p(perm.data_ptr()), C.c_void_p(inv.data_ptr()),
-                         C.c_void_p(st.data_ptr()), sp)
+                         C.c_void_p(st.data_ptr()), cur)
         if s:
             milo._check(s, "milo_route")
         milo.milo_moe_forward(layer, xin, route, out_dtype=out_dt, dev_status=st, y=y, ws=ws)
@@ -437,16 +438,20 @@ def run_milo(args):
     counts = np.diff(off.cpu().numpy())
     bytes_ = layer_bytes(wk, counts)
 
+    # --- the timed step: one CUDA graph of the whole step (route + layer), its
+    # launches and their programmatic dependencies captured once and replayed
+    run_step = capture_step(torch, dev, lambda: step(x, logits)) if args.graph else (lambda: step(x, logits))
+
     # --- warm-up and clock soak (also brings the clocks to their loaded state)
     for _ in range(args.warmup):
-        step(x, logits)
+        run_step()
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
     sampler.start()
     t_soak = time.perf_counter()
     while time.perf_counter() - t_soak < args.soak:
         for _ in range(20):
-            step(x, logits)
+            run_step()
         torch.cuda.synchronize()
 
     # --- timed region 1: K steps bracketed by events on the launching stream.
@@ -461,7 +466,7 @@ def run_milo(args):
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
-        step(x, logits)
+        run_step()
     stop.record(stream)
     torch.cuda.synchronize()
     barrier(dev)
@@ -483,6 +488,7 @@ def run_milo(args):
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {int(st.item())} after the timed region")
 
+    bytes_["graph"] = bool(args.graph)
     # --- end to end through the public API with host buffers
     if args.no_e2e:
         e2e_value, e2e_ms = None, None
@@ -490,6 +496,21 @@ def run_milo(args):
         e2e_value, e2e_ms = run_e2e(args, torch, step, x, logits, y, out_dt, T, wk, dev, stream, world)
     return finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, logits, y,
                   e2e_value, launches_per_step, clocks)
+
+
+def capture_step(torch, dev, fn):
+    """One CUDA graph of fn's launches (stream capture; the library's
+    programmatic launches become programmatic edges); returns its replay."""
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g.replay
 
 
 def run_e2e(args, torch, step, x, logits, y, out_dt, T, wk, dev, stream, world):
@@ -505,6 +526,9 @@ def run_e2e(args, torch, step, x, logits, y, out_dt, T, wk, dev, stream, world):
         l_d.copy_(l_h, non_blocking=True)
         step(x_d, l_d)
         y_h.copy_(y, non_blocking=True)
+
+    if args.graph:   # the copies in and out are part of the captured step
+        e2e_step = capture_step(torch, dev, e2e_step)
 
     for _ in range(args.warmup):
         e2e_step()
@@ -559,7 +583,9 @@ def finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, l
                    "y_dtype": "bf16",
                    "l2": f"inputs larger than L2: {bytes_['weights_only'] / 1e6:.0f} MB of packed weights "
                          f"streamed per step vs {L2_BYTES / 1e6:.0f} MB L2; no flush",
-                   "parallelism": f"replica per GPU x{world}", "active_experts": bytes_["active_experts"]},
+                   "parallelism": f"replica per GPU x{world}", "active_experts": bytes_["active_experts"],
+                   "launch": "one CUDA graph per step (route + layer)" if bytes_.get("graph")
+                   else "stream launches"},
         "roofline": roofline(args, pk, bytes_, glu_ms, glu_gbs),
         "layer_hbm": {"bytes_per_step": bytes_["step"], "achieved_gbs": step_gbs,
                       "frac": step_gbs / pk["hbm_gbs"]},
@@ -594,6 +620,8 @@ def main(argv=None):
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch the step's kernels one by one instead of replaying one CUDA graph")
     ap.add_argument("--experts", type=int, default=None, help="routed experts (profiler captures)")
     ap.add_argument("--tokens", type=int, default=None, help="tokens per step (profiler captures)")
     args = ap.parse_args(argv)
