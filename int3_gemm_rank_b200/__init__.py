@@ -177,8 +177,11 @@ def milo_unpack(packed: torch.Tensor, N: int, K: int) -> torch.Tensor:
 # ---------------------------------------------------------------------------
 
 def milo_route(logits: torch.Tensor | None, k: int, renorm: bool, E: int | None = None,
-               ids: torch.Tensor | None = None, dev_status: torch.Tensor | None = None) -> dict:
-    """Top-k router + grouping.  With `ids` given ([T, k] int32) the top-k is skipped."""
+               ids: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+               out: dict | None = None) -> dict:
+    """Top-k router + grouping.  With `ids` given ([T, k] int32) the top-k is skipped.
+    `out` (the dict a previous call returned, or one with the same keys and
+    sizes) receives the results in place, e.g. inside a CUDA graph capture."""
     flags = MILO_ROUTE_RENORM if renorm else 0
     if ids is not None:
         flags |= MILO_ROUTE_IDS_GIVEN
@@ -190,11 +193,18 @@ def milo_route(logits: torch.Tensor | None, k: int, renorm: bool, E: int | None 
         _cuda(logits, "logits")
         T, E = logits.shape
         dev = logits.device
-        ids = torch.empty((T, k), dtype=torch.int32, device=dev)
-        w = torch.empty((T, k), dtype=torch.float32, device=dev)
-    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    perm = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
-    inv = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+        ids = out["ids"] if out else torch.empty((T, k), dtype=torch.int32, device=dev)
+        w = out["w"] if out else torch.empty((T, k), dtype=torch.float32, device=dev)
+    if out:
+        for name, t, n in (("offsets", out["offsets"], E + 1), ("perm", out["perm"], T * k),
+                           ("inv_perm", out["inv_perm"], T * k)):
+            if t.dtype != torch.int32 or not t.is_contiguous() or t.numel() < n:
+                raise MiloError(MILO_ERR_INVALID_ARG, f"milo_route: out[{name!r}] must be int32[{n}]")
+        off, perm, inv = out["offsets"], out["perm"], out["inv_perm"]
+    else:
+        off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+        inv = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
     _check(lib().milo_route(_ptr(logits), T, E, k, flags, _ptr(ids), _ptr(w), _ptr(off), _ptr(perm),
                             _ptr(inv), _ptr(dev_status), _stream()), "milo_route")
     return {"ids": ids, "w": w, "offsets": off, "perm": perm[:T * k], "inv_perm": inv[:T * k]}
