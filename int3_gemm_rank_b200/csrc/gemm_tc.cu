@@ -334,10 +334,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         }
                         tc_fence_after();
                         const uint32_t d_addr = tbase + kTcDCol + kTcTok * db;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            tc_mma_ts(d_addr, tbase + kTcACol + 64 * ab + 32 * h + 8 * q,
-                                      sw128_kmajor_desc(sb_addr + h * kTcAtom + 32 * q), idesc, q > 0 ? 1u : 0u);
+                        tc_mma_ts4(d_addr, tbase + kTcACol + 64 * ab + 32 * h,
+                                   sw128_kmajor_desc(sb_addr + h * kTcAtom), idesc, 0u);
                         if (h == 1 && zs) {
                             // zero-point step of the pair into Z; the first one of an
                             // item waits until the fold has read the previous item's Z.

@@ -143,6 +143,25 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_addr, uint32_t a_addr, uint
 }
 
 // Named barrier among `count` threads (a subset of the CTA).
+// Four k16 steps D (+)= A[tmem] * B[smem]^T in one go (one elect.sync): A
+// columns a_addr + 8 q, B descriptors b_desc + 2 q (32 bytes further along
+// the 128-byte swizzled row); the first step accumulates iff `accumulate`.
+__device__ __forceinline__ void tc_mma_ts4(uint32_t d_addr, uint32_t a_addr, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e, t;\n\t.reg .b64 b1, b2, b3;\n\t.reg .b32 a1, a2, a3;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 t, %4, %4;\n\t"
+        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+        "add.s32 a1, %1, 8;\n\tadd.s32 a2, %1, 16;\n\tadd.s32 a3, %1, 24;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, t;\n\t}"
+        ::"r"(d_addr), "r"(a_addr), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, one k16 step.
 __device__ __forceinline__ void tc_mma_ss(uint32_t d_addr, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
