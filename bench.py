@@ -315,7 +315,7 @@ def sample_tokens(wk, n: int, seed: int) -> np.ndarray:
     return np.sort(np.random.default_rng(seed).choice(wk.T, size=min(n, wk.T), replace=False))
 
 
-def cpu_baseline(wk, n_tokens: int = 4, passes: int = 3, budget_s: float = 25.0) -> dict:
+def cpu_baseline(wk, n_tokens: int = 4, passes: int = 7, budget_s: float = 25.0) -> dict:
     """The oracle, as it stands, on the host cores: `passes` full-layer passes
     over `n_tokens` sampled tokens each (bounded by `budget_s`)."""
     import oracle
