@@ -43,7 +43,9 @@ _lib = None
 
 class Proj(C.Structure):
     _fields_ = [("Q", C.c_void_p), ("scale", C.c_void_p), ("zero", C.c_void_p),
-                ("U", C.c_void_p), ("V", C.c_void_p), ("rank", C.c_int32)]
+                ("U", C.c_void_p), ("V", C.c_void_p), ("rank", C.c_int32),
+                ("Uq", C.c_void_p), ("Us", C.c_void_p), ("Uz", C.c_void_p),
+                ("Vq", C.c_void_p), ("Vs", C.c_void_p), ("Vz", C.c_void_p)]
 
 
 def lib():
@@ -170,9 +172,11 @@ def route(logits_bits: np.ndarray, k: int, renorm: bool):
 
 
 class PackedProj:
-    """A quantised projection as the oracle sees it (all host arrays)."""
+    """A quantised projection as the oracle sees it (all host arrays).  With
+    `lorc3` = (Uq, Us, Uz, Vq, Vs, Vz) the compensator is int3: U^T [r, N] and
+    V [r, K] packed like weights (groups of 64 along N and K)."""
 
-    def __init__(self, Q, scale, zero, U, V):
+    def __init__(self, Q, scale, zero, U, V, lorc3=None):
         self.Q = _c(Q, np.uint32)
         self.scale = _c(scale, np.uint16)
         self.zero = _c(zero, np.uint16)
@@ -181,16 +185,26 @@ class PackedProj:
         self.rank = int(self.U.shape[1]) if self.U.ndim == 2 else 0
         self.N = self.Q.shape[0]
         self.K = self.Q.shape[1] * 32 // 3
+        self.lorc3 = None if lorc3 is None or self.rank == 0 else tuple(
+            _c(a, t) for a, t in zip(lorc3, (np.uint32, np.uint16, np.uint16) * 2))
 
     def cstruct(self) -> Proj:
+        l3 = [a.ctypes.data for a in self.lorc3] if self.lorc3 else [None] * 6
         return Proj(self.Q.ctypes.data, self.scale.ctypes.data, self.zero.ctypes.data,
                     self.U.ctypes.data if self.U.size else None,
-                    self.V.ctypes.data if self.V.size else None, self.rank)
+                    self.V.ctypes.data if self.V.size else None, self.rank, *l3)
 
 
-def quantize_projection(W_bits, U_bits, V_bits, group_size: int = 64) -> PackedProj:
+def quantize_projection(W_bits, U_bits, V_bits, group_size: int = 64, lorc_int3: bool = False) -> PackedProj:
+    """W quantised and packed; with lorc_int3 the compensator too: U^T [r, N]
+    and V [r, K] through the same quantiser (groups along N and K)."""
     q, s, z, _ = quantize(W_bits, group_size)
-    return PackedProj(pack(q), s, z, U_bits, V_bits)
+    lorc3 = None
+    if lorc_int3 and U_bits is not None and np.asarray(U_bits).size:
+        uq, us, uz, _ = quantize(np.ascontiguousarray(np.asarray(U_bits).T), group_size)
+        vq, vs, vz, _ = quantize(np.asarray(V_bits), group_size)
+        lorc3 = (pack(uq), us, uz, pack(vq), vs, vz)
+    return PackedProj(pack(q), s, z, U_bits, V_bits, lorc3)
 
 
 def linear(X: np.ndarray, P: PackedProj, group_size: int = 64, nthreads: int = 0) -> np.ndarray:

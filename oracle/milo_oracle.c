@@ -32,6 +32,10 @@
  *   - the packing layout (the page's description of the three-word packing is
  *     garbled) is the self-defined layout documented at milo_ref_code_bit();
  *   - compensator orientation: U [N_out, r], V [r, K], y += (x V^T) U^T;
+ *   - int3 compensators (the pages quantise U and V to 3 bits too): V is
+ *     quantised like a weight, groups of 64 along K; U is quantised
+ *     transposed, as U^T [r, N_out] with groups of 64 along N_out (r is at
+ *     most 64, and a group along r would not fill the 128-code blocks);
  *   - router: top-k largest logits (ties to the lower expert id), softmax
  *     weights renormalised over the top-k, or taken from the softmax over all
  *     experts when renormalisation is off;
@@ -344,15 +348,39 @@ typedef struct {
     const uint32_t* Q;      /* packed codes [N, 3K/32] */
     const uint16_t* scale;  /* fp16 [K/group, N] */
     const uint16_t* zero;   /* fp16 [K/group, N] */
-    const uint16_t* U;      /* fp16 [N, rank] */
-    const uint16_t* V;      /* fp16 [rank, K] */
+    const uint16_t* U;      /* fp16 [N, rank] (unused when Uq is set) */
+    const uint16_t* V;      /* fp16 [rank, K] (unused when Uq is set) */
     int32_t rank;
+    /* int3 compensator, optional: U^T packed [rank, 3N/32] with scale and zero
+       [N/group, rank]; V packed [rank, 3K/32] with scale and zero [K/group, rank] */
+    const uint32_t* Uq;
+    const uint16_t* Us;
+    const uint16_t* Uz;
+    const uint32_t* Vq;
+    const uint16_t* Vs;
+    const uint16_t* Vz;
 } milo_ref_proj;
+
+/* Row p of a packed matrix [R, C] (groups of `group` along C), dequantised
+   into out [C] in fp64 with the scalar unpack. */
+static void dequant_row(const uint32_t* Qm, const uint16_t* sc, const uint16_t* ze, int R, int Cc, int group,
+                        int p, double* out) {
+    uint8_t* codes = malloc((size_t)Cc);
+    milo_ref_unpack(Qm + (size_t)p * (3 * Cc / 32), 1, Cc, codes);
+    for (int c = 0; c < Cc; ++c) {
+        int j = c / group;
+        double s = milo_ref_h2d(sc[(size_t)j * R + p]);
+        double z = milo_ref_h2d(ze[(size_t)j * R + p]);
+        out[c] = ((double)codes[c] - z) * s;
+    }
+    free(codes);
+}
 
 typedef struct {
     const double* X; int M, K, N, group;
     const milo_ref_proj* P;
     const double* t;         /* [M, rank] = X V^T */
+    const double* Ud;        /* [N, rank] compensator U, fp64 */
     double* Y;               /* [M, N] */
     int n0, n1;
 } linear_job;
@@ -377,7 +405,7 @@ static void* linear_rows(void* arg) {
             for (int k = 0; k < K; ++k) acc += x[k] * wrow[k];
             double lorc = 0.0;
             for (int p = 0; p < r; ++p)
-                lorc += J->t[(size_t)m * r + p] * milo_ref_h2d(J->P->U[(size_t)n * r + p]);
+                lorc += J->t[(size_t)m * r + p] * J->Ud[(size_t)n * r + p];
             J->Y[(size_t)m * J->N + n] = acc + lorc;
         }
     }
@@ -401,12 +429,27 @@ static int default_threads(int nthreads) {
 void milo_ref_linear(const double* X, int M, int K, const milo_ref_proj* P, int N,
                      int group, double* Y, int nthreads) {
     int r = P->rank;
+    /* the compensator in fp64: fp16 values, or the dequantised int3 codes */
+    double* Vd = calloc((size_t)(r > 0 ? r : 1) * K, sizeof(double));
+    double* Ud = calloc((size_t)N * (r > 0 ? r : 1), sizeof(double));
+    double* urow = malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+    for (int p = 0; p < r; ++p) {
+        if (P->Uq) {
+            dequant_row(P->Vq, P->Vs, P->Vz, r, K, group, p, Vd + (size_t)p * K);
+            dequant_row(P->Uq, P->Us, P->Uz, r, N, group, p, urow);
+            for (int n = 0; n < N; ++n) Ud[(size_t)n * r + p] = urow[n];
+        } else {
+            for (int k = 0; k < K; ++k) Vd[(size_t)p * K + k] = milo_ref_h2d(P->V[(size_t)p * K + k]);
+            for (int n = 0; n < N; ++n) Ud[(size_t)n * r + p] = milo_ref_h2d(P->U[(size_t)n * r + p]);
+        }
+    }
+    free(urow);
     double* t = calloc((size_t)M * (r > 0 ? r : 1), sizeof(double));
     for (int m = 0; m < M; ++m)
         for (int p = 0; p < r; ++p) {
             double acc = 0.0;
             for (int k = 0; k < K; ++k)
-                acc += X[(size_t)m * K + k] * milo_ref_h2d(P->V[(size_t)p * K + k]);
+                acc += X[(size_t)m * K + k] * Vd[(size_t)p * K + k];
             t[(size_t)m * r + p] = acc;
         }
     int nt = default_threads(nthreads);
@@ -414,7 +457,7 @@ void milo_ref_linear(const double* X, int M, int K, const milo_ref_proj* P, int 
     pthread_t* th = malloc(sizeof(pthread_t) * (size_t)nt);
     linear_job* jobs = malloc(sizeof(linear_job) * (size_t)nt);
     for (int i = 0; i < nt; ++i) {
-        jobs[i] = (linear_job){X, M, K, N, group, P, t, Y,
+        jobs[i] = (linear_job){X, M, K, N, group, P, t, Ud, Y,
                                (int)((long)N * i / nt), (int)((long)N * (i + 1) / nt)};
         pthread_create(&th[i], NULL, linear_rows, &jobs[i]);
     }
@@ -422,6 +465,8 @@ void milo_ref_linear(const double* X, int M, int K, const milo_ref_proj* P, int 
     free(th);
     free(jobs);
     free(t);
+    free(Vd);
+    free(Ud);
 }
 
 /* silu(a) = a / (1 + e^-a), in fp64. */

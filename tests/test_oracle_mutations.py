@@ -17,7 +17,13 @@ SRC = os.path.join(ROOT, "oracle", "milo_oracle.c")
 MUTANTS = {
     "dequant_sign": ("wrow[k] = ((double)codes[k] - z) * s;", "wrow[k] = (z - (double)codes[k]) * s;"),
     "drop_lorc": ("J->Y[(size_t)m * J->N + n] = acc + lorc;", "J->Y[(size_t)m * J->N + n] = acc;"),
-    "transposed_U": ("J->P->U[(size_t)n * r + p]", "J->P->U[(size_t)p * J->N + n]"),
+    "transposed_U": ("milo_ref_h2d(P->U[(size_t)n * r + p])", "milo_ref_h2d(P->U[(size_t)p * N + n])"),
+    "int3_u_scale_zero_swapped": ("dequant_row(P->Uq, P->Us, P->Uz, r, N, group, p, urow);",
+                                  "dequant_row(P->Uq, P->Uz, P->Us, r, N, group, p, urow);"),
+    "int3_v_not_quantised": ("dequant_row(P->Vq, P->Vs, P->Vz, r, K, group, p, Vd + (size_t)p * K);",
+                             "for (int k = 0; k < K; ++k) Vd[(size_t)p * K + k] = milo_ref_h2d(P->V[(size_t)p * K + k]);"),
+    "int3_u_untransposed": ("for (int n = 0; n < N; ++n) Ud[(size_t)n * r + p] = urow[n];",
+                            "for (int n = 0; n < N; ++n) Ud[(size_t)n * r + p] = urow[(size_t)(n * r + p) % N];"),
     "zero_not_negated": ("float z_f = -mn / s;", "float z_f = mn / s;"),
     "scale_by_8": ("float s_f = range / 7.0f;", "float s_f = range / 8.0f;"),
     "round_half_up": ("float r = nearbyintf(v);", "float r = floorf(v + 0.5f);"),

@@ -308,6 +308,61 @@ def test_linear_rank0_equals_plain_quantized_gemm_and_matches_numpy():
     np.testing.assert_allclose(oracle.linear(X, P), X @ (wh + Uf @ Vf).T, rtol=1e-12, atol=1e-12)
 
 
+def _int3_exact_matrix(rng, R, C):
+    """fp16 bits of an R x C matrix whose every group of 64 along C holds the
+    levels (q - 3) * 2^-6 with q = 0 and q = 7 both present: the quantiser then
+    recovers s = 2^-6, z = 3 and the codes exactly."""
+    q = rng.integers(0, 8, (R, C))
+    for g0 in range(0, C, 64):
+        q[:, g0] = 0
+        q[:, g0 + 1] = 7
+    vals = ((q - 3) * 2.0 ** -6).astype(np.float16)
+    return vals.view(np.uint16), q
+
+
+def test_linear_int3_compensator_exact_levels_equal_fp16():
+    """int3 compensator (U^T grouped along N, V along K): with U and V already
+    on the int3 levels the quantised compensator equals the fp16 one exactly;
+    N != K so a transposed operand changes the result."""
+    rng = np.random.default_rng(21)
+    N, K, r = 384, 256, 8      # U^T is packed along N: N is a multiple of 128 too
+    W = wl.gen_weight(rng, N, K)
+    Ut, _ = _int3_exact_matrix(rng, r, N)       # U^T [r, N]
+    V, _ = _int3_exact_matrix(rng, r, K)
+    U = np.ascontiguousarray(Ut.T)
+    X = rng.standard_normal((4, K))
+    P16 = oracle.quantize_projection(W, U, V)
+    P3 = oracle.quantize_projection(W, U, V, lorc_int3=True)
+    assert P3.lorc3 is not None
+    assert np.array_equal(oracle.linear(X, P3), oracle.linear(X, P16))
+
+
+def test_linear_int3_compensator_rounding_bound():
+    """Random U, V: each dequantised compensator entry is within half a step
+    (s/2 plus the zero point's rounding) of its fp16 value, so the int3 and
+    fp16 outputs differ by at most the propagated bound."""
+    rng = np.random.default_rng(22)
+    N, K, r = 128, 384, 16
+    W = wl.gen_weight(rng, N, K)
+    U = wl.gen_normal_f16(rng, (N, r), 0.01)
+    V = wl.gen_normal_f16(rng, (r, K), 0.01)
+    X = rng.standard_normal((3, K))
+    qu, su, zu, _ = oracle.quantize(np.ascontiguousarray(U.T))
+    qv, sv, zv, _ = oracle.quantize(V)
+    Uh = oracle.dequant(qu, su, zu).T
+    Vh = oracle.dequant(qv, sv, zv)
+    Uf = U.view(np.float16).astype(np.float64)
+    Vf = V.view(np.float16).astype(np.float64)
+    step_u = np.repeat(su.view(np.float16).astype(np.float64).T, 64, axis=1).T   # [N, r] per entry
+    step_v = np.repeat(sv.view(np.float16).astype(np.float64).T, 64, axis=1)     # [r, K]
+    assert np.all(np.abs(Uh - Uf) <= 0.5 * step_u * (1 + 2 ** -9) + 1e-12)
+    assert np.all(np.abs(Vh - Vf) <= 0.5 * step_v * (1 + 2 ** -9) + 1e-12)
+    P16 = oracle.quantize_projection(W, U, V)
+    P3 = oracle.quantize_projection(W, U, V, lorc_int3=True)
+    d = oracle.linear(X, P3) - oracle.linear(X, P16)
+    np.testing.assert_allclose(d, (X @ Vh.T) @ Uh.T - (X @ Vf.T) @ Uf.T, rtol=1e-9, atol=1e-12)
+
+
 def test_linear_independent_of_thread_count():
     rng = np.random.default_rng(10)
     W = wl.gen_weight(rng, 37, 128)
