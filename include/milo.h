@@ -162,13 +162,21 @@ MILO_API milo_status milo_route(const uint16_t* logits, int32_t T, int32_t E, in
 /* ------------------------------------------------------------------------ */
 
 /* One quantised projection W [N, K] with its rank-r compensator (host struct
- * holding device pointers).  U fp16 [N, r] and V fp16 [r, K] row-major; both
- * may be NULL when rank == 0.  rank is a multiple of 8, at most MILO_MAX_RANK. */
+ * holding device pointers).  rank is a multiple of 8, at most MILO_MAX_RANK;
+ * U and V may be NULL when rank == 0.  The compensator is stored in one of two
+ * formats ("MiLo Algorithm": the compensators are quantised to 3 bits too):
+ *   MILO_LORC_F16   U fp16 [N, r] and V fp16 [r, K], row-major;
+ *   MILO_LORC_INT3  U points to the milo_pack blob of U^T [r, N] (groups of 64
+ *                   along N; needs N % 128 == 0) and V to the blob of V [r, K]
+ *                   (groups of 64 along K), both written by milo_pack. */
+#define MILO_LORC_F16 0
+#define MILO_LORC_INT3 1
 typedef struct milo_qweight {
     const void* packed;     /* blob written by milo_pack */
-    const uint16_t* U;
-    const uint16_t* V;
+    const void* U;
+    const void* V;
     int32_t rank;
+    int32_t lorc_format;    /* MILO_LORC_F16 or MILO_LORC_INT3 */
 } milo_qweight;
 
 /* One SwiGLU expert: w1, w3 [I, H] and w2 [H, I]. */

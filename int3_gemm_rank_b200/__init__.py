@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libmilo.so")
 
 MILO_F16, MILO_BF16, MILO_F32 = 0, 1, 2
 MILO_OK, MILO_ERR_INVALID_ARG, MILO_ERR_UNSUPPORTED_SHAPE, MILO_ERR_WORKSPACE, MILO_ERR_CUDA = range(5)
+MILO_LORC_F16, MILO_LORC_INT3 = 0, 1
 MILO_DEV_BAD_EXPERT_ID, MILO_DEV_NONFINITE, MILO_DEV_FP16_RANGE, MILO_DEV_TIMEOUT = 1, 2, 4, 8
 MILO_ROUTE_RENORM, MILO_ROUTE_IDS_GIVEN = 1, 2
 MILO_GROUP, MILO_MAX_RANK = 64, 64
@@ -41,7 +42,8 @@ class MiloError(RuntimeError):
 
 
 class milo_qweight(C.Structure):
-    _fields_ = [("packed", C.c_void_p), ("U", C.c_void_p), ("V", C.c_void_p), ("rank", C.c_int32)]
+    _fields_ = [("packed", C.c_void_p), ("U", C.c_void_p), ("V", C.c_void_p), ("rank", C.c_int32),
+                ("lorc_format", C.c_int32)]
 
 
 class milo_expert(C.Structure):
@@ -216,22 +218,33 @@ def milo_route(logits: torch.Tensor | None, k: int, renorm: bool, E: int | None 
 
 class QWeight:
     """A packed projection W [N, K] on the device: the blob of milo.h (codes,
-    scales, zeros) and the compensator U [N, r], V [r, K]."""
+    scales, zeros) and the compensator, fp16 U [N, r] and V [r, K], or
+    (lorc_int3) the blobs of U^T [r, N] and V [r, K]."""
 
-    def __init__(self, packed, N: int, K: int, U=None, V=None):
+    def __init__(self, packed, N: int, K: int, U=None, V=None, rank: int | None = None, lorc_int3: bool = False):
         self.packed = packed
         self.N, self.K = int(N), int(K)
-        self.rank = 0 if U is None or U.numel() == 0 else int(U.shape[1])
+        if rank is None:
+            rank = 0 if U is None or U.numel() == 0 else int(U.shape[1])
+        self.rank = int(rank)
         self.U = U if self.rank else None
         self.V = V if self.rank else None
+        self.lorc_int3 = bool(lorc_int3) and self.rank > 0
 
     @classmethod
-    def quantize(cls, W: torch.Tensor, U=None, V=None, dev_status=None):
-        return cls(milo_pack(W, dev_status=dev_status), W.shape[0], W.shape[1], U, V)
+    def quantize(cls, W: torch.Tensor, U=None, V=None, dev_status=None, lorc_int3: bool = False):
+        """Pack W (and, with lorc_int3, U^T and V) with milo_pack."""
+        packed = milo_pack(W, dev_status=dev_status)
+        if lorc_int3 and U is not None and U.numel():
+            r = int(U.shape[1])
+            return cls(packed, W.shape[0], W.shape[1], milo_pack(U.t().contiguous(), dev_status=dev_status),
+                       milo_pack(V, dev_status=dev_status), rank=r, lorc_int3=True)
+        return cls(packed, W.shape[0], W.shape[1], U, V)
 
     def cstruct(self) -> milo_qweight:
         return milo_qweight(self.packed.data_ptr(), self.U.data_ptr() if self.rank else None,
-                            self.V.data_ptr() if self.rank else None, self.rank)
+                            self.V.data_ptr() if self.rank else None, self.rank,
+                            MILO_LORC_INT3 if self.lorc_int3 else MILO_LORC_F16)
 
 
 def _table(n_proj: int, device) -> torch.Tensor:

@@ -94,12 +94,19 @@ static milo_status fill_proj(ProjDev* d, const milo_qweight& w, int N, int K, co
         return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": U and V are required when rank > 0");
     if (!aligned(w.packed, 16) || (w.rank > 0 && (!aligned(w.U, 16) || !aligned(w.V, 16))))
         return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": pointers must be 16-byte aligned");
+    if (w.lorc_format != MILO_LORC_F16 && w.lorc_format != MILO_LORC_INT3)
+        return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": unknown compensator format");
+    const bool int3 = w.rank > 0 && w.lorc_format == MILO_LORC_INT3;
+    if (int3 && N % 128)
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE,
+                    std::string(what) + ": an int3 compensator needs N to be a multiple of 128");
     d->packed = static_cast<const uint8_t*>(w.packed);
-    d->U = w.rank > 0 ? w.U : nullptr;
-    d->V = w.rank > 0 ? w.V : nullptr;
+    d->U = w.rank > 0 ? static_cast<const uint16_t*>(w.U) : nullptr;
+    d->V = w.rank > 0 ? static_cast<const uint16_t*>(w.V) : nullptr;
     d->rank = w.rank;
     d->N = N;
     d->K = K;
+    d->lorc3 = int3 ? 1 : 0;
     return MILO_OK;
 }
 

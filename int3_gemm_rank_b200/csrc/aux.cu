@@ -18,6 +18,10 @@
 #include "milo_host.h"
 #include "milo_kernels.h"
 
+static_assert(milo::kBlockSB == milo::kBlobBlockBytes && milo::kQTileSBWords * 4 == milo::kBlobWordBytes &&
+                  milo::kGroupBytes == milo::kBlobGroupBytes,
+              "blob block layout");
+
 namespace milo {
 
 // ---------------------------------------------------------------------------
@@ -298,6 +302,7 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
                 const int rr = (i / per_row) & 15, ch = i % per_row, isv = i / (16 * per_row);
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
                 if (isv) {
+                    if (P->lorc3) continue;   // int3 rows: below, one unit per thread
                     if (j0 + rr < r)
                         v = *reinterpret_cast<const uint4*>(P->V + static_cast<size_t>(j0 + rr) * p.K + kc + 8 * ch);
                     *reinterpret_cast<uint4*>(&vs[rr][8 * ch]) = v;
@@ -316,6 +321,34 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
                         v = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                     *reinterpret_cast<uint4*>(&xs[rr][8 * ch]) = v;
+                }
+            }
+            if (P->lorc3) {
+                // int3 V: unit c of super-block sb of rank row j0 + rr, dequantised to
+                // fp16: its first 16 codes at 16c.., its last 16 at 64 + 16c..
+                const uint8_t* vb = reinterpret_cast<const uint8_t*>(P->V);
+                for (int i = threadIdx.x; i < 16 * (cs / 32); i += blockDim.x) {
+                    const int rr = i / (cs / 32), u = i % (cs / 32), sb = u >> 2, c = u & 3;
+                    const int j = j0 + rr, b = (kc >> 7) + sb;
+                    uint32_t h0[8], h1[8];
+                    if (j < r) {
+                        const uint32_t* wp = reinterpret_cast<const uint32_t*>(vb + lorc_words_off(j, b, c));
+                        const uint32_t w3[3] = {wp[0], wp[1], wp[2]};
+                        const uint32_t sz0 = *reinterpret_cast<const uint32_t*>(vb + lorc_sz_off(j, 2 * b));
+                        const uint32_t sz1 = *reinterpret_cast<const uint32_t*>(vb + lorc_sz_off(j, 2 * b + 1));
+                        unit_half_dequant(w3, 0, sz_scale(sz0), sz_zero(sz0), h0);
+                        unit_half_dequant(w3, 1, sz_scale(sz1), sz_zero(sz1), h1);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) h0[q] = h1[q] = 0u;
+                    }
+                    uint16_t* row = &vs[rr][128 * sb + 16 * c];
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        reinterpret_cast<uint4*>(row)[q] = make_uint4(h0[4 * q], h0[4 * q + 1], h0[4 * q + 2], h0[4 * q + 3]);
+                        reinterpret_cast<uint4*>(row + 64)[q] =
+                            make_uint4(h1[4 * q], h1[4 * q + 1], h1[4 * q + 2], h1[4 * q + 3]);
+                    }
                 }
             }
             __syncthreads();
@@ -414,6 +447,12 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
         __syncthreads();
         // this thread's share of a chunk: x rows (4 x 16 B) and V rows (4 x 16 B)
         uint4 xr[4], vr[4];
+        // int3 V: a chunk of 64 positions is one group, 16 codes in each of the
+        // super-block's four units; this thread takes rank row tid / 2, units
+        // 2 (tid & 1) and 2 (tid & 1) + 1 (positions 32 (tid & 1) .. + 31)
+        const uint8_t* vb = reinterpret_cast<const uint8_t*>(P->V);
+        const int urow = threadIdx.x >> 1, uu = threadIdx.x & 1;
+        uint32_t vw[6] = {0u, 0u, 0u, 0u, 0u, 0u}, vsz = 0u;
         auto fetch = [&](int kc) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -422,8 +461,15 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
                 const int sr = src_row[rr];
                 xr[q] = sr >= 0 ? *reinterpret_cast<const uint4*>(p.src + static_cast<size_t>(sr) * p.K + kc + 8 * pc)
                                 : make_uint4(0u, 0u, 0u, 0u);
-                vr[q] = rr < r ? *reinterpret_cast<const uint4*>(P->V + static_cast<size_t>(rr) * p.K + kc + 8 * pc)
-                               : make_uint4(0u, 0u, 0u, 0u);
+                if (!P->lorc3)
+                    vr[q] = rr < r ? *reinterpret_cast<const uint4*>(P->V + static_cast<size_t>(rr) * p.K + kc + 8 * pc)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (P->lorc3 && urow < r) {
+                const uint32_t* wp = reinterpret_cast<const uint32_t*>(vb + lorc_words_off(urow, kc >> 7, 2 * uu));
+#pragma unroll
+                for (int q = 0; q < 6; ++q) vw[q] = wp[q];
+                vsz = *reinterpret_cast<const uint32_t*>(vb + lorc_sz_off(urow, kc >> 6));
             }
         };
         float acc[8][4];
@@ -446,7 +492,24 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
                     w[u] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
                 }
                 *reinterpret_cast<uint4*>(&xs[rr][8 * pc]) = make_uint4(w[0], w[1], w[2], w[3]);
-                *reinterpret_cast<uint4*>(&vs[rr][8 * pc]) = vr[q];
+                if (!P->lorc3) *reinterpret_cast<uint4*>(&vs[rr][8 * pc]) = vr[q];
+            }
+            if (P->lorc3) {
+                uint32_t h[2][8];
+                if (urow < r) {
+                    const int half = (kc >> 6) & 1;
+                    const uint32_t wa[3] = {vw[0], vw[1], vw[2]}, wb[3] = {vw[3], vw[4], vw[5]};
+                    unit_half_dequant(wa, half, sz_scale(vsz), sz_zero(vsz), h[0]);
+                    unit_half_dequant(wb, half, sz_scale(vsz), sz_zero(vsz), h[1]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) h[0][q] = h[1][q] = 0u;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4*>(&vs[urow][32 * uu + 8 * q]) =
+                        make_uint4(h[q >> 1][4 * (q & 1)], h[q >> 1][4 * (q & 1) + 1], h[q >> 1][4 * (q & 1) + 2],
+                                   h[q >> 1][4 * (q & 1) + 3]);
             }
             __syncthreads();
             if (kc + kLtK < p.K) fetch(kc + kLtK);

@@ -141,6 +141,21 @@ __device__ __forceinline__ void tc_unit(uint32_t w0, uint32_t w1, uint32_t w2, u
     tc_unit_reg<C, 15>(w, hw, a);
 }
 
+// fp16 pair (U[n][rho], U[n][rho + 1]) from an int3 U^T block (128 features):
+// feature nl's codes of rank rows rho and rho + 1, (q - z) * s.
+__device__ __forceinline__ uint32_t lorc3_value_pair(const uint8_t* blk, int rho, int nl) {
+    float v[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const uint32_t* wp = reinterpret_cast<const uint32_t*>(blk + lorc_words_off(rho + q, 0, blob_unit(nl)));
+        const uint32_t w3[3] = {wp[0], wp[1], wp[2]};
+        const uint32_t sz = *reinterpret_cast<const uint32_t*>(blk + lorc_sz_off(rho + q, nl >> 6));
+        v[q] = (static_cast<float>(unit_code(w3, blob_code(nl))) - sz_zero(sz)) * sz_scale(sz);
+    }
+    return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[0]))) |
+           (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[1]))) << 16);
+}
+
 // A fold warp reads its kTcHalf accumulator columns in chunks of kTcChunk
 // (48: three x16 loads in flight; 32: one x32 load), the caller waiting with
 // tc_wait_ld.
@@ -290,13 +305,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     fph = (fph & ~(1u << stage)) | (phase << stage);
                     const int nbox = (p.tcols + 63) / 64;
                     const int urows = min(RA, p.N - n0);
-                    const uint32_t ua = urows * ra * 2, ub = urows * rb * 2;
+                    // fp16 U rows, or the int3 U^T block holding the item's features
+                    const uint32_t ua = ra == 0 ? 0u : pa->lorc3 ? kBlockSB : urows * ra * 2;
+                    const uint32_t ub = rb == 0 ? 0u : pb->lorc3 ? kBlockSB : urows * rb * 2;
+                    const uint8_t* usa = pa->lorc3 ? reinterpret_cast<const uint8_t*>(pa->U) + (n0 >> 7) * kBlockSB
+                                                   : reinterpret_cast<const uint8_t*>(pa->U + static_cast<size_t>(n0) * ra);
+                    const uint8_t* usb = !GLU ? usa
+                                         : pb->lorc3 ? reinterpret_cast<const uint8_t*>(pb->U) + (n0 >> 7) * kBlockSB
+                                                     : reinterpret_cast<const uint8_t*>(pb->U + static_cast<size_t>(n0) * rb);
                     if (elect_one()) {
                         mbar_arrive_expect_tx(fb, nbox * kTcAtom + ua + ub);
                         for (int j = 0; j < nbox; ++j)
                             tma_load_2d(st + kTcOffB + j * kTcAtom, &p.t_map, fb, 64 * j, row0);
-                        if (ua) bulk_load_hint(st + kTcOffUA, pa->U + static_cast<size_t>(n0) * ra, ua, fb, pol);
-                        if (ub) bulk_load_hint(st + kTcOffUB, pb->U + static_cast<size_t>(n0) * rb, ub, fb, pol);
+                        if (ua) bulk_load_hint(st + kTcOffUA, usa, ua, fb, pol);
+                        if (ub) bulk_load_hint(st + kTcOffUB, usb, ub, fb, pol);
                     }
                     __syncwarp();
                     if (++stage == kTcStages) { stage = 0; phase ^= 1; }
@@ -477,20 +499,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 const uint8_t* st = smem + stage * kTcStage;
                 const uint16_t* src;
                 int lo, r;
+                bool u3;
                 if (GLU && row >= 64) {
                     src = reinterpret_cast<const uint16_t*>(st + kTcOffUB) + (row - 64) * rb;
                     lo = p.t_col_b;
                     r = rb;
+                    u3 = pb->lorc3 != 0;
                 } else {
                     src = reinterpret_cast<const uint16_t*>(st + kTcOffUA) + row * ra;
                     lo = 0;
                     r = ra;
+                    u3 = pa->lorc3 != 0;
                 }
                 uint32_t a[64];
+                if (u3) {
+                    // int3 U^T block: this row's feature, each rank row's code of it
+                    const uint8_t* blk = st + ((GLU && row >= 64) ? kTcOffUB : kTcOffUA);
+                    const int nl = ((w.ntile * RA) & 127) + (GLU ? (row & 63) : row);
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    const int slot = 2 * j;
-                    a[j] = (slot >= lo && slot < lo + r) ? *reinterpret_cast<const uint32_t*>(src + (slot - lo)) : 0u;
+                    for (int j = 0; j < 64; ++j) {
+                        const int slot = 2 * j;
+                        a[j] = (slot >= lo && slot < lo + r)
+                                   ? lorc3_value_pair(blk, slot - lo, nl)
+                                   : 0u;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) {
+                        const int slot = 2 * j;
+                        a[j] = (slot >= lo && slot < lo + r) ? *reinterpret_cast<const uint32_t*>(src + (slot - lo)) : 0u;
+                    }
                 }
                 if (!warp_wait(&aempty[ab], aph ^ 1)) {
                     fail = true;

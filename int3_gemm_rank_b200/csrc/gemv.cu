@@ -214,10 +214,31 @@ __device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2]
     }
 }
 
-// Compensator K-steps: acc += U_tile * t^T over the rank (multiple of 8).
+// Values of rank row rho of an int3 U^T block (128 features) at features nl
+// and nl + 8 (nl % 16 < 8: the same unit, codes 8 apart): (q - z) * s.
+__device__ __forceinline__ float2 lorc3_pair(const uint8_t* blk, int rho, int nl) {
+    const uint32_t* wp = reinterpret_cast<const uint32_t*>(blk + lorc_words_off(rho, 0, blob_unit(nl)));
+    const uint32_t w3[3] = {wp[0], wp[1], wp[2]};
+    const uint32_t sz = *reinterpret_cast<const uint32_t*>(blk + lorc_sz_off(rho, nl >> 6));
+    const float s = sz_scale(sz), z = sz_zero(sz);
+    const int m = blob_code(nl);
+    return make_float2((static_cast<float>(unit_code(w3, m)) - z) * s,
+                       (static_cast<float>(unit_code(w3, m + 8)) - z) * s);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(lo))) |
+           (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(hi))) << 16);
+}
+
+// Compensator K-steps: acc += U_tile * t^T over the rank (multiple of 8).  U
+// rows are fp16 [rows][r] in the stage, or (u3a for w1 / the plain
+// projection, u3b for w3) the item's int3 U^T block, whose features start at
+// `nb0` inside the block.
 template <bool GLU, int NT>
 __device__ __forceinline__ void lorc_compute(const uint8_t* st, float (&acc)[2][2][4], int warp,
-                                             int lane, int ra, int rb, int tcols, int t_col_b) {
+                                             int lane, int ra, int rb, int tcols, int t_col_b, bool u3a, bool u3b,
+                                             int nb0) {
     const int g = lane >> 2, c = lane & 3;
     const uint16_t* tt = reinterpret_cast<const uint16_t*>(st + kOffT);
 #pragma unroll
@@ -229,10 +250,26 @@ __device__ __forceinline__ void lorc_compute(const uint8_t* st, float (&acc)[2][
         for (int kk = 0; kk < r; kk += 16) {
             const int col = kk + 2 * c;
             const bool upper = col + 8 < r;
-            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(U + (rbase + g) * r + col);
-            const uint32_t a1 = *reinterpret_cast<const uint32_t*>(U + (rbase + g + 8) * r + col);
-            const uint32_t a2 = upper ? *reinterpret_cast<const uint32_t*>(U + (rbase + g) * r + col + 8) : 0u;
-            const uint32_t a3 = upper ? *reinterpret_cast<const uint32_t*>(U + (rbase + g + 8) * r + col + 8) : 0u;
+            uint32_t a0, a1, a2 = 0u, a3 = 0u;
+            if ((GLU && ti == 1) ? u3b : u3a) {
+                const uint8_t* blk = reinterpret_cast<const uint8_t*>(U);
+                const int nl = nb0 + rbase + g;
+                const float2 v0 = lorc3_pair(blk, col, nl), v1 = lorc3_pair(blk, col + 1, nl);
+                a0 = pack_half2(v0.x, v1.x);
+                a1 = pack_half2(v0.y, v1.y);
+                if (upper) {
+                    const float2 v8 = lorc3_pair(blk, col + 8, nl), v9 = lorc3_pair(blk, col + 9, nl);
+                    a2 = pack_half2(v8.x, v9.x);
+                    a3 = pack_half2(v8.y, v9.y);
+                }
+            } else {
+                a0 = *reinterpret_cast<const uint32_t*>(U + (rbase + g) * r + col);
+                a1 = *reinterpret_cast<const uint32_t*>(U + (rbase + g + 8) * r + col);
+                if (upper) {
+                    a2 = *reinterpret_cast<const uint32_t*>(U + (rbase + g) * r + col + 8);
+                    a3 = *reinterpret_cast<const uint32_t*>(U + (rbase + g + 8) * r + col + 8);
+                }
+            }
 #pragma unroll
             for (int n8 = 0; n8 < NT; ++n8) {
                 const uint16_t* trow = tt + (n8 * 8 + g) * tcols + tc0;
@@ -363,13 +400,19 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 filled |= 1u << stage;
                 fph = (fph & ~(1u << stage)) | (phase << stage);
                 const int urows = min(RA, p.N - n0);
-                const uint32_t ua = urows * ra * 2, ub = urows * rb * 2;
+                // fp16 U rows, or the int3 U^T block holding the item's features
+                const uint32_t ua = ra == 0 ? 0u : pa->lorc3 ? kBlockSB : urows * ra * 2;
+                const uint32_t ub = rb == 0 ? 0u : pb->lorc3 ? kBlockSB : urows * rb * 2;
+                const uint8_t* usa = pa->lorc3 ? reinterpret_cast<const uint8_t*>(pa->U) + (n0 >> 7) * kBlockSB
+                                               : reinterpret_cast<const uint8_t*>(pa->U + static_cast<size_t>(n0) * ra);
+                const uint8_t* usb = !GLU ? usa : pb->lorc3 ? reinterpret_cast<const uint8_t*>(pb->U) + (n0 >> 7) * kBlockSB
+                                                            : reinterpret_cast<const uint8_t*>(pb->U + static_cast<size_t>(n0) * rb);
                 const uint32_t tb = ntok * p.tcols * 2;
                 if (elect_one()) {
                     if (!header) stage_item[stage] = it;
                     mbar_arrive_expect_tx(fb, ua + ub + tb);
-                    if (ua) bulk_load_hint(st + kOffUA, pa->U + static_cast<size_t>(n0) * ra, ua, fb, pol);
-                    if (ub) bulk_load_hint(st + kOffUB, pb->U + static_cast<size_t>(n0) * rb, ub, fb, pol);
+                    if (ua) bulk_load_hint(st + kOffUA, usa, ua, fb, pol);
+                    if (ub) bulk_load_hint(st + kOffUB, usb, ub, fb, pol);
                     bulk_load(st + kOffT, p.t + static_cast<size_t>(row0) * p.tcols, tb, fb);
                 }
                 __syncwarp();
@@ -465,8 +508,10 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             }
             waited = false;
             const uint8_t* st = smem + stage * kStageBytes;
-            if (ntok > 8) lorc_compute<GLU, 2>(st, acc, warp, lane, ra, rb, p.tcols, p.t_col_b);
-            else lorc_compute<GLU, 1>(st, acc, warp, lane, ra, rb, p.tcols, p.t_col_b);
+            // int3 U^T blocks: the item's features start at n0 & 127 inside them
+            const bool u3a = pa->lorc3 != 0, u3b = GLU ? pb->lorc3 != 0 : u3a;
+            if (ntok > 8) lorc_compute<GLU, 2>(st, acc, warp, lane, ra, rb, p.tcols, p.t_col_b, u3a, u3b, n0 & 127);
+            else lorc_compute<GLU, 1>(st, acc, warp, lane, ra, rb, p.tcols, p.t_col_b, u3a, u3b, n0 & 127);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
             if (++stage == kStages) { stage = 0; phase ^= 1; }

@@ -123,6 +123,61 @@ __host__ __device__ constexpr float act_scale(int t, int f) {
 }
 
 // ---------------------------------------------------------------------------
+// int3 compensator blobs (one 64-row tile: U^T [r][N] or V [r][K], r <= 64)
+// ---------------------------------------------------------------------------
+
+// A blob block (one 64-row tile, one 128-code super-block): the rows' words
+// [64][12] u32, then the two groups' (s, z) pairs, 256 bytes each.
+constexpr int kBlobBlockBytes = 64 * 12 * 4 + 2 * 256;
+constexpr int kBlobWordBytes = 64 * 12 * 4;
+constexpr int kBlobGroupBytes = 256;
+
+// Byte offset of row j's three words of unit u of super-block b.  Unit u
+// holds the 16 codes at positions 16u..16u+15 of the super-block's first
+// group (codes 0..15 of the unit) and the 16 at 64+16u.. of its second
+// (codes 16..31).
+__device__ __forceinline__ int lorc_words_off(int j, int b, int u) { return b * kBlobBlockBytes + j * 48 + 12 * u; }
+
+// Unit and code index of position k (0..127) of a super-block.
+__device__ __forceinline__ int blob_unit(int k) { return (k & 63) >> 4; }
+__device__ __forceinline__ int blob_code(int k) { return (k & 15) + 16 * (k >> 6); }
+
+// Byte offset of row j's (s, z) fp16 pair for group g (64 codes along the row).
+__device__ __forceinline__ int lorc_sz_off(int j, int g) {
+    return (g >> 1) * kBlobBlockBytes + kBlobWordBytes + (g & 1) * kBlobGroupBytes +
+           (((j >> 4) * 8 + (j & 7)) * 4 + ((j >> 3) & 1) * 2) * 2;
+}
+
+// Code i (0..31) of a unit's three words: pair p = i / 2 < 15 sits in bits
+// 3 (p % 5) (+16 for the odd code) of word p / 5; codes 30 and 31 take bit t
+// from bits 15 and 31 of word t.
+__device__ __forceinline__ uint32_t unit_code(const uint32_t (&w)[3], int i) {
+    if (i < 30) {
+        const int p = i >> 1;
+        const uint32_t word = p < 5 ? w[0] : p < 10 ? w[1] : w[2];
+        return (word >> (3 * (p % 5) + 16 * (i & 1))) & 7u;
+    }
+    const int sh = i == 30 ? 15 : 31;
+    return ((w[0] >> sh) & 1u) | (((w[1] >> sh) & 1u) << 1) | (((w[2] >> sh) & 1u) << 2);
+}
+
+// The 16 values (q - z) * s of one group's half of a unit (codes 16 h ..
+// 16 h + 15, h = which group) as 8 fp16 pairs, in position order.
+__device__ __forceinline__ void unit_half_dequant(const uint32_t (&w)[3], int h, float s, float z,
+                                                  uint32_t (&out)[8]) {
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const float lo = (static_cast<float>(unit_code(w, 16 * h + 2 * m)) - z) * s;
+        const float hi = (static_cast<float>(unit_code(w, 16 * h + 2 * m + 1)) - z) * s;
+        out[m] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(lo))) |
+                 (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(hi))) << 16);
+    }
+}
+
+__device__ __forceinline__ float sz_scale(uint32_t sz) { return __half2float(__ushort_as_half(static_cast<uint16_t>(sz & 0xFFFFu))); }
+__device__ __forceinline__ float sz_zero(uint32_t sz) { return __half2float(__ushort_as_half(static_cast<uint16_t>(sz >> 16))); }
+
+// ---------------------------------------------------------------------------
 // PTX: mbarrier
 // ---------------------------------------------------------------------------
 

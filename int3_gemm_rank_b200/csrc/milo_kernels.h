@@ -38,9 +38,9 @@ constexpr int kTcTokens = 128;               // routed rows per tcgen05 work ite
 // One projection in the device table (device pointers and shape).
 struct alignas(64) ProjDev {
     const uint8_t* packed;      // blob of ceil(N/64) * (K/128) * kBlockSB bytes
-    const uint16_t* U;          // [N][rank] fp16, NULL when rank == 0
-    const uint16_t* V;          // [rank][K] fp16, NULL when rank == 0
-    int32_t rank, N, K, pad;
+    const uint16_t* U;          // [N][rank] fp16, or (lorc3) the blob of U^T [rank][N]; NULL when rank == 0
+    const uint16_t* V;          // [rank][K] fp16, or (lorc3) the blob of V [rank][K]; NULL when rank == 0
+    int32_t rank, N, K, lorc3;  // lorc3: the compensator is int3 (both blobs one 64-row tile high)
 };
 
 struct GemvParams {

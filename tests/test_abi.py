@@ -67,12 +67,12 @@ def test_prepare_validates_shapes_and_ranks(milo):
     nb = C.c_size_t()
     assert L.milo_table_bytes(3, C.byref(nb)) == 0 and nb.value % 64 == 0 and nb.value > 0
     fake = 0x10000
-    w = milo.milo_qweight(fake, None, None, 12)   # rank not a multiple of 8
+    w = milo.milo_qweight(fake, None, None, 12, 0)   # rank not a multiple of 8
     lin = milo.milo_linear(64, 128, 1, 64, 0, None)
     assert L.milo_linear_prepare(C.byref(lin), C.byref(w), C.c_void_p(fake), 1 << 20) == \
         milo.MILO_ERR_UNSUPPORTED_SHAPE
     lin = milo.milo_linear(64, 200, 1, 64, 0, None)            # K % 128
-    w = milo.milo_qweight(fake, None, None, 0)
+    w = milo.milo_qweight(fake, None, None, 0, 0)
     assert L.milo_linear_prepare(C.byref(lin), C.byref(w), C.c_void_p(fake), 1 << 20) == \
         milo.MILO_ERR_UNSUPPORTED_SHAPE
     lin = milo.milo_linear(64, 128, 1, 32, 0, None)            # group

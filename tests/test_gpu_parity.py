@@ -140,15 +140,15 @@ def test_route_flags_nan_logits(milo):
 # grouped linear with the compensator
 # ---------------------------------------------------------------------------
 
-def _linear_pair(milo, projs):
+def _linear_pair(milo, projs, lorc_int3=False):
     gpu = [milo.QWeight.quantize(f16_dev(p.W), f16_dev(p.U) if p.rank else None,
-                                 f16_dev(p.V) if p.rank else None) for p in projs]
-    ref = [oracle.quantize_projection(p.W, p.U, p.V) for p in projs]
+                                 f16_dev(p.V) if p.rank else None, lorc_int3=lorc_int3) for p in projs]
+    ref = [oracle.quantize_projection(p.W, p.U, p.V, lorc_int3=lorc_int3) for p in projs]
     return milo.GroupedLinear(gpu), ref
 
 
-def _linear_check(milo, projs, x_bits, x_dt, ids, k, out_dtypes=(torch.float32,)):
-    lin, ref = _linear_pair(milo, projs)
+def _linear_check(milo, projs, x_bits, x_dt, ids, k, out_dtypes=(torch.float32,), lorc_int3=False):
+    lin, ref = _linear_pair(milo, projs, lorc_int3)
     E = len(projs)
     T = x_bits.shape[0]
     r = milo.milo_route(None, k, False, E=E, ids=to_dev(ids.astype(np.int32)))
@@ -248,26 +248,26 @@ def test_linear_rejects_bad_shapes(milo):
 # full SwiGLU MoE layer (small shapes)
 # ---------------------------------------------------------------------------
 
-def gpu_layer(milo, wk):
+def gpu_layer(milo, wk, lorc_int3=False):
     experts = []
     for e in range(wk.n_experts):
         d = {}
         for name in ("w1", "w3", "w2"):
             P = wk.experts[e][name]
             d[name] = milo.QWeight.quantize(f16_dev(P.W), f16_dev(P.U) if P.rank else None,
-                                            f16_dev(P.V) if P.rank else None)
+                                            f16_dev(P.V) if P.rank else None, lorc_int3=lorc_int3)
         experts.append(d)
     return milo.MoELayer(experts, wk.n_routed, wk.n_shared, wk.top_k)
 
 
-def oracle_layer(wk):
+def oracle_layer(wk, lorc_int3=False):
     return [{name: oracle.quantize_projection(wk.experts[e][name].W, wk.experts[e][name].U,
-                                              wk.experts[e][name].V)
+                                              wk.experts[e][name].V, lorc_int3=lorc_int3)
              for name in ("w1", "w3", "w2")} for e in range(wk.n_experts)]
 
 
-def run_layer_parity(milo, wk, check_h=True, out_dtypes=(torch.float32,)):
-    layer = gpu_layer(milo, wk)
+def run_layer_parity(milo, wk, check_h=True, out_dtypes=(torch.float32,), lorc_int3=False):
+    layer = gpu_layer(milo, wk, lorc_int3)
     st = milo.new_status()
     r = milo.milo_route(f16_dev(wk.logits), wk.top_k, wk.renorm, dev_status=st)
     x = act_dev(wk.x, wk.x_dtype)
@@ -275,7 +275,7 @@ def run_layer_parity(milo, wk, check_h=True, out_dtypes=(torch.float32,)):
     assert _status(st) == 0
     ids, w, off, perm, inv, _ = oracle.route(wk.logits, wk.top_k, wk.renorm)
     assert np.array_equal(r["ids"].cpu().numpy(), ids)
-    ref = oracle_layer(wk)
+    ref = oracle_layer(wk, lorc_int3)
     y_ref, h_ref, st_ref = oracle.moe_forward(wk.x, wk.x_dtype == "bf16", ids, w, ref, wk.n_routed,
                                               wk.n_shared, wk.hidden, wk.inter, want_h=True)
     assert st_ref == 0
@@ -370,3 +370,44 @@ def test_moe_forward_cuda_graph_replay_bit_exact(milo, T):
     assert torch.equal(y_graph.view(torch.int32), y.view(torch.int32))
     assert not torch.equal(y_graph, y_eager)
     del g
+
+
+# --- int3 compensators: U^T and V packed like weights ---------------------------
+
+def test_linear_int3_compensator_decode_rows(milo, gemm_path):
+    """Few rows per expert (K-sliced down-projection), N = 256, K = 640 (odd
+    number of super-blocks), ranks 8 and 64."""
+    projs = [wl.make_projection("t_l3a", "w", e, 256, 640, r) for e, r in enumerate((8, 64))]
+    x = wl.gen_activations(np.random.default_rng(31), 6, 640, "bf16")
+    ids = np.array([[0], [1], [1], [0], [1], [1]], np.int32)
+    _linear_check(milo, projs, x, "bf16", ids, 1, lorc_int3=True)
+
+
+def test_linear_int3_compensator_many_rows(milo, gemm_path):
+    """300 rows over 2 experts (64-row down-projection tiles; the tcgen05 path
+    takes them), N = 384 (three 128-row weight tiles), K = 512, ranks 16 and 40."""
+    projs = [wl.make_projection("t_l3b", "w", e, 384, 512, r) for e, r in enumerate((16, 40))]
+    x = wl.gen_activations(np.random.default_rng(32), 300, 512, "bf16")
+    ids = np.random.default_rng(33).choice(2, size=(300, 1), p=[0.4, 0.6]).astype(np.int32)
+    _linear_check(milo, projs, x, "bf16", ids, 1, (torch.float32, torch.float16), lorc_int3=True)
+
+
+def test_moe_int3_compensator(milo, gemm_path):
+    wk = wl.small_moe("t_moe_l3", T=24, hidden=256, inter=384, n_routed=4, n_shared=1, top_k=2,
+                      rank_choices=(0, 16, 32))
+    run_layer_parity(milo, wk, lorc_int3=True)
+
+
+def test_moe_int3_compensator_many_tokens(milo, gemm_path):
+    wk = wl.small_moe("t_moe_l3b", T=200, hidden=256, inter=512, n_routed=2, n_shared=1, top_k=1,
+                      rank_choices=(8, 64))
+    run_layer_parity(milo, wk, lorc_int3=True)
+
+
+def test_int3_compensator_needs_n_multiple_of_128(milo):
+    P = wl.make_projection("t_l3c", "w", 0, 192, 256, 8)
+    w = milo.QWeight.quantize(f16_dev(P.W), f16_dev(P.U), f16_dev(P.V))
+    w.lorc_int3 = True     # fp16 factors declared int3 on an N the format cannot take
+    with pytest.raises(milo.MiloError) as e:
+        milo.GroupedLinear([w])
+    assert e.value.status == milo.MILO_ERR_UNSUPPORTED_SHAPE
