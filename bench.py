@@ -163,7 +163,7 @@ def describe(wk) -> str:
             f"T{wk.T} int3 g64 ranks={list(map(int, wk.ranks))}")
 
 
-def gpu_layer(milo, wk, torch):
+def gpu_layer(milo, wk, torch, lorc_int3: bool = False):
     experts = []
     for e in range(wk.n_experts):
         d = {}
@@ -173,13 +173,13 @@ def gpu_layer(milo, wk, torch):
             def dev(a):
                 return torch.from_numpy(a.view(np.int16)).view(torch.float16).cuda()
             d[n] = milo.QWeight.quantize(dev(P.W), dev(P.U) if P.rank else None,
-                                         dev(P.V) if P.rank else None)
+                                         dev(P.V) if P.rank else None, lorc_int3=lorc_int3)
         experts.append(d)
     torch.cuda.synchronize()
     return milo.MoELayer(experts, wk.n_routed, wk.n_shared, wk.top_k)
 
 
-def layer_bytes(wk, counts) -> dict:
+def layer_bytes(wk, counts, lorc_int3: bool = False) -> dict:
     """Algorithmic HBM bytes of one step: every active expert's packed codes
     (3/8 B per weight), fp16 scale and zero (4/64 B per weight), compensator U
     and V (fp16), plus activations in and out, for each kernel."""
@@ -189,14 +189,15 @@ def layer_bytes(wk, counts) -> dict:
     qz = lambda n, k: n * k * 3 // 8 + 2 * (k // 64) * n * 2   # codes + scale + zero
     glu = dict(weights=0, lorc_u=0, lorc_v=0)
     w2 = dict(weights=0, lorc_u=0, lorc_v=0)
+    cb = 7 / 16 if lorc_int3 else 2      # compensator bytes per element: int3 codes + s, z, or fp16
     for e in active:
         r1, r3, r2 = (wk.experts[e][n].rank for n in ("w1", "w3", "w2"))
         glu["weights"] += 2 * qz(I, H)
-        glu["lorc_u"] += (r1 + r3) * I * 2
-        glu["lorc_v"] += (r1 + r3) * H * 2
+        glu["lorc_u"] += (r1 + r3) * I * cb
+        glu["lorc_v"] += (r1 + r3) * H * cb
         w2["weights"] += qz(H, I)
-        w2["lorc_u"] += r2 * H * 2
-        w2["lorc_v"] += r2 * I * 2
+        w2["lorc_u"] += r2 * H * cb
+        w2["lorc_v"] += r2 * I * cb
     act_x = rows * H * 2
     act_h = rows * I * 2
     glu_kernel = glu["weights"] + glu["lorc_u"] + act_x + act_h + rows * 2 * 64 * 2
@@ -391,7 +392,7 @@ def run_milo(args):
     dist_init("nccl")
 
     wk = make_workload(args.workload, args.experts, args.tokens)
-    layer = gpu_layer(milo, wk, torch)
+    layer = gpu_layer(milo, wk, torch, args.lorc == "int3")
 
     def to_dev(a, dt):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(dt).to(dev)
@@ -436,7 +437,7 @@ def run_milo(args):
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {int(st.item())} on the bench workload")
     counts = np.diff(off.cpu().numpy())
-    bytes_ = layer_bytes(wk, counts)
+    bytes_ = layer_bytes(wk, counts, args.lorc == "int3")
 
     # --- the timed step: one CUDA graph of the whole step (route + layer), its
     # launches and their programmatic dependencies captured once and replayed
@@ -580,6 +581,7 @@ def finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, l
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": {"workload": describe(wk), "tokens_per_step": T, "x_dtype": wk.x_dtype,
+                   "compensator": "int3 (U^T and V packed like the weights)" if args.lorc == "int3" else "fp16",
                    "y_dtype": "bf16",
                    "l2": f"inputs larger than L2: {bytes_['weights_only'] / 1e6:.0f} MB of packed weights "
                          f"streamed per step vs {L2_BYTES / 1e6:.0f} MB L2; no flush",
@@ -620,6 +622,8 @@ def main(argv=None):
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--lorc", choices=("fp16", "int3"), default="fp16",
+                    help="compensator format: fp16 U, V (the configured workloads) or int3 blobs")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch the step's kernels one by one instead of replaying one CUDA graph")
     ap.add_argument("--experts", type=int, default=None, help="routed experts (profiler captures)")

@@ -511,31 +511,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     r = ra;
                     u3 = pa->lorc3 != 0;
                 }
-                uint32_t a[64];
-                if (u3) {
-                    // int3 U^T block: this row's feature, each rank row's code of it
-                    const uint8_t* blk = st + ((GLU && row >= 64) ? kTcOffUB : kTcOffUA);
-                    const int nl = ((w.ntile * RA) & 127) + (GLU ? (row & 63) : row);
-#pragma unroll
-                    for (int j = 0; j < 64; ++j) {
-                        const int slot = 2 * j;
-                        a[j] = (slot >= lo && slot < lo + r)
-                                   ? lorc3_value_pair(blk, slot - lo, nl)
-                                   : 0u;
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 64; ++j) {
-                        const int slot = 2 * j;
-                        a[j] = (slot >= lo && slot < lo + r) ? *reinterpret_cast<const uint32_t*>(src + (slot - lo)) : 0u;
-                    }
-                }
                 if (!warp_wait(&aempty[ab], aph ^ 1)) {
                     fail = true;
                     break;
                 }
                 tc_fence_after();
-                tc_st64(lane_base + kTcACol + 64 * ab, a);
+                if (u3) {
+                    // int3 U^T block: this row's feature, each rank row's code of
+                    // it, eight TMEM columns at a time (a rolled loop keeps the
+                    // code small)
+                    const uint8_t* blk = st + ((GLU && row >= 64) ? kTcOffUB : kTcOffUA);
+                    const int nl = ((w.ntile * RA) & 127) + (GLU ? (row & 63) : row);
+#pragma unroll 1
+                    for (int j0 = 0; j0 < 64; j0 += 8) {
+                        uint32_t v8[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int slot = 2 * (j0 + i);
+                            v8[i] = (slot >= lo && slot < lo + r) ? lorc3_value_pair(blk, slot - lo, nl) : 0u;
+                        }
+                        tc_st8(lane_base + kTcACol + 64 * ab + j0, v8);
+                    }
+                } else {
+                    uint32_t a[64];
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) {
+                        const int slot = 2 * j;
+                        a[j] = (slot >= lo && slot < lo + r) ? *reinterpret_cast<const uint32_t*>(src + (slot - lo)) : 0u;
+                    }
+                    tc_st64(lane_base + kTcACol + 64 * ab, a);
+                }
                 tc_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -552,7 +557,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     } else {
         // ---------------------------------------------------------------- fold + epilogue
         const int quarter = warp & 3;
-        const int th = (warp - 6) >> 2;                    // routed rows 48 * th .. 48 * th + 47
+        const int th = (warp - 6) >> 2;                    // routed rows kTcHalf * th .. kTcHalf * (th + 1) - 1
         const int row = 32 * quarter + lane;
         const uint32_t lane_base = tbase + (static_cast<uint32_t>(32 * quarter) << 16);
         const int half = row >> 6, r64 = row & 63;

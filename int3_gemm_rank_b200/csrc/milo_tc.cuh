@@ -40,6 +40,12 @@ __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sy
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Store 64 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tc_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                   "r"(v[7]) : "memory");
+}
+
 __device__ __forceinline__ void tc_st64(uint32_t taddr, const uint32_t (&v)[64]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {"

@@ -37,20 +37,20 @@ def milo():
 
 
 
-def _gpu_proj(milo, P):
+def _gpu_proj(milo, P, lorc_int3=False):
     return milo.QWeight.quantize(f16_dev(P.W), f16_dev(P.U) if P.rank else None,
-                                 f16_dev(P.V) if P.rank else None)
+                                 f16_dev(P.V) if P.rank else None, lorc_int3=lorc_int3)
 
 
-def _oracle_projs(projs):
+def _oracle_projs(projs, lorc_int3=False):
     with ThreadPoolExecutor(8) as ex:
-        return list(ex.map(lambda P: oracle.quantize_projection(P.W, P.U, P.V), projs))
+        return list(ex.map(lambda P: oracle.quantize_projection(P.W, P.U, P.V, lorc_int3=lorc_int3), projs))
 
 
-def _layers(milo, wk):
+def _layers(milo, wk, lorc_int3=False):
     names = ("w1", "w3", "w2")
-    gpu = [{n: _gpu_proj(milo, wk.experts[e][n]) for n in names} for e in range(wk.n_experts)]
-    flat = _oracle_projs([wk.experts[e][n] for e in range(wk.n_experts) for n in names])
+    gpu = [{n: _gpu_proj(milo, wk.experts[e][n], lorc_int3) for n in names} for e in range(wk.n_experts)]
+    flat = _oracle_projs([wk.experts[e][n] for e in range(wk.n_experts) for n in names], lorc_int3)
     ref = [{n: flat[3 * e + i] for i, n in enumerate(names)} for e in range(wk.n_experts)]
     return milo.MoELayer(gpu, wk.n_routed, wk.n_shared, wk.top_k), ref
 
@@ -82,8 +82,8 @@ def test_single_expert_decode_full(milo):
     assert err <= REL_TOL, err
 
 
-def _layer_full(milo, wk):
-    layer, ref = _layers(milo, wk)
+def _layer_full(milo, wk, lorc_int3=False):
+    layer, ref = _layers(milo, wk, lorc_int3)
     r, ids, w, inv = _route(milo, wk)
     st = milo.new_status()
     y = layer(act_dev(wk.x, wk.x_dtype), r, out_dtype=torch.float32, dev_status=st)
@@ -107,6 +107,11 @@ def test_mixtral_decode_layer_full(milo):
 
 def test_deepseek_decode_layer_full(milo):
     _layer_full(milo, wl.deepseek())
+
+
+def test_mixtral_decode_layer_full_int3_compensators(milo):
+    """The Mixtral-shaped decode layer with U^T and V quantised to int3 too."""
+    _layer_full(milo, wl.mixtral(), lorc_int3=True)
 
 
 def test_w1_sweep_zipf(milo):
