@@ -71,6 +71,10 @@ def lib():
         L.milo_ref_moe_forward.argtypes = [vp, i, i, i, i, i, i, i, i, vp, vp, C.POINTER(Proj),
                                            C.POINTER(Proj), C.POINTER(Proj), vp, vp, i]
         L.milo_ref_moe_forward.restype = i
+        f = C.c_float
+        L.milo_ref_hqq.argtypes = [vp, i, i, i, f, f, vp, vp, vp]; L.milo_ref_hqq.restype = i
+        L.milo_ref_hqq_trace.argtypes = [vp, i, f, f, vp, vp, vp, vp, vp]
+        L.milo_ref_hqq_trace.restype = i
         _lib = L
     return _lib
 
@@ -243,3 +247,138 @@ def moe_forward(x_bits: np.ndarray, x_is_bf16: bool, ids: np.ndarray, w: np.ndar
                                     _p(ids), _p(w), arr["w1"], arr["w3"], arr["w2"], _p(y),
                                     _p(h) if want_h else None, nthreads)
     return y, h, st
+
+
+# ---------------------------------------------------------------------------
+# Offline MiLo quantiser ("MiLo Algorithm: Mixture of Low-Rank Compensators":
+# HQQ initial quantisation, a rank-r compensator from the SVD of the residual,
+# and rounds that re-quantise W - U V and recompute U V from the new residual).
+
+HQQ_ITERS, HQQ_BETA, HQQ_KAPPA = 20, 10.0, 1.01
+
+
+def hqq(T: np.ndarray, iters: int = HQQ_ITERS, beta: float = HQQ_BETA, kappa: float = HQQ_KAPPA):
+    """HQQ int3 quantisation of an fp32 target [N, K] (groups of 64 along K).
+    Returns (q u8 [N, K], scale, zero fp16 bits [K/64, N], status)."""
+    T = _c(T, np.float32)
+    N, K = T.shape
+    assert K % 64 == 0
+    q = np.zeros((N, K), np.uint8)
+    sc = np.zeros((K // 64, N), np.uint16)
+    ze = np.zeros((K // 64, N), np.uint16)
+    st = lib().milo_ref_hqq(_p(T), N, K, int(iters), float(beta), float(kappa), _p(q), _p(sc), _p(ze))
+    return q, sc, ze, st
+
+
+def hqq_trace(t: np.ndarray, iters: int, beta: float, kappa: float):
+    """One group of 64 fp32 targets.  Returns (q, s bits, z bits, z before each
+    iteration and after the last [iters + 1], L1 error of each iteration [iters])."""
+    t = _c(t, np.float32)
+    assert t.shape == (64,)
+    q = np.zeros(64, np.uint8)
+    s = np.zeros(1, np.uint16)
+    z = np.zeros(1, np.uint16)
+    zt = np.zeros(iters + 1, np.float32)
+    et = np.zeros(max(iters, 1), np.float32)
+    lib().milo_ref_hqq_trace(_p(t), int(iters), float(beta), float(kappa), _p(q), _p(s), _p(z),
+                             _p(zt), _p(et))
+    return q, int(s[0]), int(z[0]), zt, et[:iters]
+
+
+def _f16(bits) -> np.ndarray:
+    return np.asarray(bits, np.uint16).view(np.float16).astype(np.float32)
+
+
+def lorc_target(W_bits: np.ndarray, U_bits=None, V_bits=None) -> np.ndarray:
+    """The quantisation target W - U V in fp32: starting from W, one rank term
+    U[:, p] V[p, :] at a time, each product and difference rounded to fp32."""
+    T = _f16(W_bits)
+    if U_bits is None or np.asarray(U_bits).size == 0:
+        return T
+    U = _f16(U_bits)
+    V = _f16(V_bits)
+    for p in range(U.shape[1]):
+        T = (T - (U[:, p:p + 1] * V[p:p + 1, :]).astype(np.float32)).astype(np.float32)
+    return T
+
+
+def residual(W_bits: np.ndarray, q: np.ndarray, scale: np.ndarray, zero: np.ndarray) -> np.ndarray:
+    """R = W - (q - z) s in fp32 (the residual the compensator approximates)."""
+    N, K = q.shape
+    s = np.repeat(_f16(scale).T, 64, axis=1)
+    z = np.repeat(_f16(zero).T, 64, axis=1)
+    d = ((q.astype(np.float32) - z).astype(np.float32) * s).astype(np.float32)
+    return (_f16(W_bits) - d).astype(np.float32)
+
+
+def _orth(Y: np.ndarray) -> np.ndarray:
+    return np.linalg.qr(Y, mode="reduced")[0]
+
+
+def _split(Y: np.ndarray, B: np.ndarray, r: int):
+    """Rayleigh-Ritz on R ~ Y B (Y orthonormal columns): the top-r singular
+    triplets of B, returned balanced as U = Y P_r S^(1/2), V = S^(-1/2) P_r^T B."""
+    lam, P = np.linalg.eigh(B @ B.T)
+    order = np.argsort(-lam, kind="stable")
+    lam, P = lam[order][:r], P[:, order][:, :r]
+    sig = np.sqrt(np.clip(lam, 0.0, None))
+    live = sig > (sig[0] * 1e-12 if r and sig[0] > 0 else np.inf)
+    root = np.where(live, np.sqrt(sig), 0.0)
+    inv = np.where(live, 1.0 / np.where(live, np.sqrt(sig), 1.0), 0.0)
+    return (Y @ P) * root[None, :], (P.T @ B) * inv[:, None]
+
+
+def rsvd(R: np.ndarray, r: int, omega: np.ndarray, power_iters: int):
+    """Rank-r compensator of R [N, K] by randomized subspace iteration (Halko,
+    Martinsson and Tropp 2011): Y = orth(R omega), then power_iters times
+    Z = orth(R^T Y), Y = orth(R Z); B = Y^T R; U, V from _split().  omega
+    [K, l] (l >= r) is the random test matrix, an input.  fp64 throughout."""
+    R = np.asarray(R, np.float64)
+    Y = _orth(R @ np.asarray(omega, np.float64))
+    for _ in range(power_iters):
+        Y = _orth(R @ _orth(R.T @ Y))
+    return _split(Y, Y.T @ R, r)
+
+
+def svd_truncated(R: np.ndarray, r: int):
+    """The exact rank-r truncated SVD of R, balanced like rsvd(); and the
+    optimal error sqrt(sum_{i >= r} sigma_i^2) (Eckart-Young)."""
+    u, sg, vt = np.linalg.svd(np.asarray(R, np.float64), full_matrices=False)
+    root = np.sqrt(sg[:r])
+    return u[:, :r] * root[None, :], vt[:r] * root[:, None], float(np.sqrt(np.sum(sg[r:] ** 2)))
+
+
+def quantize_lorc(W_bits: np.ndarray, rank: int, rounds: int, omega: np.ndarray, power_iters: int = 2,
+                  iters: int = HQQ_ITERS, beta: float = HQQ_BETA, kappa: float = HQQ_KAPPA):
+    """The offline MiLo quantiser.  Round 0: HQQ(W), R = W - W_hat, (U, V) =
+    rank-r compensator of R.  Each further round: HQQ(W - U V) with the fp16
+    U, V of the previous round, a new residual and a new compensator.  Every
+    round's error ||W - W_hat - U V||_F (fp16 U, V) is recorded; the round with
+    the lowest error (the first on ties) is returned.
+
+    Returns dict(q, scale, zero, U, V (fp16 bits), err [rounds + 1], best, status)."""
+    W = _c(W_bits, np.uint16)
+    N, K = W.shape
+    U16 = V16 = None
+    errs, best, status = [], None, 0
+    for rd in range(rounds + 1):
+        T = lorc_target(W, U16, V16)
+        q, sc, ze, st = hqq(T, iters, beta, kappa)
+        status |= st
+        R = residual(W, q, sc, ze)
+        if rank > 0:
+            U, V = rsvd(R, rank, omega, power_iters)
+            U16 = U.astype(np.float16).view(np.uint16)
+            V16 = V.astype(np.float16).view(np.uint16)
+            E = R.astype(np.float64) - _f16(U16).astype(np.float64) @ _f16(V16).astype(np.float64)
+        else:
+            U16 = np.zeros((N, 0), np.uint16)
+            V16 = np.zeros((0, K), np.uint16)
+            E = R.astype(np.float64)
+        errs.append(float(np.sqrt(np.sum(E * E))))
+        if best is None or errs[-1] < errs[best["round"]]:
+            best = dict(round=rd, q=q, scale=sc, zero=ze, U=U16, V=V16)
+        if rank == 0:
+            break
+    return dict(q=best["q"], scale=best["scale"], zero=best["zero"], U=best["U"], V=best["V"],
+                err=np.array(errs), best=best["round"], status=status)

@@ -267,6 +267,130 @@ void milo_ref_dequant(const uint8_t* q, const uint16_t* scale, const uint16_t* z
 }
 
 /* ------------------------------------------------------------------------ */
+/* HQQ: the initial quantisation of the offline MiLo quantiser              */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * "MiLo Algorithm: Mixture of Low-Rank Compensators", step 1 ("Initial
+ * Quantization"): the weights are first quantised with HQQ (half-quadratic
+ * quantisation), which needs no calibration data and treats quantisation as
+ * an optimisation problem.  The pages give no more detail; HQQ as published
+ * (Badri and Shaji, 2023) keeps the min/max scale and fits the zero point z of
+ * each group by half-quadratic splitting of an lp error (p < 1):
+ *     q      = clamp(rint(t / s + z), 0, 7)
+ *     e      = t - (q - z) s                     the group's error
+ *     w_e    = shrink(e)                          proximal step on |.|^p
+ *     z_next = mean(q - (t - w_e) / s)            least-squares zero given w_e
+ *     beta   = kappa * beta
+ * with shrink(e) = sign(e) max(|e| - |e|^(p-1) / beta, 0).
+ *
+ * Readings (listed with the design notes too):
+ *   - p = 1/2, so |e|^(p-1) / beta = 1 / (sqrt(|e|) beta) uses only IEEE
+ *     square root and division (HQQ's own default is p = 0.7);
+ *   - every step is fp32, in the order written here (no fused multiply-add),
+ *     sums run over the group's 64 values in index order; quantised codes are
+ *     decided in fp32 on both sides;
+ *   - HQQ stops when its error stops falling; here each group keeps the zero
+ *     point whose L1 error sum_i |e_i| was lowest over the iterations (the
+ *     error of a group depends only on its own zero point), first one on ties;
+ *   - the kept zero point is rounded to fp16 (the storage format), and the
+ *     codes are then re-derived from it exactly as the round-to-nearest
+ *     quantiser does, so with one iteration HQQ equals round-to-nearest.
+ *
+ * hqq_group() quantises one group of 64 fp32 targets t.  z_trace (iters + 1)
+ * and err_trace (iters), when not NULL, receive the zero point before each
+ * iteration and after the last, and each iteration's L1 error.
+ */
+static int hqq_group(const float* t, int iters, float beta0, float kappa, uint8_t* q_out,
+                     uint16_t* s_out, uint16_t* z_out, float* z_trace, float* err_trace) {
+    int status = 0;
+    float mn = INFINITY, mx = -INFINITY;
+    for (int i = 0; i < 64; ++i) {
+        float v = t[i];
+        if (!isfinite(v)) status |= REF_NONFINITE;
+        if (v < mn) mn = v;
+        if (v > mx) mx = v;
+    }
+    float range = mx - mn;
+    uint16_t s_h = milo_ref_f2h(range / 7.0f);
+    if ((s_h & 0x7FFF) == 0) s_h = 0x3C00;
+    float s = h2f(s_h);
+    float z = -mn / s;
+    float beta = beta0;
+    float best_err = INFINITY, best_z = z;
+    if (z_trace) z_trace[0] = z;
+    for (int it = 0; it < iters; ++it) {
+        float err = 0.0f, acc = 0.0f;
+        for (int i = 0; i < 64; ++i) {
+            float v = t[i] / s;
+            v = v + z;
+            float r = nearbyintf(v);
+            if (!(r >= 0.0f)) r = 0.0f;
+            if (r > 7.0f) r = 7.0f;
+            float wr = r - z;
+            wr = wr * s;
+            float e = t[i] - wr;
+            float a = fabsf(e);
+            err = err + a;
+            float w_e = 0.0f;                 /* shrink(e), p = 1/2 */
+            if (a > 0.0f) {
+                float d = sqrtf(a);
+                d = d * beta;
+                float m = a - 1.0f / d;
+                if (m > 0.0f) w_e = e < 0.0f ? -m : m;
+            }
+            float u = t[i] - w_e;
+            u = u / s;
+            acc = acc + (r - u);
+        }
+        if (err_trace) err_trace[it] = err;
+        if (err < best_err) {
+            best_err = err;
+            best_z = z;
+        }
+        z = acc * 0.015625f;                  /* mean over 64 values */
+        beta = beta * kappa;
+        if (z_trace) z_trace[it + 1] = z;
+    }
+    uint16_t z_h = milo_ref_f2h(best_z);
+    float zf = h2f(z_h);
+    if (!isfinite(s) || !isfinite(zf)) status |= REF_FP16_RANGE;
+    *s_out = s_h;
+    *z_out = z_h;
+    for (int i = 0; i < 64; ++i) {
+        float v = t[i] / s;
+        v = v + zf;
+        float r = nearbyintf(v);
+        if (!(r >= 0.0f)) r = 0.0f;
+        if (r > 7.0f) r = 7.0f;
+        q_out[i] = (uint8_t)r;
+    }
+    return status;
+}
+
+/*
+ * HQQ quantisation of an fp32 target T [N, K] (K a multiple of 64) in groups
+ * of 64 along K.  Outputs as milo_ref_quantize(): codes q [N, K], scale and
+ * zero fp16 [K/64, N].  Returns REF_* status bits.
+ */
+int milo_ref_hqq(const float* T, int N, int K, int iters, float beta0, float kappa,
+                 uint8_t* q, uint16_t* scale, uint16_t* zero) {
+    int status = 0, G = K / 64;
+    for (int n = 0; n < N; ++n)
+        for (int j = 0; j < G; ++j)
+            status |= hqq_group(T + (size_t)n * K + (size_t)j * 64, iters, beta0, kappa,
+                                q + (size_t)n * K + (size_t)j * 64, &scale[(size_t)j * N + n],
+                                &zero[(size_t)j * N + n], NULL, NULL);
+    return status;
+}
+
+/* One group with its zero-point and error trajectory (for the pins). */
+int milo_ref_hqq_trace(const float* t, int iters, float beta0, float kappa, uint8_t* q,
+                       uint16_t* s, uint16_t* z, float* z_trace, float* err_trace) {
+    return hqq_group(t, iters, beta0, kappa, q, s, z, z_trace, err_trace);
+}
+
+/* ------------------------------------------------------------------------ */
 /* routing                                                                  */
 /* ------------------------------------------------------------------------ */
 
