@@ -40,7 +40,10 @@
  *     weights renormalised over the top-k, or taken from the softmax over all
  *     experts when renormalisation is off;
  *   - SwiGLU experts, h = silu(x W1^T) * (x W3^T) rounded to fp16 because
- *     activations are FP16; shared experts have weight 1.
+ *     activations are FP16; shared experts have weight 1;
+ *   - offline quantiser: HQQ with p = 1/2 shrinkage in fp32, each group keeping
+ *     the zero point of lowest L1 error (see milo_ref_hqq()); the compensator
+ *     and the refinement rounds are in oracle/__init__.py (numpy, fp64).
  */
 #include <math.h>
 #include <pthread.h>

@@ -40,6 +40,12 @@ MUTANTS = {
     "gather_wrong_token": ("X + (size_t)(rows[m] / k) * H", "X + (size_t)(rows[m] % T) * H"),
     "perm_descending": ("int p = offsets[e] + count[e]++;", "int p = offsets[e + 1] - 1 - count[e]++;"),
     "f2h_truncate": ("double m = nearbyint(ldexp(a, 10 - e));", "double m = floor(ldexp(a, 10 - e));"),
+    "hqq_shrink_without_sqrt": ("float d = sqrtf(a);", "float d = a;"),
+    "hqq_shrink_sign": ("if (m > 0.0f) w_e = e < 0.0f ? -m : m;", "if (m > 0.0f) w_e = e < 0.0f ? m : -m;"),
+    "hqq_kappa_ignored": ("beta = beta * kappa;", "beta = beta * 1.0f;"),
+    "hqq_mean_over_63": ("z = acc * 0.015625f;", "z = acc / 63.0f;"),
+    "hqq_best_zero_not_kept": ("best_err = err;\n            best_z = z;", "best_err = err;"),
+    "hqq_l2_error": ("err = err + a;", "err = err + a * a;"),
 }
 
 
@@ -56,6 +62,7 @@ def test_mutant_is_caught(name, tmp_path):
                            "-shared", "-pthread", str(c_path), "-o", str(so_path), "-lm"])
     env = dict(os.environ, MILO_ORACLE_LIB=str(so_path))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_lorc_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
