@@ -133,6 +133,93 @@ MILO_API milo_status milo_unpack(const void* packed, int32_t N, int32_t K, uint8
                         void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Offline MiLo quantiser                                                   */
+/* ------------------------------------------------------------------------ */
+/*
+ * "MiLo: Efficient Quantized MoE Inference with Mixture of Low-Rank
+ * Compensators", section "MiLo Algorithm: Mixture of Low-Rank Compensators":
+ * (1) the weights are quantised with HQQ (half-quadratic quantisation, no
+ * calibration data); (2) the residual W - W_quant is approximated by the top-r
+ * singular triplets of its SVD, U V; then quantisation and compensation are
+ * refined in turn: W_quant from W - U V, U V from the new residual.
+ *
+ * HQQ here (per group of 64 along K, all fp32 in this order, no FMA):
+ *     s = fp16((max - min) / 7) (1 when it rounds to 0), z = -min / s, beta = hqq_beta
+ *     repeat hqq_iters times:
+ *         q = clamp(rint(t / s + z), 0, 7);  e = t - (q - z) s
+ *         L1 = sum |e| (index order); remember z if L1 is the lowest so far
+ *         w_e = sign(e) max(|e| - 1 / (sqrt|e| beta), 0)     (lp shrinkage, p = 1/2)
+ *         z = (sum over the group of q - (t - w_e) / s) * (1/64);  beta *= hqq_kappa
+ *     z := fp16(remembered z); q = clamp(rint(t / s + z), 0, 7)  (as milo_pack)
+ * With hqq_iters <= 1 this is exactly milo_pack's round-to-nearest quantiser.
+ */
+
+/*
+ * milo_hqq_pack -- HQQ-quantise the target t = W - U V and pack it.
+ *   W fp16 [N, K] row-major (K % 128 == 0).  U fp16 [N, rank], V fp16
+ *   [rank, K] row-major, or rank = 0 and both NULL (t = W).  The target is
+ *   formed in fp32 one rank term at a time: t = W, then for p = 0..rank-1
+ *   t = t - U[n, p] * V[p, k] (product and difference each rounded to fp32).
+ *   packed: the blob of milo_packed_bytes(N, K) bytes (16-byte aligned).
+ *   residual: NULL, or f32 [N, K] receiving W - (q - z) s (fp32: the
+ *   difference q - z, the product, then W minus it), the residual a
+ *   compensator approximates.
+ * Errors: K % 128 != 0, rank > 64 -> UNSUPPORTED_SHAPE; N, K <= 0, rank < 0,
+ * hqq_iters outside 0..1000, beta or kappa not finite and positive, NULL W or
+ * packed, U or V NULL with rank > 0 -> INVALID_ARG.  Device: NONFINITE for
+ * NaN/Inf targets, FP16_RANGE when s or z overflows fp16.  All pointers are
+ * caller-owned device memory; stream-ordered, no host synchronisation.
+ */
+MILO_API milo_status milo_hqq_pack(const uint16_t* W, const uint16_t* U, const uint16_t* V, int32_t rank,
+                                   int32_t N, int32_t K, int32_t hqq_iters, float hqq_beta,
+                                   float hqq_kappa, void* packed, float* residual, int32_t* dev_status,
+                                   void* stream);
+
+typedef struct milo_lorc_params {
+    int32_t rank;         /* r: 0..64 */
+    int32_t rounds;       /* refinement rounds after the first: 0..16 (ignored when r = 0) */
+    int32_t sketch;       /* l: columns of the random test matrix, r <= l <= 128 (r > 0) */
+    int32_t power_iters;  /* subspace iterations q: 0..8 */
+    int32_t hqq_iters;    /* 0..1000 */
+    float hqq_beta;       /* initial shrinkage penalty, finite and > 0 */
+    float hqq_kappa;      /* penalty growth per iteration, finite and > 0 */
+} milo_lorc_params;
+
+/* Workspace bytes of milo_quantize_lorc for a weight [N, K]. */
+MILO_API milo_status milo_quantize_lorc_workspace(int32_t N, int32_t K, const milo_lorc_params* params,
+                                                  size_t* bytes);
+
+/*
+ * milo_quantize_lorc -- the offline MiLo quantiser of one weight W fp16
+ * [N, K] (K % 128 == 0).  Round 0: HQQ(W) (milo_hqq_pack), R = W - W_hat, and
+ * the rank-r compensator of R.  Rounds 1..rounds: HQQ(W - U V) with the fp16
+ * U, V of the round before, the new residual and its compensator.
+ *
+ * Compensator of R [N, K] (randomized subspace iteration, Halko, Martinsson
+ * and Tropp 2011): Y = orth(R omega); q times Y = orth(R orth(R^T Y));
+ * B = Y^T R; the eigenpairs of B B^T (descending lambda) give sigma_i =
+ * sqrt(lambda_i), and, for the top r, U = Y P_r sigma^(1/2) [N, r],
+ * V = sigma^(-1/2) P_r^T B [r, K] (a direction with sigma below 1e-12 sigma_0
+ * gets zero U and V).  orth() is Cholesky QR applied twice (fp64 Gram and
+ * Cholesky, fp32 products); eigenpairs by cyclic Jacobi in fp64.
+ *   omega: f32 [K, sketch] row-major, the random test matrix (an input: the
+ *   caller draws it, e.g. standard normal); NULL when r = 0.
+ *   packed (milo_packed_bytes), U fp16 [N, r], V fp16 [r, K]: the round with
+ *   the lowest error (the first on ties); U, V NULL when r = 0.
+ *   err: NULL, or f32 [rounds + 1] (1 when r = 0) receiving each round's
+ *   ||W - W_hat - U V||_F (fp16 U, V; accumulated in fp64).
+ *   ws: milo_quantize_lorc_workspace bytes, 256-byte aligned, caller-owned.
+ * Errors as milo_hqq_pack, plus: params NULL, rank outside 0..64, rounds,
+ * sketch or power_iters out of range, omega / U / V NULL with r > 0, ws too
+ * small or unaligned -> INVALID_ARG / WORKSPACE.  Stream-ordered, no host
+ * synchronisation; deterministic for fixed inputs.
+ */
+MILO_API milo_status milo_quantize_lorc(const uint16_t* W, int32_t N, int32_t K,
+                                        const milo_lorc_params* params, const float* omega,
+                                        void* packed, uint16_t* U, uint16_t* V, float* err, void* ws,
+                                        size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Routing                                                                  */
 /* ------------------------------------------------------------------------ */
 /*

@@ -32,7 +32,8 @@ EXPORTS = ("milo_status_str", "milo_last_error", "milo_version", "milo_pack", "m
            "milo_route", "milo_table_bytes", "milo_linear_prepare", "milo_layer_prepare",
            "milo_linear_workspace_bytes", "milo_moe_workspace_bytes", "milo_grouped_linear",
            "milo_moe_forward", "milo_moe_h_offset", "milo_set_profile_events",
-           "milo_grouped_linear_noalloc", "milo_packed_bytes")
+           "milo_grouped_linear_noalloc", "milo_packed_bytes", "milo_hqq_pack",
+           "milo_quantize_lorc_workspace", "milo_quantize_lorc")
 
 
 class MiloError(RuntimeError):
@@ -62,6 +63,12 @@ class milo_moe_layer(C.Structure):
 
 
 _lib = None
+
+
+class milo_lorc_params(C.Structure):
+    _fields_ = [("rank", C.c_int32), ("rounds", C.c_int32), ("sketch", C.c_int32),
+                ("power_iters", C.c_int32), ("hqq_iters", C.c_int32), ("hqq_beta", C.c_float),
+                ("hqq_kappa", C.c_float)]
 
 
 def lib() -> C.CDLL:
@@ -104,6 +111,14 @@ def lib() -> C.CDLL:
         L.milo_grouped_linear_noalloc.argtypes = [C.POINTER(milo_linear), vp, C.c_int, i32, i32, vp, vp,
                                                   vp, C.c_int, vp, vp]
         L.milo_grouped_linear_noalloc.restype = C.c_int
+        f32 = C.c_float
+        L.milo_hqq_pack.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, f32, vp, vp, vp, vp]
+        L.milo_hqq_pack.restype = C.c_int
+        L.milo_quantize_lorc_workspace.argtypes = [i32, i32, C.POINTER(milo_lorc_params), C.POINTER(sz)]
+        L.milo_quantize_lorc_workspace.restype = C.c_int
+        L.milo_quantize_lorc.argtypes = [vp, i32, i32, C.POINTER(milo_lorc_params), vp, vp, vp, vp, vp, vp, sz,
+                                         vp, vp]
+        L.milo_quantize_lorc.restype = C.c_int
         _lib = L
     return _lib
 
@@ -172,6 +187,73 @@ def milo_unpack(packed: torch.Tensor, N: int, K: int) -> torch.Tensor:
     codes = torch.empty((N, K), dtype=torch.uint8, device=packed.device)
     _check(lib().milo_unpack(_ptr(packed), N, K, _ptr(codes), _stream()), "milo_unpack")
     return codes
+
+
+# ---------------------------------------------------------------------------
+# offline MiLo quantiser
+# ---------------------------------------------------------------------------
+
+HQQ_ITERS, HQQ_BETA, HQQ_KAPPA = 20, 10.0, 1.01
+
+
+def milo_hqq_pack(W: torch.Tensor, U: torch.Tensor | None = None, V: torch.Tensor | None = None,
+                  iters: int = HQQ_ITERS, beta: float = HQQ_BETA, kappa: float = HQQ_KAPPA,
+                  residual: bool = False, dev_status: torch.Tensor | None = None):
+    """HQQ-quantise W - U V (fp16 W [N, K], U [N, r], V [r, K]) and pack it.
+    Returns (blob uint8, residual f32 [N, K] = W - W_hat, or None)."""
+    _cuda(W, "W")
+    N, K = W.shape
+    r = 0 if U is None else U.shape[1]
+    for t, name in ((U, "U"), (V, "V")):
+        if t is not None:
+            _cuda(t, name)
+    nbytes = milo_packed_bytes(N, K) if K > 0 and K % 128 == 0 and N > 0 else 16
+    blob = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    R = torch.empty((N, K), dtype=torch.float32, device=W.device) if residual else None
+    _check(lib().milo_hqq_pack(_ptr(W), _ptr(U), _ptr(V), r, N, K, iters, beta, kappa, _ptr(blob), _ptr(R),
+                               _ptr(dev_status), _stream()), "milo_hqq_pack")
+    return blob, R
+
+
+def lorc_params(rank: int, rounds: int = 3, sketch: int | None = None, power_iters: int = 2,
+                iters: int = HQQ_ITERS, beta: float = HQQ_BETA, kappa: float = HQQ_KAPPA) -> milo_lorc_params:
+    if sketch is None:
+        sketch = min(128, max(16, 2 * rank)) if rank > 0 else 0
+    return milo_lorc_params(rank, rounds, sketch, power_iters, iters, beta, kappa)
+
+
+def milo_quantize_lorc_workspace(N: int, K: int, params: milo_lorc_params) -> int:
+    nb = C.c_size_t()
+    _check(lib().milo_quantize_lorc_workspace(N, K, C.byref(params), C.byref(nb)), "milo_quantize_lorc_workspace")
+    return nb.value
+
+
+def milo_quantize_lorc(W: torch.Tensor, params: milo_lorc_params, omega: torch.Tensor | None = None,
+                       dev_status: torch.Tensor | None = None):
+    """The offline MiLo quantiser of W fp16 [N, K]: HQQ, the rank-r compensator of
+    the residual, and params.rounds refinement rounds.  omega: f32 [K, sketch],
+    the random test matrix.  Returns (QWeight with fp16 U, V of the best round,
+    per-round errors f32 [rounds + 1])."""
+    _cuda(W, "W")
+    N, K = W.shape
+    r = params.rank
+    if r > 0:
+        if omega is None or omega.dtype != torch.float32 or tuple(omega.shape) != (K, params.sketch):
+            raise ValueError("omega must be float32 [K, sketch]")
+        _cuda(omega, "omega")
+    nbytes = milo_packed_bytes(N, K) if K > 0 and K % 128 == 0 and N > 0 else 16
+    blob = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    U = torch.empty((N, r), dtype=torch.float16, device=W.device) if r > 0 else None
+    V = torch.empty((r, K), dtype=torch.float16, device=W.device) if r > 0 else None
+    n_err = params.rounds + 1 if r > 0 else 1
+    err = torch.empty(n_err, dtype=torch.float32, device=W.device)
+    ws_bytes = milo_quantize_lorc_workspace(N, K, params)
+    ws = torch.empty(ws_bytes + 256, dtype=torch.uint8, device=W.device)
+    wp, _ = _aligned_view(ws, 256, ws_bytes)
+    _check(lib().milo_quantize_lorc(_ptr(W), N, K, C.byref(params), _ptr(omega), _ptr(blob), _ptr(U), _ptr(V),
+                                    _ptr(err), C.c_void_p(wp), ws_bytes, _ptr(dev_status), _stream()),
+           "milo_quantize_lorc")
+    return QWeight(blob, N, K, U, V, rank=r), err
 
 
 # ---------------------------------------------------------------------------

@@ -7,25 +7,12 @@
 // asymmetric min/max (the paper starts from HQQ; synthetic weights use RTN).
 #include <cuda_runtime.h>
 
+#include "milo_blob.cuh"
 #include "milo_device.cuh"
 #include "milo_host.h"
 #include "milo_kernels.h"
 
 namespace milo {
-
-// Device blob (milo.h): one block per (64-row tile, super-block) = the tile's
-// words for the super-block, then its two groups' scales and zeros as (s, z)
-// pairs of rows r and r + 8 of each 16-row block.  Byte offsets of row n's
-// words for super-block b and of its scale for group j (its zero follows 2
-// bytes later).
-__device__ __forceinline__ size_t blob_words(int n, int b, int SB) {
-    return (static_cast<size_t>(n / 64) * SB + b) * kBlockSB + (n % 64) * 48;
-}
-__device__ __forceinline__ size_t blob_group(int n, int j, int SB) {
-    const int r = n % 64;
-    return (static_cast<size_t>(n / 64) * SB + (j >> 1)) * kBlockSB + kQTileSBWords * 4 + (j & 1) * kGroupBytes +
-           (((r >> 4) * 8 + (r & 7)) * 4 + ((r >> 3) & 1) * 2) * 2;
-}
 
 // One thread per (row, 128-code super-block): two scale groups.  Rows N..
 // of the last tile get zero words, scales and zeros.
@@ -38,15 +25,8 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
     if (gid >= static_cast<long long>(Npad) * SB) return;
     const int n = static_cast<int>(gid / SB);
     const int b = static_cast<int>(gid % SB);
-    uint16_t* sz = reinterpret_cast<uint16_t*>(blob);
     if (n >= N) {
-        uint4* dst = reinterpret_cast<uint4*>(blob + blob_words(n, b, SB));
-        dst[0] = dst[1] = dst[2] = make_uint4(0u, 0u, 0u, 0u);
-        for (int g = 0; g < 2; ++g) {
-            const size_t o = blob_group(n, 2 * b + g, SB) / 2;
-            sz[o] = 0;
-            sz[o + 1] = 0;
-        }
+        blob_zero_row(blob, n, b, SB);
         return;
     }
     const uint16_t* w = W + static_cast<size_t>(n) * K + static_cast<size_t>(b) * 128;
@@ -69,9 +49,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
         const __half zh = __float2half_rn(__fdiv_rn(-mn, s));
         const float z = __half2float(zh);
         if (!isfinite(s) || !isfinite(z)) st |= MILO_DEV_FP16_RANGE;
-        const size_t o = blob_group(n, 2 * b + g, SB) / 2;
-        sz[o] = __half_as_ushort(sh);
-        sz[o + 1] = __half_as_ushort(zh);
+        blob_store_sz(blob, n, 2 * b + g, SB, __half_as_ushort(sh), __half_as_ushort(zh));
         for (int i = 0; i < 64; ++i) {
             const float v = __fadd_rn(__fdiv_rn(__half2float(__ushort_as_half(w[64 * g + i])), s), z);
             float r = rintf(v);
@@ -81,27 +59,9 @@ __global__ void __launch_bounds__(128) pack_kernel(const uint16_t* __restrict__ 
         }
     }
 
-    // Place the 128 codes: unit c, unit code m -> word 3c + t, see milo.h.
     uint32_t words[12];
-#pragma unroll
-    for (int i = 0; i < 12; ++i) words[i] = 0u;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int m = 0; m < 30; ++m) {
-            const int t = m / 10, r = m % 10;
-            const int pos = 16 * (r & 1) + 3 * (r >> 1);
-            words[3 * c + t] |= static_cast<uint32_t>(q[unit_k(c, m)]) << pos;
-        }
-        const uint32_t u30 = q[unit_k(c, 30)], u31 = q[unit_k(c, 31)];
-#pragma unroll
-        for (int t = 0; t < 3; ++t)
-            words[3 * c + t] |= (((u30 >> t) & 1u) << 15) | (((u31 >> t) & 1u) << 31);
-    }
-    uint4* dst = reinterpret_cast<uint4*>(blob + blob_words(n, b, SB));
-    dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-    dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
-    dst[2] = make_uint4(words[8], words[9], words[10], words[11]);
+    place_codes(q, words);
+    blob_store_words(blob, n, b, SB, words);
     flag(dev_status, st);
 }
 

@@ -1,0 +1,764 @@
+// quant.cu -- the offline MiLo quantiser on the GPU: HQQ quantise-and-pack,
+// the rank-r compensator of the residual by randomized subspace iteration,
+// and the refinement rounds (sm_100a).
+//
+// "MiLo: Efficient Quantized MoE Inference with Mixture of Low-Rank
+// Compensators", section "MiLo Algorithm: Mixture of Low-Rank Compensators":
+// the weights are first quantised with HQQ; the SVD of the residual
+// W - W_quant gives the top-r compensator U V; quantisation and compensation
+// are then refined in turn.
+//
+// Design: this runs once per weight, offline, so the kernels favour a fixed
+// arithmetic order (deterministic results, codes that are a fixed function of
+// the inputs) over speed:
+//   - hqq_pack_kernel: one thread per (row, 128-code super-block), like the
+//     round-to-nearest packer; the target W - U V, the HQQ iterations and the
+//     residual use explicitly rounded fp32 operations (no contraction).
+//   - sgemm_kernel: fp32 C = A B with arbitrary strides (64 x 64 tiles, 4 x 4
+//     per thread, the reduction never split): the sketch products R omega,
+//     R^T Y, Y^T R and the small basis changes.
+//   - gram_kernel + gram_sum_kernel: X^T X in fp64, partial sums per row chunk
+//     added in a fixed order.
+//   - chol_kernel (one block): Cholesky factor of a Gram matrix and the inverse
+//     of the factor in fp64: the basis change of Cholesky QR.
+//   - jacobi_kernel (one block): cyclic Jacobi eigenpairs of B B^T in fp64,
+//     l/2 disjoint rotations per step (round-robin ordering).
+//   - err_kernel + err_sum_kernel: ||R - U V||_F in fp64 and the best-round
+//     bookkeeping; copy_best_kernel keeps the best round's blob, U and V.
+#include <cuda_runtime.h>
+
+#include "milo_blob.cuh"
+#include "milo_device.cuh"
+#include "milo_host.h"
+
+namespace milo {
+
+namespace {
+
+__device__ __forceinline__ float f16v(uint16_t b) { return __half2float(__ushort_as_half(b)); }
+
+// ---------------------------------------------------------------------------
+// HQQ quantise and pack
+// ---------------------------------------------------------------------------
+
+struct HqqArgs {
+    const uint16_t* W;      // [N, K] fp16
+    const uint16_t* U;      // [N, r] fp16 or null
+    const uint16_t* V;      // [r, K] fp16 or null
+    uint8_t* blob;
+    float* resid;           // [N, K] or null
+    int32_t* dev_status;
+    int N, K, r, iters;
+    float beta, kappa;
+};
+
+// One group of 64 targets t: HQQ's zero-point fit with p = 1/2 shrinkage,
+// keeping the zero point of lowest L1 error; returns the fp16 scale and zero.
+__device__ __forceinline__ int32_t hqq_group(const float (&t)[64], int iters, float beta0, float kappa,
+                                             __half& sh, __half& zh) {
+    int32_t st = 0;
+    float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        if (!isfinite(t[i])) st |= MILO_DEV_NONFINITE;
+        mn = t[i] < mn ? t[i] : mn;
+        mx = t[i] > mx ? t[i] : mx;
+    }
+    sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 7.0f));
+    if ((__half_as_ushort(sh) & 0x7FFF) == 0) sh = __ushort_as_half(0x3C00);   // s := 1
+    const float s = __half2float(sh);
+    float z = __fdiv_rn(-mn, s);
+    float beta = beta0, best_err = INFINITY, best_z = z;
+    for (int it = 0; it < iters; ++it) {
+        float err = 0.0f, acc = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            float r = rintf(__fadd_rn(__fdiv_rn(t[i], s), z));
+            if (!(r >= 0.0f)) r = 0.0f;
+            if (r > 7.0f) r = 7.0f;
+            const float e = __fsub_rn(t[i], __fmul_rn(__fsub_rn(r, z), s));
+            const float a = fabsf(e);
+            err = __fadd_rn(err, a);
+            float w_e = 0.0f;
+            if (a > 0.0f) {
+                const float m = __fsub_rn(a, __fdiv_rn(1.0f, __fmul_rn(__fsqrt_rn(a), beta)));
+                if (m > 0.0f) w_e = e < 0.0f ? -m : m;
+            }
+            acc = __fadd_rn(acc, __fsub_rn(r, __fdiv_rn(__fsub_rn(t[i], w_e), s)));
+        }
+        if (err < best_err) {
+            best_err = err;
+            best_z = z;
+        }
+        z = __fmul_rn(acc, 0.015625f);
+        beta = __fmul_rn(beta, kappa);
+    }
+    zh = __float2half_rn(best_z);
+    if (!isfinite(s) || !isfinite(__half2float(zh))) st |= MILO_DEV_FP16_RANGE;
+    return st;
+}
+
+__global__ void __launch_bounds__(128) hqq_pack_kernel(const HqqArgs a) {
+    const int SB = a.K / 128;
+    const int Npad = (a.N + 63) / 64 * 64;
+    const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (gid >= static_cast<long long>(Npad) * SB) return;
+    const int n = static_cast<int>(gid / SB);
+    const int b = static_cast<int>(gid % SB);
+    if (n >= a.N) {
+        blob_zero_row(a.blob, n, b, SB);
+        return;
+    }
+    int32_t st = 0;
+    uint8_t q[128];
+#pragma unroll 1
+    for (int g = 0; g < 2; ++g) {
+        const size_t k0 = static_cast<size_t>(n) * a.K + 128 * b + 64 * g;
+        float t[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) t[i] = f16v(a.W[k0 + i]);
+        // t = W - U V, one rank term at a time
+#pragma unroll 1
+        for (int p = 0; p < a.r; ++p) {
+            const float u = f16v(a.U[static_cast<size_t>(n) * a.r + p]);
+            const uint16_t* vr = a.V + static_cast<size_t>(p) * a.K + 128 * b + 64 * g;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) t[i] = __fsub_rn(t[i], __fmul_rn(u, f16v(vr[i])));
+        }
+        __half sh, zh;
+        st |= hqq_group(t, a.iters, a.beta, a.kappa, sh, zh);
+        blob_store_sz(a.blob, n, 2 * b + g, SB, __half_as_ushort(sh), __half_as_ushort(zh));
+        const float s = __half2float(sh), z = __half2float(zh);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            float r = rintf(__fadd_rn(__fdiv_rn(t[i], s), z));
+            if (!(r >= 0.0f)) r = 0.0f;
+            if (r > 7.0f) r = 7.0f;
+            q[64 * g + i] = static_cast<uint8_t>(r);
+            if (a.resid) a.resid[k0 + i] = __fsub_rn(f16v(a.W[k0 + i]), __fmul_rn(__fsub_rn(r, z), s));
+        }
+    }
+    uint32_t words[12];
+    place_codes(q, words);
+    blob_store_words(a.blob, n, b, SB, words);
+    flag(a.dev_status, st);
+}
+
+// ---------------------------------------------------------------------------
+// fp32 GEMM with arbitrary strides
+// ---------------------------------------------------------------------------
+
+struct GemmArgs {
+    int M, Nn, Kd;
+    const float* A;          // A(m, k) = A[m * sam + k * sak]
+    long long sam, sak;
+    const float* B;          // B(k, n) = B[k * sbk + n * sbn]
+    long long sbk, sbn;
+    float* C;                // C(m, n) = C[m * ldc + n] (fp32), or
+    uint16_t* C16;           // the same in fp16 (round to nearest)
+    long long ldc;
+    int32_t* dev_status;
+};
+
+constexpr int kGT = 64;      // output tile
+constexpr int kGK = 16;      // reduction slice per shared-memory stage
+
+// C = A B over the full reduction in index order per 16-wide slice.  Tile
+// loads walk the operand's contiguous dimension across threads.
+__global__ void __launch_bounds__(256) sgemm_kernel(const GemmArgs a) {
+    __shared__ __align__(16) float As[kGK][kGT + 4];
+    __shared__ __align__(16) float Bs[kGK][kGT + 4];
+    const int tid = threadIdx.x;
+    const int m0 = blockIdx.y * kGT, n0 = blockIdx.x * kGT;
+    const int tm = (tid / 16) * 4, tn = (tid % 16) * 4;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+    for (int k0 = 0; k0 < a.Kd; k0 += kGK) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int idx = tid + 256 * i;
+            int mm, kk;
+            if (a.sak == 1) { kk = idx % kGK; mm = idx / kGK; }
+            else { mm = idx % kGT; kk = idx / kGT; }
+            const int m = m0 + mm, k = k0 + kk;
+            As[kk][mm] = (m < a.M && k < a.Kd) ? a.A[m * a.sam + k * a.sak] : 0.0f;
+            int nn;
+            if (a.sbn == 1) { nn = idx % kGT; kk = idx / kGT; }
+            else { kk = idx % kGK; nn = idx / kGK; }
+            const int n = n0 + nn, kb = k0 + kk;
+            Bs[kk][nn] = (n < a.Nn && kb < a.Kd) ? a.B[kb * a.sbk + n * a.sbn] : 0.0f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < kGK; ++kk) {
+            const float4 av = *reinterpret_cast<const float4*>(&As[kk][tm]);
+            const float4 bv = *reinterpret_cast<const float4*>(&Bs[kk][tn]);
+            const float ar[4] = {av.x, av.y, av.z, av.w}, br[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(ar[i], br[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+    int32_t st = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int m = m0 + tm + i, n = n0 + tn + j;
+            if (m >= a.M || n >= a.Nn) continue;
+            if (a.C16) {
+                const __half h = __float2half_rn(acc[i][j]);
+                if (!isfinite(__half2float(h))) st |= MILO_DEV_FP16_RANGE;
+                a.C16[m * a.ldc + n] = __half_as_ushort(h);
+            } else {
+                a.C[m * a.ldc + n] = acc[i][j];
+            }
+        }
+    flag(a.dev_status, st);
+}
+
+// ---------------------------------------------------------------------------
+// Gram matrices in fp64
+// ---------------------------------------------------------------------------
+
+struct GramArgs {
+    const float* X;          // X(i, c) = X[i * sxi + c * sxc], i < M, c < l
+    long long sxi, sxc;
+    double* part;            // [chunks][l][l]
+    int M, l, rows_per_chunk;
+};
+
+constexpr int kGramRows = 32;   // rows staged in shared memory at a time
+constexpr int kMaxSketch = 128;
+
+// Block c adds X(i, a) X(i, b) over its rows in index order; thread
+// (tid / 16, tid % 16) owns an (l/16 x l/16) tile of (a, b).
+__global__ void __launch_bounds__(256) gram_kernel(const GramArgs g) {
+    __shared__ float xs[kGramRows][kMaxSketch + 1];
+    const int tid = threadIdx.x;
+    const int ts = g.l / 16;
+    const int ta = (tid / 16) * ts, tb = (tid % 16) * ts;
+    double acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+    const int r0 = blockIdx.x * g.rows_per_chunk;
+    const int r1 = min(g.M, r0 + g.rows_per_chunk);
+    for (int base = r0; base < r1; base += kGramRows) {
+        const int nr = min(kGramRows, r1 - base);
+        for (int idx = tid; idx < kGramRows * g.l; idx += 256) {
+            int i, c;
+            if (g.sxc == 1) { c = idx % g.l; i = idx / g.l; }
+            else { i = idx % kGramRows; c = idx / kGramRows; }
+            xs[i][c] = i < nr ? g.X[(base + i) * g.sxi + c * g.sxc] : 0.0f;
+        }
+        __syncthreads();
+        for (int i = 0; i < nr; ++i) {
+#pragma unroll
+            for (int aa = 0; aa < 8; ++aa) {
+                if (aa >= ts) break;
+                const double xa = xs[i][ta + aa];
+#pragma unroll
+                for (int bb = 0; bb < 8; ++bb) {
+                    if (bb >= ts) break;
+                    acc[aa][bb] = fma(xa, static_cast<double>(xs[i][tb + bb]), acc[aa][bb]);
+                }
+            }
+        }
+        __syncthreads();
+    }
+    double* out = g.part + static_cast<size_t>(blockIdx.x) * g.l * g.l;
+#pragma unroll
+    for (int aa = 0; aa < 8; ++aa)
+#pragma unroll
+        for (int bb = 0; bb < 8; ++bb)
+            if (aa < ts && bb < ts) out[(ta + aa) * g.l + tb + bb] = acc[aa][bb];
+}
+
+// G[e] = sum over chunks of part[chunk][e], in chunk order.
+__global__ void gram_sum_kernel(const double* part, int chunks, int ll, double* G) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= ll) return;
+    double s = 0.0;
+    for (int c = 0; c < chunks; ++c) s += part[static_cast<size_t>(c) * ll + e];
+    G[e] = s;
+}
+
+// ---------------------------------------------------------------------------
+// Cholesky QR basis change (one block)
+// ---------------------------------------------------------------------------
+
+// G [l, l] fp64 (symmetric positive semi-definite) -> M fp32 [l, l] with
+// Y M = Y L^-T, L the Cholesky factor of G.  A pivot below 1e-10 of its
+// diagonal entry marks a column that lies in the span of the earlier ones:
+// its column of M is zero (the basis drops that direction).  X is fp64 [l, l]
+// scratch for the inverse.
+__global__ void __launch_bounds__(256) chol_kernel(const double* G, int l, float* M, double* X) {
+    extern __shared__ double Ls[];               // [l][l + 1]
+    __shared__ int dead[kMaxSketch];
+    const int ld = l + 1, tid = threadIdx.x;
+    for (int idx = tid; idx < l * l; idx += blockDim.x) Ls[(idx / l) * ld + idx % l] = G[idx];
+    __syncthreads();
+    for (int j = 0; j < l; ++j) {
+        if (tid == 0) {
+            double d = Ls[j * ld + j];
+            for (int k = 0; k < j; ++k) d -= Ls[j * ld + k] * Ls[j * ld + k];
+            const bool gone = !(d > 1e-10 * G[j * l + j]);
+            dead[j] = gone;
+            Ls[j * ld + j] = gone ? 1.0 : sqrt(d);
+        }
+        __syncthreads();
+        const double piv = Ls[j * ld + j];
+        for (int i = j + 1 + tid; i < l; i += blockDim.x) {
+            double v = 0.0;
+            if (!dead[j]) {
+                v = Ls[i * ld + j];
+                for (int k = 0; k < j; ++k) v -= Ls[i * ld + k] * Ls[j * ld + k];
+                v /= piv;
+            }
+            Ls[i * ld + j] = v;
+        }
+        __syncthreads();
+    }
+    // X = L^-1 by forward substitution, one column per thread
+    for (int c = tid; c < l; c += blockDim.x) {
+        for (int i = 0; i < l; ++i) {
+            double v = 0.0;
+            if (i >= c) {
+                v = i == c ? 1.0 : 0.0;
+                for (int k = c; k < i; ++k) v -= Ls[i * ld + k] * X[k * l + c];
+                v /= Ls[i * ld + i];
+            }
+            X[i * l + c] = v;
+        }
+    }
+    __syncthreads();
+    // M[k][i] = X[i][k]; the row of X of a dropped column is zero
+    for (int idx = tid; idx < l * l; idx += blockDim.x) {
+        const int k = idx / l, i = idx % l;
+        M[idx] = dead[i] ? 0.0f : static_cast<float>(X[i * l + k]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Symmetric eigenpairs by cyclic Jacobi (one block)
+// ---------------------------------------------------------------------------
+
+// C [l, l] fp64 symmetric (l even) -> the top r eigenpairs in descending
+// order of eigenvalue, emitted as MU fp32 [l, r] = P_r sigma^(1/2) and MV fp32
+// [r, l] = sigma^(-1/2) P_r^T with sigma = sqrt(max(lambda, 0)); directions
+// with sigma <= 1e-12 sigma_0 get zeros.  P is fp64 [l, l] scratch (the
+// eigenvectors).  Each sweep pairs every index with every other once
+// (round-robin: index l-1 fixed, the rest rotating), l/2 disjoint rotations
+// per step; at most kJacobiSweeps sweeps, fewer once the off-diagonal mass
+// falls below 1e-30 of the total.
+constexpr int kJacobiSweeps = 40;
+
+__global__ void __launch_bounds__(256) jacobi_kernel(const double* C, int l, int r, double* P, float* MU, float* MV) {
+    extern __shared__ double As[];               // [l][l + 1]
+    __shared__ double cs[kMaxSketch / 2], sn[kMaxSketch / 2];
+    __shared__ int pp[kMaxSketch / 2], qq[kMaxSketch / 2], order[kMaxSketch];
+    __shared__ double red[256];
+    __shared__ int stop;
+    const int ld = l + 1, tid = threadIdx.x, half = l / 2, m = l - 1;
+    for (int idx = tid; idx < l * l; idx += blockDim.x) {
+        As[(idx / l) * ld + idx % l] = C[idx];
+        P[idx] = (idx / l == idx % l) ? 1.0 : 0.0;
+    }
+    __syncthreads();
+    for (int sweep = 0; sweep < kJacobiSweeps; ++sweep) {
+        double off = 0.0, tot = 0.0;
+        for (int idx = tid; idx < l * l; idx += blockDim.x) {
+            const double v = As[(idx / l) * ld + idx % l];
+            tot += v * v;
+            if (idx / l != idx % l) off += v * v;
+        }
+        red[tid] = off;
+        __syncthreads();
+        for (int s = 128; s > 0; s >>= 1) {
+            if (tid < s) red[tid] += red[tid + s];
+            __syncthreads();
+        }
+        const double off_all = red[0];
+        __syncthreads();
+        red[tid] = tot;
+        __syncthreads();
+        for (int s = 128; s > 0; s >>= 1) {
+            if (tid < s) red[tid] += red[tid + s];
+            __syncthreads();
+        }
+        if (tid == 0) stop = !(off_all > 1e-30 * red[0]);
+        __syncthreads();
+        if (stop) break;
+        for (int step = 0; step < m; ++step) {
+            if (tid < half) {
+                int p, q;
+                if (tid == 0) { p = step % m; q = m; }
+                else { p = (step + tid) % m; q = (step - tid + m) % m; }
+                const double app = As[p * ld + p], aqq = As[q * ld + q], apq = As[p * ld + q];
+                double c = 1.0, s = 0.0;
+                if (apq != 0.0) {
+                    const double tau = (aqq - app) / (2.0 * apq);
+                    const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
+                    c = 1.0 / sqrt(1.0 + t * t);
+                    s = t * c;
+                }
+                cs[tid] = c; sn[tid] = s; pp[tid] = p; qq[tid] = q;
+            }
+            __syncthreads();
+            // rows: A <- J^T A
+            for (int idx = tid; idx < half * l; idx += blockDim.x) {
+                const int k = idx / l, j = idx % l, p = pp[k], q = qq[k];
+                const double ap = As[p * ld + j], aq = As[q * ld + j];
+                As[p * ld + j] = cs[k] * ap - sn[k] * aq;
+                As[q * ld + j] = sn[k] * ap + cs[k] * aq;
+            }
+            __syncthreads();
+            // columns: A <- A J, P <- P J
+            for (int idx = tid; idx < half * l; idx += blockDim.x) {
+                const int k = idx / l, i = idx % l, p = pp[k], q = qq[k];
+                const double ap = As[i * ld + p], aq = As[i * ld + q];
+                As[i * ld + p] = cs[k] * ap - sn[k] * aq;
+                As[i * ld + q] = sn[k] * ap + cs[k] * aq;
+                const double vp = P[i * l + p], vq = P[i * l + q];
+                P[i * l + p] = cs[k] * vp - sn[k] * vq;
+                P[i * l + q] = sn[k] * vp + cs[k] * vq;
+            }
+            __syncthreads();
+        }
+    }
+    // descending eigenvalue order, the lower index first on ties (NaN last):
+    // every index gets a distinct rank, so order[] is a permutation
+    for (int i = tid; i < l; i += blockDim.x) {
+        const double li = As[i * ld + i] == As[i * ld + i] ? As[i * ld + i] : -INFINITY;
+        int rank = 0;
+        for (int j = 0; j < l; ++j) {
+            const double lj = As[j * ld + j] == As[j * ld + j] ? As[j * ld + j] : -INFINITY;
+            rank += (lj > li || (lj == li && j < i)) ? 1 : 0;
+        }
+        order[rank] = i;
+    }
+    __syncthreads();
+    const double sig0 = sqrt(fmax(As[order[0] * ld + order[0]], 0.0));
+    for (int idx = tid; idx < l * r; idx += blockDim.x) {
+        const int a = idx / r, i = idx % r;
+        const double sig = sqrt(fmax(As[order[i] * ld + order[i]], 0.0));
+        const bool live = sig0 > 0.0 && sig > 1e-12 * sig0;
+        const double root = live ? sqrt(sig) : 0.0;
+        const double v = P[a * l + order[i]];
+        MU[a * r + i] = static_cast<float>(v * root);
+        MV[i * l + a] = live ? static_cast<float>(v / root) : 0.0f;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Error norm, best round, copies
+// ---------------------------------------------------------------------------
+
+// Block partial of sum (R - U V)^2 over (row, 128-column segment) threads, in
+// fp64 (U V summed over the rank in fp64); warp and block sums in a fixed tree.
+__global__ void __launch_bounds__(256) err_kernel(const float* R, const uint16_t* U, const uint16_t* V, int N, int K,
+                                                  int r, double* part) {
+    __shared__ double ws[8];
+    const int SB = K / 128;
+    const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    double acc = 0.0;
+    if (gid < static_cast<long long>(N) * SB) {
+        const int n = static_cast<int>(gid / SB), b = static_cast<int>(gid % SB);
+        for (int k = 128 * b; k < 128 * b + 128; ++k) {
+            double uv = 0.0;
+            for (int p = 0; p < r; ++p)
+                uv = fma(static_cast<double>(f16v(U[static_cast<size_t>(n) * r + p])),
+                         static_cast<double>(f16v(V[static_cast<size_t>(p) * K + k])), uv);
+            const double d = static_cast<double>(R[static_cast<size_t>(n) * K + k]) - uv;
+            acc = fma(d, d, acc);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+    if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double s = 0.0;
+        for (int w = 0; w < 8; ++w) s += ws[w];
+        part[blockIdx.x] = s;
+    }
+}
+
+// err[round] = sqrt(sum of parts); best[0] keeps the lowest error so far
+// (fp64), flag[0] = 1 when this round is the new best (the first round always).
+__global__ void __launch_bounds__(256) err_sum_kernel(const double* part, int nparts, int round, float* err,
+                                                      double* best, int* improved) {
+    __shared__ double red[256];
+    double s = 0.0;
+    for (int i = threadIdx.x; i < nparts; i += 256) s += part[i];
+    red[threadIdx.x] = s;
+    __syncthreads();
+    for (int o = 128; o > 0; o >>= 1) {
+        if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const double e = sqrt(red[0]);
+        if (err) err[round] = static_cast<float>(e);
+        const bool better = round == 0 || e < best[0];
+        if (better) best[0] = e;
+        improved[0] = better ? 1 : 0;
+    }
+}
+
+// dst = src (16-byte units) when improved[0] is set.
+__global__ void copy_best_kernel(const int* improved, const uint4* src0, uint4* dst0, size_t n0, const uint4* src1,
+                                 uint4* dst1, size_t n1, const uint4* src2, uint4* dst2, size_t n2) {
+    if (!improved[0]) return;
+    const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+    const size_t i0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    for (size_t i = i0; i < n0; i += stride) dst0[i] = src0[i];
+    for (size_t i = i0; i < n1; i += stride) dst1[i] = src1[i];
+    for (size_t i = i0; i < n2; i += stride) dst2[i] = src2[i];
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr int kGramChunk = 256;   // rows per Gram partial
+
+struct QuantWs {
+    size_t R, Y, Y2, Z, Z2, B, part, G, X, M, P, MU, MV, U, V, blob, epart, best, flag, total;
+    int l, chunks, eblocks;
+};
+
+QuantWs quant_layout(int N, int K, const milo_lorc_params& p) {
+    QuantWs w{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = round_up(off + bytes, 256);
+        return o;
+    };
+    const int r = p.rank;
+    const int l = r > 0 ? p.sketch : 0;
+    w.l = l;
+    w.R = take(static_cast<size_t>(N) * K * 4);
+    if (r > 0) {
+        w.Y = take(static_cast<size_t>(N) * l * 4);
+        w.Y2 = take(static_cast<size_t>(N) * l * 4);
+        w.Z = take(static_cast<size_t>(K) * l * 4);
+        w.Z2 = take(static_cast<size_t>(K) * l * 4);
+        w.B = take(static_cast<size_t>(l) * K * 4);
+        w.chunks = (std::max(N, K) + kGramChunk - 1) / kGramChunk;
+        w.part = take(static_cast<size_t>(w.chunks) * l * l * 8);
+        w.G = take(static_cast<size_t>(l) * l * 8);
+        w.X = take(static_cast<size_t>(l) * l * 8);
+        w.M = take(static_cast<size_t>(l) * l * 4);
+        w.P = take(static_cast<size_t>(l) * l * 8);
+        w.MU = take(static_cast<size_t>(l) * r * 4);
+        w.MV = take(static_cast<size_t>(r) * l * 4);
+        w.U = take(static_cast<size_t>(N) * r * 2);
+        w.V = take(static_cast<size_t>(r) * K * 2);
+    }
+    w.blob = take(static_cast<size_t>((N + 63) / 64) * (K / 128) * kBlockSB);
+    w.eblocks = static_cast<int>((static_cast<long long>(N) * (K / 128) + 255) / 256);
+    w.epart = take(static_cast<size_t>(w.eblocks) * 8);
+    w.best = take(8);
+    w.flag = take(4);
+    w.total = off;
+    return w;
+}
+
+milo_status check_hqq(int N, int K, int rank, int iters, float beta, float kappa, const char* who) {
+    const std::string f = who;
+    if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, f + ": N and K must be positive");
+    if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": K must be a multiple of 128");
+    if (N > (1 << 22)) return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": N above 4194304");
+    if (rank < 0) return fail(MILO_ERR_INVALID_ARG, f + ": negative rank");
+    if (rank > MILO_MAX_RANK) return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": rank above 64");
+    if (iters < 0 || iters > 1000) return fail(MILO_ERR_INVALID_ARG, f + ": hqq_iters outside 0..1000");
+    if (!(beta > 0.0f) || !isfinite(beta) || !(kappa > 0.0f) || !isfinite(kappa))
+        return fail(MILO_ERR_INVALID_ARG, f + ": hqq_beta and hqq_kappa must be finite and positive");
+    return MILO_OK;
+}
+
+milo_status launch_hqq(const HqqArgs& a, cudaStream_t st) {
+    const long long threads = static_cast<long long>((a.N + 63) / 64 * 64) * (a.K / 128);
+    hqq_pack_kernel<<<static_cast<unsigned>((threads + 127) / 128), 128, 0, st>>>(a);
+    return check_launch("hqq_pack_kernel");
+}
+
+milo_status gemm(cudaStream_t st, int M, int Nn, int Kd, const float* A, long long sam, long long sak, const float* B,
+                 long long sbk, long long sbn, float* C, uint16_t* C16, long long ldc, int32_t* dev_status) {
+    const GemmArgs a{M, Nn, Kd, A, sam, sak, B, sbk, sbn, C, C16, ldc, dev_status};
+    const dim3 grid((Nn + kGT - 1) / kGT, (M + kGT - 1) / kGT);
+    sgemm_kernel<<<grid, 256, 0, st>>>(a);
+    return check_launch("sgemm_kernel");
+}
+
+// G = X^T X for X(i, c) = X[i * sxi + c * sxc], i < M, c < l.
+milo_status gram(cudaStream_t st, const float* X, long long sxi, long long sxc, int M, int l, double* part,
+                 double* G) {
+    const int chunks = (M + kGramChunk - 1) / kGramChunk;
+    const GramArgs g{X, sxi, sxc, part, M, l, kGramChunk};
+    gram_kernel<<<chunks, 256, 0, st>>>(g);
+    gram_sum_kernel<<<(l * l + 255) / 256, 256, 0, st>>>(part, chunks, l * l, G);
+    return check_launch("gram_kernel");
+}
+
+size_t square_smem(int l) { return static_cast<size_t>(l) * (l + 1) * 8; }
+
+// Y [M, l] <- an orthonormal basis of its columns (Cholesky QR, twice).
+milo_status orth(cudaStream_t st, float* Y, float* Y2, int M, int l, uint8_t* base, const QuantWs& w,
+                 int32_t* dev_status) {
+    milo_status s;
+    double* G = reinterpret_cast<double*>(base + w.G);
+    float* Mm = reinterpret_cast<float*>(base + w.M);
+    for (int pass = 0; pass < 2; ++pass) {
+        if ((s = gram(st, Y, l, 1, M, l, reinterpret_cast<double*>(base + w.part), G)) != MILO_OK) return s;
+        chol_kernel<<<1, 256, square_smem(l), st>>>(G, l, Mm, reinterpret_cast<double*>(base + w.X));
+        if ((s = check_launch("chol_kernel")) != MILO_OK) return s;
+        if ((s = gemm(st, M, l, l, Y, l, 1, Mm, l, 1, Y2, nullptr, l, dev_status)) != MILO_OK) return s;
+        std::swap(Y, Y2);
+    }
+    return MILO_OK;   // two swaps: the basis is back in the first buffer
+}
+
+// U fp16 [N, r], V fp16 [r, K] from R [N, K] (randomized subspace iteration).
+milo_status compensator(cudaStream_t st, const float* R, const float* omega, int N, int K, int r, int q,
+                        uint8_t* base, const QuantWs& w, uint16_t* U, uint16_t* V, int32_t* dev_status) {
+    milo_status s;
+    const int l = w.l;
+    float* Y = reinterpret_cast<float*>(base + w.Y);
+    float* Y2 = reinterpret_cast<float*>(base + w.Y2);
+    float* Z = reinterpret_cast<float*>(base + w.Z);
+    float* Z2 = reinterpret_cast<float*>(base + w.Z2);
+    float* Bm = reinterpret_cast<float*>(base + w.B);
+    double* G = reinterpret_cast<double*>(base + w.G);
+    if ((s = gemm(st, N, l, K, R, K, 1, omega, l, 1, Y, nullptr, l, dev_status)) != MILO_OK) return s;
+    if ((s = orth(st, Y, Y2, N, l, base, w, dev_status)) != MILO_OK) return s;
+    for (int it = 0; it < q; ++it) {
+        if ((s = gemm(st, K, l, N, R, 1, K, Y, l, 1, Z, nullptr, l, dev_status)) != MILO_OK) return s;
+        if ((s = orth(st, Z, Z2, K, l, base, w, dev_status)) != MILO_OK) return s;
+        if ((s = gemm(st, N, l, K, R, K, 1, Z, l, 1, Y, nullptr, l, dev_status)) != MILO_OK) return s;
+        if ((s = orth(st, Y, Y2, N, l, base, w, dev_status)) != MILO_OK) return s;
+    }
+    if ((s = gemm(st, l, K, N, Y, 1, l, R, K, 1, Bm, nullptr, K, dev_status)) != MILO_OK) return s;
+    if ((s = gram(st, Bm, 1, K, K, l, reinterpret_cast<double*>(base + w.part), G)) != MILO_OK) return s;
+    float* MU = reinterpret_cast<float*>(base + w.MU);
+    float* MV = reinterpret_cast<float*>(base + w.MV);
+    jacobi_kernel<<<1, 256, square_smem(l), st>>>(G, l, r, reinterpret_cast<double*>(base + w.P), MU, MV);
+    if ((s = check_launch("jacobi_kernel")) != MILO_OK) return s;
+    if ((s = gemm(st, N, r, l, Y, l, 1, MU, r, 1, nullptr, U, r, dev_status)) != MILO_OK) return s;
+    return gemm(st, r, K, l, MV, l, 1, Bm, K, 1, nullptr, V, K, dev_status);
+}
+
+}  // namespace
+
+}  // namespace milo
+
+using namespace milo;
+
+extern "C" milo_status milo_hqq_pack(const uint16_t* W, const uint16_t* U, const uint16_t* V, int32_t rank,
+                                     int32_t N, int32_t K, int32_t hqq_iters, float hqq_beta, float hqq_kappa,
+                                     void* packed, float* residual, int32_t* dev_status, void* stream) {
+    clear_error();
+    milo_status s = check_hqq(N, K, rank, hqq_iters, hqq_beta, hqq_kappa, "milo_hqq_pack");
+    if (s != MILO_OK) return s;
+    if (!W || !packed) return fail(MILO_ERR_INVALID_ARG, "milo_hqq_pack: NULL W or packed");
+    if (rank > 0 && (!U || !V)) return fail(MILO_ERR_INVALID_ARG, "milo_hqq_pack: NULL U or V with rank > 0");
+    if (!aligned(packed, 16) || !aligned(W, 2) || (residual && !aligned(residual, 4)))
+        return fail(MILO_ERR_INVALID_ARG, "milo_hqq_pack: misaligned buffer (packed needs 16 bytes)");
+    const HqqArgs a{W, rank > 0 ? U : nullptr, rank > 0 ? V : nullptr, static_cast<uint8_t*>(packed), residual,
+                    dev_status, N, K, rank, hqq_iters, hqq_beta, hqq_kappa};
+    return launch_hqq(a, static_cast<cudaStream_t>(stream));
+}
+
+static milo_status check_lorc(int32_t N, int32_t K, const milo_lorc_params* p, const char* who) {
+    const std::string f = who;
+    if (!p) return fail(MILO_ERR_INVALID_ARG, f + ": NULL params");
+    milo_status s = check_hqq(N, K, p->rank, p->hqq_iters, p->hqq_beta, p->hqq_kappa, who);
+    if (s != MILO_OK) return s;
+    if (p->rank % 8) return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": rank must be a multiple of 8");
+    if (p->rounds < 0 || p->rounds > 16) return fail(MILO_ERR_INVALID_ARG, f + ": rounds outside 0..16");
+    if (p->rank > 0) {
+        if (p->sketch < p->rank || p->sketch > kMaxSketch || p->sketch % 16)
+            return fail(MILO_ERR_INVALID_ARG, f + ": sketch must be a multiple of 16 in rank..128");
+        if (p->power_iters < 0 || p->power_iters > 8)
+            return fail(MILO_ERR_INVALID_ARG, f + ": power_iters outside 0..8");
+    }
+    return MILO_OK;
+}
+
+extern "C" milo_status milo_quantize_lorc_workspace(int32_t N, int32_t K, const milo_lorc_params* params,
+                                                    size_t* bytes) {
+    clear_error();
+    milo_status s = check_lorc(N, K, params, "milo_quantize_lorc_workspace");
+    if (s != MILO_OK) return s;
+    if (!bytes) return fail(MILO_ERR_INVALID_ARG, "milo_quantize_lorc_workspace: NULL bytes");
+    *bytes = quant_layout(N, K, *params).total;
+    return MILO_OK;
+}
+
+extern "C" milo_status milo_quantize_lorc(const uint16_t* W, int32_t N, int32_t K, const milo_lorc_params* params,
+                                          const float* omega, void* packed, uint16_t* U, uint16_t* V, float* err,
+                                          void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+    clear_error();
+    milo_status s = check_lorc(N, K, params, "milo_quantize_lorc");
+    if (s != MILO_OK) return s;
+    const milo_lorc_params p = *params;
+    const int r = p.rank;
+    if (!W || !packed || !ws) return fail(MILO_ERR_INVALID_ARG, "milo_quantize_lorc: NULL W, packed or ws");
+    if (r > 0 && (!omega || !U || !V))
+        return fail(MILO_ERR_INVALID_ARG, "milo_quantize_lorc: NULL omega, U or V with rank > 0");
+    if (!aligned(packed, 16) || !aligned(ws, 256) || !aligned(W, 2) || (r > 0 && (!aligned(U, 16) ||
+        !aligned(V, 16) || !aligned(omega, 4))) || (err && !aligned(err, 4)))
+        return fail(MILO_ERR_INVALID_ARG, "milo_quantize_lorc: misaligned buffer (packed, U, V need 16 bytes, ws 256)");
+    const QuantWs w = quant_layout(N, K, p);
+    if (ws_bytes < w.total) return fail(MILO_ERR_WORKSPACE, "milo_quantize_lorc: workspace too small");
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (r > 0) {
+        const int smem = static_cast<int>(square_smem(w.l));
+        if ((s = check_cuda(cudaFuncSetAttribute(chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                            "chol_kernel attribute")) != MILO_OK)
+            return s;
+        if ((s = check_cuda(cudaFuncSetAttribute(jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                            "jacobi_kernel attribute")) != MILO_OK)
+            return s;
+    }
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    float* R = reinterpret_cast<float*>(base + w.R);
+    uint16_t* Uw = r > 0 ? reinterpret_cast<uint16_t*>(base + w.U) : nullptr;
+    uint16_t* Vw = r > 0 ? reinterpret_cast<uint16_t*>(base + w.V) : nullptr;
+    uint8_t* blob = base + w.blob;
+    double* best = reinterpret_cast<double*>(base + w.best);
+    int* improved = reinterpret_cast<int*>(base + w.flag);
+    const size_t blob_bytes = static_cast<size_t>((N + 63) / 64) * (K / 128) * kBlockSB;
+    const int rounds = r > 0 ? p.rounds : 0;
+    for (int t = 0; t <= rounds; ++t) {
+        const HqqArgs h{W, t > 0 ? Uw : nullptr, t > 0 ? Vw : nullptr, blob, R, dev_status, N, K, t > 0 ? r : 0,
+                        p.hqq_iters, p.hqq_beta, p.hqq_kappa};
+        if ((s = launch_hqq(h, st)) != MILO_OK) return s;
+        if (r > 0 && (s = compensator(st, R, omega, N, K, r, p.power_iters, base, w, Uw, Vw, dev_status)) != MILO_OK)
+            return s;
+        err_kernel<<<w.eblocks, 256, 0, st>>>(R, Uw, Vw, N, K, r, reinterpret_cast<double*>(base + w.epart));
+        err_sum_kernel<<<1, 256, 0, st>>>(reinterpret_cast<double*>(base + w.epart), w.eblocks, t, err, best,
+                                          improved);
+        copy_best_kernel<<<296, 256, 0, st>>>(improved, reinterpret_cast<const uint4*>(blob),
+                                              static_cast<uint4*>(packed), blob_bytes / 16,
+                                              reinterpret_cast<const uint4*>(Uw), reinterpret_cast<uint4*>(U),
+                                              r > 0 ? static_cast<size_t>(N) * r * 2 / 16 : 0,
+                                              reinterpret_cast<const uint4*>(Vw), reinterpret_cast<uint4*>(V),
+                                              r > 0 ? static_cast<size_t>(r) * K * 2 / 16 : 0);
+        if ((s = check_launch("milo_quantize_lorc round")) != MILO_OK) return s;
+    }
+    return MILO_OK;
+}

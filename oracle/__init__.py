@@ -320,12 +320,17 @@ def _split(Y: np.ndarray, B: np.ndarray, r: int):
     triplets of B, returned balanced as U = Y P_r S^(1/2), V = S^(-1/2) P_r^T B."""
     lam, P = np.linalg.eigh(B @ B.T)
     order = np.argsort(-lam, kind="stable")
-    lam, P = lam[order][:r], P[:, order][:, :r]
+    m = min(r, lam.size)
+    lam, P = lam[order][:m], P[:, order][:, :m]
     sig = np.sqrt(np.clip(lam, 0.0, None))
-    live = sig > (sig[0] * 1e-12 if r and sig[0] > 0 else np.inf)
+    live = sig > (sig[0] * 1e-12 if m and sig[0] > 0 else np.inf)
     root = np.where(live, np.sqrt(sig), 0.0)
     inv = np.where(live, 1.0 / np.where(live, np.sqrt(sig), 1.0), 0.0)
-    return (Y @ P) * root[None, :], (P.T @ B) * inv[:, None]
+    U = np.zeros((Y.shape[0], r))
+    V = np.zeros((r, B.shape[1]))
+    U[:, :m] = (Y @ P) * root[None, :]
+    V[:m] = (P.T @ B) * inv[:, None]
+    return U, V   # fewer than r directions (a thin R) leave zero columns / rows
 
 
 def rsvd(R: np.ndarray, r: int, omega: np.ndarray, power_iters: int):

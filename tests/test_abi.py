@@ -92,3 +92,34 @@ def test_workspace_sizes_grow_with_tokens(milo):
     assert L.milo_moe_workspace_bytes(C.byref(layer), 8192, C.byref(b)) == 0
     assert 0 < a.value < b.value
     assert L.milo_moe_h_offset(C.byref(layer), 16) % 256 == 0
+
+
+def test_quantiser_validation_and_workspace(milo):
+    L = milo.lib()
+    fake = C.c_void_p(0x1000)
+    # HQQ pack: K % 128, bad iteration count, non-positive beta, rank > 0 without U
+    assert L.milo_hqq_pack(fake, None, None, 0, 16, 100, 20, 10.0, 1.01, fake, None, None, None) == \
+        milo.MILO_ERR_UNSUPPORTED_SHAPE
+    assert L.milo_hqq_pack(fake, None, None, 0, 16, 128, 1001, 10.0, 1.01, fake, None, None, None) == \
+        milo.MILO_ERR_INVALID_ARG
+    assert L.milo_hqq_pack(fake, None, None, 0, 16, 128, 20, 0.0, 1.01, fake, None, None, None) == \
+        milo.MILO_ERR_INVALID_ARG
+    assert L.milo_hqq_pack(fake, None, None, 8, 16, 128, 20, 10.0, 1.01, fake, None, None, None) == \
+        milo.MILO_ERR_INVALID_ARG
+    nb, nb2 = C.c_size_t(), C.c_size_t()
+    p = milo.lorc_params(12)                      # rank not a multiple of 8
+    assert L.milo_quantize_lorc_workspace(64, 128, C.byref(p), C.byref(nb)) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    p = milo.lorc_params(16, sketch=24)           # sketch not a multiple of 16
+    assert L.milo_quantize_lorc_workspace(64, 128, C.byref(p), C.byref(nb)) == milo.MILO_ERR_INVALID_ARG
+    p = milo.lorc_params(16, sketch=8 * 16 + 16)  # sketch above 128
+    assert L.milo_quantize_lorc_workspace(64, 128, C.byref(p), C.byref(nb)) == milo.MILO_ERR_INVALID_ARG
+    p = milo.lorc_params(16, rounds=17)
+    assert L.milo_quantize_lorc_workspace(64, 128, C.byref(p), C.byref(nb)) == milo.MILO_ERR_INVALID_ARG
+    p = milo.lorc_params(16)
+    assert L.milo_quantize_lorc_workspace(64, 128, C.byref(p), C.byref(nb)) == 0
+    assert L.milo_quantize_lorc_workspace(640, 1280, C.byref(p), C.byref(nb2)) == 0
+    assert 64 * 128 * 4 < nb.value < nb2.value
+    # a workspace one byte short is refused before any launch
+    assert L.milo_quantize_lorc(fake, 64, 128, C.byref(p), fake, C.c_void_p(0x10000), C.c_void_p(0x20000),
+                                C.c_void_p(0x30000), None, C.c_void_p(0x40000), nb.value - 1, None, None) == \
+        milo.MILO_ERR_WORKSPACE
