@@ -3,7 +3,7 @@
 low-rank-compensator forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl milo|reference]
-                    [--workload mixtral|deepseek|prefill|single|sweep256]
+                    [--workload mixtral|deepseek|prefill|quantize] [--lorc fp16|int3]
 
 One step = one pass of the whole hot path over one batch of synthetic tokens:
 router (top-k + grouping) -> activation preparation -> compensator
@@ -612,13 +612,154 @@ def finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, l
     return 0
 
 
+# ---------------------------------------------------------------------------
+# offline quantiser (--workload quantize)
+# ---------------------------------------------------------------------------
+
+QUANT_METRIC = ("offline MiLo quantiser: weights quantised and compensated per second "
+                "(HQQ int3, rank-r compensator by subspace iteration, refinement rounds)")
+# fp32 operations of one HQQ iteration per weight outside the shrinkage (which
+# is zero for all but outlier errors): t*inv, +z, rint, two clamps, -z, *s,
+# t-w_r, |e|, err+, t-w_e, *inv, r-u, acc+, and the a^3 beta^2 pre-test's
+# first product counted once -> 15
+HQQ_OPS_PER_WEIGHT_ITER = 15
+FP32_LANES = 148 * 4 * 32
+
+
+def quant_matrices(rank_id: int, hidden: int = 4096, inter: int = 14336):
+    """One Mixtral-shaped expert's w1, w3 [inter, hidden] and w2 [hidden, inter]."""
+    return [wl.gen_weight(wl.rng_for("quantize", name, rank_id), n, k)
+            for name, n, k in (("w1", inter, hidden), ("w3", inter, hidden), ("w2", hidden, inter))]
+
+
+def quant_cpu_baseline(r: int, rounds: int, budget_rows: int = 2048) -> dict:
+    """The oracle's quantiser on a sampled [budget_rows, 4096] slice of w1."""
+    import oracle
+    W = np.ascontiguousarray(wl.gen_weight(wl.rng_for("quantize", "w1", 0), 14336, 4096)[:budget_rows])
+    rng = wl.rng_for("quantize", "omega_cpu", 0)
+    om = rng.standard_normal((W.shape[1], 2 * r))
+    t0 = time.perf_counter()
+    oracle.quantize_lorc(W, r, rounds, om)
+    dt = time.perf_counter() - t0
+    return {"value": W.size / dt, "unit": "weights/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"HQQ + rank-{r} compensator + {rounds} rounds on a [{W.shape[0]}, {W.shape[1]}] slice of "
+                      f"w1 ({dt:.1f} s; HQQ in C on one thread, the subspace iteration in numpy BLAS)"}
+
+
+def run_quantize(args):
+    import ctypes as C
+
+    import torch
+
+    import int3_gemm_rank_b200 as milo
+    from int3_gemm_rank_b200 import build as milo_build
+
+    rank, local, world = dist_env()
+    if not os.path.exists(milo.LIB_PATH):
+        milo_build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+    r, rounds = args.quant_rank, args.quant_rounds
+    params = milo.lorc_params(r, rounds=rounds)
+    L = milo.lib()
+    jobs = []
+    for i, Wn in enumerate(quant_matrices(rank)):
+        N, K = Wn.shape
+        W = torch.from_numpy(Wn.view(np.int16)).view(torch.float16).to(dev)
+        om = torch.from_numpy(wl.rng_for("quantize", "omega", i).standard_normal((K, params.sketch))
+                              .astype(np.float32)).to(dev)
+        blob = torch.empty(milo.milo_packed_bytes(N, K), dtype=torch.uint8, device=dev)
+        U = torch.empty((N, r), dtype=torch.float16, device=dev)
+        V = torch.empty((r, K), dtype=torch.float16, device=dev)
+        err = torch.empty(rounds + 1, dtype=torch.float32, device=dev)
+        nb = milo.milo_quantize_lorc_workspace(N, K, params)
+        ws = torch.empty(nb + 256, dtype=torch.uint8, device=dev)
+        wp = ws.data_ptr() + (-ws.data_ptr()) % 256
+        jobs.append((N, K, W, om, blob, U, V, err, wp, nb, ws))   # ws stays referenced: wp points into it
+    st = milo.new_status(dev)
+    sp = C.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+    def step():
+        for N, K, W, om, blob, U, V, err, wp, nb, _ws in jobs:
+            s = L.milo_quantize_lorc(C.c_void_p(W.data_ptr()), N, K, C.byref(params), C.c_void_p(om.data_ptr()),
+                                     C.c_void_p(blob.data_ptr()), C.c_void_p(U.data_ptr()),
+                                     C.c_void_p(V.data_ptr()), C.c_void_p(err.data_ptr()), C.c_void_p(wp), nb,
+                                     C.c_void_p(st.data_ptr()), sp)
+            if s != 0:
+                raise RuntimeError(f"milo_quantize_lorc: {L.milo_last_error().decode()}")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} on the quantiser workload")
+    clock = ClockSampler(local)
+    clock.start()
+    barrier(dev)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    # the HQQ kernel alone (milo_hqq_pack launches the same kernel on W), on w1
+    N1, K1, W1 = jobs[0][0], jobs[0][1], jobs[0][2]
+    blob1 = torch.empty_like(jobs[0][4])
+    hq = []
+    for _ in range(max(3, min(args.steps, 20))):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        L.milo_hqq_pack(C.c_void_p(W1.data_ptr()), None, None, 0, N1, K1, params.hqq_iters,
+                        C.c_float(params.hqq_beta), C.c_float(params.hqq_kappa), C.c_void_p(blob1.data_ptr()), None,
+                        None, sp)
+        b.record()
+        hq.append((a, b))
+    torch.cuda.synchronize()
+    clocks = clock.stop()
+    hqq_ms = statistics.median(a.elapsed_time(b) for a, b in hq[1:])
+    weights = sum(j[0] * j[1] for j in jobs)
+    sm_mhz = clocks.get("sm_mhz") or 1965.0
+    peak = FP32_LANES * sm_mhz * 1e6 / 1e12
+    achieved = HQQ_OPS_PER_WEIGHT_ITER * N1 * K1 * params.hqq_iters / (hqq_ms / 1e3) / 1e12
+    line = {
+        "metric": QUANT_METRIC, "value": weights * world / (ms / 1e3), "unit": "weights/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"quantise one Mixtral-shaped expert per GPU: w1, w3 [14336, 4096], w2 [4096, 14336]; "
+                               f"rank {r}, {rounds} refinement rounds, sketch {params.sketch}, "
+                               f"{params.power_iters} power steps, HQQ {params.hqq_iters} iterations",
+                   "l2": "inputs larger than L2 (117 MB fp16 weight plus its 235 MB fp32 residual per matrix)",
+                   "parallelism": f"replica per GPU x{world}"},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Top/s", "frac": achieved / peak,
+                     "traffic": None, "kernel": "hqq_pack_kernel (HQQ zero-point fit + pack, w1 shape)",
+                     "algorithmic_ops_per_launch": HQQ_OPS_PER_WEIGHT_ITER * N1 * K1 * params.hqq_iters,
+                     "ms_per_launch": hqq_ms,
+                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x the sampled SM clock"},
+        "gpu_launches": None, "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = quant_cpu_baseline(r, rounds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("milo", "reference"), default="milo")
-    ap.add_argument("--workload", choices=("mixtral", "deepseek", "prefill"), default="mixtral")
+    ap.add_argument("--workload", choices=("mixtral", "deepseek", "prefill", "quantize"), default="mixtral",
+                    help="quantize: the offline quantiser on one Mixtral-shaped expert (its own JSON line)")
+    ap.add_argument("--quant-rank", type=int, default=32)
+    ap.add_argument("--quant-rounds", type=int, default=3)
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -631,6 +772,12 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.workload == "quantize":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the layer forward; "
+                              "the quantiser's CPU baseline is part of its own line"}))
+            return 0
+        return run_quantize(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_milo(args)

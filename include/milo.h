@@ -146,10 +146,10 @@ MILO_API milo_status milo_unpack(const void* packed, int32_t N, int32_t K, uint8
  * HQQ here (per group of 64 along K, all fp32 in this order, no FMA):
  *     s = fp16((max - min) / 7) (1 when it rounds to 0), z = -min / s, beta = hqq_beta
  *     repeat hqq_iters times:
- *         q = clamp(rint(t / s + z), 0, 7);  e = t - (q - z) s
+ *         q = clamp(rint(t * (1/s) + z), 0, 7);  e = t - (q - z) s
  *         L1 = sum |e| (index order); remember z if L1 is the lowest so far
  *         w_e = sign(e) max(|e| - 1 / (sqrt|e| beta), 0)     (lp shrinkage, p = 1/2)
- *         z = (sum over the group of q - (t - w_e) / s) * (1/64);  beta *= hqq_kappa
+ *         z = (sum over the group of q - (t - w_e) * (1/s)) * (1/64);  beta *= hqq_kappa
  *     z := fp16(remembered z); q = clamp(rint(t / s + z), 0, 7)  (as milo_pack)
  * With hqq_iters <= 1 this is exactly milo_pack's round-to-nearest quantiser.
  */
@@ -200,15 +200,17 @@ MILO_API milo_status milo_quantize_lorc_workspace(int32_t N, int32_t K, const mi
  * B = Y^T R; the eigenpairs of B B^T (descending lambda) give sigma_i =
  * sqrt(lambda_i), and, for the top r, U = Y P_r sigma^(1/2) [N, r],
  * V = sigma^(-1/2) P_r^T B [r, K] (a direction with sigma below 1e-12 sigma_0
- * gets zero U and V).  orth() is Cholesky QR applied twice (fp64 Gram and
- * Cholesky, fp32 products); eigenpairs by cyclic Jacobi in fp64.
+ * gets zero U and V).  orth() is Cholesky QR (fp64 Gram and Cholesky, fp32
+ * products; columns dependent on earlier ones are dropped), once between
+ * power steps and twice for the final Y; eigenpairs by cyclic Jacobi in fp64.
  *   omega: f32 [K, sketch] row-major, the random test matrix (an input: the
  *   caller draws it, e.g. standard normal); NULL when r = 0.
  *   packed (milo_packed_bytes), U fp16 [N, r], V fp16 [r, K]: the round with
  *   the lowest error (the first on ties); U, V NULL when r = 0.
  *   err: NULL, or f32 [rounds + 1] (1 when r = 0) receiving each round's
  *   ||W - W_hat - U V||_F (fp16 U, V; accumulated in fp64).
- *   ws: milo_quantize_lorc_workspace bytes, 256-byte aligned, caller-owned.
+ *   ws: milo_quantize_lorc_workspace bytes, 256-byte aligned, caller-owned;
+ *   W must be 8-byte aligned.
  * Errors as milo_hqq_pack, plus: params NULL, rank outside 0..64, rounds,
  * sketch or power_iters out of range, omega / U / V NULL with r > 0, ws too
  * small or unaligned -> INVALID_ARG / WORKSPACE.  Stream-ordered, no host

@@ -23,7 +23,8 @@
 //     of the factor in fp64: the basis change of Cholesky QR.
 //   - jacobi_kernel (one block): cyclic Jacobi eigenpairs of B B^T in fp64,
 //     l/2 disjoint rotations per step (round-robin ordering).
-//   - err_kernel + err_sum_kernel: ||R - U V||_F in fp64 and the best-round
+//   - apply_kernel + err_sum_kernel: ||R - U V||_F in fp64 and the next
+//     round's target W - U V in one coalesced pass, the best-round
 //     bookkeeping; copy_best_kernel keeps the best round's blob, U and V.
 #include <cuda_runtime.h>
 
@@ -45,6 +46,7 @@ struct HqqArgs {
     const uint16_t* W;      // [N, K] fp16
     const uint16_t* U;      // [N, r] fp16 or null
     const uint16_t* V;      // [r, K] fp16 or null
+    const float* T;         // [N, K] fp32 target W - U V formed beforehand, or null
     uint8_t* blob;
     float* resid;           // [N, K] or null
     int32_t* dev_status;
@@ -68,23 +70,28 @@ __device__ __forceinline__ int32_t hqq_group(const float (&t)[64], int iters, fl
     if ((__half_as_ushort(sh) & 0x7FFF) == 0) sh = __ushort_as_half(0x3C00);   // s := 1
     const float s = __half2float(sh);
     float z = __fdiv_rn(-mn, s);
+    const float inv = __fdiv_rn(1.0f, s);   // HQQ quantises with the inverse scale
     float beta = beta0, best_err = INFINITY, best_z = z;
     for (int it = 0; it < iters; ++it) {
         float err = 0.0f, acc = 0.0f;
+        const float beta2 = __fmul_rn(beta, beta);
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-            float r = rintf(__fadd_rn(__fdiv_rn(t[i], s), z));
+            float r = rintf(__fadd_rn(__fmul_rn(t[i], inv), z));
             if (!(r >= 0.0f)) r = 0.0f;
             if (r > 7.0f) r = 7.0f;
             const float e = __fsub_rn(t[i], __fmul_rn(__fsub_rn(r, z), s));
             const float a = fabsf(e);
             err = __fadd_rn(err, a);
             float w_e = 0.0f;
-            if (a > 0.0f) {
+            // a^3 beta^2 < 1/2 means 1 / (sqrt(a) beta) > 1.41 a, so the shrinkage
+            // is zero whatever the rounding; only larger errors need the formula
+            const float a3b2 = __fmul_rn(__fmul_rn(__fmul_rn(a, a), a), beta2);
+            if (a > 0.0f && !(a3b2 < 0.5f)) {
                 const float m = __fsub_rn(a, __fdiv_rn(1.0f, __fmul_rn(__fsqrt_rn(a), beta)));
                 if (m > 0.0f) w_e = e < 0.0f ? -m : m;
             }
-            acc = __fadd_rn(acc, __fsub_rn(r, __fdiv_rn(__fsub_rn(t[i], w_e), s)));
+            acc = __fadd_rn(acc, __fsub_rn(r, __fmul_rn(__fsub_rn(t[i], w_e), inv)));
         }
         if (err < best_err) {
             best_err = err;
@@ -115,11 +122,20 @@ __global__ void __launch_bounds__(128) hqq_pack_kernel(const HqqArgs a) {
     for (int g = 0; g < 2; ++g) {
         const size_t k0 = static_cast<size_t>(n) * a.K + 128 * b + 64 * g;
         float t[64];
+        if (a.T) {
+            const float4* tp = reinterpret_cast<const float4*>(a.T + k0);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) t[i] = f16v(a.W[k0 + i]);
-        // t = W - U V, one rank term at a time
+            for (int i = 0; i < 16; ++i) {
+                const float4 v = tp[i];
+                t[4 * i] = v.x; t[4 * i + 1] = v.y; t[4 * i + 2] = v.z; t[4 * i + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) t[i] = f16v(a.W[k0 + i]);
+        }
+        // t = W - U V, one rank term at a time (when not formed beforehand)
 #pragma unroll 1
-        for (int p = 0; p < a.r; ++p) {
+        for (int p = 0; p < (a.T ? 0 : a.r); ++p) {
             const float u = f16v(a.U[static_cast<size_t>(n) * a.r + p]);
             const uint16_t* vr = a.V + static_cast<size_t>(p) * a.K + 128 * b + 64 * g;
 #pragma unroll
@@ -158,6 +174,8 @@ struct GemmArgs {
     uint16_t* C16;           // the same in fp16 (round to nearest)
     long long ldc;
     int32_t* dev_status;
+    float* Cpart;            // split reduction: slice z writes Cpart[z][m][n], else null
+    int kslice;              // reduction length per slice (multiple of kGK)
 };
 
 constexpr int kGT = 64;      // output tile
@@ -176,7 +194,9 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const GemmArgs a) {
     for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-    for (int k0 = 0; k0 < a.Kd; k0 += kGK) {
+    const int kbeg = blockIdx.z * a.kslice;
+    const int kend = min(a.Kd, kbeg + a.kslice);
+    for (int k0 = kbeg; k0 < kend; k0 += kGK) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int idx = tid + 256 * i;
@@ -184,12 +204,12 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const GemmArgs a) {
             if (a.sak == 1) { kk = idx % kGK; mm = idx / kGK; }
             else { mm = idx % kGT; kk = idx / kGT; }
             const int m = m0 + mm, k = k0 + kk;
-            As[kk][mm] = (m < a.M && k < a.Kd) ? a.A[m * a.sam + k * a.sak] : 0.0f;
+            As[kk][mm] = (m < a.M && k < kend) ? a.A[m * a.sam + k * a.sak] : 0.0f;
             int nn;
             if (a.sbn == 1) { nn = idx % kGT; kk = idx / kGT; }
             else { kk = idx % kGK; nn = idx / kGK; }
             const int n = n0 + nn, kb = k0 + kk;
-            Bs[kk][nn] = (n < a.Nn && kb < a.Kd) ? a.B[kb * a.sbk + n * a.sbn] : 0.0f;
+            Bs[kk][nn] = (n < a.Nn && kb < kend) ? a.B[kb * a.sbk + n * a.sbn] : 0.0f;
         }
         __syncthreads();
 #pragma unroll
@@ -211,7 +231,9 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const GemmArgs a) {
         for (int j = 0; j < 4; ++j) {
             const int m = m0 + tm + i, n = n0 + tn + j;
             if (m >= a.M || n >= a.Nn) continue;
-            if (a.C16) {
+            if (a.Cpart) {
+                a.Cpart[(static_cast<size_t>(blockIdx.z) * a.M + m) * a.Nn + n] = acc[i][j];
+            } else if (a.C16) {
                 const __half h = __float2half_rn(acc[i][j]);
                 if (!isfinite(__half2float(h))) st |= MILO_DEV_FP16_RANGE;
                 a.C16[m * a.ldc + n] = __half_as_ushort(h);
@@ -220,6 +242,23 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const GemmArgs a) {
             }
         }
     flag(a.dev_status, st);
+}
+
+// C(m, n) = sum over slices z, in order, of Cpart[z][m][n] (fp32 or fp16 out).
+__global__ void split_sum_kernel(const float* Cpart, int S, int M, int Nn, float* C, uint16_t* C16, long long ldc,
+                                 int32_t* dev_status) {
+    const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (e >= static_cast<long long>(M) * Nn) return;
+    float v = 0.0f;
+    for (int z = 0; z < S; ++z) v += Cpart[static_cast<size_t>(z) * M * Nn + e];
+    const int m = static_cast<int>(e / Nn), n = static_cast<int>(e % Nn);
+    if (C16) {
+        const __half h = __float2half_rn(v);
+        if (!isfinite(__half2float(h))) flag(dev_status, MILO_DEV_FP16_RANGE);
+        C16[m * ldc + n] = __half_as_ushort(h);
+    } else {
+        C[m * ldc + n] = v;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -297,52 +336,55 @@ __global__ void gram_sum_kernel(const double* part, int chunks, int ll, double* 
 // G [l, l] fp64 (symmetric positive semi-definite) -> M fp32 [l, l] with
 // Y M = Y L^-T, L the Cholesky factor of G.  A pivot below 1e-10 of its
 // diagonal entry marks a column that lies in the span of the earlier ones:
-// its column of M is zero (the basis drops that direction).  X is fp64 [l, l]
-// scratch for the inverse.
-__global__ void __launch_bounds__(256) chol_kernel(const double* G, int l, float* M, double* X) {
-    extern __shared__ double Ls[];               // [l][l + 1]
+// its column of M is zero (the basis drops that direction).  L and X = L^-1
+// are lower triangles packed in shared memory (entry (i, j), j <= i, at
+// i (i + 1) / 2 + j), fp64.
+__device__ __forceinline__ int tri(int i, int j) { return i * (i + 1) / 2 + j; }
+
+__global__ void __launch_bounds__(256) chol_kernel(const double* G, int l, float* M) {
+    extern __shared__ double sh[];
+    double* L = sh;                               // [l (l + 1) / 2]
+    double* X = sh + l * (l + 1) / 2;             // [l (l + 1) / 2]
     __shared__ int dead[kMaxSketch];
-    const int ld = l + 1, tid = threadIdx.x;
-    for (int idx = tid; idx < l * l; idx += blockDim.x) Ls[(idx / l) * ld + idx % l] = G[idx];
+    const int tid = threadIdx.x;
+    for (int i = 0; i < l; ++i)
+        for (int j = tid; j <= i; j += blockDim.x) L[tri(i, j)] = G[i * l + j];
     __syncthreads();
     for (int j = 0; j < l; ++j) {
         if (tid == 0) {
-            double d = Ls[j * ld + j];
-            for (int k = 0; k < j; ++k) d -= Ls[j * ld + k] * Ls[j * ld + k];
+            double d = L[tri(j, j)];
+            for (int k = 0; k < j; ++k) d -= L[tri(j, k)] * L[tri(j, k)];
             const bool gone = !(d > 1e-10 * G[j * l + j]);
             dead[j] = gone;
-            Ls[j * ld + j] = gone ? 1.0 : sqrt(d);
+            L[tri(j, j)] = gone ? 1.0 : sqrt(d);
         }
         __syncthreads();
-        const double piv = Ls[j * ld + j];
+        const double piv = L[tri(j, j)];
         for (int i = j + 1 + tid; i < l; i += blockDim.x) {
             double v = 0.0;
             if (!dead[j]) {
-                v = Ls[i * ld + j];
-                for (int k = 0; k < j; ++k) v -= Ls[i * ld + k] * Ls[j * ld + k];
+                v = L[tri(i, j)];
+                for (int k = 0; k < j; ++k) v -= L[tri(i, k)] * L[tri(j, k)];
                 v /= piv;
             }
-            Ls[i * ld + j] = v;
+            L[tri(i, j)] = v;
         }
         __syncthreads();
     }
     // X = L^-1 by forward substitution, one column per thread
     for (int c = tid; c < l; c += blockDim.x) {
-        for (int i = 0; i < l; ++i) {
-            double v = 0.0;
-            if (i >= c) {
-                v = i == c ? 1.0 : 0.0;
-                for (int k = c; k < i; ++k) v -= Ls[i * ld + k] * X[k * l + c];
-                v /= Ls[i * ld + i];
-            }
-            X[i * l + c] = v;
+        for (int i = c; i < l; ++i) {
+            double v = i == c ? 1.0 : 0.0;
+            for (int k = c; k < i; ++k) v -= L[tri(i, k)] * X[tri(k, c)];
+            X[tri(i, c)] = v / L[tri(i, i)];
         }
     }
     __syncthreads();
-    // M[k][i] = X[i][k]; the row of X of a dropped column is zero
+    // M[k][i] = X[i][k] (zero above the diagonal of X); the row of X of a
+    // dropped column is zero
     for (int idx = tid; idx < l * l; idx += blockDim.x) {
         const int k = idx / l, i = idx % l;
-        M[idx] = dead[i] ? 0.0f : static_cast<float>(X[i * l + k]);
+        M[idx] = (dead[i] || k > i) ? 0.0f : static_cast<float>(X[tri(i, k)]);
     }
 }
 
@@ -353,15 +395,17 @@ __global__ void __launch_bounds__(256) chol_kernel(const double* G, int l, float
 // C [l, l] fp64 symmetric (l even) -> the top r eigenpairs in descending
 // order of eigenvalue, emitted as MU fp32 [l, r] = P_r sigma^(1/2) and MV fp32
 // [r, l] = sigma^(-1/2) P_r^T with sigma = sqrt(max(lambda, 0)); directions
-// with sigma <= 1e-12 sigma_0 get zeros.  P is fp64 [l, l] scratch (the
-// eigenvectors).  Each sweep pairs every index with every other once
+// with sigma <= 1e-12 sigma_0 get zeros.  The eigenvectors P accumulate in
+// fp32 in shared memory next to the fp64 matrix.  Each sweep pairs every index with every other once
 // (round-robin: index l-1 fixed, the rest rotating), l/2 disjoint rotations
 // per step; at most kJacobiSweeps sweeps, fewer once the off-diagonal mass
-// falls below 1e-30 of the total.
+// falls below 1e-24 of the total (off-diagonal entries near 1e-12 of the
+// matrix: far below the fp32 and fp16 outputs).
 constexpr int kJacobiSweeps = 40;
 
-__global__ void __launch_bounds__(256) jacobi_kernel(const double* C, int l, int r, double* P, float* MU, float* MV) {
-    extern __shared__ double As[];               // [l][l + 1]
+__global__ void __launch_bounds__(256) jacobi_kernel(const double* C, int l, int r, float* MU, float* MV) {
+    extern __shared__ double As[];               // [l][l + 1], then P fp32 [l][l + 1]
+    float* P = reinterpret_cast<float*>(As + l * (l + 1));
     __shared__ double cs[kMaxSketch / 2], sn[kMaxSketch / 2];
     __shared__ int pp[kMaxSketch / 2], qq[kMaxSketch / 2], order[kMaxSketch];
     __shared__ double red[256];
@@ -369,7 +413,7 @@ __global__ void __launch_bounds__(256) jacobi_kernel(const double* C, int l, int
     const int ld = l + 1, tid = threadIdx.x, half = l / 2, m = l - 1;
     for (int idx = tid; idx < l * l; idx += blockDim.x) {
         As[(idx / l) * ld + idx % l] = C[idx];
-        P[idx] = (idx / l == idx % l) ? 1.0 : 0.0;
+        P[(idx / l) * ld + idx % l] = (idx / l == idx % l) ? 1.0f : 0.0f;
     }
     __syncthreads();
     for (int sweep = 0; sweep < kJacobiSweeps; ++sweep) {
@@ -393,7 +437,7 @@ __global__ void __launch_bounds__(256) jacobi_kernel(const double* C, int l, int
             if (tid < s) red[tid] += red[tid + s];
             __syncthreads();
         }
-        if (tid == 0) stop = !(off_all > 1e-30 * red[0]);
+        if (tid == 0) stop = !(off_all > 1e-24 * red[0]);
         __syncthreads();
         if (stop) break;
         for (int step = 0; step < m; ++step) {
@@ -426,9 +470,9 @@ __global__ void __launch_bounds__(256) jacobi_kernel(const double* C, int l, int
                 const double ap = As[i * ld + p], aq = As[i * ld + q];
                 As[i * ld + p] = cs[k] * ap - sn[k] * aq;
                 As[i * ld + q] = sn[k] * ap + cs[k] * aq;
-                const double vp = P[i * l + p], vq = P[i * l + q];
-                P[i * l + p] = cs[k] * vp - sn[k] * vq;
-                P[i * l + q] = sn[k] * vp + cs[k] * vq;
+                const double vp = P[i * ld + p], vq = P[i * ld + q];
+                P[i * ld + p] = static_cast<float>(cs[k] * vp - sn[k] * vq);
+                P[i * ld + q] = static_cast<float>(sn[k] * vp + cs[k] * vq);
             }
             __syncthreads();
         }
@@ -451,7 +495,7 @@ __global__ void __launch_bounds__(256) jacobi_kernel(const double* C, int l, int
         const double sig = sqrt(fmax(As[order[i] * ld + order[i]], 0.0));
         const bool live = sig0 > 0.0 && sig > 1e-12 * sig0;
         const double root = live ? sqrt(sig) : 0.0;
-        const double v = P[a * l + order[i]];
+        const double v = P[a * ld + order[i]];
         MU[a * r + i] = static_cast<float>(v * root);
         MV[i * l + a] = live ? static_cast<float>(v / root) : 0.0f;
     }
@@ -461,33 +505,56 @@ __global__ void __launch_bounds__(256) jacobi_kernel(const double* C, int l, int
 // Error norm, best round, copies
 // ---------------------------------------------------------------------------
 
-// Block partial of sum (R - U V)^2 over (row, 128-column segment) threads, in
-// fp64 (U V summed over the rank in fp64); warp and block sums in a fixed tree.
-__global__ void __launch_bounds__(256) err_kernel(const float* R, const uint16_t* U, const uint16_t* V, int N, int K,
-                                                  int r, double* part) {
-    __shared__ double ws[8];
-    const int SB = K / 128;
+// One thread per (row n, 4 consecutive columns), so a warp reads 128
+// consecutive entries of each V row.  Per entry it forms the products
+// U[n, p] V[p, k] (exact in fp32: fp16 times fp16) once and uses them twice:
+//   - the error term (R - sum_p U V)^2, summed over p in fp64;
+//   - when T is not null, the next round's target t = W, then t = t - U V for
+//     p = 0..r-1 rounded to fp32 at every step (the order milo_hqq_pack uses).
+// Block partials of the squared error go to part[] (fixed reduction tree).
+constexpr int kApplyThreads = 256;
+
+__global__ void __launch_bounds__(kApplyThreads) apply_kernel(const float* R, const uint16_t* W, const uint16_t* U,
+                                                              const uint16_t* V, int N, int K, int r, float* T,
+                                                              double* part) {
+    __shared__ double ws[kApplyThreads / 32];
+    const int K4 = K / 4;
     const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     double acc = 0.0;
-    if (gid < static_cast<long long>(N) * SB) {
-        const int n = static_cast<int>(gid / SB), b = static_cast<int>(gid % SB);
-        for (int k = 128 * b; k < 128 * b + 128; ++k) {
-            double uv = 0.0;
-            for (int p = 0; p < r; ++p)
-                uv = fma(static_cast<double>(f16v(U[static_cast<size_t>(n) * r + p])),
-                         static_cast<double>(f16v(V[static_cast<size_t>(p) * K + k])), uv);
-            const double d = static_cast<double>(R[static_cast<size_t>(n) * K + k]) - uv;
+    if (gid < static_cast<long long>(N) * K4) {
+        const int n = static_cast<int>(gid / K4), k0 = static_cast<int>(gid % K4) * 4;
+        const size_t o = static_cast<size_t>(n) * K + k0;
+        const float4 rv = *reinterpret_cast<const float4*>(R + o);
+        const uint2 wv = *reinterpret_cast<const uint2*>(W + o);
+        float t[4] = {f16v(wv.x & 0xFFFFu), f16v(wv.x >> 16), f16v(wv.y & 0xFFFFu), f16v(wv.y >> 16)};
+        double uv[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int p = 0; p < r; ++p) {
+            const float u = f16v(U[static_cast<size_t>(n) * r + p]);
+            const uint2 vv = *reinterpret_cast<const uint2*>(V + static_cast<size_t>(p) * K + k0);
+            const float v[4] = {f16v(vv.x & 0xFFFFu), f16v(vv.x >> 16), f16v(vv.y & 0xFFFFu), f16v(vv.y >> 16)};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float prod = __fmul_rn(u, v[j]);
+                t[j] = __fsub_rn(t[j], prod);
+                uv[j] += static_cast<double>(prod);
+            }
+        }
+        const float rr[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const double d = static_cast<double>(rr[j]) - uv[j];
             acc = fma(d, d, acc);
         }
+        if (T) *reinterpret_cast<float4*>(T + o) = make_float4(t[0], t[1], t[2], t[3]);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
     if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = acc;
     __syncthreads();
     if (threadIdx.x == 0) {
-        double s = 0.0;
-        for (int w = 0; w < 8; ++w) s += ws[w];
-        part[blockIdx.x] = s;
+        double sum = 0.0;
+        for (int w = 0; w < kApplyThreads / 32; ++w) sum += ws[w];
+        part[blockIdx.x] = sum;
     }
 }
 
@@ -532,10 +599,14 @@ __global__ void copy_best_kernel(const int* improved, const uint4* src0, uint4* 
 
 namespace {
 
-constexpr int kGramChunk = 256;   // rows per Gram partial
+constexpr int kGramChunk = 64;    // rows per Gram partial
+// Split reductions: a product whose output tiles fill fewer than 148 blocks and
+// whose reduction is long splits it into S slices (S x blocks <= 296) summed in
+// slice order by split_sum_kernel, so the partials fit kSplitFloats.
+constexpr int kSplitFloats = 296 * kGT * kGT;
 
 struct QuantWs {
-    size_t R, Y, Y2, Z, Z2, B, part, G, X, M, P, MU, MV, U, V, blob, epart, best, flag, total;
+    size_t R, T, Y, Y2, Z, Z2, B, part, gpart, G, M, MU, MV, U, V, blob, epart, best, flag, total;
     int l, chunks, eblocks;
 };
 
@@ -557,19 +628,19 @@ QuantWs quant_layout(int N, int K, const milo_lorc_params& p) {
         w.Z = take(static_cast<size_t>(K) * l * 4);
         w.Z2 = take(static_cast<size_t>(K) * l * 4);
         w.B = take(static_cast<size_t>(l) * K * 4);
+        w.gpart = take(static_cast<size_t>(kSplitFloats) * 4);
+        if (p.rounds > 0) w.T = take(static_cast<size_t>(N) * K * 4);
         w.chunks = (std::max(N, K) + kGramChunk - 1) / kGramChunk;
         w.part = take(static_cast<size_t>(w.chunks) * l * l * 8);
         w.G = take(static_cast<size_t>(l) * l * 8);
-        w.X = take(static_cast<size_t>(l) * l * 8);
         w.M = take(static_cast<size_t>(l) * l * 4);
-        w.P = take(static_cast<size_t>(l) * l * 8);
         w.MU = take(static_cast<size_t>(l) * r * 4);
         w.MV = take(static_cast<size_t>(r) * l * 4);
         w.U = take(static_cast<size_t>(N) * r * 2);
         w.V = take(static_cast<size_t>(r) * K * 2);
     }
     w.blob = take(static_cast<size_t>((N + 63) / 64) * (K / 128) * kBlockSB);
-    w.eblocks = static_cast<int>((static_cast<long long>(N) * (K / 128) + 255) / 256);
+    w.eblocks = static_cast<int>((static_cast<long long>(N) * (K / 4) + kApplyThreads - 1) / kApplyThreads);
     w.epart = take(static_cast<size_t>(w.eblocks) * 8);
     w.best = take(8);
     w.flag = take(4);
@@ -597,10 +668,20 @@ milo_status launch_hqq(const HqqArgs& a, cudaStream_t st) {
 }
 
 milo_status gemm(cudaStream_t st, int M, int Nn, int Kd, const float* A, long long sam, long long sak, const float* B,
-                 long long sbk, long long sbn, float* C, uint16_t* C16, long long ldc, int32_t* dev_status) {
-    const GemmArgs a{M, Nn, Kd, A, sam, sak, B, sbk, sbn, C, C16, ldc, dev_status};
-    const dim3 grid((Nn + kGT - 1) / kGT, (M + kGT - 1) / kGT);
-    sgemm_kernel<<<grid, 256, 0, st>>>(a);
+                 long long sbk, long long sbn, float* C, uint16_t* C16, long long ldc, int32_t* dev_status,
+                 float* gpart) {
+    const int gx = (Nn + kGT - 1) / kGT, gy = (M + kGT - 1) / kGT;
+    int S = 1;
+    if (gpart && gx * gy < 148 && Kd >= 2048) S = std::min(8, std::max(1, 296 / (gx * gy)));
+    const int kslice = static_cast<int>(round_up((Kd + S - 1) / S, kGK));
+    S = (Kd + kslice - 1) / kslice;
+    const GemmArgs a{M, Nn, Kd, A, sam, sak, B, sbk, sbn, C, C16, ldc, dev_status, S > 1 ? gpart : nullptr, kslice};
+    sgemm_kernel<<<dim3(gx, gy, S), 256, 0, st>>>(a);
+    if (S > 1) {
+        const long long e = static_cast<long long>(M) * Nn;
+        split_sum_kernel<<<static_cast<unsigned>((e + 255) / 256), 256, 0, st>>>(gpart, S, M, Nn, C, C16, ldc,
+                                                                                dev_status);
+    }
     return check_launch("sgemm_kernel");
 }
 
@@ -614,22 +695,30 @@ milo_status gram(cudaStream_t st, const float* X, long long sxi, long long sxc, 
     return check_launch("gram_kernel");
 }
 
-size_t square_smem(int l) { return static_cast<size_t>(l) * (l + 1) * 8; }
+size_t chol_smem(int l) { return static_cast<size_t>(l) * (l + 1) * 8; }          // two packed triangles
+size_t jacobi_smem(int l) { return static_cast<size_t>(l) * (l + 1) * (8 + 4); }  // fp64 matrix, fp32 P
 
-// Y [M, l] <- an orthonormal basis of its columns (Cholesky QR, twice).
+// Y [M, l] <- a basis of its columns: Cholesky QR once (between power steps,
+// where only the spanned subspace matters) or twice (orthonormal to fp32
+// rounding, for the Rayleigh-Ritz step).  The result is in Y either way.
 milo_status orth(cudaStream_t st, float* Y, float* Y2, int M, int l, uint8_t* base, const QuantWs& w,
-                 int32_t* dev_status) {
+                 int32_t* dev_status, int passes) {
     milo_status s;
     double* G = reinterpret_cast<double*>(base + w.G);
     float* Mm = reinterpret_cast<float*>(base + w.M);
-    for (int pass = 0; pass < 2; ++pass) {
+    float* gpart = reinterpret_cast<float*>(base + w.gpart);
+    for (int pass = 0; pass < passes; ++pass) {
         if ((s = gram(st, Y, l, 1, M, l, reinterpret_cast<double*>(base + w.part), G)) != MILO_OK) return s;
-        chol_kernel<<<1, 256, square_smem(l), st>>>(G, l, Mm, reinterpret_cast<double*>(base + w.X));
+        chol_kernel<<<1, 256, chol_smem(l), st>>>(G, l, Mm);
         if ((s = check_launch("chol_kernel")) != MILO_OK) return s;
-        if ((s = gemm(st, M, l, l, Y, l, 1, Mm, l, 1, Y2, nullptr, l, dev_status)) != MILO_OK) return s;
+        // the product lands in the other buffer; after an odd pass copy it back
+        if ((s = gemm(st, M, l, l, Y, l, 1, Mm, l, 1, Y2, nullptr, l, dev_status, gpart)) != MILO_OK) return s;
         std::swap(Y, Y2);
     }
-    return MILO_OK;   // two swaps: the basis is back in the first buffer
+    if (passes % 2)
+        return check_cuda(cudaMemcpyAsync(Y2, Y, static_cast<size_t>(M) * l * 4, cudaMemcpyDeviceToDevice, st),
+                          "orth copy");
+    return MILO_OK;
 }
 
 // U fp16 [N, r], V fp16 [r, K] from R [N, K] (randomized subspace iteration).
@@ -643,22 +732,23 @@ milo_status compensator(cudaStream_t st, const float* R, const float* omega, int
     float* Z2 = reinterpret_cast<float*>(base + w.Z2);
     float* Bm = reinterpret_cast<float*>(base + w.B);
     double* G = reinterpret_cast<double*>(base + w.G);
-    if ((s = gemm(st, N, l, K, R, K, 1, omega, l, 1, Y, nullptr, l, dev_status)) != MILO_OK) return s;
-    if ((s = orth(st, Y, Y2, N, l, base, w, dev_status)) != MILO_OK) return s;
+    float* gpart = reinterpret_cast<float*>(base + w.gpart);
+    if ((s = gemm(st, N, l, K, R, K, 1, omega, l, 1, Y, nullptr, l, dev_status, gpart)) != MILO_OK) return s;
+    if ((s = orth(st, Y, Y2, N, l, base, w, dev_status, q > 0 ? 1 : 2)) != MILO_OK) return s;
     for (int it = 0; it < q; ++it) {
-        if ((s = gemm(st, K, l, N, R, 1, K, Y, l, 1, Z, nullptr, l, dev_status)) != MILO_OK) return s;
-        if ((s = orth(st, Z, Z2, K, l, base, w, dev_status)) != MILO_OK) return s;
-        if ((s = gemm(st, N, l, K, R, K, 1, Z, l, 1, Y, nullptr, l, dev_status)) != MILO_OK) return s;
-        if ((s = orth(st, Y, Y2, N, l, base, w, dev_status)) != MILO_OK) return s;
+        if ((s = gemm(st, K, l, N, R, 1, K, Y, l, 1, Z, nullptr, l, dev_status, gpart)) != MILO_OK) return s;
+        if ((s = orth(st, Z, Z2, K, l, base, w, dev_status, 1)) != MILO_OK) return s;
+        if ((s = gemm(st, N, l, K, R, K, 1, Z, l, 1, Y, nullptr, l, dev_status, gpart)) != MILO_OK) return s;
+        if ((s = orth(st, Y, Y2, N, l, base, w, dev_status, it + 1 < q ? 1 : 2)) != MILO_OK) return s;
     }
-    if ((s = gemm(st, l, K, N, Y, 1, l, R, K, 1, Bm, nullptr, K, dev_status)) != MILO_OK) return s;
+    if ((s = gemm(st, l, K, N, Y, 1, l, R, K, 1, Bm, nullptr, K, dev_status, gpart)) != MILO_OK) return s;
     if ((s = gram(st, Bm, 1, K, K, l, reinterpret_cast<double*>(base + w.part), G)) != MILO_OK) return s;
     float* MU = reinterpret_cast<float*>(base + w.MU);
     float* MV = reinterpret_cast<float*>(base + w.MV);
-    jacobi_kernel<<<1, 256, square_smem(l), st>>>(G, l, r, reinterpret_cast<double*>(base + w.P), MU, MV);
+    jacobi_kernel<<<1, 256, jacobi_smem(l), st>>>(G, l, r, MU, MV);
     if ((s = check_launch("jacobi_kernel")) != MILO_OK) return s;
-    if ((s = gemm(st, N, r, l, Y, l, 1, MU, r, 1, nullptr, U, r, dev_status)) != MILO_OK) return s;
-    return gemm(st, r, K, l, MV, l, 1, Bm, K, 1, nullptr, V, K, dev_status);
+    if ((s = gemm(st, N, r, l, Y, l, 1, MU, r, 1, nullptr, U, r, dev_status, gpart)) != MILO_OK) return s;
+    return gemm(st, r, K, l, MV, l, 1, Bm, K, 1, nullptr, V, K, dev_status, gpart);
 }
 
 }  // namespace
@@ -677,7 +767,7 @@ extern "C" milo_status milo_hqq_pack(const uint16_t* W, const uint16_t* U, const
     if (rank > 0 && (!U || !V)) return fail(MILO_ERR_INVALID_ARG, "milo_hqq_pack: NULL U or V with rank > 0");
     if (!aligned(packed, 16) || !aligned(W, 2) || (residual && !aligned(residual, 4)))
         return fail(MILO_ERR_INVALID_ARG, "milo_hqq_pack: misaligned buffer (packed needs 16 bytes)");
-    const HqqArgs a{W, rank > 0 ? U : nullptr, rank > 0 ? V : nullptr, static_cast<uint8_t*>(packed), residual,
+    const HqqArgs a{W, rank > 0 ? U : nullptr, rank > 0 ? V : nullptr, nullptr, static_cast<uint8_t*>(packed), residual,
                     dev_status, N, K, rank, hqq_iters, hqq_beta, hqq_kappa};
     return launch_hqq(a, static_cast<cudaStream_t>(stream));
 }
@@ -719,18 +809,20 @@ extern "C" milo_status milo_quantize_lorc(const uint16_t* W, int32_t N, int32_t 
     if (!W || !packed || !ws) return fail(MILO_ERR_INVALID_ARG, "milo_quantize_lorc: NULL W, packed or ws");
     if (r > 0 && (!omega || !U || !V))
         return fail(MILO_ERR_INVALID_ARG, "milo_quantize_lorc: NULL omega, U or V with rank > 0");
-    if (!aligned(packed, 16) || !aligned(ws, 256) || !aligned(W, 2) || (r > 0 && (!aligned(U, 16) ||
+    if (!aligned(packed, 16) || !aligned(ws, 256) || !aligned(W, 8) || (r > 0 && (!aligned(U, 16) ||
         !aligned(V, 16) || !aligned(omega, 4))) || (err && !aligned(err, 4)))
-        return fail(MILO_ERR_INVALID_ARG, "milo_quantize_lorc: misaligned buffer (packed, U, V need 16 bytes, ws 256)");
+        return fail(MILO_ERR_INVALID_ARG,
+                    "milo_quantize_lorc: misaligned buffer (W needs 8 bytes, packed, U, V 16, ws 256)");
     const QuantWs w = quant_layout(N, K, p);
     if (ws_bytes < w.total) return fail(MILO_ERR_WORKSPACE, "milo_quantize_lorc: workspace too small");
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (r > 0) {
-        const int smem = static_cast<int>(square_smem(w.l));
-        if ((s = check_cuda(cudaFuncSetAttribute(chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+        if ((s = check_cuda(cudaFuncSetAttribute(chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(chol_smem(w.l))),
                             "chol_kernel attribute")) != MILO_OK)
             return s;
-        if ((s = check_cuda(cudaFuncSetAttribute(jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+        if ((s = check_cuda(cudaFuncSetAttribute(jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(jacobi_smem(w.l))),
                             "jacobi_kernel attribute")) != MILO_OK)
             return s;
     }
@@ -743,13 +835,16 @@ extern "C" milo_status milo_quantize_lorc(const uint16_t* W, int32_t N, int32_t 
     int* improved = reinterpret_cast<int*>(base + w.flag);
     const size_t blob_bytes = static_cast<size_t>((N + 63) / 64) * (K / 128) * kBlockSB;
     const int rounds = r > 0 ? p.rounds : 0;
+    float* T = p.rounds > 0 && r > 0 ? reinterpret_cast<float*>(base + w.T) : nullptr;
     for (int t = 0; t <= rounds; ++t) {
-        const HqqArgs h{W, t > 0 ? Uw : nullptr, t > 0 ? Vw : nullptr, blob, R, dev_status, N, K, t > 0 ? r : 0,
-                        p.hqq_iters, p.hqq_beta, p.hqq_kappa};
+        // round t quantises W (t = 0) or the target W - U V formed by the last round
+        const HqqArgs h{W, nullptr, nullptr, t > 0 ? T : nullptr, blob, R, dev_status, N, K, 0, p.hqq_iters,
+                        p.hqq_beta, p.hqq_kappa};
         if ((s = launch_hqq(h, st)) != MILO_OK) return s;
         if (r > 0 && (s = compensator(st, R, omega, N, K, r, p.power_iters, base, w, Uw, Vw, dev_status)) != MILO_OK)
             return s;
-        err_kernel<<<w.eblocks, 256, 0, st>>>(R, Uw, Vw, N, K, r, reinterpret_cast<double*>(base + w.epart));
+        apply_kernel<<<w.eblocks, kApplyThreads, 0, st>>>(R, W, Uw, Vw, N, K, r, t < rounds ? T : nullptr,
+                                                          reinterpret_cast<double*>(base + w.epart));
         err_sum_kernel<<<1, 256, 0, st>>>(reinterpret_cast<double*>(base + w.epart), w.eblocks, t, err, best,
                                           improved);
         copy_best_kernel<<<296, 256, 0, st>>>(improved, reinterpret_cast<const uint4*>(blob),

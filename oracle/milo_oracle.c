@@ -280,10 +280,10 @@ void milo_ref_dequant(const uint8_t* q, const uint16_t* scale, const uint16_t* z
  * an optimisation problem.  The pages give no more detail; HQQ as published
  * (Badri and Shaji, 2023) keeps the min/max scale and fits the zero point z of
  * each group by half-quadratic splitting of an lp error (p < 1):
- *     q      = clamp(rint(t / s + z), 0, 7)
+ *     q      = clamp(rint(t * (1/s) + z), 0, 7)
  *     e      = t - (q - z) s                     the group's error
  *     w_e    = shrink(e)                          proximal step on |.|^p
- *     z_next = mean(q - (t - w_e) / s)            least-squares zero given w_e
+ *     z_next = mean(q - (t - w_e) * (1/s))        least-squares zero given w_e
  *     beta   = kappa * beta
  * with shrink(e) = sign(e) max(|e| - |e|^(p-1) / beta, 0).
  *
@@ -292,7 +292,8 @@ void milo_ref_dequant(const uint8_t* q, const uint16_t* scale, const uint16_t* z
  *     square root and division (HQQ's own default is p = 0.7);
  *   - every step is fp32, in the order written here (no fused multiply-add),
  *     sums run over the group's 64 values in index order; quantised codes are
- *     decided in fp32 on both sides;
+ *     decided in fp32 on both sides; inside the iterations the target is
+ *     multiplied by the fp32 inverse 1/s, as HQQ's quantisation step does;
  *   - HQQ stops when its error stops falling; here each group keeps the zero
  *     point whose L1 error sum_i |e_i| was lowest over the iterations (the
  *     error of a group depends only on its own zero point), first one on ties;
@@ -319,13 +320,14 @@ static int hqq_group(const float* t, int iters, float beta0, float kappa, uint8_
     if ((s_h & 0x7FFF) == 0) s_h = 0x3C00;
     float s = h2f(s_h);
     float z = -mn / s;
+    float inv = 1.0f / s;                     /* HQQ quantises with the inverse scale */
     float beta = beta0;
     float best_err = INFINITY, best_z = z;
     if (z_trace) z_trace[0] = z;
     for (int it = 0; it < iters; ++it) {
         float err = 0.0f, acc = 0.0f;
         for (int i = 0; i < 64; ++i) {
-            float v = t[i] / s;
+            float v = t[i] * inv;
             v = v + z;
             float r = nearbyintf(v);
             if (!(r >= 0.0f)) r = 0.0f;
@@ -343,7 +345,7 @@ static int hqq_group(const float* t, int iters, float beta0, float kappa, uint8_
                 if (m > 0.0f) w_e = e < 0.0f ? -m : m;
             }
             float u = t[i] - w_e;
-            u = u / s;
+            u = u * inv;
             acc = acc + (r - u);
         }
         if (err_trace) err_trace[it] = err;
