@@ -717,9 +717,22 @@ def run_quantize(args):
                         None, sp)
         b.record()
         hq.append((a, b))
+    # the kurtosis reduction of the adaptive-rank policy, on w1 (HBM-bound)
+    kws = torch.empty(4 * 592, dtype=torch.float64, device=dev)
+    kout = torch.empty(1, dtype=torch.float64, device=dev)
+    kt = []
+    for _ in range(max(3, min(args.steps, 20))):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        L.milo_kurtosis(C.c_void_p(W1.data_ptr()), N1 * K1, C.c_void_p(kout.data_ptr()), C.c_void_p(kws.data_ptr()),
+                        kws.numel() * 8, None, sp)
+        b.record()
+        kt.append((a, b))
     torch.cuda.synchronize()
     clocks = clock.stop()
     hqq_ms = statistics.median(a.elapsed_time(b) for a, b in hq[1:])
+    kurt_ms = statistics.median(a.elapsed_time(b) for a, b in kt[1:])
+    kurt_gbs = 2.0 * N1 * K1 / (kurt_ms / 1e3) / 1e9
     weights = sum(j[0] * j[1] for j in jobs)
     sm_mhz = clocks.get("sm_mhz") or 1965.0
     peak = FP32_LANES * sm_mhz * 1e6 / 1e12
@@ -738,6 +751,8 @@ def run_quantize(args):
                      "algorithmic_ops_per_launch": HQQ_OPS_PER_WEIGHT_ITER * N1 * K1 * params.hqq_iters,
                      "ms_per_launch": hqq_ms,
                      "peak_source": "derived: 148 SMs x 128 fp32 lanes x the sampled SM clock"},
+        "kernels": {"hqq_pack_ms": hqq_ms, "kurtosis_ms": kurt_ms, "kurtosis_gbs": kurt_gbs,
+                    "kurtosis_frac_hbm": kurt_gbs / peaks()["hbm_gbs"]},
         "gpu_launches": None, "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

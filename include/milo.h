@@ -222,6 +222,47 @@ MILO_API milo_status milo_quantize_lorc(const uint16_t* W, int32_t N, int32_t K,
                                         size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Adaptive compensator ranks                                               */
+/* ------------------------------------------------------------------------ */
+/*
+ * "MiLo Algorithm: Mixture of Low-Rank Compensators", adaptive rank
+ * selection: a higher rank for weights with a higher kurtosis (strategy 3)
+ * and for experts activated more often (strategy 2).
+ */
+
+/* Workspace bytes of milo_kurtosis (the same for every size). */
+MILO_API milo_status milo_kurtosis_workspace(size_t* bytes);
+
+/*
+ * milo_kurtosis -- Pearson kurtosis m4 / m2^2 (not the excess; a normal
+ * distribution gives 3) of the `count` fp16 entries at W (device, 16-byte
+ * aligned), from fp64 sums of w, w^2, w^3, w^4 over a fixed grid, written to
+ * out[0] (device fp64).  A constant matrix gives 0.  Deterministic.  Device:
+ * NONFINITE for NaN/Inf entries.  ws: milo_kurtosis_workspace bytes, 8-byte
+ * aligned.
+ */
+MILO_API milo_status milo_kurtosis(const uint16_t* W, int64_t count, double* out, void* ws, size_t ws_bytes,
+                                   int32_t* dev_status, void* stream);
+
+/*
+ * milo_assign_ranks -- split a rank budget over n matrices by score (host
+ * arrays; a kurtosis, an activation frequency, ...).  Ranks are multiples of
+ * 8 in 0..max_rank (max_rank a multiple of 8, at most 64) and add up to at most
+ * n * avg_rank: the budget, in units of 8, is shared in proportion to the
+ * scores (negative scores count as 0; when no remaining score is positive the
+ * rest is shared equally); a share that reaches the cap is fixed there and the
+ * rest re-shared among the others; each matrix then takes the floor of its
+ * share and the leftover units go one at a time in decreasing order of the
+ * fractional part (ties: higher score, then lower index), pass after pass
+ * until the budget (capped at n * max_rank) is used.  A higher score never
+ * gets a lower rank.  Errors: n <= 0,
+ * NULL pointers, non-finite scores, max_rank not a multiple of 8 in 0..64,
+ * avg_rank < 0 -> INVALID_ARG.
+ */
+MILO_API milo_status milo_assign_ranks(const double* score, int32_t n, int32_t avg_rank, int32_t max_rank,
+                                       int32_t* ranks);
+
+/* ------------------------------------------------------------------------ */
 /* Routing                                                                  */
 /* ------------------------------------------------------------------------ */
 /*

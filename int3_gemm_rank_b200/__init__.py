@@ -33,7 +33,8 @@ EXPORTS = ("milo_status_str", "milo_last_error", "milo_version", "milo_pack", "m
            "milo_linear_workspace_bytes", "milo_moe_workspace_bytes", "milo_grouped_linear",
            "milo_moe_forward", "milo_moe_h_offset", "milo_set_profile_events",
            "milo_grouped_linear_noalloc", "milo_packed_bytes", "milo_hqq_pack",
-           "milo_quantize_lorc_workspace", "milo_quantize_lorc")
+           "milo_quantize_lorc_workspace", "milo_quantize_lorc", "milo_kurtosis_workspace", "milo_kurtosis",
+           "milo_assign_ranks")
 
 
 class MiloError(RuntimeError):
@@ -119,6 +120,10 @@ def lib() -> C.CDLL:
         L.milo_quantize_lorc.argtypes = [vp, i32, i32, C.POINTER(milo_lorc_params), vp, vp, vp, vp, vp, vp, sz,
                                          vp, vp]
         L.milo_quantize_lorc.restype = C.c_int
+        L.milo_kurtosis_workspace.argtypes = [C.POINTER(sz)]; L.milo_kurtosis_workspace.restype = C.c_int
+        L.milo_kurtosis.argtypes = [vp, C.c_int64, vp, vp, sz, vp, vp]; L.milo_kurtosis.restype = C.c_int
+        L.milo_assign_ranks.argtypes = [C.POINTER(C.c_double), i32, i32, i32, C.POINTER(i32)]
+        L.milo_assign_ranks.restype = C.c_int
         _lib = L
     return _lib
 
@@ -254,6 +259,29 @@ def milo_quantize_lorc(W: torch.Tensor, params: milo_lorc_params, omega: torch.T
                                     _ptr(err), C.c_void_p(wp), ws_bytes, _ptr(dev_status), _stream()),
            "milo_quantize_lorc")
     return QWeight(blob, N, K, U, V, rank=r), err
+
+
+def milo_kurtosis(W: torch.Tensor, dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """Pearson kurtosis of all entries of an fp16 CUDA tensor: a device fp64 scalar tensor."""
+    _cuda(W, "W")
+    if W.dtype != torch.float16:
+        raise ValueError("W must be float16")
+    nb = C.c_size_t()
+    _check(lib().milo_kurtosis_workspace(C.byref(nb)), "milo_kurtosis_workspace")
+    ws = torch.empty(nb.value // 8, dtype=torch.float64, device=W.device)
+    out = torch.empty(1, dtype=torch.float64, device=W.device)
+    _check(lib().milo_kurtosis(_ptr(W), W.numel(), _ptr(out), _ptr(ws), nb.value, _ptr(dev_status), _stream()),
+           "milo_kurtosis")
+    return out
+
+
+def milo_assign_ranks(scores, avg_rank: int, max_rank: int = MILO_MAX_RANK) -> list:
+    """Ranks (multiples of 8) for matrices with the given scores, within n * avg_rank in total."""
+    n = len(scores)
+    sc = (C.c_double * max(n, 1))(*[float(x) for x in scores])
+    out = (C.c_int32 * max(n, 1))()
+    _check(lib().milo_assign_ranks(sc, n, int(avg_rank), int(max_rank), out), "milo_assign_ranks")
+    return [int(out[i]) for i in range(n)]
 
 
 # ---------------------------------------------------------------------------

@@ -387,3 +387,74 @@ def quantize_lorc(W_bits: np.ndarray, rank: int, rounds: int, omega: np.ndarray,
             break
     return dict(q=best["q"], scale=best["scale"], zero=best["zero"], U=best["U"], V=best["V"],
                 err=np.array(errs), best=best["round"], status=status)
+
+
+# ---------------------------------------------------------------------------
+# Adaptive ranks ("MiLo Algorithm: Mixture of Low-Rank Compensators": a higher
+# rank for weights with a higher kurtosis, and for experts activated more often).
+
+def kurtosis(W_bits: np.ndarray) -> float:
+    """Pearson kurtosis m4 / m2^2 of all entries (fp64, centred moments); 0 for a constant matrix."""
+    w = _f16(W_bits).astype(np.float64).ravel()
+    d = w - w.mean()
+    m2 = float(np.mean(d * d))
+    return float(np.mean(d ** 4)) / (m2 * m2) if m2 > 0 else 0.0
+
+
+def assign_ranks(scores, avg_rank: int, max_rank: int = 64) -> list:
+    """Budget floor(n * avg_rank / 8) units of 8, capped at max_rank / 8 each:
+    shares proportional to max(score, 0) (no positive score left -> equal),
+    shares reaching the cap fixed there and the rest re-shared, floors, then the
+    leftover units one at a time by decreasing fractional part (ties: higher
+    score, lower index), pass after pass until used or all capped."""
+    n = len(scores)
+    cap = max_rank // 8
+    units = min(n * avg_rank // 8, cap * n)
+    s = [max(float(x), 0.0) for x in scores]
+    if not sum(s) > 0.0:
+        s = [1.0] * n
+    share = [0.0] * n
+    fixed = [False] * n
+    eff = list(s)
+    left = float(units)
+    while True:
+        active = 0.0
+        for i in range(n):
+            if not fixed[i]:
+                active += eff[i]
+        if not active > 0.0:          # only zero scores left: share the rest equally
+            for i in range(n):
+                if not fixed[i]:
+                    eff[i] = 1.0
+            active = 0.0
+            for i in range(n):
+                if not fixed[i]:
+                    active += eff[i]
+        changed = False
+        for i in range(n):
+            if fixed[i]:
+                continue
+            share[i] = left * eff[i] / active if active > 0.0 else 0.0
+            if share[i] >= cap:
+                share[i] = float(cap)
+                fixed[i] = True
+                left -= float(cap)
+                changed = True
+        if not changed:
+            break
+    u = [min(cap, int(np.floor(x))) for x in share]
+    used = sum(u)
+    frac = [x - np.floor(x) for x in share]
+    order = sorted(range(n), key=lambda i: (-frac[i], -s[i], i))
+    while used < units:               # passes until the budget is used or all are capped
+        took = False
+        for i in order:
+            if used >= units:
+                break
+            if u[i] < cap:
+                u[i] += 1
+                used += 1
+                took = True
+        if not took:
+            break
+    return [8 * x for x in u]
