@@ -28,40 +28,58 @@ namespace {
 constexpr int kKurtBlocks = 592;      // 4 blocks per SM on 148 SMs, fixed
 constexpr int kKurtThreads = 256;
 
-// Block b sums w, w^2, w^3, w^4 over the entries i = 8 (b * 256 + t) + j of a
-// grid-stride walk (8 fp16 per 16-byte load), in that order per thread, then
-// over the block in a fixed tree.
+// Thread (b, t) sums w, w^2, w^3, w^4 over the 8-entry pieces i = 8 (b * 256 +
+// t) + 8 * 592 * 256 * k, k = 0, 1, ... (16-byte loads, four issued before
+// their arithmetic so that enough bytes are in flight), in increasing k; then
+// the block adds its threads in a fixed tree.
+constexpr int kKurtUnroll = 4;
+
+__device__ __forceinline__ void kurt_piece(const uint16_t* __restrict__ W, long long i, long long count,
+                                           uint16_t (&v)[8]) {
+    if (i + 8 <= count) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(W + i));
+        const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[2 * j] = static_cast<uint16_t>(w4[j] & 0xFFFFu);
+            v[2 * j + 1] = static_cast<uint16_t>(w4[j] >> 16);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = i + j < count ? W[i + j] : 0;   // +0 adds nothing
+    }
+}
+
 __global__ void __launch_bounds__(kKurtThreads) kurt_partial_kernel(const uint16_t* __restrict__ W, long long count,
                                                                     double* __restrict__ part,
                                                                     int32_t* __restrict__ dev_status) {
     __shared__ double red[4][kKurtThreads];
     double s1 = 0.0, s2 = 0.0, s3 = 0.0, s4 = 0.0;
     int32_t st = 0;
-    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x * 8;
-    for (long long i = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8; i < count; i += stride) {
-        uint16_t v[8];
-        if (i + 8 <= count) {
-            const uint4 q = *reinterpret_cast<const uint4*>(W + i);
-            const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+    const long long piece = static_cast<long long>(gridDim.x) * blockDim.x * 8;
+    for (long long i0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8; i0 < count;
+         i0 += kKurtUnroll * piece) {
+        uint16_t v[kKurtUnroll][8];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                v[2 * j] = static_cast<uint16_t>(w4[j] & 0xFFFFu);
-                v[2 * j + 1] = static_cast<uint16_t>(w4[j] >> 16);
+        for (int u = 0; u < kKurtUnroll; ++u) {
+            const long long i = i0 + u * piece;
+            if (i < count) kurt_piece(W, i, count, v[u]);
+            else
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[u][j] = 0;
+        }
+#pragma unroll
+        for (int u = 0; u < kKurtUnroll; ++u)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const double x = static_cast<double>(__half2float(__ushort_as_half(v[u][j])));
+                if (!isfinite(x)) st |= MILO_DEV_NONFINITE;
+                const double x2 = x * x;
+                s1 += x;
+                s2 += x2;
+                s3 += x2 * x;
+                s4 += x2 * x2;
             }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = i + j < count ? W[i + j] : 0;   // +0 adds nothing
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const double x = static_cast<double>(__half2float(__ushort_as_half(v[j])));
-            if (!isfinite(x)) st |= MILO_DEV_NONFINITE;
-            const double x2 = x * x;
-            s1 += x;
-            s2 += x2;
-            s3 += x2 * x;
-            s4 += x2 * x2;
-        }
     }
     red[0][threadIdx.x] = s1;
     red[1][threadIdx.x] = s2;
