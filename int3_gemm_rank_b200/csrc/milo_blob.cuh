@@ -44,6 +44,21 @@ __device__ __forceinline__ void place_codes(const uint8_t (&q)[128], uint32_t (&
     }
 }
 
+// The same placement one code at a time: code q at super-block position k
+// (0..127) ORed into the zero-initialised words (k a compile-time constant
+// after unrolling keeps the words in registers).
+__device__ __forceinline__ void place_code(uint32_t (&words)[12], int k, uint32_t q) {
+    const int c = (k & 63) >> 4, m = (k & 15) + ((k >> 6) << 4);   // unit, unit code (unit_k inverted)
+    if (m < 30) {
+        const int t = m / 10, r = m % 10;
+        words[3 * c + t] |= q << (16 * (r & 1) + 3 * (r >> 1));
+    } else {
+        const int bit = m == 30 ? 15 : 31;
+#pragma unroll
+        for (int t = 0; t < 3; ++t) words[3 * c + t] |= ((q >> t) & 1u) << bit;
+    }
+}
+
 // Zero words, scales and zeros for a padding row n >= N of the last tile.
 __device__ __forceinline__ void blob_zero_row(uint8_t* blob, int n, int b, int SB) {
     uint4* dst = reinterpret_cast<uint4*>(blob + blob_words(n, b, SB));

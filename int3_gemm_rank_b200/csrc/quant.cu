@@ -105,7 +105,7 @@ __device__ __forceinline__ int32_t hqq_group(const float (&t)[64], int iters, fl
     return st;
 }
 
-__global__ void __launch_bounds__(128) hqq_pack_kernel(const HqqArgs a) {
+__global__ void __launch_bounds__(128, 4) hqq_pack_kernel(const HqqArgs a) {
     const int SB = a.K / 128;
     const int Npad = (a.N + 63) / 64 * 64;
     const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -117,8 +117,10 @@ __global__ void __launch_bounds__(128) hqq_pack_kernel(const HqqArgs a) {
         return;
     }
     int32_t st = 0;
-    uint8_t q[128];
-#pragma unroll 1
+    uint32_t words[12];
+#pragma unroll
+    for (int i = 0; i < 12; ++i) words[i] = 0u;
+#pragma unroll
     for (int g = 0; g < 2; ++g) {
         const size_t k0 = static_cast<size_t>(n) * a.K + 128 * b + 64 * g;
         float t[64];
@@ -150,12 +152,10 @@ __global__ void __launch_bounds__(128) hqq_pack_kernel(const HqqArgs a) {
             float r = rintf(__fadd_rn(__fdiv_rn(t[i], s), z));
             if (!(r >= 0.0f)) r = 0.0f;
             if (r > 7.0f) r = 7.0f;
-            q[64 * g + i] = static_cast<uint8_t>(r);
+            place_code(words, 64 * g + i, static_cast<uint32_t>(r));
             if (a.resid) a.resid[k0 + i] = __fsub_rn(f16v(a.W[k0 + i]), __fmul_rn(__fsub_rn(r, z), s));
         }
     }
-    uint32_t words[12];
-    place_codes(q, words);
     blob_store_words(a.blob, n, b, SB, words);
     flag(a.dev_status, st);
 }
@@ -178,34 +178,41 @@ struct GemmArgs {
     int kslice;              // reduction length per slice (multiple of kGK)
 };
 
-constexpr int kGT = 64;      // output tile
+constexpr int kGT = 64;      // output tile width (and the height of the small tile)
 constexpr int kGK = 16;      // reduction slice per shared-memory stage
 
-// C = A B over the full reduction in index order per 16-wide slice.  Tile
-// loads walk the operand's contiguous dimension across threads.
+// C = A B over the reduction in index order per 16-wide slice, TM x 64 output
+// tiles (TM = 128: 8 x 4 outputs per thread; 64: 4 x 4).  Tile loads walk the
+// operand's contiguous dimension across threads.
+template <int TM>
 __global__ void __launch_bounds__(256) sgemm_kernel(const GemmArgs a) {
-    __shared__ __align__(16) float As[kGK][kGT + 4];
+    constexpr int RM = TM / 16;          // output rows per thread
+    __shared__ __align__(16) float As[kGK][TM + 4];
     __shared__ __align__(16) float Bs[kGK][kGT + 4];
     const int tid = threadIdx.x;
-    const int m0 = blockIdx.y * kGT, n0 = blockIdx.x * kGT;
-    const int tm = (tid / 16) * 4, tn = (tid % 16) * 4;
-    float acc[4][4];
+    const int m0 = blockIdx.y * TM, n0 = blockIdx.x * kGT;
+    const int tm = (tid / 16) * RM, tn = (tid % 16) * 4;
+    float acc[RM][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < RM; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
     const int kbeg = blockIdx.z * a.kslice;
     const int kend = min(a.Kd, kbeg + a.kslice);
     for (int k0 = kbeg; k0 < kend; k0 += kGK) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < RM; ++i) {               // A: TM x 16 values, RM per thread
             const int idx = tid + 256 * i;
             int mm, kk;
             if (a.sak == 1) { kk = idx % kGK; mm = idx / kGK; }
-            else { mm = idx % kGT; kk = idx / kGT; }
+            else { mm = idx % TM; kk = idx / TM; }
             const int m = m0 + mm, k = k0 + kk;
             As[kk][mm] = (m < a.M && k < kend) ? a.A[m * a.sam + k * a.sak] : 0.0f;
-            int nn;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {                // B: 16 x 64 values, 4 per thread
+            const int idx = tid + 256 * i;
+            int kk, nn;
             if (a.sbn == 1) { nn = idx % kGT; kk = idx / kGT; }
             else { kk = idx % kGK; nn = idx / kGK; }
             const int n = n0 + nn, kb = k0 + kk;
@@ -214,11 +221,16 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const GemmArgs a) {
         __syncthreads();
 #pragma unroll
         for (int kk = 0; kk < kGK; ++kk) {
-            const float4 av = *reinterpret_cast<const float4*>(&As[kk][tm]);
-            const float4 bv = *reinterpret_cast<const float4*>(&Bs[kk][tn]);
-            const float ar[4] = {av.x, av.y, av.z, av.w}, br[4] = {bv.x, bv.y, bv.z, bv.w};
+            float ar[RM];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int h = 0; h < RM / 4; ++h) {
+                const float4 av = *reinterpret_cast<const float4*>(&As[kk][tm + 4 * h]);
+                ar[4 * h] = av.x; ar[4 * h + 1] = av.y; ar[4 * h + 2] = av.z; ar[4 * h + 3] = av.w;
+            }
+            const float4 bv = *reinterpret_cast<const float4*>(&Bs[kk][tn]);
+            const float br[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+            for (int i = 0; i < RM; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(ar[i], br[j], acc[i][j]);
         }
@@ -226,7 +238,7 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const GemmArgs a) {
     }
     int32_t st = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < RM; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int m = m0 + tm + i, n = n0 + tn + j;
@@ -603,7 +615,7 @@ constexpr int kGramChunk = 64;    // rows per Gram partial
 // Split reductions: a product whose output tiles fill fewer than 148 blocks and
 // whose reduction is long splits it into S slices (S x blocks <= 296) summed in
 // slice order by split_sum_kernel, so the partials fit kSplitFloats.
-constexpr int kSplitFloats = 296 * kGT * kGT;
+constexpr int kSplitFloats = 296 * 2 * kGT * kGT;   // S x (blocks of up to 128 x 64) <= 296 x 8192
 
 struct QuantWs {
     size_t R, T, Y, Y2, Z, Z2, B, part, gpart, G, M, MU, MV, U, V, blob, epart, best, flag, total;
@@ -670,13 +682,16 @@ milo_status launch_hqq(const HqqArgs& a, cudaStream_t st) {
 milo_status gemm(cudaStream_t st, int M, int Nn, int Kd, const float* A, long long sam, long long sak, const float* B,
                  long long sbk, long long sbn, float* C, uint16_t* C16, long long ldc, int32_t* dev_status,
                  float* gpart) {
-    const int gx = (Nn + kGT - 1) / kGT, gy = (M + kGT - 1) / kGT;
+    const bool tall = M >= 2 * kGT;                  // 128-row tiles when the output is tall
+    const int TM = tall ? 2 * kGT : kGT;
+    const int gx = (Nn + kGT - 1) / kGT, gy = (M + TM - 1) / TM;
     int S = 1;
     if (gpart && gx * gy < 148 && Kd >= 2048) S = std::min(8, std::max(1, 296 / (gx * gy)));
     const int kslice = static_cast<int>(round_up((Kd + S - 1) / S, kGK));
     S = (Kd + kslice - 1) / kslice;
     const GemmArgs a{M, Nn, Kd, A, sam, sak, B, sbk, sbn, C, C16, ldc, dev_status, S > 1 ? gpart : nullptr, kslice};
-    sgemm_kernel<<<dim3(gx, gy, S), 256, 0, st>>>(a);
+    if (tall) sgemm_kernel<2 * kGT><<<dim3(gx, gy, S), 256, 0, st>>>(a);
+    else sgemm_kernel<kGT><<<dim3(gx, gy, S), 256, 0, st>>>(a);
     if (S > 1) {
         const long long e = static_cast<long long>(M) * Nn;
         split_sum_kernel<<<static_cast<unsigned>((e + 255) / 256), 256, 0, st>>>(gpart, S, M, Nn, C, C16, ldc,
