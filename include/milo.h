@@ -67,7 +67,7 @@ typedef enum {
 #define MILO_ROUTE_RENORM 0x1u      /* renormalise the softmax over the k picked experts */
 #define MILO_ROUTE_IDS_GIVEN 0x2u   /* topk_ids are inputs (logits NULL, topk_w untouched) */
 
-/* Limits of this build. */
+/* Compile-time limits of the library. */
 #define MILO_GROUP 64               /* scale/zero group along K */
 #define MILO_MAX_RANK 64            /* compensator rank, a multiple of 8 */
 #define MILO_MAX_EXPERTS 256        /* routed + shared */
@@ -111,7 +111,8 @@ MILO_API milo_status milo_packed_bytes(int32_t N, int32_t K, size_t* bytes);
 /*
  * milo_pack -- quantise W fp16 [N, K] (row-major) to int3 and pack it.
  * Round-to-nearest asymmetric min/max per group of 64 along K (the paper's HQQ
- * initialiser is replaced by RTN for synthetic weights):
+ * initialisation is milo_hqq_pack / milo_quantize_lorc; with one iteration HQQ
+ * gives exactly this):
  *     s = fp16((max - min) / 7)   (s := 1 when it rounds to 0)
  *     z = fp16(-min / s)
  *     q = clamp(rint(w / s + z), 0, 7)    (fp32, ties to even, no FMA)

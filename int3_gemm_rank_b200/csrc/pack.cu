@@ -3,8 +3,8 @@
 // "MiLo: Efficient Quantized MoE Inference with Mixture of Low-Rank
 // Compensators", section "MiLo Kernel: Efficient Int3 Quantized GEMM Backend":
 // 32 three-bit values per three 32-bit words, no wasted bit, asymmetric
-// dequantisation with a zero point.  The quantiser is round-to-nearest
-// asymmetric min/max (the paper starts from HQQ; synthetic weights use RTN).
+// dequantisation with a zero point.  The quantiser here is round-to-nearest
+// asymmetric min/max; the paper's HQQ initialisation is in quant.cu.
 #include <cuda_runtime.h>
 
 #include "milo_blob.cuh"

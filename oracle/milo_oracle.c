@@ -25,8 +25,8 @@
  * Readings taken where the pages are silent (each also listed with the
  * design notes of the repository):
  *   - quantiser: round-to-nearest asymmetric min/max per group of 64 along K
- *     (the paper initialises with HQQ; plain RTN is used for synthetic
- *     weights); s = fp16(range / 7), z = fp16(-min / s), q = clamp(rint(w/s + z));
+ *     (milo_ref_quantize; the paper's HQQ initialisation is milo_ref_hqq
+ *     below); s = fp16(range / 7), z = fp16(-min / s), q = clamp(rint(w/s + z));
  *   - dequantisation: w_hat = (q - z) * s with fp16 s and z, z not rounded to
  *     an integer;
  *   - the packing layout (the page's description of the three-word packing is
