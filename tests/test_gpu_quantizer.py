@@ -227,3 +227,49 @@ def test_quantized_weight_runs_in_the_grouped_linear(milo):
     y = lin(f16_dev(X), route["offsets"], route["perm"], k=1).cpu().numpy()
     y_ref = oracle.linear(wl.f16_bits_to_f32(X).astype(np.float64), P)
     assert rel_err(y, y_ref) <= REL_TOL
+
+
+def test_quantize_lorc_full_size_mixtral_w1(milo):
+    """The Mixtral-shaped w1 (14336 x 4096), rank 32, one round: HQQ codes,
+    scales and zeros bit-exact on sampled rows (rows are quantised
+    independently), the fp32 residual bit-exact on those rows, and U V
+    against the oracle's fp64 subspace iteration on the full residual."""
+    rng = np.random.default_rng(59)
+    N, K, r = 14336, 4096, 32
+    W = wl.gen_weight(rng, N, K)
+    om = rng.standard_normal((K, 2 * r)).astype(np.float32)
+    qw, err = _quantize(milo, W, r, 0, om)
+    _, R_gpu = milo.milo_hqq_pack(f16_dev(W), residual=True)
+    R_gpu = R_gpu.cpu().numpy()
+    rows = np.sort(rng.choice(N, size=96, replace=False))
+    q, s, z, _ = oracle.hqq(oracle._f16(W[rows]))
+    qg, sg, zg = _unblob_rows(qw.packed.cpu().numpy(), rows, K)
+    assert np.array_equal(qg, q) and np.array_equal(sg, s) and np.array_equal(zg, z)
+    assert np.array_equal(R_gpu[rows].view(np.uint32), oracle.residual(W[rows], q, s, z).view(np.uint32))
+    U, V = oracle.rsvd(R_gpu, r, om, 2)
+    Ug = _f16(qw.U.cpu().numpy().view(np.uint16))
+    Vg = _f16(qw.V.cpu().numpy().view(np.uint16))
+    ref = U[rows] @ V
+    assert np.linalg.norm(Ug[rows] @ Vg - ref) <= UV_TOL * np.linalg.norm(ref)
+    E = R_gpu.astype(np.float64) - Ug @ Vg
+    assert abs(err[0] - np.linalg.norm(E)) <= 1e-5 * err[0]
+
+
+def _unblob_rows(blob, rows, K):
+    """Codes [len(rows), K] and scales, zeros [K/64, len(rows)] of the given rows of a blob."""
+    SB = K // 128
+    q = np.zeros((len(rows), K), np.uint8)
+    s = np.zeros((K // 64, len(rows)), np.uint16)
+    z = np.zeros((K // 64, len(rows)), np.uint16)
+    for i, n in enumerate(rows):
+        t, rr = divmod(int(n), 64)
+        for b in range(SB):
+            base = (t * SB + b) * 3584
+            words = blob[base: base + 3072].view(np.uint32).reshape(64, 12)[rr]
+            q[i, 128 * b: 128 * b + 128] = oracle.unpack(words.reshape(1, 12), 128)[0]
+            groups = blob[base + 3072: base + 3584].view(np.uint16)
+            for h in range(2):
+                o = h * 128 + ((rr // 16) * 8 + rr % 8) * 4 + ((rr % 16) // 8) * 2
+                s[2 * b + h, i] = groups[o]
+                z[2 * b + h, i] = groups[o + 1]
+    return q, s, z
