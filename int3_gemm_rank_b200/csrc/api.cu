@@ -575,7 +575,7 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
 
     PrepParams ph{reinterpret_cast<const uint16_t*>(base + w.h), nullptr,
                   reinterpret_cast<uint16_t*>(base + w.hfrag), reinterpret_cast<uint16_t*>(base + w.hg), tc ? 1 : 0,
-                  dev_status, w.R, I, 0, 0, nullptr, nullptr, nullptr, nullptr, 0, 0, 0, 0, 0};
+                  dev_status, w.R, I, 0, 0, nullptr, nullptr, nullptr, nullptr, 0, 0, 0, 0, 0, nullptr, 0};
     if ((s = check_cuda(launch_prep(ph, st), "prep h")) != MILO_OK) return s;
     if (has_t) {
         LorcParams lp{reinterpret_cast<const uint16_t*>(base + w.h), nullptr, table, grp,
