@@ -165,7 +165,8 @@ MILO_API milo_status milo_unpack(const void* packed, int32_t N, int32_t K, uint8
  *   residual: NULL, or f32 [N, K] receiving W - (q - z) s (fp32: the
  *   difference q - z, the product, then W minus it), the residual a
  *   compensator approximates.
- * Errors: K % 128 != 0, rank > 64 -> UNSUPPORTED_SHAPE; N, K <= 0, rank < 0,
+ * Errors: K % 128 != 0, rank > 64, N or K above 2^22 or N * K above 2^34 ->
+ * UNSUPPORTED_SHAPE; N, K <= 0, rank < 0,
  * hqq_iters outside 0..1000, beta or kappa not finite and positive, NULL W or
  * packed, U or V NULL with rank > 0 -> INVALID_ARG.  Device: NONFINITE for
  * NaN/Inf targets, FP16_RANGE when s or z overflows fp16.  All pointers are

@@ -664,7 +664,8 @@ milo_status check_hqq(int N, int K, int rank, int iters, float beta, float kappa
     const std::string f = who;
     if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, f + ": N and K must be positive");
     if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": K must be a multiple of 128");
-    if (N > (1 << 22)) return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": N above 4194304");
+    if (N > (1 << 22) || K > (1 << 22) || static_cast<long long>(N) * K > (1LL << 34))
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": N and K at most 4194304 and N * K at most 2^34");
     if (rank < 0) return fail(MILO_ERR_INVALID_ARG, f + ": negative rank");
     if (rank > MILO_MAX_RANK) return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": rank above 64");
     if (iters < 0 || iters > 1000) return fail(MILO_ERR_INVALID_ARG, f + ": hqq_iters outside 0..1000");
