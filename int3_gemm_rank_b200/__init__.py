@@ -284,6 +284,45 @@ def milo_assign_ranks(scores, avg_rank: int, max_rank: int = MILO_MAX_RANK) -> l
     return [int(out[i]) for i in range(n)]
 
 
+def quantize_experts(experts: list, avg_rank: int, max_rank: int = MILO_MAX_RANK, rounds: int = 3,
+                     power_iters: int = 2, score: str = "kurtosis", activation_counts=None, seed: int = 0,
+                     dev_status: torch.Tensor | None = None):
+    """The offline MiLo pipeline for a layer's experts.
+
+    experts: list of dict(w1=, w3=, w2=) fp16 CUDA weights ([I, H], [I, H], [H, I]).
+    Ranks: a budget of avg_rank per projection split by score (milo_assign_ranks),
+    the score being each projection's kurtosis (milo_kurtosis) or, with
+    score="activation", its expert's entry of activation_counts.  Then each
+    projection goes through milo_quantize_lorc (HQQ, rank-r compensator,
+    `rounds` refinement rounds) with a standard-normal test matrix drawn from a
+    generator seeded with `seed`.  Host synchronisation happens only to read the
+    kurtosis values.  Returns (list of dict(w1=, w3=, w2=) QWeight, ranks in
+    projection order w1, w3, w2 of expert 0, 1, ...)."""
+    names = ("w1", "w3", "w2")
+    mats = [e[n] for e in experts for n in names]
+    if score == "kurtosis":
+        scores = [float(milo_kurtosis(W, dev_status).item()) for W in mats]
+    elif score == "activation":
+        if activation_counts is None or len(activation_counts) != len(experts):
+            raise ValueError("activation_counts needs one count per expert")
+        scores = [float(c) for c in activation_counts for _ in names]
+    else:
+        raise ValueError("score must be 'kurtosis' or 'activation'")
+    ranks = milo_assign_ranks(scores, avg_rank, max_rank)
+    gen = torch.Generator(device=mats[0].device)
+    gen.manual_seed(seed)
+    out = []
+    for i, W in enumerate(mats):
+        p = lorc_params(ranks[i], rounds=rounds, power_iters=power_iters)
+        omega = (torch.randn(W.shape[1], p.sketch, generator=gen, device=W.device, dtype=torch.float32)
+                 if ranks[i] > 0 else None)
+        qw, _ = milo_quantize_lorc(W, p, omega, dev_status)
+        if i % 3 == 0:
+            out.append({})
+        out[-1][names[i % 3]] = qw
+    return out, ranks
+
+
 # ---------------------------------------------------------------------------
 # routing
 # ---------------------------------------------------------------------------

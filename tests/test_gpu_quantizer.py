@@ -273,3 +273,40 @@ def _unblob_rows(blob, rows, K):
                 s[2 * b + h, i] = groups[o]
                 z[2 * b + h, i] = groups[o + 1]
     return q, s, z
+
+
+def test_quantize_experts_pipeline_runs_the_layer(milo):
+    """The offline pipeline on a small layer: ranks from the kurtosis split
+    (the oracle's kurtosis and split give the same ranks), every projection
+    through the quantiser, and the layer forward with the result matches the
+    oracle's forward on the same pieces."""
+    from parity_util import REL_TOL, act_dev, rel_err
+    wk = wl.small_moe(name="t_pipeline")
+    names = ("w1", "w3", "w2")
+    experts = [{n: f16_dev(e[n].W) for n in names} for e in wk.experts]
+    st = milo.new_status()
+    qexp, ranks = milo.quantize_experts(experts, avg_rank=16, rounds=1, dev_status=st)
+    assert _status(st) == 0
+    kr = [oracle.kurtosis(e[n].W) for e in wk.experts for n in names]
+    assert ranks == oracle.assign_ranks(kr, 16)
+    assert sum(ranks) <= 16 * len(ranks)
+    # the oracle's view of the same quantised pieces
+    ref = []
+    for e in qexp:
+        d = {}
+        for n in names:
+            qw = e[n]
+            q, s, z = _unblob(qw.packed.cpu().numpy(), qw.N, qw.K)
+            U = qw.U.cpu().numpy().view(np.uint16) if qw.rank else np.zeros((qw.N, 0), np.uint16)
+            V = qw.V.cpu().numpy().view(np.uint16) if qw.rank else np.zeros((0, qw.K), np.uint16)
+            d[n] = oracle.PackedProj(oracle.pack(q), s, z, U, V)
+        ref.append(d)
+    layer = milo.MoELayer(qexp, wk.n_routed, wk.n_shared, wk.top_k)
+    r = milo.milo_route(f16_dev(wk.logits), wk.top_k, wk.renorm)
+    y = layer(act_dev(wk.x, wk.x_dtype), r, out_dtype=torch.float32, dev_status=st)
+    assert _status(st) == 0
+    ids, w, *_ = oracle.route(wk.logits, wk.top_k, wk.renorm)
+    y_ref, _, st_ref = oracle.moe_forward(wk.x, wk.x_dtype == "bf16", ids, w, ref, wk.n_routed, wk.n_shared,
+                                          wk.hidden, wk.inter)
+    assert st_ref == 0
+    assert rel_err(y.cpu().numpy(), y_ref) <= REL_TOL
