@@ -147,23 +147,25 @@ def test_quantize_lorc_rounds_track_the_oracle(milo):
     assert abs(np.linalg.norm(E) - err.min()) <= 1e-5 * err.min()
 
 
-def _unblob(blob, N, K):
-    """Codes, scales and zeros read back from a blob (layout of milo.h)."""
+def _unblob(blob, N, K, rows=None):
+    """Codes [len(rows), K] and scales, zeros [K/64, len(rows)] read back from a
+    blob (layout of milo.h), for the given rows or all N."""
+    rows = np.arange(N) if rows is None else np.asarray(rows)
     SB = K // 128
-    q = np.zeros((N, K), np.uint8)
-    s = np.zeros((K // 64, N), np.uint16)
-    z = np.zeros((K // 64, N), np.uint16)
-    for n in range(N):
-        t, rr = divmod(n, 64)
+    q = np.zeros((len(rows), K), np.uint8)
+    s = np.zeros((K // 64, len(rows)), np.uint16)
+    z = np.zeros((K // 64, len(rows)), np.uint16)
+    for i, n in enumerate(rows):
+        t, rr = divmod(int(n), 64)
         for b in range(SB):
             base = (t * SB + b) * 3584
             words = blob[base: base + 3072].view(np.uint32).reshape(64, 12)[rr]
-            q[n, 128 * b: 128 * b + 128] = oracle.unpack(words.reshape(1, 12), 128)[0]
+            q[i, 128 * b: 128 * b + 128] = oracle.unpack(words.reshape(1, 12), 128)[0]
             groups = blob[base + 3072: base + 3584].view(np.uint16)
-            for i in range(2):
-                o = i * 128 + ((rr // 16) * 8 + rr % 8) * 4 + ((rr % 16) // 8) * 2
-                s[2 * b + i, n] = groups[o]
-                z[2 * b + i, n] = groups[o + 1]
+            for h in range(2):
+                o = h * 128 + ((rr // 16) * 8 + rr % 8) * 4 + ((rr % 16) // 8) * 2
+                s[2 * b + h, i] = groups[o]
+                z[2 * b + h, i] = groups[o + 1]
     return q, s, z
 
 
@@ -243,7 +245,7 @@ def test_quantize_lorc_full_size_mixtral_w1(milo):
     R_gpu = R_gpu.cpu().numpy()
     rows = np.sort(rng.choice(N, size=96, replace=False))
     q, s, z, _ = oracle.hqq(oracle._f16(W[rows]))
-    qg, sg, zg = _unblob_rows(qw.packed.cpu().numpy(), rows, K)
+    qg, sg, zg = _unblob(qw.packed.cpu().numpy(), N, K, rows)
     assert np.array_equal(qg, q) and np.array_equal(sg, s) and np.array_equal(zg, z)
     assert np.array_equal(R_gpu[rows].view(np.uint32), oracle.residual(W[rows], q, s, z).view(np.uint32))
     U, V = oracle.rsvd(R_gpu, r, om, 2)
@@ -253,26 +255,6 @@ def test_quantize_lorc_full_size_mixtral_w1(milo):
     assert np.linalg.norm(Ug[rows] @ Vg - ref) <= UV_TOL * np.linalg.norm(ref)
     E = R_gpu.astype(np.float64) - Ug @ Vg
     assert abs(err[0] - np.linalg.norm(E)) <= 1e-5 * err[0]
-
-
-def _unblob_rows(blob, rows, K):
-    """Codes [len(rows), K] and scales, zeros [K/64, len(rows)] of the given rows of a blob."""
-    SB = K // 128
-    q = np.zeros((len(rows), K), np.uint8)
-    s = np.zeros((K // 64, len(rows)), np.uint16)
-    z = np.zeros((K // 64, len(rows)), np.uint16)
-    for i, n in enumerate(rows):
-        t, rr = divmod(int(n), 64)
-        for b in range(SB):
-            base = (t * SB + b) * 3584
-            words = blob[base: base + 3072].view(np.uint32).reshape(64, 12)[rr]
-            q[i, 128 * b: 128 * b + 128] = oracle.unpack(words.reshape(1, 12), 128)[0]
-            groups = blob[base + 3072: base + 3584].view(np.uint16)
-            for h in range(2):
-                o = h * 128 + ((rr // 16) * 8 + rr % 8) * 4 + ((rr % 16) // 8) * 2
-                s[2 * b + h, i] = groups[o]
-                z[2 * b + h, i] = groups[o + 1]
-    return q, s, z
 
 
 def test_quantize_experts_pipeline_runs_the_layer(milo):
