@@ -426,6 +426,15 @@ MILO_API milo_status milo_grouped_linear_noalloc(const milo_linear* lin, const v
 MILO_API size_t milo_moe_h_offset(const milo_moe_layer* layer, int32_t T);
 
 /*
+ * milo_selftest_wait_timeout -- self-test of the bounded waits: one block
+ * waits, with the same bounded wait the GEMM kernels use, on an mbarrier that
+ * nothing completes; after the wait limit (about two seconds of SM clock) it
+ * ORs MILO_DEV_TIMEOUT into dev_status (device memory, required) and returns.
+ * The context stays usable.  Stream-ordered; no host synchronisation.
+ */
+MILO_API milo_status milo_selftest_wait_timeout(int32_t* dev_status, void* stream);
+
+/*
  * milo_set_profile_events -- measurement hook.  `events` is a host array of n
  * cudaEvent_t (n = 0 or events = NULL disables).  While set, every
  * milo_moe_forward records events[0] / events[1] on its stream right before /

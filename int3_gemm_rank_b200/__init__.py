@@ -34,7 +34,7 @@ EXPORTS = ("milo_status_str", "milo_last_error", "milo_version", "milo_pack", "m
            "milo_moe_forward", "milo_moe_h_offset", "milo_set_profile_events",
            "milo_grouped_linear_noalloc", "milo_packed_bytes", "milo_hqq_pack",
            "milo_quantize_lorc_workspace", "milo_quantize_lorc", "milo_kurtosis_workspace", "milo_kurtosis",
-           "milo_assign_ranks")
+           "milo_assign_ranks", "milo_selftest_wait_timeout")
 
 
 class MiloError(RuntimeError):
@@ -124,6 +124,7 @@ def lib() -> C.CDLL:
         L.milo_kurtosis.argtypes = [vp, C.c_int64, vp, vp, sz, vp, vp]; L.milo_kurtosis.restype = C.c_int
         L.milo_assign_ranks.argtypes = [C.POINTER(C.c_double), i32, i32, i32, C.POINTER(i32)]
         L.milo_assign_ranks.restype = C.c_int
+        L.milo_selftest_wait_timeout.argtypes = [vp, vp]; L.milo_selftest_wait_timeout.restype = C.c_int
         _lib = L
     return _lib
 
