@@ -643,7 +643,7 @@ def quant_cpu_baseline(r: int, rounds: int, budget_rows: int = 2048) -> dict:
     dt = time.perf_counter() - t0
     return {"value": W.size / dt, "unit": "weights/s", "cores": cpu_threads(), "kind": "oracle",
             "sample": f"HQQ + rank-{r} compensator + {rounds} rounds on a [{W.shape[0]}, {W.shape[1]}] slice of "
-                      f"w1 ({dt:.1f} s; HQQ in C on one thread, the subspace iteration in numpy BLAS)"}
+                      f"w1 ({dt:.1f} s; HQQ in C over the host threads, the subspace iteration in numpy BLAS)"}
 
 
 def run_quantize(args):

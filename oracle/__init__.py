@@ -72,7 +72,7 @@ def lib():
                                            C.POINTER(Proj), C.POINTER(Proj), vp, vp, i]
         L.milo_ref_moe_forward.restype = i
         f = C.c_float
-        L.milo_ref_hqq.argtypes = [vp, i, i, i, f, f, vp, vp, vp]; L.milo_ref_hqq.restype = i
+        L.milo_ref_hqq.argtypes = [vp, i, i, i, f, f, vp, vp, vp, i]; L.milo_ref_hqq.restype = i
         L.milo_ref_hqq_trace.argtypes = [vp, i, f, f, vp, vp, vp, vp, vp]
         L.milo_ref_hqq_trace.restype = i
         _lib = L
@@ -257,8 +257,10 @@ def moe_forward(x_bits: np.ndarray, x_is_bf16: bool, ids: np.ndarray, w: np.ndar
 HQQ_ITERS, HQQ_BETA, HQQ_KAPPA = 20, 10.0, 1.01
 
 
-def hqq(T: np.ndarray, iters: int = HQQ_ITERS, beta: float = HQQ_BETA, kappa: float = HQQ_KAPPA):
-    """HQQ int3 quantisation of an fp32 target [N, K] (groups of 64 along K).
+def hqq(T: np.ndarray, iters: int = HQQ_ITERS, beta: float = HQQ_BETA, kappa: float = HQQ_KAPPA,
+        nthreads: int = 0):
+    """HQQ int3 quantisation of an fp32 target [N, K] (groups of 64 along K),
+    rows over `nthreads` host threads (0: all cores; the result is the same).
     Returns (q u8 [N, K], scale, zero fp16 bits [K/64, N], status)."""
     T = _c(T, np.float32)
     N, K = T.shape
@@ -266,7 +268,8 @@ def hqq(T: np.ndarray, iters: int = HQQ_ITERS, beta: float = HQQ_BETA, kappa: fl
     q = np.zeros((N, K), np.uint8)
     sc = np.zeros((K // 64, N), np.uint16)
     ze = np.zeros((K // 64, N), np.uint16)
-    st = lib().milo_ref_hqq(_p(T), N, K, int(iters), float(beta), float(kappa), _p(q), _p(sc), _p(ze))
+    st = lib().milo_ref_hqq(_p(T), N, K, int(iters), float(beta), float(kappa), _p(q), _p(sc), _p(ze),
+                            int(nthreads))
     return q, sc, ze, st
 
 

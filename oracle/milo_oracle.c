@@ -47,6 +47,7 @@
  */
 #include <math.h>
 #include <pthread.h>
+#include <sched.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -373,19 +374,56 @@ static int hqq_group(const float* t, int iters, float beta0, float kappa, uint8_
     return status;
 }
 
+static int default_threads(int nthreads);
+
+typedef struct {
+    const float* T;
+    int N, K, iters, n0, n1, status;
+    float beta0, kappa;
+    uint8_t* q;
+    uint16_t* scale;
+    uint16_t* zero;
+} hqq_job;
+
+static void* hqq_rows(void* arg) {
+    hqq_job* J = arg;
+    int G = J->K / 64;
+    J->status = 0;
+    for (int n = J->n0; n < J->n1; ++n)
+        for (int j = 0; j < G; ++j) {
+            size_t at = (size_t)n * J->K + (size_t)j * 64, sz = (size_t)j * J->N + n;
+            J->status |= hqq_group(J->T + at, J->iters, J->beta0, J->kappa, J->q + at, J->scale + sz,
+                                   J->zero + sz, NULL, NULL);
+        }
+    return NULL;
+}
+
 /*
  * HQQ quantisation of an fp32 target T [N, K] (K a multiple of 64) in groups
  * of 64 along K.  Outputs as milo_ref_quantize(): codes q [N, K], scale and
- * zero fp16 [K/64, N].  Returns REF_* status bits.
+ * zero fp16 [K/64, N].  Rows are split over `nthreads` threads (<= 0: every
+ * core this process may use); groups are independent, so the result does not depend on
+ * the thread count.  Returns REF_* status bits.
  */
 int milo_ref_hqq(const float* T, int N, int K, int iters, float beta0, float kappa,
-                 uint8_t* q, uint16_t* scale, uint16_t* zero) {
-    int status = 0, G = K / 64;
-    for (int n = 0; n < N; ++n)
-        for (int j = 0; j < G; ++j)
-            status |= hqq_group(T + (size_t)n * K + (size_t)j * 64, iters, beta0, kappa,
-                                q + (size_t)n * K + (size_t)j * 64, &scale[(size_t)j * N + n],
-                                &zero[(size_t)j * N + n], NULL, NULL);
+                 uint8_t* q, uint16_t* scale, uint16_t* zero, int nthreads) {
+    int nt = default_threads(nthreads);
+    if (nt > N) nt = N > 0 ? N : 1;
+    hqq_job* jobs = calloc((size_t)nt, sizeof(hqq_job));
+    pthread_t* th = calloc((size_t)nt, sizeof(pthread_t));
+    for (int t = 0; t < nt; ++t) {
+        jobs[t] = (hqq_job){T, N, K, iters, (int)((long long)N * t / nt), (int)((long long)N * (t + 1) / nt), 0,
+                            beta0, kappa, q, scale, zero};
+        if (nt > 1) pthread_create(&th[t], NULL, hqq_rows, &jobs[t]);
+    }
+    if (nt == 1) hqq_rows(&jobs[0]);
+    int status = 0;
+    for (int t = 0; t < nt; ++t) {
+        if (nt > 1) pthread_join(th[t], NULL);
+        status |= jobs[t].status;
+    }
+    free(jobs);
+    free(th);
     return status;
 }
 
@@ -543,8 +581,11 @@ static void* linear_rows(void* arg) {
     return NULL;
 }
 
+/* nthreads > 0 as given; else the cores this process may run on. */
 static int default_threads(int nthreads) {
     if (nthreads > 0) return nthreads;
+    cpu_set_t set;
+    if (sched_getaffinity(0, sizeof(set), &set) == 0 && CPU_COUNT(&set) > 0) return CPU_COUNT(&set);
     long c = sysconf(_SC_NPROCESSORS_ONLN);
     return c > 0 ? (int)c : 1;
 }
@@ -552,7 +593,7 @@ static int default_threads(int nthreads) {
 /*
  * Y [M, N] = X [M, K] * w_hat^T + (X V^T) U^T, all in fp64, where w_hat is the
  * dequantised packed weight of P.  Rows n are split over `nthreads` threads
- * (<= 0: all online cores); each output is produced by one thread in a fixed
+ * (<= 0: every core this process may use); each output is produced by one thread in a fixed
  * order, so the result does not depend on the thread count.
  */
 void milo_ref_linear(const double* X, int M, int K, const milo_ref_proj* P, int N,

@@ -26,7 +26,7 @@ MUTANTS = {
                             "for (int n = 0; n < N; ++n) Ud[(size_t)n * r + p] = urow[(size_t)(n * r + p) % N];"),
     "zero_not_negated": ("float z_f = -mn / s;", "float z_f = mn / s;"),
     "scale_by_8": ("float s_f = range / 7.0f;", "float s_f = range / 8.0f;"),
-    "round_half_up": ("float r = nearbyintf(v);", "float r = floorf(v + 0.5f);"),
+    "round_half_up": ("float r = nearbyintf(v);    /* ties to even */", "float r = floorf(v + 0.5f);"),
     "tie_to_higher_id": ("milo_ref_h2d(l[e]) > milo_ref_h2d(l[best])", "milo_ref_h2d(l[e]) >= milo_ref_h2d(l[best])"),
     "renorm_over_all": ("if (renorm) {", "if (0) {"),
     "unit_group_swap": ("int c = rr / 16, m = rr % 16 + 16 * half;", "int c = rr / 16, m = rr % 16 + 16 * (1 - half);"),
@@ -53,7 +53,7 @@ MUTANTS = {
 def test_mutant_is_caught(name, tmp_path):
     old, new = MUTANTS[name]
     src = open(SRC).read()
-    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
+    assert src.count(old) == 1, f"mutation anchor for {name} not found once"
     mutated = src.replace(old, new)
     c_path = tmp_path / "mutant.c"
     so_path = tmp_path / "mutant.so"
