@@ -113,6 +113,31 @@ def test_hqq_keeps_the_zero_point_of_lowest_l1_error():
         assert np.array_equal(q, np.clip(np.rint(t / s + zf), 0, 7).astype(np.uint8))
 
 
+def test_hqq_matrix_is_the_group_fit_at_every_thread_count():
+    """The matrix call is the one-group fit applied to each (row, group), its
+    scale and zero stored [K/64, N]; rows split over any number of host
+    threads give the same bits."""
+    rng = np.random.default_rng(36)
+    N, K = 13, 256
+    T = oracle._f16(wl.gen_weight(rng, N, K))
+    ref = None
+    for nt in (1, 3, 5, 64):
+        out = oracle.hqq(T, nthreads=nt)
+        assert out[3] == 0
+        if ref is None:
+            ref = out
+            continue
+        for a, b in zip(ref[:3], out[:3]):
+            assert np.array_equal(a, b)
+    q, sc, ze, _ = ref
+    for n in (0, 6, 12):
+        for j in range(K // 64):
+            qg, s_bits, z_bits, _, _ = oracle.hqq_trace(T[n, 64 * j:64 * (j + 1)], oracle.HQQ_ITERS,
+                                                        oracle.HQQ_BETA, oracle.HQQ_KAPPA)
+            assert np.array_equal(q[n, 64 * j:64 * (j + 1)], qg)
+            assert sc[j, n] == s_bits and ze[j, n] == z_bits
+
+
 def test_hqq_lowers_the_l1_error_of_outlier_groups():
     """The point of HQQ's sparsity-promoting fit: on weights with outliers its
     L1 reconstruction error is lower than round-to-nearest's."""

@@ -46,6 +46,7 @@ MUTANTS = {
     "hqq_mean_over_63": ("z = acc * 0.015625f;", "z = acc / 63.0f;"),
     "hqq_best_zero_not_kept": ("best_err = err;\n            best_z = z;", "best_err = err;"),
     "hqq_l2_error": ("err = err + a;", "err = err + a * a;"),
+    "hqq_scale_index_transposed": ("sz = (size_t)j * J->N + n;", "sz = (size_t)n * (J->K / 64) + j;"),
 }
 
 
