@@ -632,6 +632,49 @@ def quant_matrices(rank_id: int, hidden: int = 4096, inter: int = 14336):
             for name, n, k in (("w1", inter, hidden), ("w3", inter, hidden), ("w2", hidden, inter))]
 
 
+def quant_workload(r: int, rounds: int, sketch: int, power_iters: int, hqq_iters: int) -> str:
+    return (f"quantise one Mixtral-shaped expert per GPU: w1, w3 [14336, 4096], w2 [4096, 14336]; "
+            f"rank {r}, {rounds} refinement rounds, sketch {sketch}, {power_iters} power steps, "
+            f"HQQ {hqq_iters} iterations")
+
+
+def run_quantize_reference(args, rows: int = 256) -> int:
+    """--impl reference --workload quantize: the oracle's quantiser as the
+    reference arm (rank 0 only).  Each step quantises and compensates the next
+    [rows, 4096] slice of the same w1 the GPU arm quantises whole."""
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    r, rounds = args.quant_rank, args.quant_rounds
+    sketch = min(128, max(16, 2 * r)) if r > 0 else 0
+    W1 = wl.gen_weight(wl.rng_for("quantize", "w1", 0), 14336, 4096)
+    steps, warm = max(1, args.steps), max(0, args.warmup)
+    times = []
+    for s in range(warm + steps):
+        lo = (s * rows) % W1.shape[0]
+        W = np.ascontiguousarray(W1[lo:lo + rows])
+        om = wl.rng_for("quantize", "omega_cpu", s).standard_normal((W.shape[1], sketch))
+        t0 = time.perf_counter()
+        oracle.quantize_lorc(W, r, rounds, om)
+        if s >= warm:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = steps * rows * W1.shape[1] / total
+    nthreads = cpu_threads()
+    sample = (f"a [{rows}, {W1.shape[1]}] slice of w1 per step (HQQ in C over the host threads, "
+              f"the subspace iteration in numpy BLAS)")
+    line = {"impl": "reference", "metric": QUANT_METRIC, "value": value, "unit": "weights/s", "n_gpus": world,
+            "steps": steps, "warmup": warm, "ms_per_step": 1e3 * total / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": quant_workload(r, rounds, sketch, 2, oracle.HQQ_ITERS), "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "weights/s", "cores": nthreads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def quant_cpu_baseline(r: int, rounds: int, budget_rows: int = 2048) -> dict:
     """The oracle's quantiser on a sampled [budget_rows, 4096] slice of w1."""
     import oracle
@@ -741,9 +784,7 @@ def run_quantize(args):
         "metric": QUANT_METRIC, "value": weights * world / (ms / 1e3), "unit": "weights/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"quantise one Mixtral-shaped expert per GPU: w1, w3 [14336, 4096], w2 [4096, 14336]; "
-                               f"rank {r}, {rounds} refinement rounds, sketch {params.sketch}, "
-                               f"{params.power_iters} power steps, HQQ {params.hqq_iters} iterations",
+        "config": {"workload": quant_workload(r, rounds, params.sketch, params.power_iters, params.hqq_iters),
                    "l2": "inputs larger than L2 (117 MB fp16 weight plus its 235 MB fp32 residual per matrix)",
                    "parallelism": f"replica per GPU x{world}"},
         "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Top/s", "frac": achieved / peak,
@@ -789,9 +830,7 @@ def main(argv=None):
         args.warmup = 3
     if args.workload == "quantize":
         if args.impl == "reference":
-            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the layer forward; "
-                              "the quantiser's CPU baseline is part of its own line"}))
-            return 0
+            return run_quantize_reference(args)
         return run_quantize(args)
     if args.impl == "reference":
         return run_reference(args)

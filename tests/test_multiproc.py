@@ -53,3 +53,20 @@ def test_single_process_max_is_identity():
     import bench
     assert bench.max_over_ranks(3.25) == 3.25
     assert bench.dist_env()[2] >= 1
+
+
+def test_quantiser_reference_arm_line(capsys):
+    """The quantiser's reference arm (the oracle on row slices of w1) prints
+    one JSON line carrying the contract's keys."""
+    sys.path.insert(0, ROOT)
+    import json
+    import bench
+    args = type("A", (), {"steps": 1, "warmup": 0, "quant_rank": 8, "quant_rounds": 1})()
+    assert bench.run_quantize_reference(args, rows=64) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.QUANT_METRIC
+    assert line["value"] > 0 and line["unit"] == "weights/s" and line["steps"] == 1
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "weights/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert "[64, 4096]" in line["config"]["sample"]
