@@ -632,6 +632,44 @@ def quant_matrices(rank_id: int, hidden: int = 4096, inter: int = 14336):
             for name, n, k in (("w1", inter, hidden), ("w3", inter, hidden), ("w2", hidden, inter))]
 
 
+def _sgemm_launches(M: int, Nn: int, Kd: int) -> int:
+    """Kernels one fp32 product of the quantiser launches: the tiled GEMM, plus
+    the in-order sum of its reduction slices when a small output grid splits
+    the reduction (64-wide tiles, 128 rows when M >= 128; split when the grid
+    has fewer than 148 tiles and Kd >= 2048, at most 8 slices of a multiple of
+    16)."""
+    TM = 128 if M >= 128 else 64
+    tiles = ((Nn + 63) // 64) * ((M + TM - 1) // TM)
+    S = min(8, max(1, 296 // tiles)) if tiles < 148 and Kd >= 2048 else 1
+    kslice = -(-((Kd + S - 1) // S) // 16) * 16
+    return 2 if (Kd + kslice - 1) // kslice > 1 else 1
+
+
+def quant_launches(shapes, r: int, rounds: int, sketch: int, power_iters: int) -> int:
+    """Kernels milo_quantize_lorc launches for matrices of `shapes` [(N, K)]:
+    per round the HQQ pack, the error and next target, the error sum and the
+    copy of the best round; per compensator the products of the subspace
+    iteration, a Gram matrix (two kernels) and a Cholesky factor for every
+    basis pass, and the eigen-decomposition."""
+    total = 0
+    for N, K in shapes:
+        if r == 0:
+            total += 4
+            continue
+        l, q = sketch, power_iters
+        n = 0
+
+        def orth(M, passes):
+            return passes * (3 + _sgemm_launches(M, l, l))
+
+        n += _sgemm_launches(N, l, K) + orth(N, 1 if q > 0 else 2)
+        for it in range(q):
+            n += _sgemm_launches(K, l, N) + orth(K, 1) + _sgemm_launches(N, l, K) + orth(N, 1 if it + 1 < q else 2)
+        n += _sgemm_launches(l, K, N) + 2 + 1 + _sgemm_launches(N, r, l) + _sgemm_launches(r, K, l)
+        total += (rounds + 1) * (n + 4)
+    return total
+
+
 def quant_workload(r: int, rounds: int, sketch: int, power_iters: int, hqq_iters: int) -> str:
     return (f"quantise one Mixtral-shaped expert per GPU: w1, w3 [14336, 4096], w2 [4096, 14336]; "
             f"rank {r}, {rounds} refinement rounds, sketch {sketch}, {power_iters} power steps, "
@@ -794,7 +832,9 @@ def run_quantize(args):
                      "peak_source": "derived: 148 SMs x 128 fp32 lanes x the sampled SM clock"},
         "kernels": {"hqq_pack_ms": hqq_ms, "kurtosis_ms": kurt_ms, "kurtosis_gbs": kurt_gbs,
                     "kurtosis_frac_hbm": kurt_gbs / peaks()["hbm_gbs"]},
-        "gpu_launches": None, "clocks": clocks,
+        "gpu_launches": quant_launches([(j[0], j[1]) for j in jobs], r, rounds if r > 0 else 0, params.sketch,
+                                       params.power_iters) * args.steps,
+        "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = quant_cpu_baseline(r, rounds)

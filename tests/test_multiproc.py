@@ -70,3 +70,15 @@ def test_quantiser_reference_arm_line(capsys):
     assert line["e2e"] == {"value": line["value"], "unit": "weights/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert "[64, 4096]" in line["config"]["sample"]
+
+
+def test_quantiser_launch_count_matches_the_launch_list():
+    """The quantise line's gpu_launches: one Mixtral-shaped expert at rank 32,
+    3 refinement rounds, sketch 64, 2 power steps launched 536 kernels per step
+    in the ncu launch list (144 + 24 GEMMs, 168 Gram, 72 Cholesky, 12 each of
+    HQQ, eigen, apply, error sum and copy, 68 slice sums)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    shapes = [(14336, 4096), (14336, 4096), (4096, 14336)]
+    assert bench.quant_launches(shapes, 32, 3, 64, 2) == 536
+    assert bench.quant_launches(shapes, 0, 3, 0, 2) == 12
