@@ -426,10 +426,10 @@ def run_milo(args):
             milo._check(s, "milo_route")
         milo.milo_moe_forward(layer, xin, route, out_dtype=out_dt, dev_status=st, y=y, ws=ws)
 
-    # route, prep x, lorc w1|w3 (partial + reduce), gemm w1|w3, prep h, lorc w2 (partial + reduce),
-    # gemm w2, combine; the compensator launches drop out when no expert has one
+    # route (one kernel; from 512 tokens on a top-k kernel first), prep x, lorc w1|w3, gemm w1|w3,
+    # prep h, lorc w2, gemm w2, combine; the compensator launches drop out when no expert has one
     has_lorc = any(wk.experts[e][n].rank for e in range(wk.n_experts) for n in ("w1", "w3", "w2"))
-    launches_per_step = 8 if has_lorc else 6
+    launches_per_step = (7 if has_lorc else 5) + (2 if T >= 512 else 1)
 
     # --- correctness gate on the bench configuration itself
     step(x, logits)
