@@ -613,6 +613,141 @@ def finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, l
 
 
 # ---------------------------------------------------------------------------
+# single-projection batch sweep (--workload sweep)
+# ---------------------------------------------------------------------------
+
+SWEEP_TOKENS = (1, 4, 16, 64, 256, 1024)
+SWEEP_METRIC = ("grouped int3 + rank-32 compensator w1 projection (4096 -> 14336, 8 experts, Zipf routing): "
+                "tokens/s per batch size, with HBM and tensor rooflines")
+
+
+def sweep_cost(wk, counts) -> dict:
+    """Algorithmic bytes and FLOPs of one grouped w1 projection call: each
+    active expert's packed codes, fp16 scale and zero, and fp16 U and V, plus
+    x in (bf16) and y out (fp32); FLOPs of the int3 contraction and of both
+    compensator products."""
+    H, I, T = wk.hidden, wk.inter, wk.T
+    active = [e for e in range(wk.n_routed) if counts[e] > 0]
+    qz = I * H * 3 // 8 + 2 * (H // 64) * I * 2
+    nbytes = sum(qz + 2 * wk.experts[e]["w1"].rank * (I + H) for e in active) + T * H * 2 + T * I * 4
+    flops = sum(2 * int(counts[e]) * (I * H + wk.experts[e]["w1"].rank * (I + H)) for e in active)
+    return {"bytes": nbytes, "flops": flops, "active_experts": len(active)}
+
+
+def run_sweep(args):
+    """The w1 projection alone over 1 ... 1024 tokens, each routed to one
+    Zipf-drawn expert: the crossover from the memory-bound mma.sync kernel to
+    the tcgen05 kernel.  L2 is flushed (a 256 MB write) before every timed
+    call, since the small batches touch fewer weights than L2 holds."""
+    import torch
+
+    import int3_gemm_rank_b200 as milo
+    from int3_gemm_rank_b200 import build as milo_build
+
+    rank, local, world = dist_env()
+    if not os.path.exists(milo.LIB_PATH):
+        milo_build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+
+    def f16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.float16).to(dev)
+
+    base = wl.sweep(1)
+    projs = []
+    for e in range(base.n_routed):
+        P = base.experts[e]["w1"]
+        projs.append(milo.QWeight.quantize(f16(P.W), f16(P.U) if P.rank else None, f16(P.V) if P.rank else None))
+    lin = milo.GroupedLinear(projs)
+    st = milo.new_status(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    pk = peaks()
+    launches_per_call = 4 if any(P.rank for P in (base.experts[e]["w1"] for e in range(base.n_routed))) else 3
+    points, launches = [], 0
+    sampler = ClockSampler(local)
+    sampler.start()
+    for T in SWEEP_TOKENS:
+        wk = wl.sweep(T) if T > 1 else base
+        x = torch.from_numpy(np.ascontiguousarray(wk.x).view(np.int16)).view(torch.bfloat16).to(dev)
+        ids = torch.from_numpy(np.ascontiguousarray(wk.ids, dtype=np.int32)).to(dev)
+        r = milo.milo_route(None, 1, False, E=base.n_routed, ids=ids, dev_status=st)
+        y = torch.empty((T, wk.inter), dtype=torch.float32, device=dev)
+        ws = lin.workspace(T, 1, dev)
+
+        def call():
+            lin(x, r["offsets"], r["perm"], k=1, dev_status=st, y=y, ws=ws)
+
+        for _ in range(args.warmup):
+            call()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4 * args.steps)]
+        for e in ev:            # torch creates the CUDA event on its first record
+            e.record(stream)
+        milo.milo_set_profile_events(None)
+        barrier(dev)
+        torch.cuda.synchronize()
+        # pass 1: the whole call (prep, compensator, GEMM, combine), no event inside it
+        for i in range(args.steps):
+            flush.zero_()
+            ev[4 * i].record(stream)
+            call()
+            ev[4 * i + 1].record(stream)
+        torch.cuda.synchronize()
+        # pass 2: events around the grouped GEMM launch alone
+        for i in range(args.steps):
+            flush.zero_()
+            milo.milo_set_profile_events(ev[4 * i + 2:4 * i + 4])
+            call()
+        torch.cuda.synchronize()
+        milo.milo_set_profile_events(None)
+        launches += 2 * args.steps * launches_per_call
+        call_ms = max_over_ranks(statistics.mean(ev[4 * i].elapsed_time(ev[4 * i + 1])
+                                                 for i in range(args.steps)), dev)
+        gemm_ms = statistics.mean(ev[4 * i + 2].elapsed_time(ev[4 * i + 3]) for i in range(args.steps))
+        counts = np.bincount(wk.ids.ravel(), minlength=base.n_routed)
+        cost = sweep_cost(wk, counts)
+        forced = os.environ.get("MILO_GEMM", "")
+        tensor = forced == "tc" if forced in ("mma", "tc") else T >= 64 * base.n_routed
+        gbs = cost["bytes"] / (call_ms / 1e3) / 1e9
+        tflops = cost["flops"] / (call_ms / 1e3) / 1e12
+        points.append({"tokens": T, "kernel": "tc_gemm_kernel (tcgen05)" if tensor else "gemv_kernel (mma.sync)",
+                       "active_experts": cost["active_experts"], "us_per_call": 1e3 * call_ms,
+                       "gemm_us": 1e3 * gemm_ms, "tokens_per_s": world * T / (call_ms / 1e3),
+                       "algorithmic_bytes": cost["bytes"], "algorithmic_flops": cost["flops"],
+                       "hbm_gbs": gbs, "hbm_frac": gbs / pk["hbm_gbs"], "tflops": tflops,
+                       "tensor_frac": tflops / pk["bf16_tflops"]})
+    clocks = sampler.stop()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} on the sweep")
+    top = points[-1]
+    tensor_top = top["kernel"].startswith("tc_")
+    line = {
+        "metric": SWEEP_METRIC, "value": top["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": top["us_per_call"] / 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": f"w1 projection H{base.hidden} -> I{base.inter}, {base.n_routed} experts, rank "
+                               f"{int(base.ranks[0])}, int3 g64, k = 1 with Zipf(1.1) expert ids, x bf16, y fp32; "
+                               f"value and ms_per_step at {top['tokens']} tokens, every size under 'sweep'",
+                   "l2": "flushed by a 256 MB write before every timed call",
+                   "parallelism": f"replica per GPU x{world}"},
+        "sweep": points,
+        "roofline": ({"bound": "tensor", "achieved": top["tflops"], "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                      "frac": top["tensor_frac"], "traffic": None}
+                     if tensor_top else
+                     {"bound": "hbm", "achieved": top["hbm_gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+                      "frac": top["hbm_frac"], "traffic": None}),
+        "e2e": None, "gpu_launches": launches, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+# ---------------------------------------------------------------------------
 # offline quantiser (--workload quantize)
 # ---------------------------------------------------------------------------
 
@@ -852,8 +987,10 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("milo", "reference"), default="milo")
-    ap.add_argument("--workload", choices=("mixtral", "deepseek", "prefill", "quantize"), default="mixtral",
-                    help="quantize: the offline quantiser on one Mixtral-shaped expert (its own JSON line)")
+    ap.add_argument("--workload", choices=("mixtral", "deepseek", "prefill", "quantize", "sweep"),
+                    default="mixtral",
+                    help="quantize: the offline quantiser on one Mixtral-shaped expert; sweep: the w1 "
+                         "projection over 1 ... 1024 Zipf-routed tokens (each its own JSON line)")
     ap.add_argument("--quant-rank", type=int, default=32)
     ap.add_argument("--quant-rounds", type=int, default=3)
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing")
@@ -872,6 +1009,12 @@ def main(argv=None):
         if args.impl == "reference":
             return run_quantize_reference(args)
         return run_quantize(args)
+    if args.workload == "sweep":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the layer forward "
+                              "and the quantiser; the sweep's parity is in the GPU tests"}))
+            return 0
+        return run_sweep(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_milo(args)
