@@ -82,3 +82,21 @@ def test_quantiser_launch_count_matches_the_launch_list():
     shapes = [(14336, 4096), (14336, 4096), (4096, 14336)]
     assert bench.quant_launches(shapes, 32, 3, 64, 2) == 536
     assert bench.quant_launches(shapes, 0, 3, 0, 2) == 12
+
+
+def test_sweep_cost_counts_active_experts_only():
+    """Bytes and FLOPs of one grouped w1 call, worked by hand: codes 3/8 B,
+    fp16 scale and zero per 64 weights, fp16 U and V of each active expert,
+    bf16 x in and fp32 y out."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    P = type("P", (), {"rank": 32})()
+    wk = type("W", (), {"hidden": 4096, "inter": 14336, "T": 3, "n_routed": 8,
+                        "experts": [{"w1": P} for _ in range(8)]})()
+    counts = np.array([2, 0, 1, 0, 0, 0, 0, 0])
+    c = bench.sweep_cost(wk, counts)
+    per_expert = 14336 * 4096 * 3 // 8 + 4 * 64 * 14336 + 2 * 32 * (14336 + 4096)
+    assert c["bytes"] == 2 * per_expert + 3 * 4096 * 2 + 3 * 14336 * 4
+    assert c["flops"] == 3 * 2 * (14336 * 4096 + 32 * (14336 + 4096))
+    assert c["active_experts"] == 2
