@@ -3,7 +3,7 @@
 low-rank-compensator forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl milo|reference]
-                    [--workload mixtral|deepseek|prefill|quantize] [--lorc fp16|int3]
+                    [--workload mixtral|deepseek|prefill|quantize|sweep] [--lorc fp16|int3]
 
 One step = one pass of the whole hot path over one batch of synthetic tokens:
 router (top-k + grouping) -> activation preparation -> compensator
@@ -21,7 +21,12 @@ cross-GPU exchange on one node), the time is the max over ranks and `value`
 counts the tokens of all ranks ("weak" scaling).
 
 --impl reference times the CPU oracle (plain C, fp64) on the host cores, each
-step a bounded sample of tokens of the same workload.
+step a bounded sample of tokens of the same workload (with --workload
+quantize: the oracle's quantiser on a row slice of the same weight).
+
+Two more lines of their own: --workload quantize times the offline quantiser
+on one Mixtral-shaped expert; --workload sweep times the w1 projection alone
+over 1 ... 1024 Zipf-routed tokens (L2 flushed before each call).
 """
 from __future__ import annotations
 
