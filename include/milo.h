@@ -441,7 +441,9 @@ MILO_API milo_status milo_selftest_wait_timeout(int32_t* dev_status, void* strea
  * after the launch of the w1|w3 grouped GEMM and events[2] / events[3] around
  * the w2 grouped GEMM; milo_grouped_linear records events[0] / events[1] around
  * its grouped GEMM.  The caller owns the events and reads them with
- * cudaEventElapsedTime after the stream completes.  Process-wide setting.
+ * cudaEventElapsedTime after the stream completes.  Process-wide setting,
+ * not synchronised: change it only while no other host thread is inside the
+ * library.
  */
 MILO_API milo_status milo_set_profile_events(void* const* events, int32_t n);
 
