@@ -100,3 +100,40 @@ def test_sweep_cost_counts_active_experts_only():
     assert c["bytes"] == 2 * per_expert + 3 * 4096 * 2 + 3 * 14336 * 4
     assert c["flops"] == 3 * 2 * (14336 * 4096 + 32 * (14336 + 4096))
     assert c["active_experts"] == 2
+
+
+def test_layer_line_carries_the_contract_keys(capsys):
+    """The layer line that finish() prints holds every key of the bench
+    contract, with the roofline, e2e and clock objects complete (fed with
+    made-up timings; no GPU)."""
+    sys.path.insert(0, ROOT)
+    import json
+    import numpy as np
+    import torch
+    import bench
+    import workloads as wl
+    wk = wl.small_moe()
+    counts = np.full(wk.n_routed, 2)
+    bytes_ = bench.layer_bytes(wk, counts)
+    args = type("A", (), {"steps": 4, "warmup": 3, "lorc": "fp16", "workload": "mixtral", "tokens": None,
+                          "no_cpu_baseline": True})()
+    x = torch.zeros(wk.T, wk.hidden, dtype=torch.bfloat16)
+    logits = torch.zeros(wk.T, wk.n_routed, dtype=torch.float16)
+    y = torch.zeros(wk.T, wk.hidden, dtype=torch.bfloat16)
+    clocks = {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.finish(args, wk, 0, 1, wk.T, 0.18, 88000.0, 0.11, 0.05, bytes_, x, logits, y, 76000.0, 8,
+                        clocks) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert key in line, key
+    assert line["n_gpus"] == 1 and line["steps"] == 4 and line["gpu_launches"] == 32
+    assert line["scaling"] == "weak" and line["higher_is_better"] is True
+    rf = line["roofline"]
+    assert rf["bound"] in ("hbm", "tensor") and rf["frac"] == rf["achieved"] / rf["peak"]
+    assert "traffic" in rf and (rf["traffic"] is None or rf["traffic"] > 0)
+    e2e = line["e2e"]
+    assert e2e["value"] == 76000.0 and e2e["unit"] == "tokens/s"
+    assert e2e["h2d_bytes_per_step"] == wk.T * wk.hidden * 2 + wk.T * wk.n_routed * 2
+    assert e2e["d2h_bytes_per_step"] == wk.T * wk.hidden * 2
+    assert line["clocks"] == clocks and "workload" in line["config"]
