@@ -649,25 +649,32 @@ double milo_ref_silu(double a) { return a / (1.0 + exp(-a)); }
 /*
  * SwiGLU expert on the rows X [M, H]: a = X W1^T (+LoRC), b = X W3^T (+LoRC),
  * h = fp16(silu(a) * b), y = h W2^T (+LoRC).  h_bits [M, I] receives the fp16
- * activations, y [M, H] the fp64 outputs.
+ * activations, y [M, H] the fp64 outputs.  Returns NONFINITE when a product
+ * silu(a) * b is not finite, FP16_RANGE when a finite one rounds to an fp16
+ * infinity (h is an fp16 tensor).
  */
-static void expert_forward(const double* X, int M, int H, int I, int group,
-                           const milo_ref_proj* w1, const milo_ref_proj* w3,
-                           const milo_ref_proj* w2, uint16_t* h_bits, double* y,
-                           int nthreads) {
+static int expert_forward(const double* X, int M, int H, int I, int group,
+                          const milo_ref_proj* w1, const milo_ref_proj* w3,
+                          const milo_ref_proj* w2, uint16_t* h_bits, double* y,
+                          int nthreads) {
+    int status = 0;
     double* a = malloc(sizeof(double) * (size_t)M * I);
     double* b = malloc(sizeof(double) * (size_t)M * I);
     double* h = malloc(sizeof(double) * (size_t)M * I);
     milo_ref_linear(X, M, H, w1, I, group, a, nthreads);
     milo_ref_linear(X, M, H, w3, I, group, b, nthreads);
     for (size_t i = 0; i < (size_t)M * I; ++i) {
-        h_bits[i] = milo_ref_d2h(milo_ref_silu(a[i]) * b[i]);
+        double v = milo_ref_silu(a[i]) * b[i];
+        h_bits[i] = milo_ref_d2h(v);
         h[i] = milo_ref_h2d(h_bits[i]);
+        if (!isfinite(v)) status |= REF_NONFINITE;
+        else if (!isfinite(h[i])) status |= REF_FP16_RANGE;
     }
     milo_ref_linear(h, M, I, w2, H, group, y, nthreads);
     free(a);
     free(b);
     free(h);
+    return status;
 }
 
 /*
@@ -693,7 +700,6 @@ int milo_ref_moe_forward(const uint16_t* x, int x_is_bf16, int T, int H, int I,
     for (size_t i = 0; i < (size_t)T * H; ++i) {
         X[i] = x_is_bf16 ? milo_ref_bf2d(x[i]) : milo_ref_h2d(x[i]);
         if (!isfinite(X[i])) status |= REF_NONFINITE;
-        else if (fabs(X[i]) > 65504.0) status |= REF_FP16_RANGE;
     }
     double* y_slot = calloc((size_t)(F > 0 ? F : 1) * H, sizeof(double));
     double* y_sh = calloc((size_t)(S > 0 ? S : 1) * T * H, sizeof(double));
@@ -712,7 +718,7 @@ int milo_ref_moe_forward(const uint16_t* x, int x_is_bf16, int T, int H, int I,
         if (M == 0) continue;
         for (int m = 0; m < M; ++m)
             memcpy(Xe + (size_t)m * H, X + (size_t)(rows[m] / k) * H, sizeof(double) * H);
-        expert_forward(Xe, M, H, I, group, &w1[e], &w3[e], &w2[e], h_tmp, ye, nthreads);
+        status |= expert_forward(Xe, M, H, I, group, &w1[e], &w3[e], &w2[e], h_tmp, ye, nthreads);
         for (int m = 0; m < M; ++m) {
             memcpy(y_slot + (size_t)rows[m] * H, ye + (size_t)m * H, sizeof(double) * H);
             if (h_bits)
@@ -720,8 +726,8 @@ int milo_ref_moe_forward(const uint16_t* x, int x_is_bf16, int T, int H, int I,
         }
     }
     for (int s = 0; s < S; ++s) {
-        expert_forward(X, T, H, I, group, &w1[E + s], &w3[E + s], &w2[E + s], h_tmp,
-                       y_sh + (size_t)s * T * H, nthreads);
+        status |= expert_forward(X, T, H, I, group, &w1[E + s], &w3[E + s], &w2[E + s], h_tmp,
+                                 y_sh + (size_t)s * T * H, nthreads);
         if (h_bits)
             memcpy(h_bits + ((size_t)F + (size_t)s * T) * I, h_tmp, sizeof(uint16_t) * T * I);
     }

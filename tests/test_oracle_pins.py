@@ -537,9 +537,25 @@ def test_moe_one_hot_weights_equal_gather_and_relabelling_invariance():
     np.testing.assert_allclose(ya, yb, rtol=1e-12, atol=1e-13)
 
 
-def test_moe_flags_fp16_range():
+def test_moe_flags_fp16_range_of_h_not_of_x():
+    """Activations are FP16 up to a power-of-two row scale, so a bf16 input
+    beyond 65504 is valid (the result stays exact); the SwiGLU output h is an
+    fp16 tensor, so a finite silu(a) b that rounds to an fp16 infinity is
+    flagged."""
     H, I = 128, 256
     ex = _small_layer(E=1, S=0, H=H, I=I, ranks=(0,))
-    x = wl.f32_to_bf16_bits(np.full((1, H), 1.0e6, np.float32))
-    _, _, st = oracle.moe_forward(x, True, np.zeros((1, 1), np.int32), np.ones((1, 1)), ex, 1, 0, H, I)
-    assert st & oracle.FP16_RANGE
+    ids, w = np.zeros((1, 1), np.int32), np.ones((1, 1))
+    big = wl.f32_to_bf16_bits(np.full((1, H), 1.0e6, np.float32))
+    y, h, st = oracle.moe_forward(big, True, ids, w, ex, 1, 0, H, I, want_h=True)
+    assert st & oracle.FP16_RANGE                       # h overflows
+    hf = h.view(np.float16)
+    assert np.isinf(hf).any()
+    x = wl.f32_to_bf16_bits(np.full((1, H), 70000.0, np.float32))
+    rng = np.random.default_rng(19)
+    small = {}
+    for name, (n, kk), a in (("w1", (I, H), -16), ("w3", (I, H), -16), ("w2", (H, I), 0)):
+        W = wl.f32_to_f16_bits(wl.f16_bits_to_f32(wl.gen_weight(rng, n, kk)) * np.float32(2.0 ** a))
+        small[name] = oracle.quantize_projection(W, np.zeros((n, 0), np.uint16), np.zeros((0, kk), np.uint16))
+    y2, h2, st2 = oracle.moe_forward(x, True, ids, w, [small], 1, 0, H, I, want_h=True)
+    assert st2 == 0 and np.isfinite(h2.view(np.float16)).all() and np.isfinite(y2).all()
+    assert np.abs(h2.view(np.float16)).max() > 0
