@@ -3,7 +3,7 @@
 low-rank-compensator forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl milo|reference]
-                    [--workload mixtral|deepseek|prefill|quantize|sweep] [--lorc fp16|int3]
+                    [--workload mixtral|deepseek|prefill|single|quantize|sweep] [--lorc fp16|int3]
 
 One step = one pass of the whole hot path over one batch of synthetic tokens:
 router (top-k + grouping) -> activation preparation -> compensator
@@ -24,9 +24,11 @@ counts the tokens of all ranks ("weak" scaling).
 step a bounded sample of tokens of the same workload (with --workload
 quantize: the oracle's quantiser on a row slice of the same weight).
 
-Two more lines of their own: --workload quantize times the offline quantiser
-on one Mixtral-shaped expert; --workload sweep times the w1 projection alone
-over 1 ... 1024 Zipf-routed tokens (L2 flushed before each call).
+More lines of their own: --workload single times the single-expert decode
+call (1 x 1024 -> 1024, rank 16) over rotated weight copies; --workload
+quantize times the offline quantiser on one Mixtral-shaped expert;
+--workload sweep times the w1 projection alone over 1 ... 1024 Zipf-routed
+tokens (L2 flushed before each call).
 """
 from __future__ import annotations
 
@@ -753,6 +755,213 @@ def run_sweep(args):
 
 
 # ---------------------------------------------------------------------------
+# single expert, decode (--workload single)
+# ---------------------------------------------------------------------------
+
+SINGLE_METRIC = ("single int3 expert with a rank-16 compensator, decode (1 token, 1024 -> 1024): "
+                 "time per call and achieved HBM bandwidth over rotated weight copies")
+
+
+def single_cost(P) -> dict:
+    """Algorithmic bytes of one single-expert call (codes, fp16 scale and zero,
+    fp16 U and V, x in fp16, y out fp32) and of its grouped GEMM launch (all
+    but V, which the compensator's down-projection reads); FLOPs of the int3
+    contraction and both compensator products."""
+    n, k, r = P.n, P.k, P.rank
+    blob = n * k * 3 // 8 + 2 * (k // 64) * n * 2
+    act = k * 2 + n * 4
+    return {"call": blob + 2 * r * (n + k) + act, "gemm": blob + 2 * r * n + act,
+            "flops": 2 * (n * k + r * (n + k)), "copy": blob + 2 * r * (n + k)}
+
+
+def run_single(args):
+    """The single-expert decode call, milo_grouped_linear on one token (no
+    routing: one expert).  Its 0.53 MB of weights fit in L2, so the step
+    rotates over distinct copies of the packed weight and its compensator,
+    at least 3 x L2 of them, and L2 is flushed (a 256 MB write) before each
+    timed region; within a region a copy comes back only after 3 x L2 of
+    other copies.  One step = one call; the K steps are one CUDA graph."""
+    import torch
+
+    import int3_gemm_rank_b200 as milo
+    from int3_gemm_rank_b200 import build as milo_build
+
+    rank, local, world = dist_env()
+    if not os.path.exists(milo.LIB_PATH):
+        milo_build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+
+    x_bits, P = wl.single()
+    cost = single_cost(P)
+    n_copies = -(-3 * L2_BYTES // cost["copy"])
+
+    def f16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.float16).to(dev)
+
+    q0 = milo.QWeight.quantize(f16(P.W), f16(P.U), f16(P.V))
+    lins = [milo.GroupedLinear([milo.QWeight(q0.packed.clone(), P.n, P.k, q0.U.clone(), q0.V.clone())])
+            for _ in range(n_copies)]
+    x = f16(x_bits)
+    st = milo.new_status(dev)
+    r = milo.milo_route(None, 1, False, E=1, ids=torch.zeros((1, 1), dtype=torch.int32, device=dev),
+                        dev_status=st)
+    off, perm = r["offsets"], r["perm"]
+    y = torch.empty((1, P.n), dtype=torch.float32, device=dev)
+    ws = lins[0].workspace(1, 1, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    K = args.steps
+    launches_per_call = 4          # prep, compensator down-projection, grouped GEMM, per-slot combine
+
+    def calls(xin, base=0):
+        for j in range(K):
+            milo.milo_grouped_linear(lins[(base + j) % n_copies], xin, off, perm, 1, torch.float32, st, y, ws)
+
+    # gate on the bench configuration: the calls run with a clean device status
+    # (their parity with the oracle is tests/test_gpu_fullsize.py's single-expert case)
+    calls(x)
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} on the single-expert workload")
+    graph = capture_step(torch, dev, lambda: calls(x))
+    for _ in range(args.warmup):
+        graph()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_soak = time.perf_counter()
+    while time.perf_counter() - t_soak < args.soak:
+        graph()
+        torch.cuda.synchronize()
+    flush.zero_()
+    barrier(dev)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    graph()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(dev)
+    ms_total = max_over_ranks(start.elapsed_time(stop), dev)
+    # region 2: the calls launched one by one with events around the grouped GEMM
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K)]
+    for e in ev:
+        e.record(stream)
+    flush.zero_()
+    torch.cuda.synchronize()
+    for j in range(K):
+        milo.milo_set_profile_events(ev[2 * j:2 * j + 2])
+        milo.milo_grouped_linear(lins[j % n_copies], x, off, perm, 1, torch.float32, st, y, ws)
+    torch.cuda.synchronize()
+    milo.milo_set_profile_events(None)
+    clocks = sampler.stop()
+    gemm_ms = statistics.mean(ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(K))
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} after the timed region")
+    ms_call = ms_total / K
+    pk = peaks()
+    call_gbs = cost["call"] / (ms_call / 1e3) / 1e9
+    gemm_gbs = cost["gemm"] / (gemm_ms / 1e3) / 1e9
+
+    # end to end: x from pinned host memory and y back every call
+    e2e = None
+    if not args.no_e2e:
+        x_h = x.cpu().pin_memory()
+        y_h = torch.empty((1, P.n), dtype=torch.float32).pin_memory()
+        x_d = torch.empty_like(x)
+
+        def e2e_calls():
+            for j in range(K):
+                x_d.copy_(x_h, non_blocking=True)
+                milo.milo_grouped_linear(lins[j % n_copies], x_d, off, perm, 1, torch.float32, st, y, ws)
+                y_h.copy_(y, non_blocking=True)
+
+        g2 = capture_step(torch, dev, e2e_calls)
+        for _ in range(args.warmup):
+            g2()
+        flush.zero_()
+        torch.cuda.synchronize()
+        barrier(dev)
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        g2()
+        e2.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(s2.elapsed_time(e2), dev)
+        e2e = {"value": world * K / (e2e_ms / 1e3), "unit": "tokens/s", "us_per_call": 1e3 * e2e_ms / K,
+               "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 4}
+    line = {
+        "metric": SINGLE_METRIC, "value": world * K / (ms_total / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms_call, "us_per_call": 1e3 * ms_call,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": f"single expert decode: x fp16 [1 x {P.k}], W [{P.n} x {P.k}] int3 g64 "
+                               f"(N(0, 0.02), 0.1 % outliers x20), rank {P.rank} fp16 U, V; y fp32",
+                   "l2": f"{n_copies} rotated copies of the packed weight and compensator "
+                         f"({n_copies * cost['copy'] / 1e6:.0f} MB, 3 x L2) and a 256 MB flush before each "
+                         f"timed region",
+                   "launch": f"one CUDA graph of the {K} calls", "parallelism": f"replica per GPU x{world}"},
+        "roofline": {"bound": "hbm", "achieved": gemm_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": gemm_gbs / pk["hbm_gbs"], "traffic": None,
+                     "kernel": "gemv_kernel<false> (grouped int3 GEMM + compensator, split-K)",
+                     "algorithmic_bytes_per_launch": cost["gemm"], "ms_per_launch": gemm_ms,
+                     "peak_source": f"{pk['source']} HBM copy bandwidth"},
+        "call_hbm": {"bytes_per_call": cost["call"], "achieved_gbs": call_gbs, "frac": call_gbs / pk["hbm_gbs"],
+                     "roofline_us": 1e6 * cost["call"] / (pk["hbm_gbs"] * 1e9)},
+        "e2e": e2e, "gpu_launches": launches_per_call * K, "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = single_cpu_baseline(x_bits, P)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def single_oracle_calls(x_bits, P, budget_s: float, max_calls: int = 1 << 30):
+    """Oracle single-expert calls (the layer's linear, fp64) until budget_s."""
+    import oracle
+    ref = oracle.quantize_projection(P.W, P.U, P.V)
+    X = wl.f16_bits_to_f32(x_bits).astype(np.float64)
+    nthreads = cpu_threads()
+    t0 = time.perf_counter()
+    n = 0
+    while n < max_calls and (n == 0 or time.perf_counter() - t0 < budget_s):
+        oracle.linear(X, ref, nthreads=nthreads)
+        n += 1
+    return n, time.perf_counter() - t0, nthreads
+
+
+def single_cpu_baseline(x_bits, P) -> dict:
+    n, secs, nthreads = single_oracle_calls(x_bits, P, 10.0)
+    return {"value": n / secs, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"{n} oracle calls of the single-expert decode projection (1 token), {secs:.1f} s"}
+
+
+def run_single_reference(args) -> int:
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    x_bits, P = wl.single()
+    single_oracle_calls(x_bits, P, 0.0, max_calls=max(0, args.warmup))
+    n, secs, nthreads = single_oracle_calls(x_bits, P, 1e9, max_calls=max(1, args.steps))
+    value = n / secs
+    line = {"impl": "reference", "metric": SINGLE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": n, "warmup": args.warmup, "ms_per_step": 1e3 * secs / n, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"single expert decode: x fp16 [1 x {P.k}], W [{P.n} x {P.k}] int3 g64, "
+                                   f"rank {P.rank} fp16 U, V; y fp32"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                             "sample": f"{n} oracle calls of the whole projection, one per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
 # offline quantiser (--workload quantize)
 # ---------------------------------------------------------------------------
 
@@ -992,10 +1201,11 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("milo", "reference"), default="milo")
-    ap.add_argument("--workload", choices=("mixtral", "deepseek", "prefill", "quantize", "sweep"),
+    ap.add_argument("--workload", choices=("mixtral", "deepseek", "prefill", "single", "quantize", "sweep"),
                     default="mixtral",
-                    help="quantize: the offline quantiser on one Mixtral-shaped expert; sweep: the w1 "
-                         "projection over 1 ... 1024 Zipf-routed tokens (each its own JSON line)")
+                    help="single: one 1024 x 1024 expert with a rank-16 compensator, 1 token; quantize: the "
+                         "offline quantiser on one Mixtral-shaped expert; sweep: the w1 projection over "
+                         "1 ... 1024 Zipf-routed tokens (each its own JSON line)")
     ap.add_argument("--quant-rank", type=int, default=32)
     ap.add_argument("--quant-rounds", type=int, default=3)
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing")
@@ -1014,6 +1224,10 @@ def main(argv=None):
         if args.impl == "reference":
             return run_quantize_reference(args)
         return run_quantize(args)
+    if args.workload == "single":
+        if args.impl == "reference":
+            return run_single_reference(args)
+        return run_single(args)
     if args.workload == "sweep":
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the layer forward "

@@ -60,7 +60,7 @@ typedef enum {
 /* Device status bits, OR-ed into *dev_status by the kernels. */
 #define MILO_DEV_BAD_EXPERT_ID 0x1  /* a routed id outside [0, E): the slot is dropped */
 #define MILO_DEV_NONFINITE 0x2      /* NaN/Inf in weights, logits or activations */
-#define MILO_DEV_FP16_RANGE 0x4     /* a value does not fit fp16 (activation, s or z) */
+#define MILO_DEV_FP16_RANGE 0x4     /* a value does not fit fp16 (s, z, h, an fp16 output) */
 #define MILO_DEV_TIMEOUT 0x8        /* a bounded pipeline wait gave up; outputs invalid */
 
 /* Router flags. */
@@ -356,6 +356,16 @@ MILO_API milo_status milo_linear_workspace_bytes(const milo_linear* lin, int32_t
 MILO_API milo_status milo_moe_workspace_bytes(const milo_moe_layer* layer, int32_t T, size_t* bytes);
 
 /*
+ * Activations (milo_grouped_linear, milo_moe_forward): the GEMMs multiply the
+ * int3 codes with FP16 activations (W3A16).  Each activation row (a token's
+ * x, or a routed slot's SwiGLU output h) is first multiplied by a power of two
+ * 2^a that brings its largest magnitude into [1, 2) and then rounded to fp16;
+ * the result is multiplied by 2^-a.  So every fp16 activation, and every bf16
+ * one within 2^17 of its row's largest magnitude, enters the product exactly,
+ * whatever the row's scale: bf16 rows beyond the fp16 range are accepted too.
+ */
+
+/*
  * milo_grouped_linear -- per routed slot, y = x W_e^T + (x V_e^T) U_e^T.
  *   x        [T, K] fp16 or bf16 (x_dt), row-major
  *   expert_offsets, perm  from milo_route over n_experts experts and k slots
@@ -363,7 +373,8 @@ MILO_API milo_status milo_moe_workspace_bytes(const milo_moe_layer* layer, int32
  *   y        [T*k, N] in y_dt (F32, F16 or BF16), row f = t*k + j; rows of
  *            dropped slots are written as zeros
  *   ws       >= milo_linear_workspace_bytes(lin, T, k), 256-byte aligned
- * Device: FP16_RANGE (|x| > 65504), NONFINITE, TIMEOUT.
+ * Device: NONFINITE (NaN/Inf in x), FP16_RANGE (an fp16 output or the
+ * compensator's fp16 t = x V^T overflows), TIMEOUT.
  */
 MILO_API milo_status milo_grouped_linear(const milo_linear* lin, const void* x, milo_dtype x_dt,
                                 int32_t T, int32_t k, const int32_t* expert_offsets,
@@ -383,7 +394,7 @@ MILO_API milo_status milo_grouped_linear(const milo_linear* lin, const void* x, 
  *            fp16 SwiGLU activations h [T*k + n_shared*T, inter] sit at byte
  *            offset milo_moe_h_offset(layer, T) of ws after the call, row p =
  *            expert-sorted slot p (shared-expert rows after the routed ones).
- * Device: FP16_RANGE, NONFINITE, TIMEOUT.
+ * Device: NONFINITE, FP16_RANGE (h, t or an fp16 output overflows), TIMEOUT.
  */
 MILO_API milo_status milo_moe_forward(const milo_moe_layer* layer, const void* x, milo_dtype x_dt,
                              int32_t T, const float* topk_w, const int32_t* expert_offsets,
@@ -408,8 +419,11 @@ MILO_API milo_status milo_moe_forward(const milo_moe_layer* layer, const void* x
  *     lin, T, k) exceeds MILO_NOALLOC_SCRATCH_BYTES returns MILO_ERR_WORKSPACE
  *     and enqueues nothing; decode-sized calls (tens of rows) fit.
  *   - The first call on each device looks up the buffer's device address
- *     with that device current (cudaGetSymbolAddress); make that first call
- *     before any stream capture.  A failed lookup returns MILO_ERR_CUDA.
+ *     with that device current (cudaGetSymbolAddress) and keeps it for the
+ *     life of the process; make that first call before any stream capture,
+ *     and do not reset the device (cudaDeviceReset) while the library is
+ *     loaded, which would leave the kept address stale.  A failed lookup
+ *     returns MILO_ERR_CUDA.
  *   - Every call on a device shares the one buffer and finds the previous
  *     call's contents in it; nothing in it needs to start at zero (each call
  *     writes what it reads).  Calls that overlap on the GPU (other streams,
@@ -433,6 +447,21 @@ MILO_API size_t milo_moe_h_offset(const milo_moe_layer* layer, int32_t T);
  * The context stays usable.  Stream-ordered; no host synchronisation.
  */
 MILO_API milo_status milo_selftest_wait_timeout(int32_t* dev_status, void* stream);
+
+/*
+ * milo_set_gemm_path -- measurement and test hook: which grouped GEMM kernel
+ * milo_moe_forward and milo_grouped_linear use.  MILO_GEMM_AUTO: chosen per
+ * call from the routed rows per expert (the tcgen05 kernel when they are many,
+ * the mma.sync kernel when they are few); MILO_GEMM_MMA / MILO_GEMM_TC force
+ * one (both compute the same results within fp32 rounding).  The initial
+ * value comes from the environment variable MILO_GEMM ("mma" or "tc"), read
+ * once, the first time a call needs it.  Process-wide; applies to calls made
+ * after it returns.  Errors: an unknown mode -> INVALID_ARG.
+ */
+#define MILO_GEMM_AUTO 0
+#define MILO_GEMM_MMA 1
+#define MILO_GEMM_TC 2
+MILO_API milo_status milo_set_gemm_path(int32_t mode);
 
 /*
  * milo_set_profile_events -- measurement hook.  `events` is a host array of n

@@ -25,6 +25,7 @@ MILO_OK, MILO_ERR_INVALID_ARG, MILO_ERR_UNSUPPORTED_SHAPE, MILO_ERR_WORKSPACE, M
 MILO_LORC_F16, MILO_LORC_INT3 = 0, 1
 MILO_DEV_BAD_EXPERT_ID, MILO_DEV_NONFINITE, MILO_DEV_FP16_RANGE, MILO_DEV_TIMEOUT = 1, 2, 4, 8
 MILO_ROUTE_RENORM, MILO_ROUTE_IDS_GIVEN = 1, 2
+MILO_GEMM_AUTO, MILO_GEMM_MMA, MILO_GEMM_TC = 0, 1, 2
 MILO_GROUP, MILO_MAX_RANK = 64, 64
 
 # The C ABI symbols of include/milo.h (checked by the tests).
@@ -34,7 +35,7 @@ EXPORTS = ("milo_status_str", "milo_last_error", "milo_version", "milo_pack", "m
            "milo_moe_forward", "milo_moe_h_offset", "milo_set_profile_events",
            "milo_grouped_linear_noalloc", "milo_packed_bytes", "milo_hqq_pack",
            "milo_quantize_lorc_workspace", "milo_quantize_lorc", "milo_kurtosis_workspace", "milo_kurtosis",
-           "milo_assign_ranks", "milo_selftest_wait_timeout")
+           "milo_assign_ranks", "milo_selftest_wait_timeout", "milo_set_gemm_path")
 
 
 class MiloError(RuntimeError):
@@ -125,6 +126,7 @@ def lib() -> C.CDLL:
         L.milo_assign_ranks.argtypes = [C.POINTER(C.c_double), i32, i32, i32, C.POINTER(i32)]
         L.milo_assign_ranks.restype = C.c_int
         L.milo_selftest_wait_timeout.argtypes = [vp, vp]; L.milo_selftest_wait_timeout.restype = C.c_int
+        L.milo_set_gemm_path.argtypes = [i32]; L.milo_set_gemm_path.restype = C.c_int
         _lib = L
     return _lib
 
@@ -160,6 +162,13 @@ def milo_set_profile_events(events: list | None):
         return
     arr = (C.c_void_p * len(events))(*[e.cuda_event for e in events])
     _check(lib().milo_set_profile_events(arr, len(events)), "milo_set_profile_events")
+
+
+def milo_set_gemm_path(path: str):
+    """Which grouped GEMM kernel the forward calls use: "auto", "mma" (mma.sync)
+    or "tc" (tcgen05); process-wide."""
+    mode = {"auto": MILO_GEMM_AUTO, "mma": MILO_GEMM_MMA, "tc": MILO_GEMM_TC}[path]
+    _check(lib().milo_set_gemm_path(mode), "milo_set_gemm_path")
 
 
 def new_status(device=None) -> torch.Tensor:

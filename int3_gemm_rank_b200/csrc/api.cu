@@ -13,6 +13,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <mutex>
 #include <string>
@@ -155,7 +156,7 @@ struct LorcPlan {
 static int lorc_counters(int n_exp) { return n_exp * 2 * ((MILO_MAX_RANK + 15) / 16) * 8; }
 
 struct LinearWs {
-    size_t grp, rows, inv, frag, gsum, t, tpart, done, part, total;
+    size_t grp, rows, inv, rscale, frag, gsum, t, tpart, done, part, total;
     int R, splits, tcols;
     LorcPlan lp;
 };
@@ -211,6 +212,7 @@ static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
     w.grp = c.take(static_cast<size_t>(n_exp) * 8);
     w.rows = c.take(static_cast<size_t>(w.R) * 4);
     w.inv = c.take(static_cast<size_t>(w.R) * 4);
+    w.rscale = c.take(static_cast<size_t>(w.R) * 4);
     w.frag = c.take(frag_bytes(lin->K, w.R));
     w.gsum = c.take(gsum_bytes(lin->K, w.R));
     w.t = c.take(static_cast<size_t>(w.R) * w.tcols * 2);
@@ -223,7 +225,7 @@ static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
 }
 
 struct MoeWs {
-    size_t grp, rows, xfrag, xg, t13, h, hfrag, hg, t2, tpart, done, part, total;
+    size_t grp, rows, xscale, xfrag, xg, t13, h, hscale, hfrag, hg, t2, tpart, done, part, total;
     int R, R_routed, splits, tc13, tc2;
     LorcPlan lp13, lp2;
 };
@@ -242,10 +244,12 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
     w.tc2 = std::max(8, L->max_rank);
     w.grp = c.take(static_cast<size_t>(n_exp) * 8);
     w.rows = c.take(static_cast<size_t>(w.R) * 4);
+    w.xscale = c.take(static_cast<size_t>(w.R) * 4);
     w.xfrag = c.take(frag_bytes(H, w.R));
     w.xg = c.take(gsum_bytes(H, w.R));
     w.t13 = c.take(static_cast<size_t>(w.R) * w.tc13 * 2);
     w.h = c.take(static_cast<size_t>(w.R) * I * 2);
+    w.hscale = c.take(static_cast<size_t>(w.R) * 4);
     w.hfrag = c.take(frag_bytes(I, w.R));
     w.hg = c.take(gsum_bytes(I, w.R));
     w.t2 = c.take(static_cast<size_t>(w.R) * w.tc2 * 2);
@@ -263,8 +267,9 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
 // ---------------------------------------------------------------------------
 // launch helpers
 // ---------------------------------------------------------------------------
-static void act_ptrs(GemvParams& g, void* frag, void* t, int R, int K, int tcols, bool has_t) {
+static void act_ptrs(GemvParams& g, void* frag, void* rscale, void* t, int R, int K, int tcols, bool has_t) {
     g.x = static_cast<const uint16_t*>(frag);
+    g.rscale = static_cast<const float*>(rscale);
     g.t = has_t ? static_cast<const uint16_t*>(t) : nullptr;
     g.R = R;
     g.K = K;
@@ -283,12 +288,30 @@ static milo_status run_gemv(GemvParams& g, bool glu, cudaStream_t st, const char
 // Which grouped GEMM runs.  The mma.sync kernel suits a few routed rows per
 // expert (decode): a tcgen05.mma of N = 16 costs as much to issue as one of
 // N = 64.  With many rows per expert (prefill) the weights are reused across
-// 128-row tiles and the tcgen05 kernel takes over.  MILO_GEMM=mma|tc forces
-// one (both give the same results within fp32 rounding).
+// 128-row tiles and the tcgen05 kernel takes over.  milo_set_gemm_path (or
+// MILO_GEMM=mma|tc in the environment, read once) forces one; both give the
+// same results within fp32 rounding.
+static std::atomic<int> g_gemm_path{-1};   // -1: not yet read from the environment
+
+static int gemm_path() {
+    int v = g_gemm_path.load(std::memory_order_relaxed);
+    if (v >= 0) return v;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const char* e = getenv("MILO_GEMM");
+        int m = MILO_GEMM_AUTO;
+        if (e && e[0] == 't') m = MILO_GEMM_TC;
+        else if (e && e[0] == 'm') m = MILO_GEMM_MMA;
+        int unset = -1;
+        g_gemm_path.compare_exchange_strong(unset, m);
+    });
+    return g_gemm_path.load(std::memory_order_relaxed);
+}
+
 static bool use_tc(long long routed_rows, int n_routed) {
-    const char* v = getenv("MILO_GEMM");
-    if (v && v[0] == 't') return true;
-    if (v && v[0] == 'm') return false;
+    const int path = gemm_path();
+    if (path == MILO_GEMM_TC) return true;
+    if (path == MILO_GEMM_MMA) return false;
     return routed_rows >= 64LL * std::max(1, n_routed);
 }
 
@@ -312,6 +335,7 @@ static milo_status run_tc(const GemvParams& g, bool glu, void* xcol, void* gsum,
                                  static_cast<uint64_t>(g.tcols) * 2, 64, kTcTokens, "compensator rows",
                                  CU_TENSOR_MAP_SWIZZLE_128B)) != MILO_OK)
         return s;
+    p.rscale = g.rscale;
     p.table = g.table;
     p.grp = g.grp;
     p.y_part = g.y_part;
@@ -365,6 +389,14 @@ extern "C" milo_status milo_set_profile_events(void* const* events, int32_t n) {
         return fail(MILO_ERR_INVALID_ARG, "milo_set_profile_events: n must be in [0, 4]");
     for (int i = 0; i < 4; ++i) g_prof[i] = i < n ? static_cast<cudaEvent_t>(events[i]) : nullptr;
     g_prof_n = n;
+    return MILO_OK;
+}
+
+extern "C" milo_status milo_set_gemm_path(int32_t mode) {
+    clear_error();
+    if (mode != MILO_GEMM_AUTO && mode != MILO_GEMM_MMA && mode != MILO_GEMM_TC)
+        return fail(MILO_ERR_INVALID_ARG, "milo_set_gemm_path: mode must be MILO_GEMM_AUTO, _MMA or _TC");
+    g_gemm_path.store(mode, std::memory_order_relaxed);
     return MILO_OK;
 }
 
@@ -468,26 +500,63 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     int32_t* inv = reinterpret_cast<int32_t*>(base + w.inv);
 
     const bool tc = use_tc(static_cast<long long>(T) * k, lin->n_experts);
-    PrepParams pp{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.frag),
-                  reinterpret_cast<uint16_t*>(base + w.gsum), tc ? 1 : 0, dev_status, w.R, lin->K, x_dt == MILO_BF16,
-                  1, expert_offsets, perm, grp, inv, T, k, lin->n_experts, 0, w.R,
-                  reinterpret_cast<int32_t*>(base + w.done), lorc_counters(lin->n_experts)};
+    float* rscale = reinterpret_cast<float*>(base + w.rscale);
+    PrepParams pp = {};
+    pp.src = static_cast<const uint16_t*>(x);
+    pp.row_src = rows;
+    pp.frag = reinterpret_cast<uint16_t*>(base + w.frag);
+    pp.gsum = reinterpret_cast<uint16_t*>(base + w.gsum);
+    pp.rscale = rscale;
+    pp.layout = tc ? 1 : 0;
+    pp.dev_status = dev_status;
+    pp.R = w.R;
+    pp.K = lin->K;
+    pp.src_bf16 = x_dt == MILO_BF16;
+    pp.rows = 1;
+    pp.offsets = expert_offsets;
+    pp.perm = perm;
+    pp.grp = grp;
+    pp.inv = inv;
+    pp.T = T;
+    pp.k = k;
+    pp.E = lin->n_experts;
+    pp.S = 0;
+    pp.R_routed = w.R;
+    pp.zero = reinterpret_cast<int32_t*>(base + w.done);
+    pp.nzero = lorc_counters(lin->n_experts);
     milo_status s = check_cuda(launch_prep(pp, st), "prep");
     if (s != MILO_OK) return s;
 
     const bool has_t = lin->max_rank > 0;
     const ProjDev* table = static_cast<const ProjDev*>(lin->table);
     if (has_t) {
-        LorcParams lp{static_cast<const uint16_t*>(x), rows, table, grp,
-                      reinterpret_cast<uint16_t*>(base + w.t), reinterpret_cast<float*>(base + w.tpart),
-                      reinterpret_cast<int32_t*>(base + w.done), dev_status, 1, 0, -1, lin->n_experts, lin->K, w.R, w.tcols, 0, x_dt == MILO_BF16,
-                      w.lp.splits, w.lp.row_groups};
+        LorcParams lp = {};
+        lp.src = static_cast<const uint16_t*>(x);
+        lp.row_src = rows;
+        lp.rscale = rscale;
+        lp.table = table;
+        lp.grp = grp;
+        lp.t = reinterpret_cast<uint16_t*>(base + w.t);
+        lp.part = reinterpret_cast<float*>(base + w.tpart);
+        lp.done = reinterpret_cast<int32_t*>(base + w.done);
+        lp.dev_status = dev_status;
+        lp.stride = 1;
+        lp.proj_a = 0;
+        lp.proj_b = -1;
+        lp.n_exp = lin->n_experts;
+        lp.K = lin->K;
+        lp.R = w.R;
+        lp.tcols = w.tcols;
+        lp.t_col_b = 0;
+        lp.src_bf16 = x_dt == MILO_BF16;
+        lp.splits = w.lp.splits;
+        lp.row_groups = w.lp.row_groups;
         if ((s = check_cuda(launch_lorc(lp, st), "lorc")) != MILO_OK) return s;
     }
 
     GemvParams g;
     memset(&g, 0, sizeof(g));
-    act_ptrs(g, base + w.frag, base + w.t, w.R, lin->K, w.tcols, has_t);
+    act_ptrs(g, base + w.frag, rscale, base + w.t, w.R, lin->K, w.tcols, has_t);
     g.table = table;
     g.grp = grp;
     g.y_part = reinterpret_cast<float*>(base + w.part);
@@ -539,22 +608,60 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     milo_status s;
 
     const bool tc = use_tc(w.R_routed, L->n_routed);
-    PrepParams px{static_cast<const uint16_t*>(x), rows, reinterpret_cast<uint16_t*>(base + w.xfrag),
-                  reinterpret_cast<uint16_t*>(base + w.xg), tc ? 1 : 0, dev_status, w.R, H, x_dt == MILO_BF16, 1,
-                  expert_offsets, perm, grp, nullptr, T, L->top_k, L->n_routed, L->n_shared, w.R_routed,
-                  reinterpret_cast<int32_t*>(base + w.done), lorc_counters(n_exp)};
+    float* xscale = reinterpret_cast<float*>(base + w.xscale);
+    float* hscale = reinterpret_cast<float*>(base + w.hscale);
+    PrepParams px = {};
+    px.src = static_cast<const uint16_t*>(x);
+    px.row_src = rows;
+    px.frag = reinterpret_cast<uint16_t*>(base + w.xfrag);
+    px.gsum = reinterpret_cast<uint16_t*>(base + w.xg);
+    px.rscale = xscale;
+    px.layout = tc ? 1 : 0;
+    px.dev_status = dev_status;
+    px.R = w.R;
+    px.K = H;
+    px.src_bf16 = x_dt == MILO_BF16;
+    px.rows = 1;
+    px.offsets = expert_offsets;
+    px.perm = perm;
+    px.grp = grp;
+    px.inv = nullptr;
+    px.T = T;
+    px.k = L->top_k;
+    px.E = L->n_routed;
+    px.S = L->n_shared;
+    px.R_routed = w.R_routed;
+    px.zero = reinterpret_cast<int32_t*>(base + w.done);
+    px.nzero = lorc_counters(n_exp);
     if ((s = check_cuda(launch_prep(px, st), "prep x")) != MILO_OK) return s;
     if (has_t) {
-        LorcParams lp{static_cast<const uint16_t*>(x), rows, table, grp,
-                      reinterpret_cast<uint16_t*>(base + w.t13), reinterpret_cast<float*>(base + w.tpart),
-                      reinterpret_cast<int32_t*>(base + w.done), dev_status, 3, 0, 1, n_exp, H, w.R, w.tc13, L->max_rank, x_dt == MILO_BF16,
-                      w.lp13.splits, w.lp13.row_groups};
+        LorcParams lp = {};
+        lp.src = static_cast<const uint16_t*>(x);
+        lp.row_src = rows;
+        lp.rscale = xscale;
+        lp.table = table;
+        lp.grp = grp;
+        lp.t = reinterpret_cast<uint16_t*>(base + w.t13);
+        lp.part = reinterpret_cast<float*>(base + w.tpart);
+        lp.done = reinterpret_cast<int32_t*>(base + w.done);
+        lp.dev_status = dev_status;
+        lp.stride = 3;
+        lp.proj_a = 0;
+        lp.proj_b = 1;
+        lp.n_exp = n_exp;
+        lp.K = H;
+        lp.R = w.R;
+        lp.tcols = w.tc13;
+        lp.t_col_b = L->max_rank;
+        lp.src_bf16 = x_dt == MILO_BF16;
+        lp.splits = w.lp13.splits;
+        lp.row_groups = w.lp13.row_groups;
         if ((s = check_cuda(launch_lorc(lp, st), "lorc w1|w3")) != MILO_OK) return s;
     }
 
     GemvParams g1;
     memset(&g1, 0, sizeof(g1));
-    act_ptrs(g1, base + w.xfrag, base + w.t13, w.R, H, w.tc13, has_t);
+    act_ptrs(g1, base + w.xfrag, xscale, base + w.t13, w.R, H, w.tc13, has_t);
     g1.table = table;
     g1.grp = grp;
     g1.h = reinterpret_cast<uint16_t*>(base + w.h);
@@ -573,20 +680,47 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     if (s != MILO_OK) return s;
     prof_record(1, st);
 
-    PrepParams ph{reinterpret_cast<const uint16_t*>(base + w.h), nullptr,
-                  reinterpret_cast<uint16_t*>(base + w.hfrag), reinterpret_cast<uint16_t*>(base + w.hg), tc ? 1 : 0,
-                  dev_status, w.R, I, 0, 0, nullptr, nullptr, nullptr, nullptr, 0, 0, 0, 0, 0, nullptr, 0};
+    PrepParams ph = {};
+    ph.src = reinterpret_cast<const uint16_t*>(base + w.h);
+    ph.row_src = nullptr;
+    ph.frag = reinterpret_cast<uint16_t*>(base + w.hfrag);
+    ph.gsum = reinterpret_cast<uint16_t*>(base + w.hg);
+    ph.rscale = hscale;
+    ph.layout = tc ? 1 : 0;
+    ph.dev_status = dev_status;
+    ph.R = w.R;
+    ph.K = I;
+    ph.src_bf16 = 0;
+    ph.rows = 0;
     if ((s = check_cuda(launch_prep(ph, st), "prep h")) != MILO_OK) return s;
     if (has_t) {
-        LorcParams lp{reinterpret_cast<const uint16_t*>(base + w.h), nullptr, table, grp,
-                      reinterpret_cast<uint16_t*>(base + w.t2), reinterpret_cast<float*>(base + w.tpart),
-                      reinterpret_cast<int32_t*>(base + w.done), dev_status, 3, 2, -1, n_exp, I, w.R, w.tc2, 0, 0, w.lp2.splits, w.lp2.row_groups};
+        LorcParams lp = {};
+        lp.src = reinterpret_cast<const uint16_t*>(base + w.h);
+        lp.row_src = nullptr;
+        lp.rscale = hscale;
+        lp.table = table;
+        lp.grp = grp;
+        lp.t = reinterpret_cast<uint16_t*>(base + w.t2);
+        lp.part = reinterpret_cast<float*>(base + w.tpart);
+        lp.done = reinterpret_cast<int32_t*>(base + w.done);
+        lp.dev_status = dev_status;
+        lp.stride = 3;
+        lp.proj_a = 2;
+        lp.proj_b = -1;
+        lp.n_exp = n_exp;
+        lp.K = I;
+        lp.R = w.R;
+        lp.tcols = w.tc2;
+        lp.t_col_b = 0;
+        lp.src_bf16 = 0;
+        lp.splits = w.lp2.splits;
+        lp.row_groups = w.lp2.row_groups;
         if ((s = check_cuda(launch_lorc(lp, st), "lorc w2")) != MILO_OK) return s;
     }
 
     GemvParams g2;
     memset(&g2, 0, sizeof(g2));
-    act_ptrs(g2, base + w.hfrag, base + w.t2, w.R, I, w.tc2, has_t);
+    act_ptrs(g2, base + w.hfrag, hscale, base + w.t2, w.R, I, w.tc2, has_t);
     g2.table = table;
     g2.grp = grp;
     g2.y_part = reinterpret_cast<float*>(base + w.part);

@@ -1,6 +1,7 @@
 // aux.cu -- the kernels around the grouped int3 GEMM:
-//   prep_kernel    activations -> fp16 MMA fragments (power-of-2 factors of the
-//                  int3 field extraction folded in) and per-group sums; the
+//   prep_kernel    activations -> fp16 MMA fragments (the row's power-of-2
+//                  scale and those of the int3 field extraction folded in)
+//                  and per-group sums; the
 //                  first one of a call also does the row bookkeeping (expert
 //                  groups, row -> token) from the router's offsets and perm
 //   lorc_*_kernel  compensator down-projection t = x V^T per expert
@@ -27,6 +28,8 @@ namespace milo {
 // ---------------------------------------------------------------------------
 // prep: fragment-ordered activations and group sums, one block per row
 // ---------------------------------------------------------------------------
+// Activations of register (word t, field f) times 2^(6 - e): exact, the
+// scaled row's values being below 2 (see act_scale).
 template <int S, int H>
 __device__ __forceinline__ uint32_t frag_pair(const __half (&x)[32]) {
     constexpr int t = sched_word(S, H), f = sched_field(S, H);
@@ -109,6 +112,30 @@ __device__ __forceinline__ int row_source(const PrepParams& p, int row, int32_t&
     return f / p.k;
 }
 
+// Largest magnitude of row `src` (K elements, fp16 or bf16), over the whole
+// block; 0 for a zero row.  NaN counts as larger than everything (the caller's
+// scale then falls back to 1 and the conversion flags it).
+__device__ __forceinline__ uint32_t row_max_bits(const PrepParams& p, int src) {
+    __shared__ uint32_t wmax[4];
+    uint32_t mx = 0u;
+    if (src >= 0) {
+        const uint4* rowv = reinterpret_cast<const uint4*>(p.src + static_cast<size_t>(src) * p.K);
+        for (int i = threadIdx.x; i < p.K / 8; i += blockDim.x) {
+            const uint4 u = rowv[i];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                mx = max(mx, __float_as_uint(fabsf(act_f32(static_cast<uint16_t>(w[q] & 0xFFFFu), p.src_bf16))));
+                mx = max(mx, __float_as_uint(fabsf(act_f32(static_cast<uint16_t>(w[q] >> 16), p.src_bf16))));
+            }
+        }
+    }
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    return max(max(wmax[0], wmax[1]), max(wmax[2], wmax[3]));
+}
+
 __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     grid_dep_launch();
     grid_dep_wait();
@@ -127,6 +154,10 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     } else {
         src = p.row_src ? p.row_src[row] : row;
     }
+    // the row's scale 2^a: every block of the row reads the whole row (the
+    // blocks of one row are few, and only while rows are few)
+    const float scale = row_scale_for(row_max_bits(p, src));
+    if (blockIdx.y == 0 && threadIdx.x == 0) p.rscale[row] = scale;
     for (int base = blockIdx.y * blockDim.x; base < SB * 4; base += gridDim.y * blockDim.x) {
         const int idx = base + threadIdx.x;
         const bool active = idx < SB * 4;
@@ -142,8 +173,8 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
                 const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    x[16 * half + 2 * i] = to_half(static_cast<uint16_t>(w[i] & 0xFFFFu), p.src_bf16, st);
-                    x[16 * half + 2 * i + 1] = to_half(static_cast<uint16_t>(w[i] >> 16), p.src_bf16, st);
+                    x[16 * half + 2 * i] = to_half_scaled(static_cast<uint16_t>(w[i] & 0xFFFFu), p.src_bf16, scale, st);
+                    x[16 * half + 2 * i + 1] = to_half_scaled(static_cast<uint16_t>(w[i] >> 16), p.src_bf16, scale, st);
                 }
             }
 #pragma unroll
@@ -173,16 +204,15 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
             o2[0] = make_uint4(f4.x, f4.y, f5.x, f5.y);
             o2[1] = make_uint4(f6.x, f6.y, f7.x, f7.y);
             if (c == 0) {
-                // the two group sums split exactly enough into fp16 hi + lo
-                // (2^-22 relative), slots (hi, lo, hi, lo) per group; a pair of
-                // super-blocks shares 16 slots, the odd tail's second half is 0
+                // the two group sums (|sum| <= 128) split exactly enough into
+                // fp16 hi + lo (2^-22 relative), slots (hi, lo, hi, lo) per group; a
+                // pair of super-blocks shares 16 slots, the odd tail's second half is 0
                 uint32_t v[4];
                 const float gs[2] = {s0, s1};
 #pragma unroll
                 for (int g = 0; g < 2; ++g) {
                     const __half hi = __float2half_rn(gs[g]);
                     const __half lo = __float2half_rn(gs[g] - __half2float(hi));
-                    if (__hisinf(hi)) st |= MILO_DEV_FP16_RANGE;
                     v[2 * g] = v[2 * g + 1] =
                         static_cast<uint32_t>(__half_as_ushort(hi)) | (static_cast<uint32_t>(__half_as_ushort(lo)) << 16);
                 }
@@ -216,13 +246,16 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
 
 cudaError_t launch_prep(const PrepParams& p, cudaStream_t s) {
     if (p.R <= 0) return cudaSuccess;
-    // 32 super-blocks per block; enough blocks per row to fill the GPU at decode sizes
-    const int chunks = (p.K / 128 * 4 + 127) / 128;
+    // 32 super-blocks per block; several blocks per row fill the GPU at decode
+    // sizes, one block per row once rows are many (each block of a row reads
+    // the whole row for its scale)
+    const int chunks = p.R >= 256 ? 1 : (p.K / 128 * 4 + 127) / 128;
     return launch_pdl(prep_kernel, dim3(p.R, chunks), dim3(128), 0, s, p);
 }
 
 // ---------------------------------------------------------------------------
-// lorc: t[p, col0 + j] = sum_k x[p, k] V[j, k] for the rows of each expert.
+// lorc: t[p, col0 + j] = sum_k x'[p, k] V[j, k] for the rows of each expert,
+// x' = fp16(x 2^a) with the row's scale (so t carries the row's 2^a too).
 // One block per (expert, projection, 16-rank block, K slice, row-tile group);
 // its four warps split the K slice and their 16x16 tiles are added in a fixed
 // order into part[slice].  The block that finishes a (expert, projection,
@@ -230,11 +263,23 @@ cudaError_t launch_prep(const PrepParams& p, cudaStream_t s) {
 // (a counter per tile says which block that is).  Both orders are fixed, so
 // the result does not depend on scheduling.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t load_x_pair(const uint16_t* row, int k, bool bf16, int32_t& st) {
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(row + k);
-    const __half lo = to_half(static_cast<uint16_t>(w & 0xFFFFu), bf16, st);
-    const __half hi = to_half(static_cast<uint16_t>(w >> 16), bf16, st);
-    return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+// Four packed activation pairs times the row's scale, as fp16 pairs.
+__device__ __forceinline__ uint4 scale_pairs(uint4 v, bool bf16, float scale, int32_t& st) {
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const __half lo = to_half_scaled(static_cast<uint16_t>(w[q] & 0xFFFFu), bf16, scale, st);
+        const __half hi = to_half_scaled(static_cast<uint16_t>(w[q] >> 16), bf16, scale, st);
+        w[q] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// t value rounded to fp16 (FP16_RANGE if it overflows).
+__device__ __forceinline__ uint16_t t_half(float v, int32_t& st) {
+    const __half h = __float2half_rn(v);
+    if (__hisinf(h)) st |= MILO_DEV_FP16_RANGE;
+    return __half_as_ushort(h);
 }
 
 constexpr int kLorcRankBlocks = (MILO_MAX_RANK + 15) / 16;
@@ -248,6 +293,7 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
     __shared__ __align__(16) uint16_t vs[16][kLorcPitch];
     __shared__ float part[4][16][17];
     __shared__ int src_row[16];
+    __shared__ float src_scale[16];
     const int nproj = p.proj_b >= 0 ? 2 : 1;
     int b = blockIdx.x;
     const int split = b % p.splits;
@@ -289,6 +335,7 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
         if (threadIdx.x < 16) {
             const int i = threadIdx.x;
             src_row[i] = mt + i < m ? (p.row_src ? p.row_src[row0 + mt + i] : row0 + mt + i) : -1;
+            src_scale[i] = mt + i < m ? p.rscale[row0 + mt + i] : 1.0f;
         }
         float acc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
         for (int kc = kbeg; kc < kend; kc += kLorcChunk) {
@@ -308,18 +355,9 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
                     *reinterpret_cast<uint4*>(&vs[rr][8 * ch]) = v;
                 } else {
                     const int sr = src_row[rr];
-                    if (sr >= 0) {
-                        v = *reinterpret_cast<const uint4*>(p.src + static_cast<size_t>(sr) * p.K + kc + 8 * ch);
-                        uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const __half lo = to_half(static_cast<uint16_t>(w[q] & 0xFFFFu), p.src_bf16, st);
-                            const __half hi = to_half(static_cast<uint16_t>(w[q] >> 16), p.src_bf16, st);
-                            w[q] = static_cast<uint32_t>(__half_as_ushort(lo)) |
-                                   (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
-                        }
-                        v = make_uint4(w[0], w[1], w[2], w[3]);
-                    }
+                    if (sr >= 0)
+                        v = scale_pairs(*reinterpret_cast<const uint4*>(p.src + static_cast<size_t>(sr) * p.K + kc + 8 * ch),
+                                        p.src_bf16, src_scale[rr], st);
                     *reinterpret_cast<uint4*>(&xs[rr][8 * ch]) = v;
                 }
             }
@@ -377,7 +415,7 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
             const float v = ((part[0][rr][jj] + part[1][rr][jj]) + part[2][rr][jj]) + part[3][rr][jj];
             if (mt + rr < m && j0 + jj < span) {
                 const size_t o = static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j0 + jj;
-                if (single) p.t[o] = __half_as_ushort(__float2half_rn(j0 + jj < r ? v : 0.0f));
+                if (single) p.t[o] = t_half(j0 + jj < r ? v : 0.0f, st);
                 else out[o] = j0 + jj < r ? v : 0.0f;
             }
         }
@@ -401,10 +439,11 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
                 const size_t o = static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j0 + jj;
                 float v = 0.0f;
                 for (int sp = 0; sp < p.splits; ++sp) v += __ldcg(p.part + sp * slice + o);
-                p.t[o] = __half_as_ushort(__float2half_rn(v));
+                p.t[o] = t_half(v, st);
             }
         }
     if (threadIdx.x == 0) *ctr = 0;   // ready for the next launch
+    flag(p.dev_status, st);
 }
 
 // Many rows per expert (no K split): one block per (expert, projection, 64-row
@@ -420,6 +459,7 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
     __shared__ __align__(16) uint16_t xs[kLtRows][kLtPitch];
     __shared__ __align__(16) uint16_t vs[MILO_MAX_RANK][kLtPitch];
     __shared__ int src_row[kLtRows];
+    __shared__ float src_scale[kLtRows];
     const int nproj = p.proj_b >= 0 ? 2 : 1;
     const int which = blockIdx.x % nproj, e = blockIdx.x / nproj;
     const ProjDev* P = p.table + e * p.stride + (which == 0 ? p.proj_a : p.proj_b);
@@ -443,6 +483,7 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
         if (threadIdx.x < kLtRows) {
             const int i = threadIdx.x;
             src_row[i] = mt + i < m ? (p.row_src ? p.row_src[row0 + mt + i] : row0 + mt + i) : -1;
+            src_scale[i] = mt + i < m ? p.rscale[row0 + mt + i] : 1.0f;
         }
         __syncthreads();
         // this thread's share of a chunk: x rows (4 x 16 B) and V rows (4 x 16 B)
@@ -484,14 +525,7 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
             for (int q = 0; q < 4; ++q) {
                 const int i = threadIdx.x + 128 * q;
                 const int rr = i >> 3, pc = i & 7;
-                uint32_t w[4] = {xr[q].x, xr[q].y, xr[q].z, xr[q].w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const __half lo = to_half(static_cast<uint16_t>(w[u] & 0xFFFFu), p.src_bf16, st);
-                    const __half hi = to_half(static_cast<uint16_t>(w[u] >> 16), p.src_bf16, st);
-                    w[u] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
-                }
-                *reinterpret_cast<uint4*>(&xs[rr][8 * pc]) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4*>(&xs[rr][8 * pc]) = scale_pairs(xr[q], p.src_bf16, src_scale[rr], st);
                 if (!P->lorc3) *reinterpret_cast<uint4*>(&vs[rr][8 * pc]) = vr[q];
             }
             if (P->lorc3) {
@@ -538,8 +572,7 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
             for (int i = 0; i < 4; ++i) {
                 const int rr = 16 * warp + g + 8 * (i >> 1), j = 8 * n + 2 * c + (i & 1);
                 if (mt + rr < m && j < span)
-                    p.t[static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j] =
-                        __half_as_ushort(__float2half_rn(j < r ? acc[n][i] : 0.0f));
+                    p.t[static_cast<size_t>(row0 + mt + rr) * p.tcols + col0 + j] = t_half(j < r ? acc[n][i] : 0.0f, st);
             }
     }
     flag(p.dev_status, st);

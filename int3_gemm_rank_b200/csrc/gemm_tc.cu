@@ -14,8 +14,9 @@
 //     stage of each super-block pair, the pair's group-sum tile.
 //   - Four extraction warps (one thread per weight row) turn the row's 32
 //     code pairs into exact fp16 patterns code * 2^e * 2^-24 (one LOP3 per
-//     pair, the 2^e folded into the activations) and store them to TMEM: the
-//     A operand.  They also write -s_g * z_g of the row's groups, split into
+//     pair; the activations carry 2^(6 - e) and their row's scale 2^a) and
+//     store them to TMEM: the A operand.  They also write -s_g * z_g of the
+//     row's groups, times a power of two of the row (zp_scale) and split into
 //     fp16 hi + lo, to shared memory (32-byte swizzle).
 //   - The MMA warp issues tcgen05.mma M=128, N=kTcTok, K=16 (one elected lane)
 //     with A from TMEM and B from shared memory, per 64-code scale group into
@@ -23,10 +24,11 @@
 //     zero-point step Z += (-s z)_hi,lo x (X_g)_hi,lo over the pair's four
 //     groups (four K slots each: the four hi/lo cross products).
 //   - Eight fold warps (two per weight row: kTcTok / 2 routed rows and fp32
-//     accumulators each) read D_g and fold acc += s * 2^24 * D_g (packed
-//     FFMA2), then add Z once per item, so the scale and the zero point cost
-//     no per-weight work; -s z splits exactly, X_g to 2^-22 relative, and
-//     the rest is fp32 accumulation.
+//     accumulators each) read D_g and fold acc += s * 2^18 * D_g (packed
+//     FFMA2), then add Z once per item and multiply each routed row by its
+//     2^-a, so the scale and the zero point cost no per-weight work; -s z
+//     splits exactly, X_g to 2^-22 relative, and the rest is fp32
+//     accumulation.
 //   - The compensator is one more stage: A = U rows, B = t = x V^T.
 //   - Epilogue: SwiGLU through a shared-memory exchange between the w1 and w3
 //     rows of each output feature (each side finishes half the tokens), or
@@ -34,6 +36,8 @@
 //   - Every wait is bounded; on a timeout the kernel flags MILO_DEV_TIMEOUT,
 //     drains its copies and MMAs and frees TMEM before leaving.
 #include <cuda_runtime.h>
+
+#include <atomic>
 
 #include "milo_device.cuh"
 #include "milo_host.h"
@@ -154,6 +158,17 @@ __device__ __forceinline__ uint32_t lorc3_value_pair(const uint8_t* blk, int rho
     }
     return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[0]))) |
            (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[1]))) << 16);
+}
+
+// Power of two 2^c that brings a weight row's first group scale s into
+// [2^-3, 2^-2).  The zero-point operand -s z 2^c of each of the row's groups
+// (|s z| <= 7 s for codes 0..7) then splits into normal fp16 hi + lo however
+// small the weights are; the fold multiplies the row's Z by 2^-c.  Extraction
+// and fold warps derive it from the same s; 1 for a zero row.
+__device__ __forceinline__ float zp_scale(float s) {
+    const uint32_t b = __float_as_uint(s);
+    if (!(s > 0.0f) || b >= 0x7F800000u) return 1.0f;
+    return __uint_as_float(static_cast<uint32_t>(127 + 124 - static_cast<int>(b >> 23)) << 23);
 }
 
 // A fold warp reads its kTcHalf accumulator columns in chunks of kTcChunk
@@ -425,6 +440,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         bool fail = false;
         int32_t st_bits = 0;
         uint4 zprev = make_uint4(0u, 0u, 0u, 0u);   // A_z slots of the pair's first super-block
+        float zsc = 1.0f;                           // the item's zero-point scale 2^c of this row
         for (int it = blockIdx.x; it < n_items && !fail; it += gridDim.x) {
             const TcItem w = tc_decode(it, start, cnt, p.n_exp, n_tiles, p.ntile_fast);
             const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
@@ -452,8 +468,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 for (int h = 0; h < 2; ++h) {
                     const uint32_t szv = *reinterpret_cast<const uint32_t*>(
                         st + kTcOffW + half * kBlockSB + kQTileSBWords * 4 + h * kGroupBytes + pair_off);
-                    const float c = live ? -__half2float(__ushort_as_half(static_cast<uint16_t>(szv & 0xFFFFu))) *
-                                               __half2float(__ushort_as_half(static_cast<uint16_t>(szv >> 16)))
+                    const float sv = __half2float(__ushort_as_half(static_cast<uint16_t>(szv & 0xFFFFu)));
+                    if (b == 0 && h == 0) zsc = zp_scale(sv);
+                    const float c = live ? -(sv * __half2float(__ushort_as_half(static_cast<uint16_t>(szv >> 16)))) * zsc
                                          : 0.0f;
                     const __half hi = __float2half_rn(c);
                     const __half lo = __float2half_rn(c - __half2float(hi));
@@ -576,6 +593,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             const int row0 = row0s[w.e] + w.tt * kTcTok;
             const int ntok = min(kTcTok, cnt[w.e] - w.tt * kTcTok);
             float2 acc[kTcHalf / 2];      // routed rows kTcHalf * th + 2i, +1
+            float zinv = 1.0f;            // 2^-c of the row's zero-point scale (zp_scale)
 #pragma unroll
             for (int i = 0; i < kTcHalf / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
 
@@ -587,10 +605,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 const uint8_t* st = smem + stage * kTcStage;
                 float s24[2];
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-                    s24[h] = 16777216.0f * __half2float(*reinterpret_cast<const __half*>(
-                                               st + kTcOffW + half * kBlockSB + kQTileSBWords * 4 + h * kGroupBytes +
-                                               pair_off));
+                for (int h = 0; h < 2; ++h) {
+                    const float sv = __half2float(*reinterpret_cast<const __half*>(
+                        st + kTcOffW + half * kBlockSB + kQTileSBWords * 4 + h * kGroupBytes + pair_off));
+                    if (b == 0 && h == 0) zinv = inv_pow2(zp_scale(sv));
+                    s24[h] = kFoldScale * sv;
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[stage]);
                 if (++stage == kTcStages) { stage = 0; phase ^= 1; }
@@ -624,8 +644,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 if (fail) break;
             }
             if (fail) break;
-            // the zero-point sums Z = sum_g (-s_g z_g) X_g: the last D_g's commit
-            // covered the item's last zero-point step
+            // the zero-point sums Z = 2^c sum_g (-s_g z_g) X_g: the last D_g's
+            // commit covered the item's last zero-point step
 #pragma unroll
             for (int j = 0; j < kTcChunks; ++j) {
                 uint32_t d[kTcChunk];
@@ -633,8 +653,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 tc_wait_ld();
 #pragma unroll
                 for (int i = 0; i < kTcChunk / 2; ++i) {
-                    acc[kTcChunk / 2 * j + i].x += __uint_as_float(d[2 * i]);
-                    acc[kTcChunk / 2 * j + i].y += __uint_as_float(d[2 * i + 1]);
+                    acc[kTcChunk / 2 * j + i].x = fmaf(__uint_as_float(d[2 * i]), zinv, acc[kTcChunk / 2 * j + i].x);
+                    acc[kTcChunk / 2 * j + i].y = fmaf(__uint_as_float(d[2 * i + 1]), zinv, acc[kTcChunk / 2 * j + i].y);
                 }
             }
             tc_fence_before();
@@ -670,6 +690,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&dempty[db]);
                 if (++db == kTcDBufs) { db = 0; dph ^= 1; }
+            }
+
+            // undo the rows' scale 2^a: token kTcHalf * th + 32 u + lane's scale
+            // in register u of that lane, broadcast to the whole warp
+            {
+                float sc[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int t = kTcHalf * th + 32 * u + lane;
+                    sc[u] = t < ntok ? inv_pow2(p.rscale[row0 + t]) : 0.0f;
+                }
+#pragma unroll
+                for (int i = 0; i < kTcHalf / 2; ++i) {
+                    const float s0 = __shfl_sync(0xFFFFFFFFu, sc[(2 * i) >> 5], (2 * i) & 31);
+                    const float s1 = __shfl_sync(0xFFFFFFFFu, sc[(2 * i + 1) >> 5], (2 * i + 1) & 31);
+                    acc[i].x *= s0;
+                    acc[i].y *= s1;
+                }
             }
 
             // ------------------------------------------------------------ epilogue
@@ -753,15 +791,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 size_t tc_smem_bytes() { return kTcSmemBytes; }
 
 cudaError_t launch_tc_gemm(const TcParams& p, bool glu, int grid, cudaStream_t s) {
-    static bool configured[64][2] = {};
+    static std::atomic<bool> configured[64][2];   // set once per device and kernel (a repeat is harmless)
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !configured[dev][glu]) {
+    if (dev < 0 || dev >= 64 || !configured[dev][glu].load(std::memory_order_acquire)) {
         e = glu ? cudaFuncSetAttribute(tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes)
                 : cudaFuncSetAttribute(tc_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) configured[dev][glu] = true;
+        if (dev >= 0 && dev < 64) configured[dev][glu].store(true, std::memory_order_release);
     }
     // normal stream ordering, like the other persistent GEMM
     if (glu) tc_gemm_kernel<true><<<grid, kTcThreads, kTcSmemBytes, s>>>(p);

@@ -23,11 +23,13 @@
 //   - Four consumer warps each own 32 weight rows.  A lane reads its 3-word
 //     unit of two rows and extracts code pairs with one LOP3 each (plus one
 //     shift per word): the masked fp16 pattern already is code * 2^e * 2^-24,
-//     and the power of 2 is folded into the activations, which are shared by
-//     all rows.  mma.sync m16n8k16 (A = codes, B = tokens) accumulates
-//     D_g = 2^-24 * sum_k x_k q_k per scale group g; after each group the lane
-//     folds  acc += s * 2^24 * D_g - s * z * sum_k x_k  in fp32.  The zero point
-//     thus costs nothing per weight and the result is exact to fp32 rounding.
+//     and 2^(6 - e) is folded into the activations, which are shared by all
+//     rows (as is the row's own scale 2^a, see kFoldScale).  mma.sync m16n8k16
+//     (A = codes, B = tokens) accumulates D_g = 2^-18 * sum_k x'_k q_k per
+//     scale group g; after each group the lane folds
+//     acc += s * 2^18 * D_g - s * z * sum_k x'_k  in fp32, and the epilogue
+//     multiplies by 2^-a.  The zero point thus costs nothing per weight and
+//     the result is exact to fp32 rounding.
 //   - The compensator runs as extra K-steps on the same accumulators:
 //     A = U rows (fp16), B = t = x V^T (fp16, computed beforehand per expert).
 //   - Epilogue: SwiGLU h = silu(a) * b in the w1|w3 kernel (both rows live in
@@ -41,6 +43,8 @@
 //     The consumers learn each item from a header the producer writes into
 //     the item's first stage.
 #include <cuda_runtime.h>
+
+#include <atomic>
 
 #include "milo_device.cuh"
 #include "milo_host.h"
@@ -136,7 +140,7 @@ struct TileMap {
     }
 };
 
-// acc += s * 2^24 * D_g - s * z * X_g for group `grp` (0..3) of the chunk;
+// acc += s * 2^18 * D_g - s * z * X_g for group `grp` (0..3) of the chunk;
 // super-block grp / 2's scales follow its codes, as (s, z) pairs of rows j and
 // j + 8 of each 16-row block, so one 64-bit load brings the lane's two rows.
 // xg[n8][j]: X_g of its tokens.
@@ -154,7 +158,7 @@ __device__ __forceinline__ void fold_group(float (&acc)[2][2][4], const float (&
             const uint32_t v = rr ? q.y : q.x;
             const float sv = __half2float(__ushort_as_half(static_cast<uint16_t>(v & 0xFFFFu)));
             const float zv = __half2float(__ushort_as_half(static_cast<uint16_t>(v >> 16)));
-            s24[rr] = sv * 16777216.0f;
+            s24[rr] = sv * kFoldScale;
             nsz[rr] = -sv * zv;
         }
 #pragma unroll
@@ -523,6 +527,15 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         }
 
         // ------------------------------------------------------------ epilogue
+        // the lane's tokens n8 * 8 + 2c + j: undo their rows' scale 2^a
+        float inv[2][2];
+#pragma unroll
+        for (int n8 = 0; n8 < 2; ++n8)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int tok = n8 * 8 + 2 * c + j;
+                inv[n8][j] = tok < ntok ? inv_pow2(p.rscale[row0 + tok]) : 0.0f;
+            }
         if constexpr (GLU) {
             int32_t st = 0;
 #pragma unroll
@@ -532,7 +545,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                     const int f = n0 + 16 * warp + g + 8 * (i >> 1);
                     const int tok = n8 * 8 + 2 * c + (i & 1);
                     if (tok < ntok && f < p.N) {
-                        const float a = acc[0][n8][i], b = acc[1][n8][i];
+                        const float a = acc[0][n8][i] * inv[n8][i & 1], b = acc[1][n8][i] * inv[n8][i & 1];
                         const float hv = __fdividef(a, 1.0f + __expf(-a)) * b;
                         const __half hh = __float2half_rn(hv);
                         if (!isfinite(hv)) st |= MILO_DEV_NONFINITE;
@@ -552,7 +565,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                         const int n = n0 + 32 * warp + 16 * ti + g + 8 * (i >> 1);
                         const int tok = n8 * 8 + 2 * c + (i & 1);
                         if (tok < ntok && n < p.N)
-                            out[static_cast<size_t>(row0 + tok) * p.N + n] = acc[ti][n8][i];
+                            out[static_cast<size_t>(row0 + tok) * p.N + n] = acc[ti][n8][i] * inv[n8][i & 1];
                     }
         }
     }
@@ -562,15 +575,15 @@ size_t gemv_smem_bytes(bool) { return kSmemBytes; }
 
 cudaError_t launch_gemv(const GemvParams& p, bool glu, int grid, cudaStream_t s) {
     // The shared-memory opt-in is a per-device function attribute.
-    static bool configured[64][2] = {};
+    static std::atomic<bool> configured[64][2];   // set once per device and kernel (a repeat is harmless)
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !configured[dev][glu]) {
+    if (dev < 0 || dev >= 64 || !configured[dev][glu].load(std::memory_order_acquire)) {
         e = glu ? cudaFuncSetAttribute(gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)
                 : cudaFuncSetAttribute(gemv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) configured[dev][glu] = true;
+        if (dev >= 0 && dev < 64) configured[dev][glu].store(true, std::memory_order_release);
     }
     // A normal launch: the persistent grid starts once the previous kernel has
     // left every SM, so its CTAs are spread evenly over the SMs (an early,

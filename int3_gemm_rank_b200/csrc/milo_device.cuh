@@ -40,18 +40,35 @@ __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol
 // conversions
 // ---------------------------------------------------------------------------
 
-// Activation element -> fp16, round to nearest even.  bf16 values between
-// 2^-17 and 65504 in magnitude convert exactly; larger ones set FP16_RANGE.
-__device__ __forceinline__ __half to_half(uint16_t bits, bool is_bf16, int32_t& st) {
-    float f;
-    if (is_bf16) {
-        f = __uint_as_float(static_cast<uint32_t>(bits) << 16);
-    } else {
-        f = __half2float(__ushort_as_half(bits));
-    }
+// Activation element (fp16 or bf16 bits) as f32, exactly.
+__device__ __forceinline__ float act_f32(uint16_t bits, bool is_bf16) {
+    return is_bf16 ? __uint_as_float(static_cast<uint32_t>(bits) << 16) : __half2float(__ushort_as_half(bits));
+}
+
+// Activation element times its row's scale 2^a, rounded to fp16 (nearest
+// even).  The product is exact in f32; the rounding keeps every bit of an
+// fp16 or bf16 element down to 2^-17 of the row's largest magnitude, and the
+// scaled values are below 2 (FP16_RANGE guards a scale that does not match).
+__device__ __forceinline__ __half to_half_scaled(uint16_t bits, bool is_bf16, float scale, int32_t& st) {
+    const float f = act_f32(bits, is_bf16) * scale;
     if (!isfinite(f)) st |= MILO_DEV_NONFINITE;
     else if (fabsf(f) > 65504.0f) st |= MILO_DEV_FP16_RANGE;
     return __float2half_rn(f);
+}
+
+// The row scale 2^a for a row whose largest magnitude is `mx` (f32 bits of a
+// non-negative value): max * 2^a in [1, 2), a clamped to [-126, 126] so that
+// 2^a and 2^-a are normal floats; 1 for a zero or non-finite maximum.
+__device__ __forceinline__ float row_scale_for(uint32_t mx_bits) {
+    if (mx_bits == 0u || mx_bits >= 0x7F800000u) return 1.0f;
+    int a = 127 - static_cast<int>(mx_bits >> 23);     // a subnormal maximum (exponent field 0) clamps
+    a = a < -126 ? -126 : (a > 126 ? 126 : a);
+    return __uint_as_float(static_cast<uint32_t>(127 + a) << 23);
+}
+
+// 2^-a from 2^a (both normal powers of two): exact.
+__device__ __forceinline__ float inv_pow2(float s) {
+    return __uint_as_float(0x7F000000u - __float_as_uint(s));
 }
 
 // ---------------------------------------------------------------------------
@@ -113,13 +130,16 @@ __host__ __device__ constexpr int reg_code(int t, int f) { return f < 5 ? 10 * t
 __host__ __device__ constexpr int unit_k(int c, int m) {
     return m < 16 ? 16 * c + m : 64 + 16 * c + (m - 16);
 }
-// Power of 2 left in the extracted value of register (word t, field f), and
-// its inverse, which multiplies the activation paired with it.
+// Power of 2 left in the extracted value of register (word t, field f), 2^e
+// with e <= 6, and the factor 2^(6 - e) >= 1 that multiplies the activation
+// paired with it, so that every product carries the same 2^6 (undone with
+// the 2^-24 of the fp16 pattern by kFoldScale = 2^18).  Scaling up keeps
+// fp16 activations exact, subnormal ones included.
 __host__ __device__ constexpr int field_shift(int t, int f) {
     return f == 0 ? 0 : f == 1 ? 3 : f == 2 ? 6 : f == 3 ? t : f == 4 ? 3 + t : 6;
 }
 __host__ __device__ constexpr float act_scale(int t, int f) {
-    return 1.0f / static_cast<float>(1 << field_shift(t, f));
+    return static_cast<float>(1 << (6 - field_shift(t, f)));
 }
 
 // ---------------------------------------------------------------------------

@@ -21,6 +21,16 @@ constexpr int kChunkK = 256;       // K per pipeline stage (two 128-code super-b
 // so that the rows of a 16-row tile fall on different shared-memory banks
 // (row pitch 136 words, 8 mod 32): 272 fp16 (544 bytes).
 // The first 8 padding fp16 hold the chunk's four group sums (f32).
+//
+// Row scaling: every activation row v (an x row or an h row) is multiplied by
+// a power of two 2^a chosen from its largest magnitude (max |v| 2^a in [1, 2))
+// before it is rounded to fp16, so that small rows keep their precision and
+// large ones fit; the power of two of the int3 field it meets is then applied
+// upwards (x 2^(6 - e), exact: the values stay below 2^7).  The products in
+// the MMA are thus 2^a * 2^-18 * v * code, the group sums are sums of
+// fp16(v 2^a), the compensator's t = fp16(2^a v V^T), and the GEMM epilogue
+// multiplies the row's result by 2^-a.  Both factors are exact.
+constexpr float kFoldScale = 262144.0f;   // 2^18: undoes the 2^-18 of the code operand
 constexpr int kFragHalvesPerSB = 128;
 constexpr int kFragRowHalves = 2 * kFragHalvesPerSB + 16;
 constexpr int kGsumHalf = 2 * kFragHalvesPerSB;
@@ -46,7 +56,8 @@ struct alignas(64) ProjDev {
 struct GemvParams {
     const uint16_t* x;          // prepared activations [chunks][R][kFragRowHalves] fp16
                                 // (group sums in each row's padding, see kGsumHalf)
-    const uint16_t* t;          // LoRC down-projection [R][tcols] fp16
+    const float* rscale;        // [R]: the row's activation scale 2^a (see kFoldScale)
+    const uint16_t* t;          // LoRC down-projection [R][tcols] fp16 (times the row's 2^a)
     const ProjDev* table;       // device table
     const int32_t* grp;         // [n_exp][2]: first row, row count of each group (expert)
     float* y_part;              // plain: [splits][R][N] f32 partial sums
@@ -65,6 +76,7 @@ struct TcParams {
     CUtensorMap b_map;          // activations [R][K] fp16, box {64, kTcTokens}, 128-byte swizzle
     CUtensorMap z_map;          // group sums [R][chunks][16] fp16 (hi, lo, hi, lo per group), box {16, kTcTokens}
     CUtensorMap t_map;          // LoRC down-projection [R][tcols] fp16, box {64, kTcTokens}, 128-byte swizzle
+    const float* rscale;        // [R]: the row's activation scale 2^a
     const ProjDev* table;
     const int32_t* grp;
     float* y_part;              // plain: [R][N] f32
@@ -84,6 +96,7 @@ struct PrepParams {
     uint16_t* frag;             // layout 0: [chunks][R][kFragRowHalves] fp16, chunks = ceil(K/256);
                                 // layout 1: [R][K] fp16 in tcgen05 A-column order
     uint16_t* gsum;             // layout 1: group sums [R][chunks][16] fp16: per group (hi, lo, hi, lo)
+    float* rscale;              // [R]: written, the row's scale 2^a (1 for a zero row)
     int layout;
     int32_t* dev_status;
     int R, K, src_bf16;
@@ -102,9 +115,10 @@ struct PrepParams {
 struct LorcParams {
     const uint16_t* src;        // [*, K] bf16/fp16 rows
     const int32_t* row_src;     // row p -> source row (NULL: identity); -1 = zero row
+    const float* rscale;        // [R]: the row's activation scale 2^a (written by prep)
     const ProjDev* table;
     const int32_t* grp;         // [n_exp][2]
-    uint16_t* t;                // [R, tcols] fp16
+    uint16_t* t;                // [R, tcols] fp16: 2^a x V^T
     float* part;                // [splits][R][tcols] f32 partial sums over K slices
     int32_t* done;              // per (expert, projection, rank block, row group): slices finished; 0 on entry
     int32_t* dev_status;

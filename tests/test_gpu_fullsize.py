@@ -9,8 +9,9 @@ times (same entry points, same workspace sizing):
 * w1 batch sweep with Zipf routing, T = 1 ... 1024: all rows up to 64 tokens,
   a seeded sample of rows beyond;
 * Mixtral-shaped prefill (8192 tokens, rank 64): routing bit-exact for all
-  tokens, layer outputs on a seeded sample of tokens (tokens are independent
-  in an MoE layer, so the oracle runs the sampled tokens alone).
+  tokens, layer outputs and SwiGLU activations on at least 256 tokens that
+  reach every (expert, 128-row tile) of both grouped GEMMs (tokens are
+  independent in an MoE layer, so the oracle runs the sampled tokens alone).
 """
 from concurrent.futures import ThreadPoolExecutor
 
@@ -139,7 +140,28 @@ def test_w1_sweep_zipf(milo):
         assert err <= REL_TOL, (T, err)
 
 
+def prefill_sample(off: np.ndarray, perm: np.ndarray, k: int, T: int, tile: int = 128,
+                   at_least: int = 256, seed: int = 55) -> np.ndarray:
+    """Tokens whose rows reach every work item of the grouped GEMMs: for each
+    expert, the first and the last routed row of each of its `tile`-row
+    tiles (the ragged last tile included), the first and the last token, then
+    seeded random tokens up to `at_least`."""
+    tok = {0, T - 1}
+    for e in range(off.size - 1):
+        for p0 in range(int(off[e]), int(off[e + 1]), tile):
+            p1 = min(p0 + tile, int(off[e + 1])) - 1
+            tok.add(int(perm[p0]) // k)
+            tok.add(int(perm[p1]) // k)
+    rng = np.random.default_rng(seed)
+    while len(tok) < at_least:
+        tok.add(int(rng.integers(T)))
+    return np.array(sorted(tok))
+
+
 def test_mixtral_prefill_sampled(milo):
+    """8192 tokens on the tcgen05 path: every output feature and every SwiGLU
+    activation of the sampled tokens, the sample reaching every (expert,
+    128-row tile) of both grouped GEMMs at its first and last row."""
     wk = wl.prefill()
     layer, ref = _layers(milo, wk)
     r, ids, w, inv = _route(milo, wk)
@@ -147,8 +169,21 @@ def test_mixtral_prefill_sampled(milo):
     y = layer(act_dev(wk.x, wk.x_dtype), r, out_dtype=torch.float32, dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    tok = np.sort(np.random.default_rng(55).choice(wk.T, size=16, replace=False))
-    y_ref, _, _ = oracle.moe_forward(wk.x[tok], True, ids[tok], w[tok], ref, wk.n_routed,
-                                     wk.n_shared, wk.hidden, wk.inter)
+    off, perm = r["offsets"].cpu().numpy(), r["perm"].cpu().numpy()
+    tok = prefill_sample(off, perm, wk.top_k, wk.T)
+    assert tok.size >= 256
+    covered = {(e, (int(inv[t * wk.top_k + j]) - int(off[e])) // 128)
+               for t in tok for j in range(wk.top_k) for e in [int(ids[t, j])]}
+    every = {(e, q) for e in range(wk.n_routed) for q in range((int(off[e + 1] - off[e]) + 127) // 128)}
+    assert covered == every
+    y_ref, h_ref, st_ref = oracle.moe_forward(wk.x[tok], True, ids[tok], w[tok], ref, wk.n_routed,
+                                              wk.n_shared, wk.hidden, wk.inter, want_h=True)
+    assert st_ref == 0
     err = rel_err(y.cpu().numpy()[tok], y_ref)
     assert err <= REL_TOL, err
+    # h rows of the sampled slots: GPU row inv[t k + j] against the oracle's slot i k + j
+    h = layer.h_view(wk.T).cpu().numpy().view(np.uint16)
+    rows = np.array([inv[t * wk.top_k + j] for t in tok for j in range(wk.top_k)])
+    h_gpu = h[rows].view(np.float16).astype(np.float64)
+    herr = rel_err(h_gpu, h_ref.view(np.float16).astype(np.float64))
+    assert herr <= REL_TOL, herr

@@ -31,11 +31,12 @@ def milo():
 
 
 @pytest.fixture(params=["mma", "tc"])
-def gemm_path(request, monkeypatch):
+def gemm_path(request, milo):
     """Run a test on the mma.sync grouped GEMM (chosen for few rows per expert)
     and on the tcgen05 one (chosen for many)."""
-    monkeypatch.setenv("MILO_GEMM", request.param)
-    return request.param
+    milo.milo_set_gemm_path(request.param)
+    yield request.param
+    milo.milo_set_gemm_path("auto")
 
 
 def _status(st):
@@ -227,13 +228,21 @@ def test_linear_bad_ids_dropped_and_zero(milo, gemm_path):
     assert rel_err(y[2], oracle.linear(X[2:], ref[1])[0]) <= REL_TOL
 
 
-def test_linear_flags_fp16_range(milo):
+def test_linear_large_bf16_rows_and_fp16_output_range(milo):
+    """bf16 activations of 1e6 (beyond fp16) are valid input: the f32 result
+    matches the oracle; the same result requested as fp16 overflows, which
+    sets FP16_RANGE."""
     projs = [wl.make_projection("t_rng", "w", 0, 128, 128, 0)]
-    lin, _ = _linear_pair(milo, projs)
+    lin, ref = _linear_pair(milo, projs)
     x = wl.f32_to_bf16_bits(np.full((1, 128), 1.0e6, np.float32))
     r = milo.milo_route(None, 1, False, E=1, ids=to_dev(np.zeros((1, 1), np.int32)))
     st = milo.new_status()
-    lin(act_dev(x, "bf16"), r["offsets"], r["perm"], k=1, dev_status=st)
+    y = lin(act_dev(x, "bf16"), r["offsets"], r["perm"], k=1, dev_status=st)
+    assert _status(st) == 0
+    y_ref = oracle.linear(act_f64(x, "bf16"), ref[0])
+    assert rel_err(y.cpu().numpy(), y_ref) <= REL_TOL
+    assert np.abs(y_ref).max() > 65504
+    lin(act_dev(x, "bf16"), r["offsets"], r["perm"], k=1, out_dtype=torch.float16, dev_status=st)
     assert _status(st) & milo.MILO_DEV_FP16_RANGE
 
 
