@@ -433,10 +433,11 @@ def run_milo(args):
             milo._check(s, "milo_route")
         milo.milo_moe_forward(layer, xin, route, out_dtype=out_dt, dev_status=st, y=y, ws=ws)
 
-    # route (one kernel; from 512 tokens on a top-k kernel first), prep x, lorc w1|w3, gemm w1|w3,
-    # prep h, lorc w2, gemm w2, combine; the compensator launches drop out when no expert has one
+    # route (one kernel; from 512 tokens on a top-k kernel first), then the forward:
+    # mma.sync path: prep x, gemm w1|w3 (compensator inside), prep h, gemm w2 (compensator and
+    # combine inside); tcgen05 path: prep x, lorc w1|w3, gemm w1|w3, prep h, lorc w2, gemm w2,
+    # combine, the compensator launches dropping out when no expert has one
     has_lorc = any(wk.experts[e][n].rank for e in range(wk.n_experts) for n in ("w1", "w3", "w2"))
-    launches_per_step = (7 if has_lorc else 5) + (2 if T >= 512 else 1)
 
     # --- correctness gate on the bench configuration itself
     step(x, logits)
@@ -445,6 +446,8 @@ def run_milo(args):
         raise RuntimeError(f"device status {int(st.item())} on the bench workload")
     counts = np.diff(off.cpu().numpy())
     bytes_ = layer_bytes(wk, counts, args.lorc == "int3")
+    forward = (7 if has_lorc else 5) if uses_tensor_path(bytes_) else 5
+    launches_per_step = forward + (2 if T >= 512 else 1)
 
     # --- the timed step: one CUDA graph of the whole step (route + layer), its
     # launches and their programmatic dependencies captured once and replayed
@@ -671,7 +674,9 @@ def run_sweep(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     pk = peaks()
-    launches_per_call = 4 if any(P.rank for P in (base.experts[e]["w1"] for e in range(base.n_routed))) else 3
+    # prep and the grouped GEMM (compensator and combine inside) on the mma.sync path; prep,
+    # compensator down-projection, grouped GEMM and combine on the tcgen05 path
+    has_lorc = any(P.rank for P in (base.experts[e]["w1"] for e in range(base.n_routed)))
     points, launches = [], 0
     sampler = ClockSampler(local)
     sampler.start()
@@ -688,17 +693,20 @@ def run_sweep(args):
 
         for _ in range(args.warmup):
             call()
+        # the timed call is one CUDA graph (its launches back to back on the
+        # device, as in a decode loop); the flush before it is not timed
+        graph_call = capture_step(torch, dev, call)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(4 * args.steps)]
         for e in ev:            # torch creates the CUDA event on its first record
             e.record(stream)
         milo.milo_set_profile_events(None)
         barrier(dev)
         torch.cuda.synchronize()
-        # pass 1: the whole call (prep, compensator, GEMM, combine), no event inside it
+        # pass 1: the whole call (all its kernels), no event inside it
         for i in range(args.steps):
             flush.zero_()
             ev[4 * i].record(stream)
-            call()
+            graph_call()
             ev[4 * i + 1].record(stream)
         torch.cuda.synchronize()
         # pass 2: events around the grouped GEMM launch alone
@@ -708,7 +716,6 @@ def run_sweep(args):
             call()
         torch.cuda.synchronize()
         milo.milo_set_profile_events(None)
-        launches += 2 * args.steps * launches_per_call
         call_ms = max_over_ranks(statistics.mean(ev[4 * i].elapsed_time(ev[4 * i + 1])
                                                  for i in range(args.steps)), dev)
         gemm_ms = statistics.mean(ev[4 * i + 2].elapsed_time(ev[4 * i + 3]) for i in range(args.steps))
@@ -716,6 +723,7 @@ def run_sweep(args):
         cost = sweep_cost(wk, counts)
         forced = os.environ.get("MILO_GEMM", "")
         tensor = forced == "tc" if forced in ("mma", "tc") else T >= 64 * base.n_routed
+        launches += 2 * args.steps * ((4 if has_lorc else 3) if tensor else 3)
         gbs = cost["bytes"] / (call_ms / 1e3) / 1e9
         tflops = cost["flops"] / (call_ms / 1e3) / 1e12
         points.append({"tokens": T, "kernel": "tc_gemm_kernel (tcgen05)" if tensor else "gemv_kernel (mma.sync)",
@@ -737,6 +745,8 @@ def run_sweep(args):
                                f"{int(base.ranks[0])}, int3 g64, k = 1 with Zipf(1.1) expert ids, x bf16, y fp32; "
                                f"value and ms_per_step at {top['tokens']} tokens, every size under 'sweep'",
                    "l2": "flushed by a 256 MB write before every timed call",
+                   "launch": "each timed call one CUDA graph replay; gemm_us from a second pass of stream "
+                             "launches with events around the grouped GEMM",
                    "parallelism": f"replica per GPU x{world}"},
         "sweep": points,
         "roofline": ({"bound": "tensor", "achieved": top["tflops"], "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
@@ -813,7 +823,7 @@ def run_single(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     K = args.steps
-    launches_per_call = 4          # prep, compensator down-projection, grouped GEMM, per-slot combine
+    launches_per_call = 3          # prep, grouped GEMM (compensator inside), per-slot combine
 
     def calls(xin, base=0):
         for j in range(K):

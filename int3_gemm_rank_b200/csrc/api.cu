@@ -4,8 +4,12 @@
 // The sequence for one MoE layer ("MiLo: Efficient Quantized MoE Inference
 // with Mixture of Low-Rank Compensators": routed experts, each a quantised
 // weight plus a rank-r compensator, outputs mixed by the router weights):
-//   prep(x, row bookkeeping) -> lorc(x, V1|V3) -> gemv<SwiGLU>(w1|w3)
-//        -> prep(h) -> lorc(h, V2) -> gemv(w2) -> combine
+//   few rows per expert (mma.sync GEMMs):
+//     prep(x, row bookkeeping) -> gemv<SwiGLU>(w1|w3, t = x V1|V3^T inside)
+//        -> prep(h) -> gemv(w2, t = h V2^T inside, combine inside)
+//   many rows per expert (tcgen05 GEMMs):
+//     prep(x, row bookkeeping) -> lorc(x, V1|V3) -> tc<SwiGLU>(w1|w3)
+//        -> prep(h) -> lorc(h, V2) -> tc(w2) -> combine
 // Every step is a kernel on the caller's stream; the host never waits.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -126,6 +130,36 @@ static milo_status upload(void* device_table, size_t table_bytes, const std::vec
     return check_cuda(cudaMemcpy(device_table, t.data(), need, cudaMemcpyHostToDevice), "table upload");
 }
 
+// Which grouped GEMM runs.  The mma.sync kernel suits a few routed rows per
+// expert (decode): a tcgen05.mma of N = 16 costs as much to issue as one of
+// N = 64.  With many rows per expert (prefill) the weights are reused across
+// 128-row tiles and the tcgen05 kernel takes over.  milo_set_gemm_path (or
+// MILO_GEMM=mma|tc in the environment, read once) forces one; both give the
+// same results within fp32 rounding.
+static std::atomic<int> g_gemm_path{-1};   // -1: not yet read from the environment
+
+static int gemm_path() {
+    int v = g_gemm_path.load(std::memory_order_relaxed);
+    if (v >= 0) return v;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const char* e = getenv("MILO_GEMM");
+        int m = MILO_GEMM_AUTO;
+        if (e && e[0] == 't') m = MILO_GEMM_TC;
+        else if (e && e[0] == 'm') m = MILO_GEMM_MMA;
+        int unset = -1;
+        g_gemm_path.compare_exchange_strong(unset, m);
+    });
+    return g_gemm_path.load(std::memory_order_relaxed);
+}
+
+static bool use_tc(long long routed_rows, int n_routed) {
+    const int path = gemm_path();
+    if (path == MILO_GEMM_TC) return true;
+    if (path == MILO_GEMM_MMA) return false;
+    return routed_rows >= 64LL * std::max(1, n_routed);
+}
+
 // ---------------------------------------------------------------------------
 // workspace layouts
 // ---------------------------------------------------------------------------
@@ -156,8 +190,9 @@ struct LorcPlan {
 static int lorc_counters(int n_exp) { return n_exp * 2 * ((MILO_MAX_RANK + 15) / 16) * 8; }
 
 struct LinearWs {
-    size_t grp, rows, inv, rscale, frag, gsum, t, tpart, done, part, total;
-    int R, splits, tcols;
+    size_t grp, rows, inv, rscale, frag, gsum, t, tpart, done, part, plain, total;
+    int R, splits, tcols, nzero;
+    bool tc;
     LorcPlan lp;
 };
 
@@ -199,10 +234,19 @@ static LorcPlan lorc_plan(int n_exp, int nproj, int K, long long max_rows) {
     return pl;
 }
 
+// K slices of the compensator's t-items inside the mma.sync GEMM: short
+// enough that all of a slice's loads are in flight at once (a lane loads 8
+// values per 32 of K), so that t is ready long before the first GEMM items
+// reach their compensator stage; longer for very long K, where the number of
+// slices to add up would grow.
+static int t_slice_len(int K) { return K <= 4096 ? 256 : 512; }
+static int t_slices(int K) { return (K + t_slice_len(K) - 1) / t_slice_len(K); }
+
 static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
     LinearWs w;
     Carve c;
     w.R = T * k;
+    w.tc = use_tc(static_cast<long long>(T) * k, lin->n_experts);
     const int n_exp = lin->n_experts;
     const int chunks = (lin->K + kChunkK - 1) / kChunkK;
     const long long groups = std::min<long long>(n_exp, std::max(1LL, static_cast<long long>(T) * k));
@@ -217,16 +261,22 @@ static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
     w.gsum = c.take(gsum_bytes(lin->K, w.R));
     w.t = c.take(static_cast<size_t>(w.R) * w.tcols * 2);
     w.lp = lorc_plan(n_exp, 1, lin->K, static_cast<long long>(T) * k);   // at most all rows in one expert
-    w.tpart = c.take(static_cast<size_t>(w.lp.splits) * w.R * w.tcols * 4);
-    w.done = c.take(static_cast<size_t>(lorc_counters(n_exp)) * 4);
+    // the tcgen05 path: the down-projection kernel's K slices; the mma.sync
+    // path: its t-items' K slices, the rows' plain copy, and their counters
+    const int tslices = w.tc ? w.lp.splits : t_slices(lin->K);
+    w.tpart = c.take(static_cast<size_t>(tslices) * w.R * w.tcols * 4);
+    w.nzero = lorc_counters(n_exp) + (w.tc ? 0 : gemv_sync_ints(w.R, n_exp, lin->N));
+    w.done = c.take(static_cast<size_t>(w.nzero) * 4);
     w.part = c.take(static_cast<size_t>(w.splits) * w.R * lin->N * 4);
+    w.plain = w.tc ? 0 : c.take(static_cast<size_t>(w.R) * lin->K * 2);
     w.total = c.off;
     return w;
 }
 
 struct MoeWs {
-    size_t grp, rows, xscale, xfrag, xg, t13, h, hscale, hfrag, hg, t2, tpart, done, part, total;
-    int R, R_routed, splits, tc13, tc2;
+    size_t grp, rows, xscale, xfrag, xg, t13, h, hscale, hfrag, hg, t2, tpart, done, part, xplain, hplain, total;
+    int R, R_routed, splits, tc13, tc2, nzero, sync13, sync2;
+    bool tc;
     LorcPlan lp13, lp2;
 };
 
@@ -236,6 +286,7 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
     const int H = L->hidden, I = L->inter;
     w.R_routed = T * L->top_k;
     w.R = w.R_routed + L->n_shared * T;
+    w.tc = use_tc(w.R_routed, L->n_routed);
     const int n_exp = L->n_routed + L->n_shared;
     const int chunks = (I + kChunkK - 1) / kChunkK;
     const long long groups = std::min<long long>(L->n_routed, std::max(1LL, static_cast<long long>(w.R_routed))) + L->n_shared;
@@ -256,10 +307,18 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
     // a token meets an expert at most once, and a shared expert sees every token
     w.lp13 = lorc_plan(n_exp, 2, H, T);
     w.lp2 = lorc_plan(n_exp, 1, I, T);
-    w.tpart = c.take(std::max(static_cast<size_t>(w.lp13.splits) * w.tc13,
-                              static_cast<size_t>(w.lp2.splits) * w.tc2) * w.R * 4);
-    w.done = c.take(static_cast<size_t>(lorc_counters(n_exp)) * 4);
+    // the down-projection kernels' slices (tcgen05 path) or the t-items' (mma.sync path)
+    const size_t s13 = w.tc ? w.lp13.splits : t_slices(H), s2 = w.tc ? w.lp2.splits : t_slices(I);
+    w.tpart = c.take(std::max(s13 * w.tc13, s2 * w.tc2) * w.R * 4);
+    // counters, all zeroed by the first preparation: the down-projection
+    // kernels', then (mma.sync path) those of the w1|w3 and w2 GEMMs
+    w.sync13 = w.tc ? 0 : gemv_sync_ints(w.R, n_exp, I);
+    w.sync2 = w.tc ? 0 : gemv_sync_ints(w.R, n_exp, H);
+    w.nzero = lorc_counters(n_exp) + w.sync13 + w.sync2;
+    w.done = c.take(static_cast<size_t>(w.nzero) * 4);
     w.part = c.take(static_cast<size_t>(w.splits) * w.R * H * 4);
+    w.xplain = w.tc ? 0 : c.take(static_cast<size_t>(w.R) * H * 2);
+    w.hplain = w.tc ? 0 : c.take(static_cast<size_t>(w.R) * I * 2);
     w.total = c.off;
     return w;
 }
@@ -270,7 +329,7 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
 static void act_ptrs(GemvParams& g, void* frag, void* rscale, void* t, int R, int K, int tcols, bool has_t) {
     g.x = static_cast<const uint16_t*>(frag);
     g.rscale = static_cast<const float*>(rscale);
-    g.t = has_t ? static_cast<const uint16_t*>(t) : nullptr;
+    g.t = has_t ? static_cast<uint16_t*>(t) : nullptr;
     g.R = R;
     g.K = K;
     g.SB = K / 128;
@@ -281,38 +340,21 @@ static void act_ptrs(GemvParams& g, void* frag, void* rscale, void* t, int R, in
 }
 
 static milo_status run_gemv(GemvParams& g, bool glu, cudaStream_t st, const char* what) {
-    const int grid = 3 * sm_count();
-    return check_cuda(launch_gemv(g, glu, grid, st), what);
+    return check_cuda(launch_gemv(g, glu, sm_count(), st), what);
 }
 
-// Which grouped GEMM runs.  The mma.sync kernel suits a few routed rows per
-// expert (decode): a tcgen05.mma of N = 16 costs as much to issue as one of
-// N = 64.  With many rows per expert (prefill) the weights are reused across
-// 128-row tiles and the tcgen05 kernel takes over.  milo_set_gemm_path (or
-// MILO_GEMM=mma|tc in the environment, read once) forces one; both give the
-// same results within fp32 rounding.
-static std::atomic<int> g_gemm_path{-1};   // -1: not yet read from the environment
-
-static int gemm_path() {
-    int v = g_gemm_path.load(std::memory_order_relaxed);
-    if (v >= 0) return v;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        const char* e = getenv("MILO_GEMM");
-        int m = MILO_GEMM_AUTO;
-        if (e && e[0] == 't') m = MILO_GEMM_TC;
-        else if (e && e[0] == 'm') m = MILO_GEMM_MMA;
-        int unset = -1;
-        g_gemm_path.compare_exchange_strong(unset, m);
-    });
-    return g_gemm_path.load(std::memory_order_relaxed);
-}
-
-static bool use_tc(long long routed_rows, int n_routed) {
-    const int path = gemm_path();
-    if (path == MILO_GEMM_TC) return true;
-    if (path == MILO_GEMM_MMA) return false;
-    return routed_rows >= 64LL * std::max(1, n_routed);
+// The t-items of a grouped GEMM on the mma.sync path: the compensator's t from
+// the rows' plain copy, K slices and counters in the workspace.
+static void t_items(GemvParams& g, const void* plain, void* tpart, int32_t* sync) {
+    g.t_items = g.has_t ? 1 : 0;
+    g.src = static_cast<const uint16_t*>(plain);
+    g.kslice = t_slice_len(g.K);
+    g.nks = t_slices(g.K);
+    g.tpart = static_cast<float*>(tpart);
+    const int tiles = (g.R + kTokTile - 1) / kTokTile + g.n_exp;   // as gemv_sync_ints
+    g.tctr = sync;
+    g.tdone = sync + 4 * tiles;
+    g.nctr = sync + 5 * tiles;
 }
 
 // The grouped GEMM described by g on the tcgen05 kernel: activations in
@@ -499,7 +541,7 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     int32_t* rows = reinterpret_cast<int32_t*>(base + w.rows);
     int32_t* inv = reinterpret_cast<int32_t*>(base + w.inv);
 
-    const bool tc = use_tc(static_cast<long long>(T) * k, lin->n_experts);
+    const bool tc = w.tc;
     float* rscale = reinterpret_cast<float*>(base + w.rscale);
     PrepParams pp = {};
     pp.src = static_cast<const uint16_t*>(x);
@@ -523,13 +565,16 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     pp.S = 0;
     pp.R_routed = w.R;
     pp.zero = reinterpret_cast<int32_t*>(base + w.done);
-    pp.nzero = lorc_counters(lin->n_experts);
+    pp.nzero = w.nzero;
+    pp.plain = tc ? nullptr : reinterpret_cast<uint16_t*>(base + w.plain);
     milo_status s = check_cuda(launch_prep(pp, st), "prep");
     if (s != MILO_OK) return s;
 
     const bool has_t = lin->max_rank > 0;
     const ProjDev* table = static_cast<const ProjDev*>(lin->table);
-    if (has_t) {
+    // the tcgen05 path takes t from the down-projection kernel; the mma.sync
+    // GEMM computes it itself (t-items) and combines its own output tiles
+    if (has_t && tc) {
         LorcParams lp = {};
         lp.src = static_cast<const uint16_t*>(x);
         lp.row_src = rows;
@@ -569,14 +614,17 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     const int splits = tc ? 1 : w.splits;   // the tcgen05 kernel does not split K
     g.splits = splits;
     g.cps = (g.chunks + splits - 1) / splits;
-    prof_record(0, st);
-    if (tc) s = run_tc(g, false, base + w.frag, base + w.gsum, st, "tc gemm");
-    else s = run_gemv(g, false, st, "gemv");
-    if (s != MILO_OK) return s;
-    prof_record(1, st);
-
     CombineParams cp{reinterpret_cast<const float*>(base + w.part), inv, nullptr, y, dev_status,
                      T, k, 0, lin->N, w.R, splits, w.R, static_cast<int>(y_dt), 1};
+    prof_record(0, st);
+    if (tc) {
+        s = run_tc(g, false, base + w.frag, base + w.gsum, st, "tc gemm");
+    } else {
+        t_items(g, base + w.plain, base + w.tpart, reinterpret_cast<int32_t*>(base + w.done) + lorc_counters(lin->n_experts));
+        s = run_gemv(g, false, st, "gemv");
+    }
+    if (s != MILO_OK) return s;
+    prof_record(1, st);
     return check_cuda(launch_combine(cp, st), "combine");
 }
 
@@ -607,7 +655,8 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     const bool has_t = L->max_rank > 0;
     milo_status s;
 
-    const bool tc = use_tc(w.R_routed, L->n_routed);
+    const bool tc = w.tc;
+    int32_t* sync = reinterpret_cast<int32_t*>(base + w.done) + lorc_counters(n_exp);
     float* xscale = reinterpret_cast<float*>(base + w.xscale);
     float* hscale = reinterpret_cast<float*>(base + w.hscale);
     PrepParams px = {};
@@ -632,9 +681,10 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     px.S = L->n_shared;
     px.R_routed = w.R_routed;
     px.zero = reinterpret_cast<int32_t*>(base + w.done);
-    px.nzero = lorc_counters(n_exp);
+    px.nzero = w.nzero;
+    px.plain = tc ? nullptr : reinterpret_cast<uint16_t*>(base + w.xplain);
     if ((s = check_cuda(launch_prep(px, st), "prep x")) != MILO_OK) return s;
-    if (has_t) {
+    if (has_t && tc) {
         LorcParams lp = {};
         lp.src = static_cast<const uint16_t*>(x);
         lp.row_src = rows;
@@ -675,8 +725,12 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     g1.cps = g1.chunks;
     g1.t_col_b = L->max_rank;
     prof_record(0, st);
-    if (tc) s = run_tc(g1, true, base + w.xfrag, base + w.xg, st, "tc gemm w1|w3");
-    else s = run_gemv(g1, true, st, "gemv w1|w3");
+    if (tc) {
+        s = run_tc(g1, true, base + w.xfrag, base + w.xg, st, "tc gemm w1|w3");
+    } else {
+        t_items(g1, base + w.xplain, base + w.tpart, sync);
+        s = run_gemv(g1, true, st, "gemv w1|w3");
+    }
     if (s != MILO_OK) return s;
     prof_record(1, st);
 
@@ -692,8 +746,9 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     ph.K = I;
     ph.src_bf16 = 0;
     ph.rows = 0;
+    ph.plain = tc ? nullptr : reinterpret_cast<uint16_t*>(base + w.hplain);
     if ((s = check_cuda(launch_prep(ph, st), "prep h")) != MILO_OK) return s;
-    if (has_t) {
+    if (has_t && tc) {
         LorcParams lp = {};
         lp.src = reinterpret_cast<const uint16_t*>(base + w.h);
         lp.row_src = nullptr;
@@ -733,13 +788,16 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     const int splits = tc ? 1 : w.splits;   // the tcgen05 kernel does not split K
     g2.splits = splits;
     g2.cps = (g2.chunks + splits - 1) / splits;
-    prof_record(2, st);
-    if (tc) s = run_tc(g2, false, base + w.hfrag, base + w.hg, st, "tc gemm w2");
-    else s = run_gemv(g2, false, st, "gemv w2");
-    if (s != MILO_OK) return s;
-    prof_record(3, st);
-
     CombineParams cp{reinterpret_cast<const float*>(base + w.part), inv_perm, topk_w, y, dev_status,
                      T, L->top_k, L->n_shared, H, w.R, splits, w.R_routed, static_cast<int>(y_dt), 0};
+    prof_record(2, st);
+    if (tc) {
+        s = run_tc(g2, false, base + w.hfrag, base + w.hg, st, "tc gemm w2");
+    } else {
+        t_items(g2, base + w.hplain, base + w.tpart, sync + w.sync13);
+        s = run_gemv(g2, false, st, "gemv w2");
+    }
+    if (s != MILO_OK) return s;
+    prof_record(3, st);
     return check_cuda(launch_combine(cp, st), "combine");
 }

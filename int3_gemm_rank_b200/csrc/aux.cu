@@ -15,6 +15,7 @@
 
 #include <climits>
 
+#include "milo_combine.cuh"
 #include "milo_device.cuh"
 #include "milo_host.h"
 #include "milo_kernels.h"
@@ -181,9 +182,29 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
             for (int m = 0; m < 16; ++m) s0 += __half2float(x[m]);
 #pragma unroll
             for (int m = 16; m < 32; ++m) s1 += __half2float(x[m]);
+            if (p.plain) {
+                // the row's scaled values, plain: 16 at 128 sb + 16c, 16 at + 64
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    w[i] = static_cast<uint32_t>(__half_as_ushort(x[2 * i])) |
+                           (static_cast<uint32_t>(__half_as_ushort(x[2 * i + 1])) << 16);
+                uint4* o = reinterpret_cast<uint4*>(p.plain + static_cast<size_t>(row) * p.K + 128 * sb + 16 * c);
+                o[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                o[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                uint4* o2 = reinterpret_cast<uint4*>(p.plain + static_cast<size_t>(row) * p.K + 128 * sb + 64 + 16 * c);
+                o2[0] = make_uint4(w[8], w[9], w[10], w[11]);
+                o2[1] = make_uint4(w[12], w[13], w[14], w[15]);
+            }
         } else {
 #pragma unroll
             for (int m = 0; m < 32; ++m) x[m] = __ushort_as_half(0);
+            if (active && p.plain) {
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                uint4* o = reinterpret_cast<uint4*>(p.plain + static_cast<size_t>(row) * p.K + 128 * sb + 16 * c);
+                uint4* o2 = reinterpret_cast<uint4*>(p.plain + static_cast<size_t>(row) * p.K + 128 * sb + 64 + 16 * c);
+                o[0] = o[1] = o2[0] = o2[1] = z;
+            }
         }
         // group sums over the four units of the super-block (lanes 4j..4j+3)
         s0 += __shfl_xor_sync(0xFFFFFFFFu, s0, 1);
@@ -263,25 +284,6 @@ cudaError_t launch_prep(const PrepParams& p, cudaStream_t s) {
 // (a counter per tile says which block that is).  Both orders are fixed, so
 // the result does not depend on scheduling.
 // ---------------------------------------------------------------------------
-// Four packed activation pairs times the row's scale, as fp16 pairs.
-__device__ __forceinline__ uint4 scale_pairs(uint4 v, bool bf16, float scale, int32_t& st) {
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const __half lo = to_half_scaled(static_cast<uint16_t>(w[q] & 0xFFFFu), bf16, scale, st);
-        const __half hi = to_half_scaled(static_cast<uint16_t>(w[q] >> 16), bf16, scale, st);
-        w[q] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// t value rounded to fp16 (FP16_RANGE if it overflows).
-__device__ __forceinline__ uint16_t t_half(float v, int32_t& st) {
-    const __half h = __float2half_rn(v);
-    if (__hisinf(h)) st |= MILO_DEV_FP16_RANGE;
-    return __half_as_ushort(h);
-}
-
 constexpr int kLorcRankBlocks = (MILO_MAX_RANK + 15) / 16;
 constexpr int kLorcChunk = 256;             // K staged per step (per block)
 constexpr int kLorcPitch = kLorcChunk + 8;  // fp16; rows fall on different banks
@@ -356,7 +358,7 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
                 } else {
                     const int sr = src_row[rr];
                     if (sr >= 0)
-                        v = scale_pairs(*reinterpret_cast<const uint4*>(p.src + static_cast<size_t>(sr) * p.K + kc + 8 * ch),
+                        v = scaled_pairs(*reinterpret_cast<const uint4*>(p.src + static_cast<size_t>(sr) * p.K + kc + 8 * ch),
                                         p.src_bf16, src_scale[rr], st);
                     *reinterpret_cast<uint4*>(&xs[rr][8 * ch]) = v;
                 }
@@ -525,7 +527,7 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
             for (int q = 0; q < 4; ++q) {
                 const int i = threadIdx.x + 128 * q;
                 const int rr = i >> 3, pc = i & 7;
-                *reinterpret_cast<uint4*>(&xs[rr][8 * pc]) = scale_pairs(xr[q], p.src_bf16, src_scale[rr], st);
+                *reinterpret_cast<uint4*>(&xs[rr][8 * pc]) = scaled_pairs(xr[q], p.src_bf16, src_scale[rr], st);
                 if (!P->lorc3) *reinterpret_cast<uint4*>(&vs[rr][8 * pc]) = vr[q];
             }
             if (P->lorc3) {
@@ -595,64 +597,18 @@ cudaError_t launch_lorc(const LorcParams& p, cudaStream_t s) {
 // combine: y[t] = sum_j w[t,j] * y_slot[inv[t*k+j]] + sum_s y_shared[s, t]
 // (or, per slot, y[f] = y_slot[inv[f]]), split-K partials summed in order.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float4 row_sum(const float* part, int splits, size_t split_stride,
-                                          size_t off) {
-    float4 a = *reinterpret_cast<const float4*>(part + off);
-    for (int s = 1; s < splits; ++s) {
-        const float4 b = *reinterpret_cast<const float4*>(part + s * split_stride + off);
-        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
-    }
-    return a;
-}
-
 __global__ void __launch_bounds__(64) combine_kernel(const CombineParams p) {
     grid_dep_launch();
     grid_dep_wait();
     const int H4 = p.H / 4;
     const int rows_out = p.per_slot ? p.T * p.k : p.T;
     const long long total = static_cast<long long>(rows_out) * H4;
-    const size_t sstride = static_cast<size_t>(p.R) * p.H;
     int32_t st = 0;
     for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
         const int o = static_cast<int>(i / H4);
         const int n = static_cast<int>(i % H4) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (p.per_slot) {
-            const int r = p.inv_perm[o];
-            if (r >= 0) acc = row_sum(p.y_part, p.splits, sstride, static_cast<size_t>(r) * p.H + n);
-        } else {
-            for (int j = 0; j < p.k; ++j) {
-                const int f = o * p.k + j;
-                const int r = p.inv_perm[f];
-                if (r < 0 || r >= p.R_routed) continue;
-                const float wj = p.w[f];
-                const float4 v = row_sum(p.y_part, p.splits, sstride, static_cast<size_t>(r) * p.H + n);
-                acc.x = fmaf(wj, v.x, acc.x);
-                acc.y = fmaf(wj, v.y, acc.y);
-                acc.z = fmaf(wj, v.z, acc.z);
-                acc.w = fmaf(wj, v.w, acc.w);
-            }
-            for (int s = 0; s < p.S; ++s) {
-                const float4 v = row_sum(p.y_part, p.splits, sstride,
-                                         static_cast<size_t>(p.R_routed + s * p.T + o) * p.H + n);
-                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-            }
-        }
-        const size_t off = static_cast<size_t>(o) * p.H + n;
-        if (p.y_dt == MILO_F32) {
-            *reinterpret_cast<float4*>(static_cast<float*>(p.y) + off) = acc;
-        } else if (p.y_dt == MILO_F16) {
-            const __half2 lo = __floats2half2_rn(acc.x, acc.y), hi = __floats2half2_rn(acc.z, acc.w);
-            if (__hisinf(lo.x) || __hisinf(lo.y) || __hisinf(hi.x) || __hisinf(hi.y)) st |= MILO_DEV_FP16_RANGE;
-            __half2* dst = reinterpret_cast<__half2*>(static_cast<__half*>(p.y) + off);
-            dst[0] = lo;
-            dst[1] = hi;
-        } else {
-            __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.y) + off);
-            dst[0] = __floats2bfloat162_rn(acc.x, acc.y);
-            dst[1] = __floats2bfloat162_rn(acc.z, acc.w);
-        }
+        store4(p, static_cast<size_t>(o) * p.H + n, combine4(p, o, n), st);
     }
     flag(p.dev_status, st);
 }

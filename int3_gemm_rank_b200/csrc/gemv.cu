@@ -46,6 +46,7 @@
 
 #include <atomic>
 
+#include "milo_combine.cuh"
 #include "milo_device.cuh"
 #include "milo_host.h"
 #include "milo_kernels.h"
@@ -66,7 +67,9 @@ constexpr int kOffX = 2 * kTileBlk;                       // 14336
 constexpr int kStageBytes = kOffX + kTokTile * kFragRowHalves * 2;
 constexpr int kOffUA = 0, kOffUB = 8192, kOffT = 16384;   // compensator stage
 constexpr int kBarOffset = kStages * kStageBytes;
-constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 3 * (MILO_MAX_EXPERTS + 1) * 4 + kStages * 4 + 16;
+// barriers, then the item tables cnt, row0s, ttb, tstart [MILO_MAX_EXPERTS + 1],
+// the stage headers and the consumers' broadcast word
+constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 4 * (MILO_MAX_EXPERTS + 1) * 4 + kStages * 4 + 16;
 
 static_assert(kStageBytes % 16 == 0 && kOffX % 16 == 0 && kTileBlk % 16 == 0, "bulk-copy alignment");
 static_assert(kOffT >= kRowsPlain * MILO_MAX_RANK * 2, "compensator stage: U rows");
@@ -76,23 +79,155 @@ struct Item {
     int e, ntile, split, tt;
 };
 
-__device__ __forceinline__ Item decode_item(int it, const int* start, const int* cnt, int n_exp,
-                                            int splits) {
+// Largest e in [0, n_exp) with first[e] * mul <= it (first[] non-decreasing).
+__device__ __forceinline__ int find_expert(int it, const int* first, int mul, int n_exp) {
     int lo = 0, hi = n_exp - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (start[mid] <= it) lo = mid;
+        if (first[mid] * mul <= it) lo = mid;
         else hi = mid - 1;
     }
+    return lo;
+}
+
+// GEMM item `it`: expert e owns items [ttb[e], ttb[e+1]) * n_tiles * splits
+// (ttb: prefix of the experts' 16-row token tiles), its token tiles fastest,
+// then the K splits, then the weight-row tiles.
+__device__ __forceinline__ Item decode_item(int it, const int* ttb, const int* cnt, int n_exp, int n_tiles,
+                                            int splits) {
     Item r;
-    r.e = lo;
-    const int local = it - start[lo];
-    const int tte = (cnt[lo] + kTokTile - 1) / kTokTile;
+    r.e = find_expert(it, ttb, n_tiles * splits, n_exp);
+    const int local = it - ttb[r.e] * n_tiles * splits;
+    const int tte = (cnt[r.e] + kTokTile - 1) / kTokTile;
     r.tt = local % tte;
     const int rest = local / tte;
     r.split = rest % splits;
     r.ntile = rest / splits;
     return r;
+}
+
+// Rank blocks of 32 of a projection (t-items).
+__device__ __forceinline__ int rank_blocks(int r) { return (r + 31) >> 5; }
+
+// Named barrier of the four consumer warps (the producer warp is not in it).
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Eight consecutive values k .. k + 7 (k % 8 == 0) of rank row j of an int3
+// V blob (milo_pack layout, one 64-row tile), dequantised (q - z) s to fp16
+// pairs: they are codes m0 .. m0 + 7 of one unit of super-block k / 128.
+__device__ __forceinline__ uint4 lorc3_v8(const uint8_t* blob, int j, int k) {
+    const int kin = k & 127;
+    const uint32_t* wp = reinterpret_cast<const uint32_t*>(blob + lorc_words_off(j, k >> 7, blob_unit(kin)));
+    const uint32_t w3[3] = {__ldg(wp), __ldg(wp + 1), __ldg(wp + 2)};
+    const uint32_t sz = __ldg(reinterpret_cast<const uint32_t*>(blob + lorc_sz_off(j, k >> 6)));
+    const float sc = sz_scale(sz), z = sz_zero(sz);
+    const int m0 = blob_code(kin);
+    uint32_t h[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float lo = (static_cast<float>(unit_code(w3, m0 + 2 * q)) - z) * sc;
+        const float hi = (static_cast<float>(unit_code(w3, m0 + 2 * q + 1)) - z) * sc;
+        h[q] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(lo))) |
+               (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(hi))) << 16);
+    }
+    return make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+// t-item j (consumer warps): t[row][col] = fp16(sum_k x'[row][k] V[rank][k])
+// for the 16 rows of one token tile of expert e, 32 ranks of one projection
+// (8 per warp) and one K slice; x' is the prepared rows' plain fp16 copy
+// (already times their scale 2^a).  Each lane loads 8 consecutive k of its
+// two rows and of its V row with 16-byte loads and uses them as two k16 MMA
+// steps (the same relabelling of k on both operands, so the sum is
+// unchanged).  The slice's f32 partials go to tpart; the slice that finishes
+// last adds the slices in order (deterministic) and writes t, then counts
+// the rank block done for the token tile.
+template <bool GLU>
+__device__ void titem_run(const GemvParams& p, int j, const int* tstart, const int* ttb, const int* cnt,
+                          const int* row0s, int warp, int lane, volatile int* bcast) {
+    const int e = find_expert(j, tstart, 1, p.n_exp);
+    const ProjDev* pa = p.table + e * p.stride + p.proj_a;
+    const ProjDev* pb = p.table + e * p.stride + p.proj_b;
+    const int na = rank_blocks(pa->rank), nb = GLU ? rank_blocks(pb->rank) : 0;
+    const int local = j - tstart[e];
+    const int ks = local % p.nks, rest = local / p.nks;
+    const int rbi = rest % (na + nb), tt = rest / (na + nb);
+    const bool second = rbi >= na;
+    const ProjDev* P = second ? pb : pa;
+    const int r = P->rank;
+    const int rk0 = 32 * (second ? rbi - na : rbi) + 8 * warp;        // the warp's first rank
+    const int col0 = (second ? p.t_col_b : 0) + rk0;
+    const int row0 = row0s[e] + kTokTile * tt, ntok = min(kTokTile, cnt[e] - kTokTile * tt);
+    const int g = lane >> 2, c = lane & 3;
+    int32_t st = 0;
+    const uint16_t* xr0 = g < ntok ? p.src + static_cast<size_t>(row0 + g) * p.K : nullptr;
+    const uint16_t* xr1 = g + 8 < ntok ? p.src + static_cast<size_t>(row0 + g + 8) * p.K : nullptr;
+    const int jr = rk0 + g;                      // the lane's V row
+    const bool vrow = jr < r;
+    const int kb0 = ks * p.kslice, kb1 = min(p.K, kb0 + p.kslice);
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 16
+    for (int kb = kb0; kb < kb1; kb += 32) {
+        const int k = kb + 8 * c;
+        const uint4 xa = xr0 ? __ldg(reinterpret_cast<const uint4*>(xr0 + k)) : z4;
+        const uint4 xb = xr1 ? __ldg(reinterpret_cast<const uint4*>(xr1 + k)) : z4;
+        const uint4 v = !vrow ? z4
+                        : P->lorc3 ? lorc3_v8(reinterpret_cast<const uint8_t*>(P->V), jr, k)
+                                   : __ldg(reinterpret_cast<const uint4*>(P->V + static_cast<size_t>(jr) * p.K + k));
+        mma16816(acc, xa.x, xb.x, xa.y, xb.y, v.x, v.y);
+        mma16816(acc, xa.z, xb.z, xa.w, xb.w, v.z, v.w);
+    }
+    // acc[i]: row g + 8 (i >> 1), rank rk0 + 2c + (i & 1); only ranks < r are stored
+    if (p.nks == 1) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int rr = g + 8 * (i >> 1), rk = rk0 + 2 * c + (i & 1);
+            if (rr < ntok && rk < r)
+                p.t[static_cast<size_t>(row0 + rr) * p.tcols + col0 + 2 * c + (i & 1)] = t_half(acc[i], st);
+        }
+    } else {
+        float* part = p.tpart + static_cast<size_t>(ks) * p.R * p.tcols;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int rr = g + 8 * (i >> 1), rk = rk0 + 2 * c + (i & 1);
+            if (rr < ntok && rk < r) part[static_cast<size_t>(row0 + rr) * p.tcols + col0 + 2 * c + (i & 1)] = acc[i];
+        }
+        __threadfence();
+        consumer_sync();
+        if (threadIdx.x == 0) *bcast = atomicAdd(&p.tctr[j / p.nks], 1) == p.nks - 1;
+        consumer_sync();
+        const bool last = *bcast != 0;
+        if (last) {
+            __threadfence();
+            const size_t slice = static_cast<size_t>(p.R) * p.tcols;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int rr = g + 8 * (i >> 1), rk = rk0 + 2 * c + (i & 1);
+                if (rr < ntok && rk < r) {
+                    const size_t o = static_cast<size_t>(row0 + rr) * p.tcols + col0 + 2 * c + (i & 1);
+                    float v = 0.0f;
+                    for (int s2 = 0; s2 < p.nks; ++s2) v += __ldcg(p.tpart + s2 * slice + o);
+                    p.t[o] = t_half(v, st);
+                }
+            }
+        }
+        consumer_sync();          // every warp has read bcast before it is reused
+        if (!last) {
+            flag(p.dev_status, st);
+            return;
+        }
+    }
+    __threadfence();
+    consumer_sync();
+    if (threadIdx.x == 0) atomicAdd(&p.tdone[ttb[e] + tt], 1);
+    flag(p.dev_status, st);
 }
 
 // One k16 step of the code part: extract the A fragments of both row tiles
@@ -290,11 +425,14 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
     uint64_t* empty = full + kStages;
-    int* start = reinterpret_cast<int*>(empty + kStages);
-    int* cnt = start + (MILO_MAX_EXPERTS + 1);
+    int* cnt = reinterpret_cast<int*>(empty + kStages);
     int* row0s = cnt + (MILO_MAX_EXPERTS + 1);
-    // header of each stage: the work item whose first stage it is (-1: no more items)
-    volatile int* stage_item = row0s + (MILO_MAX_EXPERTS + 1);
+    int* ttb = row0s + (MILO_MAX_EXPERTS + 1);       // prefix of the experts' token tiles
+    int* tstart = ttb + (MILO_MAX_EXPERTS + 1);      // prefix of the experts' t-items
+    // header of each stage: the work item whose first stage it is (-1: no more
+    // items, -2 - j: t-item j, a stage with no data)
+    volatile int* stage_item = tstart + (MILO_MAX_EXPERTS + 1);
+    volatile int* bcast = stage_item + kStages;      // consumers' broadcast word
 
     constexpr int RA = GLU ? kRowsGlu : kRowsPlain;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -308,34 +446,51 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         fence_barrier_init();
     }
     grid_dep_wait();
-    // Item table from the expert groups: all threads load groups (independent
-    // global loads), then warp 0 scans the per-expert item counts.
+    // Item tables from the expert groups: all threads load the groups (and the
+    // ranks, for the t-items), then warp 0 scans the token tiles and t-items.
     for (int e = threadIdx.x; e < p.n_exp; e += blockDim.x) {
         const int r0 = p.grp[2 * e], m = p.grp[2 * e + 1];
         const bool ok = m > 0 && r0 >= 0 && r0 + m <= p.R;
         cnt[e] = ok ? m : 0;
         row0s[e] = r0;
+        const int tte = ok ? (m + kTokTile - 1) / kTokTile : 0;
+        ttb[e] = tte;
+        int nt = 0;
+        if (p.t_items && tte > 0) {
+            const int na = rank_blocks(p.table[e * p.stride + p.proj_a].rank);
+            const int nb = GLU ? rank_blocks(p.table[e * p.stride + p.proj_b].rank) : 0;
+            nt = tte * (na + nb) * p.nks;
+        }
+        tstart[e] = nt;
     }
     __syncthreads();
     if (warp == 0) {
-        int run = 0;
+        int run = 0, trun = 0;
         for (int base = 0; base < p.n_exp; base += 32) {
             const int e = base + lane;
-            const int m = e < p.n_exp ? cnt[e] : 0;
-            const int items = m > 0 ? ((m + kTokTile - 1) / kTokTile) * n_tiles * p.splits : 0;
-            int incl = items;
+            const int a = e < p.n_exp ? ttb[e] : 0, b = e < p.n_exp ? tstart[e] : 0;
+            int ia = a, ib = b;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-                if (lane >= o) incl += y;
+                const int ya = __shfl_up_sync(0xFFFFFFFFu, ia, o);
+                const int yb = __shfl_up_sync(0xFFFFFFFFu, ib, o);
+                if (lane >= o) { ia += ya; ib += yb; }
             }
-            if (e < p.n_exp) start[e] = run + incl - items;
-            run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+            if (e < p.n_exp) {
+                ttb[e] = run + ia - a;
+                tstart[e] = trun + ib - b;
+            }
+            run += __shfl_sync(0xFFFFFFFFu, ia, 31);
+            trun += __shfl_sync(0xFFFFFFFFu, ib, 31);
         }
-        if (lane == 0) start[p.n_exp] = run;
+        if (lane == 0) {
+            ttb[p.n_exp] = run;
+            tstart[p.n_exp] = trun;
+        }
     }
     __syncthreads();
-    const int n_items = start[p.n_exp];
+    const int n_items = ttb[p.n_exp] * n_tiles * p.splits;
+    const int n_t = tstart[p.n_exp];
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------------ producer
@@ -347,16 +502,37 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         uint32_t phase = 0;
         uint32_t filled = 0, fph = 0;     // per stage: has a fill, parity of its last fill
         bool fail = false;
-        // Items are taken round-robin (item b, b + gridDim.x, ...).  A global
-        // work queue balanced the skewed DeepSeekMoE-shaped layer no better
-        // and cost the Mixtral-shaped one 15 %; the static split is kept.
+        // This CTA's t-items first (j = G - 1 - b, + G, ...: one per CTA from
+        // the last one down, so that every t is ready early; the last CTAs
+        // have the fewest GEMM items), then its GEMM items, taken round-robin
+        // (item b, b + G, ...).  A global work queue balanced the skewed
+        // DeepSeekMoE-shaped layer no better and cost the Mixtral-shaped one
+        // 15 %; the static split is kept.
+        const int S = static_cast<int>(gridDim.x);
+        int tj = S - 1 - static_cast<int>(blockIdx.x);
         int next = blockIdx.x;
         for (;;) {
+            if (tj < n_t) {      // a t-item: a header-only stage
+                if (!warp_wait(&empty[stage], phase ^ 1)) {
+                    fail = true;
+                    break;
+                }
+                filled |= 1u << stage;
+                fph = (fph & ~(1u << stage)) | (phase << stage);
+                if (elect_one()) {
+                    stage_item[stage] = -2 - tj;
+                    mbar_arrive(&full[stage]);
+                }
+                __syncwarp();
+                if (++stage == kStages) { stage = 0; phase ^= 1; }
+                tj += S;
+                continue;
+            }
             const int it = next;
             if (it < 0 || it >= n_items) break;
             next += gridDim.x;
             bool header = false;      // the item's first stage has been filled
-            const Item w = decode_item(it, start, cnt, p.n_exp, p.splits);
+            const Item w = decode_item(it, ttb, cnt, p.n_exp, n_tiles, p.splits);
             const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
             const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
             const int n0 = w.ntile * RA;
@@ -393,8 +569,29 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 header = true;
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
             }
+            if (fail) break;
             const int ra = pa->rank, rb = GLU ? pb->rank : 0;
-            if (!fail && w.split == 0 && p.has_t && (ra > 0 || rb > 0)) {
+            if (w.split == 0 && p.has_t && (ra > 0 || rb > 0)) {
+                if (p.t_items) {
+                    // this token tile's t comes from t-items of this launch:
+                    // wait (bounded) until all its rank blocks are done
+                    const int need = rank_blocks(ra) + (GLU ? rank_blocks(rb) : 0);
+                    const int32_t* done = p.tdone + ttb[w.e] + w.tt;
+                    if (ld_acquire(done) < need) {
+                        const long long t0 = clock64();
+                        while (ld_acquire(done) < need) {
+                            if (clock64() - t0 > kWaitCycles) {
+                                fail = true;
+                                break;
+                            }
+                            __nanosleep(64);
+                        }
+                    }
+                    fail = __any_sync(0xFFFFFFFFu, fail);
+                    if (fail) break;
+                    // t was written by ordinary stores; the bulk copy reads it
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                }
                 if (!warp_wait(&empty[stage], phase ^ 1)) {
                     fail = true;
                     break;
@@ -472,9 +669,16 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             return;
         }
         const int it = stage_item[stage];
-        if (it < 0) break;
+        if (it == -1) break;
+        if (it < -1) {           // a t-item: its stage carries no data
+            titem_run<GLU>(p, -2 - it, tstart, ttb, cnt, row0s, warp, lane, bcast);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == kStages) { stage = 0; phase ^= 1; }
+            continue;
+        }
         bool waited = true;       // the next stage's barrier has been passed already
-        const Item w = decode_item(it, start, cnt, p.n_exp, p.splits);
+        const Item w = decode_item(it, ttb, cnt, p.n_exp, n_tiles, p.splits);
         const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
         const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
         const int n0 = w.ntile * RA;
@@ -567,31 +771,87 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                         if (tok < ntok && n < p.N)
                             out[static_cast<size_t>(row0 + tok) * p.N + n] = acc[ti][n8][i] * inv[n8][i & 1];
                     }
+            if (p.fuse_combine) {
+                // the item that completes this output tile combines its columns
+                __threadfence();
+                consumer_sync();
+                if (threadIdx.x == 0)
+                    *bcast = atomicAdd(&p.nctr[w.ntile], 1) == ttb[p.n_exp] * p.splits - 1;
+                consumer_sync();
+                const bool last = *bcast != 0;
+                consumer_sync();
+                if (last) {
+                    __threadfence();
+                    int32_t cst = 0;
+                    const int rows_out = p.comb.per_slot ? p.comb.T * p.comb.k : p.comb.T;
+                    const int quads = min(RA, p.N - n0) / 4;
+                    for (int i = threadIdx.x; i < rows_out * quads; i += 32 * kConsumerWarps) {
+                        const int o = i / quads, n = n0 + 4 * (i % quads);
+                        store4(p.comb, static_cast<size_t>(o) * p.N + n, combine4(p.comb, o, n), cst);
+                    }
+                    flag(p.dev_status, cst);
+                }
+            }
         }
+    }
+    // No rows at all: nothing completes an output tile, so the CTAs combine
+    // (zeros, for dropped slots) tile by tile.
+    if (!GLU && p.fuse_combine && n_items == 0) {
+        int32_t cst = 0;
+        const int rows_out = p.comb.per_slot ? p.comb.T * p.comb.k : p.comb.T;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            const int n0 = tile * RA, quads = min(RA, p.N - n0) / 4;
+            for (int i = threadIdx.x; i < rows_out * quads; i += 32 * kConsumerWarps) {
+                const int o = i / quads, n = n0 + 4 * (i % quads);
+                store4(p.comb, static_cast<size_t>(o) * p.N + n, combine4(p.comb, o, n), cst);
+            }
+        }
+        flag(p.dev_status, cst);
     }
 }
 
 size_t gemv_smem_bytes(bool) { return kSmemBytes; }
 
-cudaError_t launch_gemv(const GemvParams& p, bool glu, int grid, cudaStream_t s) {
-    // The shared-memory opt-in is a per-device function attribute.
-    static std::atomic<bool> configured[64][2];   // set once per device and kernel (a repeat is harmless)
+// Resident CTAs per SM of the kernel (its shared memory opted in), per device.
+static int gemv_occupancy(bool glu, int dev) {
+    static std::atomic<int> occ[64][2];
+    int v = dev >= 0 && dev < 64 ? occ[dev][glu].load(std::memory_order_acquire) : 0;
+    if (v > 0) return v;
+    cudaError_t e = glu ? cudaFuncSetAttribute(gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)
+                        : cudaFuncSetAttribute(gemv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return -static_cast<int>(e);
+    int n = 0;
+    e = glu ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_kernel<true>, kGemvThreads, kSmemBytes)
+            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_kernel<false>, kGemvThreads, kSmemBytes);
+    if (e != cudaSuccess) return -static_cast<int>(e);
+    if (n < 1) return -static_cast<int>(cudaErrorInvalidConfiguration);
+    if (dev >= 0 && dev < 64) occ[dev][glu].store(n, std::memory_order_release);
+    return n;
+}
+
+cudaError_t launch_gemv(const GemvParams& p, bool glu, int sms, cudaStream_t s) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !configured[dev][glu].load(std::memory_order_acquire)) {
-        e = glu ? cudaFuncSetAttribute(gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)
-                : cudaFuncSetAttribute(gemv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) configured[dev][glu].store(true, std::memory_order_release);
-    }
-    // A normal launch: the persistent grid starts once the previous kernel has
-    // left every SM, so its CTAs are spread evenly over the SMs (an early,
-    // programmatic launch places them wherever resources free up first, and
-    // the per-SM load of the static item split then goes uneven).
-    if (glu) gemv_kernel<true><<<grid, kGemvThreads, kSmemBytes, s>>>(p);
-    else gemv_kernel<false><<<grid, kGemvThreads, kSmemBytes, s>>>(p);
-    return cudaGetLastError();
+    const int occ = gemv_occupancy(glu, dev);
+    if (occ < 0) return static_cast<cudaError_t>(-occ);
+    // A normal (not programmatic) launch: the persistent grid starts once the
+    // previous kernel has left every SM, so its CTAs are spread evenly over
+    // the SMs (an early, programmatic launch places them wherever resources
+    // free up first, and the per-SM load of the static item split then goes
+    // uneven).  When CTAs wait on one another (t-items), the launch is
+    // cooperative: every CTA is resident at once.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(occ * sms));
+    cfg.blockDim = dim3(kGemvThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
+    return glu ? cudaLaunchKernelEx(&cfg, gemv_kernel<true>, p) : cudaLaunchKernelEx(&cfg, gemv_kernel<false>, p);
 }
 
 }  // namespace milo

@@ -71,6 +71,25 @@ __device__ __forceinline__ float inv_pow2(float s) {
     return __uint_as_float(0x7F000000u - __float_as_uint(s));
 }
 
+// Four packed activation pairs times their row's scale, as fp16 pairs.
+__device__ __forceinline__ uint4 scaled_pairs(uint4 v, bool bf16, float scale, int32_t& st) {
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const __half lo = to_half_scaled(static_cast<uint16_t>(w[q] & 0xFFFFu), bf16, scale, st);
+        const __half hi = to_half_scaled(static_cast<uint16_t>(w[q] >> 16), bf16, scale, st);
+        w[q] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// A compensator value t rounded to fp16 (FP16_RANGE if it overflows).
+__device__ __forceinline__ uint16_t t_half(float v, int32_t& st) {
+    const __half h = __float2half_rn(v);
+    if (__hisinf(h)) st |= MILO_DEV_FP16_RANGE;
+    return __half_as_ushort(h);
+}
+
 // ---------------------------------------------------------------------------
 // int3 format: field extraction
 // ---------------------------------------------------------------------------

@@ -53,11 +53,21 @@ struct alignas(64) ProjDev {
     int32_t rank, N, K, lorc3;  // lorc3: the compensator is int3 (both blobs one 64-row tile high)
 };
 
+struct CombineParams {
+    const float* y_part;        // [splits][R][H]
+    const int32_t* inv_perm;    // [T*k] row of each flat slot (-1 = dropped)
+    const float* w;             // [T*k] combine weights (NULL: 1, and k slots are rows)
+    void* y;                    // output
+    int32_t* dev_status;
+    int T, k, S, H, R, splits, R_routed, y_dt;
+    int per_slot;               // 1: y row per flat slot (grouped linear), 0: per token
+};
+
 struct GemvParams {
     const uint16_t* x;          // prepared activations [chunks][R][kFragRowHalves] fp16
                                 // (group sums in each row's padding, see kGsumHalf)
     const float* rscale;        // [R]: the row's activation scale 2^a (see kFoldScale)
-    const uint16_t* t;          // LoRC down-projection [R][tcols] fp16 (times the row's 2^a)
+    uint16_t* t;                // LoRC down-projection [R][tcols] fp16 (times the row's 2^a)
     const ProjDev* table;       // device table
     const int32_t* grp;         // [n_exp][2]: first row, row count of each group (expert)
     float* y_part;              // plain: [splits][R][N] f32 partial sums
@@ -67,7 +77,30 @@ struct GemvParams {
     int n_exp, N, K, R, SB, G;  // G = K / 64 groups
     int splits, chunks, cps;    // split-K count, K chunks, chunks per split
     int has_t, tcols, t_col_b;  // LoRC activations present; row width; first column of w3's
+    // Compensator down-projection computed in the kernel ("t-items", first on
+    // the CTAs with the fewest GEMM items): t = fp16(x' V^T) per (expert,
+    // projection, 32 ranks, 16-row token tile, K slice); the slice that
+    // finishes last adds the slices in order, and a GEMM item waits (bounded)
+    // until its token tile's t is complete before copying it.
+    int t_items;                // 0: t was computed beforehand
+    const uint16_t* src;        // the rows' plain fp16 copy [R][K] (times their scale 2^a)
+    int nks, kslice;            // K slices per t-item and their length (multiple of 32)
+    float* tpart;               // [nks][R][tcols] f32 slice partials
+    int32_t* tctr;              // per (expert, token tile, rank block): slices finished (0 on entry)
+    int32_t* tdone;             // per (expert, token tile): rank blocks finished (0 on entry)
+    // Fused combine (plain kernel): the last item of each 128-row output tile
+    // combines the tile's columns of every output row.
+    int fuse_combine;
+    int32_t* nctr;              // per output tile: items finished (0 on entry)
+    CombineParams comb;
 };
+
+// Ints of the t-item and combine counters of a grouped GEMM over R rows,
+// n_exp experts and N outputs (zeroed before each launch).
+inline int gemv_sync_ints(int R, int n_exp, int N) {
+    const int tiles = (R + kTokTile - 1) / kTokTile + n_exp;   // token tiles of all experts, at most
+    return tiles * 4 + tiles + (N + kRowsPlain - 1) / kRowsPlain;
+}
 
 // Parameters of the tcgen05 grouped GEMM for large per-expert row counts
 // (gemm_tc.cu).  Activations in MMA column order [R][K] fp16 and their group
@@ -97,6 +130,7 @@ struct PrepParams {
                                 // layout 1: [R][K] fp16 in tcgen05 A-column order
     uint16_t* gsum;             // layout 1: group sums [R][chunks][16] fp16: per group (hi, lo, hi, lo)
     float* rscale;              // [R]: written, the row's scale 2^a (1 for a zero row)
+    uint16_t* plain;            // optional [R][K]: written, the row's fp16 values times 2^a
     int layout;
     int32_t* dev_status;
     int R, K, src_bf16;
@@ -131,15 +165,6 @@ struct LorcParams {
 // groups); zeroed by prep_kernel and left at zero.
 constexpr int kLorcCounters = MILO_MAX_EXPERTS * 2 * ((MILO_MAX_RANK + 15) / 16) * 8;
 
-struct CombineParams {
-    const float* y_part;        // [splits][R][H]
-    const int32_t* inv_perm;    // [T*k] row of each flat slot (-1 = dropped)
-    const float* w;             // [T*k] combine weights (NULL: 1, and k slots are rows)
-    void* y;                    // output
-    int32_t* dev_status;
-    int T, k, S, H, R, splits, R_routed, y_dt;
-    int per_slot;               // 1: y row per flat slot (grouped linear), 0: per token
-};
 
 size_t tc_smem_bytes();
 cudaError_t launch_tc_gemm(const TcParams& p, bool glu, int grid, cudaStream_t s);
