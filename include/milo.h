@@ -133,6 +133,20 @@ MILO_API milo_status milo_pack(const uint16_t* W, int32_t N, int32_t K, int32_t 
 MILO_API milo_status milo_unpack(const void* packed, int32_t N, int32_t K, uint8_t* codes,
                         void* stream);
 
+/*
+ * milo_dequantize -- the dequantised weights of a packed blob, as fp16:
+ * W_hat[n, k] = fp16((q[n, k] - z[n, k/64]) * s[n, k/64]), row-major [N, K],
+ * rounded once to nearest even (the product is formed exactly).  This is the
+ * first pass of the unfused pipeline the paper compares its fused kernel
+ * against ("Experimental Setup & Results": the int3 GEMM is several times
+ * faster than the unfused implementation, a dequantisation pass followed by
+ * an FP16 GEMM); the fused GEMMs of this library never materialise W_hat.
+ *   packed: the blob (16-byte aligned); W_hat: fp16 [N, K] (16-byte aligned).
+ * Errors: K % 128 != 0 -> UNSUPPORTED_SHAPE; N, K <= 0, NULL or misaligned
+ * pointers -> INVALID_ARG.  Stream-ordered.
+ */
+MILO_API milo_status milo_dequantize(const void* packed, int32_t N, int32_t K, uint16_t* W_hat, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Offline MiLo quantiser                                                   */
 /* ------------------------------------------------------------------------ */
@@ -350,7 +364,11 @@ MILO_API milo_status milo_linear_prepare(milo_linear* lin, const milo_qweight* w
 MILO_API milo_status milo_layer_prepare(milo_moe_layer* layer, const milo_expert* experts,
                                void* device_table, size_t table_bytes);
 
-/* Workspace bytes for milo_grouped_linear / milo_moe_forward over T tokens. */
+/* Workspace bytes for milo_grouped_linear / milo_moe_forward over T tokens.
+ * The size depends on which grouped GEMM the call takes (see
+ * milo_set_gemm_path: the mma.sync kernel also keeps a plain fp16 copy of the
+ * scaled rows and its counters in the workspace), so query it again after
+ * changing that setting; a call given less returns MILO_ERR_WORKSPACE. */
 MILO_API milo_status milo_linear_workspace_bytes(const milo_linear* lin, int32_t T, int32_t k,
                                         size_t* bytes);
 MILO_API milo_status milo_moe_workspace_bytes(const milo_moe_layer* layer, int32_t T, size_t* bytes);

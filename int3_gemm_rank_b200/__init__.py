@@ -35,7 +35,7 @@ EXPORTS = ("milo_status_str", "milo_last_error", "milo_version", "milo_pack", "m
            "milo_moe_forward", "milo_moe_h_offset", "milo_set_profile_events",
            "milo_grouped_linear_noalloc", "milo_packed_bytes", "milo_hqq_pack",
            "milo_quantize_lorc_workspace", "milo_quantize_lorc", "milo_kurtosis_workspace", "milo_kurtosis",
-           "milo_assign_ranks", "milo_selftest_wait_timeout", "milo_set_gemm_path")
+           "milo_assign_ranks", "milo_selftest_wait_timeout", "milo_set_gemm_path", "milo_dequantize")
 
 
 class MiloError(RuntimeError):
@@ -127,6 +127,7 @@ def lib() -> C.CDLL:
         L.milo_assign_ranks.restype = C.c_int
         L.milo_selftest_wait_timeout.argtypes = [vp, vp]; L.milo_selftest_wait_timeout.restype = C.c_int
         L.milo_set_gemm_path.argtypes = [i32]; L.milo_set_gemm_path.restype = C.c_int
+        L.milo_dequantize.argtypes = [vp, i32, i32, vp, vp]; L.milo_dequantize.restype = C.c_int
         _lib = L
     return _lib
 
@@ -194,6 +195,14 @@ def milo_pack(W: torch.Tensor, group: int = MILO_GROUP, dev_status: torch.Tensor
     blob = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
     _check(lib().milo_pack(_ptr(W), N, K, group, _ptr(blob), _ptr(dev_status), _stream()), "milo_pack")
     return blob
+
+
+def milo_dequantize(packed: torch.Tensor, N: int, K: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    """fp16 [N, K] dequantised weights (q - z) s of a packed blob."""
+    _cuda(packed, "packed")
+    W = torch.empty((N, K), dtype=torch.float16, device=packed.device) if out is None else out
+    _check(lib().milo_dequantize(_ptr(packed), N, K, _ptr(W), _stream()), "milo_dequantize")
+    return W
 
 
 def milo_unpack(packed: torch.Tensor, N: int, K: int) -> torch.Tensor:

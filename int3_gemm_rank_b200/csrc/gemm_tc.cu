@@ -771,7 +771,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     for (int i = 0; i < kTcHalf; ++i) {
                         const int t = kTcHalf * th + i;
                         if (t < ntok)
-                            p.y_part[static_cast<size_t>(row0 + t) * p.N + n] = (i & 1) ? acc[i >> 1].y : acc[i >> 1].x;
+                            // streaming stores: the output is read once, by the
+                            // combine, and must not push the routed rows out of L2
+                            __stcs(p.y_part + static_cast<size_t>(row0 + t) * p.N + n,
+                                   (i & 1) ? acc[i >> 1].y : acc[i >> 1].x);
                     }
                 }
             }

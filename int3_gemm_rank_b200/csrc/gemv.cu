@@ -542,6 +542,11 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             const int ntok = min(kTokTile, cnt[w.e] - w.tt * kTokTile);
             const int c0 = w.split * p.cps;
             const int c1 = min(p.chunks, c0 + p.cps);
+            // the compensator stage's fields, loaded with the item's first ones
+            const int ra = pa->rank, rb = GLU ? pb->rank : 0;
+            const bool l3a = pa->lorc3 != 0, l3b = GLU ? pb->lorc3 != 0 : false;
+            const uint16_t* Ua = pa->U;
+            const uint16_t* Ub = pb->U;
             for (int ch = c0; ch < c1; ++ch) {
                 if (!warp_wait(&empty[stage], phase ^ 1)) {
                     fail = true;
@@ -570,7 +575,6 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
             }
             if (fail) break;
-            const int ra = pa->rank, rb = GLU ? pb->rank : 0;
             if (w.split == 0 && p.has_t && (ra > 0 || rb > 0)) {
                 if (p.t_items) {
                     // this token tile's t comes from t-items of this launch:
@@ -602,12 +606,12 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 fph = (fph & ~(1u << stage)) | (phase << stage);
                 const int urows = min(RA, p.N - n0);
                 // fp16 U rows, or the int3 U^T block holding the item's features
-                const uint32_t ua = ra == 0 ? 0u : pa->lorc3 ? kBlockSB : urows * ra * 2;
-                const uint32_t ub = rb == 0 ? 0u : pb->lorc3 ? kBlockSB : urows * rb * 2;
-                const uint8_t* usa = pa->lorc3 ? reinterpret_cast<const uint8_t*>(pa->U) + (n0 >> 7) * kBlockSB
-                                               : reinterpret_cast<const uint8_t*>(pa->U + static_cast<size_t>(n0) * ra);
-                const uint8_t* usb = !GLU ? usa : pb->lorc3 ? reinterpret_cast<const uint8_t*>(pb->U) + (n0 >> 7) * kBlockSB
-                                                            : reinterpret_cast<const uint8_t*>(pb->U + static_cast<size_t>(n0) * rb);
+                const uint32_t ua = ra == 0 ? 0u : l3a ? kBlockSB : urows * ra * 2;
+                const uint32_t ub = rb == 0 ? 0u : l3b ? kBlockSB : urows * rb * 2;
+                const uint8_t* usa = l3a ? reinterpret_cast<const uint8_t*>(Ua) + (n0 >> 7) * kBlockSB
+                                         : reinterpret_cast<const uint8_t*>(Ua + static_cast<size_t>(n0) * ra);
+                const uint8_t* usb = !GLU ? usa : l3b ? reinterpret_cast<const uint8_t*>(Ub) + (n0 >> 7) * kBlockSB
+                                                      : reinterpret_cast<const uint8_t*>(Ub + static_cast<size_t>(n0) * rb);
                 const uint32_t tb = ntok * p.tcols * 2;
                 if (elect_one()) {
                     if (!header) stage_item[stage] = it;
@@ -686,6 +690,19 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         const int ntok = min(kTokTile, cnt[w.e] - w.tt * kTokTile);
         const int c0 = w.split * p.cps;
         const int c1 = min(p.chunks, c0 + p.cps);
+        // what the item's end needs from global memory, loaded now so that the
+        // loads overlap the K loop (the barrier waits keep the compiler from
+        // moving them): the projections' ranks and formats, the rows' scales
+        const int ra = pa->rank, rb = GLU ? pb->rank : 0;
+        const bool u3a = pa->lorc3 != 0, u3b = GLU ? pb->lorc3 != 0 : u3a;
+        float inv[2][2];
+#pragma unroll
+        for (int n8 = 0; n8 < 2; ++n8)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int tok = n8 * 8 + 2 * c + j;
+                inv[n8][j] = tok < ntok ? inv_pow2(p.rscale[row0 + tok]) : 0.0f;
+            }
         float acc[2][2][4];
 #pragma unroll
         for (int a = 0; a < 2; ++a)
@@ -708,7 +725,6 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             if (lane == 0) mbar_arrive(&empty[stage]);
             if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
-        const int ra = pa->rank, rb = GLU ? pb->rank : 0;
         if (w.split == 0 && p.has_t && (ra > 0 || rb > 0)) {
             if (!waited && !warp_wait(&full[stage], phase)) {
                 flag(p.dev_status, MILO_DEV_TIMEOUT);
@@ -717,7 +733,6 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             waited = false;
             const uint8_t* st = smem + stage * kStageBytes;
             // int3 U^T blocks: the item's features start at n0 & 127 inside them
-            const bool u3a = pa->lorc3 != 0, u3b = GLU ? pb->lorc3 != 0 : u3a;
             if (ntok > 8) lorc_compute<GLU, 2>(st, acc, warp, lane, ra, rb, p.tcols, p.t_col_b, u3a, u3b, n0 & 127);
             else lorc_compute<GLU, 1>(st, acc, warp, lane, ra, rb, p.tcols, p.t_col_b, u3a, u3b, n0 & 127);
             __syncwarp();
@@ -731,15 +746,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         }
 
         // ------------------------------------------------------------ epilogue
-        // the lane's tokens n8 * 8 + 2c + j: undo their rows' scale 2^a
-        float inv[2][2];
-#pragma unroll
-        for (int n8 = 0; n8 < 2; ++n8)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int tok = n8 * 8 + 2 * c + j;
-                inv[n8][j] = tok < ntok ? inv_pow2(p.rscale[row0 + tok]) : 0.0f;
-            }
+        // the lane's tokens n8 * 8 + 2c + j: inv undoes their rows' scale 2^a
         if constexpr (GLU) {
             int32_t st = 0;
 #pragma unroll

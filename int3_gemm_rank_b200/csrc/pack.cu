@@ -113,6 +113,51 @@ __global__ void __launch_bounds__(128) unpack_kernel(const uint8_t* __restrict__
     for (int m = 0; m < 32; ++m) out[unit_k(c, m)] = u[m];
 }
 
+// fp64 value -> fp16 bits, rounded once to nearest even: to fp32 rounding
+// towards zero with a sticky last bit (round to odd keeps the information a
+// second rounding needs), then fp32 -> fp16 to nearest even.
+__device__ __forceinline__ uint16_t d2h_rn(double d) {
+    float f = __double2float_rz(d);
+    if (static_cast<double>(f) != d) f = __uint_as_float(__float_as_uint(f) | 1u);
+    return __half_as_ushort(__float2half_rn(f));
+}
+
+// Dequantisation of one 32-code unit of one row: w_hat = (q - z) s for the
+// unit's two groups, written as fp16 (the unfused baseline's weights).  The
+// product is exact in fp64, so each value is rounded once.
+__global__ void __launch_bounds__(128) dequant_kernel(const uint8_t* __restrict__ blob, int N, int K,
+                                                       uint16_t* __restrict__ out) {
+    const int SB = K / 128;
+    const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (gid >= static_cast<long long>(N) * SB * 4) return;
+    const int c = static_cast<int>(gid & 3);
+    const long long nb = gid / 4;
+    const int n = static_cast<int>(nb / SB), b = static_cast<int>(nb % SB);
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(blob + blob_words(n, b, SB)) + 3 * c;
+    const uint32_t w[3] = {src[0], src[1], src[2]};
+    uint16_t v[32];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint16_t* sz = reinterpret_cast<const uint16_t*>(blob + blob_group(n, 2 * b + h, SB));
+        const double s = static_cast<double>(__half2float(__ushort_as_half(sz[0])));
+        const double z = static_cast<double>(__half2float(__ushort_as_half(sz[1])));
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+            v[16 * h + m] = d2h_rn((static_cast<double>(unit_code(w, 16 * h + m)) - z) * s);
+    }
+    uint16_t* row = out + static_cast<size_t>(n) * K + 128 * b;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint4* o = reinterpret_cast<uint4*>(row + 64 * h + 16 * c);
+        uint32_t p[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            p[i] = static_cast<uint32_t>(v[16 * h + 2 * i]) | (static_cast<uint32_t>(v[16 * h + 2 * i + 1]) << 16);
+        o[0] = make_uint4(p[0], p[1], p[2], p[3]);
+        o[1] = make_uint4(p[4], p[5], p[6], p[7]);
+    }
+}
+
 }  // namespace milo
 
 using namespace milo;
@@ -156,4 +201,20 @@ extern "C" milo_status milo_packed_bytes(int32_t N, int32_t K, size_t* bytes) {
     if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_packed_bytes: K must be a multiple of 128");
     *bytes = static_cast<size_t>((N + 63) / 64) * (K / 128) * kBlockSB;
     return MILO_OK;
+}
+
+extern "C" milo_status milo_dequantize(const void* packed, int32_t N, int32_t K, uint16_t* W_hat, void* stream) {
+    clear_error();
+    if (!packed || !W_hat) return fail(MILO_ERR_INVALID_ARG, "milo_dequantize: NULL pointer");
+    if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, "milo_dequantize: N and K must be positive");
+    if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_dequantize: K must be a multiple of 128");
+    if (!aligned(packed, 16) || !aligned(W_hat, 16))
+        return fail(MILO_ERR_INVALID_ARG, "milo_dequantize: pointers must be 16-byte aligned");
+    const long long threads = static_cast<long long>(N) * (K / 128) * 4;
+    const int block = 128;
+    const long long grid = (threads + block - 1) / block;
+    if (grid > 0x7FFFFFFFLL) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_dequantize: too large");
+    dequant_kernel<<<static_cast<unsigned>(grid), block, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint8_t*>(packed), N, K, W_hat);
+    return check_launch("milo_dequantize");
 }

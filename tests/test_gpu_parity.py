@@ -87,6 +87,20 @@ def test_unpack_bit_exact(milo, N, K):
     assert np.array_equal(codes.cpu().numpy(), q)
 
 
+@pytest.mark.parametrize("N,K,mul", [(48, 384, 1.0), (130, 1408, 1.0), (64, 256, 2.0 ** -12), (16, 128, 2.0 ** 8)])
+def test_dequantize_bit_exact(milo, N, K, mul):
+    """milo_dequantize (the unfused baseline's first pass): fp16((q - z) s) for
+    every weight, bit for bit against the oracle's fp64 dequantisation rounded
+    by its own fp16 conversion; tiny weights (subnormal s) and large ones too."""
+    W = wl.gen_weight(np.random.default_rng(N + K), N, K)
+    W = wl.f32_to_f16_bits(wl.f16_bits_to_f32(W) * np.float32(mul))
+    blob = milo.milo_pack(f16_dev(W))
+    W_hat = milo.milo_dequantize(blob, N, K).cpu().numpy().view(np.uint16)
+    q, s, z, _ = oracle.quantize(W)
+    ref = oracle.d2h(oracle.dequant(q, s, z)).reshape(N, K)
+    assert np.array_equal(W_hat, ref)
+
+
 # ---------------------------------------------------------------------------
 # routing
 # ---------------------------------------------------------------------------
