@@ -271,7 +271,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         // ---------------------------------------------------------------- producer
         // the whole warp runs the loop; one elected lane issues the copies
         {
-            const uint64_t pol = l2_evict_first();
+            // weights keep the default L2 policy here: every weight tile serves
+            // all of its expert's routed-row tiles (an evict-first hint, right
+            // for the decode GEMM that reads each tile once, made them re-read)
             int stage = 0;
             uint32_t phase = 0, filled = 0, fph = 0;
             bool fail = false;
@@ -300,8 +302,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         mbar_arrive_expect_tx(fb, kTcStageTx + ntl * kBlockSB + (zs ? kTcZTile : 0));
                         tma_load_2d(st + kTcOffB, &p.b_map, fb, 128 * b, row0);
                         tma_load_2d(st + kTcOffB + kTcAtom, &p.b_map, fb, 128 * b + 64, row0);
-                        bulk_load_hint(st + kTcOffW, w0, kBlockSB, fb, pol);
-                        if (ntl == 2) bulk_load_hint(st + kTcOffW + kBlockSB, w1, kBlockSB, fb, pol);
+                        bulk_load(st + kTcOffW, w0, kBlockSB, fb);
+                        if (ntl == 2) bulk_load(st + kTcOffW + kBlockSB, w1, kBlockSB, fb);
                         if (zs) tma_load_2d(st + kTcOffZB, &p.z_map, fb, 16 * (b >> 1), row0);
                     }
                     __syncwarp();
@@ -332,8 +334,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         mbar_arrive_expect_tx(fb, nbox * kTcAtom + ua + ub);
                         for (int j = 0; j < nbox; ++j)
                             tma_load_2d(st + kTcOffB + j * kTcAtom, &p.t_map, fb, 64 * j, row0);
-                        if (ua) bulk_load_hint(st + kTcOffUA, usa, ua, fb, pol);
-                        if (ub) bulk_load_hint(st + kTcOffUB, usb, ub, fb, pol);
+                        if (ua) bulk_load(st + kTcOffUA, usa, ua, fb);
+                        if (ub) bulk_load(st + kTcOffUB, usb, ub, fb);
                     }
                     __syncwarp();
                     if (++stage == kTcStages) { stage = 0; phase ^= 1; }
@@ -757,7 +759,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                             const __half hh = __float2half_rn(hv);
                             if (!isfinite(hv)) st_bits |= MILO_DEV_NONFINITE;
                             else if (__hisinf(hh)) st_bits |= MILO_DEV_FP16_RANGE;
-                            p.h[static_cast<size_t>(row0 + t) * p.N + f] = __half_as_ushort(hh);
+                            // streaming: h (R x I fp16) is far larger than L2 and is
+                            // read once, by the next kernel
+                            __stcs(p.h + static_cast<size_t>(row0 + t) * p.N + f, __half_as_ushort(hh));
                         }
                     }
                 }
