@@ -265,7 +265,7 @@ static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
     // path: its t-items' K slices, the rows' plain copy, and their counters
     const int tslices = w.tc ? w.lp.splits : t_slices(lin->K);
     w.tpart = c.take(static_cast<size_t>(tslices) * w.R * w.tcols * 4);
-    w.nzero = lorc_counters(n_exp) + (w.tc ? 0 : gemv_sync_ints(w.R, n_exp, lin->N));
+    w.nzero = lorc_counters(n_exp) + (w.tc ? 0 : gemv_sync_ints(w.R, n_exp));
     w.done = c.take(static_cast<size_t>(w.nzero) * 4);
     w.part = c.take(static_cast<size_t>(w.splits) * w.R * lin->N * 4);
     w.plain = w.tc ? 0 : c.take(static_cast<size_t>(w.R) * lin->K * 2);
@@ -312,8 +312,8 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
     w.tpart = c.take(std::max(s13 * w.tc13, s2 * w.tc2) * w.R * 4);
     // counters, all zeroed by the first preparation: the down-projection
     // kernels', then (mma.sync path) those of the w1|w3 and w2 GEMMs
-    w.sync13 = w.tc ? 0 : gemv_sync_ints(w.R, n_exp, I);
-    w.sync2 = w.tc ? 0 : gemv_sync_ints(w.R, n_exp, H);
+    w.sync13 = w.tc ? 0 : gemv_sync_ints(w.R, n_exp);
+    w.sync2 = w.tc ? 0 : gemv_sync_ints(w.R, n_exp);
     w.nzero = lorc_counters(n_exp) + w.sync13 + w.sync2;
     w.done = c.take(static_cast<size_t>(w.nzero) * 4);
     w.part = c.take(static_cast<size_t>(w.splits) * w.R * H * 4);
@@ -354,7 +354,6 @@ static void t_items(GemvParams& g, const void* plain, void* tpart, int32_t* sync
     const int tiles = (g.R + kTokTile - 1) / kTokTile + g.n_exp;   // as gemv_sync_ints
     g.tctr = sync;
     g.tdone = sync + 4 * tiles;
-    g.nctr = sync + 5 * tiles;
 }
 
 // The grouped GEMM described by g on the tcgen05 kernel: activations in

@@ -46,7 +46,6 @@
 
 #include <atomic>
 
-#include "milo_combine.cuh"
 #include "milo_device.cuh"
 #include "milo_host.h"
 #include "milo_kernels.h"
@@ -778,42 +777,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                         if (tok < ntok && n < p.N)
                             out[static_cast<size_t>(row0 + tok) * p.N + n] = acc[ti][n8][i] * inv[n8][i & 1];
                     }
-            if (p.fuse_combine) {
-                // the item that completes this output tile combines its columns
-                __threadfence();
-                consumer_sync();
-                if (threadIdx.x == 0)
-                    *bcast = atomicAdd(&p.nctr[w.ntile], 1) == ttb[p.n_exp] * p.splits - 1;
-                consumer_sync();
-                const bool last = *bcast != 0;
-                consumer_sync();
-                if (last) {
-                    __threadfence();
-                    int32_t cst = 0;
-                    const int rows_out = p.comb.per_slot ? p.comb.T * p.comb.k : p.comb.T;
-                    const int quads = min(RA, p.N - n0) / 4;
-                    for (int i = threadIdx.x; i < rows_out * quads; i += 32 * kConsumerWarps) {
-                        const int o = i / quads, n = n0 + 4 * (i % quads);
-                        store4(p.comb, static_cast<size_t>(o) * p.N + n, combine4(p.comb, o, n), cst);
-                    }
-                    flag(p.dev_status, cst);
-                }
-            }
         }
-    }
-    // No rows at all: nothing completes an output tile, so the CTAs combine
-    // (zeros, for dropped slots) tile by tile.
-    if (!GLU && p.fuse_combine && n_items == 0) {
-        int32_t cst = 0;
-        const int rows_out = p.comb.per_slot ? p.comb.T * p.comb.k : p.comb.T;
-        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-            const int n0 = tile * RA, quads = min(RA, p.N - n0) / 4;
-            for (int i = threadIdx.x; i < rows_out * quads; i += 32 * kConsumerWarps) {
-                const int o = i / quads, n = n0 + 4 * (i % quads);
-                store4(p.comb, static_cast<size_t>(o) * p.N + n, combine4(p.comb, o, n), cst);
-            }
-        }
-        flag(p.dev_status, cst);
     }
 }
 

@@ -88,18 +88,13 @@ struct GemvParams {
     float* tpart;               // [nks][R][tcols] f32 slice partials
     int32_t* tctr;              // per (expert, token tile, rank block): slices finished (0 on entry)
     int32_t* tdone;             // per (expert, token tile): rank blocks finished (0 on entry)
-    // Fused combine (plain kernel): the last item of each 128-row output tile
-    // combines the tile's columns of every output row.
-    int fuse_combine;
-    int32_t* nctr;              // per output tile: items finished (0 on entry)
-    CombineParams comb;
 };
 
-// Ints of the t-item and combine counters of a grouped GEMM over R rows,
-// n_exp experts and N outputs (zeroed before each launch).
-inline int gemv_sync_ints(int R, int n_exp, int N) {
+// Ints of the t-item counters of a grouped GEMM over R rows and n_exp experts
+// (zeroed before each launch).
+inline int gemv_sync_ints(int R, int n_exp) {
     const int tiles = (R + kTokTile - 1) / kTokTile + n_exp;   // token tiles of all experts, at most
-    return tiles * 4 + tiles + (N + kRowsPlain - 1) / kRowsPlain;
+    return tiles * 4 + tiles;
 }
 
 // Parameters of the tcgen05 grouped GEMM for large per-expert row counts
