@@ -111,6 +111,18 @@ __device__ __forceinline__ int rank_blocks(int r) { return (r + 31) >> 5; }
 // Named barrier of the four consumer warps (the producer warp is not in it).
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// GPU-scope counters: an acquire-release add (returns the old value) and a
+// release add.  A CTA barrier before them orders the CTA's other threads'
+// writes too (the release is cumulative).
+__device__ __forceinline__ int atom_add_acq_rel(int32_t* p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ void red_add_release(int32_t* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ int ld_acquire(const int32_t* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -198,13 +210,13 @@ __device__ void titem_run(const GemvParams& p, int j, const int* tstart, const i
             const int rr = g + 8 * (i >> 1), rk = rk0 + 2 * c + (i & 1);
             if (rr < ntok && rk < r) part[static_cast<size_t>(row0 + rr) * p.tcols + col0 + 2 * c + (i & 1)] = acc[i];
         }
-        __threadfence();
+        // the CTA's partials, then one thread's acquire-release count: the last
+        // slice to count sees every other slice's partials
         consumer_sync();
-        if (threadIdx.x == 0) *bcast = atomicAdd(&p.tctr[j / p.nks], 1) == p.nks - 1;
+        if (threadIdx.x == 0) *bcast = atom_add_acq_rel(&p.tctr[j / p.nks], 1) == p.nks - 1;
         consumer_sync();
         const bool last = *bcast != 0;
         if (last) {
-            __threadfence();
             const size_t slice = static_cast<size_t>(p.R) * p.tcols;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -223,9 +235,8 @@ __device__ void titem_run(const GemvParams& p, int j, const int* tstart, const i
             return;
         }
     }
-    __threadfence();
-    consumer_sync();
-    if (threadIdx.x == 0) atomicAdd(&p.tdone[ttb[e] + tt], 1);
+    consumer_sync();          // t is written; one release publishes it
+    if (threadIdx.x == 0) red_add_release(&p.tdone[ttb[e] + tt], 1);
     flag(p.dev_status, st);
 }
 
