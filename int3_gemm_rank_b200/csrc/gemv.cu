@@ -160,14 +160,14 @@ __device__ __forceinline__ uint4 lorc3_v8(const uint8_t* blob, int j, int k) {
 // last adds the slices in order (deterministic) and writes t, then counts
 // the rank block done for the token tile.
 template <bool GLU>
-__device__ void titem_run(const GemvParams& p, int j, const int* tstart, const int* ttb, const int* cnt,
-                          const int* row0s, int warp, int lane, volatile int* bcast) {
-    const int e = find_expert(j, tstart, 1, p.n_exp);
+__device__ void titem_run(const GemvParams& p, int j, int nks, int kslice, const int* tstart, const int* ttb,
+                          const int* cnt, const int* row0s, int warp, int lane, volatile int* bcast) {
+    const int e = find_expert(j, tstart, nks, p.n_exp);
     const ProjDev* pa = p.table + e * p.stride + p.proj_a;
     const ProjDev* pb = p.table + e * p.stride + p.proj_b;
     const int na = rank_blocks(pa->rank), nb = GLU ? rank_blocks(pb->rank) : 0;
-    const int local = j - tstart[e];
-    const int ks = local % p.nks, rest = local / p.nks;
+    const int local = j - tstart[e] * nks;
+    const int ks = local % nks, rest = local / nks;
     const int rbi = rest % (na + nb), tt = rest / (na + nb);
     const bool second = rbi >= na;
     const ProjDev* P = second ? pb : pa;
@@ -181,7 +181,7 @@ __device__ void titem_run(const GemvParams& p, int j, const int* tstart, const i
     const uint16_t* xr1 = g + 8 < ntok ? p.src + static_cast<size_t>(row0 + g + 8) * p.K : nullptr;
     const int jr = rk0 + g;                      // the lane's V row
     const bool vrow = jr < r;
-    const int kb0 = ks * p.kslice, kb1 = min(p.K, kb0 + p.kslice);
+    const int kb0 = ks * kslice, kb1 = min(p.K, kb0 + kslice);
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll 16
@@ -196,7 +196,7 @@ __device__ void titem_run(const GemvParams& p, int j, const int* tstart, const i
         mma16816(acc, xa.z, xb.z, xa.w, xb.w, v.z, v.w);
     }
     // acc[i]: row g + 8 (i >> 1), rank rk0 + 2c + (i & 1); only ranks < r are stored
-    if (p.nks == 1) {
+    if (nks == 1) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int rr = g + 8 * (i >> 1), rk = rk0 + 2 * c + (i & 1);
@@ -213,7 +213,7 @@ __device__ void titem_run(const GemvParams& p, int j, const int* tstart, const i
         // the CTA's partials, then one thread's acquire-release count: the last
         // slice to count sees every other slice's partials
         consumer_sync();
-        if (threadIdx.x == 0) *bcast = atom_add_acq_rel(&p.tctr[j / p.nks], 1) == p.nks - 1;
+        if (threadIdx.x == 0) *bcast = atom_add_acq_rel(&p.tctr[j / nks], 1) == nks - 1;
         consumer_sync();
         const bool last = *bcast != 0;
         if (last) {
@@ -224,7 +224,7 @@ __device__ void titem_run(const GemvParams& p, int j, const int* tstart, const i
                 if (rr < ntok && rk < r) {
                     const size_t o = static_cast<size_t>(row0 + rr) * p.tcols + col0 + 2 * c + (i & 1);
                     float v = 0.0f;
-                    for (int s2 = 0; s2 < p.nks; ++s2) v += __ldcg(p.tpart + s2 * slice + o);
+                    for (int s2 = 0; s2 < nks; ++s2) v += __ldcg(p.tpart + s2 * slice + o);
                     p.t[o] = t_half(v, st);
                 }
             }
@@ -469,7 +469,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         if (p.t_items && tte > 0) {
             const int na = rank_blocks(p.table[e * p.stride + p.proj_a].rank);
             const int nb = GLU ? rank_blocks(p.table[e * p.stride + p.proj_b].rank) : 0;
-            nt = tte * (na + nb) * p.nks;
+            nt = tte * (na + nb);
         }
         tstart[e] = nt;
     }
@@ -500,7 +500,16 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     }
     __syncthreads();
     const int n_items = ttb[p.n_exp] * n_tiles * p.splits;
-    const int n_t = tstart[p.n_exp];
+    // K slices of the t-items: about one t-item per CTA (each slice pays a
+    // fixed cost in counting and partial sums), at most p.nks slices of at
+    // least p.kslice; every CTA derives the same values from the same tables
+    int nks = 1, kslice = p.K;
+    if (p.t_items && tstart[p.n_exp] > 0) {
+        nks = max(1, min(p.nks, static_cast<int>(gridDim.x) / tstart[p.n_exp]));
+        kslice = (((p.K + nks - 1) / nks) + 31) / 32 * 32;
+        nks = (p.K + kslice - 1) / kslice;
+    }
+    const int n_t = tstart[p.n_exp] * nks;
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------------ producer
@@ -685,7 +694,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         const int it = stage_item[stage];
         if (it == -1) break;
         if (it < -1) {           // a t-item: its stage carries no data
-            titem_run<GLU>(p, -2 - it, tstart, ttb, cnt, row0s, warp, lane, bcast);
+            titem_run<GLU>(p, -2 - it, nks, kslice, tstart, ttb, cnt, row0s, warp, lane, bcast);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
             if (++stage == kStages) { stage = 0; phase ^= 1; }

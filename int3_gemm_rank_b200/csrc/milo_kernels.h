@@ -84,7 +84,8 @@ struct GemvParams {
     // until its token tile's t is complete before copying it.
     int t_items;                // 0: t was computed beforehand
     const uint16_t* src;        // the rows' plain fp16 copy [R][K] (times their scale 2^a)
-    int nks, kslice;            // K slices per t-item and their length (multiple of 32)
+    int nks, kslice;            // the most K slices per t-item and their least length (multiple of
+                                // 32): the kernel picks fewer, longer slices when t-items are many
     float* tpart;               // [nks][R][tcols] f32 slice partials
     int32_t* tctr;              // per (expert, token tile, rank block): slices finished (0 on entry)
     int32_t* tdone;             // per (expert, token tile): rank blocks finished (0 on entry)
