@@ -112,6 +112,11 @@ static milo_status fill_proj(ProjDev* d, const milo_qweight& w, int N, int K, co
     d->N = N;
     d->K = K;
     d->lorc3 = int3 ? 1 : 0;
+    // fp16 V for the mma.sync GEMM's t-items: 32 rank rows x 64 of K per box
+    // (rows past the rank read as zeros)
+    if (w.rank > 0 && !int3)
+        return make_map(&d->vmap, w.V, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, static_cast<uint64_t>(K), w.rank,
+                        static_cast<uint64_t>(K) * 2, 64, 32, "V", CU_TENSOR_MAP_SWIZZLE_128B);
     return MILO_OK;
 }
 
@@ -234,12 +239,10 @@ static LorcPlan lorc_plan(int n_exp, int nproj, int K, long long max_rows) {
     return pl;
 }
 
-// K slices of the compensator's t-items inside the mma.sync GEMM: short
-// enough that all of a slice's loads are in flight at once (a lane loads 8
-// values per 32 of K), so that t is ready long before the first GEMM items
-// reach their compensator stage; longer for very long K, where the number of
-// slices to add up would grow.
-static int t_slice_len(int K) { return K <= 4096 ? 256 : 512; }
+// K slices of the compensator's t-items inside the mma.sync GEMM: at least
+// two pipeline stages (256 of K each) per slice, and at most this many slices
+// (the kernel takes fewer, longer ones when the t-items outnumber the CTAs).
+static int t_slice_len(int) { return 512; }
 static int t_slices(int K) { return (K + t_slice_len(K) - 1) / t_slice_len(K); }
 
 static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
@@ -345,7 +348,7 @@ static milo_status run_gemv(GemvParams& g, bool glu, cudaStream_t st, const char
 
 // The t-items of a grouped GEMM on the mma.sync path: the compensator's t from
 // the rows' plain copy, K slices and counters in the workspace.
-static void t_items(GemvParams& g, const void* plain, void* tpart, int32_t* sync) {
+static milo_status t_items(GemvParams& g, const void* plain, void* tpart, int32_t* sync) {
     g.t_items = g.has_t ? 1 : 0;
     g.src = static_cast<const uint16_t*>(plain);
     g.kslice = t_slice_len(g.K);
@@ -354,6 +357,10 @@ static void t_items(GemvParams& g, const void* plain, void* tpart, int32_t* sync
     const int tiles = (g.R + kTokTile - 1) / kTokTile + g.n_exp;   // as gemv_sync_ints
     g.tctr = sync;
     g.tdone = sync + 4 * tiles;
+    if (!g.has_t) return MILO_OK;
+    return make_map(&g.smap, plain, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, static_cast<uint64_t>(g.K),
+                    static_cast<uint64_t>(g.R), static_cast<uint64_t>(g.K) * 2, 64, kTokTile, "plain rows",
+                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // The grouped GEMM described by g on the tcgen05 kernel: activations in
@@ -619,8 +626,9 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     if (tc) {
         s = run_tc(g, false, base + w.frag, base + w.gsum, st, "tc gemm");
     } else {
-        t_items(g, base + w.plain, base + w.tpart, reinterpret_cast<int32_t*>(base + w.done) + lorc_counters(lin->n_experts));
-        s = run_gemv(g, false, st, "gemv");
+        s = t_items(g, base + w.plain, base + w.tpart,
+                    reinterpret_cast<int32_t*>(base + w.done) + lorc_counters(lin->n_experts));
+        if (s == MILO_OK) s = run_gemv(g, false, st, "gemv");
     }
     if (s != MILO_OK) return s;
     prof_record(1, st);
@@ -727,8 +735,8 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     if (tc) {
         s = run_tc(g1, true, base + w.xfrag, base + w.xg, st, "tc gemm w1|w3");
     } else {
-        t_items(g1, base + w.xplain, base + w.tpart, sync);
-        s = run_gemv(g1, true, st, "gemv w1|w3");
+        s = t_items(g1, base + w.xplain, base + w.tpart, sync);
+        if (s == MILO_OK) s = run_gemv(g1, true, st, "gemv w1|w3");
     }
     if (s != MILO_OK) return s;
     prof_record(1, st);
@@ -793,8 +801,8 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     if (tc) {
         s = run_tc(g2, false, base + w.hfrag, base + w.hg, st, "tc gemm w2");
     } else {
-        t_items(g2, base + w.hplain, base + w.tpart, sync + w.sync13);
-        s = run_gemv(g2, false, st, "gemv w2");
+        s = t_items(g2, base + w.hplain, base + w.tpart, sync + w.sync13);
+        if (s == MILO_OK) s = run_gemv(g2, false, st, "gemv w2");
     }
     if (s != MILO_OK) return s;
     prof_record(3, st);

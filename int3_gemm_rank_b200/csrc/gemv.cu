@@ -59,17 +59,22 @@ constexpr int kGemvThreads = 32 * (kConsumerWarps + 1);
 // (tile, super-block) blocks of the packed blob: per super-block the codes
 // [64 rows][12 words], then its two groups' (s, z) pairs (GLU: w1's tile,
 // then w3's; plain: rows 0-63, then 64-127).  Then the activations
-// [16 rows][272 fp16].
+// [16 rows][272 fp16].  Stages are 1024-byte aligned for the t-items' swizzled
+// TMA boxes, which fill a whole stage.
 constexpr int kTileBlk = 2 * kBlockSB;                    // 7168
 constexpr int kOffQ = 0;
 constexpr int kOffX = 2 * kTileBlk;                       // 14336
-constexpr int kStageBytes = kOffX + kTokTile * kFragRowHalves * 2;
+constexpr int kStageBytes = 23552;
 constexpr int kOffUA = 0, kOffUB = 8192, kOffT = 16384;   // compensator stage
 constexpr int kBarOffset = kStages * kStageBytes;
 // barriers, then the item tables cnt, row0s, ttb, tstart [MILO_MAX_EXPERTS + 1],
-// the stage headers and the consumers' broadcast word
-constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 4 * (MILO_MAX_EXPERTS + 1) * 4 + kStages * 4 + 16;
+// the stage headers and the consumers' broadcast word; 1 KB of slack to align
+// the base
+constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 4 * (MILO_MAX_EXPERTS + 1) * 4 + kStages * 4 + 16 + 1024;
 
+static_assert(kOffX + kTokTile * kFragRowHalves * 2 <= kStageBytes, "GEMM stage");
+static_assert(kStageBytes % 1024 == 0, "stage alignment");
+static_assert(3 * (kSmemBytes + 1024) <= 228 * 1024, "three CTAs per SM (1 KB reserved per CTA)");
 static_assert(kStageBytes % 16 == 0 && kOffX % 16 == 0 && kTileBlk % 16 == 0, "bulk-copy alignment");
 static_assert(kOffT >= kRowsPlain * MILO_MAX_RANK * 2, "compensator stage: U rows");
 static_assert(kOffT + kTokTile * 2 * MILO_MAX_RANK * 2 <= kStageBytes, "compensator stage: t rows");
@@ -150,52 +155,118 @@ __device__ __forceinline__ uint4 lorc3_v8(const uint8_t* blob, int j, int k) {
     return make_uint4(h[0], h[1], h[2], h[3]);
 }
 
-// t-item j (consumer warps): t[row][col] = fp16(sum_k x'[row][k] V[rank][k])
-// for the 16 rows of one token tile of expert e, 32 ranks of one projection
-// (8 per warp) and one K slice; x' is the prepared rows' plain fp16 copy
-// (already times their scale 2^a).  Each lane loads 8 consecutive k of its
-// two rows and of its V row with 16-byte loads and uses them as two k16 MMA
-// steps (the same relabelling of k on both operands, so the sum is
-// unchanged).  The slice's f32 partials go to tpart; the slice that finishes
-// last adds the slices in order (deterministic) and writes t, then counts
-// the rank block done for the token tile.
+// A t-item: t[row][col] = fp16(sum_k x'[row][k] V[rank][k]) for the 16 rows
+// of one token tile of expert e, 32 ranks of one projection (8 per consumer
+// warp) and one K slice; x' is the prepared rows' plain fp16 copy (already
+// times their scale 2^a).  Items j of expert e are [tstart[e], tstart[e+1])
+// * nks, K slices fastest, then rank blocks, then token tiles.
+struct TItem {
+    const ProjDev* P;     // the projection whose V it multiplies
+    int e, ks, tt;        // expert, K slice, token tile
+    int rb;               // first rank of the block
+    int col;              // column of that rank in t
+};
+
 template <bool GLU>
-__device__ void titem_run(const GemvParams& p, int j, int nks, int kslice, const int* tstart, const int* ttb,
-                          const int* cnt, const int* row0s, int warp, int lane, volatile int* bcast) {
-    const int e = find_expert(j, tstart, nks, p.n_exp);
-    const ProjDev* pa = p.table + e * p.stride + p.proj_a;
-    const ProjDev* pb = p.table + e * p.stride + p.proj_b;
+__device__ __forceinline__ TItem decode_titem(const GemvParams& p, int j, int nks, const int* tstart) {
+    TItem t;
+    t.e = find_expert(j, tstart, nks, p.n_exp);
+    const ProjDev* pa = p.table + t.e * p.stride + p.proj_a;
+    const ProjDev* pb = p.table + t.e * p.stride + p.proj_b;
     const int na = rank_blocks(pa->rank), nb = GLU ? rank_blocks(pb->rank) : 0;
-    const int local = j - tstart[e] * nks;
-    const int ks = local % nks, rest = local / nks;
-    const int rbi = rest % (na + nb), tt = rest / (na + nb);
+    const int local = j - tstart[t.e] * nks;
+    t.ks = local % nks;
+    const int rest = local / nks;
+    const int rbi = rest % (na + nb);
+    t.tt = rest / (na + nb);
     const bool second = rbi >= na;
-    const ProjDev* P = second ? pb : pa;
-    const int r = P->rank;
-    const int rk0 = 32 * (second ? rbi - na : rbi) + 8 * warp;        // the warp's first rank
-    const int col0 = (second ? p.t_col_b : 0) + rk0;
-    const int row0 = row0s[e] + kTokTile * tt, ntok = min(kTokTile, cnt[e] - kTokTile * tt);
+    t.P = second ? pb : pa;
+    t.rb = 32 * (second ? rbi - na : rbi);
+    t.col = (second ? p.t_col_b : 0) + t.rb;
+    return t;
+}
+
+// t-item stage (fp16 V): per 64 of K one TMA box of the 16 rows' plain copy
+// and one of the block's 32 V rows, both 128-byte rows with the 128-byte
+// swizzle; three of each per stage.
+constexpr int kTBoxes = 3;
+constexpr int kTStageK = 64 * kTBoxes;                    // 192
+constexpr int kOffTX = 0, kTXBox = kTokTile * 128;        // 2048
+constexpr int kOffTV = kTBoxes * kTXBox, kTVBox = 32 * 128;   // 6144, 4096
+static_assert(kOffTV + kTBoxes * kTVBox <= kStageBytes && kOffTV % 1024 == 0, "t-item stage");
+
+// Consumer side of a t-item with fp16 V: its stages (the first one already
+// waited for) as m16n8k16 MMAs, A = the 16 rows (ldmatrix), B = the warp's 8
+// V rows (ldmatrix), each stage released after use.  False on a timeout.
+__device__ bool titem_tma(const TItem& ti, int kb0, int kb1, const uint8_t* smem, uint64_t* full,
+                          uint64_t* empty, int& stage, uint32_t& phase, int warp, int lane, float (&acc)[4]) {
+    const bool active = ti.rb + 8 * warp < ti.P->rank;   // the warp's 8 ranks exist
+    const int arow = (lane & 7) + 8 * ((lane >> 3) & 1), achk = lane >> 4;
+    const int brow = 8 * warp + (lane & 7), bchk = lane >> 3;
+    for (int kc = kb0; kc < kb1; kc += kTStageK) {
+        if (kc != kb0 && !warp_wait(&full[stage], phase)) return false;
+        const uint8_t* st = smem + stage * kStageBytes;
+        const int nbox = min(kTBoxes, (kb1 - kc) / 64);
+        if (active) {
+#pragma unroll
+            for (int q = 0; q < kTBoxes; ++q) {
+                if (q == nbox) break;
+                const uint8_t* xb = st + kOffTX + q * kTXBox;
+                const uint8_t* vb = st + kOffTV + q * kTVBox;
+#pragma unroll
+                for (int s2 = 0; s2 < 4; s2 += 2) {
+                    uint32_t b[4];
+                    ldmatrix_x4(b, vb + swz128(brow, 2 * s2 + bchk));
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t a[4];
+                        ldmatrix_x4(a, xb + swz128(arow, 2 * (s2 + h) + achk));
+                        mma16816(acc, a[0], a[1], a[2], a[3], b[2 * h], b[2 * h + 1]);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+    }
+    return true;
+}
+
+// t-item with an int3 V (no stage data): each lane loads 8 consecutive k of
+// its two rows and dequantises 8 of its V row, used as two k16 MMA steps (the
+// same relabelling of k on both operands, so the sum is unchanged).
+__device__ void titem_lorc3(const GemvParams& p, const TItem& ti, int kb0, int kb1, int row0, int ntok, int warp,
+                            int lane, float (&acc)[4]) {
     const int g = lane >> 2, c = lane & 3;
-    int32_t st = 0;
     const uint16_t* xr0 = g < ntok ? p.src + static_cast<size_t>(row0 + g) * p.K : nullptr;
     const uint16_t* xr1 = g + 8 < ntok ? p.src + static_cast<size_t>(row0 + g + 8) * p.K : nullptr;
-    const int jr = rk0 + g;                      // the lane's V row
-    const bool vrow = jr < r;
-    const int kb0 = ks * kslice, kb1 = min(p.K, kb0 + kslice);
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const int jr = ti.rb + 8 * warp + g;          // the lane's V row
+    const uint8_t* blob = reinterpret_cast<const uint8_t*>(ti.P->V);
+    if (ti.rb + 8 * warp >= ti.P->rank) return;
     const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll 16
+#pragma unroll 4
     for (int kb = kb0; kb < kb1; kb += 32) {
         const int k = kb + 8 * c;
         const uint4 xa = xr0 ? __ldg(reinterpret_cast<const uint4*>(xr0 + k)) : z4;
         const uint4 xb = xr1 ? __ldg(reinterpret_cast<const uint4*>(xr1 + k)) : z4;
-        const uint4 v = !vrow ? z4
-                        : P->lorc3 ? lorc3_v8(reinterpret_cast<const uint8_t*>(P->V), jr, k)
-                                   : __ldg(reinterpret_cast<const uint4*>(P->V + static_cast<size_t>(jr) * p.K + k));
+        const uint4 v = lorc3_v8(blob, jr, k);
         mma16816(acc, xa.x, xb.x, xa.y, xb.y, v.x, v.y);
         mma16816(acc, xa.z, xb.z, xa.w, xb.w, v.z, v.w);
     }
-    // acc[i]: row g + 8 (i >> 1), rank rk0 + 2c + (i & 1); only ranks < r are stored
+}
+
+// End of t-item j: acc[i] is row g + 8 (i >> 1), rank 2c + (i & 1) of the
+// warp's 8 (only ranks below the projection's are stored).  One slice: t
+// directly.  Otherwise the slice's f32 partials go to tpart; the slice that
+// counts last adds the slices in order (deterministic) and writes t.  The
+// CTA that writes t then counts the rank block done for the token tile.
+template <bool GLU>
+__device__ void titem_finish(const GemvParams& p, const TItem& ti, int j, int nks, int row0, int ntok,
+                             const int* ttb, const float (&acc)[4], int warp, int lane, volatile int* bcast) {
+    const int g = lane >> 2, c = lane & 3;
+    const int rk0 = ti.rb + 8 * warp, col0 = ti.col + 8 * warp, r = ti.P->rank;
+    int32_t st = 0;
     if (nks == 1) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -204,7 +275,7 @@ __device__ void titem_run(const GemvParams& p, int j, int nks, int kslice, const
                 p.t[static_cast<size_t>(row0 + rr) * p.tcols + col0 + 2 * c + (i & 1)] = t_half(acc[i], st);
         }
     } else {
-        float* part = p.tpart + static_cast<size_t>(ks) * p.R * p.tcols;
+        float* part = p.tpart + static_cast<size_t>(ti.ks) * p.R * p.tcols;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int rr = g + 8 * (i >> 1), rk = rk0 + 2 * c + (i & 1);
@@ -236,7 +307,7 @@ __device__ void titem_run(const GemvParams& p, int j, int nks, int kslice, const
         }
     }
     consumer_sync();          // t is written; one release publishes it
-    if (threadIdx.x == 0) red_add_release(&p.tdone[ttb[e] + tt], 1);
+    if (threadIdx.x == 0) red_add_release(&p.tdone[ttb[ti.e] + ti.tt], 1);
     flag(p.dev_status, st);
 }
 
@@ -432,7 +503,8 @@ __device__ __forceinline__ void lorc_compute(const uint8_t* st, float (&acc)[2][
 
 template <bool GLU>
 __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_constant__ GemvParams p) {
-    extern __shared__ __align__(1024) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
     uint64_t* empty = full + kStages;
     int* cnt = reinterpret_cast<int*>(empty + kStages);
@@ -501,12 +573,13 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     __syncthreads();
     const int n_items = ttb[p.n_exp] * n_tiles * p.splits;
     // K slices of the t-items: about one t-item per CTA (each slice pays a
-    // fixed cost in counting and partial sums), at most p.nks slices of at
-    // least p.kslice; every CTA derives the same values from the same tables
+    // fixed cost in counting and partial sums), at most p.nks slices, each a
+    // whole number of stages; every CTA derives the same values from the same
+    // tables
     int nks = 1, kslice = p.K;
     if (p.t_items && tstart[p.n_exp] > 0) {
         nks = max(1, min(p.nks, static_cast<int>(gridDim.x) / tstart[p.n_exp]));
-        kslice = (((p.K + nks - 1) / nks) + 31) / 32 * 32;
+        kslice = (((p.K + nks - 1) / nks) + kTStageK - 1) / kTStageK * kTStageK;
         nks = (p.K + kslice - 1) / kslice;
     }
     const int n_t = tstart[p.n_exp] * nks;
@@ -531,19 +604,40 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         int tj = S - 1 - static_cast<int>(blockIdx.x);
         int next = blockIdx.x;
         for (;;) {
-            if (tj < n_t) {      // a t-item: a header-only stage
-                if (!warp_wait(&empty[stage], phase ^ 1)) {
-                    fail = true;
-                    break;
+            if (tj < n_t) {
+                // a t-item: with fp16 V its stages of plain rows and V rows by
+                // TMA; with an int3 V one header-only stage
+                const TItem ti = decode_titem<GLU>(p, tj, nks, tstart);
+                const int kb0 = ti.ks * kslice, kb1 = min(p.K, kb0 + kslice);
+                const int trow0 = row0s[ti.e] + kTokTile * ti.tt;
+                const bool l3 = ti.P->lorc3 != 0;
+                for (int kc = kb0; kc < kb1; kc += kTStageK) {
+                    if (!warp_wait(&empty[stage], phase ^ 1)) {
+                        fail = true;
+                        break;
+                    }
+                    uint8_t* st = smem + stage * kStageBytes;
+                    uint64_t* fb = &full[stage];
+                    filled |= 1u << stage;
+                    fph = (fph & ~(1u << stage)) | (phase << stage);
+                    const int nbox = min(kTBoxes, (kb1 - kc) / 64);
+                    if (elect_one()) {
+                        if (kc == kb0) stage_item[stage] = -2 - tj;
+                        if (l3) {
+                            mbar_arrive(fb);
+                        } else {
+                            mbar_arrive_expect_tx(fb, nbox * (kTXBox + kTVBox));
+                            for (int q = 0; q < nbox; ++q) {
+                                tma_load_2d(st + kOffTX + q * kTXBox, &p.smap, fb, kc + 64 * q, trow0);
+                                tma_load_2d(st + kOffTV + q * kTVBox, &ti.P->vmap, fb, kc + 64 * q, ti.rb);
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (++stage == kStages) { stage = 0; phase ^= 1; }
+                    if (l3) break;
                 }
-                filled |= 1u << stage;
-                fph = (fph & ~(1u << stage)) | (phase << stage);
-                if (elect_one()) {
-                    stage_item[stage] = -2 - tj;
-                    mbar_arrive(&full[stage]);
-                }
-                __syncwarp();
-                if (++stage == kStages) { stage = 0; phase ^= 1; }
+                if (fail) break;
                 tj += S;
                 continue;
             }
@@ -693,11 +787,23 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         }
         const int it = stage_item[stage];
         if (it == -1) break;
-        if (it < -1) {           // a t-item: its stage carries no data
-            titem_run<GLU>(p, -2 - it, nks, kslice, tstart, ttb, cnt, row0s, warp, lane, bcast);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
-            if (++stage == kStages) { stage = 0; phase ^= 1; }
+        if (it < -1) {           // a t-item
+            const int j = -2 - it;
+            const TItem ti = decode_titem<GLU>(p, j, nks, tstart);
+            const int kb0 = ti.ks * kslice, kb1 = min(p.K, kb0 + kslice);
+            const int trow0 = row0s[ti.e] + kTokTile * ti.tt;
+            const int tntok = min(kTokTile, cnt[ti.e] - kTokTile * ti.tt);
+            float tacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            if (ti.P->lorc3) {   // its one stage carries no data
+                titem_lorc3(p, ti, kb0, kb1, trow0, tntok, warp, lane, tacc);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
+                if (++stage == kStages) { stage = 0; phase ^= 1; }
+            } else if (!titem_tma(ti, kb0, kb1, smem, full, empty, stage, phase, warp, lane, tacc)) {
+                flag(p.dev_status, MILO_DEV_TIMEOUT);
+                return;
+            }
+            titem_finish<GLU>(p, ti, j, nks, trow0, tntok, ttb, tacc, warp, lane, bcast);
             continue;
         }
         bool waited = true;       // the next stage's barrier has been passed already

@@ -318,6 +318,21 @@ __device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint3
         ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy) : "memory");
 }
 
+// Four 8x8 b16 matrices from shared memory: lane l gives the address of row
+// l % 8 of matrix l / 8; lane t receives, of each matrix, row t / 4, elements
+// 2 (t % 4) and 2 (t % 4) + 1.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(smem_u32(p)));
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a tile of
+// 128-byte rows written by TMA with the 128-byte swizzle (tile base 1024-byte
+// aligned): the chunk index is XORed with the row index modulo 8.
+__device__ __forceinline__ uint32_t swz128(int row, int chunk) {
+    return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
 // ---------------------------------------------------------------------------
 // PTX: warp-level MMA  D[16x8] (+)= A[16x16] * B[16x8], fp16 in, fp32 accumulate
 // ---------------------------------------------------------------------------

@@ -47,6 +47,7 @@ constexpr int kTcTokens = 128;               // routed rows per tcgen05 work ite
 
 // One projection in the device table (device pointers and shape).
 struct alignas(64) ProjDev {
+    CUtensorMap vmap;           // fp16 V [rank][K]: box {64, 32}, 128-byte swizzle (unset for lorc3 or rank 0)
     const uint8_t* packed;      // blob of ceil(N/64) * (K/128) * kBlockSB bytes
     const uint16_t* U;          // [N][rank] fp16, or (lorc3) the blob of U^T [rank][N]; NULL when rank == 0
     const uint16_t* V;          // [rank][K] fp16, or (lorc3) the blob of V [rank][K]; NULL when rank == 0
@@ -64,6 +65,7 @@ struct CombineParams {
 };
 
 struct GemvParams {
+    CUtensorMap smap;           // the rows' plain fp16 copy `src` [R][K]: box {64, 16}, 128-byte swizzle
     const uint16_t* x;          // prepared activations [chunks][R][kFragRowHalves] fp16
                                 // (group sums in each row's padding, see kGsumHalf)
     const float* rscale;        // [R]: the row's activation scale 2^a (see kFoldScale)
@@ -85,7 +87,7 @@ struct GemvParams {
     int t_items;                // 0: t was computed beforehand
     const uint16_t* src;        // the rows' plain fp16 copy [R][K] (times their scale 2^a)
     int nks, kslice;            // the most K slices per t-item and their least length (multiple of
-                                // 32): the kernel picks fewer, longer slices when t-items are many
+                                // 256): the kernel picks fewer, longer slices when t-items are many
     float* tpart;               // [nks][R][tcols] f32 slice partials
     int32_t* tctr;              // per (expert, token tile, rank block): slices finished (0 on entry)
     int32_t* tdone;             // per (expert, token tile): rank blocks finished (0 on entry)
