@@ -110,8 +110,13 @@ __device__ __forceinline__ Item decode_item(int it, const int* ttb, const int* c
     return r;
 }
 
-// Rank blocks of 32 of a projection (t-items).
+// t-items of a projection per token tile and K slice: one per 32 ranks of an
+// fp16 V, one for an int3 V (its one 64-row tile).
 __device__ __forceinline__ int rank_blocks(int r) { return (r + 31) >> 5; }
+__device__ __forceinline__ int t_blocks(const ProjDev* P) {
+    const int r = P->rank;
+    return r == 0 ? 0 : P->lorc3 ? 1 : rank_blocks(r);
+}
 
 // Named barrier of the four consumer warps (the producer warp is not in it).
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -134,27 +139,6 @@ __device__ __forceinline__ int ld_acquire(const int32_t* p) {
     return v;
 }
 
-// Eight consecutive values k .. k + 7 (k % 8 == 0) of rank row j of an int3
-// V blob (milo_pack layout, one 64-row tile), dequantised (q - z) s to fp16
-// pairs: they are codes m0 .. m0 + 7 of one unit of super-block k / 128.
-__device__ __forceinline__ uint4 lorc3_v8(const uint8_t* blob, int j, int k) {
-    const int kin = k & 127;
-    const uint32_t* wp = reinterpret_cast<const uint32_t*>(blob + lorc_words_off(j, k >> 7, blob_unit(kin)));
-    const uint32_t w3[3] = {__ldg(wp), __ldg(wp + 1), __ldg(wp + 2)};
-    const uint32_t sz = __ldg(reinterpret_cast<const uint32_t*>(blob + lorc_sz_off(j, k >> 6)));
-    const float sc = sz_scale(sz), z = sz_zero(sz);
-    const int m0 = blob_code(kin);
-    uint32_t h[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float lo = (static_cast<float>(unit_code(w3, m0 + 2 * q)) - z) * sc;
-        const float hi = (static_cast<float>(unit_code(w3, m0 + 2 * q + 1)) - z) * sc;
-        h[q] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(lo))) |
-               (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(hi))) << 16);
-    }
-    return make_uint4(h[0], h[1], h[2], h[3]);
-}
-
 // A t-item: t[row][col] = fp16(sum_k x'[row][k] V[rank][k]) for the 16 rows
 // of one token tile of expert e, 32 ranks of one projection (8 per consumer
 // warp) and one K slice; x' is the prepared rows' plain fp16 copy (already
@@ -173,7 +157,7 @@ __device__ __forceinline__ TItem decode_titem(const GemvParams& p, int j, int nk
     t.e = find_expert(j, tstart, nks, p.n_exp);
     const ProjDev* pa = p.table + t.e * p.stride + p.proj_a;
     const ProjDev* pb = p.table + t.e * p.stride + p.proj_b;
-    const int na = rank_blocks(pa->rank), nb = GLU ? rank_blocks(pb->rank) : 0;
+    const int na = t_blocks(pa), nb = GLU ? t_blocks(pb) : 0;
     const int local = j - tstart[t.e] * nks;
     t.ks = local % nks;
     const int rest = local / nks;
@@ -191,6 +175,10 @@ __device__ __forceinline__ TItem decode_titem(const GemvParams& p, int j, int nk
 // swizzle; three of each per stage.
 constexpr int kTBoxes = 3;
 constexpr int kTStageK = 64 * kTBoxes;                    // 192
+// K slices are whole stages of both kinds of t-item (192 of K with fp16 V,
+// one 256 chunk with int3 V)
+constexpr int kTSliceAlign = 768;
+static_assert(kTSliceAlign % kTStageK == 0 && kTSliceAlign % kChunkK == 0, "t-item slices");
 constexpr int kOffTX = 0, kTXBox = kTokTile * 128;        // 2048
 constexpr int kOffTV = kTBoxes * kTXBox, kTVBox = 32 * 128;   // 6144, 4096
 static_assert(kOffTV + kTBoxes * kTVBox <= kStageBytes && kOffTV % 1024 == 0, "t-item stage");
@@ -233,54 +221,28 @@ __device__ bool titem_tma(const TItem& ti, int kb0, int kb1, const uint8_t* smem
     return true;
 }
 
-// t-item with an int3 V (no stage data): each lane loads 8 consecutive k of
-// its two rows and dequantises 8 of its V row, used as two k16 MMA steps (the
-// same relabelling of k on both operands, so the sum is unchanged).
-__device__ void titem_lorc3(const GemvParams& p, const TItem& ti, int kb0, int kb1, int row0, int ntok, int warp,
-                            int lane, float (&acc)[4]) {
-    const int g = lane >> 2, c = lane & 3;
-    const uint16_t* xr0 = g < ntok ? p.src + static_cast<size_t>(row0 + g) * p.K : nullptr;
-    const uint16_t* xr1 = g + 8 < ntok ? p.src + static_cast<size_t>(row0 + g + 8) * p.K : nullptr;
-    const int jr = ti.rb + 8 * warp + g;          // the lane's V row
-    const uint8_t* blob = reinterpret_cast<const uint8_t*>(ti.P->V);
-    if (ti.rb + 8 * warp >= ti.P->rank) return;
-    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll 4
-    for (int kb = kb0; kb < kb1; kb += 32) {
-        const int k = kb + 8 * c;
-        const uint4 xa = xr0 ? __ldg(reinterpret_cast<const uint4*>(xr0 + k)) : z4;
-        const uint4 xb = xr1 ? __ldg(reinterpret_cast<const uint4*>(xr1 + k)) : z4;
-        const uint4 v = lorc3_v8(blob, jr, k);
-        mma16816(acc, xa.x, xb.x, xa.y, xb.y, v.x, v.y);
-        mma16816(acc, xa.z, xb.z, xa.w, xb.w, v.z, v.w);
-    }
-}
-
-// End of t-item j: acc[i] is row g + 8 (i >> 1), rank 2c + (i & 1) of the
-// warp's 8 (only ranks below the projection's are stored).  One slice: t
-// directly.  Otherwise the slice's f32 partials go to tpart; the slice that
-// counts last adds the slices in order (deterministic) and writes t.  The
-// CTA that writes t then counts the rank block done for the token tile.
-template <bool GLU>
+// End of t-item j: the lane's n results v[i] of token tok[i] and rank rk[i]
+// (only those of the tile's tokens and the projection's ranks are stored).
+// One slice: t directly.  Otherwise the slice's f32 partials go to tpart;
+// the slice that counts last adds the slices in order (deterministic) and
+// writes t.  The CTA that writes t then counts the t-item done for the token
+// tile.
+template <bool GLU, int N>
 __device__ void titem_finish(const GemvParams& p, const TItem& ti, int j, int nks, int row0, int ntok,
-                             const int* ttb, const float (&acc)[4], int warp, int lane, volatile int* bcast) {
-    const int g = lane >> 2, c = lane & 3;
-    const int rk0 = ti.rb + 8 * warp, col0 = ti.col + 8 * warp, r = ti.P->rank;
+                             const int* ttb, const float (&v)[N], const int (&tok)[N], const int (&rk)[N],
+                             volatile int* bcast) {
+    const int r = ti.P->rank, col0 = ti.col - ti.rb;
     int32_t st = 0;
     if (nks == 1) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int rr = g + 8 * (i >> 1), rk = rk0 + 2 * c + (i & 1);
-            if (rr < ntok && rk < r)
-                p.t[static_cast<size_t>(row0 + rr) * p.tcols + col0 + 2 * c + (i & 1)] = t_half(acc[i], st);
-        }
+        for (int i = 0; i < N; ++i)
+            if (tok[i] < ntok && rk[i] < r)
+                p.t[static_cast<size_t>(row0 + tok[i]) * p.tcols + col0 + rk[i]] = t_half(v[i], st);
     } else {
         float* part = p.tpart + static_cast<size_t>(ti.ks) * p.R * p.tcols;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int rr = g + 8 * (i >> 1), rk = rk0 + 2 * c + (i & 1);
-            if (rr < ntok && rk < r) part[static_cast<size_t>(row0 + rr) * p.tcols + col0 + 2 * c + (i & 1)] = acc[i];
-        }
+        for (int i = 0; i < N; ++i)
+            if (tok[i] < ntok && rk[i] < r) part[static_cast<size_t>(row0 + tok[i]) * p.tcols + col0 + rk[i]] = v[i];
         // the CTA's partials, then one thread's acquire-release count: the last
         // slice to count sees every other slice's partials
         consumer_sync();
@@ -290,15 +252,13 @@ __device__ void titem_finish(const GemvParams& p, const TItem& ti, int j, int nk
         if (last) {
             const size_t slice = static_cast<size_t>(p.R) * p.tcols;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int rr = g + 8 * (i >> 1), rk = rk0 + 2 * c + (i & 1);
-                if (rr < ntok && rk < r) {
-                    const size_t o = static_cast<size_t>(row0 + rr) * p.tcols + col0 + 2 * c + (i & 1);
-                    float v = 0.0f;
-                    for (int s2 = 0; s2 < nks; ++s2) v += __ldcg(p.tpart + s2 * slice + o);
-                    p.t[o] = t_half(v, st);
+            for (int i = 0; i < N; ++i)
+                if (tok[i] < ntok && rk[i] < r) {
+                    const size_t o = static_cast<size_t>(row0 + tok[i]) * p.tcols + col0 + rk[i];
+                    float a = 0.0f;
+                    for (int s2 = 0; s2 < nks; ++s2) a += __ldcg(p.tpart + s2 * slice + o);
+                    p.t[o] = t_half(a, st);
                 }
-            }
         }
         consumer_sync();          // every warp has read bcast before it is reused
         if (!last) {
@@ -313,7 +273,7 @@ __device__ void titem_finish(const GemvParams& p, const TItem& ti, int j, int nk
 
 // One k16 step of the code part: extract the A fragments of both row tiles
 // and multiply them with the prepared activation fragments of NT n8 tiles.
-template <int S, int NT>
+template <int S, int NT, int NTI>
 __device__ __forceinline__ void code_step(const uint32_t (&wd)[2][2][3], const uint32_t (&hw)[2][2][3],
                                           const uint8_t* xs, int g, int c, float (&dz)[2][2][4]) {
     constexpr int t0 = sched_word(S, 0), f0 = sched_field(S, 0);
@@ -324,7 +284,7 @@ __device__ __forceinline__ void code_step(const uint32_t (&wd)[2][2][3], const u
     for (int n8 = 0; n8 < NT; ++n8)
         b[n8] = *reinterpret_cast<const uint2*>(xs + ((n8 * 8 + g) * kFragRowHalves + S * 16 + c * 4) * 2);
 #pragma unroll
-    for (int ti = 0; ti < 2; ++ti) {
+    for (int ti = 0; ti < NTI; ++ti) {
         const uint32_t a0 = unit_reg<t0, f0>(wd[ti][0], hw[ti][0]);
         const uint32_t a1 = unit_reg<t0, f0>(wd[ti][1], hw[ti][1]);
         const uint32_t a2 = unit_reg<t1, f1>(wd[ti][0], hw[ti][0]);
@@ -360,12 +320,12 @@ struct TileMap {
 // super-block grp / 2's scales follow its codes, as (s, z) pairs of rows j and
 // j + 8 of each 16-row block, so one 64-bit load brings the lane's two rows.
 // xg[n8][j]: X_g of its tokens.
-template <int NT>
+template <int NT, int NTI>
 __device__ __forceinline__ void fold_group(float (&acc)[2][2][4], const float (&dz)[2][2][4],
                                            const uint8_t* st, int grp, const int (&reg)[2],
                                            const int (&rbase)[2], int g, const float (&xg)[NT][2]) {
 #pragma unroll
-    for (int ti = 0; ti < 2; ++ti) {
+    for (int ti = 0; ti < NTI; ++ti) {
         const uint2 q = *reinterpret_cast<const uint2*>(st + reg[ti] + (grp >> 1) * kBlockSB + kQTileSBWords * 4 +
                                                         (grp & 1) * kGroupBytes + ((rbase[ti] >> 4) * 8 + g) * 8);
         float s24[2], nsz[2];
@@ -388,7 +348,9 @@ __device__ __forceinline__ void fold_group(float (&acc)[2][2][4], const float (&
     }
 }
 
-template <bool GLU, int NT>
+// One stage's K chunk (nsb super-blocks) on the warp's NTI m16 row tiles
+// (NTI = 1: only tile 0, for the int3 compensator's t-items).
+template <bool GLU, int NT, int NTI = 2>
 __device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2][2][4], const TileMap<GLU>& tm,
                                               int nsb, int lane) {
     const int g = lane >> 2, c = lane & 3;
@@ -397,7 +359,7 @@ __device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2]
         if (sbl == nsb) break;
         uint32_t wd[2][2][3], hw[2][2][3];
 #pragma unroll
-        for (int ti = 0; ti < 2; ++ti) {
+        for (int ti = 0; ti < NTI; ++ti) {
             const uint32_t* qt = reinterpret_cast<const uint32_t*>(st + tm.reg[ti] + sbl * kBlockSB);
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr)
@@ -421,16 +383,16 @@ __device__ __forceinline__ void chunk_compute(const uint8_t* st, float (&acc)[2]
                 xb[n8][j] = v.y;
             }
         float dz[2][2][4];
-        code_step<0, NT>(wd, hw, xs, g, c, dz);
-        code_step<1, NT>(wd, hw, xs, g, c, dz);
-        code_step<2, NT>(wd, hw, xs, g, c, dz);
-        code_step<3, NT>(wd, hw, xs, g, c, dz);
-        fold_group<NT>(acc, dz, st, 2 * sbl, tm.reg, tm.r, g, xa);
-        code_step<4, NT>(wd, hw, xs, g, c, dz);
-        code_step<5, NT>(wd, hw, xs, g, c, dz);
-        code_step<6, NT>(wd, hw, xs, g, c, dz);
-        code_step<7, NT>(wd, hw, xs, g, c, dz);
-        fold_group<NT>(acc, dz, st, 2 * sbl + 1, tm.reg, tm.r, g, xb);
+        code_step<0, NT, NTI>(wd, hw, xs, g, c, dz);
+        code_step<1, NT, NTI>(wd, hw, xs, g, c, dz);
+        code_step<2, NT, NTI>(wd, hw, xs, g, c, dz);
+        code_step<3, NT, NTI>(wd, hw, xs, g, c, dz);
+        fold_group<NT, NTI>(acc, dz, st, 2 * sbl, tm.reg, tm.r, g, xa);
+        code_step<4, NT, NTI>(wd, hw, xs, g, c, dz);
+        code_step<5, NT, NTI>(wd, hw, xs, g, c, dz);
+        code_step<6, NT, NTI>(wd, hw, xs, g, c, dz);
+        code_step<7, NT, NTI>(wd, hw, xs, g, c, dz);
+        fold_group<NT, NTI>(acc, dz, st, 2 * sbl + 1, tm.reg, tm.r, g, xb);
     }
 }
 
@@ -539,8 +501,8 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         ttb[e] = tte;
         int nt = 0;
         if (p.t_items && tte > 0) {
-            const int na = rank_blocks(p.table[e * p.stride + p.proj_a].rank);
-            const int nb = GLU ? rank_blocks(p.table[e * p.stride + p.proj_b].rank) : 0;
+            const int na = t_blocks(p.table + e * p.stride + p.proj_a);
+            const int nb = GLU ? t_blocks(p.table + e * p.stride + p.proj_b) : 0;
             nt = tte * (na + nb);
         }
         tstart[e] = nt;
@@ -579,7 +541,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     int nks = 1, kslice = p.K;
     if (p.t_items && tstart[p.n_exp] > 0) {
         nks = max(1, min(p.nks, static_cast<int>(gridDim.x) / tstart[p.n_exp]));
-        kslice = (((p.K + nks - 1) / nks) + kTStageK - 1) / kTStageK * kTStageK;
+        kslice = (((p.K + nks - 1) / nks) + kTSliceAlign - 1) / kTSliceAlign * kTSliceAlign;
         nks = (p.K + kslice - 1) / kslice;
     }
     const int n_t = tstart[p.n_exp] * nks;
@@ -611,7 +573,10 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 const int kb0 = ti.ks * kslice, kb1 = min(p.K, kb0 + kslice);
                 const int trow0 = row0s[ti.e] + kTokTile * ti.tt;
                 const bool l3 = ti.P->lorc3 != 0;
-                for (int kc = kb0; kc < kb1; kc += kTStageK) {
+                // stages of 192 of K (fp16 V) or of one K chunk (int3 V)
+                const int kstep = l3 ? kChunkK : kTStageK;
+                const int tntok = min(kTokTile, cnt[ti.e] - kTokTile * ti.tt);
+                for (int kc = kb0; kc < kb1; kc += kstep) {
                     if (!warp_wait(&empty[stage], phase ^ 1)) {
                         fail = true;
                         break;
@@ -620,12 +585,21 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                     uint64_t* fb = &full[stage];
                     filled |= 1u << stage;
                     fph = (fph & ~(1u << stage)) | (phase << stage);
-                    const int nbox = min(kTBoxes, (kb1 - kc) / 64);
                     if (elect_one()) {
                         if (kc == kb0) stage_item[stage] = -2 - tj;
                         if (l3) {
-                            mbar_arrive(fb);
+                            // the V blob's K chunk (its one 64-row tile) and the
+                            // rows' prepared activations, as for a GEMM item
+                            const int ch = kc / kChunkK;
+                            const uint32_t vb = min(2, p.SB - 2 * ch) * kBlockSB;
+                            const uint32_t xb = tntok * kFragRowHalves * 2;
+                            mbar_arrive_expect_tx(fb, vb + xb);
+                            bulk_load_hint(st + kOffQ, reinterpret_cast<const uint8_t*>(ti.P->V) + 2 * ch * kBlockSB,
+                                           vb, fb, pol);
+                            bulk_load(st + kOffX, p.x + (static_cast<size_t>(ch) * p.R + trow0) * kFragRowHalves, xb,
+                                      fb);
                         } else {
+                            const int nbox = min(kTBoxes, (kb1 - kc) / 64);
                             mbar_arrive_expect_tx(fb, nbox * (kTXBox + kTVBox));
                             for (int q = 0; q < nbox; ++q) {
                                 tma_load_2d(st + kOffTX + q * kTXBox, &p.smap, fb, kc + 64 * q, trow0);
@@ -635,7 +609,6 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                     }
                     __syncwarp();
                     if (++stage == kStages) { stage = 0; phase ^= 1; }
-                    if (l3) break;
                 }
                 if (fail) break;
                 tj += S;
@@ -692,7 +665,8 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 if (p.t_items) {
                     // this token tile's t comes from t-items of this launch:
                     // wait (bounded) until all its rank blocks are done
-                    const int need = rank_blocks(ra) + (GLU ? rank_blocks(rb) : 0);
+                    const int need = (ra == 0 ? 0 : l3a ? 1 : rank_blocks(ra)) +
+                                     (GLU && rb > 0 ? (l3b ? 1 : rank_blocks(rb)) : 0);
                     const int32_t* done = p.tdone + ttb[w.e] + w.tt;
                     if (ld_acquire(done) < need) {
                         const long long t0 = clock64();
@@ -793,17 +767,53 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             const int kb0 = ti.ks * kslice, kb1 = min(p.K, kb0 + kslice);
             const int trow0 = row0s[ti.e] + kTokTile * ti.tt;
             const int tntok = min(kTokTile, cnt[ti.e] - kTokTile * ti.tt);
-            float tacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            if (ti.P->lorc3) {   // its one stage carries no data
-                titem_lorc3(p, ti, kb0, kb1, trow0, tntok, warp, lane, tacc);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[stage]);
-                if (++stage == kStages) { stage = 0; phase ^= 1; }
-            } else if (!titem_tma(ti, kb0, kb1, smem, full, empty, stage, phase, warp, lane, tacc)) {
-                flag(p.dev_status, MILO_DEV_TIMEOUT);
-                return;
+            if (ti.P->lorc3) {
+                // int3 V: the GEMM's own decode of the V blob (rows = ranks)
+                // against the rows' prepared activations; acc[0][n8][i] is
+                // rank 16 warp + g + 8 (i >> 1) of token 8 n8 + 2c + (i & 1),
+                // already times the row's 2^a
+                float acc[2][2][4] = {};
+                const TileMap<true> tmv(warp);
+                const bool active = 16 * warp < ti.P->rank;
+                for (int kc = kb0; kc < kb1; kc += kChunkK) {
+                    if (kc != kb0 && !warp_wait(&full[stage], phase)) {
+                        flag(p.dev_status, MILO_DEV_TIMEOUT);
+                        return;
+                    }
+                    const int nsb = min(2, p.SB - 2 * (kc / kChunkK));
+                    if (active) {
+                        if (tntok > 8) chunk_compute<true, 2, 1>(smem + stage * kStageBytes, acc, tmv, nsb, lane);
+                        else chunk_compute<true, 1, 1>(smem + stage * kStageBytes, acc, tmv, nsb, lane);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[stage]);
+                    if (++stage == kStages) { stage = 0; phase ^= 1; }
+                }
+                float v[8];
+                int tok[8], rk[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int n8 = q >> 2, i = q & 3;
+                    v[q] = acc[0][n8][i];
+                    tok[q] = 8 * n8 + 2 * c + (i & 1);
+                    rk[q] = 16 * warp + g + 8 * (i >> 1);
+                }
+                titem_finish<GLU, 8>(p, ti, j, nks, trow0, tntok, ttb, v, tok, rk, bcast);
+            } else {
+                float tacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                if (!titem_tma(ti, kb0, kb1, smem, full, empty, stage, phase, warp, lane, tacc)) {
+                    flag(p.dev_status, MILO_DEV_TIMEOUT);
+                    return;
+                }
+                // tacc[i]: token g + 8 (i >> 1), rank 8 warp + 2c + (i & 1) of the block
+                int tok[4], rk[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    tok[i] = g + 8 * (i >> 1);
+                    rk[i] = ti.rb + 8 * warp + 2 * c + (i & 1);
+                }
+                titem_finish<GLU, 4>(p, ti, j, nks, trow0, tntok, ttb, tacc, tok, rk, bcast);
             }
-            titem_finish<GLU>(p, ti, j, nks, trow0, tntok, ttb, tacc, warp, lane, bcast);
             continue;
         }
         bool waited = true;       // the next stage's barrier has been passed already

@@ -415,6 +415,17 @@ def test_linear_int3_compensator_many_rows(milo, gemm_path):
     _linear_check(milo, projs, x, "bf16", ids, 1, (torch.float32, torch.float16), lorc_int3=True)
 
 
+@pytest.mark.parametrize("lorc_int3", [False, True])
+def test_linear_compensator_long_k(milo, gemm_path, lorc_int3):
+    """K = 4224 (33 super-blocks): the compensator's down-projection runs in
+    several K slices, the last one ragged (a half chunk, a partial stage);
+    ranks 8, 40 (a partial 32-rank block) and 64; 5 rows over 3 experts."""
+    projs = [wl.make_projection("t_longk", "w", e, 256, 4224, r) for e, r in enumerate((8, 40, 64))]
+    x = wl.gen_activations(np.random.default_rng(34), 5, 4224, "bf16")
+    ids = np.array([[2], [0], [1], [2], [2]], np.int32)
+    _linear_check(milo, projs, x, "bf16", ids, 1, lorc_int3=lorc_int3)
+
+
 def test_moe_int3_compensator(milo, gemm_path):
     wk = wl.small_moe("t_moe_l3", T=24, hidden=256, inter=384, n_routed=4, n_shared=1, top_k=2,
                       rank_choices=(0, 16, 32))
