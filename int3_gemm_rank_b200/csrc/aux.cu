@@ -250,6 +250,7 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
             float* gs = reinterpret_cast<float*>(p.frag + crow * kFragRowHalves + kGsumHalf);
             gs[2 * (sb & 1)] = s0;
             gs[2 * (sb & 1) + 1] = s1;
+            if (!(sb & 1)) gs[kInvSlot] = inv_pow2(scale);   // the GEMM epilogue's 2^-a
         }
         // per super-block: step-major, lane-in-quad c, 4 fp16 each
         uint2* out = reinterpret_cast<uint2*>(p.frag + crow * kFragRowHalves + (sb & 1) * kFragHalvesPerSB) + c;

@@ -68,9 +68,11 @@ constexpr int kStageBytes = 23552;
 constexpr int kOffUA = 0, kOffUB = 8192, kOffT = 16384;   // compensator stage
 constexpr int kBarOffset = kStages * kStageBytes;
 // barriers, then the item tables cnt, row0s, ttb, tstart [MILO_MAX_EXPERTS + 1],
-// the stage headers and the consumers' broadcast word; 1 KB of slack to align
-// the base
-constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 4 * (MILO_MAX_EXPERTS + 1) * 4 + kStages * 4 + 16 + 1024;
+// the stage headers (kHdrInts each) and the consumers' broadcast word; 1 KB
+// of slack to align the base
+constexpr int kHdrInts = 8;
+constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 4 * (MILO_MAX_EXPERTS + 1) * 4 + kStages * kHdrInts * 4 + 16 +
+                           1024;
 
 static_assert(kOffX + kTokTile * kFragRowHalves * 2 <= kStageBytes, "GEMM stage");
 static_assert(kStageBytes % 1024 == 0, "stage alignment");
@@ -463,6 +465,16 @@ __device__ __forceinline__ void lorc_compute(const uint8_t* st, float (&acc)[2][
     }
 }
 
+// A GEMM item's stage header: its index, what the producer decoded for it,
+// and its projections' ranks and compensator formats (info).
+__device__ __forceinline__ void write_hdr(volatile int* h, int it, const Item& w, int info) {
+    h[1] = w.e;
+    h[2] = w.ntile;
+    h[3] = w.tt | (w.split << 16);
+    h[4] = info;
+    h[0] = it;
+}
+
 template <bool GLU>
 __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_constant__ GemvParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -474,9 +486,11 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     int* ttb = row0s + (MILO_MAX_EXPERTS + 1);       // prefix of the experts' token tiles
     int* tstart = ttb + (MILO_MAX_EXPERTS + 1);      // prefix of the experts' t-items
     // header of each stage: the work item whose first stage it is (-1: no more
-    // items, -2 - j: t-item j, a stage with no data)
-    volatile int* stage_item = tstart + (MILO_MAX_EXPERTS + 1);
-    volatile int* bcast = stage_item + kStages;      // consumers' broadcast word
+    // items, -2 - j: t-item j), then for a GEMM item what the producer decoded
+    // for it (expert, weight tile, token tile and K split, the ranks and
+    // compensator formats), so that the consumers need no global loads for it
+    volatile int* hdr = tstart + (MILO_MAX_EXPERTS + 1);
+    volatile int* bcast = hdr + kStages * kHdrInts;   // consumers' broadcast word
 
     constexpr int RA = GLU ? kRowsGlu : kRowsPlain;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -586,7 +600,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                     filled |= 1u << stage;
                     fph = (fph & ~(1u << stage)) | (phase << stage);
                     if (elect_one()) {
-                        if (kc == kb0) stage_item[stage] = -2 - tj;
+                        if (kc == kb0) hdr[stage * kHdrInts] = -2 - tj;
                         if (l3) {
                             // the V blob's K chunk (its one 64-row tile) and the
                             // rows' prepared activations, as for a GEMM item
@@ -631,6 +645,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             // the compensator stage's fields, loaded with the item's first ones
             const int ra = pa->rank, rb = GLU ? pb->rank : 0;
             const bool l3a = pa->lorc3 != 0, l3b = GLU ? pb->lorc3 != 0 : false;
+            const int hinfo = ra | (rb << 8) | (l3a ? 1 << 16 : 0) | (l3b ? 1 << 17 : 0);
             const uint16_t* Ua = pa->U;
             const uint16_t* Ub = pb->U;
             for (int ch = c0; ch < c1; ++ch) {
@@ -650,7 +665,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                                         : w0 + static_cast<size_t>(p.SB) * kBlockSB;
                 const uint16_t* xsrc = p.x + (static_cast<size_t>(ch) * p.R + row0) * kFragRowHalves;
                 if (elect_one()) {
-                    if (!header) stage_item[stage] = it;
+                    if (!header) write_hdr(hdr + stage * kHdrInts, it, w, hinfo);
                     mbar_arrive_expect_tx(fb, ntl * wb + xb);
                     bulk_load_hint(st + kOffQ, w0, wb, fb, pol);
                     if (ntl == 2) bulk_load_hint(st + kOffQ + kTileBlk, w1, wb, fb, pol);
@@ -701,7 +716,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                                                       : reinterpret_cast<const uint8_t*>(Ub + static_cast<size_t>(n0) * rb);
                 const uint32_t tb = ntok * p.tcols * 2;
                 if (elect_one()) {
-                    if (!header) stage_item[stage] = it;
+                    if (!header) write_hdr(hdr + stage * kHdrInts, it, w, hinfo);
                     mbar_arrive_expect_tx(fb, ua + ub + tb);
                     if (ua) bulk_load_hint(st + kOffUA, usa, ua, fb, pol);
                     if (ub) bulk_load_hint(st + kOffUB, usb, ub, fb, pol);
@@ -719,7 +734,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 filled |= 1u << stage;
                 fph = (fph & ~(1u << stage)) | (phase << stage);
                 if (elect_one()) {
-                    stage_item[stage] = it;
+                    write_hdr(hdr + stage * kHdrInts, it, w, hinfo);
                     mbar_arrive(&full[stage]);
                 }
                 __syncwarp();
@@ -733,7 +748,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 filled |= 1u << stage;
                 fph = (fph & ~(1u << stage)) | (phase << stage);
                 if (elect_one()) {
-                    stage_item[stage] = -1;
+                    hdr[stage * kHdrInts] = -1;
                     mbar_arrive(&full[stage]);
                 }
                 __syncwarp();
@@ -759,7 +774,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             flag(p.dev_status, MILO_DEV_TIMEOUT);
             return;
         }
-        const int it = stage_item[stage];
+        const int it = hdr[stage * kHdrInts];
         if (it == -1) break;
         if (it < -1) {           // a t-item
             const int j = -2 - it;
@@ -817,27 +832,29 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             continue;
         }
         bool waited = true;       // the next stage's barrier has been passed already
-        const Item w = decode_item(it, ttb, cnt, p.n_exp, n_tiles, p.splits);
-        const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
-        const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
+        Item w;
+        int ra, rb;
+        bool u3a, u3b;
+        {
+            const volatile int* h = hdr + stage * kHdrInts;
+            w.e = h[1];
+            w.ntile = h[2];
+            w.tt = h[3] & 0xFFFF;
+            w.split = h[3] >> 16;
+            const int info = h[4];
+            ra = info & 255;
+            rb = (info >> 8) & 255;
+            u3a = (info >> 16) & 1;
+            u3b = GLU ? (info >> 17) & 1 : u3a;
+        }
         const int n0 = w.ntile * RA;
         const int row0 = row0s[w.e] + w.tt * kTokTile;
         const int ntok = min(kTokTile, cnt[w.e] - w.tt * kTokTile);
         const int c0 = w.split * p.cps;
         const int c1 = min(p.chunks, c0 + p.cps);
-        // what the item's end needs from global memory, loaded now so that the
-        // loads overlap the K loop (the barrier waits keep the compiler from
-        // moving them): the projections' ranks and formats, the rows' scales
-        const int ra = pa->rank, rb = GLU ? pb->rank : 0;
-        const bool u3a = pa->lorc3 != 0, u3b = GLU ? pb->lorc3 != 0 : u3a;
-        float inv[2][2];
-#pragma unroll
-        for (int n8 = 0; n8 < 2; ++n8)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int tok = n8 * 8 + 2 * c + j;
-                inv[n8][j] = tok < ntok ? inv_pow2(p.rscale[row0 + tok]) : 0.0f;
-            }
+        // the lane's tokens n8 * 8 + 2c + j: 2^-a undoes their rows' scale
+        // 2^a; it sits in every activation row's padding (the first stage)
+        float inv[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
         float acc[2][2][4];
 #pragma unroll
         for (int a = 0; a < 2; ++a)
@@ -854,6 +871,17 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             waited = false;
             const uint8_t* st = smem + stage * kStageBytes;
             const int nsb = min(2, p.SB - 2 * ch);
+            if (ch == c0) {
+#pragma unroll
+                for (int n8 = 0; n8 < 2; ++n8)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int tok = n8 * 8 + 2 * c + j;
+                        inv[n8][j] = tok < ntok ? reinterpret_cast<const float*>(
+                                                      st + kOffX + (tok * kFragRowHalves + kGsumHalf) * 2)[kInvSlot]
+                                                : 0.0f;
+                    }
+            }
             if (ntok > 8) chunk_compute<GLU, 2>(st, acc, tm, nsb, lane);
             else chunk_compute<GLU, 1>(st, acc, tm, nsb, lane);
             __syncwarp();
@@ -881,7 +909,6 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         }
 
         // ------------------------------------------------------------ epilogue
-        // the lane's tokens n8 * 8 + 2c + j: inv undoes their rows' scale 2^a
         if constexpr (GLU) {
             int32_t st = 0;
 #pragma unroll

@@ -34,6 +34,9 @@ constexpr float kFoldScale = 262144.0f;   // 2^18: undoes the 2^-18 of the code 
 constexpr int kFragHalvesPerSB = 128;
 constexpr int kFragRowHalves = 2 * kFragHalvesPerSB + 16;
 constexpr int kGsumHalf = 2 * kFragHalvesPerSB;
+// Row padding of a chunk (f32 slots from kGsumHalf): the chunk's four group
+// sums, then the row's 2^-a.
+constexpr int kInvSlot = 4;
 
 // Packed weights (milo.h): rows in tiles of 64; each (tile, super-block)
 // block -- the codes, then the two groups' scales and zeros -- is contiguous,
@@ -67,7 +70,7 @@ struct CombineParams {
 struct GemvParams {
     CUtensorMap smap;           // the rows' plain fp16 copy `src` [R][K]: box {64, 16}, 128-byte swizzle
     const uint16_t* x;          // prepared activations [chunks][R][kFragRowHalves] fp16
-                                // (group sums in each row's padding, see kGsumHalf)
+                                // (group sums and 2^-a in each row's padding, see kGsumHalf)
     const float* rscale;        // [R]: the row's activation scale 2^a (see kFoldScale)
     uint16_t* t;                // LoRC down-projection [R][tcols] fp16 (times the row's 2^a)
     const ProjDev* table;       // device table
