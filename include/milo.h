@@ -62,6 +62,10 @@ typedef enum {
 #define MILO_DEV_NONFINITE 0x2      /* NaN/Inf in weights, logits or activations */
 #define MILO_DEV_FP16_RANGE 0x4     /* a value does not fit fp16 (s, z, h, an fp16 output) */
 #define MILO_DEV_TIMEOUT 0x8        /* a bounded pipeline wait gave up; outputs invalid */
+/* Checked build only (libmilo_checked.so, compiled with MILO_CHECKED): an
+ * index or copy range fell outside its buffer; that access was skipped and
+ * the outputs are invalid.  The normal build performs no such checks. */
+#define MILO_DEV_BOUNDS 0x10
 
 /* Router flags. */
 #define MILO_ROUTE_RENORM 0x1u      /* renormalise the softmax over the k picked experts */

@@ -18,12 +18,16 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmilo.so")
+# MILO_LIBRARY=checked loads the checked build (range checks in every kernel,
+# MILO_DEV_BOUNDS on a violation), built by `python -m int3_gemm_rank_b200.build
+# --checked`.
+LIB_PATH = os.path.join(_HERE, "libmilo_checked.so" if os.environ.get("MILO_LIBRARY") == "checked"
+                        else "libmilo.so")
 
 MILO_F16, MILO_BF16, MILO_F32 = 0, 1, 2
 MILO_OK, MILO_ERR_INVALID_ARG, MILO_ERR_UNSUPPORTED_SHAPE, MILO_ERR_WORKSPACE, MILO_ERR_CUDA = range(5)
 MILO_LORC_F16, MILO_LORC_INT3 = 0, 1
-MILO_DEV_BAD_EXPERT_ID, MILO_DEV_NONFINITE, MILO_DEV_FP16_RANGE, MILO_DEV_TIMEOUT = 1, 2, 4, 8
+MILO_DEV_BAD_EXPERT_ID, MILO_DEV_NONFINITE, MILO_DEV_FP16_RANGE, MILO_DEV_TIMEOUT, MILO_DEV_BOUNDS = 1, 2, 4, 8, 16
 MILO_ROUTE_RENORM, MILO_ROUTE_IDS_GIVEN = 1, 2
 MILO_GEMM_AUTO, MILO_GEMM_MMA, MILO_GEMM_TC = 0, 1, 2
 MILO_GROUP, MILO_MAX_RANK = 64, 64
@@ -79,7 +83,8 @@ def lib() -> C.CDLL:
     if _lib is None:
         if not os.path.exists(LIB_PATH):
             raise RuntimeError(f"{LIB_PATH} is missing: build it with "
-                               "`python -m int3_gemm_rank_b200.build` (nvcc, sm_100a)")
+                               "`python -m int3_gemm_rank_b200.build` (nvcc, sm_100a; --checked "
+                               "for the checked build)")
         L = C.CDLL(LIB_PATH)
         vp, i32, u32, sz = C.c_void_p, C.c_int32, C.c_uint32, C.c_size_t
         L.milo_status_str.argtypes = [C.c_int]; L.milo_status_str.restype = C.c_char_p

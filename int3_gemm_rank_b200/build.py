@@ -1,11 +1,17 @@
 """Build libmilo.so (the sm_100a kernels and the C ABI of include/milo.h) in-tree.
 
-    python -m int3_gemm_rank_b200.build [--force]
+    python -m int3_gemm_rank_b200.build [--force] [--checked]
 
 Each .cu file is compiled with nvcc for sm_100a only (-gencode
 arch=compute_100a,code=sm_100a), with -lineinfo for the profilers, and linked
 into int3_gemm_rank_b200/libmilo.so next to this file.  The CUDA runtime is
 linked statically, so the library only needs the driver at run time.
+
+--checked builds libmilo_checked.so instead: the same sources with
+MILO_CHECKED defined, so that the kernels check their indices and copy ranges
+against their buffers and flag MILO_DEV_BOUNDS instead of making an access out
+of range (the stand-in for a memory checker).  MILO_LIBRARY=checked makes the
+Python binding load it.
 """
 from __future__ import annotations
 
@@ -19,6 +25,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmilo.so")
+LIB_CHECKED = os.path.join(HERE, "libmilo_checked.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
@@ -36,21 +43,24 @@ def _deps():
                   [os.path.join(HERE, "..", "include", "milo.h"), os.path.abspath(__file__)])
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB
+    if not force and up_to_date(lib):
+        return lib
+    bdir = BUILD + ("_checked" if checked else "")
+    os.makedirs(bdir, exist_ok=True)
+    extra = ["-DMILO_CHECKED"] if checked else []
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-        cmd = [NVCC, *FLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
+        cmd = [NVCC, *FLAGS, *extra, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
@@ -60,14 +70,14 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     with ThreadPoolExecutor(max(1, min(8, os.cpu_count() or 1))) as ex:
         objs = list(ex.map(compile_one, _sources()))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     r = subprocess.run([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs,
                         "-o", tmp, "-Xcompiler", "-fvisibility=hidden"], capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, checked="--checked" in sys.argv))

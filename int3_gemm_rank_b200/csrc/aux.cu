@@ -155,6 +155,8 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     } else {
         src = p.row_src ? p.row_src[row] : row;
     }
+    // the source has T rows (tokens) when rows come from the router, else R
+    if (src >= 0 && !in_range(p.dev_status, src < (p.rows || p.row_src ? p.T : p.R))) src = -1;
     // the row's scale 2^a: every block of the row reads the whole row (the
     // blocks of one row are few, and only while rows are few)
     const float scale = row_scale_for(row_max_bits(p, src));
@@ -315,6 +317,11 @@ __global__ void __launch_bounds__(128) lorc_partial_kernel(const LorcParams p) {
     const int row0 = p.grp[2 * e], m = p.grp[2 * e + 1];
     if (m <= 0 || row0 < 0 || row0 + m > p.R) return;
     const int col0 = which == 0 ? 0 : p.t_col_b;
+    // t's columns, and (K split) the slice counter of this tile
+    if (!in_range(p.dev_status, col0 + span <= p.tcols &&
+                                    (p.splits == 1 || ((e * nproj + which) * kLorcRankBlocks + rblk) * p.row_groups +
+                                                              static_cast<int>(blockIdx.y) < kLorcCounters)))
+        return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
     // K slice of this block: whole super-blocks, the last slice may be shorter
     const int slice_sb = (p.K / 128 + p.splits - 1) / p.splits;
@@ -471,6 +478,7 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
     const int col0 = which == 0 ? 0 : p.t_col_b;
     const int row0 = p.grp[2 * e], m = p.grp[2 * e + 1];
     if (m <= 0 || row0 < 0 || row0 + m > p.R) return;
+    if (!in_range(p.dev_status, col0 + span <= p.tcols)) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
     const int nr8 = (r + 7) / 8;                      // n8 rank tiles that hold ranks < r
     int32_t st = 0;

@@ -299,12 +299,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     const uint8_t* w1 = GLU ? pb->packed + (static_cast<size_t>(tile0) * p.SB + b) * kBlockSB
                                             : w0 + static_cast<size_t>(p.SB) * kBlockSB;
                     if (elect_one()) {
-                        mbar_arrive_expect_tx(fb, kTcStageTx + ntl * kBlockSB + (zs ? kTcZTile : 0));
-                        tma_load_2d(st + kTcOffB, &p.b_map, fb, 128 * b, row0);
-                        tma_load_2d(st + kTcOffB + kTcAtom, &p.b_map, fb, 128 * b + 64, row0);
-                        bulk_load(st + kTcOffW, w0, kBlockSB, fb);
-                        if (ntl == 2) bulk_load(st + kTcOffW + kBlockSB, w1, kBlockSB, fb);
-                        if (zs) tma_load_2d(st + kTcOffZB, &p.z_map, fb, 16 * (b >> 1), row0);
+                        // each blob's ceil(N / 64) tiles of SB blocks (SwiGLU: tile
+                        // tile0 of w1's and of w3's), the routed rows
+                        if (in_range(p.dev_status, tile0 + (GLU ? 1 : ntl) <= (p.N + kTileRows - 1) / kTileRows &&
+                                                       row0 >= 0 &&
+                                                       row0 < p.R)) {
+                            mbar_arrive_expect_tx(fb, kTcStageTx + ntl * kBlockSB + (zs ? kTcZTile : 0));
+                            tma_load_2d(st + kTcOffB, &p.b_map, fb, 128 * b, row0);
+                            tma_load_2d(st + kTcOffB + kTcAtom, &p.b_map, fb, 128 * b + 64, row0);
+                            bulk_load(st + kTcOffW, w0, kBlockSB, fb);
+                            if (ntl == 2) bulk_load(st + kTcOffW + kBlockSB, w1, kBlockSB, fb);
+                            if (zs) tma_load_2d(st + kTcOffZB, &p.z_map, fb, 16 * (b >> 1), row0);
+                        } else {
+                            mbar_arrive(fb);
+                        }
                     }
                     __syncwarp();
                     if (++stage == kTcStages) { stage = 0; phase ^= 1; }
@@ -331,11 +339,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                                          : pb->lorc3 ? reinterpret_cast<const uint8_t*>(pb->U) + (n0 >> 7) * kBlockSB
                                                      : reinterpret_cast<const uint8_t*>(pb->U + static_cast<size_t>(n0) * rb);
                     if (elect_one()) {
-                        mbar_arrive_expect_tx(fb, nbox * kTcAtom + ua + ub);
-                        for (int j = 0; j < nbox; ++j)
-                            tma_load_2d(st + kTcOffB + j * kTcAtom, &p.t_map, fb, 64 * j, row0);
-                        if (ua) bulk_load(st + kTcOffUA, usa, ua, fb);
-                        if (ub) bulk_load(st + kTcOffUB, usb, ub, fb);
+                        // U rows n0 .. n0 + urows or the int3 U^T block of
+                        // super-block n0 / 128, and the stage's room for them
+                        if (in_range(p.dev_status, n0 + urows <= p.N && nbox <= 2 && row0 >= 0 && row0 < p.R &&
+                                                       ua <= (GLU ? kTcOffUB : kTcStage) - kTcOffUA && kTcOffUB + ub <= kTcStage &&
+                                                       (!(ra && pa->lorc3) || (n0 >> 7) < p.N / 128) &&
+                                                       (!(rb && pb->lorc3) || (n0 >> 7) < p.N / 128))) {
+                            mbar_arrive_expect_tx(fb, nbox * kTcAtom + ua + ub);
+                            for (int j = 0; j < nbox; ++j)
+                                tma_load_2d(st + kTcOffB + j * kTcAtom, &p.t_map, fb, 64 * j, row0);
+                            if (ua) bulk_load(st + kTcOffUA, usa, ua, fb);
+                            if (ub) bulk_load(st + kTcOffUB, usb, ub, fb);
+                        } else {
+                            mbar_arrive(fb);
+                        }
                     }
                     __syncwarp();
                     if (++stage == kTcStages) { stage = 0; phase ^= 1; }
@@ -701,7 +718,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     const int t = kTcHalf * th + 32 * u + lane;
-                    sc[u] = t < ntok ? inv_pow2(p.rscale[row0 + t]) : 0.0f;
+                    sc[u] = t < ntok && in_range(p.dev_status, row0 + t < p.R) ? inv_pow2(p.rscale[row0 + t]) : 0.0f;
                 }
 #pragma unroll
                 for (int i = 0; i < kTcHalf / 2; ++i) {
@@ -754,7 +771,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         const float av = is_w1 ? own : other;
                         const float bv = is_w1 ? other : own;
                         const int t = kTcHalf * th + tl;
-                        if (t < ntok && f < p.N) {
+                        if (t < ntok && f < p.N && in_range(p.dev_status, row0 + t < p.R)) {
                             const float hv = __fdividef(av, 1.0f + __expf(-av)) * bv;
                             const __half hh = __float2half_rn(hv);
                             if (!isfinite(hv)) st_bits |= MILO_DEV_NONFINITE;
@@ -774,7 +791,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 #pragma unroll
                     for (int i = 0; i < kTcHalf; ++i) {
                         const int t = kTcHalf * th + i;
-                        if (t < ntok)
+                        if (t < ntok && in_range(p.dev_status, row0 + t < p.R))
                             // streaming stores: the output is read once, by the
                             // combine, and must not push the routed rows out of L2
                             __stcs(p.y_part + static_cast<size_t>(row0 + t) * p.N + n,

@@ -234,28 +234,35 @@ __device__ void titem_finish(const GemvParams& p, const TItem& ti, int j, int nk
                              const int* ttb, const float (&v)[N], const int (&tok)[N], const int (&rk)[N],
                              volatile int* bcast) {
     const int r = ti.P->rank, col0 = ti.col - ti.rb;
+    const int n_ttiles = (p.R + kTokTile - 1) / kTokTile + p.n_exp;   // as gemv_sync_ints
     int32_t st = 0;
+    bool ok[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+        ok[i] = tok[i] < ntok && rk[i] < r &&
+                in_range(p.dev_status, row0 + tok[i] >= 0 && row0 + tok[i] < p.R && col0 + rk[i] < p.tcols &&
+                                           ti.ks < p.nks);
     if (nks == 1) {
 #pragma unroll
         for (int i = 0; i < N; ++i)
-            if (tok[i] < ntok && rk[i] < r)
-                p.t[static_cast<size_t>(row0 + tok[i]) * p.tcols + col0 + rk[i]] = t_half(v[i], st);
+            if (ok[i]) p.t[static_cast<size_t>(row0 + tok[i]) * p.tcols + col0 + rk[i]] = t_half(v[i], st);
     } else {
         float* part = p.tpart + static_cast<size_t>(ti.ks) * p.R * p.tcols;
 #pragma unroll
         for (int i = 0; i < N; ++i)
-            if (tok[i] < ntok && rk[i] < r) part[static_cast<size_t>(row0 + tok[i]) * p.tcols + col0 + rk[i]] = v[i];
+            if (ok[i]) part[static_cast<size_t>(row0 + tok[i]) * p.tcols + col0 + rk[i]] = v[i];
         // the CTA's partials, then one thread's acquire-release count: the last
         // slice to count sees every other slice's partials
         consumer_sync();
-        if (threadIdx.x == 0) *bcast = atom_add_acq_rel(&p.tctr[j / nks], 1) == nks - 1;
+        if (threadIdx.x == 0)
+            *bcast = in_range(p.dev_status, j / nks < 4 * n_ttiles) && atom_add_acq_rel(&p.tctr[j / nks], 1) == nks - 1;
         consumer_sync();
         const bool last = *bcast != 0;
         if (last) {
             const size_t slice = static_cast<size_t>(p.R) * p.tcols;
 #pragma unroll
             for (int i = 0; i < N; ++i)
-                if (tok[i] < ntok && rk[i] < r) {
+                if (ok[i]) {
                     const size_t o = static_cast<size_t>(row0 + tok[i]) * p.tcols + col0 + rk[i];
                     float a = 0.0f;
                     for (int s2 = 0; s2 < nks; ++s2) a += __ldcg(p.tpart + s2 * slice + o);
@@ -269,7 +276,8 @@ __device__ void titem_finish(const GemvParams& p, const TItem& ti, int j, int nk
         }
     }
     consumer_sync();          // t is written; one release publishes it
-    if (threadIdx.x == 0) red_add_release(&p.tdone[ttb[ti.e] + ti.tt], 1);
+    if (threadIdx.x == 0 && in_range(p.dev_status, ttb[ti.e] + ti.tt < n_ttiles))
+        red_add_release(&p.tdone[ttb[ti.e] + ti.tt], 1);
     flag(p.dev_status, st);
 }
 
@@ -607,17 +615,28 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                             const int ch = kc / kChunkK;
                             const uint32_t vb = min(2, p.SB - 2 * ch) * kBlockSB;
                             const uint32_t xb = tntok * kFragRowHalves * 2;
-                            mbar_arrive_expect_tx(fb, vb + xb);
-                            bulk_load_hint(st + kOffQ, reinterpret_cast<const uint8_t*>(ti.P->V) + 2 * ch * kBlockSB,
-                                           vb, fb, pol);
-                            bulk_load(st + kOffX, p.x + (static_cast<size_t>(ch) * p.R + trow0) * kFragRowHalves, xb,
-                                      fb);
+                            if (in_range(p.dev_status, ch < p.chunks && 2 * ch < p.SB && tntok > 0 && trow0 >= 0 &&
+                                                           trow0 + tntok <= p.R)) {
+                                mbar_arrive_expect_tx(fb, vb + xb);
+                                bulk_load_hint(st + kOffQ,
+                                               reinterpret_cast<const uint8_t*>(ti.P->V) + 2 * ch * kBlockSB, vb, fb,
+                                               pol);
+                                bulk_load(st + kOffX, p.x + (static_cast<size_t>(ch) * p.R + trow0) * kFragRowHalves,
+                                          xb, fb);
+                            } else {
+                                mbar_arrive(fb);
+                            }
                         } else {
                             const int nbox = min(kTBoxes, (kb1 - kc) / 64);
+                            if (!in_range(p.dev_status, kc + 64 * nbox <= p.K && trow0 >= 0 && trow0 < p.R &&
+                                                            ti.rb < ti.P->rank)) {
+                                mbar_arrive(fb);
+                            } else {
                             mbar_arrive_expect_tx(fb, nbox * (kTXBox + kTVBox));
                             for (int q = 0; q < nbox; ++q) {
                                 tma_load_2d(st + kOffTX + q * kTXBox, &p.smap, fb, kc + 64 * q, trow0);
                                 tma_load_2d(st + kOffTV + q * kTVBox, &ti.P->vmap, fb, kc + 64 * q, ti.rb);
+                            }
                             }
                         }
                     }
@@ -666,10 +685,19 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 const uint16_t* xsrc = p.x + (static_cast<size_t>(ch) * p.R + row0) * kFragRowHalves;
                 if (elect_one()) {
                     if (!header) write_hdr(hdr + stage * kHdrInts, it, w, hinfo);
-                    mbar_arrive_expect_tx(fb, ntl * wb + xb);
-                    bulk_load_hint(st + kOffQ, w0, wb, fb, pol);
-                    if (ntl == 2) bulk_load_hint(st + kOffQ + kTileBlk, w1, wb, fb, pol);
-                    bulk_load(st + kOffX, xsrc, xb, fb);
+                    // each blob holds ceil(N / 64) tiles of SB blocks (SwiGLU: tile
+                    // tile0 of w1's and of w3's; plain: tiles tile0 and tile0 + 1
+                    // of one); the rows exist
+                    if (in_range(p.dev_status, tile0 + (GLU ? 1 : ntl) <= (p.N + kTileRows - 1) / kTileRows &&
+                                                   2 * ch + nsb <= p.SB && ch < p.chunks && ntok > 0 &&
+                                                   row0 >= 0 && row0 + ntok <= p.R)) {
+                        mbar_arrive_expect_tx(fb, ntl * wb + xb);
+                        bulk_load_hint(st + kOffQ, w0, wb, fb, pol);
+                        if (ntl == 2) bulk_load_hint(st + kOffQ + kTileBlk, w1, wb, fb, pol);
+                        bulk_load(st + kOffX, xsrc, xb, fb);
+                    } else {
+                        mbar_arrive(fb);
+                    }
                 }
                 __syncwarp();
                 header = true;
@@ -683,7 +711,9 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                     const int need = (ra == 0 ? 0 : l3a ? 1 : rank_blocks(ra)) +
                                      (GLU && rb > 0 ? (l3b ? 1 : rank_blocks(rb)) : 0);
                     const int32_t* done = p.tdone + ttb[w.e] + w.tt;
-                    if (ld_acquire(done) < need) {
+                    const int n_ttiles = (p.R + kTokTile - 1) / kTokTile + p.n_exp;   // as gemv_sync_ints
+                    const bool dok = in_range(p.dev_status, ttb[w.e] + w.tt < n_ttiles);
+                    if (dok && ld_acquire(done) < need) {
                         const long long t0 = clock64();
                         while (ld_acquire(done) < need) {
                             if (clock64() - t0 > kWaitCycles) {
@@ -717,10 +747,20 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 const uint32_t tb = ntok * p.tcols * 2;
                 if (elect_one()) {
                     if (!header) write_hdr(hdr + stage * kHdrInts, it, w, hinfo);
-                    mbar_arrive_expect_tx(fb, ua + ub + tb);
-                    if (ua) bulk_load_hint(st + kOffUA, usa, ua, fb, pol);
-                    if (ub) bulk_load_hint(st + kOffUB, usb, ub, fb, pol);
-                    bulk_load(st + kOffT, p.t + static_cast<size_t>(row0) * p.tcols, tb, fb);
+                    // U rows n0 .. n0 + urows (fp16) or the int3 U^T block of
+                    // super-block n0 / 128 (N / 128 of them), the rows' t, and
+                    // the stage's room for each
+                    if (in_range(p.dev_status, n0 + urows <= p.N && ua <= (GLU ? kOffUB : kOffT) - kOffUA && ub <= kOffT - kOffUB &&
+                                                   (!l3a || (n0 >> 7) < p.N / 128) &&
+                                                   (!l3b || (n0 >> 7) < p.N / 128) && row0 >= 0 &&
+                                                   row0 + ntok <= p.R && tb <= kStageBytes - kOffT)) {
+                        mbar_arrive_expect_tx(fb, ua + ub + tb);
+                        if (ua) bulk_load_hint(st + kOffUA, usa, ua, fb, pol);
+                        if (ub) bulk_load_hint(st + kOffUB, usb, ub, fb, pol);
+                        bulk_load(st + kOffT, p.t + static_cast<size_t>(row0) * p.tcols, tb, fb);
+                    } else {
+                        mbar_arrive(fb);
+                    }
                 }
                 __syncwarp();
                 header = true;
@@ -917,7 +957,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 for (int i = 0; i < 4; ++i) {
                     const int f = n0 + 16 * warp + g + 8 * (i >> 1);
                     const int tok = n8 * 8 + 2 * c + (i & 1);
-                    if (tok < ntok && f < p.N) {
+                    if (tok < ntok && f < p.N && in_range(p.dev_status, row0 + tok < p.R)) {
                         const float a = acc[0][n8][i] * inv[n8][i & 1], b = acc[1][n8][i] * inv[n8][i & 1];
                         const float hv = __fdividef(a, 1.0f + __expf(-a)) * b;
                         const __half hh = __float2half_rn(hv);
@@ -937,7 +977,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                     for (int i = 0; i < 4; ++i) {
                         const int n = n0 + 32 * warp + 16 * ti + g + 8 * (i >> 1);
                         const int tok = n8 * 8 + 2 * c + (i & 1);
-                        if (tok < ntok && n < p.N)
+                        if (tok < ntok && n < p.N && in_range(p.dev_status, row0 + tok < p.R && w.split < p.splits))
                             out[static_cast<size_t>(row0 + tok) * p.N + n] = acc[ti][n8][i] * inv[n8][i & 1];
                     }
         }

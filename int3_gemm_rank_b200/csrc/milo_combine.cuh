@@ -36,7 +36,8 @@ __device__ __forceinline__ float4 combine4(const CombineParams& p, int o, int n)
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (p.per_slot) {
         const int r = p.inv_perm[o];
-        if (r >= 0) acc = split_sum4(p.y_part, p.splits, sstride, static_cast<size_t>(r) * p.H + n);
+        if (r >= 0 && in_range(p.dev_status, r < p.R))
+            acc = split_sum4(p.y_part, p.splits, sstride, static_cast<size_t>(r) * p.H + n);
         return acc;
     }
     for (int j = 0; j < p.k; ++j) {
@@ -51,6 +52,7 @@ __device__ __forceinline__ float4 combine4(const CombineParams& p, int o, int n)
         acc.w = fmaf(wj, v.w, acc.w);
     }
     for (int s = 0; s < p.S; ++s) {
+        if (!in_range(p.dev_status, p.R_routed + s * p.T + o < p.R)) break;
         const float4 v = split_sum4(p.y_part, p.splits, sstride, static_cast<size_t>(p.R_routed + s * p.T + o) * p.H + n);
         acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }

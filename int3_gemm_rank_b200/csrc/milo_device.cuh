@@ -22,6 +22,19 @@ __device__ __forceinline__ void flag(int32_t* st, int32_t bits) {
     if (st != nullptr && bits) atomicOr(st, bits);
 }
 
+// Range checks of the checked build (MILO_CHECKED): in_range(st, cond) is
+// true when cond holds; otherwise it flags MILO_DEV_BOUNDS and returns false,
+// and the caller skips the access.  In the normal build it is always true and
+// costs nothing.
+#ifdef MILO_CHECKED
+__device__ __forceinline__ bool in_range(int32_t* st, bool cond) {
+    if (!cond) flag(st, MILO_DEV_BOUNDS);
+    return cond;
+}
+#else
+__device__ __forceinline__ constexpr bool in_range(int32_t*, bool) { return true; }
+#endif
+
 // ---------------------------------------------------------------------------
 // programmatic dependent launch
 // ---------------------------------------------------------------------------

@@ -181,8 +181,10 @@ route_kernel(const uint16_t* __restrict__ logits, int T, int E, int k, uint32_t 
         __syncthreads();
         if (valid) {
             const int p = wcnt[warp][e] + rank;
-            perm[p] = f;
-            inv_perm[f] = p;
+            if (in_range(dev_status, p >= 0 && p < F)) {
+                perm[p] = f;
+                inv_perm[f] = p;
+            }
         } else if (f < F) {
             inv_perm[f] = -1;
         }

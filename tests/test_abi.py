@@ -36,6 +36,17 @@ def test_library_exports_every_declared_symbol(milo):
     assert set(milo.EXPORTS) == set(_declared())
 
 
+def test_checked_build_exports_every_declared_symbol():
+    """The checked build (MILO_CHECKED: range checks in the kernels) is the
+    same library with the same entry points."""
+    from int3_gemm_rank_b200 import build
+    path = build.build(checked=True)
+    assert path.endswith("libmilo_checked.so")
+    L = C.CDLL(path)
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
 def test_status_strings_and_version(milo):
     L = milo.lib()
     assert L.milo_version() >= 1
