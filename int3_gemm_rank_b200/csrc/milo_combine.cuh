@@ -18,12 +18,24 @@
 namespace milo {
 
 // Sum over the split-K partials of one row, columns n..n+3, in split order
-// (L2 loads: the partials may come from other CTAs of the same grid).
+// (L2 loads: the partials come from the previous kernel), four loads in
+// flight at a time.
 __device__ __forceinline__ float4 split_sum4(const float* part, int splits, size_t split_stride, size_t off) {
-    float4 a = __ldcg(reinterpret_cast<const float4*>(part + off));
-    for (int s = 1; s < splits; ++s) {
-        const float4 b = __ldcg(reinterpret_cast<const float4*>(part + s * split_stride + off));
-        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < splits; s0 += 4) {
+        float4 v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if (s0 + q < splits) v[q] = __ldcg(reinterpret_cast<const float4*>(part + (s0 + q) * split_stride + off));
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if (s0 + q < splits) {
+                if (s0 + q == 0) {
+                    a = v[0];
+                } else {
+                    a.x += v[q].x; a.y += v[q].y; a.z += v[q].z; a.w += v[q].w;
+                }
+            }
     }
     return a;
 }
@@ -40,16 +52,46 @@ __device__ __forceinline__ float4 combine4(const CombineParams& p, int o, int n)
             acc = split_sum4(p.y_part, p.splits, sstride, static_cast<size_t>(r) * p.H + n);
         return acc;
     }
-    for (int j = 0; j < p.k; ++j) {
-        const int f = o * p.k + j;
-        const int r = p.inv_perm[f];
-        if (r < 0 || r >= p.R_routed) continue;
-        const float wj = p.w[f];
-        const float4 v = split_sum4(p.y_part, p.splits, sstride, static_cast<size_t>(r) * p.H + n);
-        acc.x = fmaf(wj, v.x, acc.x);
-        acc.y = fmaf(wj, v.y, acc.y);
-        acc.z = fmaf(wj, v.z, acc.z);
-        acc.w = fmaf(wj, v.w, acc.w);
+    if (p.splits == 1) {
+        // one partial per slot: eight slots at a time, their rows and weights
+        // first, then all their partial rows in flight at once, added in slot
+        // order
+        for (int j0 = 0; j0 < p.k; j0 += 8) {
+            int rows[8];
+            float wts[8];
+            float4 v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j0 + j < p.k) {
+                    const int f = o * p.k + j0 + j;
+                    rows[j] = p.inv_perm[f];
+                    wts[j] = p.w[f];
+                }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j0 + j < p.k && rows[j] >= 0 && rows[j] < p.R_routed)
+                    v[j] = __ldcg(reinterpret_cast<const float4*>(p.y_part + static_cast<size_t>(rows[j]) * p.H + n));
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j0 + j < p.k && rows[j] >= 0 && rows[j] < p.R_routed) {
+                    acc.x = fmaf(wts[j], v[j].x, acc.x);
+                    acc.y = fmaf(wts[j], v[j].y, acc.y);
+                    acc.z = fmaf(wts[j], v[j].z, acc.z);
+                    acc.w = fmaf(wts[j], v[j].w, acc.w);
+                }
+        }
+    } else {
+        for (int j = 0; j < p.k; ++j) {
+            const int f = o * p.k + j;
+            const int r = p.inv_perm[f];
+            if (r < 0 || r >= p.R_routed) continue;
+            const float wj = p.w[f];
+            const float4 v = split_sum4(p.y_part, p.splits, sstride, static_cast<size_t>(r) * p.H + n);
+            acc.x = fmaf(wj, v.x, acc.x);
+            acc.y = fmaf(wj, v.y, acc.y);
+            acc.z = fmaf(wj, v.z, acc.z);
+            acc.w = fmaf(wj, v.w, acc.w);
+        }
     }
     for (int s = 0; s < p.S; ++s) {
         if (!in_range(p.dev_status, p.R_routed + s * p.T + o < p.R)) break;

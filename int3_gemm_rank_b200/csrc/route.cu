@@ -23,45 +23,46 @@ constexpr int kRouteSplitT = 512;            // from this many tokens the top-k 
 
 // Top-k of token t, one warp: the lanes hold the token's logits (expert e at
 // lane e % 32, slot e / 32) and k rounds of a warp arg-max pick the largest
-// remaining logit, ties to the lower expert id (a key orders by value, then by
-// descending id).  NaN counts as -inf (and is flagged).  Slot j = j-th pick.
+// remaining logit, ties to the lower expert id.  A 32-bit key orders by value
+// (the fp16 bits made order-preserving) in its high half and by descending id
+// in its low half, so one warp max-reduction picks; 0 marks empty or picked.
+// NaN counts as -inf (and is flagged).  Slot j = j-th pick.
 __device__ __forceinline__ void topk_token(const uint16_t* __restrict__ logits, int t, int E, int k, uint32_t flags,
                                            int32_t* __restrict__ ids, float* __restrict__ wts, int lane,
                                            int32_t& st) {
     constexpr int kSlots = (MILO_MAX_EXPERTS + 31) / 32;
     const uint16_t* l = logits + static_cast<size_t>(t) * E;
     float v[kSlots];
-    unsigned long long key[kSlots];
+    uint32_t key[kSlots];
 #pragma unroll
     for (int i = 0; i < kSlots; ++i) {
         const int e = 32 * i + lane;
         v[i] = -INFINITY;
-        key[i] = 0ull;   // below every real key: empty or already picked
+        key[i] = 0u;   // below every real key: empty or already picked
         if (e < E) {
-            float x = __half2float(__ushort_as_half(l[e]));
+            uint32_t b = l[e];
+            float x = __half2float(__ushort_as_half(static_cast<uint16_t>(b)));
             if (!isfinite(x)) st |= MILO_DEV_NONFINITE;
-            if (x != x) x = -INFINITY;
+            if (x != x) {
+                x = -INFINITY;
+                b = 0xFC00u;   // fp16 -inf
+            }
             v[i] = x;
-            const uint32_t b = __float_as_uint(x);
-            const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-            key[i] = (static_cast<unsigned long long>(ord) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e));
+            const uint32_t ord = (b & 0x8000u) ? (~b & 0xFFFFu) : (b | 0x8000u);
+            key[i] = (ord << 16) | (0xFFFFu - static_cast<uint32_t>(e));
         }
     }
     // lane j keeps pick j (k <= 16 < 32); the renormalising sum runs in slot order
     int my_e = 0;
     float my_v = 0.0f, m = 0.0f, den = 0.0f;
     for (int j = 0; j < k; ++j) {
-        unsigned long long best = 0ull;
+        uint32_t best = 0u;
 #pragma unroll
-        for (int i = 0; i < kSlots; ++i) best = key[i] > best ? key[i] : best;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, best, o);
-            best = other > best ? other : best;
-        }
-        const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best & 0xFFFFFFFFull));
-        const uint32_t ord = static_cast<uint32_t>(best >> 32);
-        const float val = __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
+        for (int i = 0; i < kSlots; ++i) best = max(best, key[i]);
+        best = __reduce_max_sync(0xFFFFFFFFu, best);
+        const int e = static_cast<int>(0xFFFFu - (best & 0xFFFFu));
+        const uint32_t ord = best >> 16;
+        const float val = __half2float(__ushort_as_half(static_cast<uint16_t>((ord & 0x8000u) ? (ord & 0x7FFFu) : (~ord & 0xFFFFu))));
         if (j == 0) m = val;
         if (flags & MILO_ROUTE_RENORM) den += expf(val - m);
         if (lane == j) {
@@ -70,7 +71,7 @@ __device__ __forceinline__ void topk_token(const uint16_t* __restrict__ logits, 
         }
 #pragma unroll
         for (int i = 0; i < kSlots; ++i)
-            if (32 * i + lane == e) key[i] = 0ull;
+            if (32 * i + lane == e) key[i] = 0u;
     }
     if (!(flags & MILO_ROUTE_RENORM)) {
 #pragma unroll
