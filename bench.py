@@ -253,7 +253,7 @@ def kernel_source_hash(tensor: bool = False) -> str:
     """Hash of the sources the profiled GEMM kernel is built from."""
     h = hashlib.sha256()
     files = ("int3_gemm_rank_b200/csrc/gemm_tc.cu", "int3_gemm_rank_b200/csrc/milo_tc.cuh") if tensor else \
-        ("int3_gemm_rank_b200/csrc/gemv.cu", "int3_gemm_rank_b200/csrc/milo_combine.cuh")
+        ("int3_gemm_rank_b200/csrc/gemv.cu",)
     for rel in files + ("int3_gemm_rank_b200/csrc/milo_device.cuh", "int3_gemm_rank_b200/csrc/milo_kernels.h"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
