@@ -67,12 +67,14 @@ constexpr int kOffX = 2 * kTileBlk;                       // 14336
 constexpr int kStageBytes = 23552;
 constexpr int kOffUA = 0, kOffUB = 8192, kOffT = 16384;   // compensator stage
 constexpr int kBarOffset = kStages * kStageBytes;
-// barriers, then the item tables cnt, row0s, ttb, tstart [MILO_MAX_EXPERTS + 1],
-// the stage headers (kHdrInts each) and the consumers' broadcast word; 1 KB
-// of slack to align the base
+// barriers, then the item tables cnt, row0s, tpos, tstart [MILO_MAX_EXPERTS +
+// 1], the stage headers (kHdrInts each), the consumers' broadcast word and
+// the expert order ord, pos [MILO_MAX_EXPERTS] (bytes); 1 KB of slack to
+// align the base
 constexpr int kHdrInts = 8;
 constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 4 * (MILO_MAX_EXPERTS + 1) * 4 + kStages * kHdrInts * 4 + 16 +
-                           1024;
+                           2 * MILO_MAX_EXPERTS + 1024;
+static_assert(MILO_MAX_EXPERTS <= 256, "expert order in bytes");
 
 static_assert(kOffX + kTokTile * kFragRowHalves * 2 <= kStageBytes, "GEMM stage");
 static_assert(kStageBytes % 1024 == 0, "stage alignment");
@@ -96,14 +98,16 @@ __device__ __forceinline__ int find_expert(int it, const int* first, int mul, in
     return lo;
 }
 
-// GEMM item `it`: expert e owns items [ttb[e], ttb[e+1]) * n_tiles * splits
-// (ttb: prefix of the experts' 16-row token tiles), its token tiles fastest,
-// then the K splits, then the weight-row tiles.
-__device__ __forceinline__ Item decode_item(int it, const int* ttb, const int* cnt, int n_exp, int n_tiles,
-                                            int splits) {
+// GEMM item `it`: the experts take turns in the order ord (most routed rows
+// first); the expert at position k owns items [tpos[k], tpos[k+1]) * n_tiles
+// * splits (tpos: prefix of the 16-row token tiles in that order), its token
+// tiles fastest, then the K splits, then the weight-row tiles.
+__device__ __forceinline__ Item decode_item(int it, const int* tpos, const uint8_t* ord, const int* cnt, int n_exp,
+                                            int n_tiles, int splits) {
     Item r;
-    r.e = find_expert(it, ttb, n_tiles * splits, n_exp);
-    const int local = it - ttb[r.e] * n_tiles * splits;
+    const int k = find_expert(it, tpos, n_tiles * splits, n_exp);
+    r.e = ord[k];
+    const int local = it - tpos[k] * n_tiles * splits;
     const int tte = (cnt[r.e] + kTokTile - 1) / kTokTile;
     r.tt = local % tte;
     const int rest = local / tte;
@@ -231,7 +235,8 @@ __device__ bool titem_tma(const TItem& ti, int kb0, int kb1, const uint8_t* smem
 // tile.
 template <bool GLU, int N>
 __device__ void titem_finish(const GemvParams& p, const TItem& ti, int j, int nks, int row0, int ntok,
-                             const int* ttb, const float (&v)[N], const int (&tok)[N], const int (&rk)[N],
+                             const int* tpos, const uint8_t* pos, const float (&v)[N], const int (&tok)[N],
+                             const int (&rk)[N],
                              volatile int* bcast) {
     const int r = ti.P->rank, col0 = ti.col - ti.rb;
     const int n_ttiles = (p.R + kTokTile - 1) / kTokTile + p.n_exp;   // as gemv_sync_ints
@@ -276,8 +281,8 @@ __device__ void titem_finish(const GemvParams& p, const TItem& ti, int j, int nk
         }
     }
     consumer_sync();          // t is written; one release publishes it
-    if (threadIdx.x == 0 && in_range(p.dev_status, ttb[ti.e] + ti.tt < n_ttiles))
-        red_add_release(&p.tdone[ttb[ti.e] + ti.tt], 1);
+    const int tile = tpos[pos[ti.e]] + ti.tt;   // the token tile's slot
+    if (threadIdx.x == 0 && in_range(p.dev_status, tile < n_ttiles)) red_add_release(&p.tdone[tile], 1);
     flag(p.dev_status, st);
 }
 
@@ -491,14 +496,18 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
     uint64_t* empty = full + kStages;
     int* cnt = reinterpret_cast<int*>(empty + kStages);
     int* row0s = cnt + (MILO_MAX_EXPERTS + 1);
-    int* ttb = row0s + (MILO_MAX_EXPERTS + 1);       // prefix of the experts' token tiles
-    int* tstart = ttb + (MILO_MAX_EXPERTS + 1);      // prefix of the experts' t-items
+    int* tpos = row0s + (MILO_MAX_EXPERTS + 1);      // prefix of the token tiles in expert order ord
+    int* tstart = tpos + (MILO_MAX_EXPERTS + 1);     // prefix of the experts' t-items (expert index order)
     // header of each stage: the work item whose first stage it is (-1: no more
     // items, -2 - j: t-item j), then for a GEMM item what the producer decoded
     // for it (expert, weight tile, token tile and K split, the ranks and
     // compensator formats), so that the consumers need no global loads for it
     volatile int* hdr = tstart + (MILO_MAX_EXPERTS + 1);
     volatile int* bcast = hdr + kStages * kHdrInts;   // consumers' broadcast word
+    // the GEMM items' expert order (most routed rows first, then by index) and
+    // each expert's position in it
+    uint8_t* ord = reinterpret_cast<uint8_t*>(const_cast<int*>(bcast) + 4);
+    uint8_t* pos = ord + MILO_MAX_EXPERTS;
 
     constexpr int RA = GLU ? kRowsGlu : kRowsPlain;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -520,7 +529,6 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         cnt[e] = ok ? m : 0;
         row0s[e] = r0;
         const int tte = ok ? (m + kTokTile - 1) / kTokTile : 0;
-        ttb[e] = tte;
         int nt = 0;
         if (p.t_items && tte > 0) {
             const int na = t_blocks(p.table + e * p.stride + p.proj_a);
@@ -530,11 +538,23 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         tstart[e] = nt;
     }
     __syncthreads();
+    // Whole waves of round-robin items are even; the last, partial one is not,
+    // so the costlier items (more routed rows: 16-token tiles, several tiles)
+    // go first and the last wave holds the cheapest.
+    for (int e = threadIdx.x; e < p.n_exp; e += blockDim.x) {
+        int rank = 0;
+        for (int f = 0; f < p.n_exp; ++f) rank += cnt[f] > cnt[e] || (cnt[f] == cnt[e] && f < e);
+        pos[e] = static_cast<uint8_t>(rank);
+        ord[rank] = static_cast<uint8_t>(e);
+    }
+    __syncthreads();
+    for (int k = threadIdx.x; k < p.n_exp; k += blockDim.x) tpos[k] = (cnt[ord[k]] + kTokTile - 1) / kTokTile;
+    __syncthreads();
     if (warp == 0) {
         int run = 0, trun = 0;
         for (int base = 0; base < p.n_exp; base += 32) {
             const int e = base + lane;
-            const int a = e < p.n_exp ? ttb[e] : 0, b = e < p.n_exp ? tstart[e] : 0;
+            const int a = e < p.n_exp ? tpos[e] : 0, b = e < p.n_exp ? tstart[e] : 0;
             int ia = a, ib = b;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -543,19 +563,19 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                 if (lane >= o) { ia += ya; ib += yb; }
             }
             if (e < p.n_exp) {
-                ttb[e] = run + ia - a;
+                tpos[e] = run + ia - a;
                 tstart[e] = trun + ib - b;
             }
             run += __shfl_sync(0xFFFFFFFFu, ia, 31);
             trun += __shfl_sync(0xFFFFFFFFu, ib, 31);
         }
         if (lane == 0) {
-            ttb[p.n_exp] = run;
+            tpos[p.n_exp] = run;
             tstart[p.n_exp] = trun;
         }
     }
     __syncthreads();
-    const int n_items = ttb[p.n_exp] * n_tiles * p.splits;
+    const int n_items = tpos[p.n_exp] * n_tiles * p.splits;
     // K slices of the t-items: about one t-item per CTA (each slice pays a
     // fixed cost in counting and partial sums), at most p.nks slices, each a
     // whole number of stages; every CTA derives the same values from the same
@@ -651,7 +671,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
             if (it < 0 || it >= n_items) break;
             next += gridDim.x;
             bool header = false;      // the item's first stage has been filled
-            const Item w = decode_item(it, ttb, cnt, p.n_exp, n_tiles, p.splits);
+            const Item w = decode_item(it, tpos, ord, cnt, p.n_exp, n_tiles, p.splits);
             const ProjDev* pa = p.table + w.e * p.stride + p.proj_a;
             const ProjDev* pb = p.table + w.e * p.stride + p.proj_b;
             const int n0 = w.ntile * RA;
@@ -710,9 +730,9 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                     // wait (bounded) until all its rank blocks are done
                     const int need = (ra == 0 ? 0 : l3a ? 1 : rank_blocks(ra)) +
                                      (GLU && rb > 0 ? (l3b ? 1 : rank_blocks(rb)) : 0);
-                    const int32_t* done = p.tdone + ttb[w.e] + w.tt;
+                    const int32_t* done = p.tdone + tpos[pos[w.e]] + w.tt;
                     const int n_ttiles = (p.R + kTokTile - 1) / kTokTile + p.n_exp;   // as gemv_sync_ints
-                    const bool dok = in_range(p.dev_status, ttb[w.e] + w.tt < n_ttiles);
+                    const bool dok = in_range(p.dev_status, tpos[pos[w.e]] + w.tt < n_ttiles);
                     if (dok && ld_acquire(done) < need) {
                         const long long t0 = clock64();
                         while (ld_acquire(done) < need) {
@@ -853,7 +873,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                     tok[q] = 8 * n8 + 2 * c + (i & 1);
                     rk[q] = 16 * warp + g + 8 * (i >> 1);
                 }
-                titem_finish<GLU, 8>(p, ti, j, nks, trow0, tntok, ttb, v, tok, rk, bcast);
+                titem_finish<GLU, 8>(p, ti, j, nks, trow0, tntok, tpos, pos, v, tok, rk, bcast);
             } else {
                 float tacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                 if (!titem_tma(ti, kb0, kb1, smem, full, empty, stage, phase, warp, lane, tacc)) {
@@ -867,7 +887,7 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
                     tok[i] = g + 8 * (i >> 1);
                     rk[i] = ti.rb + 8 * warp + 2 * c + (i & 1);
                 }
-                titem_finish<GLU, 4>(p, ti, j, nks, trow0, tntok, ttb, tacc, tok, rk, bcast);
+                titem_finish<GLU, 4>(p, ti, j, nks, trow0, tntok, tpos, pos, tacc, tok, rk, bcast);
             }
             continue;
         }
