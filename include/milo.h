@@ -355,13 +355,16 @@ MILO_API milo_status milo_table_bytes(int32_t n_projections, size_t* bytes);
 /*
  * milo_linear_prepare / milo_layer_prepare -- validate the weights (host
  * array `weights` / `experts` of device pointers) and write the device table
- * (pointers and shapes) to `device_table`, which the caller keeps
- * alive and unmodified while the layer is used.  One-time set-up: the table is
- * copied with a synchronous cudaMemcpy.  lin/layer are host structs; the
- * caller fills the shape fields and the call sets max_rank and table.
+ * (pointers, shapes and, for an fp16 V, a TMA tensor map of V) to
+ * `device_table`, which the caller keeps alive and unmodified while the layer
+ * is used; the weights, U and V must stay at the same addresses too (the
+ * tensor map holds V's).  One-time set-up: the table is copied with a
+ * synchronous cudaMemcpy.  lin/layer are host structs; the caller fills the
+ * shape fields and the call sets max_rank and table.
  * Errors: UNSUPPORTED_SHAPE (K % 128, N % 16, group != 64, rank not a multiple
  * of 8 or above MILO_MAX_RANK), WORKSPACE (table too small or not 64-byte
- * aligned), INVALID_ARG (NULL or misaligned weight pointers).
+ * aligned), INVALID_ARG (NULL or misaligned weight pointers, or a tensor map
+ * the driver refuses to encode), CUDA (no tensor-map encoder in the driver).
  */
 MILO_API milo_status milo_linear_prepare(milo_linear* lin, const milo_qweight* weights,
                                 void* device_table, size_t table_bytes);
