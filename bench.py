@@ -565,8 +565,9 @@ def roofline(args, pk, bytes_, glu_ms, glu_gbs) -> dict:
         peak = pk["bf16_tflops"]
         return {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
                 "frac_of_sustained": tf / pk["bf16_tflops_sustained"],
+                # the captures are of the default workloads (fp16 compensators)
                 "traffic": profiled_traffic("tc_gemm_glu_prefill.md", tensor=True)
-                if args.workload == "prefill" and args.tokens is None else None,
+                if args.workload == "prefill" and args.tokens is None and args.lorc == "fp16" else None,
                 "kernel": "tc_gemm_kernel<true> (w1|w3 grouped int3 GEMM on tcgen05 + compensator + SwiGLU)",
                 "algorithmic_flops_per_launch": bytes_["glu_flops"], "ms_per_launch": glu_ms,
                 "peak_source": "measured cuBLAS bf16 GEMM, burst (MEASURED_PEAKS.json bf16_tflops); "
@@ -574,7 +575,7 @@ def roofline(args, pk, bytes_, glu_ms, glu_gbs) -> dict:
                 else "fallback 1590 TFLOP/s"}
     return {"bound": "hbm", "achieved": glu_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": glu_gbs / pk["hbm_gbs"], "traffic": profiled_traffic("gemv_glu_mixtral_decode.md")
-            if args.workload == "mixtral" and args.tokens is None else None,
+            if args.workload == "mixtral" and args.tokens is None and args.lorc == "fp16" else None,
             "kernel": "gemv_kernel<true> (w1|w3 grouped int3 GEMM + compensator + SwiGLU)",
             "algorithmic_bytes_per_launch": bytes_["glu_kernel"], "ms_per_launch": glu_ms,
             "peak_source": f"{pk['source']} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
