@@ -473,10 +473,7 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
     const int nproj = p.proj_b >= 0 ? 2 : 1;
     const int which = blockIdx.x % nproj, e = blockIdx.x / nproj;
     const ProjDev* P = p.table + e * p.stride + (which == 0 ? p.proj_a : p.proj_b);
-    // the projection's fields, read once (the loop's stores could alias them)
     const int r = P->rank;
-    const bool l3 = P->lorc3 != 0;
-    const uint16_t* const Vp = P->V;
     const int span = p.proj_b >= 0 ? p.t_col_b : p.tcols;
     const int col0 = which == 0 ? 0 : p.t_col_b;
     const int row0 = p.grp[2 * e], m = p.grp[2 * e + 1];
@@ -505,7 +502,7 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
         // int3 V: a chunk of 64 positions is one group, 16 codes in each of the
         // super-block's four units; this thread takes rank row tid / 2, units
         // 2 (tid & 1) and 2 (tid & 1) + 1 (positions 32 (tid & 1) .. + 31)
-        const uint8_t* vb = reinterpret_cast<const uint8_t*>(Vp);
+        const uint8_t* vb = reinterpret_cast<const uint8_t*>(P->V);
         const int urow = threadIdx.x >> 1, uu = threadIdx.x & 1;
         uint32_t vw[6] = {0u, 0u, 0u, 0u, 0u, 0u}, vsz = 0u;
         auto fetch = [&](int kc) {
@@ -516,11 +513,11 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
                 const int sr = src_row[rr];
                 xr[q] = sr >= 0 ? *reinterpret_cast<const uint4*>(p.src + static_cast<size_t>(sr) * p.K + kc + 8 * pc)
                                 : make_uint4(0u, 0u, 0u, 0u);
-                if (!l3)
-                    vr[q] = rr < r ? *reinterpret_cast<const uint4*>(Vp + static_cast<size_t>(rr) * p.K + kc + 8 * pc)
+                if (!P->lorc3)
+                    vr[q] = rr < r ? *reinterpret_cast<const uint4*>(P->V + static_cast<size_t>(rr) * p.K + kc + 8 * pc)
                                    : make_uint4(0u, 0u, 0u, 0u);
             }
-            if (l3 && urow < r) {
+            if (P->lorc3 && urow < r) {
                 const uint32_t* wp = reinterpret_cast<const uint32_t*>(vb + lorc_words_off(urow, kc >> 7, 2 * uu));
 #pragma unroll
                 for (int q = 0; q < 6; ++q) vw[q] = wp[q];
@@ -540,9 +537,9 @@ __global__ void __launch_bounds__(128) lorc_tile_kernel(const LorcParams p) {
                 const int i = threadIdx.x + 128 * q;
                 const int rr = i >> 3, pc = i & 7;
                 *reinterpret_cast<uint4*>(&xs[rr][8 * pc]) = scaled_pairs(xr[q], p.src_bf16, src_scale[rr], st);
-                if (!l3) *reinterpret_cast<uint4*>(&vs[rr][8 * pc]) = vr[q];
+                if (!P->lorc3) *reinterpret_cast<uint4*>(&vs[rr][8 * pc]) = vr[q];
             }
-            if (l3) {
+            if (P->lorc3) {
                 uint32_t h[2][8];
                 if (urow < r) {
                     const int half = (kc >> 6) & 1;
