@@ -594,6 +594,7 @@ def finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, l
         "config": {"workload": describe(wk), "tokens_per_step": T, "x_dtype": wk.x_dtype,
                    "compensator": "int3 (U^T and V packed like the weights)" if args.lorc == "int3" else "fp16",
                    "y_dtype": "bf16",
+                   "compute_dtype": "int3 codes x f16 activations (exact f16 code patterns), f32 accumulate",
                    "l2": f"inputs larger than L2: {bytes_['weights_only'] / 1e6:.0f} MB of packed weights "
                          f"streamed per step vs {L2_BYTES / 1e6:.0f} MB L2; no flush",
                    "parallelism": f"replica per GPU x{world}", "active_experts": bytes_["active_experts"],
