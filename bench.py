@@ -34,6 +34,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -249,14 +250,23 @@ def peaks() -> dict:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def _code_only(text: str) -> str:
+    """Source text without its comments and blank lines (comment edits leave
+    the kernel, and so its captured traffic, unchanged)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash(tensor: bool = False) -> str:
-    """Hash of the sources the profiled GEMM kernel is built from."""
+    """Hash of the code (comments stripped) of the sources the profiled GEMM
+    kernel is built from."""
     h = hashlib.sha256()
     files = ("int3_gemm_rank_b200/csrc/gemm_tc.cu", "int3_gemm_rank_b200/csrc/milo_tc.cuh") if tensor else \
         ("int3_gemm_rank_b200/csrc/gemv.cu",)
     for rel in files + ("int3_gemm_rank_b200/csrc/milo_device.cuh", "int3_gemm_rank_b200/csrc/milo_kernels.h"):
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

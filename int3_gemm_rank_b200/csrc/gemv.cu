@@ -31,7 +31,11 @@
 //     multiplies by 2^-a.  The zero point thus costs nothing per weight and
 //     the result is exact to fp32 rounding.
 //   - The compensator runs as extra K-steps on the same accumulators:
-//     A = U rows (fp16), B = t = x V^T (fp16, computed beforehand per expert).
+//     A = U rows (fp16, or decoded from the int3 U^T blob), B = t = x V^T
+//     (fp16).  t itself comes from "t-items" of the same launch, which every
+//     CTA runs first (see decode_titem): the rows' plain copy times V by
+//     ldmatrix + mma.sync from TMA boxes (fp16 V), or the V blob decoded by
+//     this kernel's own chunk code (int3 V).
 //   - Epilogue: SwiGLU h = silu(a) * b in the w1|w3 kernel (both rows live in
 //     the same lane), or fp32 partial sums per K split for the plain one.
 //   - A K chunk is two super-blocks; when K/128 is odd the last chunk has one,
@@ -40,8 +44,10 @@
 //     on the device from the expert offsets, so the host never synchronises;
 //     CTAs are persistent (three per SM) and walk the items round-robin, the
 //     token tiles of one weight tile being adjacent so that they share L2.
-//     The consumers learn each item from a header the producer writes into
-//     the item's first stage.
+//     The consumers learn each item, and what the producer decoded for it,
+//     from a header the producer writes into the item's first stage; the
+//     experts take turns in order of routed rows, most first, so that the
+//     partial last round holds the cheapest items.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -610,7 +616,8 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_kernel(const __grid_cons
         for (;;) {
             if (tj < n_t) {
                 // a t-item: with fp16 V its stages of plain rows and V rows by
-                // TMA; with an int3 V one header-only stage
+                // TMA; with an int3 V, like a GEMM item, its V-blob chunks and
+                // the rows' prepared activations by bulk copies
                 const TItem ti = decode_titem<GLU>(p, tj, nks, tstart);
                 const int kb0 = ti.ks * kslice, kb1 = min(p.K, kb0 + kslice);
                 const int trow0 = row0s[ti.e] + kTokTile * ti.tt;

@@ -1,8 +1,6 @@
 // milo_combine.cuh -- the weighted un-permute of the MoE layer's expert
 // outputs back to token order (or, for the grouped linear, the copy of each
-// routed slot's row), four output columns at a time.  Used by the combine
-// kernel and by the grouped GEMM's fused combine (the last work item of an
-// output tile combines that tile).
+// routed slot's row), four output columns at a time (the combine kernel).
 //
 // "MiLo: Efficient Quantized MoE Inference with Mixture of Low-Rank
 // Compensators", "Background": an MoE layer sends each token to a subset of
