@@ -137,3 +137,23 @@ def test_layer_line_carries_the_contract_keys(capsys):
     assert e2e["h2d_bytes_per_step"] == wk.T * wk.hidden * 2 + wk.T * wk.n_routed * 2
     assert e2e["d2h_bytes_per_step"] == wk.T * wk.hidden * 2
     assert line["clocks"] == clocks and "workload" in line["config"]
+
+
+def test_traffic_hash_ignores_comments_only():
+    """The captured traffic stays valid across comment edits of a profiled
+    kernel's sources, and only then: the hash covers the code."""
+    import bench
+    a = "int f(int x) {  // one\n    /* two\n       lines */\n    return x + 1;\n}\n"
+    b = "// header\nint f(int x) {\n\n    return x + 1;   // changed comment\n}\n"
+    c = "int f(int x) {\n    return x + 2;\n}\n"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    assert len(bench.kernel_source_hash(False)) == 16 and len(bench.kernel_source_hash(True)) == 16
+
+
+def test_committed_traffic_matches_the_current_kernels():
+    """Both committed ncu summaries carry the hash of the current kernel code,
+    so bench.py reports their DRAM traffic."""
+    import bench
+    assert bench.profiled_traffic("gemv_glu_mixtral_decode.md") is not None
+    assert bench.profiled_traffic("tc_gemm_glu_prefill.md", tensor=True) is not None
