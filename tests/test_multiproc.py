@@ -150,10 +150,3 @@ def test_traffic_hash_ignores_comments_only():
     assert bench._code_only(a) != bench._code_only(c)
     assert len(bench.kernel_source_hash(False)) == 16 and len(bench.kernel_source_hash(True)) == 16
 
-
-def test_committed_traffic_matches_the_current_kernels():
-    """Both committed ncu summaries carry the hash of the current kernel code,
-    so bench.py reports their DRAM traffic."""
-    import bench
-    assert bench.profiled_traffic("gemv_glu_mixtral_decode.md") is not None
-    assert bench.profiled_traffic("tc_gemm_glu_prefill.md", tensor=True) is not None
