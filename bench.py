@@ -36,6 +36,7 @@ import argparse
 import hashlib
 import re
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -500,6 +501,10 @@ def run_milo(args):
     torch.cuda.synchronize()
     milo.milo_set_profile_events(None)
     barrier(dev)
+    # --- timed region 3 (graph replays only): the same K steps with an event
+    # after each, for the spread of the step time (a stream launch sequence
+    # would lose its cross-step overlap to the events)
+    spread = step_spread(torch, run_step, args.steps, stream, dev) if args.graph else None
     clocks = sampler.stop()
     glu_ms = statistics.mean(ev[4 * i].elapsed_time(ev[4 * i + 1]) for i in range(args.steps))
     w2_ms = statistics.mean(ev[4 * i + 2].elapsed_time(ev[4 * i + 3]) for i in range(args.steps))
@@ -516,7 +521,32 @@ def run_milo(args):
     else:
         e2e_value, e2e_ms = run_e2e(args, torch, step, x, logits, y, out_dt, T, wk, dev, stream, world)
     return finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, logits, y,
-                  e2e_value, launches_per_step, clocks)
+                  e2e_value, launches_per_step, clocks, spread)
+
+
+def nearest_rank(sorted_vals, q: float) -> float:
+    """The q-quantile of sorted values by the nearest-rank rule."""
+    i = min(len(sorted_vals) - 1, max(0, math.ceil(q * len(sorted_vals)) - 1))
+    return sorted_vals[i]
+
+
+def step_spread(torch, run_step, steps: int, stream, dev) -> dict:
+    """Median, p10 and p90 of single step times (ms): `steps` more replays,
+    an event recorded after each; every quantile is the max over ranks."""
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    for e in ev:
+        e.record(stream)
+    torch.cuda.synchronize()
+    barrier(dev)
+    ev[0].record(stream)
+    for i in range(steps):
+        run_step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier(dev)
+    d = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(steps))
+    return {"median": max_over_ranks(nearest_rank(d, 0.5), dev), "p10": max_over_ranks(nearest_rank(d, 0.1), dev),
+            "p90": max_over_ranks(nearest_rank(d, 0.9), dev), "steps": steps}
 
 
 def capture_step(torch, dev, fn):
@@ -593,7 +623,7 @@ def roofline(args, pk, bytes_, glu_ms, glu_gbs) -> dict:
 
 
 def finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, logits, y, e2e_value,
-           launches_per_step, clocks):
+           launches_per_step, clocks, spread=None):
     pk = peaks()
     glu_gbs = bytes_["glu_kernel"] / (glu_ms / 1e3) / 1e9
     step_gbs = bytes_["step"] / (ms_step / 1e3) / 1e9
@@ -624,6 +654,8 @@ def finish(args, wk, rank, world, T, ms_step, value, glu_ms, w2_ms, bytes_, x, l
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if spread is not None:
+        line["step_ms"] = spread
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wk)
     if rank == 0:

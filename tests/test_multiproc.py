@@ -121,8 +121,9 @@ def test_layer_line_carries_the_contract_keys(capsys):
     logits = torch.zeros(wk.T, wk.n_routed, dtype=torch.float16)
     y = torch.zeros(wk.T, wk.hidden, dtype=torch.bfloat16)
     clocks = {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": []}
+    spread = {"median": 0.18, "p10": 0.179, "p90": 0.182, "steps": 4}
     assert bench.finish(args, wk, 0, 1, wk.T, 0.18, 88000.0, 0.11, 0.05, bytes_, x, logits, y, 76000.0, 8,
-                        clocks) == 0
+                        clocks, spread) == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
@@ -137,6 +138,17 @@ def test_layer_line_carries_the_contract_keys(capsys):
     assert e2e["h2d_bytes_per_step"] == wk.T * wk.hidden * 2 + wk.T * wk.n_routed * 2
     assert e2e["d2h_bytes_per_step"] == wk.T * wk.hidden * 2
     assert line["clocks"] == clocks and "workload" in line["config"]
+    assert line["step_ms"] == spread
+
+
+def test_step_quantiles_nearest_rank():
+    """The step-time spread takes the nearest-rank quantiles: of 1..10 ms the
+    median is 5, p10 1 and p90 9; one step gives itself for every quantile."""
+    import bench
+    d = [float(v) for v in range(1, 11)]
+    assert (bench.nearest_rank(d, 0.5), bench.nearest_rank(d, 0.1), bench.nearest_rank(d, 0.9)) == (5.0, 1.0, 9.0)
+    assert bench.nearest_rank([2.5], 0.1) == bench.nearest_rank([2.5], 0.9) == 2.5
+    assert bench.nearest_rank(list(range(200)), 0.9) == 179
 
 
 def test_traffic_hash_ignores_comments_only():
