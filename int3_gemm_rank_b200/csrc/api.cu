@@ -292,8 +292,13 @@ static MoeWs moe_ws(const milo_moe_layer* L, int T) {
     w.tc = use_tc(w.R_routed, L->n_routed);
     const int n_exp = L->n_routed + L->n_shared;
     const int chunks = (I + kChunkK - 1) / kChunkK;
-    const long long groups = std::min<long long>(L->n_routed, std::max(1LL, static_cast<long long>(w.R_routed))) + L->n_shared;
-    w.splits = choose_splits(groups * tiles_of(H, kRowsPlain), chunks);
+    // 16-row token tiles: the routed rows fill at least one per expert they
+    // reach and at least R_routed / 16 in all; each shared expert sees all T
+    // tokens
+    const long long routed_tt = std::max(std::min<long long>(L->n_routed, std::max(1LL, static_cast<long long>(w.R_routed))),
+                                         (static_cast<long long>(w.R_routed) + kTokTile - 1) / kTokTile);
+    const long long token_tiles = routed_tt + static_cast<long long>(L->n_shared) * ((T + kTokTile - 1) / kTokTile);
+    w.splits = choose_splits(token_tiles * tiles_of(H, kRowsPlain), chunks);
     w.tc13 = std::max(8, 2 * L->max_rank);
     w.tc2 = std::max(8, L->max_rank);
     w.grp = c.take(static_cast<size_t>(n_exp) * 8);
