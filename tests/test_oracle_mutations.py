@@ -47,6 +47,16 @@ MUTANTS = {
     "hqq_best_zero_not_kept": ("best_err = err;\n            best_z = z;", "best_err = err;"),
     "hqq_l2_error": ("err = err + a;", "err = err + a * a;"),
     "hqq_scale_index_transposed": ("sz = (size_t)j * J->N + n;", "sz = (size_t)n * (J->K / 64) + j;"),
+    "swiglu_gate_swapped": ("double v = milo_ref_silu(a[i]) * b[i];", "double v = milo_ref_silu(b[i]) * a[i];"),
+    "bf16_read_as_fp16": ("X[i] = x_is_bf16 ? milo_ref_bf2d(x[i]) : milo_ref_h2d(x[i]);",
+                          "X[i] = milo_ref_h2d(x[i]);"),
+    "h_overflow_not_flagged": ("else if (!isfinite(h[i])) status |= REF_FP16_RANGE;", ";"),
+    "d2h_binade_carry_lost": ("if (m == 2048.0) { m = 1024.0; e += 1; }", "if (m == 2048.0) { m = 2047.0; }"),
+    "codes_clamped_at_6": ("/* also maps NaN to 0 */\n                if (r > 7.0f) r = 7.0f;",
+                           "/* also maps NaN to 0 */\n                if (r > 6.0f) r = 6.0f;"),
+    "zero_point_unrounded": ("float z = h2f(z_h);", "float z = z_f;"),
+    "int3_compensator_scale_index_transposed": ("double s = milo_ref_h2d(sc[(size_t)j * R + p]);",
+                                                "double s = milo_ref_h2d(sc[(size_t)p * (Cc / group) + j]);"),
 }
 
 
