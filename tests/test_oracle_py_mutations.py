@@ -36,6 +36,16 @@ MUTANTS = {
     "ranks_negative_scores_by_magnitude": ("""    s = [max(float(x), 0.0) for x in scores]""",
                                            """    s = [abs(float(x)) for x in scores]"""),
     "ranks_budget_off_by_one": ("""    units = min(n * avg_rank // 8, cap * n)""", """    units = min(n * avg_rank // 8 + 1, cap * n)"""),
+    "rsvd_no_power_iterations": ("""    for _ in range(power_iters):
+        Y = _orth(R @ _orth(R.T @ Y))""", """    for _ in range(0):
+        Y = _orth(R @ _orth(R.T @ Y))"""),
+    "rounds_ignore_compensator": ("""        T = lorc_target(W, U16, V16)""", """        T = lorc_target(W)"""),
+    "round_error_of_unrounded_pieces": ("""            E = R.astype(np.float64) - _f16(U16).astype(np.float64) @ _f16(V16).astype(np.float64)""",
+                                        """            E = R.astype(np.float64) - U @ V"""),
+    "kurtosis_over_m2": ("""    return float(np.mean(d ** 4)) / (m2 * m2) if m2 > 0 else 0.0""",
+                         """    return float(np.mean(d ** 4)) / m2 if m2 > 0 else 0.0"""),
+    "ranks_cap_not_refilled": ("""                left -= float(cap)
+                changed = True""", """                left -= float(cap)"""),
 }
 
 PINS = [getattr(m, n) for m in (lorc_pins, rank_pins) for n in sorted(dir(m))
