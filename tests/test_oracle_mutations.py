@@ -55,6 +55,10 @@ MUTANTS = {
     "codes_clamped_at_6": ("/* also maps NaN to 0 */\n                if (r > 7.0f) r = 7.0f;",
                            "/* also maps NaN to 0 */\n                if (r > 6.0f) r = 6.0f;"),
     "zero_point_unrounded": ("float z = h2f(z_h);", "float z = z_f;"),
+    "tile_pack_rows_j_and_j8_swapped": ("int q = i * 128 + ((r / 16) * 8 + r % 8) * 4 + ((r % 16) / 8) * 2;",
+                                        "int q = i * 128 + ((r / 16) * 8 + r % 8) * 4 + (1 - (r % 16) / 8) * 2;"),
+    "tile_pack_scale_zero_swapped": ("groups[q] = scale[(size_t)g * N + n];\n                    groups[q + 1] = zero[(size_t)g * N + n];",
+                                     "groups[q] = zero[(size_t)g * N + n];\n                    groups[q + 1] = scale[(size_t)g * N + n];"),
     "int3_compensator_scale_index_transposed": ("double s = milo_ref_h2d(sc[(size_t)j * R + p]);",
                                                 "double s = milo_ref_h2d(sc[(size_t)p * (Cc / group) + j]);"),
 }
