@@ -420,6 +420,79 @@ class QWeight:
                             MILO_LORC_INT3 if self.lorc_int3 else MILO_LORC_F16)
 
 
+# ---------------------------------------------------------------------------
+# saving packed experts (the quantiser is offline and slow; a saved layer
+# loads in seconds)
+# ---------------------------------------------------------------------------
+
+SAVE_FORMAT = 1
+
+
+def _qweight_shapes(qw: QWeight) -> dict:
+    """Expected host array shapes and dtypes of a projection's pieces."""
+    out = {"packed": ((milo_packed_bytes(qw.N, qw.K),), "uint8")}
+    if qw.rank and qw.lorc_int3:
+        out["U"] = ((milo_packed_bytes(qw.rank, qw.N),), "uint8")
+        out["V"] = ((milo_packed_bytes(qw.rank, qw.K),), "uint8")
+    elif qw.rank:
+        out["U"] = ((qw.N, qw.rank), "float16")
+        out["V"] = ((qw.rank, qw.K), "float16")
+    return out
+
+
+def save_experts(path, experts: list) -> None:
+    """Write packed experts (list of dict(w1=, w3=, w2=) QWeight, as
+    quantize_experts returns them) to an .npz file: each projection's blob,
+    its shape and rank, and its compensator (fp16 U and V, or their int3
+    blobs), copied to the host."""
+    import json
+
+    import numpy as np
+    arrays, meta = {}, []
+    for e, d in enumerate(experts):
+        for name, qw in d.items():
+            key = f"e{e}.{name}"
+            pieces = {"packed": qw.packed}
+            if qw.rank:
+                pieces.update(U=qw.U, V=qw.V)
+            for part, (shape, dt) in _qweight_shapes(qw).items():
+                a = pieces[part].detach().cpu().numpy()
+                if a.shape != shape or a.dtype != np.dtype(dt):
+                    raise ValueError(f"{key}.{part}: {a.dtype}{list(a.shape)}, expected {dt}{list(shape)}")
+                arrays[f"{key}.{part}"] = a
+            meta.append({"expert": e, "name": name, "N": qw.N, "K": qw.K, "rank": qw.rank,
+                         "lorc_int3": qw.lorc_int3})
+    arrays["meta"] = np.frombuffer(json.dumps({"format": SAVE_FORMAT, "projections": meta}).encode(), np.uint8)
+    np.savez(path, **arrays)
+
+
+def load_experts(path, device="cuda") -> list:
+    """The experts save_experts wrote, as QWeights on `device` (sizes checked
+    against the packed layout of milo.h)."""
+    import json
+
+    import numpy as np
+    with np.load(path, allow_pickle=False) as f:
+        meta = json.loads(bytes(f["meta"]).decode())
+        if meta.get("format") != SAVE_FORMAT:
+            raise ValueError(f"{path}: unknown format {meta.get('format')}")
+        experts = []
+        for m in meta["projections"]:
+            key = f"e{m['expert']}.{m['name']}"
+            probe = QWeight(None, m["N"], m["K"], rank=m["rank"], lorc_int3=m["lorc_int3"])
+            got = {}
+            for part, (shape, dt) in _qweight_shapes(probe).items():
+                a = f[f"{key}.{part}"]
+                if a.shape != shape or a.dtype != np.dtype(dt):
+                    raise ValueError(f"{path}: {key}.{part} is {a.dtype}{list(a.shape)}, expected {dt}{list(shape)}")
+                got[part] = torch.from_numpy(np.ascontiguousarray(a)).to(device)
+            while len(experts) <= m["expert"]:
+                experts.append({})
+            experts[m["expert"]][m["name"]] = QWeight(got["packed"], m["N"], m["K"], got.get("U"), got.get("V"),
+                                                      rank=m["rank"], lorc_int3=m["lorc_int3"])
+    return experts
+
+
 def _table(n_proj: int, device) -> torch.Tensor:
     nb = C.c_size_t()
     _check(lib().milo_table_bytes(n_proj, C.byref(nb)), "milo_table_bytes")
