@@ -486,19 +486,23 @@ def run_milo(args):
     barrier(dev)
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("milo/timed_steps")      # NVTX ranges name the regions for ncu --nvtx
     start.record(stream)
     for i in range(args.steps):
         run_step()
     stop.record(stream)
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     barrier(dev)
     ms_total = start.elapsed_time(stop)
     # --- timed region 2: the same K steps with events around the two grouped
     # GEMM launches, for their average launch durations (roofline)
+    torch.cuda.nvtx.range_push("milo/gemm_events")
     for i in range(args.steps):
         milo.milo_set_profile_events(ev[4 * i:4 * i + 4])
         step(x, logits)
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     milo.milo_set_profile_events(None)
     barrier(dev)
     # --- timed region 3 (graph replays only): the same K steps with an event
@@ -538,11 +542,13 @@ def step_spread(torch, run_step, steps: int, stream, dev) -> dict:
         e.record(stream)
     torch.cuda.synchronize()
     barrier(dev)
+    torch.cuda.nvtx.range_push("milo/step_spread")
     ev[0].record(stream)
     for i in range(steps):
         run_step()
         ev[i + 1].record(stream)
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     barrier(dev)
     d = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(steps))
     return {"median": max_over_ranks(nearest_rank(d, 0.5), dev), "p10": max_over_ranks(nearest_rank(d, 0.1), dev),
@@ -586,11 +592,13 @@ def run_e2e(args, torch, step, x, logits, y, out_dt, T, wk, dev, stream, world):
     torch.cuda.synchronize()
     barrier(dev)
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("milo/e2e_steps")
     s2.record(stream)
     for _ in range(args.steps):
         e2e_step()
     e2.record(stream)
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     e2e_ms = max_over_ranks(s2.elapsed_time(e2), dev)
     e2e_value = world * T * args.steps / (e2e_ms / 1e3)
     return e2e_value, e2e_ms
