@@ -6,7 +6,7 @@
 // weight plus a rank-r compensator, outputs mixed by the router weights):
 //   few rows per expert (mma.sync GEMMs):
 //     prep(x, row bookkeeping) -> gemv<SwiGLU>(w1|w3, t = x V1|V3^T inside)
-//        -> prep(h) -> gemv(w2, t = h V2^T inside, combine inside)
+//        -> prep(h) -> gemv(w2, t = h V2^T inside) -> combine
 //   many rows per expert (tcgen05 GEMMs):
 //     prep(x, row bookkeeping) -> lorc(x, V1|V3) -> tc<SwiGLU>(w1|w3)
 //        -> prep(h) -> lorc(h, V2) -> tc(w2) -> combine
