@@ -76,6 +76,10 @@ typedef enum {
 #define MILO_MAX_RANK 64            /* compensator rank, a multiple of 8 */
 #define MILO_MAX_EXPERTS 256        /* routed + shared */
 #define MILO_MAX_TOPK 16
+/* Rows of one call: T*k for milo_route and milo_grouped_linear, T*(top_k +
+ * n_shared) for milo_moe_forward.  Row indices and counts are 32-bit on the
+ * device; a call above this returns MILO_ERR_UNSUPPORTED_SHAPE. */
+#define MILO_MAX_ROWS 0x3FFFFFFF
 
 MILO_API const char* milo_status_str(milo_status s);
 /* Host string describing the last failure on the calling thread ("" if none). */
@@ -298,7 +302,8 @@ MILO_API milo_status milo_assign_ranks(const double* score, int32_t n, int32_t a
  *   perm        int32 [T*k]: the flat slots f = t*k + j of expert 0 in
  *               ascending order, then expert 1, ...
  *   inv_perm    int32 [T*k]: inv_perm[perm[p]] = p; -1 for a dropped slot
- * Limits: 1 <= E <= MILO_MAX_EXPERTS, 1 <= k <= min(E, MILO_MAX_TOPK), T >= 0.
+ * Limits: 1 <= E <= MILO_MAX_EXPERTS, 1 <= k <= min(E, MILO_MAX_TOPK), T >= 0,
+ * T*k <= MILO_MAX_ROWS (else UNSUPPORTED_SHAPE).
  * Device: BAD_EXPERT_ID (given ids outside [0, E); the slot is dropped),
  * NONFINITE (NaN/Inf logits; ids then unspecified).
  */
@@ -371,7 +376,9 @@ MILO_API milo_status milo_linear_prepare(milo_linear* lin, const milo_qweight* w
 MILO_API milo_status milo_layer_prepare(milo_moe_layer* layer, const milo_expert* experts,
                                void* device_table, size_t table_bytes);
 
-/* Workspace bytes for milo_grouped_linear / milo_moe_forward over T tokens.
+/* Workspace bytes for milo_grouped_linear / milo_moe_forward over T tokens
+ * (UNSUPPORTED_SHAPE when the call's rows exceed MILO_MAX_ROWS, or for a
+ * layer whose top_k or n_shared milo_layer_prepare would reject).
  * The size depends on which grouped GEMM the call takes (see
  * milo_set_gemm_path: the mma.sync kernel also keeps a plain fp16 copy of the
  * scaled rows and its counters in the workspace), so query it again after
@@ -398,6 +405,9 @@ MILO_API milo_status milo_moe_workspace_bytes(const milo_moe_layer* layer, int32
  *   y        [T*k, N] in y_dt (F32, F16 or BF16), row f = t*k + j; rows of
  *            dropped slots are written as zeros
  *   ws       >= milo_linear_workspace_bytes(lin, T, k), 256-byte aligned
+ * Errors: INVALID_ARG (NULL or misaligned pointers, bad T, k or dtype),
+ * UNSUPPORTED_SHAPE (T*k above MILO_MAX_ROWS, N not a multiple of 4),
+ * WORKSPACE (ws too small or misaligned).
  * Device: NONFINITE (NaN/Inf in x), FP16_RANGE (an fp16 output or the
  * compensator's fp16 t = x V^T overflows), TIMEOUT.
  */
@@ -419,6 +429,8 @@ MILO_API milo_status milo_grouped_linear(const milo_linear* lin, const void* x, 
  *            fp16 SwiGLU activations h [T*k + n_shared*T, inter] sit at byte
  *            offset milo_moe_h_offset(layer, T) of ws after the call, row p =
  *            expert-sorted slot p (shared-expert rows after the routed ones).
+ * Errors: INVALID_ARG (NULL or misaligned pointers, T < 0, bad dtype),
+ * UNSUPPORTED_SHAPE (T*(top_k + n_shared) above MILO_MAX_ROWS), WORKSPACE.
  * Device: NONFINITE, FP16_RANGE (h, t or an fp16 output overflows), TIMEOUT.
  */
 MILO_API milo_status milo_moe_forward(const milo_moe_layer* layer, const void* x, milo_dtype x_dt,
@@ -461,7 +473,8 @@ MILO_API milo_status milo_grouped_linear_noalloc(const milo_linear* lin, const v
                                                  const int32_t* perm, void* y, milo_dtype y_dt,
                                                  int32_t* dev_status, void* stream);
 
-/* Byte offset of h inside the forward workspace (see milo_moe_forward). */
+/* Byte offset of h inside the forward workspace (see milo_moe_forward); 0
+ * where milo_moe_workspace_bytes rejects the layer or T. */
 MILO_API size_t milo_moe_h_offset(const milo_moe_layer* layer, int32_t T);
 
 /*

@@ -245,6 +245,24 @@ static LorcPlan lorc_plan(int n_exp, int nproj, int K, long long max_rows) {
 static int t_slice_len(int) { return 512; }
 static int t_slices(int K) { return (K + t_slice_len(K) - 1) / t_slice_len(K); }
 
+// The rows of one call, counted in 64 bits before the 32-bit planning below:
+// T*k routed slots (grouped linear), plus n_shared*T shared-expert rows (MoE
+// layer).  A call above MILO_MAX_ROWS, or a layer with a top_k or n_shared
+// that its preparation rejects, is refused before anything is planned.
+static milo_status check_linear_rows(int T, int k, const char* what) {
+    if (static_cast<long long>(T) * k > MILO_MAX_ROWS)
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": T*k above MILO_MAX_ROWS");
+    return MILO_OK;
+}
+
+static milo_status check_moe_rows(const milo_moe_layer* L, int T, const char* what) {
+    if (L->top_k < 1 || L->top_k > MILO_MAX_TOPK || L->n_shared < 0 || L->n_shared > MILO_MAX_EXPERTS)
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": top_k or n_shared out of range");
+    if (static_cast<long long>(T) * (L->top_k + L->n_shared) > MILO_MAX_ROWS)
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": T*(top_k + n_shared) above MILO_MAX_ROWS");
+    return MILO_OK;
+}
+
 static LinearWs linear_ws(const milo_linear* lin, int T, int k) {
     LinearWs w;
     Carve c;
@@ -514,6 +532,8 @@ extern "C" milo_status milo_linear_workspace_bytes(const milo_linear* lin, int32
                                                    size_t* bytes) {
     clear_error();
     if (!lin || !bytes || T < 0 || k < 1) return fail(MILO_ERR_INVALID_ARG, "milo_linear_workspace_bytes");
+    const milo_status s = check_linear_rows(T, k, "milo_linear_workspace_bytes");
+    if (s != MILO_OK) return s;
     *bytes = linear_ws(lin, T, k).total;
     return MILO_OK;
 }
@@ -521,12 +541,15 @@ extern "C" milo_status milo_linear_workspace_bytes(const milo_linear* lin, int32
 extern "C" milo_status milo_moe_workspace_bytes(const milo_moe_layer* L, int32_t T, size_t* bytes) {
     clear_error();
     if (!L || !bytes || T < 0) return fail(MILO_ERR_INVALID_ARG, "milo_moe_workspace_bytes");
+    const milo_status s = check_moe_rows(L, T, "milo_moe_workspace_bytes");
+    if (s != MILO_OK) return s;
     *bytes = moe_ws(L, T).total;
     return MILO_OK;
 }
 
 extern "C" size_t milo_moe_h_offset(const milo_moe_layer* L, int32_t T) {
-    return L ? moe_ws(L, T).h : 0;
+    if (!L || T < 0 || check_moe_rows(L, T, "milo_moe_h_offset") != MILO_OK) return 0;
+    return moe_ws(L, T).h;
 }
 
 extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x, milo_dtype x_dt,
@@ -536,6 +559,7 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
     clear_error();
     if (!lin || !lin->table) return fail(MILO_ERR_INVALID_ARG, "milo_grouped_linear: layer not prepared");
     if (T < 0 || k < 1 || k > MILO_MAX_TOPK) return fail(MILO_ERR_INVALID_ARG, "milo_grouped_linear: bad T or k");
+    if (check_linear_rows(T, k, "milo_grouped_linear") != MILO_OK) return MILO_ERR_UNSUPPORTED_SHAPE;
     if (x_dt != MILO_F16 && x_dt != MILO_BF16) return fail(MILO_ERR_INVALID_ARG, "x must be fp16 or bf16");
     if (y_dt != MILO_F16 && y_dt != MILO_BF16 && y_dt != MILO_F32) return fail(MILO_ERR_INVALID_ARG, "bad y dtype");
     if (!perm && k != 1) return fail(MILO_ERR_INVALID_ARG, "perm may be NULL only with k == 1");
@@ -648,6 +672,7 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
     clear_error();
     if (!L || !L->table) return fail(MILO_ERR_INVALID_ARG, "milo_moe_forward: layer not prepared");
     if (T < 0) return fail(MILO_ERR_INVALID_ARG, "milo_moe_forward: T must be >= 0");
+    if (check_moe_rows(L, T, "milo_moe_forward") != MILO_OK) return MILO_ERR_UNSUPPORTED_SHAPE;
     if (x_dt != MILO_F16 && x_dt != MILO_BF16) return fail(MILO_ERR_INVALID_ARG, "x must be fp16 or bf16");
     if (y_dt != MILO_F16 && y_dt != MILO_BF16 && y_dt != MILO_F32) return fail(MILO_ERR_INVALID_ARG, "bad y dtype");
     if (T == 0) return MILO_OK;

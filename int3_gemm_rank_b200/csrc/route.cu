@@ -214,8 +214,8 @@ extern "C" milo_status milo_route(const uint16_t* logits, int32_t T, int32_t E, 
         return fail(MILO_ERR_INVALID_ARG, "milo_route: NULL output");
     if (!(flags & MILO_ROUTE_IDS_GIVEN) && T > 0 && (!logits || !topk_w))
         return fail(MILO_ERR_INVALID_ARG, "milo_route: logits and topk_w are required");
-    if (static_cast<long long>(T) * k > 0x3FFFFFFFLL)
-        return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_route: T*k too large");
+    if (static_cast<long long>(T) * k > MILO_MAX_ROWS)
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_route: T*k above MILO_MAX_ROWS");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool want_topk = !(flags & MILO_ROUTE_IDS_GIVEN) && T > 0;
     const bool split = want_topk && T >= kRouteSplitT;

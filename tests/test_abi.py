@@ -105,6 +105,56 @@ def test_workspace_sizes_grow_with_tokens(milo):
     assert L.milo_moe_h_offset(C.byref(layer), 16) % 256 == 0
 
 
+MAX_ROWS = 0x3FFFFFFF   # MILO_MAX_ROWS
+
+
+def test_header_states_the_row_limit():
+    src = open(os.path.join(ROOT, "include", "milo.h")).read()
+    assert re.search(r"#define MILO_MAX_ROWS 0x3FFFFFFF\b", src)
+
+
+def test_calls_above_the_row_limit_are_refused_before_planning(milo):
+    """T*k (grouped linear, router) or T*(top_k + n_shared) (MoE layer) above
+    the row limit: the size queries and the calls refuse the shape instead of
+    sizing a workspace from a wrapped 32-bit row count.  Every call here
+    returns before any CUDA call, so no device is needed."""
+    L = milo.lib()
+    nb = C.c_size_t(123)
+    lin = milo.milo_linear(4096, 4096, 8, 64, 0, None)
+    # at the limit the query succeeds; one token more (k = 2) does not
+    assert L.milo_linear_workspace_bytes(C.byref(lin), MAX_ROWS // 2, 2, C.byref(nb)) == 0 and nb.value > 0
+    assert L.milo_linear_workspace_bytes(C.byref(lin), MAX_ROWS // 2 + 1, 2, C.byref(nb)) == \
+        milo.MILO_ERR_UNSUPPORTED_SHAPE
+    assert b"MILO_MAX_ROWS" in L.milo_last_error()
+    # T * k wraps a signed 32-bit count: 2^31 - 1 tokens, k = 16
+    assert L.milo_linear_workspace_bytes(C.byref(lin), 0x7FFFFFFF, 16, C.byref(nb)) == \
+        milo.MILO_ERR_UNSUPPORTED_SHAPE
+    fake = C.c_void_p(0x10000)
+    lin.table = fake
+    assert L.milo_grouped_linear(C.byref(lin), fake, milo.MILO_F16, 0x7FFFFFFF, 16, fake, fake, fake,
+                                 milo.MILO_F32, fake, 1 << 40, None, None) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    assert L.milo_grouped_linear_noalloc(C.byref(lin), fake, milo.MILO_F16, 0x7FFFFFFF, 16, fake, fake, fake,
+                                         milo.MILO_F32, None, None) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    # MoE layer: the shared experts' rows count too
+    layer = milo.milo_moe_layer(2048, 1408, 64, 2, 6, 64, 0, None)
+    t_max = MAX_ROWS // 8
+    assert L.milo_moe_workspace_bytes(C.byref(layer), t_max, C.byref(nb)) == 0 and nb.value > 0
+    assert L.milo_moe_h_offset(C.byref(layer), t_max) > 0
+    assert L.milo_moe_workspace_bytes(C.byref(layer), t_max + 1, C.byref(nb)) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    assert L.milo_moe_h_offset(C.byref(layer), t_max + 1) == 0
+    layer.table = fake
+    assert L.milo_moe_forward(C.byref(layer), fake, milo.MILO_BF16, 0x7FFFFFFF, fake, fake, fake, fake, fake,
+                              milo.MILO_F32, fake, 1 << 40, None, None) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    # a layer struct whose top_k or n_shared preparation would reject
+    bad = milo.milo_moe_layer(2048, 1408, 64, -1, 6, 64, 0, None)
+    assert L.milo_moe_workspace_bytes(C.byref(bad), 16, C.byref(nb)) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    bad = milo.milo_moe_layer(2048, 1408, 64, 0, 0, 64, 0, None)
+    assert L.milo_moe_workspace_bytes(C.byref(bad), 16, C.byref(nb)) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    # the router keeps the same limit
+    assert L.milo_route(fake, 0x7FFFFFFF, 8, 2, 0, fake, fake, fake, fake, fake, None, None) == \
+        milo.MILO_ERR_UNSUPPORTED_SHAPE
+
+
 def test_quantiser_validation_and_workspace(milo):
     L = milo.lib()
     fake = C.c_void_p(0x1000)

@@ -132,7 +132,7 @@ def test_quantize_lorc_rounds_track_the_oracle(milo):
     ref = oracle.quantize_lorc(W, r, rounds, om)
     assert err.shape == (rounds + 1,)
     # Rounds 0 and 1 quantise the same targets on both sides (W, then W minus a
-    # compensator that agrees to fp16 rounding); from round 2 on, a code decided
+    # compensator that agrees to fp16 rounding); from refinement round 2 on, a code decided
     # differently near a rounding boundary moves its group's zero-point fit, so
     # the two runs agree only statistically.
     assert np.all(np.abs(err[:2] - ref["err"][:2]) <= ERR_TOL * ref["err"][:2])
