@@ -111,6 +111,8 @@ MILO_API int32_t milo_version(void);
  * codes, scales and zeros -- with one copy.
  * Dequantisation: w_hat[n, k] = (q[n, k] - z[n, k/64]) * s[n, k/64].
  * The blob has ceil(N/64) * (K/128) * 3584 bytes (milo_packed_bytes).
+ * N is at most 2^31 - 64, so that the padded row count stays a 32-bit
+ * integer (UNSUPPORTED_SHAPE above).
  */
 
 /* Bytes of the packed blob of a weight [N, K] (K % 128 == 0). */

@@ -122,6 +122,7 @@ static milo_status fill_proj(ProjDev* d, const milo_qweight& w, int N, int K, co
 
 static milo_status check_nk(int N, int K, const char* what) {
     if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": sizes must be positive");
+    if (N > kMaxWeightRows) return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": N above 2^31 - 64");
     if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": K must be a multiple of 128");
     if (N % 16) return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": N must be a multiple of 16");
     return MILO_OK;

@@ -38,6 +38,10 @@ inline milo_status check_cuda(cudaError_t e, const char* what) {
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Weight rows whose count padded to whole 64-row tiles (the blob's layout)
+// still fits the 32-bit row counts of the kernels.
+constexpr int32_t kMaxWeightRows = 0x7FFFFFFF - 63;
+
 // Launch with programmatic stream serialization (see grid_dep_wait in
 // milo_device.cuh): the kernel may be scheduled while the previous kernel of
 // the stream drains.

@@ -166,6 +166,7 @@ extern "C" milo_status milo_pack(const uint16_t* W, int32_t N, int32_t K, int32_
                                  int32_t* dev_status, void* stream) {
     clear_error();
     if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, "milo_pack: N and K must be positive");
+    if (N > kMaxWeightRows) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_pack: N above 2^31 - 64");
     if (group != MILO_GROUP) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_pack: group must be 64");
     if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_pack: K must be a multiple of 128");
     if (!W || !packed) return fail(MILO_ERR_INVALID_ARG, "milo_pack: NULL pointer");
@@ -184,6 +185,7 @@ extern "C" milo_status milo_unpack(const void* packed, int32_t N, int32_t K, uin
     clear_error();
     if (!packed || !codes) return fail(MILO_ERR_INVALID_ARG, "milo_unpack: NULL pointer");
     if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, "milo_unpack: N and K must be positive");
+    if (N > kMaxWeightRows) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_unpack: N above 2^31 - 64");
     if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_unpack: K must be a multiple of 128");
     if (!aligned(packed, 4)) return fail(MILO_ERR_INVALID_ARG, "milo_unpack: the packed buffer must be 4-byte aligned");
     const long long threads = static_cast<long long>(N) * (K / 128) * 4;
@@ -198,6 +200,7 @@ extern "C" milo_status milo_unpack(const void* packed, int32_t N, int32_t K, uin
 extern "C" milo_status milo_packed_bytes(int32_t N, int32_t K, size_t* bytes) {
     clear_error();
     if (N <= 0 || K <= 0 || !bytes) return fail(MILO_ERR_INVALID_ARG, "milo_packed_bytes: bad argument");
+    if (N > kMaxWeightRows) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_packed_bytes: N above 2^31 - 64");
     if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_packed_bytes: K must be a multiple of 128");
     *bytes = static_cast<size_t>((N + 63) / 64) * (K / 128) * kBlockSB;
     return MILO_OK;
@@ -207,6 +210,7 @@ extern "C" milo_status milo_dequantize(const void* packed, int32_t N, int32_t K,
     clear_error();
     if (!packed || !W_hat) return fail(MILO_ERR_INVALID_ARG, "milo_dequantize: NULL pointer");
     if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, "milo_dequantize: N and K must be positive");
+    if (N > kMaxWeightRows) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_dequantize: N above 2^31 - 64");
     if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "milo_dequantize: K must be a multiple of 128");
     if (!aligned(packed, 16) || !aligned(W_hat, 16))
         return fail(MILO_ERR_INVALID_ARG, "milo_dequantize: pointers must be 16-byte aligned");

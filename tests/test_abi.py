@@ -155,6 +155,29 @@ def test_calls_above_the_row_limit_are_refused_before_planning(milo):
         milo.MILO_ERR_UNSUPPORTED_SHAPE
 
 
+def test_weight_rows_bounded_so_the_tile_padding_fits_32_bits(milo):
+    """A weight of N rows is stored in 64-row tiles; N up to 2^31 - 64 pads to
+    a 32-bit count, and above it pack, unpack, dequantise, the size query and
+    preparation refuse the shape (no device needed: all return before a
+    launch)."""
+    L = milo.lib()
+    nb = C.c_size_t()
+    n_max = 0x7FFFFFFF - 63
+    assert L.milo_packed_bytes(n_max, 128, C.byref(nb)) == 0
+    assert nb.value == (n_max // 64) * 3584
+    for n in (n_max + 1, 0x7FFFFFFF):
+        assert L.milo_packed_bytes(n, 128, C.byref(nb)) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+        assert b"2^31 - 64" in L.milo_last_error()
+    fake = C.c_void_p(0x1000)
+    assert L.milo_pack(fake, 0x7FFFFFFF, 128, 64, fake, None, None) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    assert L.milo_unpack(fake, 0x7FFFFFFF, 128, fake, None) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    assert L.milo_dequantize(fake, 0x7FFFFFFF, 128, fake, None) == milo.MILO_ERR_UNSUPPORTED_SHAPE
+    w = milo.milo_qweight(0x10000, None, None, 0, 0)
+    lin = milo.milo_linear(0x7FFFFFF0, 128, 1, 64, 0, None)   # a multiple of 16 above the bound
+    assert L.milo_linear_prepare(C.byref(lin), C.byref(w), C.c_void_p(0x10000), 1 << 20) == \
+        milo.MILO_ERR_UNSUPPORTED_SHAPE
+
+
 def test_quantiser_validation_and_workspace(milo):
     L = milo.lib()
     fake = C.c_void_p(0x1000)
