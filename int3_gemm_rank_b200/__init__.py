@@ -161,6 +161,57 @@ def _cuda(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
 
 
+_ACT = (torch.float16, torch.bfloat16)               # activations x
+_OUT = (torch.float16, torch.bfloat16, torch.float32)  # outputs y
+
+
+def _dname(d) -> str:
+    return str(d).replace("torch.", "")
+
+
+def _arg(t, name: str, dtypes=None, shape=None, min_numel: int | None = None, device=None):
+    """Check a tensor before its pointer crosses the C ABI.  The library reads
+    and writes through the raw pointer with the sizes the call states, so a
+    tensor of another dtype or size would be read or written out of bounds.
+    dtype and size are checked first (they need no device), then contiguity,
+    then that the tensor is a CUDA tensor on the call's device."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, not {type(t).__name__}")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name} must be {' or '.join(_dname(d) for d in dtypes)}, not {_dname(t.dtype)}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name} must hold at least {min_numel} elements, not {t.numel()}")
+    _cuda(t, name)
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}; the call's other tensors are on {device}")
+
+
+def _rows_arg(x, name: str, width: int):
+    """Activation rows [T, width] in fp16 or bf16; returns their device."""
+    if not isinstance(x, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, not {type(x).__name__}")
+    if x.dim() != 2 or x.shape[1] != width:
+        raise ValueError(f"{name} must be [T, {width}], not {tuple(x.shape)}")
+    _arg(x, name, _ACT)
+    return x.device
+
+
+def _status_arg(dev_status, device):
+    if dev_status is not None:
+        _arg(dev_status, "dev_status", (torch.int32,), min_numel=1, device=device)
+
+
+def _ws_arg(ws, device) -> tuple:
+    """The 256-byte-aligned start of a caller's workspace and the bytes from
+    there to its end (0 when the buffer ends before that boundary)."""
+    _arg(ws, "ws", device=device)
+    start = ws.data_ptr()
+    off = (-start) % 256
+    return start + off, max(0, ws.numel() * ws.element_size() - off)
+
+
 def milo_set_profile_events(events: list | None):
     """Record torch.cuda.Event objects around the grouped GEMM launches (None disables)."""
     if not events:
@@ -204,17 +255,23 @@ def milo_pack(W: torch.Tensor, group: int = MILO_GROUP, dev_status: torch.Tensor
 
 def milo_dequantize(packed: torch.Tensor, N: int, K: int, out: torch.Tensor | None = None) -> torch.Tensor:
     """fp16 [N, K] dequantised weights (q - z) s of a packed blob."""
-    _cuda(packed, "packed")
-    W = torch.empty((N, K), dtype=torch.float16, device=packed.device) if out is None else out
-    _check(lib().milo_dequantize(_ptr(packed), N, K, _ptr(W), _stream()), "milo_dequantize")
+    _arg(packed, "packed", (torch.uint8,), min_numel=milo_packed_bytes(N, K))
+    if out is None:
+        W = torch.empty((N, K), dtype=torch.float16, device=packed.device)
+    else:
+        _arg(out, "out", (torch.float16,), shape=(N, K), device=packed.device)
+        W = out
+    with torch.cuda.device(packed.device):
+        _check(lib().milo_dequantize(_ptr(packed), N, K, _ptr(W), _stream()), "milo_dequantize")
     return W
 
 
 def milo_unpack(packed: torch.Tensor, N: int, K: int) -> torch.Tensor:
     """Codes u8 [N, K] of a packed blob."""
-    _cuda(packed, "packed")
+    _arg(packed, "packed", (torch.uint8,), min_numel=milo_packed_bytes(N, K))
     codes = torch.empty((N, K), dtype=torch.uint8, device=packed.device)
-    _check(lib().milo_unpack(_ptr(packed), N, K, _ptr(codes), _stream()), "milo_unpack")
+    with torch.cuda.device(packed.device):
+        _check(lib().milo_unpack(_ptr(packed), N, K, _ptr(codes), _stream()), "milo_unpack")
     return codes
 
 
@@ -360,28 +417,40 @@ def milo_route(logits: torch.Tensor | None, k: int, renorm: bool, E: int | None 
     flags = MILO_ROUTE_RENORM if renorm else 0
     if ids is not None:
         flags |= MILO_ROUTE_IDS_GIVEN
-        _cuda(ids, "ids")
+        if E is None:
+            raise ValueError("milo_route: E (the number of experts) is required when ids are given")
+        if not isinstance(ids, torch.Tensor) or ids.dim() != 2 or ids.shape[1] != k:
+            raise ValueError(f"milo_route: ids must be [T, {k}]")
+        _arg(ids, "ids", (torch.int32,))
         T = ids.shape[0]
         dev = ids.device
         w = None
     else:
-        _cuda(logits, "logits")
+        if not isinstance(logits, torch.Tensor) or logits.dim() != 2:
+            raise ValueError("milo_route: logits must be a [T, E] tensor")
+        _arg(logits, "logits", (torch.float16,))
         T, E = logits.shape
         dev = logits.device
+        if out:
+            _arg(out["ids"], "out['ids']", (torch.int32,), shape=(T, k), device=dev)
+            _arg(out["w"], "out['w']", (torch.float32,), shape=(T, k), device=dev)
         ids = out["ids"] if out else torch.empty((T, k), dtype=torch.int32, device=dev)
         w = out["w"] if out else torch.empty((T, k), dtype=torch.float32, device=dev)
+    _status_arg(dev_status, dev)
     if out:
         for name, t, n in (("offsets", out["offsets"], E + 1), ("perm", out["perm"], T * k),
                            ("inv_perm", out["inv_perm"], T * k)):
             if t.dtype != torch.int32 or not t.is_contiguous() or t.numel() < n:
                 raise MiloError(MILO_ERR_INVALID_ARG, f"milo_route: out[{name!r}] must be int32[{n}]")
+            _arg(t, f"out[{name!r}]", device=dev)
         off, perm, inv = out["offsets"], out["perm"], out["inv_perm"]
     else:
         off = torch.empty(E + 1, dtype=torch.int32, device=dev)
         perm = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
         inv = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
-    _check(lib().milo_route(_ptr(logits), T, E, k, flags, _ptr(ids), _ptr(w), _ptr(off), _ptr(perm),
-                            _ptr(inv), _ptr(dev_status), _stream()), "milo_route")
+    with torch.cuda.device(dev):
+        _check(lib().milo_route(_ptr(logits), T, E, k, flags, _ptr(ids), _ptr(w), _ptr(off), _ptr(perm),
+                                _ptr(inv), _ptr(dev_status), _stream()), "milo_route")
     return {"ids": ids, "w": w, "offsets": off, "perm": perm[:T * k], "inv_perm": inv[:T * k]}
 
 
@@ -414,7 +483,26 @@ class QWeight:
                        milo_pack(V, dev_status=dev_status), rank=r, lorc_int3=True)
         return cls(packed, W.shape[0], W.shape[1], U, V)
 
+    def check(self):
+        """Checks the pieces' dtypes and sizes against N, K and the rank before
+        their pointers go into a layer table: the kernels read each piece
+        with the sizes the shape implies.  Int3 factors need N and K to be
+        multiples of 128 (the packed format's rows); milo_packed_bytes
+        refuses other sizes with UNSUPPORTED_SHAPE."""
+        _arg(self.packed, "packed", (torch.uint8,), min_numel=milo_packed_bytes(self.N, self.K))
+        dev = self.packed.device
+        if not self.rank:
+            return
+        if self.lorc_int3:
+            nu, nv = milo_packed_bytes(self.rank, self.N), milo_packed_bytes(self.rank, self.K)
+            _arg(self.U, "U (int3 blob of U^T)", (torch.uint8,), min_numel=nu, device=dev)
+            _arg(self.V, "V (int3 blob)", (torch.uint8,), min_numel=nv, device=dev)
+        else:
+            _arg(self.U, "U", (torch.float16,), shape=(self.N, self.rank), device=dev)
+            _arg(self.V, "V", (torch.float16,), shape=(self.rank, self.K), device=dev)
+
     def cstruct(self) -> milo_qweight:
+        self.check()
         return milo_qweight(self.packed.data_ptr(), self.U.data_ptr() if self.rank else None,
                             self.V.data_ptr() if self.rank else None, self.rank,
                             MILO_LORC_INT3 if self.lorc_int3 else MILO_LORC_F16)
@@ -533,18 +621,33 @@ class GroupedLinear:
         return milo_grouped_linear(self, x, offsets, perm, k, out_dtype, dev_status, y, ws)
 
 
+def _linear_args(lin: GroupedLinear, x, offsets, perm, k, out_dtype, dev_status, y):
+    """Checks the tensors of a grouped-linear call against the projection's
+    shape; returns (T, device, y)."""
+    dev = _rows_arg(x, "x", lin.cs.K)
+    T = x.shape[0]
+    if T > 0:
+        _arg(offsets, "offsets", (torch.int32,), min_numel=lin.cs.n_experts + 1, device=dev)
+        if perm is not None:
+            _arg(perm, "perm", (torch.int32,), min_numel=T * k, device=dev)
+    if y is None:
+        y = torch.empty((T * k, lin.cs.N), dtype=out_dtype, device=dev)
+    else:
+        _arg(y, "y", _OUT, shape=(T * k, lin.cs.N), device=dev)
+    _status_arg(dev_status, dev)
+    return T, dev, y
+
+
 def milo_grouped_linear(lin: GroupedLinear, x, offsets, perm, k=1, out_dtype=torch.float32,
                         dev_status=None, y=None, ws=None) -> torch.Tensor:
-    _cuda(x, "x")
-    T = x.shape[0]
-    if y is None:
-        y = torch.empty((T * k, lin.cs.N), dtype=out_dtype, device=x.device)
+    T, dev, y = _linear_args(lin, x, offsets, perm, k, out_dtype, dev_status, y)
     if ws is None:
-        ws = lin.workspace(T, k, x.device)
-    wp, wn = _aligned_view(ws, 256, ws.numel() - 256)
-    _check(lib().milo_grouped_linear(C.byref(lin.cs), _ptr(x), _dt(x), T, k, _ptr(offsets), _ptr(perm),
-                                     _ptr(y), _dt(y), C.c_void_p(wp), wn, _ptr(dev_status), _stream()),
-           "milo_grouped_linear")
+        ws = lin.workspace(T, k, dev)
+    wp, wn = _ws_arg(ws, dev)
+    with torch.cuda.device(dev):
+        _check(lib().milo_grouped_linear(C.byref(lin.cs), _ptr(x), _dt(x), T, k, _ptr(offsets), _ptr(perm),
+                                         _ptr(y), _dt(y), C.c_void_p(wp), wn, _ptr(dev_status), _stream()),
+               "milo_grouped_linear")
     return y
 
 
@@ -552,13 +655,11 @@ def milo_grouped_linear_noalloc(lin: GroupedLinear, x, offsets, perm, k=1, out_d
                                 dev_status=None, y=None) -> torch.Tensor:
     """milo_grouped_linear without a workspace argument: for callers that cannot
     allocate device memory; the scratch is the library's built-in buffer."""
-    _cuda(x, "x")
-    T = x.shape[0]
-    if y is None:
-        y = torch.empty((T * k, lin.cs.N), dtype=out_dtype, device=x.device)
-    _check(lib().milo_grouped_linear_noalloc(C.byref(lin.cs), _ptr(x), _dt(x), T, k, _ptr(offsets),
-                                             _ptr(perm), _ptr(y), _dt(y), _ptr(dev_status), _stream()),
-           "milo_grouped_linear_noalloc")
+    T, dev, y = _linear_args(lin, x, offsets, perm, k, out_dtype, dev_status, y)
+    with torch.cuda.device(dev):
+        _check(lib().milo_grouped_linear_noalloc(C.byref(lin.cs), _ptr(x), _dt(x), T, k, _ptr(offsets),
+                                                 _ptr(perm), _ptr(y), _dt(y), _ptr(dev_status), _stream()),
+               "milo_grouped_linear_noalloc")
     return y
 
 
@@ -602,15 +703,28 @@ class MoELayer:
 
 def milo_moe_forward(layer: MoELayer, x, route: dict, out_dtype=torch.float32, dev_status=None,
                      y=None, ws=None) -> torch.Tensor:
-    _cuda(x, "x")
+    dev = _rows_arg(x, "x", layer.cs.hidden)
     T = x.shape[0]
+    Tk = T * layer.cs.top_k
+    if T > 0:
+        # milo_route's outputs over the routed experts (k = top_k)
+        for key, dt, n in (("w", torch.float32, Tk), ("offsets", torch.int32, layer.cs.n_routed + 1),
+                           ("perm", torch.int32, Tk), ("inv_perm", torch.int32, Tk)):
+            if route.get(key) is None:
+                raise ValueError(f"route[{key!r}] is required")
+            _arg(route[key], f"route[{key!r}]", (dt,), min_numel=n, device=dev)
     if y is None:
-        y = torch.empty((T, layer.cs.hidden), dtype=out_dtype, device=x.device)
+        y = torch.empty((T, layer.cs.hidden), dtype=out_dtype, device=dev)
+    else:
+        _arg(y, "y", _OUT, shape=(T, layer.cs.hidden), device=dev)
+    _status_arg(dev_status, dev)
     if ws is None:
-        ws = layer.workspace(T, x.device)
-    wp, wn = _aligned_view(ws, 256, ws.numel() - 256)
-    _check(lib().milo_moe_forward(C.byref(layer.cs), _ptr(x), _dt(x), T, _ptr(route["w"]),
-                                  _ptr(route["offsets"]), _ptr(route["perm"]), _ptr(route["inv_perm"]),
-                                  _ptr(y), _dt(y), C.c_void_p(wp), wn, _ptr(dev_status), _stream()),
-           "milo_moe_forward")
+        ws = layer.workspace(T, dev)
+    wp, wn = _ws_arg(ws, dev)
+    with torch.cuda.device(dev):
+        _check(lib().milo_moe_forward(C.byref(layer.cs), _ptr(x), _dt(x), T, _ptr(route.get("w")),
+                                      _ptr(route.get("offsets")), _ptr(route.get("perm")),
+                                      _ptr(route.get("inv_perm")), _ptr(y), _dt(y), C.c_void_p(wp), wn,
+                                      _ptr(dev_status), _stream()),
+               "milo_moe_forward")
     return y
