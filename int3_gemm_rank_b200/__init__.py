@@ -198,6 +198,14 @@ def _rows_arg(x, name: str, width: int):
     return x.device
 
 
+def _weight_arg(W):
+    """A weight matrix W [N, K] in fp16 (the quantiser and packer read N*K
+    halves)."""
+    if not isinstance(W, torch.Tensor) or W.dim() != 2:
+        raise ValueError("W must be a [N, K] tensor")
+    _arg(W, "W", (torch.float16,))
+
+
 def _status_arg(dev_status, device):
     if dev_status is not None:
         _arg(dev_status, "dev_status", (torch.int32,), min_numel=1, device=device)
@@ -245,8 +253,9 @@ def milo_packed_bytes(N: int, K: int) -> int:
 
 def milo_pack(W: torch.Tensor, group: int = MILO_GROUP, dev_status: torch.Tensor | None = None):
     """Quantise W fp16 [N, K] to int3 and pack it: the device blob (uint8 tensor) of milo.h."""
-    _cuda(W, "W")
+    _weight_arg(W)
     N, K = W.shape
+    _status_arg(dev_status, W.device)
     nbytes = milo_packed_bytes(N, K) if K > 0 and K % 128 == 0 and N > 0 else 16
     blob = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
     _check(lib().milo_pack(_ptr(W), N, K, group, _ptr(blob), _ptr(dev_status), _stream()), "milo_pack")
@@ -287,12 +296,15 @@ def milo_hqq_pack(W: torch.Tensor, U: torch.Tensor | None = None, V: torch.Tenso
                   residual: bool = False, dev_status: torch.Tensor | None = None):
     """HQQ-quantise W - U V (fp16 W [N, K], U [N, r], V [r, K]) and pack it.
     Returns (blob uint8, residual f32 [N, K] = W - W_hat, or None)."""
-    _cuda(W, "W")
+    _weight_arg(W)
     N, K = W.shape
-    r = 0 if U is None else U.shape[1]
-    for t, name in ((U, "U"), (V, "V")):
-        if t is not None:
-            _cuda(t, name)
+    if (U is None) != (V is None):
+        raise ValueError("milo_hqq_pack: give both U and V, or neither")
+    r = 0 if U is None or U.dim() != 2 else U.shape[1]
+    if U is not None:
+        _arg(U, "U", (torch.float16,), shape=(N, r), device=W.device)
+        _arg(V, "V", (torch.float16,), shape=(r, K), device=W.device)
+    _status_arg(dev_status, W.device)
     nbytes = milo_packed_bytes(N, K) if K > 0 and K % 128 == 0 and N > 0 else 16
     blob = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
     R = torch.empty((N, K), dtype=torch.float32, device=W.device) if residual else None
@@ -320,8 +332,9 @@ def milo_quantize_lorc(W: torch.Tensor, params: milo_lorc_params, omega: torch.T
     the residual, and params.rounds refinement rounds.  omega: f32 [K, sketch],
     the random test matrix.  Returns (QWeight with fp16 U, V of the best round,
     per-round errors f32 [rounds + 1])."""
-    _cuda(W, "W")
+    _weight_arg(W)
     N, K = W.shape
+    _status_arg(dev_status, W.device)
     r = params.rank
     if r > 0:
         if omega is None or omega.dtype != torch.float32 or tuple(omega.shape) != (K, params.sketch):

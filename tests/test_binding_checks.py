@@ -179,3 +179,26 @@ def test_qweight_pieces_checked_before_the_table_is_written(no_device_check):
     with pytest.raises(milo.MiloError) as e:
         milo.QWeight(blob192, 192, K, U, V, rank=r, lorc_int3=True).check()
     assert e.value.status == milo.MILO_ERR_UNSUPPORTED_SHAPE
+
+
+def test_packers_and_quantiser_need_fp16_weights_and_matching_factors(no_device_check):
+    milo = no_device_check
+    W = torch.zeros((128, 256), dtype=torch.float16)
+    for bad in (torch.zeros((128, 256), dtype=torch.uint8), torch.zeros((128, 256), dtype=torch.bfloat16)):
+        with pytest.raises(ValueError, match="float16"):
+            milo.milo_pack(bad)
+        with pytest.raises(ValueError, match="float16"):
+            milo.milo_hqq_pack(bad)
+        with pytest.raises(ValueError, match="float16"):
+            milo.milo_quantize_lorc(bad, milo.lorc_params(0))
+    with pytest.raises(ValueError, match=r"\[N, K\]"):
+        milo.milo_pack(torch.zeros(256, dtype=torch.float16))
+    U, V = torch.zeros((128, 8), dtype=torch.float16), torch.zeros((8, 256), dtype=torch.float16)
+    with pytest.raises(ValueError, match="both"):
+        milo.milo_hqq_pack(W, U, None)
+    with pytest.raises(ValueError, match=r"V must have shape \(8, 256\)"):
+        milo.milo_hqq_pack(W, U, V[:, :128])
+    with pytest.raises(ValueError, match=r"U must have shape \(128, 8\)"):
+        milo.milo_hqq_pack(W, U[:64], V)
+    with pytest.raises(ValueError, match="dev_status"):
+        milo.milo_pack(W, dev_status=torch.zeros(1, dtype=torch.float32))
