@@ -549,6 +549,7 @@ extern "C" milo_status milo_moe_workspace_bytes(const milo_moe_layer* L, int32_t
 }
 
 extern "C" size_t milo_moe_h_offset(const milo_moe_layer* L, int32_t T) {
+    clear_error();
     if (!L || T < 0 || check_moe_rows(L, T, "milo_moe_h_offset") != MILO_OK) return 0;
     return moe_ws(L, T).h;
 }
