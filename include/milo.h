@@ -368,8 +368,9 @@ MILO_API milo_status milo_table_bytes(int32_t n_projections, size_t* bytes);
  * tensor map holds V's).  One-time set-up: the table is copied with a
  * synchronous cudaMemcpy.  lin/layer are host structs; the caller fills the
  * shape fields and the call sets max_rank and table.
- * Errors: UNSUPPORTED_SHAPE (K % 128, N % 16, group != 64, rank not a multiple
- * of 8 or above MILO_MAX_RANK), WORKSPACE (table too small or not 64-byte
+ * Errors: UNSUPPORTED_SHAPE (K % 128, N % 16, K above 2^24, group != 64,
+ * rank not a multiple of 8 or above MILO_MAX_RANK, n_experts outside 1..256,
+ * top_k outside 1..min(n_routed, 16)), WORKSPACE (table too small or not 64-byte
  * aligned), INVALID_ARG (NULL or misaligned weight pointers, or a tensor map
  * the driver refuses to encode), CUDA (no tensor-map encoder in the driver).
  */
@@ -378,10 +379,14 @@ MILO_API milo_status milo_linear_prepare(milo_linear* lin, const milo_qweight* w
 MILO_API milo_status milo_layer_prepare(milo_moe_layer* layer, const milo_expert* experts,
                                void* device_table, size_t table_bytes);
 
-/* Workspace bytes for milo_grouped_linear / milo_moe_forward over T tokens
- * (UNSUPPORTED_SHAPE when the call's rows exceed MILO_MAX_ROWS, or for a
- * layer whose top_k or n_shared milo_layer_prepare would reject).
- * The size depends on which grouped GEMM the call takes (see
+/* Workspace bytes for milo_grouped_linear / milo_moe_forward over T tokens,
+ * for a prepared lin / layer (the size depends on the max_rank that the
+ * preparation sets).  UNSUPPORTED_SHAPE for shape fields the preparation
+ * would refuse or when the call's rows exceed MILO_MAX_ROWS; INVALID_ARG for
+ * a max_rank outside 0..64 or not a multiple of 8.  The size is not monotone
+ * in T (the split-K count and the GEMM kernel change with the rows), so a
+ * caller reusing one workspace takes the largest size over the T it will
+ * call with.  The size depends on which grouped GEMM the call takes (see
  * milo_set_gemm_path: the mma.sync kernel also keeps a plain fp16 copy of the
  * scaled rows and its counters in the workspace), so query it again after
  * changing that setting; a call given less returns MILO_ERR_WORKSPACE. */

@@ -120,11 +120,45 @@ static milo_status fill_proj(ProjDev* d, const milo_qweight& w, int N, int K, co
     return MILO_OK;
 }
 
-static milo_status check_nk(int N, int K, const char* what) {
-    if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, std::string(what) + ": sizes must be positive");
-    if (N > kMaxWeightRows) return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": N above 2^31 - 64");
-    if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": K must be a multiple of 128");
-    if (N % 16) return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": N must be a multiple of 16");
+static milo_status check_nk(int N, int K, const std::string& what) {
+    if (N <= 0 || K <= 0) return fail(MILO_ERR_INVALID_ARG, what + ": sizes must be positive");
+    if (N > kMaxWeightRows) return fail(MILO_ERR_UNSUPPORTED_SHAPE, what + ": N above 2^31 - 64");
+    if (K > kMaxProjK) return fail(MILO_ERR_UNSUPPORTED_SHAPE, what + ": K above 2^24");
+    if (K % 128) return fail(MILO_ERR_UNSUPPORTED_SHAPE, what + ": K must be a multiple of 128");
+    if (N % 16) return fail(MILO_ERR_UNSUPPORTED_SHAPE, what + ": N must be a multiple of 16");
+    return MILO_OK;
+}
+
+// The shape fields of a grouped projection or a layer as the preparation
+// accepts them.  The size queries and the calls check them again, and once
+// prepared also max_rank (it sizes the compensator's rows and stages), since
+// the planning divides by and multiplies with every one of them.
+static milo_status check_linear(const milo_linear* lin, bool prepared, const char* what) {
+    const std::string f = what;
+    if (lin->group != MILO_GROUP) return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": group must be 64");
+    if (lin->n_experts < 1 || lin->n_experts > MILO_MAX_EXPERTS)
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": n_experts must be in [1, 256]");
+    const milo_status s = check_nk(lin->N, lin->K, f);
+    if (s != MILO_OK) return s;
+    if (prepared && (lin->max_rank < 0 || lin->max_rank > MILO_MAX_RANK || lin->max_rank % 8))
+        return fail(MILO_ERR_INVALID_ARG, f + ": max_rank is not one milo_linear_prepare sets (0..64, multiple of 8)");
+    return MILO_OK;
+}
+
+static milo_status check_layer(const milo_moe_layer* L, bool prepared, const char* what) {
+    const std::string f = what;
+    if (L->group != MILO_GROUP) return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": group must be 64");
+    if (L->n_routed < 1 || L->n_shared < 0 || L->n_routed > MILO_MAX_EXPERTS || L->n_shared > MILO_MAX_EXPERTS ||
+        L->n_routed + L->n_shared > MILO_MAX_EXPERTS)
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": experts: need n_routed >= 1 and n_routed + n_shared <= 256");
+    if (L->top_k < 1 || L->top_k > L->n_routed || L->top_k > MILO_MAX_TOPK)
+        return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": top_k must be in [1, min(n_routed, 16)]");
+    milo_status s;
+    if ((s = check_nk(L->inter, L->hidden, f + " (w1/w3)")) != MILO_OK) return s;
+    if ((s = check_nk(L->hidden, L->inter, f + " (w2)")) != MILO_OK) return s;
+    if (L->hidden % 4) return fail(MILO_ERR_UNSUPPORTED_SHAPE, f + ": hidden must be a multiple of 4");
+    if (prepared && (L->max_rank < 0 || L->max_rank > MILO_MAX_RANK || L->max_rank % 8))
+        return fail(MILO_ERR_INVALID_ARG, f + ": max_rank is not one milo_layer_prepare sets (0..64, multiple of 8)");
     return MILO_OK;
 }
 
@@ -248,8 +282,7 @@ static int t_slices(int K) { return (K + t_slice_len(K) - 1) / t_slice_len(K); }
 
 // The rows of one call, counted in 64 bits before the 32-bit planning below:
 // T*k routed slots (grouped linear), plus n_shared*T shared-expert rows (MoE
-// layer).  A call above MILO_MAX_ROWS, or a layer with a top_k or n_shared
-// that its preparation rejects, is refused before anything is planned.
+// layer).  A call above MILO_MAX_ROWS is refused before anything is planned.
 static milo_status check_linear_rows(int T, int k, const char* what) {
     if (static_cast<long long>(T) * k > MILO_MAX_ROWS)
         return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": T*k above MILO_MAX_ROWS");
@@ -257,8 +290,7 @@ static milo_status check_linear_rows(int T, int k, const char* what) {
 }
 
 static milo_status check_moe_rows(const milo_moe_layer* L, int T, const char* what) {
-    if (L->top_k < 1 || L->top_k > MILO_MAX_TOPK || L->n_shared < 0 || L->n_shared > MILO_MAX_EXPERTS)
-        return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": top_k or n_shared out of range");
+    // top_k and n_shared are in range here (check_layer first)
     if (static_cast<long long>(T) * (L->top_k + L->n_shared) > MILO_MAX_ROWS)
         return fail(MILO_ERR_UNSUPPORTED_SHAPE, std::string(what) + ": T*(top_k + n_shared) above MILO_MAX_ROWS");
     return MILO_OK;
@@ -483,10 +515,7 @@ extern "C" milo_status milo_linear_prepare(milo_linear* lin, const milo_qweight*
                                            void* device_table, size_t table_bytes) {
     clear_error();
     if (!lin || !weights) return fail(MILO_ERR_INVALID_ARG, "milo_linear_prepare: NULL argument");
-    if (lin->group != MILO_GROUP) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "group must be 64");
-    if (lin->n_experts < 1 || lin->n_experts > MILO_MAX_EXPERTS)
-        return fail(MILO_ERR_UNSUPPORTED_SHAPE, "n_experts must be in [1, 256]");
-    milo_status s = check_nk(lin->N, lin->K, "milo_linear_prepare");
+    milo_status s = check_linear(lin, false, "milo_linear_prepare");
     if (s != MILO_OK) return s;
     std::vector<ProjDev> t(lin->n_experts);
     int rmax = 0;
@@ -505,16 +534,9 @@ extern "C" milo_status milo_layer_prepare(milo_moe_layer* L, const milo_expert* 
                                           void* device_table, size_t table_bytes) {
     clear_error();
     if (!L || !experts) return fail(MILO_ERR_INVALID_ARG, "milo_layer_prepare: NULL argument");
-    if (L->group != MILO_GROUP) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "group must be 64");
+    milo_status s = check_layer(L, false, "milo_layer_prepare");
+    if (s != MILO_OK) return s;
     const int n_exp = L->n_routed + L->n_shared;
-    if (L->n_routed < 1 || L->n_shared < 0 || n_exp > MILO_MAX_EXPERTS)
-        return fail(MILO_ERR_UNSUPPORTED_SHAPE, "experts: need n_routed >= 1 and n_routed + n_shared <= 256");
-    if (L->top_k < 1 || L->top_k > L->n_routed || L->top_k > MILO_MAX_TOPK)
-        return fail(MILO_ERR_UNSUPPORTED_SHAPE, "top_k must be in [1, min(n_routed, 16)]");
-    milo_status s;
-    if ((s = check_nk(L->inter, L->hidden, "w1/w3")) != MILO_OK) return s;
-    if ((s = check_nk(L->hidden, L->inter, "w2")) != MILO_OK) return s;
-    if (L->hidden % 4) return fail(MILO_ERR_UNSUPPORTED_SHAPE, "hidden must be a multiple of 4");
     std::vector<ProjDev> t(3 * static_cast<size_t>(n_exp));
     int rmax = 0;
     for (int e = 0; e < n_exp; ++e) {
@@ -533,8 +555,9 @@ extern "C" milo_status milo_linear_workspace_bytes(const milo_linear* lin, int32
                                                    size_t* bytes) {
     clear_error();
     if (!lin || !bytes || T < 0 || k < 1) return fail(MILO_ERR_INVALID_ARG, "milo_linear_workspace_bytes");
-    const milo_status s = check_linear_rows(T, k, "milo_linear_workspace_bytes");
+    milo_status s = check_linear(lin, true, "milo_linear_workspace_bytes");
     if (s != MILO_OK) return s;
+    if ((s = check_linear_rows(T, k, "milo_linear_workspace_bytes")) != MILO_OK) return s;
     *bytes = linear_ws(lin, T, k).total;
     return MILO_OK;
 }
@@ -542,15 +565,18 @@ extern "C" milo_status milo_linear_workspace_bytes(const milo_linear* lin, int32
 extern "C" milo_status milo_moe_workspace_bytes(const milo_moe_layer* L, int32_t T, size_t* bytes) {
     clear_error();
     if (!L || !bytes || T < 0) return fail(MILO_ERR_INVALID_ARG, "milo_moe_workspace_bytes");
-    const milo_status s = check_moe_rows(L, T, "milo_moe_workspace_bytes");
+    milo_status s = check_layer(L, true, "milo_moe_workspace_bytes");
     if (s != MILO_OK) return s;
+    if ((s = check_moe_rows(L, T, "milo_moe_workspace_bytes")) != MILO_OK) return s;
     *bytes = moe_ws(L, T).total;
     return MILO_OK;
 }
 
 extern "C" size_t milo_moe_h_offset(const milo_moe_layer* L, int32_t T) {
     clear_error();
-    if (!L || T < 0 || check_moe_rows(L, T, "milo_moe_h_offset") != MILO_OK) return 0;
+    if (!L || T < 0 || check_layer(L, true, "milo_moe_h_offset") != MILO_OK ||
+        check_moe_rows(L, T, "milo_moe_h_offset") != MILO_OK)
+        return 0;
     return moe_ws(L, T).h;
 }
 
@@ -560,6 +586,7 @@ extern "C" milo_status milo_grouped_linear(const milo_linear* lin, const void* x
                                            size_t ws_bytes, int32_t* dev_status, void* stream) {
     clear_error();
     if (!lin || !lin->table) return fail(MILO_ERR_INVALID_ARG, "milo_grouped_linear: layer not prepared");
+    if (const milo_status s0 = check_linear(lin, true, "milo_grouped_linear"); s0 != MILO_OK) return s0;
     if (T < 0 || k < 1 || k > MILO_MAX_TOPK) return fail(MILO_ERR_INVALID_ARG, "milo_grouped_linear: bad T or k");
     if (check_linear_rows(T, k, "milo_grouped_linear") != MILO_OK) return MILO_ERR_UNSUPPORTED_SHAPE;
     if (x_dt != MILO_F16 && x_dt != MILO_BF16) return fail(MILO_ERR_INVALID_ARG, "x must be fp16 or bf16");
@@ -673,6 +700,7 @@ extern "C" milo_status milo_moe_forward(const milo_moe_layer* L, const void* x, 
                                         int32_t* dev_status, void* stream) {
     clear_error();
     if (!L || !L->table) return fail(MILO_ERR_INVALID_ARG, "milo_moe_forward: layer not prepared");
+    if (const milo_status s0 = check_layer(L, true, "milo_moe_forward"); s0 != MILO_OK) return s0;
     if (T < 0) return fail(MILO_ERR_INVALID_ARG, "milo_moe_forward: T must be >= 0");
     if (check_moe_rows(L, T, "milo_moe_forward") != MILO_OK) return MILO_ERR_UNSUPPORTED_SHAPE;
     if (x_dt != MILO_F16 && x_dt != MILO_BF16) return fail(MILO_ERR_INVALID_ARG, "x must be fp16 or bf16");

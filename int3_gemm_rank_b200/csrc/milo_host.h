@@ -42,6 +42,10 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // still fits the 32-bit row counts of the kernels.
 constexpr int32_t kMaxWeightRows = 0x7FFFFFFF - 63;
 
+// Largest K (input features) of a projection the forward calls take: the
+// planning's chunk, slice and byte counts of a row stay far inside 32 bits.
+constexpr int32_t kMaxProjK = 1 << 24;
+
 // Launch with programmatic stream serialization (see grid_dep_wait in
 // milo_device.cuh): the kernel may be scheduled while the previous kernel of
 // the stream drains.

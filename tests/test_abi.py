@@ -178,6 +178,56 @@ def test_weight_rows_bounded_so_the_tile_padding_fits_32_bits(milo):
         milo.MILO_ERR_UNSUPPORTED_SHAPE
 
 
+def test_size_queries_check_the_struct_fields(milo):
+    """The size queries (and the calls) check the shape fields as preparation
+    does, and max_rank as preparation sets it: the planning divides by and
+    multiplies with them (an expert count of 0 used to divide by zero)."""
+    L = milo.lib()
+    nb = C.c_size_t()
+    U, I = milo.MILO_ERR_UNSUPPORTED_SHAPE, milo.MILO_ERR_INVALID_ARG
+    for fields, want in (((256, 512, 0, 64, 0), U),        # no experts
+                         ((256, 512, 257, 64, 0), U),      # too many experts
+                         ((256, 512, 4, 32, 0), U),        # group
+                         ((256, 500, 4, 64, 0), U),        # K % 128
+                         ((250, 512, 4, 64, 0), U),        # N % 16
+                         ((256, (1 << 24) + 128, 4, 64, 0), U),
+                         ((256, 512, 4, 64, 12), I),       # max_rank not a multiple of 8
+                         ((256, 512, 4, 64, 72), I),
+                         ((256, 512, 4, 64, -8), I),
+                         ((256, 512, 4, 64, 64), 0)):
+        lin = milo.milo_linear(*fields, None)
+        assert L.milo_linear_workspace_bytes(C.byref(lin), 16, 2, C.byref(nb)) == want, fields
+    for fields, want in (((2048, 1408, 0, 0, 1, 64, 0), U),      # no routed experts
+                         ((2048, 1408, 200, 57, 2, 64, 0), U),   # 257 experts
+                         ((2048, 1408, 2**31 - 1, 1, 2, 64, 0), U),
+                         ((2048, 1408, 4, 0, 5, 64, 0), U),      # top_k > n_routed
+                         ((2048, 1408, 64, 0, 17, 64, 0), U),    # top_k > 16
+                         ((2048, 1400, 8, 0, 2, 64, 0), U),      # inter % 128
+                         ((2056, 1408, 8, 0, 2, 64, 0), U),      # hidden % 128
+                         ((2048, 1408, 8, 0, 2, 64, 65), I),
+                         ((2048, 1408, 64, 2, 6, 64, 64), 0)):
+        lay = milo.milo_moe_layer(*fields, None)
+        assert L.milo_moe_workspace_bytes(C.byref(lay), 16, C.byref(nb)) == want, fields
+        assert (L.milo_moe_h_offset(C.byref(lay), 16) > 0) == (want == 0)
+
+
+def test_size_queries_survive_arbitrary_fields(milo):
+    """Seeded fuzz of the size queries over extreme field values: each returns
+    a status (or 0 for the h offset), never crashes the process."""
+    import random
+    L = milo.lib()
+    rnd = random.Random(7)
+    vals = [-2**31, -129, -1, 0, 1, 7, 8, 16, 64, 100, 128, 1408, 4096, 14336, 2**20, 2**24, 2**30, 2**31 - 1]
+    nb = C.c_size_t()
+    for _ in range(3000):
+        lin = milo.milo_linear(*(rnd.choice(vals) for _ in range(5)), None)
+        T, k = rnd.choice(vals), rnd.choice(vals)
+        assert L.milo_linear_workspace_bytes(C.byref(lin), T, k, C.byref(nb)) in range(5)
+        lay = milo.milo_moe_layer(*(rnd.choice(vals) for _ in range(7)), None)
+        assert L.milo_moe_workspace_bytes(C.byref(lay), T, C.byref(nb)) in range(5)
+        L.milo_moe_h_offset(C.byref(lay), T)
+
+
 def test_quantiser_validation_and_workspace(milo):
     L = milo.lib()
     fake = C.c_void_p(0x1000)
