@@ -17,7 +17,7 @@
 namespace {
 
 constexpr size_t kScratchBytes = MILO_NOALLOC_SCRATCH_BYTES;
-__device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
