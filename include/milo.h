@@ -115,7 +115,9 @@ MILO_API int32_t milo_version(void);
  * integer (UNSUPPORTED_SHAPE above).
  */
 
-/* Bytes of the packed blob of a weight [N, K] (K % 128 == 0). */
+/* Bytes of the packed blob of a weight [N, K] (K % 128 == 0), written to the
+ * host size_t *bytes.  Errors: K % 128 != 0 or N above 2^31 - 64 ->
+ * UNSUPPORTED_SHAPE; N, K <= 0 or bytes NULL -> INVALID_ARG. */
 MILO_API milo_status milo_packed_bytes(int32_t N, int32_t K, size_t* bytes);
 
 /*
@@ -128,9 +130,11 @@ MILO_API milo_status milo_packed_bytes(int32_t N, int32_t K, size_t* bytes);
  *     q = clamp(rint(w / s + z), 0, 7)    (fp32, ties to even, no FMA)
  * Writes the blob in the device layout above, padding rows included (size
  * from milo_packed_bytes; 16-byte aligned).
- * Errors: group != 64 or K % 128 != 0 -> UNSUPPORTED_SHAPE; N, K <= 0 or NULL
- * pointers -> INVALID_ARG.  Device: NONFINITE for NaN/Inf weights, FP16_RANGE
- * when s or z overflows fp16.  dev_status may be NULL.
+ * Errors: group != 64, K % 128 != 0 or N above 2^31 - 64 -> UNSUPPORTED_SHAPE;
+ * N, K <= 0, NULL pointers or a packed buffer not 16-byte aligned ->
+ * INVALID_ARG.  Device: NONFINITE for NaN/Inf weights, FP16_RANGE when s or z
+ * overflows fp16.  dev_status may be NULL.  W and packed are caller-owned
+ * device memory; stream-ordered.
  */
 MILO_API milo_status milo_pack(const uint16_t* W, int32_t N, int32_t K, int32_t group, void* packed,
                       int32_t* dev_status, void* stream);
@@ -138,7 +142,10 @@ MILO_API milo_status milo_pack(const uint16_t* W, int32_t N, int32_t K, int32_t 
 /*
  * milo_unpack -- extract the codes of a packed blob (device layout above)
  * into codes u8 [N, K] row-major, with the same register-level field
- * extraction the GEMM kernels use.
+ * extraction the GEMM kernels use.  packed (4-byte aligned) and codes are
+ * caller-owned device memory; stream-ordered.
+ * Errors: K % 128 != 0 or N above 2^31 - 64 -> UNSUPPORTED_SHAPE; N, K <= 0,
+ * NULL or misaligned pointers -> INVALID_ARG.
  */
 MILO_API milo_status milo_unpack(const void* packed, int32_t N, int32_t K, uint8_t* codes,
                         void* stream);
@@ -152,8 +159,8 @@ MILO_API milo_status milo_unpack(const void* packed, int32_t N, int32_t K, uint8
  * faster than the unfused implementation, a dequantisation pass followed by
  * an FP16 GEMM); the fused GEMMs of this library never materialise W_hat.
  *   packed: the blob (16-byte aligned); W_hat: fp16 [N, K] (16-byte aligned).
- * Errors: K % 128 != 0 -> UNSUPPORTED_SHAPE; N, K <= 0, NULL or misaligned
- * pointers -> INVALID_ARG.  Stream-ordered.
+ * Errors: K % 128 != 0 or N above 2^31 - 64 -> UNSUPPORTED_SHAPE; N, K <= 0,
+ * NULL or misaligned pointers -> INVALID_ARG.  Stream-ordered.
  */
 MILO_API milo_status milo_dequantize(const void* packed, int32_t N, int32_t K, uint16_t* W_hat, void* stream);
 
@@ -211,7 +218,8 @@ typedef struct milo_lorc_params {
     float hqq_kappa;      /* penalty growth per iteration, finite and > 0 */
 } milo_lorc_params;
 
-/* Workspace bytes of milo_quantize_lorc for a weight [N, K]. */
+/* Workspace bytes of milo_quantize_lorc for a weight [N, K] (host size_t
+ * *bytes); the same shape and parameter errors as milo_quantize_lorc. */
 MILO_API milo_status milo_quantize_lorc_workspace(int32_t N, int32_t K, const milo_lorc_params* params,
                                                   size_t* bytes);
 
@@ -256,7 +264,8 @@ MILO_API milo_status milo_quantize_lorc(const uint16_t* W, int32_t N, int32_t K,
  * and for experts activated more often (strategy 2).
  */
 
-/* Workspace bytes of milo_kurtosis (the same for every size). */
+/* Workspace bytes of milo_kurtosis (the same for every size; host size_t
+ * *bytes, INVALID_ARG when NULL). */
 MILO_API milo_status milo_kurtosis_workspace(size_t* bytes);
 
 /*
